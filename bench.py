@@ -1,0 +1,417 @@
+#!/usr/bin/env python
+"""Benchmark of the CKDA recurrence library on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload fwdbwd|fwd|varlen|decode]
+
+Default workload (the headline): one step = ckda_chunk_fwd (saving chunk
+states) + ckda_chunk_bwd on B=8, H=16, T=4096, dk=dv=128, bf16 I/O, fp32
+gate and state -- the shape of one 1.3B-model token-mixer layer.  Inputs are
+seeded synthetic tensors (chunked_gated_delta_ckda_b200.workloads), resident
+in HBM when the timed region starts; each step streams ~2 GB, more than L2.
+
+Prints ONE JSON line (rank 0).  Under torchrun each rank runs its own batch
+(weak scaling, no collective on the data path); ``value`` = tokens of all
+ranks / the slowest rank's device time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from chunked_gated_delta_ckda_b200 import workloads as W  # noqa: E402
+
+METRIC = "CKDA fwd+bwd tokens/s (H=16,d=128,T=4096,bf16); % tensor/HBM roofline"
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+# Algorithmic work per token per head (chunk 64, dk = dv = 128; causal masks
+# counted at half; recomputation and padding excluded):
+#   forward  139 264 flop, 1666 B (q, k, v bf16; g fp32; sign int8; beta; o)
+#   backward 278 528 flop, 2948 B (inputs and dO again; dq, dk, dv, dg, dbeta)
+FWD_FLOP, FWD_BYTES = 139264, 1666
+BWD_FLOP, BWD_BYTES = 278528, 2948
+DECODE_BYTES_PER_NH = 131072 + 1666  # state read + write, per-token inputs and output
+
+# Which per-unit figure a kernel's roofline uses (the call it implements).
+KERNEL_UNITS = {
+    "v1_grad": ("bwd", BWD_BYTES, BWD_FLOP),
+    "v1_state_bwd": ("bwd", BWD_BYTES, BWD_FLOP),
+    "v1_intra": ("fwd", FWD_BYTES, FWD_FLOP),
+    "v1_state_fwd": ("fwd", FWD_BYTES, FWD_FLOP),
+    "v1_state_fwd_recompute": ("fwd", FWD_BYTES, FWD_FLOP),
+    "decode": ("decode", DECODE_BYTES_PER_NH, 0),
+}
+
+# DRAM traffic per launch measured by ncu (dram__bytes_read.sum +
+# dram__bytes_write.sum) for the kernel as it stands, keyed by kernel and
+# workload; None until captured for the current kernel version.
+NCU_TRAFFIC = {}
+
+
+# ---------------------------------------------------------------------------
+# host-side helpers (unit-tested on CPU with gloo)
+# ---------------------------------------------------------------------------
+
+def rank_seed(base: int, rank: int) -> int:
+    """Each rank draws its own batch (weak scaling)."""
+    return base + 1000 * rank
+
+
+def reduce_max(x: float, world: int) -> float:
+    """Slowest rank's value (max over ranks); identity for one process."""
+    if world <= 1:
+        return float(x)
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([float(x)], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate(tokens_per_rank: int, world: int, max_ms_per_step: float) -> float:
+    """Whole-job throughput: tokens of all ranks per second of the slowest rank."""
+    return tokens_per_rank * world / (max_ms_per_step / 1e3)
+
+
+def measured_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return dict(hbm_gbs=d.get("hbm_gbs", FALLBACK_HBM_GBS),
+                    bf16_tflops=d.get("bf16_tflops", FALLBACK_BF16_TFLOPS),
+                    bf16_tflops_sustained=d.get("bf16_tflops_sustained", FALLBACK_BF16_TFLOPS),
+                    source="measured")
+    return dict(hbm_gbs=FALLBACK_HBM_GBS, bf16_tflops=FALLBACK_BF16_TFLOPS,
+                bf16_tflops_sustained=1400.0, source="fallback")
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.path = None
+        self.dev = device_index
+
+    def start(self):
+        try:
+            uuid = str(torch.cuda.get_device_properties(self.dev).uuid)
+            sel = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", sel, "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) == 7:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(r[0]) for r in rows if r[0].replace(".", "").isdigit()]
+        mx = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[3 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------
+# our implementation
+# ---------------------------------------------------------------------------
+
+def _fwdbwd_setup(inp, dev):
+    from chunked_gated_delta_ckda_b200 import _abi, api
+    d = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+    B, T, H, dk = d["q"].shape
+    dv = d["v"].shape[-1]
+    NC = (T + 63) // 64
+    e = lambda *s, dt: torch.empty(*s, dtype=dt, device=dev)
+    io = d["q"].dtype
+    buf = dict(o=e(B, T, H, dv, dt=io), ST=e(B, H, dk, dv, dt=torch.float32),
+               cs=e(B, H, NC, dk, dv, dt=torch.float32), dq=e(B, T, H, dk, dt=io),
+               dk=e(B, T, H, dk, dt=io), dv=e(B, T, H, dv, dt=io),
+               dg=e(B, T, H, dk, dt=torch.float32), dbeta=e(B, T, H, dt=io),
+               dS0=e(B, H, dk, dv, dt=torch.float32))
+    wsf = api.workspace(_abi.CKDA_OP_CHUNK_FWD, B, T, H, dk, dv, device=dev, cache=False)
+    wsb = api.workspace(_abi.CKDA_OP_CHUNK_BWD, B, T, H, dk, dv, device=dev, cache=False)
+    code = api.io_code(io)
+
+    def step():
+        _abi.ckda_chunk_fwd(B, T, H, dk, dv, code, d["q"], d["k"], d["v"], d["g"], d["sign"],
+                            d["beta"], None, buf["o"], buf["ST"], buf["cs"], wsf)
+        _abi.ckda_chunk_bwd(B, T, H, dk, dv, code, d["q"], d["k"], d["v"], d["g"], d["sign"],
+                            d["beta"], None, d["dO"], None, buf["cs"], buf["dq"], buf["dk"],
+                            buf["dv"], buf["dg"], buf["dbeta"], buf["dS0"], wsb)
+    return d, buf, step
+
+
+def _time_steps(step, steps, warmup, world):
+    import torch.distributed as dist
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    s = torch.cuda.current_stream()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(s)
+    for _ in range(steps):
+        step()
+    b.record(s)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / steps
+
+
+def run_ours(args, rank, world, local_rank):
+    from chunked_gated_delta_ckda_b200 import _abi
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    wl = W.LAYER_FWDBWD
+    w = W.Workload(**{**wl.__dict__, "seed": rank_seed(wl.seed, rank)})
+    inp = W.make(w)
+    B, T, H = w.B, w.T, w.H
+    tokens = B * T
+    d, buf, step = _fwdbwd_setup(inp, dev)
+
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    _abi.ckda_profile_reset()
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    _abi.ckda_profile_enable(True)
+    ms = _time_steps(step, args.steps, 0, world)
+    _abi.ckda_profile_enable(False)
+    prof = _abi.ckda_profile_collect()
+    clk = clocks.stop()
+    ms_max = reduce_max(ms, world)
+    value = aggregate(tokens, world, ms_max)
+
+    # dominant kernel, timed live with CUDA events on the launch stream
+    peaks = measured_peaks()
+    total = sum(t for _, t in prof.values())
+    kernels = {k: {"launches": n, "ms_per_launch": t / n, "share": t / total if total else None}
+               for k, (n, t) in sorted(prof.items(), key=lambda kv: -kv[1][1])}
+    top = max(prof.items(), key=lambda kv: kv[1][1])[0] if prof else None
+    roof = None
+    if top is not None:
+        n, t = prof[top]
+        unit, bytes_per, _ = KERNEL_UNITS.get(top, ("bwd", BWD_BYTES, BWD_FLOP))
+        alg_bytes = bytes_per * B * T * H
+        achieved = alg_bytes / (t / n / 1e3) / 1e9
+        roof = {"bound": "hbm", "kernel": top, "achieved": achieved, "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                "traffic": NCU_TRAFFIC.get((top, w.name)),
+                "algorithmic_bytes_per_launch": alg_bytes, "per_unit": "%d B per token-head (%s)" % (bytes_per, unit),
+                "peak_source": peaks["source"]}
+    # whole step against both roofs
+    t_hbm = (FWD_BYTES + BWD_BYTES) * B * T * H / (peaks["hbm_gbs"] * 1e9) * 1e3
+    t_tc = (FWD_FLOP + BWD_FLOP) * B * T * H / (peaks["bf16_tflops_sustained"] * 1e12) * 1e3
+    step_roof = {"t_hbm_ms": t_hbm, "t_tensor_ms": t_tc, "hbm_frac": t_hbm / ms_max,
+                 "tensor_frac": t_tc / ms_max, "binding_frac": max(t_hbm, t_tc) / ms_max}
+
+    # end to end through the public API with host buffers
+    e2e = run_e2e(inp, dev, args, world)
+
+    out = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+           "dtype": "f32", "data": "synthetic",
+           "config": {"workload": w.name, "B": B, "T": T, "H": H, "dk": w.dk, "dv": w.dv,
+                      "io_dtype": "bf16", "gate_dtype": "f32", "state_dtype": "f32",
+                      "step": "ckda_chunk_fwd(save chunk states) + ckda_chunk_bwd",
+                      "global_batch": B * world, "seq_len": T, "parallelism": "dp%d" % world,
+                      "l2": "inputs larger than L2 (about 2 GB streamed per step)"},
+           "roofline": roof, "step_roofline": step_roof, "kernels": kernels,
+           "gpu_launches": int(sum(n for n, _ in prof.values())), "clocks": clk, "e2e": e2e}
+    return out, inp
+
+
+def run_e2e(inp, dev, args, world):
+    """Same step through the public API from pinned HOST buffers: H2D of the
+    inputs and D2H of every output inside the timed region."""
+    from chunked_gated_delta_ckda_b200 import _abi, api
+    host_in = {k: inp[k].pin_memory() for k in ("q", "k", "v", "g", "sign", "beta", "dO")}
+    dev_in = {k: torch.empty_like(v, device=dev) for k, v in host_in.items()}
+    B, T, H, dk = inp["q"].shape
+    dv = inp["v"].shape[-1]
+    d, buf, _ = _fwdbwd_setup({**inp}, dev)
+    host_out = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True)
+                for k, v in buf.items() if k not in ("cs",)}
+    wsf = api.workspace(_abi.CKDA_OP_CHUNK_FWD, B, T, H, dk, dv, device=dev, cache=False)
+    wsb = api.workspace(_abi.CKDA_OP_CHUNK_BWD, B, T, H, dk, dv, device=dev, cache=False)
+    code = api.io_code(inp["q"].dtype)
+    h2d = sum(v.numel() * v.element_size() for v in host_in.values())
+    d2h = sum(v.numel() * v.element_size() for v in host_out.values())
+
+    def step():
+        for k, v in host_in.items():
+            dev_in[k].copy_(v, non_blocking=True)
+        x = dev_in
+        _abi.ckda_chunk_fwd(B, T, H, dk, dv, code, x["q"], x["k"], x["v"], x["g"], x["sign"],
+                            x["beta"], None, buf["o"], buf["ST"], buf["cs"], wsf)
+        _abi.ckda_chunk_bwd(B, T, H, dk, dv, code, x["q"], x["k"], x["v"], x["g"], x["sign"],
+                            x["beta"], None, x["dO"], None, buf["cs"], buf["dq"], buf["dk"],
+                            buf["dv"], buf["dg"], buf["dbeta"], buf["dS0"], wsb)
+        for k, v in host_out.items():
+            v.copy_(buf[k], non_blocking=True)
+
+    steps = max(1, min(args.steps, 10))
+    ms = _time_steps(step, steps, max(1, min(args.warmup, 3)), world)
+    ms = reduce_max(ms, world)
+    return {"value": aggregate(B * T, world, ms), "unit": "tokens/s", "ms_per_step": ms,
+            "steps": steps, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+
+# ---------------------------------------------------------------------------
+# the fp64 CPU oracle (baseline / reference arm)
+# ---------------------------------------------------------------------------
+
+def oracle_fwdbwd_sample(inp, pairs, nthreads):
+    """Oracle forward + backward over the sampled (batch, head) sequences."""
+    import numpy as np
+    import oracle
+    T = inp["q"].shape[1]
+    P = lambda x, b, h: x[b, :, h:h + 1].to(torch.float64).numpy()
+    # pack the sampled sequences as independent documents of one head
+    cat = lambda key: np.concatenate([P(inp[key], b, h) for b, h in pairs], axis=0)
+    sg = np.concatenate([inp["sign"][b, :, h:h + 1].numpy() for b, h in pairs], axis=0)
+    cu = np.arange(len(pairs) + 1, dtype=np.int64) * T
+    q, k, v, g, beta, dO = (cat(x) for x in ("q", "k", "v", "g", "beta", "dO"))
+    t0 = time.perf_counter()
+    oracle.fwd(cu, q, k, v, g, sg, beta, nthreads=nthreads)
+    oracle.bwd(cu, q, k, v, g, sg, beta, dO, nthreads=nthreads)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(inp, H, n_pairs=None):
+    import oracle
+    cores = oracle.default_threads()
+    n_pairs = n_pairs or max(8, min(128, 12 * cores))
+    B = inp["q"].shape[0]
+    pairs = [(i % B, (i * 7) % H) for i in range(n_pairs)]
+    threads = min(cores, n_pairs)
+    dt = oracle_fwdbwd_sample(inp, pairs, threads)
+    T = inp["q"].shape[1]
+    tokens = n_pairs * T / H  # a token carries H heads
+    return {"value": tokens / dt, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": "%d of %d (batch, head) sequences of %d tokens, forward + backward, fp64, "
+                      "%d threads, %.1f s" % (n_pairs, B * H, T, threads, dt)}
+
+
+def run_reference(args, rank, world):
+    """The oracle as it stands, timed on the host cores, on this workload."""
+    import oracle
+    if rank != 0:
+        return None
+    oracle.build()
+    w = W.LAYER_FWDBWD
+    inp = W.make(w)
+    cores = oracle.default_threads()
+    n_pairs = max(2, min(8, cores))
+    pairs = [(i % w.B, (i * 5) % w.H) for i in range(n_pairs)]
+    threads = min(cores, n_pairs)
+    for _ in range(args.warmup):
+        oracle_fwdbwd_sample(inp, pairs[:1], 1)
+    dts = [oracle_fwdbwd_sample(inp, pairs, threads) for _ in range(args.steps)]
+    dt = sum(dts) / len(dts)
+    value = n_pairs * w.T / w.H / dt
+    sample = ("%d of %d (batch, head) sequences of %d tokens per step, forward + backward, "
+              "fp64, %d threads" % (n_pairs, w.B * w.H, w.T, threads))
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "dk": w.dk, "dv": w.dv,
+                       "io_dtype": "bf16", "global_batch": w.B, "seq_len": w.T,
+                       "parallelism": "host cores"},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+# ---------------------------------------------------------------------------
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        out = run_reference(args, rank, world)
+        if out is not None:
+            print(json.dumps(out), flush=True)
+        return 0
+
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        out, inp = run_ours(args, rank, world, local_rank)
+        if rank == 0:
+            if world == 1 and not args.no_cpu_baseline:
+                out["cpu_baseline"] = cpu_baseline(inp, W.LAYER_FWDBWD.H)
+            print(json.dumps(out), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+            dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,120 @@
+"""Tensor-level helpers over the C ABI: allocate outputs and workspaces with
+torch (device memory is torch's job here) and call the library.
+
+    o, ST, cs = chunk_fwd(q, k, v, g, sign, beta, S0=None, save_chunk_states=True)
+    grads     = chunk_bwd(q, k, v, g, sign, beta, dO, S0=None, dST=None, chunk_states=cs)
+    o         = decode_step(q, k, v, g, sign, beta, state)     # state updated in place
+    o, ST     = varlen_fwd(q, k, v, g, sign, beta, cu_seqlens, max_seqlen, S0=None)
+
+Shapes and dtypes are those of include/ckda.h: q, k, g, sign [B,T,H,dk]; v
+[B,T,H,dv]; beta [B,T,H]; g fp32; sign int8; q, k, v, beta either fp32 or
+bf16 (all the same); states fp32 [B,H,dk,dv].
+"""
+from __future__ import annotations
+
+from typing import Optional
+
+import torch
+
+from . import _abi
+from ._abi import CKDA_BF16, CKDA_F32, CKDA_OP_CHUNK_BWD, CKDA_OP_CHUNK_FWD, CKDA_OP_VARLEN_FWD
+
+_ws_cache: dict = {}
+
+
+def io_code(dtype: torch.dtype) -> int:
+    if dtype == torch.float32:
+        return CKDA_F32
+    if dtype == torch.bfloat16:
+        return CKDA_BF16
+    raise TypeError("q, k, v, beta must be float32 or bfloat16, got %s" % dtype)
+
+
+def workspace(op: int, B: int, T: int, H: int, dk: int, dv: int, N: int = 0,
+              device=None, cache: bool = True) -> torch.Tensor:
+    """A workspace of at least ckda_workspace_size(...) bytes (256-aligned)."""
+    n = _abi.ckda_workspace_size(op, B, T, H, dk, dv, N)
+    device = torch.device(device or "cuda")
+    key = (device, torch.cuda.current_stream(device).cuda_stream)
+    if cache:
+        ws = _ws_cache.get(key)
+        if ws is not None and ws.numel() >= max(n, 1):
+            return ws
+    ws = torch.empty(max(n, 256), dtype=torch.uint8, device=device)
+    if cache:
+        _ws_cache[key] = ws
+    return ws
+
+
+def _c(x: Optional[torch.Tensor]) -> Optional[torch.Tensor]:
+    if x is None:
+        return None
+    if not x.is_cuda:
+        raise ValueError("tensors must be on a CUDA device")
+    return x if x.is_contiguous() else x.contiguous()
+
+
+def chunk_fwd(q, k, v, g, sign, beta, S0=None, output_final_state=True, save_chunk_states=False,
+              ws=None):
+    q, k, v, g, sign, beta, S0 = map(_c, (q, k, v, g, sign, beta, S0))
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    io = io_code(q.dtype)
+    o = torch.empty(B, T, H, dv, dtype=q.dtype, device=q.device)
+    ST = torch.empty(B, H, dk, dv, dtype=torch.float32, device=q.device) if output_final_state else None
+    NC = (T + 63) // 64
+    cs = (torch.empty(B, H, NC, dk, dv, dtype=torch.float32, device=q.device)
+          if save_chunk_states else None)
+    if ws is None:
+        ws = workspace(CKDA_OP_CHUNK_FWD, B, T, H, dk, dv, device=q.device)
+    _abi.ckda_chunk_fwd(B, T, H, dk, dv, io, q, k, v, g, sign, beta, S0, o, ST, cs, ws)
+    return o, ST, cs
+
+
+def chunk_bwd(q, k, v, g, sign, beta, dO, S0=None, dST=None, chunk_states=None, need_dS0=True,
+              ws=None):
+    q, k, v, g, sign, beta, dO, S0, dST, chunk_states = map(
+        _c, (q, k, v, g, sign, beta, dO, S0, dST, chunk_states))
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    io = io_code(q.dtype)
+    dq = torch.empty_like(q)
+    dk_ = torch.empty_like(k)
+    dv_ = torch.empty_like(v)
+    dg = torch.empty_like(g)
+    dbeta = torch.empty_like(beta)
+    dS0 = torch.empty(B, H, dk, dv, dtype=torch.float32, device=q.device) if need_dS0 else None
+    if ws is None:
+        ws = workspace(CKDA_OP_CHUNK_BWD, B, T, H, dk, dv, device=q.device)
+    _abi.ckda_chunk_bwd(B, T, H, dk, dv, io, q, k, v, g, sign, beta, S0, dO, dST, chunk_states,
+                        dq, dk_, dv_, dg, dbeta, dS0, ws)
+    return dict(dq=dq, dk=dk_, dv=dv_, dg=dg, dbeta=dbeta, dS0=dS0)
+
+
+def decode_step(q, k, v, g, sign, beta, state, o=None):
+    q, k, v, g, sign, beta = map(_c, (q, k, v, g, sign, beta))
+    if not state.is_contiguous() or state.dtype != torch.float32:
+        raise ValueError("state must be a contiguous float32 tensor (updated in place)")
+    N, H, dk = q.shape
+    dv = v.shape[-1]
+    if o is None:
+        o = torch.empty(N, H, dv, dtype=q.dtype, device=q.device)
+    _abi.ckda_decode_step(N, H, dk, dv, io_code(q.dtype), q, k, v, g, sign, beta, state, o)
+    return o
+
+
+def varlen_fwd(q, k, v, g, sign, beta, cu_seqlens, max_seqlen, S0=None, output_final_state=True,
+               ws=None):
+    q, k, v, g, sign, beta, S0, cu_seqlens = map(_c, (q, k, v, g, sign, beta, S0, cu_seqlens))
+    if cu_seqlens.dtype != torch.int32:
+        raise TypeError("cu_seqlens must be int32")
+    _, T, H, dk = q.shape
+    dv = v.shape[-1]
+    N = cu_seqlens.numel() - 1
+    o = torch.empty(1, T, H, dv, dtype=q.dtype, device=q.device)
+    ST = torch.empty(N, H, dk, dv, dtype=torch.float32, device=q.device) if output_final_state else None
+    if ws is None:
+        ws = workspace(CKDA_OP_VARLEN_FWD, 1, T, H, dk, dv, N, device=q.device)
+    _abi.ckda_varlen_fwd(T, N, cu_seqlens, int(max_seqlen), H, dk, dv, io_code(q.dtype), q, k, v,
+                         g, sign, beta, S0, o, ST, ws)
+    return o, ST

@@ -1,0 +1,260 @@
+// ckda_api.cu -- the extern "C" entry points of include/ckda.h: argument
+// validation, workspace layout and dispatch to the kernels.  Host only.
+#include <cstdint>
+#include <cstring>
+
+#include "ckda_internal.cuh"
+
+namespace ckda {
+
+WsLayout ws_layout(int op, int B, int T, int H, int dk, int dv, int N) {
+  WsLayout L;
+  const bool packed = (op == CKDA_OP_VARLEN_FWD);
+  int64_t nch;
+  int NC = 0;
+  if (packed) {
+    const int64_t bound = (int64_t)T / C + N;
+    nch = bound < T ? bound : T;
+  } else {
+    NC = (T + C - 1) / C;
+    nch = (int64_t)B * NC;
+  }
+  L.n_chunks_bound = (int)nch;
+  size_t off = align256(sizeof(DevStatus));
+  if (packed) {
+    L.table = off;
+    off += align256((size_t)nch * 4 * sizeof(int32_t));
+    L.seq_first = off;
+    off += align256((size_t)(N + 1) * sizeof(int32_t));
+  }
+  L.intra_stride = intra_floats(dk, dv);
+  L.intra = off;
+  off += align256((size_t)nch * H * L.intra_stride * sizeof(float));
+  L.fscratch = off;
+  off += align256(v1_fwd_scratch_floats(dk, dv) * sizeof(float));
+  if (op == CKDA_OP_CHUNK_BWD) {
+    const size_t st = (size_t)B * H * NC * dk * dv * sizeof(float);
+    L.states = off;
+    off += align256(st);
+    L.dsend = off;
+    off += align256(st);
+    L.du = off;
+    off += align256((size_t)nch * H * C * dv * sizeof(float));
+    L.scratch = off;
+    off += align256(bwd_scratch_floats(dk, dv) * kBwdCtas * sizeof(float));
+  }
+  L.total = off;
+  return L;
+}
+
+}  // namespace ckda
+
+using namespace ckda;
+
+namespace {
+
+bool a16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool a256(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 255u) == 0; }
+bool dim_ok(int d) { return d == 64 || d == 128; }
+
+int check_common(int B, int T, int H, int dk, int dv, int io_dtype) {
+  if (B < 0 || T < 0 || H < 1) return CKDA_ERR_INVALID_ARG;
+  if (io_dtype != CKDA_F32 && io_dtype != CKDA_BF16) return CKDA_ERR_INVALID_ARG;
+  if (!dim_ok(dk) || !dim_ok(dv)) return CKDA_ERR_UNSUPPORTED;
+  // index arithmetic is 64-bit; chunk ids and token offsets are 32-bit
+  if ((int64_t)B * T > INT32_MAX / 2) return CKDA_ERR_UNSUPPORTED;
+  return CKDA_OK;
+}
+
+int check_ptrs(std::initializer_list<const void *> required,
+               std::initializer_list<const void *> optional) {
+  for (const void *p : required)
+    if (!p) return CKDA_ERR_INVALID_ARG;
+  for (const void *p : required)
+    if (!a16(p)) return CKDA_ERR_ALIGNMENT;
+  for (const void *p : optional)
+    if (p && !a16(p)) return CKDA_ERR_ALIGNMENT;
+  return CKDA_OK;
+}
+
+int check_ws(const void *ws, size_t ws_bytes, size_t need) {
+  if (!ws || ws_bytes < need) return CKDA_ERR_WORKSPACE;
+  if (!a256(ws)) return CKDA_ERR_ALIGNMENT;
+  return CKDA_OK;
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? CKDA_OK : CKDA_ERR_CUDA; }
+
+#define CKDA_TRY(expr)                          \
+  do {                                          \
+    int _rc = (expr);                           \
+    if (_rc != CKDA_OK) return _rc;             \
+  } while (0)
+#define CKDA_CUDA(expr) CKDA_TRY(cuda_status(expr))
+
+}  // namespace
+
+extern "C" {
+
+size_t ckda_workspace_size(int op, int B, int T, int H, int dk, int dv, int N) {
+  if (op < CKDA_OP_CHUNK_FWD || op > CKDA_OP_VARLEN_FWD) return 0;
+  if (op == CKDA_OP_VARLEN_FWD) {
+    if (B != 1 || N < 0) return 0;
+  }
+  if (check_common(B, T, H, dk, dv, CKDA_F32) != CKDA_OK) return 0;
+  return ws_layout(op, B, T, H, dk, dv, N).total;
+}
+
+int ckda_chunk_fwd(int B, int T, int H, int dk, int dv, int io_dtype, const void *q,
+                   const void *k, const void *v, const float *g, const int8_t *sign,
+                   const void *beta, const float *S0, void *o, float *ST, float *chunk_states,
+                   void *ws, size_t ws_bytes, cudaStream_t stream) {
+  CKDA_TRY(check_common(B, T, H, dk, dv, io_dtype));
+  const bool empty = (int64_t)B * T == 0;
+  if (!empty) CKDA_TRY(check_ptrs({q, k, v, g, sign, beta, o}, {S0, ST, chunk_states}));
+  else CKDA_TRY(check_ptrs({}, {S0, ST, chunk_states}));
+  const WsLayout L = ws_layout(CKDA_OP_CHUNK_FWD, B, T, H, dk, dv, 0);
+  CKDA_TRY(check_ws(ws, ws_bytes, L.total));
+  char *w = static_cast<char *>(ws);
+  CKDA_CUDA(cudaMemsetAsync(w, 0, sizeof(DevStatus), stream));
+  FwdArgs a{};
+  a.B = B; a.T = T; a.H = H; a.dk = dk; a.dv = dv;
+  a.q = q; a.k = k; a.v = v; a.beta = beta; a.g = g; a.sign = sign;
+  a.S0 = S0; a.o = o; a.ST = ST; a.chunk_states = chunk_states;
+  a.map.T = T;
+  a.map.NC = (T + C - 1) / C;
+  a.map.n_seq = B;
+  a.map.n_chunks_bound = L.n_chunks_bound;
+  a.intra = reinterpret_cast<float *>(w + L.intra);
+  a.status = reinterpret_cast<DevStatus *>(w);
+  const bool bf16 = io_dtype == CKDA_BF16;
+  CKDA_CUDA(v1_intra(a, bf16, reinterpret_cast<float *>(w + L.fscratch), stream));
+  CKDA_CUDA(v1_state_fwd(a, bf16, true, chunk_states, stream));
+  return CKDA_OK;
+}
+
+int ckda_chunk_bwd(int B, int T, int H, int dk, int dv, int io_dtype, const void *q,
+                   const void *k, const void *v, const float *g, const int8_t *sign,
+                   const void *beta, const float *S0, const void *dO, const float *dST,
+                   const float *chunk_states, void *dq, void *dk_out, void *dv_out, float *dg,
+                   void *dbeta, float *dS0, void *ws, size_t ws_bytes, cudaStream_t stream) {
+  CKDA_TRY(check_common(B, T, H, dk, dv, io_dtype));
+  const bool empty = (int64_t)B * T == 0;
+  if (!empty)
+    CKDA_TRY(check_ptrs({q, k, v, g, sign, beta, dO, dq, dk_out, dv_out, dg, dbeta},
+                        {S0, dST, chunk_states, dS0}));
+  else
+    CKDA_TRY(check_ptrs({}, {S0, dST, chunk_states, dS0}));
+  const WsLayout L = ws_layout(CKDA_OP_CHUNK_BWD, B, T, H, dk, dv, 0);
+  CKDA_TRY(check_ws(ws, ws_bytes, L.total));
+  char *w = static_cast<char *>(ws);
+  CKDA_CUDA(cudaMemsetAsync(w, 0, sizeof(DevStatus), stream));
+  const bool bf16 = io_dtype == CKDA_BF16;
+  FwdArgs f{};
+  f.B = B; f.T = T; f.H = H; f.dk = dk; f.dv = dv;
+  f.q = q; f.k = k; f.v = v; f.beta = beta; f.g = g; f.sign = sign; f.S0 = S0;
+  f.map.T = T;
+  f.map.NC = (T + C - 1) / C;
+  f.map.n_seq = B;
+  f.map.n_chunks_bound = L.n_chunks_bound;
+  f.intra = reinterpret_cast<float *>(w + L.intra);
+  f.status = reinterpret_cast<DevStatus *>(w);
+  CKDA_CUDA(v1_intra(f, bf16, reinterpret_cast<float *>(w + L.fscratch), stream));
+  const float *states = chunk_states;
+  if (!states) {
+    float *st = reinterpret_cast<float *>(w + L.states);
+    CKDA_CUDA(v1_state_fwd(f, bf16, false, st, stream));
+    states = st;
+  }
+  BwdArgs a{};
+  a.B = B; a.T = T; a.H = H; a.dk = dk; a.dv = dv;
+  a.q = q; a.k = k; a.v = v; a.beta = beta; a.dO = dO; a.g = g; a.sign = sign;
+  a.S0 = S0; a.dST = dST; a.states = states;
+  a.dq = dq; a.dkg = dk_out; a.dvg = dv_out; a.dbeta = dbeta; a.dg = dg; a.dS0 = dS0;
+  a.map = f.map;
+  a.intra = f.intra;
+  a.dsend = reinterpret_cast<float *>(w + L.dsend);
+  a.du = reinterpret_cast<float *>(w + L.du);
+  a.scratch = reinterpret_cast<float *>(w + L.scratch);
+  a.status = f.status;
+  CKDA_CUDA(v1_backward(a, bf16, stream));
+  return CKDA_OK;
+}
+
+int ckda_decode_step(int N, int H, int dk, int dv, int io_dtype, const void *q, const void *k,
+                     const void *v, const float *g, const int8_t *sign, const void *beta,
+                     float *state, void *o, cudaStream_t stream) {
+  CKDA_TRY(check_common(N, 1, H, dk, dv, io_dtype));
+  if (N == 0) return CKDA_OK;
+  CKDA_TRY(check_ptrs({q, k, v, g, sign, beta, state, o}, {}));
+  return cuda_status(decode_step(N, H, dk, dv, io_dtype == CKDA_BF16, q, k, v, g, sign, beta,
+                                 state, o, stream));
+}
+
+int ckda_varlen_fwd(int total_T, int N, const int32_t *cu_seqlens, int max_seqlen, int H,
+                    int dk, int dv, int io_dtype, const void *q, const void *k, const void *v,
+                    const float *g, const int8_t *sign, const void *beta, const float *S0,
+                    void *o, float *ST, void *ws, size_t ws_bytes, cudaStream_t stream) {
+  CKDA_TRY(check_common(1, total_T, H, dk, dv, io_dtype));
+  if (N < 0) return CKDA_ERR_INVALID_ARG;
+  if (N == 0) return total_T == 0 ? CKDA_OK : CKDA_ERR_INVALID_ARG;
+  if (!cu_seqlens) return CKDA_ERR_INVALID_ARG;
+  if (total_T > 0 && (max_seqlen < 1 || max_seqlen > total_T)) return CKDA_ERR_INVALID_ARG;
+  if (total_T > 0) CKDA_TRY(check_ptrs({q, k, v, g, sign, beta, o}, {S0, ST}));
+  else CKDA_TRY(check_ptrs({}, {S0, ST}));
+  if ((reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) != 0) return CKDA_ERR_ALIGNMENT;
+  const WsLayout L = ws_layout(CKDA_OP_VARLEN_FWD, 1, total_T, H, dk, dv, N);
+  CKDA_TRY(check_ws(ws, ws_bytes, L.total));
+  char *w = static_cast<char *>(ws);
+  CKDA_CUDA(cudaMemsetAsync(w, 0, sizeof(DevStatus), stream));
+  FwdArgs a{};
+  a.B = 1; a.T = total_T; a.H = H; a.dk = dk; a.dv = dv;
+  a.q = q; a.k = k; a.v = v; a.beta = beta; a.g = g; a.sign = sign;
+  a.S0 = S0; a.o = o; a.ST = ST; a.chunk_states = nullptr;
+  a.map.table = reinterpret_cast<const int32_t *>(w + L.table);
+  a.map.seq_first = reinterpret_cast<const int32_t *>(w + L.seq_first);
+  a.map.status = reinterpret_cast<const DevStatus *>(w);
+  a.map.T = total_T;
+  a.map.NC = 0;
+  a.map.n_seq = N;
+  a.map.n_chunks_bound = L.n_chunks_bound;
+  a.intra = reinterpret_cast<float *>(w + L.intra);
+  a.status = reinterpret_cast<DevStatus *>(w);
+  CKDA_CUDA(build_chunk_table(cu_seqlens, N, total_T, total_T > 0 ? max_seqlen : 0,
+                              L.n_chunks_bound, reinterpret_cast<int32_t *>(w + L.table),
+                              reinterpret_cast<int32_t *>(w + L.seq_first),
+                              reinterpret_cast<DevStatus *>(w), stream));
+  const bool bf16 = io_dtype == CKDA_BF16;
+  CKDA_CUDA(v1_intra(a, bf16, reinterpret_cast<float *>(w + L.fscratch), stream));
+  CKDA_CUDA(v1_state_fwd(a, bf16, true, nullptr, stream));
+  return CKDA_OK;
+}
+
+int ckda_check_device_status(const void *ws, cudaStream_t stream) {
+  if (!ws) return CKDA_ERR_INVALID_ARG;
+  DevStatus st;
+  if (cudaMemcpyAsync(&st, ws, sizeof(st), cudaMemcpyDeviceToHost, stream) != cudaSuccess)
+    return CKDA_ERR_CUDA;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return CKDA_ERR_CUDA;
+  if (st.flags & kFlagTimeout) return CKDA_ERR_TIMEOUT;
+  if (st.flags & kFlagBadSeqlens) return CKDA_ERR_DEVICE_ARG;
+  return CKDA_OK;
+}
+
+const char *ckda_status_string(int status) {
+  switch (status) {
+    case CKDA_OK: return "ok";
+    case CKDA_ERR_INVALID_ARG: return "invalid argument (null pointer, negative size or bad enum)";
+    case CKDA_ERR_UNSUPPORTED: return "unsupported shape (dk and dv must be 64 or 128)";
+    case CKDA_ERR_ALIGNMENT: return "misaligned pointer (tensors 16-byte, workspace 256-byte)";
+    case CKDA_ERR_WORKSPACE: return "workspace missing or smaller than ckda_workspace_size()";
+    case CKDA_ERR_CUDA: return "CUDA launch or runtime error";
+    case CKDA_ERR_TIMEOUT: return "a bounded device wait gave up";
+    case CKDA_ERR_DEVICE_ARG: return "malformed cu_seqlens (found on the device)";
+    default: return "unknown status";
+  }
+}
+
+int ckda_version(void) { return 100; }
+
+}  // extern "C"

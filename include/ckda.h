@@ -1,0 +1,180 @@
+/*
+ * ckda.h -- C ABI of the B200 (sm_100a) Complex KDA (CKDA) recurrence library.
+ *
+ * The operation (one head of one sequence):
+ *
+ *   alpha_t = sign_t * exp(g_t)          signed per-channel gate, |alpha| <= 1
+ *   S_t     = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T
+ *   o_t     = S_t^T q_t
+ *
+ * with S in R^{dk x dv} (rows: key channels, columns: value channels),
+ * beta_t in [0, 2].  Sources: "openeurollm/complex-kda-1.3B-100B" model card,
+ * introduction (signed decay alpha in [-1, 1]; |alpha| carried in log space;
+ * the +-1 part carried as a running product folded onto queries and keys so
+ * the kernels run the unsigned recurrence); "Complex KDA: Understanding and
+ * Enhancing the Expressivity of Kimi Delta Attention", section 2 (Related
+ * work, "Linear RNNs": delta-rule transition, KDA's channel-wise gate, WY-based
+ * chunk-wise implementations) and section 3 ("CKDA": gate in [-1, 1], beta in
+ * [0, 2]).  No output scaling is applied: callers pre-scale q if they want one.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  Layout     Activations are [B, T, H, D] contiguous (head-interleaved, the
+ *             layout of a [B, T, H*D] projection).  beta is [B, T, H]; g and
+ *             sign are [B, T, H, dk]; states are [B, H, dk, dv].  The packed
+ *             variable-length call uses B = 1 and cu_seqlens.
+ *  Dtypes     io_dtype (CKDA_F32 or CKDA_BF16) applies to q, k, v, beta, o and,
+ *             in the backward, to dO, dq, dk, dv and dbeta.  g, dg and every
+ *             state (S0, ST, chunk_states, dST, dS0, the decode state) are fp32.
+ *             sign is int8 holding +1 or -1 (any other value: undefined
+ *             output).  g = log|alpha| should be <= 0; the library computes
+ *             exactly what it is given, and very negative g (a gate near 0) is
+ *             supported.
+ *  Shapes     dk, dv in {64, 128}; any T >= 0; the chunk length is 64.
+ *  States     Every state crossing this ABI is in the true (signed) frame, so
+ *             the final state of a chunked or packed forward can seed a decode
+ *             step directly.  The sign folding is internal.
+ *  Ownership  All pointers are caller-owned DEVICE memory unless stated.  The
+ *             library never allocates, frees or synchronises: all work is
+ *             enqueued on `stream`.  Scratch comes from the caller's workspace
+ *             `ws` of `ws_bytes` bytes, at least ckda_workspace_size(...);
+ *             its contents between calls are unspecified except for the
+ *             status word read by ckda_check_device_status.  Calls that share
+ *             a workspace must be ordered on the device (same stream).
+ *  Alignment  Every tensor pointer must be 16-byte aligned, ws 256-byte
+ *             aligned (CKDA_ERR_ALIGNMENT otherwise).
+ *  Errors     Each call returns a status.  Argument errors are detected on the
+ *             host before anything is enqueued.  Launch failures return
+ *             CKDA_ERR_CUDA.  Errors found on the device (a bounded wait that
+ *             ran out, malformed cu_seqlens) are recorded in the workspace's
+ *             status word; ckda_check_device_status reads it (synchronising
+ *             the stream).  Outputs are unspecified after any error.
+ */
+#ifndef CKDA_H_
+#define CKDA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* I/O dtypes */
+#define CKDA_F32 0
+#define CKDA_BF16 1
+
+/* status codes */
+#define CKDA_OK 0
+#define CKDA_ERR_INVALID_ARG 1 /* null required pointer, negative size, bad enum  */
+#define CKDA_ERR_UNSUPPORTED 2 /* dk or dv outside {64, 128}                       */
+#define CKDA_ERR_ALIGNMENT 3   /* a pointer breaks the alignment rule above        */
+#define CKDA_ERR_WORKSPACE 4   /* ws null or smaller than ckda_workspace_size()    */
+#define CKDA_ERR_CUDA 5        /* a kernel launch or runtime call failed           */
+#define CKDA_ERR_TIMEOUT 6     /* device: a bounded wait gave up (kernel returned)  */
+#define CKDA_ERR_DEVICE_ARG 7  /* device: malformed cu_seqlens                     */
+
+/* operations, for ckda_workspace_size */
+#define CKDA_OP_CHUNK_FWD 0
+#define CKDA_OP_CHUNK_BWD 1
+#define CKDA_OP_VARLEN_FWD 2
+
+#define CKDA_CHUNK 64
+
+/* Workspace bytes an operation needs.  For CKDA_OP_CHUNK_FWD / _BWD pass the
+ * batched shape (N ignored); for CKDA_OP_VARLEN_FWD pass B = 1, T = total
+ * tokens and N = number of sequences.  Returns 0 for invalid arguments. */
+size_t ckda_workspace_size(int op, int B, int T, int H, int dk, int dv, int N);
+
+/* Chunked forward over B independent sequences of length T.
+ *   q, k  [B,T,H,dk] io;  v [B,T,H,dv] io;  g [B,T,H,dk] f32;
+ *   sign  [B,T,H,dk] int8;  beta [B,T,H] io
+ *   S0    [B,H,dk,dv] f32, nullable (zero initial state)
+ *   o     [B,T,H,dv] io (written)
+ *   ST    [B,H,dk,dv] f32, nullable: final state
+ *   chunk_states [B,H,ceil(T/64),dk,dv] f32, nullable: the state at the start
+ *         of every 64-token chunk (true frame); pass it to ckda_chunk_bwd to
+ *         skip the backward's forward recomputation.
+ * The algorithm is the chunk-wise (WY / UT-transform) form the second source
+ * names: per 64-token chunk a unit-lower-triangular intra-chunk system is
+ * inverted, then a sequential pass carries the state across chunks. */
+int ckda_chunk_fwd(int B, int T, int H, int dk, int dv, int io_dtype,
+                   const void *q, const void *k, const void *v, const float *g,
+                   const int8_t *sign, const void *beta, const float *S0,
+                   void *o, float *ST, float *chunk_states, void *ws,
+                   size_t ws_bytes, cudaStream_t stream);
+
+/* Gradients of L(o, ST) through ckda_chunk_fwd.
+ *   dO    [B,T,H,dv] io: dL/do
+ *   dST   [B,H,dk,dv] f32, nullable (zero): dL/dST
+ *   chunk_states: nullable; the buffer ckda_chunk_fwd filled for the same
+ *         inputs (else the forward chunk states are recomputed in ws)
+ *   dq, dk_out [B,T,H,dk] io;  dv_out [B,T,H,dv] io;  dg [B,T,H,dk] f32
+ *         (dL/d log|alpha|);  dbeta [B,T,H] io;  dS0 [B,H,dk,dv] f32, nullable
+ * The sign gets no gradient (piecewise constant); dg is the exact gradient
+ * for the g given (the pages defer their gate-floor and backward convention
+ * to an appendix that is not in the text). */
+int ckda_chunk_bwd(int B, int T, int H, int dk, int dv, int io_dtype,
+                   const void *q, const void *k, const void *v, const float *g,
+                   const int8_t *sign, const void *beta, const float *S0,
+                   const void *dO, const float *dST, const float *chunk_states,
+                   void *dq, void *dk_out, void *dv_out, float *dg, void *dbeta,
+                   float *dS0, void *ws, size_t ws_bytes, cudaStream_t stream);
+
+/* One recurrent step of N*H independent states, in place (the model card's
+ * "purely recurrent" inference form).
+ *   q, k [N,H,dk] io;  v [N,H,dv] io;  g [N,H,dk] f32;  sign [N,H,dk] int8;
+ *   beta [N,H] io;  state [N,H,dk,dv] f32 read and written in place (true
+ *   frame);  o [N,H,dv] io.  No workspace. */
+int ckda_decode_step(int N, int H, int dk, int dv, int io_dtype, const void *q,
+                     const void *k, const void *v, const float *g,
+                     const int8_t *sign, const void *beta, float *state,
+                     void *o, cudaStream_t stream);
+
+/* Chunked forward over N packed documents (training packs documents back to
+ * back; the state restarts at each boundary).
+ *   cu_seqlens [N+1] int32 DEVICE: cu[0] = 0, non-decreasing, cu[N] = total_T
+ *   max_seqlen: an upper bound on every document's length (1..total_T);
+ *         a document longer than it is reported as CKDA_ERR_DEVICE_ARG
+ *   q, k [1,total_T,H,dk] ... as ckda_chunk_fwd with B = 1, T = total_T
+ *   S0, ST [N,H,dk,dv] f32, nullable: per-document initial / final states
+ * Chunks restart at each document start; a document's last chunk may be
+ * partial.  Malformed cu_seqlens are detected on the device
+ * (CKDA_ERR_DEVICE_ARG via ckda_check_device_status; no output is written). */
+int ckda_varlen_fwd(int total_T, int N, const int32_t *cu_seqlens,
+                    int max_seqlen, int H, int dk, int dv, int io_dtype,
+                    const void *q, const void *k, const void *v, const float *g,
+                    const int8_t *sign, const void *beta, const float *S0,
+                    void *o, float *ST, void *ws, size_t ws_bytes,
+                    cudaStream_t stream);
+
+/* Reads the device-side status recorded in ws by the last call that used it
+ * (synchronises `stream`).  Returns CKDA_OK, CKDA_ERR_TIMEOUT,
+ * CKDA_ERR_DEVICE_ARG or CKDA_ERR_CUDA. */
+int ckda_check_device_status(const void *ws, cudaStream_t stream);
+
+/* Static message for a status code. */
+const char *ckda_status_string(int status);
+
+/* ---- optional per-kernel timing (host side, off by default) -------------
+ * Not part of the recurrence: a measurement aid.  While enabled, every kernel
+ * launch of the library is bracketed by a pair of CUDA events recorded on the
+ * launch stream.  ckda_profile_collect synchronises those events and folds
+ * them into per-kernel totals; ckda_profile_get reads total i (name copied
+ * into `name`, at most name_len bytes with the terminator).  The library
+ * creates the events lazily (no device memory). */
+int ckda_profile_enable(int on); /* returns the previous setting */
+int ckda_profile_collect(void);  /* number of kernels with totals, or -status */
+int ckda_profile_get(int i, char *name, int name_len, int *count, double *total_ms);
+void ckda_profile_reset(void);
+
+/* Library ABI version (major * 10000 + minor * 100 + patch). */
+int ckda_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CKDA_H_ */

@@ -1,0 +1,80 @@
+"""The C-ABI library loads, exports every function include/ckda.h declares,
+and its host-side argument checks answer without touching a GPU."""
+import ctypes
+
+import pytest
+
+from chunked_gated_delta_ckda_b200 import _abi
+
+P = None
+
+
+def test_exports_every_header_symbol():
+    lib = _abi.library()
+    names = _abi.header_functions()
+    assert {"ckda_chunk_fwd", "ckda_chunk_bwd", "ckda_decode_step", "ckda_varlen_fwd",
+            "ckda_workspace_size", "ckda_check_device_status", "ckda_status_string",
+            "ckda_version"} <= set(names)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_strings_and_version():
+    assert _abi.ckda_status_string(0) == "ok"
+    for code in range(1, 8):
+        assert _abi.ckda_status_string(code) != "unknown status"
+    assert _abi.ckda_version() >= 100
+
+
+def test_workspace_size_rules():
+    ws = _abi.ckda_workspace_size
+    assert ws(0, 8, 4096, 16, 128, 128, 0) > 0
+    assert ws(1, 8, 4096, 16, 128, 128, 0) > ws(0, 8, 4096, 16, 128, 128, 0)
+    assert ws(2, 1, 65536, 16, 128, 128, 44) > 0
+    assert ws(0, 1, 100, 2, 96, 64, 0) == 0      # unsupported dk
+    assert ws(2, 2, 100, 2, 64, 64, 3) == 0      # packed call needs B == 1
+    assert ws(7, 1, 100, 2, 64, 64, 0) == 0      # unknown op
+    assert ws(0, 1, 0, 2, 64, 64, 0) > 0         # empty input still has a status block
+
+
+def _raw():
+    return _abi.library()
+
+
+def test_host_validation_without_gpu():
+    lib = _raw()
+    fake = ctypes.c_void_p(1 << 20)     # never dereferenced: the calls fail validation first
+    odd = ctypes.c_void_p((1 << 20) + 4)
+    args = [fake] * 11
+    # unsupported head size
+    assert lib.ckda_chunk_fwd(1, 64, 2, 96, 64, 0, *args, 1 << 30, None) == 2
+    # bad io dtype
+    assert lib.ckda_chunk_fwd(1, 64, 2, 64, 64, 5, *args, 1 << 30, None) == 1
+    # negative sizes
+    assert lib.ckda_chunk_fwd(-1, 64, 2, 64, 64, 0, *args, 1 << 30, None) == 1
+    # null required pointer
+    a = list(args)
+    a[0] = None
+    assert lib.ckda_chunk_fwd(1, 64, 2, 64, 64, 0, *a, 1 << 30, None) == 1
+    # misaligned tensor
+    a = list(args)
+    a[1] = odd
+    assert lib.ckda_chunk_fwd(1, 64, 2, 64, 64, 0, *a, 1 << 30, None) == 3
+    # workspace too small
+    assert lib.ckda_chunk_fwd(1, 64, 2, 64, 64, 0, *args, 16, None) == 4
+    # decode: unsupported / null
+    assert lib.ckda_decode_step(4, 2, 64, 32, 0, *([fake] * 8), None) == 2
+    assert lib.ckda_decode_step(4, 2, 64, 64, 0, *([None] * 8), None) == 1
+    # packed: bad max_seqlen, N < 0
+    v = [fake] * 9
+    assert lib.ckda_varlen_fwd(100, 2, fake, 0, 2, 64, 64, 0, *v, fake, 1 << 30, None) == 1
+    assert lib.ckda_varlen_fwd(100, -1, fake, 50, 2, 64, 64, 0, *v, fake, 1 << 30, None) == 1
+    # backward: missing gradient output
+    b = [fake] * 17
+    b[13] = None  # dg
+    assert lib.ckda_chunk_bwd(1, 64, 2, 64, 64, 1, *b, 1 << 30, None) == 1
+    # backward: workspace too small
+    b[13] = fake
+    assert lib.ckda_chunk_bwd(1, 64, 2, 64, 64, 1, *b, 16, None) == 4
+    # zero-sized decode is a no-op
+    assert lib.ckda_decode_step(0, 2, 64, 64, 0, *([None] * 8), None) == 0

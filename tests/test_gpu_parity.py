@@ -1,0 +1,305 @@
+"""CUDA path vs the fp64 oracle, element by element, through the C ABI.
+
+Small cases span several chunks and a ragged tail; full-size workloads are
+checked on sampled heads the oracle computes one by one.  Tolerances: fp32
+I/O relative L2 <= 1e-4; bf16 I/O relative L2 <= 1e-2 and max-abs <=
+2e-2 * max|ref| (per whole tensor: o, final state and every gradient)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from chunked_gated_delta_ckda_b200 import _abi, api
+from chunked_gated_delta_ckda_b200 import workloads as W
+from tests.gpu_util import (check, f64, oracle_bwd_batched, oracle_fwd_batched, random_inputs,
+                            to_dev)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    _abi.library()  # fails loudly if the library is missing
+    torch.manual_seed(0)
+
+
+def _fwd(inp, S0=None, chunk_states=False):
+    d = to_dev(inp)
+    o, ST, cs = api.chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["sign"], d["beta"],
+                              S0=None if S0 is None else S0.cuda(), save_chunk_states=chunk_states)
+    torch.cuda.synchronize()
+    return o, ST, cs
+
+
+# ---------------------------------------------------------------------------
+# forward
+# ---------------------------------------------------------------------------
+
+def test_tiny_fp32_forward_workload():
+    """The tiny fp32 workload (B=1, H=2, T=256, d=64, zero initial state)."""
+    inp = W.make(W.TINY)
+    o, ST, _ = _fwd(inp)
+    o_ref, ST_ref, _ = oracle_fwd_batched(inp)
+    check("o", o, o_ref, torch.float32)
+    check("ST", ST, ST_ref, torch.float32)
+
+
+@pytest.mark.parametrize("io", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("B,T,H,dk,dv", [(2, 200, 3, 64, 128), (1, 64, 2, 128, 64),
+                                         (3, 1, 2, 64, 64), (1, 129, 1, 128, 128)])
+def test_forward_ragged_with_state(io, B, T, H, dk, dv):
+    inp = random_inputs(B, T, H, dk, dv, io, seed=B * 1000 + T, extreme_p=0.05)
+    o, ST, cs = _fwd(inp, S0=inp["S0"], chunk_states=True)
+    o_ref, ST_ref, cs_ref = oracle_fwd_batched(inp, S0=inp["S0"], chunk=64)
+    check("o", o, o_ref, io)
+    check("ST", ST, ST_ref, io)
+    NC = (T + 63) // 64
+    cs_ref = cs_ref.reshape(B, NC, H, dk, dv).transpose(0, 2, 1, 3, 4)
+    check("chunk_states", cs, cs_ref, io)
+
+
+@pytest.mark.parametrize("io", [torch.float32, torch.bfloat16])
+def test_forward_strong_decay_exact_pair_path(io):
+    """Decay strong enough (|g| ~ 3 per token) that the factored pair sums
+    would overflow: the kernels must take the exact per-pair path."""
+    inp = random_inputs(2, 160, 2, 64, 64, io, seed=5, gscale=3.0)
+    o, ST, _ = _fwd(inp, S0=inp["S0"])
+    o_ref, ST_ref, _ = oracle_fwd_batched(inp, S0=inp["S0"])
+    check("o", o, o_ref, io)
+    check("ST", ST, ST_ref, io)
+
+
+def test_empty_and_zero_length():
+    inp = random_inputs(2, 1, 2, 64, 64, torch.float32, seed=9)
+    S0 = inp["S0"].cuda()
+    e = lambda *s, dt=torch.float32: torch.empty(*s, dtype=dt, device="cuda")
+    q = e(2, 0, 2, 64)
+    o = e(2, 0, 2, 64)
+    ST = e(2, 2, 64, 64)
+    ws = api.workspace(_abi.CKDA_OP_CHUNK_FWD, 2, 0, 2, 64, 64)
+    _abi.ckda_chunk_fwd(2, 0, 2, 64, 64, 0, q, q, q, q, e(2, 0, 2, 64, dt=torch.int8), e(2, 0, 2), S0,
+                        o, ST, None, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(ST, S0)
+    _abi.ckda_chunk_fwd(0, 5, 2, 64, 64, 0, None, None, None, None, None, None, None, None, None,
+                        None, ws)
+
+
+# ---------------------------------------------------------------------------
+# backward
+# ---------------------------------------------------------------------------
+
+def _bwd(inp, S0, dST, cs=None):
+    d = to_dev(inp)
+    r = api.chunk_bwd(d["q"], d["k"], d["v"], d["g"], d["sign"], d["beta"], d["dO"],
+                      S0=None if S0 is None else S0.cuda(), dST=None if dST is None else dST.cuda(),
+                      chunk_states=cs)
+    torch.cuda.synchronize()
+    return r
+
+
+@pytest.mark.parametrize("io", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("B,T,H,dk,dv,gscale", [(2, 150, 2, 64, 64, 0.05), (1, 256, 2, 128, 128, 0.05),
+                                                (1, 70, 3, 64, 128, 3.0), (2, 33, 1, 128, 64, 0.3)])
+def test_backward_against_oracle(io, B, T, H, dk, dv, gscale):
+    inp = random_inputs(B, T, H, dk, dv, io, seed=T + dk, gscale=gscale, extreme_p=0.05)
+    got = _bwd(inp, inp["S0"], inp["dST"])
+    ref = oracle_bwd_batched(inp, inp["dO"], S0=inp["S0"], dST=inp["dST"])
+    for key in ("dq", "dk", "dv", "dg", "dbeta", "dS0"):
+        check(key, got[key], ref[key], io)
+
+
+def test_backward_uses_saved_chunk_states():
+    io = torch.bfloat16
+    inp = random_inputs(2, 300, 2, 128, 128, io, seed=11, extreme_p=0.05)
+    _, _, cs = _fwd(inp, S0=inp["S0"], chunk_states=True)
+    a = _bwd(inp, inp["S0"], inp["dST"], cs=cs)
+    b = _bwd(inp, inp["S0"], inp["dST"], cs=None)
+    for key in a:
+        assert torch.allclose(a[key].float(), b[key].float(), rtol=1e-3, atol=1e-3), key
+
+
+def test_backward_without_state_inputs():
+    io = torch.float32
+    inp = random_inputs(1, 100, 2, 64, 64, io, seed=12)
+    got = _bwd(inp, None, None)
+    ref = oracle_bwd_batched(inp, inp["dO"])
+    for key in ("dq", "dk", "dv", "dg", "dbeta", "dS0"):
+        check(key, got[key], ref[key], io)
+
+
+# ---------------------------------------------------------------------------
+# packed variable-length forward
+# ---------------------------------------------------------------------------
+
+def _varlen(lens, io, seed, with_S0=True, gscale=0.05):
+    T = int(sum(lens))
+    inp = random_inputs(1, T, 2, 128, 128, io, seed=seed, gscale=gscale, extreme_p=0.05)
+    N = len(lens)
+    cu = torch.tensor(np.concatenate([[0], np.cumsum(lens)]), dtype=torch.int32)
+    S0 = 0.1 * torch.randn(N, 2, 128, 128, generator=torch.Generator().manual_seed(seed)) if with_S0 else None
+    d = to_dev(inp)
+    o, ST = api.varlen_fwd(d["q"], d["k"], d["v"], d["g"], d["sign"], d["beta"], cu.cuda(),
+                           max(max(lens), 1), S0=None if S0 is None else S0.cuda())
+    torch.cuda.synchronize()
+    P = lambda x: f64(x[0])
+    o_ref, ST_ref, _ = oracle.fwd(cu.numpy().astype(np.int64), P(inp["q"]), P(inp["k"]), P(inp["v"]),
+                                  P(inp["g"]), inp["sign"][0].numpy(), P(inp["beta"]), S0=f64(S0))
+    return o, ST, o_ref, ST_ref
+
+
+@pytest.mark.parametrize("io", [torch.float32, torch.bfloat16])
+def test_varlen_forward(io):
+    o, ST, o_ref, ST_ref = _varlen([1, 16, 64, 65, 200, 5, 128], io, seed=21)
+    check("o", o[0], o_ref, io)
+    check("ST", ST, ST_ref, io)
+
+
+def test_varlen_zero_length_documents_and_no_state():
+    o, ST, o_ref, ST_ref = _varlen([0, 70, 0, 3, 0], torch.float32, seed=22, with_S0=False)
+    check("o", o[0], o_ref, torch.float32)
+    check("ST", ST, ST_ref, torch.float32)
+
+
+def test_varlen_strong_decay():
+    o, ST, o_ref, ST_ref = _varlen([100, 37], torch.float32, seed=23, gscale=3.0)
+    check("o", o[0], o_ref, torch.float32)
+    check("ST", ST, ST_ref, torch.float32)
+
+
+def test_varlen_malformed_cu_seqlens_reported_on_device():
+    inp = random_inputs(1, 64, 2, 64, 64, torch.float32, seed=24)
+    d = to_dev(inp)
+    for cu in ([0, 40, 30, 64], [0, 40, 64, 70], [1, 40, 64]):
+        cu_t = torch.tensor(cu, dtype=torch.int32, device="cuda")
+        N = len(cu) - 1
+        ws = api.workspace(_abi.CKDA_OP_VARLEN_FWD, 1, 64, 2, 64, 64, N, cache=False)
+        o = torch.empty(1, 64, 2, 64, device="cuda")
+        _abi.ckda_varlen_fwd(64, N, cu_t, 64, 2, 64, 64, 0, d["q"], d["k"], d["v"], d["g"], d["sign"],
+                             d["beta"], None, o, None, ws)
+        assert _abi.ckda_check_device_status(ws) == 7
+    # a well-formed call on the same workspace clears the status
+    cu_t = torch.tensor([0, 30, 64], dtype=torch.int32, device="cuda")
+    _abi.ckda_varlen_fwd(64, 2, cu_t, 64, 2, 64, 64, 0, d["q"], d["k"], d["v"], d["g"], d["sign"],
+                         d["beta"], None, o, None, ws)
+    assert _abi.ckda_check_device_status(ws) == 0
+
+
+# ---------------------------------------------------------------------------
+# decode
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("io", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("dk,dv", [(128, 128), (64, 64), (128, 64), (64, 128)])
+def test_decode_steps(io, dk, dv):
+    N, H, steps = 5, 3, 4
+    state = 0.1 * torch.randn(N, H, dk, dv, generator=torch.Generator().manual_seed(dk + dv))
+    st_ref = f64(state)
+    st_dev = state.cuda()
+    for t in range(steps):
+        x = random_inputs(N, 1, H, dk, dv, io, seed=100 * t + dk)
+        x = {k: (v[:, 0] if k in ("q", "k", "v", "g", "sign", "beta") else v) for k, v in x.items()}
+        d = to_dev(x)
+        o = api.decode_step(d["q"], d["k"], d["v"], d["g"], d["sign"], d["beta"], st_dev)
+        torch.cuda.synchronize()
+        o_ref, st_ref = oracle.decode(f64(x["q"]), f64(x["k"]), f64(x["v"]), f64(x["g"]),
+                                      x["sign"].numpy(), f64(x["beta"]), st_ref)
+        check("o[%d]" % t, o, o_ref, io)
+        check("state[%d]" % t, st_dev, st_ref, io)
+
+
+def test_decode_continues_chunked_final_state():
+    """States cross the ABI in the true frame: decode after a chunked forward
+    equals one forward over the concatenation."""
+    io = torch.float32
+    inp = random_inputs(2, 101, 2, 64, 64, io, seed=31)
+    pre = {k: (v[:, :100] if k in ("q", "k", "v", "g", "sign", "beta") else v) for k, v in inp.items()}
+    _, ST, _ = _fwd(pre, S0=inp["S0"])
+    last = {k: inp[k][:, 100].contiguous() for k in ("q", "k", "v", "g", "sign", "beta")}
+    d = to_dev(last)
+    o = api.decode_step(d["q"], d["k"], d["v"], d["g"], d["sign"], d["beta"], ST)
+    o_ref, ST_ref, _ = oracle_fwd_batched(inp, S0=inp["S0"])
+    check("o_last", o, o_ref[:, 100], io)
+    check("ST", ST, ST_ref, io)
+
+
+# ---------------------------------------------------------------------------
+# full-size workloads, sampled heads
+# ---------------------------------------------------------------------------
+
+def _sample_heads(B, H, n, seed):
+    rng = np.random.default_rng(seed)
+    return [(int(b), int(h)) for b, h in zip(rng.integers(0, B, n), rng.integers(0, H, n))]
+
+
+def test_full_layer_fwd_bwd_sampled_heads():
+    """B=8, H=16, T=4096, d=128, bf16: the forward+backward the benchmark times,
+    checked on sampled (batch, head) pairs."""
+    w = W.LAYER_FWDBWD
+    inp = W.make(w)
+    d = to_dev(inp)
+    o, ST, cs = api.chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["sign"], d["beta"], save_chunk_states=True)
+    gr = api.chunk_bwd(d["q"], d["k"], d["v"], d["g"], d["sign"], d["beta"], d["dO"], chunk_states=cs)
+    torch.cuda.synchronize()
+    for b, h in _sample_heads(w.B, w.H, 3, seed=1):
+        sub = {k: inp[k][b:b + 1, :, h:h + 1].contiguous() for k in ("q", "k", "v", "g", "sign", "beta", "dO")}
+        o_ref, ST_ref, _ = oracle_fwd_batched(sub)
+        check("o[%d,%d]" % (b, h), o[b:b + 1, :, h:h + 1], o_ref, w.io_dtype)
+        check("ST[%d,%d]" % (b, h), ST[b:b + 1, h:h + 1], ST_ref, w.io_dtype)
+        ref = oracle_bwd_batched(sub, sub["dO"])
+        for key in ("dq", "dk", "dv", "dg", "dbeta"):
+            check("%s[%d,%d]" % (key, b, h), gr[key][b:b + 1, :, h:h + 1], ref[key], w.io_dtype)
+        check("dS0[%d,%d]" % (b, h), gr["dS0"][b:b + 1, h:h + 1], ref["dS0"], w.io_dtype)
+
+
+def test_full_varlen_sampled():
+    """65536 packed tokens (geometric document lengths), H=16, d=128, bf16."""
+    w = W.VARLEN
+    inp = W.make_varlen(w)
+    d = to_dev(inp)
+    cu = inp["cu_seqlens"]
+    o, ST = api.varlen_fwd(d["q"], d["k"], d["v"], d["g"], d["sign"], d["beta"], cu.cuda(),
+                           max(inp["lens"]))
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(3)
+    docs = rng.choice(len(inp["lens"]), 3, replace=False)
+    for i in docs:
+        a, b = int(cu[i]), int(cu[i + 1])
+        h = int(rng.integers(0, w.H))
+        sl = lambda x: f64(x[0, a:b, h:h + 1])
+        o_ref, ST_ref, _ = oracle.fwd([0, b - a], sl(inp["q"]), sl(inp["k"]), sl(inp["v"]), sl(inp["g"]),
+                                      inp["sign"][0, a:b, h:h + 1].numpy(), sl(inp["beta"]))
+        check("o[doc %d]" % i, o[0, a:b, h:h + 1], o_ref, w.io_dtype)
+        check("ST[doc %d]" % i, ST[i:i + 1, h:h + 1], ST_ref, w.io_dtype)
+
+
+def test_full_long_sequence_sampled():
+    """One 65536-token sequence with an N(0, 0.1^2) initial state."""
+    w = W.LONG
+    inp = W.make(w)
+    d = to_dev(inp)
+    o, ST, _ = api.chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["sign"], d["beta"], S0=d["S0"])
+    torch.cuda.synchronize()
+    h = 5
+    sub = {k: inp[k][:, :, h:h + 1].contiguous() for k in ("q", "k", "v", "g", "sign", "beta")}
+    o_ref, ST_ref, _ = oracle_fwd_batched(sub, S0=inp["S0"][:, h:h + 1])
+    check("o", o[:, :, h:h + 1], o_ref, w.io_dtype)
+    check("ST", ST[:, h:h + 1], ST_ref, w.io_dtype)
+
+
+def test_full_decode_steps():
+    """N=256, H=16, d=128 states, bf16 I/O, a few consecutive steps, all heads."""
+    w = W.DECODE
+    state = W.make_decode_state(w)
+    st_dev = state.cuda()
+    st_ref = f64(state)
+    for t in range(3):
+        x = W.make_decode_step(w, t)
+        d = to_dev(x)
+        o = api.decode_step(d["q"], d["k"], d["v"], d["g"], d["sign"], d["beta"], st_dev)
+        torch.cuda.synchronize()
+        o_ref, st_ref = oracle.decode(f64(x["q"]), f64(x["k"]), f64(x["v"]), f64(x["g"]),
+                                      x["sign"].numpy(), f64(x["beta"]), st_ref)
+        check("o[%d]" % t, o, o_ref, w.io_dtype)
+    check("state", st_dev, st_ref, w.io_dtype)
