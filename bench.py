@@ -206,7 +206,8 @@ def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     wl = W.LAYER_FWDBWD
-    w = W.Workload(**{**wl.__dict__, "seed": rank_seed(wl.seed, rank)})
+    w = W.Workload(**{**wl.__dict__, "seed": rank_seed(wl.seed, rank),
+                      "B": args.batch or wl.B})
     inp = W.make(w)
     B, T, H = w.B, w.T, w.H
     tokens = B * T
@@ -250,7 +251,7 @@ def run_ours(args, rank, world, local_rank):
                  "tensor_frac": t_tc / ms_max, "binding_frac": max(t_hbm, t_tc) / ms_max}
 
     # end to end through the public API with host buffers
-    e2e = run_e2e(inp, dev, args, world)
+    e2e = None if args.no_e2e else run_e2e(inp, dev, args, world)
 
     out = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
@@ -379,6 +380,9 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer pass")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="override B (profiling a smaller case; not a bench line)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
