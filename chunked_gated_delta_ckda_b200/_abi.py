@@ -26,7 +26,7 @@ CKDA_CHUNK = 64
 
 STATUS = {0: "CKDA_OK", 1: "CKDA_ERR_INVALID_ARG", 2: "CKDA_ERR_UNSUPPORTED",
           3: "CKDA_ERR_ALIGNMENT", 4: "CKDA_ERR_WORKSPACE", 5: "CKDA_ERR_CUDA",
-          6: "CKDA_ERR_TIMEOUT", 7: "CKDA_ERR_DEVICE_ARG"}
+          6: "CKDA_ERR_TIMEOUT", 7: "CKDA_ERR_DEVICE_ARG", 8: "CKDA_ERR_NOALLOC_CAPACITY"}
 
 _lib = None
 
@@ -51,6 +51,7 @@ def _load():
         lib.ckda_chunk_bwd.argtypes = [I] * 6 + [P] * 17 + [Z, P]
         lib.ckda_decode_step.argtypes = [I] * 5 + [P] * 9
         lib.ckda_varlen_fwd.argtypes = [I, I, P, I, I, I, I, I] + [P] * 10 + [Z, P]
+        lib.ckda_chunk_fwd_noalloc.argtypes = [I] * 6 + [P] * 11
         lib.ckda_check_device_status.argtypes = [P, P]
         lib.ckda_status_string.argtypes = [I]
         lib.ckda_status_string.restype = ctypes.c_char_p
@@ -62,7 +63,7 @@ def _load():
         lib.ckda_profile_reset.argtypes = []
         lib.ckda_profile_reset.restype = None
         for f in ("ckda_chunk_fwd", "ckda_chunk_bwd", "ckda_decode_step", "ckda_varlen_fwd",
-                  "ckda_check_device_status", "ckda_version", "ckda_profile_enable",
+                  "ckda_chunk_fwd_noalloc", "ckda_check_device_status", "ckda_version", "ckda_profile_enable",
                   "ckda_profile_collect", "ckda_profile_get"):
             getattr(lib, f).restype = I
         _lib = lib
@@ -138,6 +139,15 @@ def ckda_varlen_fwd(total_T, N, cu_seqlens, max_seqlen, H, dk, dv, io_dtype, q, 
                                    _p(q), _p(k), _p(v), _p(g), _p(sign), _p(beta), _p(S0), _p(o),
                                    _p(ST), _p(ws), _nbytes(ws, ws_bytes), _s(stream)),
            "ckda_varlen_fwd")
+
+
+def ckda_chunk_fwd_noalloc(B, T, H, dk, dv, io_dtype, q, k, v, g, sign, beta, S0, o, ST,
+                           chunk_states, stream=None):
+    """ckda_chunk_fwd without a workspace: the library's fixed scratch array
+    is used instead (for callers that cannot allocate device memory)."""
+    _check(_load().ckda_chunk_fwd_noalloc(B, T, H, dk, dv, io_dtype, _p(q), _p(k), _p(v), _p(g),
+                                          _p(sign), _p(beta), _p(S0), _p(o), _p(ST),
+                                          _p(chunk_states), _s(stream)), "ckda_chunk_fwd_noalloc")
 
 
 def ckda_check_device_status(ws, stream=None) -> int:

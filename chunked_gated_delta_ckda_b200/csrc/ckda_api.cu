@@ -251,6 +251,8 @@ const char *ckda_status_string(int status) {
     case CKDA_ERR_CUDA: return "CUDA launch or runtime error";
     case CKDA_ERR_TIMEOUT: return "a bounded device wait gave up";
     case CKDA_ERR_DEVICE_ARG: return "malformed cu_seqlens (found on the device)";
+    case CKDA_ERR_NOALLOC_CAPACITY:
+      return "problem does not fit the fixed scratch of ckda_chunk_fwd_noalloc";
     default: return "unknown status";
   }
 }

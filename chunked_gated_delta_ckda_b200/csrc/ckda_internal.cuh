@@ -179,6 +179,9 @@ cudaError_t build_chunk_table(const int32_t *cu, int N, int total_T, int max_seq
                               DevStatus *status, cudaStream_t s);
 size_t v1_fwd_scratch_floats(int dk, int dv);
 cudaError_t v1_intra(const FwdArgs &a, bool bf16, float *scratch, cudaStream_t s);
+size_t v1_fwd_scratch_floats_per_cta(int dk, int dv);
+cudaError_t v1_intra_on_ctas(const FwdArgs &a, bool bf16, float *scratch, int ctas,
+                             cudaStream_t s);
 cudaError_t v1_state_fwd(const FwdArgs &a, bool bf16, bool write_o, float *states_out,
                          cudaStream_t s);
 cudaError_t v1_backward(const BwdArgs &a, bool bf16, cudaStream_t s);

@@ -681,6 +681,32 @@ cudaError_t launch_backward(const BwdArgs &a, cudaStream_t s) {
 
 size_t v1_fwd_scratch_floats(int dk, int dv) { return fwd_scratch_floats(dk, dv) * kBwdCtas; }
 
+// Same intra-chunk kernel on a caller-chosen number of persistent CTAs (each
+// needs fwd_scratch_floats(dk, dv) floats of scratch); used by the entry
+// point that runs out of a fixed static scratch area.
+cudaError_t v1_intra_on_ctas(const FwdArgs &a, bool bf16, float *scratch, int ctas,
+                             cudaStream_t s) {
+  const size_t sm_intra = intra_smem_floats(0) * sizeof(float);
+  if (bf16) {
+    cudaError_t e = cudaFuncSetAttribute(intra_fwd_kernel<__nv_bfloat16>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)sm_intra);
+    if (e != cudaSuccess) return e;
+    ProfScope prof("v1_intra", s);
+    intra_fwd_kernel<__nv_bfloat16><<<ctas, NT, sm_intra, s>>>(a, scratch);
+  } else {
+    cudaError_t e = cudaFuncSetAttribute(intra_fwd_kernel<float>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)sm_intra);
+    if (e != cudaSuccess) return e;
+    ProfScope prof("v1_intra", s);
+    intra_fwd_kernel<float><<<ctas, NT, sm_intra, s>>>(a, scratch);
+  }
+  return cudaGetLastError();
+}
+
+size_t v1_fwd_scratch_floats_per_cta(int dk, int dv) { return fwd_scratch_floats(dk, dv); }
+
 cudaError_t v1_intra(const FwdArgs &a, bool bf16, float *scratch, cudaStream_t s) {
   return bf16 ? launch_intra<__nv_bfloat16>(a, scratch, s) : launch_intra<float>(a, scratch, s);
 }

@@ -75,6 +75,7 @@ extern "C" {
 #define CKDA_ERR_CUDA 5        /* a kernel launch or runtime call failed           */
 #define CKDA_ERR_TIMEOUT 6     /* device: a bounded wait gave up (kernel returned)  */
 #define CKDA_ERR_DEVICE_ARG 7  /* device: malformed cu_seqlens                     */
+#define CKDA_ERR_NOALLOC_CAPACITY 8 /* problem too large for the no-alloc scratch  */
 
 /* operations, for ckda_workspace_size */
 #define CKDA_OP_CHUNK_FWD 0
@@ -149,6 +150,34 @@ int ckda_varlen_fwd(int total_T, int N, const int32_t *cu_seqlens,
                     const int8_t *sign, const void *beta, const float *S0,
                     void *o, float *ST, void *ws, size_t ws_bytes,
                     cudaStream_t stream);
+
+/* ---- chunked forward without any allocation --------------------------------
+ * The pages have no counterpart to this call; it serves callers that cannot
+ * allocate device memory: a plug-in inside a host application that owns every
+ * device allocation (a fixed pool or its own allocator, and no workspace to
+ * hand over), or a latency-critical path that must not call cudaMalloc, which
+ * can synchronise the device and fail at run time.
+ *
+ * Same arguments, semantics and outputs as ckda_chunk_fwd, minus the
+ * workspace: scratch comes from one fixed array of CKDA_NOALLOC_SCRATCH_BYTES
+ * that the library holds on every GPU that loads it, until the process exits.
+ * Nothing is allocated or freed by the call.
+ *  - Capacity: one 148 KiB record per (64-token chunk, head) at dk = dv = 128
+ *    (72 KiB at 64) plus ~4.7 MiB of fixed scratch must fit: e.g. 194
+ *    chunk-heads at d = 128 (B=1, T=4096, H=3).  Larger problems return
+ *    CKDA_ERR_NOALLOC_CAPACITY before anything is enqueued.
+ *  - The first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before any stream capture starts.
+ *  - Every call uses the same array, which keeps the previous call's
+ *    contents; calls whose work may overlap on the GPU (other streams, other
+ *    host threads) race on it and must be serialised by the caller. */
+#define CKDA_NOALLOC_SCRATCH_BYTES (32u << 20)
+int ckda_chunk_fwd_noalloc(int B, int T, int H, int dk, int dv, int io_dtype,
+                           const void *q, const void *k, const void *v,
+                           const float *g, const int8_t *sign, const void *beta,
+                           const float *S0, void *o, float *ST,
+                           float *chunk_states, cudaStream_t stream);
 
 /* Reads the device-side status recorded in ws by the last call that used it
  * (synchronises `stream`).  Returns CKDA_OK, CKDA_ERR_TIMEOUT,

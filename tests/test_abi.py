@@ -21,7 +21,7 @@ def test_exports_every_header_symbol():
 
 def test_status_strings_and_version():
     assert _abi.ckda_status_string(0) == "ok"
-    for code in range(1, 8):
+    for code in range(1, 9):
         assert _abi.ckda_status_string(code) != "unknown status"
     assert _abi.ckda_version() >= 100
 
