@@ -85,6 +85,12 @@ int check_ws(const void *ws, size_t ws_bytes, size_t need) {
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? CKDA_OK : CKDA_ERR_CUDA; }
 
+// bf16 I/O at dk = dv = 128 runs on the tensor cores; other shapes and fp32
+// I/O (whose 1e-4 accuracy target bf16 operands cannot meet) on CUDA cores.
+bool use_tensor_cores(int io_dtype, int dk, int dv) {
+  return io_dtype == CKDA_BF16 && dk == 128 && dv == 128;
+}
+
 #define CKDA_TRY(expr)                          \
   do {                                          \
     int _rc = (expr);                           \
@@ -128,6 +134,11 @@ int ckda_chunk_fwd(int B, int T, int H, int dk, int dv, int io_dtype, const void
   a.intra = reinterpret_cast<float *>(w + L.intra);
   a.status = reinterpret_cast<DevStatus *>(w);
   const bool bf16 = io_dtype == CKDA_BF16;
+  if (use_tensor_cores(io_dtype, dk, dv)) {
+    CKDA_CUDA(tc_forward(a, reinterpret_cast<unsigned char *>(w + L.intra),
+                         reinterpret_cast<float *>(w + L.fscratch), true, chunk_states, stream));
+    return CKDA_OK;
+  }
   CKDA_CUDA(v1_intra(a, bf16, reinterpret_cast<float *>(w + L.fscratch), stream));
   CKDA_CUDA(v1_state_fwd(a, bf16, true, chunk_states, stream));
   return CKDA_OK;
@@ -225,6 +236,11 @@ int ckda_varlen_fwd(int total_T, int N, const int32_t *cu_seqlens, int max_seqle
                               reinterpret_cast<int32_t *>(w + L.seq_first),
                               reinterpret_cast<DevStatus *>(w), stream));
   const bool bf16 = io_dtype == CKDA_BF16;
+  if (use_tensor_cores(io_dtype, dk, dv)) {
+    CKDA_CUDA(tc_forward(a, reinterpret_cast<unsigned char *>(w + L.intra),
+                         reinterpret_cast<float *>(w + L.fscratch), true, nullptr, stream));
+    return CKDA_OK;
+  }
   CKDA_CUDA(v1_intra(a, bf16, reinterpret_cast<float *>(w + L.fscratch), stream));
   CKDA_CUDA(v1_state_fwd(a, bf16, true, nullptr, stream));
   return CKDA_OK;

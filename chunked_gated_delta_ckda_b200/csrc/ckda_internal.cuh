@@ -185,6 +185,10 @@ cudaError_t v1_intra_on_ctas(const FwdArgs &a, bool bf16, float *scratch, int ct
 cudaError_t v1_state_fwd(const FwdArgs &a, bool bf16, bool write_o, float *states_out,
                          cudaStream_t s);
 cudaError_t v1_backward(const BwdArgs &a, bool bf16, cudaStream_t s);
+size_t tc_fwd_fallback_floats(int ctas);
+int tc_intra_ctas();
+cudaError_t tc_forward(const FwdArgs &f, unsigned char *recs, float *fb, bool write_o,
+                       float *states_out, cudaStream_t s);
 cudaError_t decode_step(int N, int H, int dk, int dv, bool bf16, const void *q,
                         const void *k, const void *v, const float *g, const int8_t *sign,
                         const void *beta, float *state, void *o, cudaStream_t s);

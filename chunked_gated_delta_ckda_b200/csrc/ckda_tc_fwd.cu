@@ -1,0 +1,700 @@
+// ckda_tc_fwd.cu -- chunked CKDA forward on 5th-generation tensor cores
+// (tcgen05, TMEM accumulators), bf16 I/O, dk = dv = 128.
+//
+// Same algorithm as the CUDA-core path (chunk-wise WY / UT form with the
+// gate sign folded per chunk; "Complex KDA: Understanding and Enhancing the
+// Expressivity of Kimi Delta Attention", section 2, and the
+// "openeurollm/complex-kda-1.3B-100B" model card introduction), split in two
+// kernels:
+//
+//  tc_intra_kernel  (persistent, 2 CTAs / SM, one (chunk, head) at a time)
+//    prep on CUDA cores: chunk-local cumsum Gam and sign product p, the
+//      factored operands Q~ = q' e^{Gam-Gam_m}, K~l = k' e^{Gam-Gam_m},
+//      K~r = k' e^{Gam_m-Gam}, KG = k' e^Gam, QG = q' e^Gam,
+//      Khat = p_C k' e^{Gam_C-Gam}, d = p_C e^{Gam_C}
+//    MMA1  [A_q ; A] = [Q~ ; K~l] K~r^T           (M=128, N=64, K=128)
+//    triangular inverse M = (I + Diag(beta) A)^{-1}, 16x16 blocks, fp32
+//    MMA2  W^T = KG^T T^T, U0^T = V^T T^T          (M=128, N=64, K=64 each)
+//    -> one record per (chunk, head), written in the shared-memory image
+//       the state kernel consumes (128-byte-swizzled operand tiles).
+//
+//  tc_state_kernel  (one CTA per (sequence, head), sequential over chunks)
+//    the state is kept transposed, S^T (lanes = value channel), fp32 in TMEM;
+//    records arrive by one bulk async copy each, double-buffered.
+//    MMA3  [(W S)^T | (QG S)^T] = S^T [W^T | QG^T]  (M=128, N=128, K=128)
+//    U^T = U0^T - (W S)^T                           (CUDA cores, -> bf16 tile)
+//    MMA4  O^T += U^T A_q^T                         (M=128, N=64,  K=64)
+//    MMA5  S^T += U^T Khat                          (M=128, N=128, K=64)
+//    S^T <- Diag(d_next) S^T and its bf16 copy for the next MMA3.
+//
+// Chunks whose decay is too strong for the factored operands (any
+// |Gam_r - Gam_m| > kTau) compute A and A_q exactly per pair on CUDA cores.
+#include <cmath>
+
+#include "ckda_tc.cuh"
+
+namespace ckda {
+namespace {
+
+using namespace tc;
+
+constexpr int D = 128;
+constexpr float kTau = 40.f;
+constexpr float kLog2e = 1.4426950408889634f;
+
+// record layout (bytes); each tile 1024-byte aligned inside the record
+constexpr uint32_t R1 = 0;       // [W^T | QG^T]: MN-major B tile, K = c (128), N = r' (128)
+constexpr uint32_t R2 = 32768;   // U0^T: K-major tile [v][s] (128 x 64)
+constexpr uint32_t R3 = 49152;   // A_q: K-major tile [r][s] (64 x 64)
+constexpr uint32_t R4 = 57344;   // Khat^T: K-major tile [c][s] (128 x 64)
+constexpr uint32_t R5 = 73728;   // d[128] fp32
+constexpr uint32_t REC = 74240;  // bytes per (chunk, head) record
+constexpr uint32_t REC_PAD = 74752;  // record slot in shared memory (73 x 1024)
+
+__device__ __forceinline__ float fast_exp(float x) { return exp2f(x * kLog2e); }
+
+__device__ __forceinline__ void st_bf16(unsigned char *base, uint32_t off, float x) {
+  *reinterpret_cast<__nv_bfloat16 *>(base + off) = __float2bfloat16_rn(x);
+}
+
+// ===========================================================================
+// intra-chunk kernel
+// ===========================================================================
+constexpr int kIntraThreads = 256;
+// shared memory map (offsets from a 1024-aligned base)
+constexpr uint32_t I_A1 = 0;          // [Q~; K~l]  K-major 128 x 128      32 KiB
+constexpr uint32_t I_B1 = 32768;      // K~r        K-major  64 x 128      16 KiB
+constexpr uint32_t I_KG = 49152;      // KG         MN-major A (K=64, M=128) 16 KiB
+constexpr uint32_t I_V = 65536;       // V          MN-major A (K=64, M=128) 16 KiB
+constexpr uint32_t I_T = 81920;       // T          K-major 64 x 64         8 KiB
+constexpr uint32_t I_MISC = 90112;    // small arrays
+constexpr uint32_t I_NF = 0;          // fp32 N [64][65]  (reuses A1 after MMA1)
+constexpr uint32_t I_MF = 16640;      // fp32 M [64][65]  (reuses A1/B1 after MMA1)
+constexpr int LDF = 65;
+
+struct IntraMisc {
+  uint64_t mbar1, mbar2, mfin;
+  uint32_t tmem;
+  int flag;
+  float beta[64];
+  float totG[2][128];
+  uint32_t totP[2][128];
+  float Gm[128], eGm[128], eCm[128], GamC[128];
+  uint32_t pC[128];
+  float X[3][16][16];
+};
+
+struct TcArgs {
+  FwdArgs f;
+  unsigned char *recs;  // (chunk, head) records
+  float *fb;            // per-CTA fallback scratch: Gam, k', q' (3 x 64 x 128 fp32)
+  float *states_out;    // chunk-start states (batched only) or null
+  bool write_o;
+};
+
+__global__ void __launch_bounds__(kIntraThreads, 2) tc_intra_kernel(TcArgs ta) {
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char *sm = reinterpret_cast<unsigned char *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  IntraMisc &ms = *reinterpret_cast<IntraMisc *>(sm + I_MISC);
+  const FwdArgs &a = ta.f;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int H = a.H;
+  const __nv_bfloat16 *q = (const __nv_bfloat16 *)a.q, *k = (const __nv_bfloat16 *)a.k;
+  const __nv_bfloat16 *v = (const __nv_bfloat16 *)a.v, *beta = (const __nv_bfloat16 *)a.beta;
+
+  if (tid == 0) {
+    mbar_init(&ms.mbar1, 1);
+    mbar_init(&ms.mbar2, 1);
+    mbar_init(&ms.mfin, 1);
+    mbar_fence_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(&ms.tmem, 256);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ms.tmem;
+  const uint32_t sA1 = smem_u32(sm + I_A1), sB1 = smem_u32(sm + I_B1);
+  const uint32_t sKG = smem_u32(sm + I_KG), sV = smem_u32(sm + I_V), sT = smem_u32(sm + I_T);
+  float *Nf = reinterpret_cast<float *>(sm + I_NF);
+  float *Mf = reinterpret_cast<float *>(sm + I_MF);
+  float *fb = ta.fb + (size_t)blockIdx.x * 3 * 64 * D;
+
+  const int c = tid & 127, hf = tid >> 7;
+  const int nitems = a.map.n_chunks() * H;
+  uint32_t it = 0;
+  bool abort = false;
+  for (int item = blockIdx.x; item < nitems && !abort; item += gridDim.x, ++it) {
+    const int cid = item / H, h = item % H;
+    int seq, len, jl;
+    int64_t tok0;
+    a.map.info(cid, seq, tok0, len, jl);
+    unsigned char *rec = ta.recs + (size_t)item * REC;
+
+    // ---------------- prep, pass 1: local scans over 32 rows ----------------
+    float G[32];
+    uint32_t kq[32];   // bf16 k (low half) and q (high half) of each row
+    uint32_t neg = 0;  // bit i: sign of row 32*hf + i is negative
+    {
+      float acc = 0.f;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const int r = 32 * hf + i;
+        float gg = 0.f;
+        uint32_t kk = 0, qq = 0;
+        int8_t sg = 1;
+        if (r < len) {
+          const size_t off = ((size_t)(tok0 + r) * H + h) * D + c;
+          gg = a.g[off];
+          sg = a.sign[off];
+          kk = __bfloat16_as_ushort(k[off]);
+          qq = __bfloat16_as_ushort(q[off]);
+        }
+        acc += gg;
+        G[i] = acc;
+        kq[i] = kk | (qq << 16);
+        if (sg < 0) neg |= 1u << i;
+      }
+    }
+    // prefix parity of the sign bits
+    uint32_t par = 0, pre = 0;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      par ^= (neg >> i) & 1u;
+      pre |= par << i;
+    }
+    ms.totG[hf][c] = G[31];
+    ms.totP[hf][c] = par;
+    // V tile (MN-major A operand, K = token j, M = value channel)
+    for (int e = tid; e < 64 * 16; e += kIntraThreads) {
+      const int j = e >> 4, cc = e & 15;
+      uint4 val = make_uint4(0, 0, 0, 0);
+      if (j < len)
+        val = *reinterpret_cast<const uint4 *>(v + ((size_t)(tok0 + j) * H + h) * D + cc * 8);
+      *reinterpret_cast<uint4 *>(sm + I_V + mnmaj_off(j, cc * 8, 64)) = val;
+    }
+    if (tid < 64) ms.beta[tid] = tid < len ? __bfloat162float(beta[(size_t)(tok0 + tid) * H + h]) : 0.f;
+    __syncthreads();
+
+    // ---------------- carry, reference row, range check ----------------
+    if (hf == 1) {
+      const float cg = ms.totG[0][c];
+      const uint32_t cp = ms.totP[0][c] ? 0xffffffffu : 0u;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) G[i] += cg;
+      pre ^= cp;
+    }
+    const float Gm = ms.totG[0][c];
+    const float GC = ms.totG[0][c] + ms.totG[1][c];
+    const uint32_t pCneg = ms.totP[0][c] ^ ms.totP[1][c];
+    int bad = 0;
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+      if (!(fabsf(G[i] - Gm) <= kTau)) bad = 1;
+    const bool fast = !__syncthreads_or(bad);
+    const float eGm = fast_exp(Gm);
+    const float eCm = fast_exp(GC - Gm);
+    const float pCs = pCneg ? -1.f : 1.f;
+    if (hf == 0) {
+      reinterpret_cast<float *>(rec + R5)[c] = pCs * fast_exp(GC);
+      ms.Gm[c] = Gm;
+      ms.GamC[c] = GC;
+      ms.pC[c] = pCneg;
+    }
+
+    // ---------------- prep, pass 2: operand tiles and record tiles ----------------
+    if (fast) {
+      uint32_t qg_pack[16], kh_pack[16];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const int r = 32 * hf + i;
+        const float p = ((pre >> i) & 1u) ? -1.f : 1.f;
+        const float kp = p * __uint_as_float(kq[i] << 16), qp = p * __uint_as_float(kq[i] & 0xffff0000u);
+        const float el = fast_exp(G[i] - Gm);
+        const float er = __frcp_rn(el);
+        const float ql = qp * el, kl = kp * el, kr = kp * er;
+        st_bf16(sm + I_A1, kmaj_off(r, c, 128), ql);
+        st_bf16(sm + I_A1, kmaj_off(64 + r, c, 128), kl);
+        st_bf16(sm + I_B1, kmaj_off(r, c, 64), kr);
+        st_bf16(sm + I_KG, mnmaj_off(r, c, 64), kl * eGm);
+        const float qg = ql * eGm, kh = pCs * kr * eCm;
+        if (i & 1) {
+          qg_pack[i >> 1] |= (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(qg)) << 16;
+          kh_pack[i >> 1] |= (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(kh)) << 16;
+        } else {
+          qg_pack[i >> 1] = __bfloat16_as_ushort(__float2bfloat16_rn(qg));
+          kh_pack[i >> 1] = __bfloat16_as_ushort(__float2bfloat16_rn(kh));
+        }
+      }
+      // QG^T row c (N index 64 + r) and Khat^T row c (K index r): 4 chunks each
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const uint4 vq = make_uint4(qg_pack[4 * m], qg_pack[4 * m + 1], qg_pack[4 * m + 2], qg_pack[4 * m + 3]);
+        const uint4 vk = make_uint4(kh_pack[4 * m], kh_pack[4 * m + 1], kh_pack[4 * m + 2], kh_pack[4 * m + 3]);
+        *reinterpret_cast<uint4 *>(rec + R1 + mnmaj_off(c, 64 + 32 * hf + 8 * m, 128)) = vq;
+        *reinterpret_cast<uint4 *>(rec + R4 + kmaj_off(c, 32 * hf + 8 * m, 128)) = vk;
+      }
+    } else {
+      // exact path: keep Gam, k', q' for the per-pair sums; KG, QG, Khat direct
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const int r = 32 * hf + i;
+        const float p = ((pre >> i) & 1u) ? -1.f : 1.f;
+        const float kp = p * __uint_as_float(kq[i] << 16), qp = p * __uint_as_float(kq[i] & 0xffff0000u);
+        fb[r * D + c] = G[i];
+        fb[64 * D + r * D + c] = kp;
+        fb[128 * D + r * D + c] = qp;
+        const float E = fast_exp(G[i]);
+        st_bf16(sm + I_KG, mnmaj_off(r, c, 64), kp * E);
+        st_bf16(rec, R1 + mnmaj_off(c, 64 + r, 128), qp * E);
+        st_bf16(rec, R4 + kmaj_off(c, r, 128), pCs * kp * fast_exp(GC - G[i]));
+      }
+    }
+    fence_async_smem();
+    __syncthreads();
+
+    // ---------------- A_q and N = Diag(beta) A ----------------
+    if (fast) {
+      if (tid == 0) {
+        tc_fence_after();
+        const uint32_t id = idesc_bf16(128, 64, false, false);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t ad = sdesc(sA1 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+          const uint64_t bd = sdesc(sB1 + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024);
+          mma_bf16(tmem, ad, bd, id, kk > 0);
+        }
+        mma_commit(&ms.mbar1);
+      }
+      const bool ok = mbar_wait(&ms.mbar1, it & 1, a.status, 101);
+      if (__syncthreads_or(!ok)) { abort = true; break; }
+      tc_fence_after();
+      const int qd = warp & 3, ch = warp >> 2;
+      const int L = 32 * qd + lane;
+      float x[16], y[16];
+      tmem_ld16(tmem + ((uint32_t)(32 * qd) << 16) + 32 * ch, x);
+      tmem_ld16(tmem + ((uint32_t)(32 * qd) << 16) + 32 * ch + 16, y);
+      tmem_wait_ld();
+      if (L < 64) {
+        const int r = L;
+        uint32_t pk[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const int s0 = 32 * ch + 2 * j;
+          const float v0 = (j < 8 ? x[2 * j] : y[2 * j - 16]);
+          const float v1 = (j < 8 ? x[2 * j + 1] : y[2 * j + 1 - 16]);
+          pk[j] = pack_bf16(s0 <= r ? v0 : 0.f, s0 + 1 <= r ? v1 : 0.f);
+        }
+#pragma unroll
+        for (int m = 0; m < 4; ++m)
+          *reinterpret_cast<uint4 *>(rec + R3 + kmaj_off(r, 32 * ch + 8 * m, 64)) =
+              make_uint4(pk[4 * m], pk[4 * m + 1], pk[4 * m + 2], pk[4 * m + 3]);
+      }
+      tc_fence_before();
+      __syncthreads();  // all TMEM reads of MMA1's accumulator done before A1 is reused
+      if (L >= 64) {
+        const int r = L - 64;
+        const float br = ms.beta[r];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const int s = 32 * ch + j;
+          const float val = j < 16 ? x[j] : y[j - 16];
+          Nf[r * LDF + s] = s < r ? br * val : 0.f;
+        }
+      }
+    } else {
+      // exact per-pair sums (fallback scratch is per CTA, global)
+      for (int e = tid; e < 64 * 64; e += kIntraThreads) {
+        const int r = e >> 6, s = e & 63;
+        float aa = 0.f, aq = 0.f;
+        if (s <= r)
+          for (int cc = 0; cc < D; ++cc) {
+            const float ex = expf(fb[r * D + cc] - fb[s * D + cc]);
+            const float ks = fb[64 * D + s * D + cc] * ex;
+            aa += fb[64 * D + r * D + cc] * ks;
+            aq += fb[128 * D + r * D + cc] * ks;
+          }
+        Nf[r * LDF + s] = s < r ? ms.beta[r] * aa : 0.f;
+        st_bf16(rec, R3 + kmaj_off(r, s, 64), s <= r ? aq : 0.f);
+      }
+    }
+    __syncthreads();
+
+    // ---------------- M = (I + N)^{-1}, 16 x 16 blocks ----------------
+    for (int e = tid; e < 64 * 64; e += kIntraThreads) Mf[(e >> 6) * LDF + (e & 63)] = 0.f;
+    __syncthreads();
+    if (tid < 64) {
+      const int bI = tid >> 4, j = tid & 15, o = 16 * bI;
+      float xc[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        float s = 0.f;
+#pragma unroll
+        for (int kk = 0; kk < i; ++kk) s += Nf[(o + i) * LDF + o + kk] * xc[kk];
+        xc[i] = (i == j) ? 1.f : (i < j ? 0.f : -s);
+      }
+#pragma unroll
+      for (int i = 0; i < 16; ++i) Mf[(o + i) * LDF + o + j] = xc[i];
+    }
+    __syncthreads();
+    for (int d = 1; d < 4; ++d) {
+      const int nb = 4 - d;
+      for (int e = tid; e < nb * 256; e += kIntraThreads) {
+        const int J = e >> 8, I = J + d, aa = (e >> 4) & 15, bb = e & 15;
+        float s = 0.f;
+        for (int u = 16 * J; u < 16 * I; ++u) s += Nf[(16 * I + aa) * LDF + u] * Mf[u * LDF + 16 * J + bb];
+        ms.X[J][aa][bb] = s;
+      }
+      __syncthreads();
+      for (int e = tid; e < nb * 256; e += kIntraThreads) {
+        const int J = e >> 8, I = J + d, aa = (e >> 4) & 15, bb = e & 15;
+        float s = 0.f;
+#pragma unroll
+        for (int t = 0; t < 16; ++t) s += Mf[(16 * I + aa) * LDF + 16 * I + t] * ms.X[J][t][bb];
+        Mf[(16 * I + aa) * LDF + 16 * J + bb] = -s;
+      }
+      __syncthreads();
+    }
+    // T = M Diag(beta) -> bf16 K-major B tile [r][j]
+    {
+      const int r = tid >> 2, j0 = (tid & 3) * 16;
+      uint32_t pk[8];
+#pragma unroll
+      for (int m = 0; m < 8; ++m)
+        pk[m] = pack_bf16(Mf[r * LDF + j0 + 2 * m] * ms.beta[j0 + 2 * m],
+                          Mf[r * LDF + j0 + 2 * m + 1] * ms.beta[j0 + 2 * m + 1]);
+      *reinterpret_cast<uint4 *>(sm + I_T + kmaj_off(r, j0, 64)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      *reinterpret_cast<uint4 *>(sm + I_T + kmaj_off(r, j0 + 8, 64)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+    }
+    fence_async_smem();
+    __syncthreads();
+
+    // ---------------- W^T = KG^T T^T, U0^T = V^T T^T ----------------
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t id = idesc_bf16(128, 64, true, false);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        const uint64_t bd = sdesc(sT + kk * 32, 16, 1024);
+        mma_bf16(tmem + 64, sdesc(sKG + kk * 2048, 8192, 1024), bd, id, kk > 0);
+        mma_bf16(tmem + 128, sdesc(sV + kk * 2048, 8192, 1024), bd, id, kk > 0);
+      }
+      mma_commit(&ms.mbar2);
+    }
+    {
+      const bool ok = mbar_wait(&ms.mbar2, it & 1, a.status, 102);
+      if (__syncthreads_or(!ok)) { abort = true; break; }
+    }
+    tc_fence_after();
+    {
+      const int qd = warp & 3, ch = warp >> 2;
+      const int L = 32 * qd + lane;  // c for W^T, v for U0^T
+      const uint32_t lanebase = tmem + ((uint32_t)(32 * qd) << 16);
+      float x[16], y[16];
+      tmem_ld16(lanebase + 64 + 32 * ch, x);
+      tmem_ld16(lanebase + 64 + 32 * ch + 16, y);
+      tmem_wait_ld();
+      uint32_t pk[16];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) pk[j] = pack_bf16(x[2 * j], x[2 * j + 1]);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) pk[8 + j] = pack_bf16(y[2 * j], y[2 * j + 1]);
+#pragma unroll
+      for (int m = 0; m < 4; ++m)
+        *reinterpret_cast<uint4 *>(rec + R1 + mnmaj_off(L, 32 * ch + 8 * m, 128)) =
+            make_uint4(pk[4 * m], pk[4 * m + 1], pk[4 * m + 2], pk[4 * m + 3]);
+      tmem_ld16(lanebase + 128 + 32 * ch, x);
+      tmem_ld16(lanebase + 128 + 32 * ch + 16, y);
+      tmem_wait_ld();
+#pragma unroll
+      for (int j = 0; j < 8; ++j) pk[j] = pack_bf16(x[2 * j], x[2 * j + 1]);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) pk[8 + j] = pack_bf16(y[2 * j], y[2 * j + 1]);
+#pragma unroll
+      for (int m = 0; m < 4; ++m)
+        *reinterpret_cast<uint4 *>(rec + R2 + kmaj_off(L, 32 * ch + 8 * m, 128)) =
+            make_uint4(pk[4 * m], pk[4 * m + 1], pk[4 * m + 2], pk[4 * m + 3]);
+    }
+    tc_fence_before();
+    __syncthreads();
+  }
+  // wind down: make sure no MMA is still writing TMEM before freeing it
+  if (abort && tid == 0) {
+    mma_commit(&ms.mfin);
+    mbar_wait(&ms.mfin, 0, a.status, 109);
+  }
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, 256);
+}
+
+// ===========================================================================
+// sequential state kernel
+// ===========================================================================
+constexpr int kStateThreads = 128;
+constexpr uint32_t S_REC0 = 0;
+constexpr uint32_t S_REC1 = REC_PAD;
+constexpr uint32_t S_TS = 2 * REC_PAD;          // S^T bf16, K-major [v][c] 128 x 128
+constexpr uint32_t S_TU = S_TS + 32768;         // U^T bf16, K-major [v][s] 128 x 64
+constexpr uint32_t S_MISC = S_TU + 16384;
+
+struct StateMisc {
+  uint64_t mrec[2], m3, m4, mfin;
+  uint32_t tmem;
+};
+
+__global__ void __launch_bounds__(kStateThreads, 1) tc_state_kernel(TcArgs ta) {
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char *sm = reinterpret_cast<unsigned char *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  StateMisc &ms = *reinterpret_cast<StateMisc *>(sm + S_MISC);
+  const FwdArgs &a = ta.f;
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int h = blockIdx.x, seq = blockIdx.y, H = a.H;
+  const int v = tid;  // value channel = TMEM lane
+  __nv_bfloat16 *o = (__nv_bfloat16 *)a.o;
+
+  int first;
+  const int nc = a.map.seq_chunks(seq, first);
+  const size_t sbase = ((size_t)seq * H + h) * D * D;
+  const int NCb = a.map.NC;
+
+  if (tid == 0) {
+    mbar_init(&ms.mrec[0], 1);
+    mbar_init(&ms.mrec[1], 1);
+    mbar_init(&ms.m3, 1);
+    mbar_init(&ms.m4, 1);
+    mbar_init(&ms.mfin, 1);
+    mbar_fence_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(&ms.tmem, 256);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ms.tmem;
+  const uint32_t lanebase = tmem + ((uint32_t)(32 * warp) << 16);
+  unsigned char *recbuf[2] = {sm + S_REC0, sm + S_REC1};
+  auto record = [&](int j) -> const unsigned char * {
+    return ta.recs + ((size_t)(first + j) * H + h) * REC;
+  };
+  if (tid == 0) {
+    for (int j = 0; j < 2 && j < nc; ++j) {
+      mbar_arrive_expect_tx(&ms.mrec[j], REC);
+      bulk_g2s(recbuf[j], record(j), REC, &ms.mrec[j]);
+    }
+  }
+  bool abort = false;
+  // initial state: S^T row v = column v of S0; bf16 copy and Diag(d_0)-scaled fp32
+  {
+    bool ok = true;
+    if (nc > 0) ok = mbar_wait(&ms.mrec[0], 0, a.status, 201);
+    if (__syncthreads_or(!ok)) abort = true;
+    if (!abort) {
+      const float *d0 = reinterpret_cast<const float *>(recbuf[0] + R5);
+      for (int c0 = 0; c0 < D; c0 += 16) {
+        float sv[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) sv[i] = a.S0 ? a.S0[sbase + (size_t)(c0 + i) * D + v] : 0.f;
+        if (nc == 0) {
+          if (a.ST)
+            for (int i = 0; i < 16; ++i) a.ST[sbase + (size_t)(c0 + i) * D + v] = sv[i];
+          continue;
+        }
+        if (ta.states_out)
+          for (int i = 0; i < 16; ++i)
+            ta.states_out[(((size_t)seq * H + h) * NCb + 0) * D * D + (size_t)(c0 + i) * D + v] = sv[i];
+        uint32_t pk[8];
+#pragma unroll
+        for (int m = 0; m < 8; ++m) pk[m] = pack_bf16(sv[2 * m], sv[2 * m + 1]);
+        *reinterpret_cast<uint4 *>(sm + S_TS + kmaj_off(v, c0, 128)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        *reinterpret_cast<uint4 *>(sm + S_TS + kmaj_off(v, c0 + 8, 128)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) sv[i] *= d0[c0 + i];
+        tmem_st16(lanebase + c0, sv);
+      }
+      tmem_wait_st();
+    }
+  }
+  fence_async_smem();
+  tc_fence_before();
+  __syncthreads();
+
+  for (int j = 0; j < nc && !abort; ++j) {
+    const int buf = j & 1;
+    unsigned char *rec = recbuf[buf];
+    int sq, len, jl;
+    int64_t tok0;
+    a.map.info(first + j, sq, tok0, len, jl);
+    {
+      const bool ok = mbar_wait(&ms.mrec[buf], (j >> 1) & 1, a.status, 202);
+      if (__syncthreads_or(!ok)) { abort = true; break; }
+    }
+    // MMA3: [(W S)^T | (QG S)^T] = S^T [W^T | QG^T]
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t id = idesc_bf16(128, 128, false, true);
+      const uint32_t sS = smem_u32(sm + S_TS), sR = smem_u32(rec + R1);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk)
+        mma_bf16(tmem + 128, sdesc(sS + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                 sdesc(sR + kk * 2048, 16384, 1024), id, kk > 0);
+      mma_commit(&ms.m3);
+    }
+    {
+      const bool ok = mbar_wait(&ms.m3, j & 1, a.status, 203);
+      if (__syncthreads_or(!ok)) { abort = true; break; }
+    }
+    tc_fence_after();
+    // U^T = U0^T - (W S)^T  -> bf16 K-major tile [v][s]
+    for (int s0 = 0; s0 < 64; s0 += 16) {
+      float w[16];
+      tmem_ld16(lanebase + 128 + s0, w);
+      tmem_wait_ld();
+      const uint4 u0a = *reinterpret_cast<const uint4 *>(rec + R2 + kmaj_off(v, s0, 128));
+      const uint4 u0b = *reinterpret_cast<const uint4 *>(rec + R2 + kmaj_off(v, s0 + 8, 128));
+      const __nv_bfloat16 *ua = reinterpret_cast<const __nv_bfloat16 *>(&u0a);
+      const __nv_bfloat16 *ub = reinterpret_cast<const __nv_bfloat16 *>(&u0b);
+      uint32_t pk[8];
+#pragma unroll
+      for (int m = 0; m < 4; ++m)
+        pk[m] = pack_bf16(__bfloat162float(ua[2 * m]) - w[2 * m], __bfloat162float(ua[2 * m + 1]) - w[2 * m + 1]);
+#pragma unroll
+      for (int m = 0; m < 4; ++m)
+        pk[4 + m] = pack_bf16(__bfloat162float(ub[2 * m]) - w[8 + 2 * m],
+                              __bfloat162float(ub[2 * m + 1]) - w[8 + 2 * m + 1]);
+      *reinterpret_cast<uint4 *>(sm + S_TU + kmaj_off(v, s0, 128)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      *reinterpret_cast<uint4 *>(sm + S_TU + kmaj_off(v, s0 + 8, 128)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    // MMA4: O^T += U^T A_q^T ; MMA5: S^T += U^T Khat
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t sU = smem_u32(sm + S_TU);
+      const uint32_t id4 = idesc_bf16(128, 64, false, false);
+      const uint32_t id5 = idesc_bf16(128, 128, false, false);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        const uint64_t ad = sdesc(sU + kk * 32, 16, 1024);
+        mma_bf16(tmem + 192, ad, sdesc(smem_u32(rec + R3) + kk * 32, 16, 1024), id4, true);
+        mma_bf16(tmem + 0, ad, sdesc(smem_u32(rec + R4) + kk * 32, 16, 1024), id5, true);
+      }
+      mma_commit(&ms.m4);
+    }
+    {
+      const bool ok = mbar_wait(&ms.m4, j & 1, a.status, 204);
+      if (__syncthreads_or(!ok)) { abort = true; break; }
+    }
+    tc_fence_after();
+    // the record buffer is free again: fetch chunk j + 2 into it
+    if (tid == 0 && j + 2 < nc) {
+      mbar_arrive_expect_tx(&ms.mrec[buf], REC);
+      bulk_g2s(rec, record(j + 2), REC, &ms.mrec[buf]);
+    }
+    // output rows of this chunk
+    if (ta.write_o) {
+      for (int r0 = 0; r0 < 64; r0 += 16) {
+        float ov[16];
+        tmem_ld16(lanebase + 192 + r0, ov);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          if (r0 + i < len) o[((size_t)(tok0 + r0 + i) * H + h) * D + v] = __float2bfloat16_rn(ov[i]);
+      }
+    }
+    // next state
+    const bool last = (j + 1 == nc);
+    const float *dn = nullptr;
+    if (!last) {
+      const bool ok = mbar_wait(&ms.mrec[buf ^ 1], ((j + 1) >> 1) & 1, a.status, 205);
+      if (__syncthreads_or(!ok)) { abort = true; break; }
+      dn = reinterpret_cast<const float *>(recbuf[buf ^ 1] + R5);
+    }
+    for (int c0 = 0; c0 < D; c0 += 16) {
+      float sv[16];
+      tmem_ld16(lanebase + c0, sv);
+      tmem_wait_ld();
+      if (last) {
+        if (a.ST)
+          for (int i = 0; i < 16; ++i) a.ST[sbase + (size_t)(c0 + i) * D + v] = sv[i];
+        continue;
+      }
+      if (ta.states_out)
+        for (int i = 0; i < 16; ++i)
+          ta.states_out[(((size_t)seq * H + h) * NCb + j + 1) * D * D + (size_t)(c0 + i) * D + v] = sv[i];
+      uint32_t pk[8];
+#pragma unroll
+      for (int m = 0; m < 8; ++m) pk[m] = pack_bf16(sv[2 * m], sv[2 * m + 1]);
+      *reinterpret_cast<uint4 *>(sm + S_TS + kmaj_off(v, c0, 128)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      *reinterpret_cast<uint4 *>(sm + S_TS + kmaj_off(v, c0 + 8, 128)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) sv[i] *= dn[c0 + i];
+      tmem_st16(lanebase + c0, sv);
+    }
+    tmem_wait_st();
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+  }
+  if (abort && tid == 0) {
+    mma_commit(&ms.mfin);
+    mbar_wait(&ms.mfin, 0, a.status, 209);
+  }
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, 256);
+}
+
+int g_num_sms = 0;
+
+}  // namespace
+
+size_t tc_fwd_fallback_floats(int ctas) { return (size_t)ctas * 3 * 64 * D; }
+
+int tc_intra_ctas() {
+  if (g_num_sms == 0) {
+    int dev = 0, n = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+      cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    g_num_sms = n > 0 ? n : 148;
+  }
+  const int want = 2 * g_num_sms;
+  return want < kBwdCtas ? want : kBwdCtas;
+}
+
+// Forward on tensor cores.  recs: n_chunks_bound * H records of REC bytes;
+// fb: tc_fwd_fallback_floats(tc_intra_ctas()) floats.
+cudaError_t tc_forward(const FwdArgs &f, unsigned char *recs, float *fb, bool write_o,
+                       float *states_out, cudaStream_t s) {
+  TcArgs ta;
+  ta.f = f;
+  ta.recs = recs;
+  ta.fb = fb;
+  ta.states_out = states_out;
+  ta.write_o = write_o;
+  const size_t sm_intra = I_MISC + sizeof(IntraMisc) + 1024;
+  const size_t sm_state = S_MISC + sizeof(StateMisc) + 1024;
+  cudaError_t e = cudaFuncSetAttribute(tc_intra_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)sm_intra);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(tc_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_state);
+  if (e != cudaSuccess) return e;
+  {
+    ProfScope prof("tc_intra", s);
+    tc_intra_kernel<<<tc_intra_ctas(), kIntraThreads, sm_intra, s>>>(ta);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  if (f.map.n_seq > 0) {
+    ProfScope prof(write_o ? "tc_state_fwd" : "tc_state_fwd_recompute", s);
+    tc_state_kernel<<<dim3(f.H, f.map.n_seq), kStateThreads, sm_state, s>>>(ta);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+}  // namespace ckda
