@@ -161,6 +161,7 @@ int ckda_chunk_bwd(int B, int T, int H, int dk, int dv, int io_dtype, const void
   char *w = static_cast<char *>(ws);
   CKDA_CUDA(cudaMemsetAsync(w, 0, sizeof(DevStatus), stream));
   const bool bf16 = io_dtype == CKDA_BF16;
+  const bool tcp = use_tensor_cores(io_dtype, dk, dv);
   FwdArgs f{};
   f.B = B; f.T = T; f.H = H; f.dk = dk; f.dv = dv;
   f.q = q; f.k = k; f.v = v; f.beta = beta; f.g = g; f.sign = sign; f.S0 = S0;
@@ -170,12 +171,20 @@ int ckda_chunk_bwd(int B, int T, int H, int dk, int dv, int io_dtype, const void
   f.map.n_chunks_bound = L.n_chunks_bound;
   f.intra = reinterpret_cast<float *>(w + L.intra);
   f.status = reinterpret_cast<DevStatus *>(w);
-  CKDA_CUDA(v1_intra(f, bf16, reinterpret_cast<float *>(w + L.fscratch), stream));
   const float *states = chunk_states;
-  if (!states) {
+  if (tcp) {
     float *st = reinterpret_cast<float *>(w + L.states);
-    CKDA_CUDA(v1_state_fwd(f, bf16, false, st, stream));
-    states = st;
+    CKDA_CUDA(tc_forward(f, reinterpret_cast<unsigned char *>(w + L.intra),
+                         reinterpret_cast<float *>(w + L.fscratch), false, st, stream,
+                         /*state_pass=*/states == nullptr));
+    if (!states) states = st;
+  } else {
+    CKDA_CUDA(v1_intra(f, bf16, reinterpret_cast<float *>(w + L.fscratch), stream));
+    if (!states) {
+      float *st = reinterpret_cast<float *>(w + L.states);
+      CKDA_CUDA(v1_state_fwd(f, bf16, false, st, stream));
+      states = st;
+    }
   }
   BwdArgs a{};
   a.B = B; a.T = T; a.H = H; a.dk = dk; a.dv = dv;
@@ -188,6 +197,13 @@ int ckda_chunk_bwd(int B, int T, int H, int dk, int dv, int io_dtype, const void
   a.du = reinterpret_cast<float *>(w + L.du);
   a.scratch = reinterpret_cast<float *>(w + L.scratch);
   a.status = f.status;
+  if (tcp) {
+    CKDA_CUDA(tc_backward(a, reinterpret_cast<unsigned char *>(w + L.intra),
+                          reinterpret_cast<unsigned char *>(w + L.dsend),
+                          reinterpret_cast<unsigned char *>(w + L.du),
+                          reinterpret_cast<float *>(w + L.fscratch), stream));
+    return CKDA_OK;
+  }
   CKDA_CUDA(v1_backward(a, bf16, stream));
   return CKDA_OK;
 }

@@ -205,5 +205,60 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<uint32_t *>(&v);
 }
 
+// ---------------------------------------------------------------------------
+// per (chunk, head) record of the intra-chunk kernel (bf16 I/O, dk = dv = 128),
+// laid out as the shared-memory image its consumers read (tiles 1024-aligned)
+// ---------------------------------------------------------------------------
+constexpr int D = 128;
+constexpr float kTau = 40.f;  // bound on |Gam_r - Gam_m| for the factored operands
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr uint32_t R1 = 0;       // [W^T | QG^T]: MN-major B tile, K = c (128), N = r' (128)
+constexpr uint32_t R2 = 32768;   // U0^T: K-major tile [v][s] (128 x 64)
+constexpr uint32_t R3 = 49152;   // A_q: K-major tile [r][s] (64 x 64)
+constexpr uint32_t R4 = 57344;   // Khat^T: K-major tile [c][s] (128 x 64)
+constexpr uint32_t R5 = 73728;   // d[128] fp32
+constexpr uint32_t REC = 74240;  // bytes per (chunk, head) record
+
+__device__ __forceinline__ float fast_exp(float x) { return exp2f(x * kLog2e); }
+
+__device__ __forceinline__ void st_bf16(unsigned char *base, uint32_t off, float x) {
+  *reinterpret_cast<__nv_bfloat16 *>(base + off) = __float2bfloat16_rn(x);
+}
+
+// Chunk rows 32*hf .. 32*hf+31 of key channel c: local inclusive cumsum of g,
+// raw bf16 k | q << 16, sign bits.  Rows >= len are padding (g = 0, k = q = 0,
+// sign +1).  All loads are issued before any use (clamped row index).
+__device__ __forceinline__ void load_rows(const float *g, const int8_t *sign,
+                                          const __nv_bfloat16 *k, const __nv_bfloat16 *q,
+                                          int64_t tok0, int len, int h, int H, int c, int hf,
+                                          float (&G)[32], uint32_t (&kq)[32], uint32_t &neg) {
+  float acc = 0.f;
+  neg = 0;
+#pragma unroll
+  for (int b = 0; b < 2; ++b) {  // two batches of 16 rows: all loads of a batch in flight
+    float gg[16];
+    int sg[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int r = 32 * hf + 16 * b + i;
+      const int rr = r < len ? r : len - 1;
+      const size_t off = ((size_t)(tok0 + rr) * H + h) * D + c;
+      gg[i] = g[off];
+      sg[i] = sign[off];
+      kq[16 * b + i] = (uint32_t)__bfloat16_as_ushort(k[off]) |
+                       ((uint32_t)__bfloat16_as_ushort(q[off]) << 16);
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int ii = 16 * b + i;
+      const bool valid = 32 * hf + ii < len;
+      acc += valid ? gg[i] : 0.f;
+      G[ii] = acc;
+      if (!valid) kq[ii] = 0;
+      if (valid && sg[i] < 0) neg |= 1u << ii;
+    }
+  }
+}
+
 }  // namespace tc
 }  // namespace ckda

@@ -1,0 +1,982 @@
+// ckda_tc_bwd.cu -- chunked CKDA backward on tcgen05 tensor cores (bf16 I/O,
+// dk = dv = 128).  Reverse mode of the chunk-wise WY / UT form ("Complex KDA:
+// Understanding and Enhancing the Expressivity of Kimi Delta Attention",
+// section 2, "Linear RNNs"; sign folding per the "openeurollm/
+// complex-kda-1.3B-100B" model card introduction), derived by hand:
+//
+//   reverse state pass (per sequence and head, chunks in reverse):
+//     dU    = A_q^T dO + Khat dS_{c+1}
+//     dS_c  = Diag(d) dS_{c+1} + QG^T dO - W^T dU
+//   per-chunk gradients (parallel over chunks):
+//     U = U0 - W S_c;  dQG = dO S_c^T;  dW = -dU S_c^T;  dKhat = U dS_{c+1}^T
+//     dd = rowsum(S_c . dS_{c+1});  dA_q = tril(dO U^T);  dT = tril(dU V^T + dW KG^T)
+//     dV = T^T dU;  dKG = T^T dW;  dM = dT Diag(beta);  dL = -M^T dM M^T
+//     dA = Diag(beta) strict_tril(dL);  dbeta from dT.M and dL.A
+//     pair terms through the reference row: X1 = dA K~r, X2 = dA_q K~r,
+//     Y1 = dA^T K~l + dA_q^T Q~, then the exponential factors, a reverse
+//     in-chunk cumsum for dg, and the sign unfold of dq, dk.
+//
+// Kernels: tc_state_bwd_kernel (reverse pass; state gradient kept transposed
+// in TMEM, lanes = value channel) writes per chunk the dL/dS_{c+1} and dU
+// tiles; tc_grad_kernel (persistent, one CTA per SM) does everything else.
+#include <cmath>
+
+#include "ckda_tc.cuh"
+
+namespace ckda {
+namespace {
+
+using namespace tc;
+
+// bytes of the per-(chunk, head) tiles the reverse pass hands to the gradient kernel
+constexpr uint32_t DS_TILE = 32768;  // dL/dS_{c+1}: bf16 K-major [c][v], 128 rows
+constexpr uint32_t DU_TILE = 16384;  // dU: bf16 K-major [i][v], 64 rows
+
+struct BwdTcArgs {
+  BwdArgs b;
+  const unsigned char *recs;  // intra-chunk records (forward layout)
+  unsigned char *dS_tiles;    // [n_chunks][H] DS_TILE
+  unsigned char *dU_tiles;    // [n_chunks][H] DU_TILE
+  float *fb;                  // per-CTA fallback scratch (3 x 64 x 128 fp32)
+};
+
+__device__ __forceinline__ void cp_async16(void *smem_dst, const void *gsrc, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(smem_dst)), "l"(gsrc),
+               "r"(valid ? 16 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+// ===========================================================================
+// reverse state pass
+// ===========================================================================
+constexpr int kSbThreads = 128;
+constexpr uint32_t RB_SIZE = 58368;            // compact record: R1 | R3 | R4 | R5
+constexpr uint32_t RB_R1 = 0, RB_R3 = 32768, RB_R4 = 40960, RB_R5 = 57344;
+constexpr uint32_t SB_RB0 = 0, SB_RB1 = RB_SIZE;
+constexpr uint32_t SB_O0 = 2 * RB_SIZE;        // dO tile K-major [r][v], 64 rows (16 KiB)
+constexpr uint32_t SB_O1 = SB_O0 + 16384;
+constexpr uint32_t SB_DS = SB_O1 + 16384;      // dS^T bf16 K-major [v][c], 128 rows
+constexpr uint32_t SB_DU = SB_DS + 32768;      // dU^T bf16 K-major [v][s], 128 rows x 64
+constexpr uint32_t SB_MISC = SB_DU + 16384;
+
+struct SbMisc {
+  uint64_t mrec[2], mu, ms, mfin;
+  uint32_t tmem;
+};
+
+__global__ void __launch_bounds__(kSbThreads, 1) tc_state_bwd_kernel(BwdTcArgs ta) {
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char *sm = reinterpret_cast<unsigned char *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  SbMisc &ms = *reinterpret_cast<SbMisc *>(sm + SB_MISC);
+  const BwdArgs &a = ta.b;
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int h = blockIdx.x, seq = blockIdx.y, H = a.H;
+  const int v = tid;
+  const __nv_bfloat16 *dO = (const __nv_bfloat16 *)a.dO;
+  int first;
+  const int nc = a.map.seq_chunks(seq, first);
+  const size_t sbase = ((size_t)seq * H + h) * D * D;
+
+  if (tid == 0) {
+    mbar_init(&ms.mrec[0], 1);
+    mbar_init(&ms.mrec[1], 1);
+    mbar_init(&ms.mu, 1);
+    mbar_init(&ms.ms, 1);
+    mbar_init(&ms.mfin, 1);
+    mbar_fence_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(&ms.tmem, 256);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ms.tmem;
+  const uint32_t lanebase = tmem + ((uint32_t)(32 * warp) << 16);
+  unsigned char *rb[2] = {sm + SB_RB0, sm + SB_RB1};
+  unsigned char *ob[2] = {sm + SB_O0, sm + SB_O1};
+
+  // step s handles chunk j = nc - 1 - s
+  auto issue_record = [&](int s) {
+    const int j = nc - 1 - s;
+    const unsigned char *src = ta.recs + ((size_t)(first + j) * H + h) * REC;
+    unsigned char *dst = rb[s & 1];
+    mbar_arrive_expect_tx(&ms.mrec[s & 1], 32768 + 25088);
+    bulk_g2s(dst + RB_R1, src + R1, 32768, &ms.mrec[s & 1]);
+    bulk_g2s(dst + RB_R3, src + R3, 25088, &ms.mrec[s & 1]);
+  };
+  auto issue_dO = [&](int s) {
+    const int j = nc - 1 - s;
+    int sq, len, jl;
+    int64_t tok0;
+    a.map.info(first + j, sq, tok0, len, jl);
+    unsigned char *dst = ob[s & 1];
+    for (int e = tid; e < 64 * 16; e += kSbThreads) {
+      const int r = e >> 4, cc = e & 15;
+      const int rr = r < len ? r : 0;
+      cp_async16(dst + kmaj_off(r, cc * 8, 64), dO + ((size_t)(tok0 + rr) * H + h) * D + cc * 8, r < len);
+    }
+    cp_async_commit();
+  };
+  // dL/dS_{c+1} snapshot of chunk j from the fp32 values of dS^T row v
+  auto snapshot = [&](int j, int c0, const float (&sv)[16]) {
+    unsigned char *dst = ta.dS_tiles + ((size_t)(first + j) * H + h) * DS_TILE;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) st_bf16(dst, kmaj_off(c0 + i, v, 128), sv[i]);
+  };
+
+  if (tid == 0 && nc > 0) {
+    issue_record(0);
+    if (nc > 1) issue_record(1);
+  }
+  if (nc > 0) issue_dO(0);
+  // dS_T (true frame) -> dS^T rows; bf16 copy for the MMA, fp32 in TMEM
+  for (int c0 = 0; c0 < D; c0 += 16) {
+    float sv[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) sv[i] = a.dST ? a.dST[sbase + (size_t)(c0 + i) * D + v] : 0.f;
+    if (nc == 0) {
+      if (a.dS0)
+        for (int i = 0; i < 16; ++i) a.dS0[sbase + (size_t)(c0 + i) * D + v] = sv[i];
+      continue;
+    }
+    snapshot(nc - 1, c0, sv);
+    uint32_t pk[8];
+#pragma unroll
+    for (int m = 0; m < 8; ++m) pk[m] = pack_bf16(sv[2 * m], sv[2 * m + 1]);
+    *reinterpret_cast<uint4 *>(sm + SB_DS + kmaj_off(v, c0, 128)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+    *reinterpret_cast<uint4 *>(sm + SB_DS + kmaj_off(v, c0 + 8, 128)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+    tmem_st16(lanebase + c0, sv);
+  }
+  tmem_wait_st();
+  fence_async_smem();
+  tc_fence_before();
+  __syncthreads();
+
+  bool abort = false;
+  for (int s = 0; s < nc && !abort; ++s) {
+    const int j = nc - 1 - s;
+    const int b = s & 1;
+    unsigned char *rec = rb[b];
+    unsigned char *ot = ob[b];
+    int sq, len, jl;
+    int64_t tok0;
+    a.map.info(first + j, sq, tok0, len, jl);
+    if (s + 1 < nc) issue_dO(s + 1);  // prefetch next dO into the other buffer
+    {
+      // dO of this step landed (all but the group just committed)
+      if (s + 1 < nc) asm volatile("cp.async.wait_group 1;" ::: "memory");
+      else cp_async_wait_all();
+      fence_async_smem();
+      const bool ok = mbar_wait(&ms.mrec[b], (s >> 1) & 1, a.status, 301);
+      if (__syncthreads_or(!ok)) { abort = true; break; }
+    }
+    // dU^T = dO^T A_q + dS1^T Khat^T
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t sO = smem_u32(ot), sRec = smem_u32(rec), sDS = smem_u32(sm + SB_DS);
+      const uint32_t id1 = idesc_bf16(128, 64, true, true);
+      const uint32_t id2 = idesc_bf16(128, 64, false, true);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+        mma_bf16(tmem + 128, sdesc(sO + kk * 2048, 8192, 1024), sdesc(sRec + RB_R3 + kk * 2048, 8192, 1024),
+                 id1, kk > 0);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk)
+        mma_bf16(tmem + 128, sdesc(sDS + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                 sdesc(sRec + RB_R4 + kk * 2048, 8192, 1024), id2, true);
+      mma_commit(&ms.mu);
+    }
+    // meanwhile: dS^T <- dS^T Diag(d_j)
+    {
+      const float *dj = reinterpret_cast<const float *>(rec + RB_R5);
+      for (int c0 = 0; c0 < D; c0 += 16) {
+        float sv[16];
+        tmem_ld16(lanebase + c0, sv);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) sv[i] *= dj[c0 + i];
+        tmem_st16(lanebase + c0, sv);
+      }
+      tmem_wait_st();
+    }
+    {
+      const bool ok = mbar_wait(&ms.mu, s & 1, a.status, 302);
+      if (__syncthreads_or(!ok)) { abort = true; break; }
+    }
+    tc_fence_after();
+    // dU^T -> bf16 operand tile and the dU tile of this chunk
+    {
+      unsigned char *gdu = ta.dU_tiles + ((size_t)(first + j) * H + h) * DU_TILE;
+      for (int s0 = 0; s0 < 64; s0 += 16) {
+        float w[16];
+        tmem_ld16(lanebase + 128 + s0, w);
+        tmem_wait_ld();
+        uint32_t pk[8];
+#pragma unroll
+        for (int m = 0; m < 8; ++m) pk[m] = pack_bf16(w[2 * m], w[2 * m + 1]);
+        *reinterpret_cast<uint4 *>(sm + SB_DU + kmaj_off(v, s0, 128)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        *reinterpret_cast<uint4 *>(sm + SB_DU + kmaj_off(v, s0 + 8, 128)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) st_bf16(gdu, kmaj_off(s0 + i, v, 64), w[i]);
+      }
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    // dS^T += dO^T QG - dU^T W
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t sO = smem_u32(ot), sRec = smem_u32(rec), sDU = smem_u32(sm + SB_DU);
+      const uint32_t id1 = idesc_bf16(128, 128, true, false);
+      const uint32_t id2 = idesc_bf16(128, 128, false, false) | (1u << 13);  // negate A
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+        mma_bf16(tmem, sdesc(sO + kk * 2048, 8192, 1024), sdesc(sRec + RB_R1 + 16384 + kk * 32, 16, 1024),
+                 id1, true);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+        mma_bf16(tmem, sdesc(sDU + kk * 32, 16, 1024), sdesc(sRec + RB_R1 + kk * 32, 16, 1024), id2, true);
+      mma_commit(&ms.ms);
+    }
+    {
+      const bool ok = mbar_wait(&ms.ms, s & 1, a.status, 303);
+      if (__syncthreads_or(!ok)) { abort = true; break; }
+    }
+    tc_fence_after();
+    if (tid == 0 && s + 2 < nc) issue_record(s + 2);
+    // dS at the start of chunk j: next step's operand, snapshot of chunk j-1, or dS0
+    for (int c0 = 0; c0 < D; c0 += 16) {
+      float sv[16];
+      tmem_ld16(lanebase + c0, sv);
+      tmem_wait_ld();
+      if (j == 0) {
+        if (a.dS0)
+          for (int i = 0; i < 16; ++i) a.dS0[sbase + (size_t)(c0 + i) * D + v] = sv[i];
+        continue;
+      }
+      snapshot(j - 1, c0, sv);
+      uint32_t pk[8];
+#pragma unroll
+      for (int m = 0; m < 8; ++m) pk[m] = pack_bf16(sv[2 * m], sv[2 * m + 1]);
+      *reinterpret_cast<uint4 *>(sm + SB_DS + kmaj_off(v, c0, 128)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      *reinterpret_cast<uint4 *>(sm + SB_DS + kmaj_off(v, c0 + 8, 128)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+  }
+  cp_async_wait_all();
+  if (abort && tid == 0) {
+    mma_commit(&ms.mfin);
+    mbar_wait(&ms.mfin, 0, a.status, 309);
+  }
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, 256);
+}
+
+// ===========================================================================
+// per-chunk gradient kernel
+// ===========================================================================
+constexpr int kGThreads = 256;
+constexpr uint32_t G_A1 = 0;          // [Q~; K~l] K-major 128 x 128
+constexpr uint32_t G_B1 = 32768;      // K~r K-major 64 x 128
+constexpr uint32_t G_KG = 49152;      // KG (== K-major [j][c] 64 rows); later tmp fp32 [64][64]
+constexpr uint32_t G_UV = 65536;      // [U; V] K-major 128 x 128
+constexpr uint32_t G_TT = 98304;      // T K-major [r][j] 64 x 64
+constexpr uint32_t G_OU = 106496;     // [dO; dU] K-major 128 x 128
+constexpr uint32_t G_SC = 139264;     // S_c bf16 K-major [c][v]; later dW in rows 64..127
+constexpr uint32_t G_WN = 172032;     // N fp32 | W tile | dS1 tile | [dA; dAq] + dT fp32
+constexpr uint32_t G_DT = G_WN + 16384;
+constexpr uint32_t G_MF = 205824;     // M fp32 [64][65]
+constexpr uint32_t G_MISC = 222464;
+constexpr int LDF = 65;
+
+struct GMisc {
+  uint64_t bar[6], mdu, mds, mfin;
+  uint32_t tmem;
+  int pad;
+  float beta[64], dbc[64], dbr[2][64];
+  float totG[2][128];
+  uint32_t totP[2][128];
+  float dd[2][128];
+  float gcp[2][128];
+  float acc1[128];
+  float X[3][16][16];
+};
+
+__device__ __forceinline__ bool wait_all(uint64_t *bar, uint32_t phase, DevStatus *st, uint32_t site) {
+  const bool ok = mbar_wait(bar, phase, st, site);
+  return !__syncthreads_or(!ok);
+}
+
+__global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(BwdTcArgs ta) {
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char *sm = reinterpret_cast<unsigned char *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  GMisc &ms = *reinterpret_cast<GMisc *>(sm + G_MISC);
+  const BwdArgs &a = ta.b;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int H = a.H;
+  const __nv_bfloat16 *q = (const __nv_bfloat16 *)a.q, *k = (const __nv_bfloat16 *)a.k;
+  const __nv_bfloat16 *v = (const __nv_bfloat16 *)a.v, *beta = (const __nv_bfloat16 *)a.beta;
+  const __nv_bfloat16 *dO = (const __nv_bfloat16 *)a.dO;
+  __nv_bfloat16 *dq = (__nv_bfloat16 *)a.dq, *dk = (__nv_bfloat16 *)a.dkg;
+  __nv_bfloat16 *dv = (__nv_bfloat16 *)a.dvg, *dbeta = (__nv_bfloat16 *)a.dbeta;
+
+  if (tid == 0) {
+    for (int i = 0; i < 6; ++i) mbar_init(&ms.bar[i], 1);
+    mbar_init(&ms.mdu, 1);
+    mbar_init(&ms.mds, 1);
+    mbar_init(&ms.mfin, 1);
+    mbar_fence_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(&ms.tmem, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ms.tmem;
+  const uint32_t sA1 = smem_u32(sm + G_A1), sB1 = smem_u32(sm + G_B1), sKG = smem_u32(sm + G_KG);
+  const uint32_t sUV = smem_u32(sm + G_UV), sTT = smem_u32(sm + G_TT), sOU = smem_u32(sm + G_OU);
+  const uint32_t sSC = smem_u32(sm + G_SC), sWN = smem_u32(sm + G_WN);
+  float *Nf = reinterpret_cast<float *>(sm + G_WN);
+  float *dTf = reinterpret_cast<float *>(sm + G_DT);
+  float *Mf = reinterpret_cast<float *>(sm + G_MF);
+  float *tmpf = reinterpret_cast<float *>(sm + G_KG);  // [64][64]
+  float *fb = ta.fb + (size_t)blockIdx.x * 3 * 64 * D;
+
+  const int c = tid & 127, hf = tid >> 7;
+  const int qd = warp & 3;  // TMEM lane quadrant of this warp
+  const uint32_t lanebase = tmem + ((uint32_t)(32 * qd) << 16);
+  const int nitems = a.map.n_chunks() * H;
+  uint32_t it = 0;
+  bool abort = false;
+  for (int item = blockIdx.x; item < nitems && !abort; item += gridDim.x, ++it) {
+    const uint32_t ph = it & 1;
+    const int cid = item / H, h = item % H;
+    int seq, len, jl;
+    int64_t tok0;
+    a.map.info(cid, seq, tok0, len, jl);
+    const size_t sidx = (((size_t)seq * H + h) * a.map.NC + jl) * D * D;
+    const float *Sc = a.states + sidx;
+    const unsigned char *gdS = ta.dS_tiles + (size_t)item * DS_TILE;
+    const unsigned char *gdU = ta.dU_tiles + (size_t)item * DU_TILE;
+
+    // ---------------- loads ----------------
+    if (tid == 0) {
+      mbar_arrive_expect_tx(&ms.mdu, DU_TILE);
+      bulk_g2s(sm + G_OU + 8192, gdU, 8192, &ms.mdu);
+      bulk_g2s(sm + G_OU + 16384 + 8192, gdU + 8192, 8192, &ms.mdu);
+    }
+    float G[32];
+    uint32_t kq[32];
+    uint32_t neg;
+    load_rows(a.g, a.sign, k, q, tok0, len, h, H, c, hf, G, kq, neg);
+    for (int e = tid; e < 64 * 16; e += kGThreads) {
+      const int j = e >> 4, cc = e & 15;
+      uint4 vv = make_uint4(0, 0, 0, 0), oo = vv;
+      if (j < len) {
+        const size_t off = ((size_t)(tok0 + j) * H + h) * D + cc * 8;
+        vv = *reinterpret_cast<const uint4 *>(v + off);
+        oo = *reinterpret_cast<const uint4 *>(dO + off);
+      }
+      *reinterpret_cast<uint4 *>(sm + G_UV + kmaj_off(64 + j, cc * 8, 128)) = vv;
+      *reinterpret_cast<uint4 *>(sm + G_OU + kmaj_off(j, cc * 8, 128)) = oo;
+    }
+    for (int rr = warp; rr < D; rr += 8) {  // S_c fp32 row rr -> bf16 K-major [c][v]
+      const float4 x = *reinterpret_cast<const float4 *>(Sc + (size_t)rr * D + 4 * lane);
+      uint2 pk = make_uint2(pack_bf16(x.x, x.y), pack_bf16(x.z, x.w));
+      *reinterpret_cast<uint2 *>(sm + G_SC + kmaj_off(rr, 4 * lane, 128)) = pk;
+    }
+    if (tid < 64) ms.beta[tid] = tid < len ? __bfloat162float(beta[(size_t)(tok0 + tid) * H + h]) : 0.f;
+    uint32_t par = 0, pre = 0;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      par ^= (neg >> i) & 1u;
+      pre |= par << i;
+    }
+    ms.totG[hf][c] = G[31];
+    ms.totP[hf][c] = par;
+    __syncthreads();
+    if (hf == 1) {
+      const float cg = ms.totG[0][c];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) G[i] += cg;
+      if (ms.totP[0][c]) pre = ~pre;
+    }
+    const float Gm = ms.totG[0][c];
+    const float GC = ms.totG[0][c] + ms.totG[1][c];
+    const float pCs = (ms.totP[0][c] ^ ms.totP[1][c]) ? -1.f : 1.f;
+    int bad = 0;
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+      if (!(fabsf(G[i] - Gm) <= kTau)) bad = 1;
+    const bool fast = !__syncthreads_or(bad);
+    const float eGm = fast_exp(Gm), eCm = fast_exp(GC - Gm);
+    const float dC = pCs * fast_exp(GC);
+
+    // ---------------- operand tiles ----------------
+    if (fast) {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const int r = 32 * hf + i;
+        const float p = ((pre >> i) & 1u) ? -1.f : 1.f;
+        const float kp = p * __uint_as_float(kq[i] << 16), qp = p * __uint_as_float(kq[i] & 0xffff0000u);
+        const float el = fast_exp(G[i] - Gm), er = __frcp_rn(el);
+        st_bf16(sm + G_A1, kmaj_off(r, c, 128), qp * el);
+        st_bf16(sm + G_A1, kmaj_off(64 + r, c, 128), kp * el);
+        st_bf16(sm + G_B1, kmaj_off(r, c, 64), kp * er);
+        st_bf16(sm + G_KG, mnmaj_off(r, c, 64), kp * el * eGm);
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const int r = 32 * hf + i;
+        const float p = ((pre >> i) & 1u) ? -1.f : 1.f;
+        const float kp = p * __uint_as_float(kq[i] << 16), qp = p * __uint_as_float(kq[i] & 0xffff0000u);
+        fb[r * D + c] = G[i];
+        fb[64 * D + r * D + c] = kp;
+        fb[128 * D + r * D + c] = qp;
+        st_bf16(sm + G_KG, mnmaj_off(r, c, 64), kp * fast_exp(G[i]));
+      }
+    }
+    fence_async_smem();
+    __syncthreads();
+
+    // ---------------- A (-> N = Diag(beta) A) ----------------
+    if (fast) {
+      if (tid == 0) {
+        tc_fence_after();
+        const uint32_t id = idesc_bf16(128, 64, false, false);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_bf16(tmem, sdesc(sA1 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                   sdesc(sB1 + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), id, kk > 0);
+        mma_commit(&ms.bar[0]);
+      }
+      if (!wait_all(&ms.bar[0], ph, a.status, 401)) { abort = true; break; }
+      tc_fence_after();
+      if (qd >= 2) {  // lanes 64..127: rows of A
+        const int r = 32 * qd + lane - 64, ch = warp >> 2;
+        float x[16], y[16];
+        tmem_ld16(lanebase + 32 * ch, x);
+        tmem_ld16(lanebase + 32 * ch + 16, y);
+        tmem_wait_ld();
+        const float br = ms.beta[r];
+#pragma unroll
+        for (int jj = 0; jj < 32; ++jj) {
+          const int s = 32 * ch + jj;
+          const float val = jj < 16 ? x[jj] : y[jj - 16];
+          Nf[r * LDF + s] = s < r ? br * val : 0.f;
+        }
+      }
+    } else {
+      for (int e = tid; e < 64 * 64; e += kGThreads) {
+        const int r = e >> 6, s = e & 63;
+        float aa = 0.f;
+        if (s < r)
+          for (int cc = 0; cc < D; ++cc)
+            aa += fb[64 * D + r * D + cc] * fb[64 * D + s * D + cc] * expf(fb[r * D + cc] - fb[s * D + cc]);
+        Nf[r * LDF + s] = s < r ? ms.beta[r] * aa : 0.f;
+      }
+    }
+    __syncthreads();
+
+    // ---------------- M = (I + N)^{-1} ----------------
+    for (int e = tid; e < 64 * 64; e += kGThreads) Mf[(e >> 6) * LDF + (e & 63)] = 0.f;
+    __syncthreads();
+    if (tid < 64) {
+      const int bI = tid >> 4, j = tid & 15, o = 16 * bI;
+      float xc[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        float s = 0.f;
+#pragma unroll
+        for (int kk = 0; kk < i; ++kk) s += Nf[(o + i) * LDF + o + kk] * xc[kk];
+        xc[i] = (i == j) ? 1.f : (i < j ? 0.f : -s);
+      }
+#pragma unroll
+      for (int i = 0; i < 16; ++i) Mf[(o + i) * LDF + o + j] = xc[i];
+    }
+    __syncthreads();
+    for (int d = 1; d < 4; ++d) {
+      const int nb = 4 - d;
+      for (int e = tid; e < nb * 256; e += kGThreads) {
+        const int J = e >> 8, I = J + d, aa = (e >> 4) & 15, bb = e & 15;
+        float s = 0.f;
+        for (int u = 16 * J; u < 16 * I; ++u) s += Nf[(16 * I + aa) * LDF + u] * Mf[u * LDF + 16 * J + bb];
+        ms.X[J][aa][bb] = s;
+      }
+      __syncthreads();
+      for (int e = tid; e < nb * 256; e += kGThreads) {
+        const int J = e >> 8, I = J + d, aa = (e >> 4) & 15, bb = e & 15;
+        float s = 0.f;
+#pragma unroll
+        for (int t = 0; t < 16; ++t) s += Mf[(16 * I + aa) * LDF + 16 * I + t] * ms.X[J][t][bb];
+        Mf[(16 * I + aa) * LDF + 16 * J + bb] = -s;
+      }
+      __syncthreads();
+    }
+    {
+      const int r = tid >> 2, j0 = (tid & 3) * 16;
+      uint32_t pk[8];
+#pragma unroll
+      for (int m = 0; m < 8; ++m)
+        pk[m] = pack_bf16(Mf[r * LDF + j0 + 2 * m] * ms.beta[j0 + 2 * m],
+                          Mf[r * LDF + j0 + 2 * m + 1] * ms.beta[j0 + 2 * m + 1]);
+      *reinterpret_cast<uint4 *>(sm + G_TT + kmaj_off(r, j0, 64)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      *reinterpret_cast<uint4 *>(sm + G_TT + kmaj_off(r, j0 + 8, 64)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+    }
+    fence_async_smem();
+    __syncthreads();
+
+    // ---------------- W^T, U0^T ----------------
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t id = idesc_bf16(128, 64, true, false);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        const uint64_t bd = sdesc(sTT + kk * 32, 16, 1024);
+        mma_bf16(tmem + 64, sdesc(sKG + kk * 2048, 8192, 1024), bd, id, kk > 0);
+        mma_bf16(tmem + 128, sdesc(sUV + 8192 + kk * 2048, 16384, 1024), bd, id, kk > 0);
+      }
+      mma_commit(&ms.bar[1]);
+    }
+    if (!wait_all(&ms.bar[1], ph, a.status, 402)) { abort = true; break; }
+    tc_fence_after();
+    {  // W^T -> W tile, MN-major B [K = c][N = r] (over the dead N matrix)
+      const int ch = warp >> 2;
+      float x[16], y[16];
+      tmem_ld16(lanebase + 64 + 32 * ch, x);
+      tmem_ld16(lanebase + 64 + 32 * ch + 16, y);
+      tmem_wait_ld();
+      uint32_t pk[16];
+#pragma unroll
+      for (int m = 0; m < 8; ++m) pk[m] = pack_bf16(x[2 * m], x[2 * m + 1]);
+#pragma unroll
+      for (int m = 0; m < 8; ++m) pk[8 + m] = pack_bf16(y[2 * m], y[2 * m + 1]);
+#pragma unroll
+      for (int m = 0; m < 4; ++m)
+        *reinterpret_cast<uint4 *>(sm + G_WN + mnmaj_off(c, 32 * ch + 8 * m, 128)) =
+            make_uint4(pk[4 * m], pk[4 * m + 1], pk[4 * m + 2], pk[4 * m + 3]);
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+
+    // ---------------- (W S)^T -> U ----------------
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t id = idesc_bf16(128, 64, true, true);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk)
+        mma_bf16(tmem + 192, sdesc(sSC + kk * 2048, 16384, 1024), sdesc(sWN + kk * 2048, 16384, 1024), id,
+                 kk > 0);
+      mma_commit(&ms.bar[2]);
+    }
+    if (!wait_all(&ms.bar[2], ph, a.status, 403)) { abort = true; break; }
+    tc_fence_after();
+    if (tid == 0) {  // the W tile is dead: bring dL/dS_{c+1} into its place
+      mbar_arrive_expect_tx(&ms.mds, DS_TILE);
+      bulk_g2s(sm + G_WN, gdS, DS_TILE, &ms.mds);
+    }
+    {  // U^T = U0^T - (W S)^T ; U rows s (K-major [s][v]) of the [U; V] tile
+      const int ch = warp >> 2;
+#pragma unroll
+      for (int h16 = 0; h16 < 2; ++h16) {
+        float u0[16], ws[16];
+        tmem_ld16(lanebase + 128 + 32 * ch + 16 * h16, u0);
+        tmem_ld16(lanebase + 192 + 32 * ch + 16 * h16, ws);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) st_bf16(sm + G_UV, kmaj_off(32 * ch + 16 * h16 + i, c, 128), u0[i] - ws[i]);
+      }
+    }
+    // dd partial: sum over v of S_c[c][v] * dS1[c][v] (dS1 arrives meanwhile)
+    if (!wait_all(&ms.mds, ph, a.status, 404)) { abort = true; break; }
+    {
+      float s = 0.f;
+      for (int vv = 64 * hf; vv < 64 * hf + 64; vv += 8) {
+        const uint4 xa = *reinterpret_cast<const uint4 *>(sm + G_SC + kmaj_off(c, vv, 128));
+        const uint4 xb = *reinterpret_cast<const uint4 *>(sm + G_WN + kmaj_off(c, vv, 128));
+        const __nv_bfloat16 *pa = reinterpret_cast<const __nv_bfloat16 *>(&xa);
+        const __nv_bfloat16 *pb = reinterpret_cast<const __nv_bfloat16 *>(&xb);
+#pragma unroll
+        for (int m = 0; m < 8; ++m) s += __bfloat162float(pa[m]) * __bfloat162float(pb[m]);
+      }
+      ms.dd[hf][c] = s;
+    }
+    if (!wait_all(&ms.mdu, ph, a.status, 405)) { abort = true; break; }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+
+    // ---------------- [dQG^T | S dU^T], dKhat^T ----------------
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t id1 = idesc_bf16(128, 128, false, false);
+      const uint32_t id2 = idesc_bf16(128, 64, false, false);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t ko = (kk >> 2) * 16384 + (kk & 3) * 32;
+        mma_bf16(tmem + 256, sdesc(sSC + ko, 16, 1024), sdesc(sOU + ko, 16, 1024), id1, kk > 0);
+        mma_bf16(tmem + 384, sdesc(sWN + ko, 16, 1024), sdesc(sUV + ko, 16, 1024), id2, kk > 0);
+      }
+      mma_commit(&ms.bar[3]);
+    }
+    if (!wait_all(&ms.bar[3], ph, a.status, 406)) { abort = true; break; }
+    tc_fence_after();
+    {  // dW = -dU S_c^T -> rows 64..127 of the S_c tile (K-major [i][c]); S_c is dead
+      const int ch = warp >> 2;
+#pragma unroll
+      for (int h16 = 0; h16 < 2; ++h16) {
+        float w[16];
+        tmem_ld16(lanebase + 320 + 32 * ch + 16 * h16, w);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) st_bf16(sm + G_SC, kmaj_off(64 + 32 * ch + 16 * h16 + i, c, 128), -w[i]);
+      }
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+
+    // ---------------- D7 = [dO; dU][U; V]^T + [.; dW] KG^T ----------------
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t id1 = idesc_bf16(128, 128, false, false);
+      const uint32_t id2 = idesc_bf16(128, 64, false, false);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t ko = (kk >> 2) * 16384 + (kk & 3) * 32;
+        mma_bf16(tmem + 128, sdesc(sOU + ko, 16, 1024), sdesc(sUV + ko, 16, 1024), id1, kk > 0);
+      }
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk)
+        mma_bf16(tmem + 192, sdesc(sSC + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                 sdesc(sKG + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), id2, true);
+      mma_commit(&ms.bar[4]);
+    }
+    if (!wait_all(&ms.bar[4], ph, a.status, 407)) { abort = true; break; }
+    tc_fence_after();
+    {
+      const int ch = warp >> 2;
+      const int L = 32 * qd + lane;
+      float x[16], y[16];
+      if (L < 64) {  // dA_q rows -> bf16 rows 64..127 of the [dA; dA_q] tile
+        tmem_ld16(lanebase + 128 + 32 * ch, x);
+        tmem_ld16(lanebase + 128 + 32 * ch + 16, y);
+        tmem_wait_ld();
+        const int r = L;
+        uint32_t pk[16];
+#pragma unroll
+        for (int jj = 0; jj < 16; ++jj) {
+          const int s0 = 32 * ch + 2 * jj;
+          const float v0 = jj < 8 ? x[2 * jj] : y[2 * jj - 16];
+          const float v1 = jj < 8 ? x[2 * jj + 1] : y[2 * jj + 1 - 16];
+          pk[jj] = pack_bf16(s0 <= r ? v0 : 0.f, s0 + 1 <= r ? v1 : 0.f);
+        }
+#pragma unroll
+        for (int m = 0; m < 4; ++m)
+          *reinterpret_cast<uint4 *>(sm + G_WN + kmaj_off(64 + r, 32 * ch + 8 * m, 128)) =
+              make_uint4(pk[4 * m], pk[4 * m + 1], pk[4 * m + 2], pk[4 * m + 3]);
+      } else {  // dT rows (masked j <= i) -> fp32
+        tmem_ld16(lanebase + 192 + 32 * ch, x);
+        tmem_ld16(lanebase + 192 + 32 * ch + 16, y);
+        tmem_wait_ld();
+        const int i = L - 64;
+#pragma unroll
+        for (int jj = 0; jj < 32; ++jj) {
+          const int j = 32 * ch + jj;
+          const float val = jj < 16 ? x[jj] : y[jj - 16];
+          dTf[i * LDF + j] = j <= i ? val : 0.f;
+        }
+      }
+    }
+    tc_fence_before();
+    __syncthreads();
+    // dbeta (column part) and dM = dT Diag(beta)
+    if (tid < 64) {
+      const int j = tid;
+      float s = 0.f;
+      for (int i = j; i < 64; ++i) s += dTf[i * LDF + j] * Mf[i * LDF + j];
+      ms.dbc[j] = s;
+    }
+    __syncthreads();
+    for (int e = tid; e < 64 * 64; e += kGThreads) dTf[(e >> 6) * LDF + (e & 63)] *= ms.beta[e & 63];
+    __syncthreads();
+    // tmp = dM M^T  (tmp[i][kk] = sum_{j <= min(i, kk)} dM[i][j] M[kk][j])
+    for (int e = tid; e < 64 * 64; e += kGThreads) {
+      const int i = e >> 6, kk = e & 63;
+      const int jm = i < kk ? i : kk;
+      float s = 0.f;
+      for (int j = 0; j <= jm; ++j) s += dTf[i * LDF + j] * Mf[kk * LDF + j];
+      tmpf[i * 64 + kk] = s;
+    }
+    __syncthreads();
+    // dL = -M^T tmp, strict lower -> dN (into dTf)
+    for (int e = tid; e < 64 * 64; e += kGThreads) {
+      const int aa = e >> 6, kk = e & 63;
+      float s = 0.f;
+      if (kk < aa)
+        for (int i = aa; i < 64; ++i) s -= Mf[i * LDF + aa] * tmpf[i * 64 + kk];
+      dTf[aa * LDF + kk] = s;  // overwrites dM row aa: dM is dead (tmp holds it)
+    }
+    __syncthreads();
+    // dA = Diag(beta) dN -> bf16 rows 0..63 of the [dA; dA_q] tile; dbeta (row part)
+    {
+      const int r = tid >> 2, j0 = (tid & 3) * 16;
+      const float br = ms.beta[r];
+      uint32_t pk[8];
+#pragma unroll
+      for (int m = 0; m < 8; ++m)
+        pk[m] = pack_bf16(br * dTf[r * LDF + j0 + 2 * m], br * dTf[r * LDF + j0 + 2 * m + 1]);
+      *reinterpret_cast<uint4 *>(sm + G_WN + kmaj_off(r, j0, 128)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      *reinterpret_cast<uint4 *>(sm + G_WN + kmaj_off(r, j0 + 8, 128)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+    }
+    if (fast) {
+      if (qd >= 2) {
+        const int r = 32 * qd + lane - 64, ch = warp >> 2;
+        float x[16], y[16];
+        tmem_ld16(lanebase + 32 * ch, x);
+        tmem_ld16(lanebase + 32 * ch + 16, y);
+        tmem_wait_ld();
+        float s = 0.f;
+#pragma unroll
+        for (int jj = 0; jj < 32; ++jj) {
+          const int j = 32 * ch + jj;
+          if (j < r) s += dTf[r * LDF + j] * (jj < 16 ? x[jj] : y[jj - 16]);
+        }
+        ms.dbr[ch][r] = s;
+      }
+    } else {
+      // exact path: recompute the needed A entries from the fallback scratch
+      if (tid < 128) {
+        const int r = tid & 63, ch = tid >> 6;
+        float s = 0.f;
+        for (int j = 32 * ch; j < 32 * ch + 32; ++j) {
+          if (j >= r) break;
+          float aa = 0.f;
+          for (int cc = 0; cc < D; ++cc)
+            aa += fb[64 * D + r * D + cc] * fb[64 * D + j * D + cc] * expf(fb[r * D + cc] - fb[j * D + cc]);
+          s += dTf[r * LDF + j] * aa;
+        }
+        ms.dbr[ch][r] = s;
+      }
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+
+    // ---------------- dV^T, dKG^T, X^T, Y^T ----------------
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t idT = idesc_bf16(128, 64, true, true);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        const uint64_t bd = sdesc(sTT + kk * 2048, 8192, 1024);
+        mma_bf16(tmem + 448, sdesc(sOU + 8192 + kk * 2048, 16384, 1024), bd, idT, kk > 0);
+        mma_bf16(tmem + 64, sdesc(sSC + 8192 + kk * 2048, 16384, 1024), bd, idT, kk > 0);
+      }
+      if (fast) {
+        const uint32_t idX = idesc_bf16(128, 128, true, false);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_bf16(tmem + 128, sdesc(sB1 + kk * 2048, 8192, 1024), sdesc(sWN + kk * 32, 16, 1024), idX, kk > 0);
+        const uint32_t idY = idesc_bf16(128, 64, true, true);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_bf16(tmem + 320, sdesc(sA1 + 8192 + kk * 2048, 16384, 1024), sdesc(sWN + kk * 2048, 8192, 1024),
+                   idY, kk > 0);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_bf16(tmem + 320, sdesc(sA1 + kk * 2048, 16384, 1024), sdesc(sWN + 8192 + kk * 2048, 8192, 1024),
+                   idY, true);
+      }
+      mma_commit(&ms.bar[5]);
+    }
+    if (!fast) {
+      // exact pair terms into the TMEM columns the fast path fills:
+      // X1 (128 + r), X2 (192 + r), Y1 (320 + r) of lane c
+      const float *Gc = fb, *kpc = fb + 64 * D, *qpc = fb + 128 * D;
+
+      auto dAv = [&](int r, int s) {  // dA (rows 0..63) / dA_q (rows 64..127) from the bf16 tile
+        return __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(sm + G_WN + kmaj_off(r, s, 128)));
+      };
+
+      for (int b16 = 0; b16 < 2; ++b16) {
+        float x1[16], x2[16], y1[16];
+        for (int i = 0; i < 16; ++i) {
+          const int r = 32 * hf + 16 * b16 + i;
+          const float gr = Gc[r * D + c];
+          float a1 = 0.f, a2 = 0.f, b1 = 0.f;
+          for (int s = 0; s <= r; ++s) {
+            const float e = expf(gr - Gc[s * D + c]) * kpc[s * D + c];
+            a1 += dAv(r, s) * e;
+            a2 += dAv(64 + r, s) * e;
+          }
+          for (int t = r; t < 64; ++t) {
+            const float e = expf(Gc[t * D + c] - gr);
+            b1 += (dAv(t, r) * kpc[t * D + c] + dAv(64 + t, r) * qpc[t * D + c]) * e;
+          }
+          x1[i] = a1;
+          x2[i] = a2;
+          y1[i] = b1;
+        }
+        const uint32_t colo = 32 * hf + 16 * b16;
+        tmem_st16(lanebase + 128 + colo, x1);
+        tmem_st16(lanebase + 192 + colo, x2);
+        tmem_st16(lanebase + 320 + colo, y1);
+      }
+      tmem_wait_st();
+    }
+    if (!wait_all(&ms.bar[5], ph, a.status, 408)) { abort = true; break; }
+    tc_fence_after();
+
+    // ---------------- final elementwise gradients ----------------
+    {
+      // thread (c, hf): rows 32 hf .. 32 hf + 31 of key channel c
+      float dG[32];
+      float gcp = 0.f;
+#pragma unroll
+      for (int b16 = 0; b16 < 2; ++b16) {
+        const uint32_t colo = 32 * hf + 16 * b16;
+        float X1[16], X2[16], Y1[16], dQG[16], dKG[16], dKh[16];
+        tmem_ld16(lanebase + 128 + colo, X1);
+        tmem_ld16(lanebase + 192 + colo, X2);
+        tmem_ld16(lanebase + 320 + colo, Y1);
+        tmem_ld16(lanebase + 256 + colo, dQG);
+        tmem_ld16(lanebase + 64 + colo, dKG);
+        tmem_ld16(lanebase + 384 + colo, dKh);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int ii = 16 * b16 + i;
+          const int r = 32 * hf + ii;
+          const float p = ((pre >> ii) & 1u) ? -1.f : 1.f;
+          const float kp = p * __uint_as_float(kq[ii] << 16), qp = p * __uint_as_float(kq[ii] & 0xffff0000u);
+          float el, er, E, eC;
+          if (fast) {
+            el = fast_exp(G[ii] - Gm);
+            er = __frcp_rn(el);
+            E = el * eGm;
+            eC = er * eCm;
+          } else {
+            el = 1.f;
+            er = 1.f;
+            E = fast_exp(G[ii]);
+            eC = fast_exp(GC - G[ii]);
+          }
+          const float x1 = el * X1[i], x2 = el * X2[i], y1 = er * Y1[i];
+          const float KG = kp * E, QG = qp * E, Kh = pCs * kp * eC;
+          const float dkp = x1 + y1 + dKG[i] * E + pCs * dKh[i] * eC;
+          const float dqp = x2 + dQG[i] * E;
+          dG[ii] = kp * x1 + qp * x2 - kp * y1 + dKG[i] * KG + dQG[i] * QG - dKh[i] * Kh;
+          gcp += dKh[i] * Kh;
+          if (r < len) {
+            const size_t off = ((size_t)(tok0 + r) * H + h) * D + c;
+            dq[off] = __float2bfloat16_rn(p * dqp);
+            dk[off] = __float2bfloat16_rn(p * dkp);
+          }
+        }
+        // dV^T lanes = value channel, columns = token
+        float dVv[16];
+        tmem_ld16(lanebase + 448 + colo, dVv);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int j = 32 * hf + 16 * b16 + i;
+          if (j < len) dv[((size_t)(tok0 + j) * H + h) * D + c] = __float2bfloat16_rn(dVv[i]);
+        }
+      }
+      ms.gcp[hf][c] = gcp;
+      __syncthreads();
+      const float gC = ms.gcp[0][c] + ms.gcp[1][c] + (ms.dd[0][c] + ms.dd[1][c]) * dC;
+      // reverse in-chunk cumsum: the upper half first, then the lower half continues
+      if (hf == 1) {
+        float acc = gC;
+#pragma unroll
+        for (int ii = 31; ii >= 0; --ii) {
+          acc += dG[ii];
+          const int r = 32 + ii;
+          if (r < len) a.dg[((size_t)(tok0 + r) * H + h) * D + c] = acc;
+        }
+        ms.acc1[c] = acc;
+      }
+      __syncthreads();
+      if (hf == 0) {
+        float acc = ms.acc1[c];
+#pragma unroll
+        for (int ii = 31; ii >= 0; --ii) {
+          acc += dG[ii];
+          if (ii < len) a.dg[((size_t)(tok0 + ii) * H + h) * D + c] = acc;
+        }
+      }
+      if (tid < 64 && tid < len)
+        dbeta[(size_t)(tok0 + tid) * H + h] =
+            __float2bfloat16_rn(ms.dbc[tid] + ms.dbr[0][tid] + ms.dbr[1][tid]);
+    }
+    tc_fence_before();
+    __syncthreads();
+  }
+  if (abort && tid == 0) {
+    mma_commit(&ms.mfin);
+    mbar_wait(&ms.mfin, 0, a.status, 409);
+  }
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, 512);
+}
+
+int g_sms = 0;
+int num_sms() {
+  if (g_sms == 0) {
+    int dev = 0, n = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    g_sms = n > 0 ? n : 148;
+  }
+  return g_sms;
+}
+
+}  // namespace
+
+// Backward on tensor cores.  recs: records of tc_forward's intra kernel for
+// these inputs; dS_tiles / dU_tiles: n_chunks * H tiles of 32 KiB / 16 KiB.
+cudaError_t tc_backward(const BwdArgs &b, const unsigned char *recs, unsigned char *dS_tiles,
+                        unsigned char *dU_tiles, float *fb, cudaStream_t s) {
+  BwdTcArgs ta;
+  ta.b = b;
+  ta.recs = recs;
+  ta.dS_tiles = dS_tiles;
+  ta.dU_tiles = dU_tiles;
+  ta.fb = fb;
+  const size_t sm_sb = SB_MISC + sizeof(SbMisc) + 1024;
+  const size_t sm_g = G_MISC + sizeof(GMisc) + 1024;
+  cudaError_t e = cudaFuncSetAttribute(tc_state_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)sm_sb);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(tc_grad_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_g);
+  if (e != cudaSuccess) return e;
+  if (b.map.n_seq == 0) return cudaSuccess;
+  {
+    ProfScope prof("tc_state_bwd", s);
+    tc_state_bwd_kernel<<<dim3(b.H, b.map.n_seq), kSbThreads, sm_sb, s>>>(ta);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  {
+    ProfScope prof("tc_grad", s);
+    tc_grad_kernel<<<num_sms(), kGThreads, sm_g, s>>>(ta);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+size_t tc_bwd_smem_bytes() { return G_MISC + sizeof(GMisc) + 1024; }
+
+}  // namespace ckda

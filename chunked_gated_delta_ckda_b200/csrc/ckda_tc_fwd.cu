@@ -38,24 +38,7 @@ namespace {
 
 using namespace tc;
 
-constexpr int D = 128;
-constexpr float kTau = 40.f;
-constexpr float kLog2e = 1.4426950408889634f;
-
-// record layout (bytes); each tile 1024-byte aligned inside the record
-constexpr uint32_t R1 = 0;       // [W^T | QG^T]: MN-major B tile, K = c (128), N = r' (128)
-constexpr uint32_t R2 = 32768;   // U0^T: K-major tile [v][s] (128 x 64)
-constexpr uint32_t R3 = 49152;   // A_q: K-major tile [r][s] (64 x 64)
-constexpr uint32_t R4 = 57344;   // Khat^T: K-major tile [c][s] (128 x 64)
-constexpr uint32_t R5 = 73728;   // d[128] fp32
-constexpr uint32_t REC = 74240;  // bytes per (chunk, head) record
 constexpr uint32_t REC_PAD = 74752;  // record slot in shared memory (73 x 1024)
-
-__device__ __forceinline__ float fast_exp(float x) { return exp2f(x * kLog2e); }
-
-__device__ __forceinline__ void st_bf16(unsigned char *base, uint32_t off, float x) {
-  *reinterpret_cast<__nv_bfloat16 *>(base + off) = __float2bfloat16_rn(x);
-}
 
 // ===========================================================================
 // intra-chunk kernel
@@ -138,27 +121,7 @@ __global__ void __launch_bounds__(kIntraThreads, 2) tc_intra_kernel(TcArgs ta) {
     float G[32];
     uint32_t kq[32];   // bf16 k (low half) and q (high half) of each row
     uint32_t neg = 0;  // bit i: sign of row 32*hf + i is negative
-    {
-      float acc = 0.f;
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const int r = 32 * hf + i;
-        float gg = 0.f;
-        uint32_t kk = 0, qq = 0;
-        int8_t sg = 1;
-        if (r < len) {
-          const size_t off = ((size_t)(tok0 + r) * H + h) * D + c;
-          gg = a.g[off];
-          sg = a.sign[off];
-          kk = __bfloat16_as_ushort(k[off]);
-          qq = __bfloat16_as_ushort(q[off]);
-        }
-        acc += gg;
-        G[i] = acc;
-        kq[i] = kk | (qq << 16);
-        if (sg < 0) neg |= 1u << i;
-      }
-    }
+    load_rows(a.g, a.sign, k, q, tok0, len, h, H, c, hf, G, kq, neg);
     // prefix parity of the sign bits
     uint32_t par = 0, pre = 0;
 #pragma unroll
@@ -670,7 +633,7 @@ int tc_intra_ctas() {
 // Forward on tensor cores.  recs: n_chunks_bound * H records of REC bytes;
 // fb: tc_fwd_fallback_floats(tc_intra_ctas()) floats.
 cudaError_t tc_forward(const FwdArgs &f, unsigned char *recs, float *fb, bool write_o,
-                       float *states_out, cudaStream_t s) {
+                       float *states_out, cudaStream_t s, bool state_pass) {
   TcArgs ta;
   ta.f = f;
   ta.recs = recs;
@@ -689,7 +652,7 @@ cudaError_t tc_forward(const FwdArgs &f, unsigned char *recs, float *fb, bool wr
     tc_intra_kernel<<<tc_intra_ctas(), kIntraThreads, sm_intra, s>>>(ta);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
-  if (f.map.n_seq > 0) {
+  if (state_pass && f.map.n_seq > 0) {
     ProfScope prof(write_o ? "tc_state_fwd" : "tc_state_fwd_recompute", s);
     tc_state_kernel<<<dim3(f.H, f.map.n_seq), kStateThreads, sm_state, s>>>(ta);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;

@@ -102,7 +102,8 @@ def _bwd(inp, S0, dST, cs=None):
 
 @pytest.mark.parametrize("io", [torch.float32, torch.bfloat16])
 @pytest.mark.parametrize("B,T,H,dk,dv,gscale", [(2, 150, 2, 64, 64, 0.05), (1, 256, 2, 128, 128, 0.05),
-                                                (1, 70, 3, 64, 128, 3.0), (2, 33, 1, 128, 64, 0.3)])
+                                                (1, 70, 3, 64, 128, 3.0), (2, 33, 1, 128, 64, 0.3),
+                                                (1, 100, 2, 128, 128, 3.0), (3, 130, 2, 128, 128, 0.05)])
 def test_backward_against_oracle(io, B, T, H, dk, dv, gscale):
     inp = random_inputs(B, T, H, dk, dv, io, seed=T + dk, gscale=gscale, extreme_p=0.05)
     got = _bwd(inp, inp["S0"], inp["dST"])
