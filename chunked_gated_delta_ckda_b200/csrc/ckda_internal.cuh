@@ -6,7 +6,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
-#include "../../include/ckda.h"
+#include "ckda.h"
 
 namespace ckda {
 

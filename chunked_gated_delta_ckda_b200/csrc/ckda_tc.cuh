@@ -260,5 +260,128 @@ __device__ __forceinline__ void load_rows(const float *g, const int8_t *sign,
   }
 }
 
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8]) {
+  uint32_t r[8];
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+                 "=r"(r[7])
+               : "r"(taddr));
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// ---------------------------------------------------------------------------
+// Chunk preprocessing in the "row-group" thread layout (256 threads):
+// warp w owns chunk rows 8w .. 8w+7, lane l owns key channels 4l .. 4l+3.
+// Every load is a coalesced vector load of a full 128-channel row.
+// ---------------------------------------------------------------------------
+struct PrepTot {  // per-group totals exchanged through shared memory
+  float G[8][128];
+  uint8_t P[8][128];
+};
+
+struct Prep {
+  float G[8][4];     // chunk-local inclusive cumsum of g (after the carry)
+  uint32_t k2[8][2]; // raw bf16 k, two channels per word
+  uint32_t q2[8][2];
+  uint32_t pre;      // bit 4*rr+m: sign product of row 8w+rr, channel 4l+m is negative
+  float Gm[4], GC[4];
+  uint32_t pC;       // bit m: chunk sign product of channel 4l+m is negative
+};
+
+// Loads the 8 x 4 block of this thread, local scans, writes the group totals.
+__device__ __forceinline__ void prep_load(const float *g, const int8_t *sign, const __nv_bfloat16 *k,
+                                          const __nv_bfloat16 *q, int64_t tok0, int len, int h, int H,
+                                          int w, int l, Prep &P, PrepTot &tot) {
+  float4 gv[8];
+  uint32_t sg[8];
+#pragma unroll
+  for (int rr = 0; rr < 8; ++rr) {
+    const int r = 8 * w + rr;
+    const int rrow = r < len ? r : len - 1;
+    const size_t off = ((size_t)(tok0 + rrow) * H + h) * D + 4 * l;
+    gv[rr] = *reinterpret_cast<const float4 *>(g + off);
+    sg[rr] = *reinterpret_cast<const uint32_t *>(sign + off);
+    const uint2 kv = *reinterpret_cast<const uint2 *>(k + off);
+    const uint2 qv = *reinterpret_cast<const uint2 *>(q + off);
+    P.k2[rr][0] = kv.x; P.k2[rr][1] = kv.y;
+    P.q2[rr][0] = qv.x; P.q2[rr][1] = qv.y;
+  }
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  uint32_t par = 0, pre = 0;
+#pragma unroll
+  for (int rr = 0; rr < 8; ++rr) {
+    const bool valid = 8 * w + rr < len;
+    const float gg[4] = {gv[rr].x, gv[rr].y, gv[rr].z, gv[rr].w};
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      acc[m] += valid ? gg[m] : 0.f;
+      P.G[rr][m] = acc[m];
+      const bool neg = valid && (int8_t)((sg[rr] >> (8 * m)) & 0xffu) < 0;
+      par ^= (neg ? 1u : 0u) << m;
+    }
+    pre |= par << (4 * rr);
+    if (!valid) {
+      P.k2[rr][0] = P.k2[rr][1] = 0u;
+      P.q2[rr][0] = P.q2[rr][1] = 0u;
+    }
+  }
+  P.pre = pre;
+  *reinterpret_cast<float4 *>(&tot.G[w][4 * l]) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+#pragma unroll
+  for (int m = 0; m < 4; ++m) tot.P[w][4 * l + m] = (uint8_t)((par >> m) & 1u);
+}
+
+// After a barrier: add the carry of the earlier row groups; reference row 31
+// and chunk totals per channel.
+__device__ __forceinline__ void prep_carry(int w, int l, Prep &P, const PrepTot &tot) {
+  float cg[4] = {0.f, 0.f, 0.f, 0.f}, gm[4] = {0.f, 0.f, 0.f, 0.f}, gc[4] = {0.f, 0.f, 0.f, 0.f};
+  uint32_t cp = 0, pc = 0;
+#pragma unroll
+  for (int ww = 0; ww < 8; ++ww) {
+    const float4 t = *reinterpret_cast<const float4 *>(&tot.G[ww][4 * l]);
+    const float tt[4] = {t.x, t.y, t.z, t.w};
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const uint32_t pb = tot.P[ww][4 * l + m];
+      if (ww < w) { cg[m] += tt[m]; cp ^= pb << m; }
+      if (ww <= 3) gm[m] += tt[m];
+      gc[m] += tt[m];
+      pc ^= pb << m;
+    }
+  }
+#pragma unroll
+  for (int rr = 0; rr < 8; ++rr)
+#pragma unroll
+    for (int m = 0; m < 4; ++m) P.G[rr][m] += cg[m];
+  uint32_t rep = 0;  // replicate the 4-bit carry parity over the 8 rows
+#pragma unroll
+  for (int rr = 0; rr < 8; ++rr) rep |= cp << (4 * rr);
+  P.pre ^= rep;
+#pragma unroll
+  for (int m = 0; m < 4; ++m) { P.Gm[m] = gm[m]; P.GC[m] = gc[m]; }
+  P.pC = pc;
+}
+
+__device__ __forceinline__ float bf_lo(uint32_t x) { return __uint_as_float(x << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t x) { return __uint_as_float(x & 0xffff0000u); }
+// raw k (q) of row rr, channel m of this thread
+__device__ __forceinline__ float prep_k(const Prep &P, int rr, int m) {
+  const uint32_t w2 = P.k2[rr][m >> 1];
+  return (m & 1) ? bf_hi(w2) : bf_lo(w2);
+}
+__device__ __forceinline__ float prep_q(const Prep &P, int rr, int m) {
+  const uint32_t w2 = P.q2[rr][m >> 1];
+  return (m & 1) ? bf_hi(w2) : bf_lo(w2);
+}
+__device__ __forceinline__ float prep_p(const Prep &P, int rr, int m) {
+  return ((P.pre >> (4 * rr + m)) & 1u) ? -1.f : 1.f;
+}
+// 4 consecutive bf16 (8 bytes) of a row of a 128-byte-swizzled tile
+__device__ __forceinline__ void st_bf16x4(unsigned char *base, uint32_t off, float a, float b, float c,
+                                          float d) {
+  *reinterpret_cast<uint2 *>(base + off) = make_uint2(pack_bf16(a, b), pack_bf16(c, d));
+}
+
 }  // namespace tc
 }  // namespace ckda

@@ -51,7 +51,7 @@ __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wai
 // ===========================================================================
 // reverse state pass
 // ===========================================================================
-constexpr int kSbThreads = 128;
+constexpr int kSbThreads = 256;  // two warps per TMEM lane quadrant
 constexpr uint32_t RB_SIZE = 58368;            // compact record: R1 | R3 | R4 | R5
 constexpr uint32_t RB_R1 = 0, RB_R3 = 32768, RB_R4 = 40960, RB_R5 = 57344;
 constexpr uint32_t SB_RB0 = 0, SB_RB1 = RB_SIZE;
@@ -72,9 +72,10 @@ __global__ void __launch_bounds__(kSbThreads, 1) tc_state_bwd_kernel(BwdTcArgs t
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   SbMisc &ms = *reinterpret_cast<SbMisc *>(sm + SB_MISC);
   const BwdArgs &a = ta.b;
-  const int tid = threadIdx.x, warp = tid >> 5;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int qd = warp & 3, ch = warp >> 2;
   const int h = blockIdx.x, seq = blockIdx.y, H = a.H;
-  const int v = tid;
+  const int v = 32 * qd + lane;
   const __nv_bfloat16 *dO = (const __nv_bfloat16 *)a.dO;
   int first;
   const int nc = a.map.seq_chunks(seq, first);
@@ -96,7 +97,7 @@ __global__ void __launch_bounds__(kSbThreads, 1) tc_state_bwd_kernel(BwdTcArgs t
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = ms.tmem;
-  const uint32_t lanebase = tmem + ((uint32_t)(32 * warp) << 16);
+  const uint32_t lanebase = tmem + ((uint32_t)(32 * qd) << 16);
   unsigned char *rb[2] = {sm + SB_RB0, sm + SB_RB1};
   unsigned char *ob[2] = {sm + SB_O0, sm + SB_O1};
 
@@ -135,7 +136,7 @@ __global__ void __launch_bounds__(kSbThreads, 1) tc_state_bwd_kernel(BwdTcArgs t
   }
   if (nc > 0) issue_dO(0);
   // dS_T (true frame) -> dS^T rows; bf16 copy for the MMA, fp32 in TMEM
-  for (int c0 = 0; c0 < D; c0 += 16) {
+  for (int c0 = 64 * ch; c0 < 64 * ch + 64; c0 += 16) {
     float sv[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) sv[i] = a.dST ? a.dST[sbase + (size_t)(c0 + i) * D + v] : 0.f;
@@ -194,7 +195,7 @@ __global__ void __launch_bounds__(kSbThreads, 1) tc_state_bwd_kernel(BwdTcArgs t
     // meanwhile: dS^T <- dS^T Diag(d_j)
     {
       const float *dj = reinterpret_cast<const float *>(rec + RB_R5);
-      for (int c0 = 0; c0 < D; c0 += 16) {
+      for (int c0 = 64 * ch; c0 < 64 * ch + 64; c0 += 16) {
         float sv[16];
         tmem_ld16(lanebase + c0, sv);
         tmem_wait_ld();
@@ -205,14 +206,15 @@ __global__ void __launch_bounds__(kSbThreads, 1) tc_state_bwd_kernel(BwdTcArgs t
       tmem_wait_st();
     }
     {
-      const bool ok = mbar_wait(&ms.mu, s & 1, a.status, 302);
+      bool ok = true;
+      if (tid == 0) ok = mbar_wait(&ms.mu, s & 1, a.status, 302);
       if (__syncthreads_or(!ok)) { abort = true; break; }
     }
     tc_fence_after();
     // dU^T -> bf16 operand tile and the dU tile of this chunk
     {
       unsigned char *gdu = ta.dU_tiles + ((size_t)(first + j) * H + h) * DU_TILE;
-      for (int s0 = 0; s0 < 64; s0 += 16) {
+      for (int s0 = 32 * ch; s0 < 32 * ch + 32; s0 += 16) {
         float w[16];
         tmem_ld16(lanebase + 128 + s0, w);
         tmem_wait_ld();
@@ -244,13 +246,14 @@ __global__ void __launch_bounds__(kSbThreads, 1) tc_state_bwd_kernel(BwdTcArgs t
       mma_commit(&ms.ms);
     }
     {
-      const bool ok = mbar_wait(&ms.ms, s & 1, a.status, 303);
+      bool ok = true;
+      if (tid == 0) ok = mbar_wait(&ms.ms, s & 1, a.status, 303);
       if (__syncthreads_or(!ok)) { abort = true; break; }
     }
     tc_fence_after();
     if (tid == 0 && s + 2 < nc) issue_record(s + 2);
     // dS at the start of chunk j: next step's operand, snapshot of chunk j-1, or dS0
-    for (int c0 = 0; c0 < D; c0 += 16) {
+    for (int c0 = 64 * ch; c0 < 64 * ch + 64; c0 += 16) {
       float sv[16];
       tmem_ld16(lanebase + c0, sv);
       tmem_wait_ld();
@@ -301,14 +304,22 @@ struct GMisc {
   uint32_t tmem;
   int pad;
   float beta[64], dbc[64], dbr[2][64];
-  float totG[2][128];
-  uint32_t totP[2][128];
+  PrepTot tot;
+  uint8_t pbits[8][128];
   float dd[2][128];
-  float gcp[2][128];
-  float acc1[128];
-  float X[3][16][16];
 };
+// scratch that lives in tiles idle at the time: inverse blocks in the free
+// tail of the N-matrix region, final-epilogue sums in the [U; V] tile
+constexpr uint32_t G_XS = G_WN + 17408;  // float [3][16][16]
 
+// Completion of MMAs (or of a copy only MMAs consume): one thread polls the
+// mbarrier, the others wait at the CTA barrier (no spinning issue slots).
+__device__ __forceinline__ bool wait_one(uint64_t *bar, uint32_t phase, DevStatus *st, uint32_t site) {
+  bool ok = true;
+  if (threadIdx.x == 0) ok = mbar_wait(bar, phase, st, site);
+  return !__syncthreads_or(!ok);
+}
+// Completion of a copy whose data every thread reads: every thread observes it.
 __device__ __forceinline__ bool wait_all(uint64_t *bar, uint32_t phase, DevStatus *st, uint32_t site) {
   const bool ok = mbar_wait(bar, phase, st, site);
   return !__syncthreads_or(!ok);
@@ -350,6 +361,9 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(BwdTcArgs ta) {
   float *dTf = reinterpret_cast<float *>(sm + G_DT);
   float *Mf = reinterpret_cast<float *>(sm + G_MF);
   float *tmpf = reinterpret_cast<float *>(sm + G_KG);  // [64][64]
+  float(*Xs)[16][16] = reinterpret_cast<float(*)[16][16]>(sm + G_XS);
+  float *gcps = reinterpret_cast<float *>(sm + G_UV);         // [2][128], final epilogue only
+  float *acc1s = gcps + 256;                                  // [128]
   float *fb = ta.fb + (size_t)blockIdx.x * 3 * 64 * D;
 
   const int c = tid & 127, hf = tid >> 7;
@@ -375,77 +389,78 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(BwdTcArgs ta) {
       bulk_g2s(sm + G_OU + 8192, gdU, 8192, &ms.mdu);
       bulk_g2s(sm + G_OU + 16384 + 8192, gdU + 8192, 8192, &ms.mdu);
     }
-    float G[32];
-    uint32_t kq[32];
-    uint32_t neg;
-    load_rows(a.g, a.sign, k, q, tok0, len, h, H, c, hf, G, kq, neg);
-    for (int e = tid; e < 64 * 16; e += kGThreads) {
-      const int j = e >> 4, cc = e & 15;
-      uint4 vv = make_uint4(0, 0, 0, 0), oo = vv;
-      if (j < len) {
-        const size_t off = ((size_t)(tok0 + j) * H + h) * D + cc * 8;
-        vv = *reinterpret_cast<const uint4 *>(v + off);
-        oo = *reinterpret_cast<const uint4 *>(dO + off);
+    Prep P;  // row-group layout: rows 8 warp .., channels 4 lane ..
+    prep_load(a.g, a.sign, k, q, tok0, len, h, H, warp, lane, P, ms.tot);
+    {  // V and dO rows (all loads in flight before the stores)
+      uint4 vv[4], oo[4];
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const int e = tid + kGThreads * m, j = e >> 4, cc = e & 15;
+        const int jj = j < len ? j : len - 1;
+        const size_t off = ((size_t)(tok0 + jj) * H + h) * D + cc * 8;
+        vv[m] = *reinterpret_cast<const uint4 *>(v + off);
+        oo[m] = *reinterpret_cast<const uint4 *>(dO + off);
       }
-      *reinterpret_cast<uint4 *>(sm + G_UV + kmaj_off(64 + j, cc * 8, 128)) = vv;
-      *reinterpret_cast<uint4 *>(sm + G_OU + kmaj_off(j, cc * 8, 128)) = oo;
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const int e = tid + kGThreads * m, j = e >> 4, cc = e & 15;
+        if (j >= len) vv[m] = oo[m] = make_uint4(0, 0, 0, 0);
+        *reinterpret_cast<uint4 *>(sm + G_UV + kmaj_off(64 + j, cc * 8, 128)) = vv[m];
+        *reinterpret_cast<uint4 *>(sm + G_OU + kmaj_off(j, cc * 8, 128)) = oo[m];
+      }
     }
-    for (int rr = warp; rr < D; rr += 8) {  // S_c fp32 row rr -> bf16 K-major [c][v]
-      const float4 x = *reinterpret_cast<const float4 *>(Sc + (size_t)rr * D + 4 * lane);
-      uint2 pk = make_uint2(pack_bf16(x.x, x.y), pack_bf16(x.z, x.w));
-      *reinterpret_cast<uint2 *>(sm + G_SC + kmaj_off(rr, 4 * lane, 128)) = pk;
+    {  // S_c fp32 rows -> bf16 K-major [c][v]; 16 rows per warp, all loads in flight
+      float4 x[16];
+#pragma unroll
+      for (int m = 0; m < 16; ++m) x[m] = *reinterpret_cast<const float4 *>(Sc + (size_t)(warp + 8 * m) * D + 4 * lane);
+#pragma unroll
+      for (int m = 0; m < 16; ++m)
+        *reinterpret_cast<uint2 *>(sm + G_SC + kmaj_off(warp + 8 * m, 4 * lane, 128)) =
+            make_uint2(pack_bf16(x[m].x, x[m].y), pack_bf16(x[m].z, x[m].w));
     }
     if (tid < 64) ms.beta[tid] = tid < len ? __bfloat162float(beta[(size_t)(tok0 + tid) * H + h]) : 0.f;
-    uint32_t par = 0, pre = 0;
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      par ^= (neg >> i) & 1u;
-      pre |= par << i;
-    }
-    ms.totG[hf][c] = G[31];
-    ms.totP[hf][c] = par;
     __syncthreads();
-    if (hf == 1) {
-      const float cg = ms.totG[0][c];
-#pragma unroll
-      for (int i = 0; i < 32; ++i) G[i] += cg;
-      if (ms.totP[0][c]) pre = ~pre;
-    }
-    const float Gm = ms.totG[0][c];
-    const float GC = ms.totG[0][c] + ms.totG[1][c];
-    const float pCs = (ms.totP[0][c] ^ ms.totP[1][c]) ? -1.f : 1.f;
+    prep_carry(warp, lane, P, ms.tot);
     int bad = 0;
 #pragma unroll
-    for (int i = 0; i < 32; ++i)
-      if (!(fabsf(G[i] - Gm) <= kTau)) bad = 1;
+    for (int rr = 0; rr < 8; ++rr)
+#pragma unroll
+      for (int m = 0; m < 4; ++m)
+        if (!(fabsf(P.G[rr][m] - P.Gm[m]) <= kTau)) bad = 1;
     const bool fast = !__syncthreads_or(bad);
-    const float eGm = fast_exp(Gm), eCm = fast_exp(GC - Gm);
-    const float dC = pCs * fast_exp(GC);
 
     // ---------------- operand tiles ----------------
-    if (fast) {
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const int r = 32 * hf + i;
-        const float p = ((pre >> i) & 1u) ? -1.f : 1.f;
-        const float kp = p * __uint_as_float(kq[i] << 16), qp = p * __uint_as_float(kq[i] & 0xffff0000u);
-        const float el = fast_exp(G[i] - Gm), er = __frcp_rn(el);
-        st_bf16(sm + G_A1, kmaj_off(r, c, 128), qp * el);
-        st_bf16(sm + G_A1, kmaj_off(64 + r, c, 128), kp * el);
-        st_bf16(sm + G_B1, kmaj_off(r, c, 64), kp * er);
-        st_bf16(sm + G_KG, mnmaj_off(r, c, 64), kp * el * eGm);
-      }
-    } else {
+    for (int rr = 0; rr < 8; ++rr) {
+      const int r = 8 * warp + rr;
+      float ql[4], kl[4], kr[4], kgv[4];
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const int r = 32 * hf + i;
-        const float p = ((pre >> i) & 1u) ? -1.f : 1.f;
-        const float kp = p * __uint_as_float(kq[i] << 16), qp = p * __uint_as_float(kq[i] & 0xffff0000u);
-        fb[r * D + c] = G[i];
-        fb[64 * D + r * D + c] = kp;
-        fb[128 * D + r * D + c] = qp;
-        st_bf16(sm + G_KG, mnmaj_off(r, c, 64), kp * fast_exp(G[i]));
+      for (int m = 0; m < 4; ++m) {
+        const float p = prep_p(P, rr, m);
+        const float kp = p * prep_k(P, rr, m), qp = p * prep_q(P, rr, m);
+        if (fast) {
+          const float el = fast_exp(P.G[rr][m] - P.Gm[m]), er = __frcp_rn(el);
+          ql[m] = qp * el;
+          kl[m] = kp * el;
+          kr[m] = kp * er;
+          kgv[m] = kl[m] * fast_exp(P.Gm[m]);
+        } else {
+          ql[m] = qp;
+          kl[m] = kp;
+          kr[m] = P.G[rr][m];
+          kgv[m] = kp * fast_exp(P.G[rr][m]);
+        }
       }
+      if (fast) {
+        st_bf16x4(sm + G_A1, kmaj_off(r, 4 * lane, 128), ql[0], ql[1], ql[2], ql[3]);
+        st_bf16x4(sm + G_A1, kmaj_off(64 + r, 4 * lane, 128), kl[0], kl[1], kl[2], kl[3]);
+        st_bf16x4(sm + G_B1, kmaj_off(r, 4 * lane, 64), kr[0], kr[1], kr[2], kr[3]);
+      } else {
+        *reinterpret_cast<float4 *>(fb + r * D + 4 * lane) = make_float4(kr[0], kr[1], kr[2], kr[3]);
+        *reinterpret_cast<float4 *>(fb + 64 * D + r * D + 4 * lane) = make_float4(kl[0], kl[1], kl[2], kl[3]);
+        *reinterpret_cast<float4 *>(fb + 128 * D + r * D + 4 * lane) = make_float4(ql[0], ql[1], ql[2], ql[3]);
+      }
+      st_bf16x4(sm + G_KG, mnmaj_off(r, 4 * lane, 64), kgv[0], kgv[1], kgv[2], kgv[3]);
     }
     fence_async_smem();
     __syncthreads();
@@ -461,7 +476,7 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(BwdTcArgs ta) {
                    sdesc(sB1 + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), id, kk > 0);
         mma_commit(&ms.bar[0]);
       }
-      if (!wait_all(&ms.bar[0], ph, a.status, 401)) { abort = true; break; }
+      if (!wait_one(&ms.bar[0], ph, a.status, 401)) { abort = true; break; }
       tc_fence_after();
       if (qd >= 2) {  // lanes 64..127: rows of A
         const int r = 32 * qd + lane - 64, ch = warp >> 2;
@@ -512,14 +527,14 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(BwdTcArgs ta) {
         const int J = e >> 8, I = J + d, aa = (e >> 4) & 15, bb = e & 15;
         float s = 0.f;
         for (int u = 16 * J; u < 16 * I; ++u) s += Nf[(16 * I + aa) * LDF + u] * Mf[u * LDF + 16 * J + bb];
-        ms.X[J][aa][bb] = s;
+        Xs[J][aa][bb] = s;
       }
       __syncthreads();
       for (int e = tid; e < nb * 256; e += kGThreads) {
         const int J = e >> 8, I = J + d, aa = (e >> 4) & 15, bb = e & 15;
         float s = 0.f;
 #pragma unroll
-        for (int t = 0; t < 16; ++t) s += Mf[(16 * I + aa) * LDF + 16 * I + t] * ms.X[J][t][bb];
+        for (int t = 0; t < 16; ++t) s += Mf[(16 * I + aa) * LDF + 16 * I + t] * Xs[J][t][bb];
         Mf[(16 * I + aa) * LDF + 16 * J + bb] = -s;
       }
       __syncthreads();
@@ -549,7 +564,7 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(BwdTcArgs ta) {
       }
       mma_commit(&ms.bar[1]);
     }
-    if (!wait_all(&ms.bar[1], ph, a.status, 402)) { abort = true; break; }
+    if (!wait_one(&ms.bar[1], ph, a.status, 402)) { abort = true; break; }
     tc_fence_after();
     {  // W^T -> W tile, MN-major B [K = c][N = r] (over the dead N matrix)
       const int ch = warp >> 2;
@@ -581,7 +596,7 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(BwdTcArgs ta) {
                  kk > 0);
       mma_commit(&ms.bar[2]);
     }
-    if (!wait_all(&ms.bar[2], ph, a.status, 403)) { abort = true; break; }
+    if (!wait_one(&ms.bar[2], ph, a.status, 403)) { abort = true; break; }
     tc_fence_after();
     if (tid == 0) {  // the W tile is dead: bring dL/dS_{c+1} into its place
       mbar_arrive_expect_tx(&ms.mds, DS_TILE);
@@ -613,7 +628,7 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(BwdTcArgs ta) {
       }
       ms.dd[hf][c] = s;
     }
-    if (!wait_all(&ms.mdu, ph, a.status, 405)) { abort = true; break; }
+    if (!wait_one(&ms.mdu, ph, a.status, 405)) { abort = true; break; }
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -631,7 +646,7 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(BwdTcArgs ta) {
       }
       mma_commit(&ms.bar[3]);
     }
-    if (!wait_all(&ms.bar[3], ph, a.status, 406)) { abort = true; break; }
+    if (!wait_one(&ms.bar[3], ph, a.status, 406)) { abort = true; break; }
     tc_fence_after();
     {  // dW = -dU S_c^T -> rows 64..127 of the S_c tile (K-major [i][c]); S_c is dead
       const int ch = warp >> 2;
@@ -664,7 +679,7 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(BwdTcArgs ta) {
                  sdesc(sKG + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), id2, true);
       mma_commit(&ms.bar[4]);
     }
-    if (!wait_all(&ms.bar[4], ph, a.status, 407)) { abort = true; break; }
+    if (!wait_one(&ms.bar[4], ph, a.status, 407)) { abort = true; break; }
     tc_fence_after();
     {
       const int ch = warp >> 2;
@@ -712,22 +727,61 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(BwdTcArgs ta) {
     __syncthreads();
     for (int e = tid; e < 64 * 64; e += kGThreads) dTf[(e >> 6) * LDF + (e & 63)] *= ms.beta[e & 63];
     __syncthreads();
-    // tmp = dM M^T  (tmp[i][kk] = sum_{j <= min(i, kk)} dM[i][j] M[kk][j])
-    for (int e = tid; e < 64 * 64; e += kGThreads) {
-      const int i = e >> 6, kk = e & 63;
-      const int jm = i < kk ? i : kk;
-      float s = 0.f;
-      for (int j = 0; j <= jm; ++j) s += dTf[i * LDF + j] * Mf[kk * LDF + j];
-      tmpf[i * 64 + kk] = s;
+    // tmp = dM M^T  (tmp[i][kk] = sum_{j <= min(i, kk)} dM[i][j] M[kk][j]), 4 x 4 per thread;
+    // dM and M are lower triangular, so the extra j of a tile contribute zeros
+    {
+      const int i0 = (tid >> 4) * 4, k0 = (tid & 15) * 4;
+      const int jmax = (i0 < k0 ? i0 : k0) + 3;
+      float acc[4][4];
+#pragma unroll
+      for (int m = 0; m < 4; ++m)
+#pragma unroll
+        for (int n = 0; n < 4; ++n) acc[m][n] = 0.f;
+      for (int j = 0; j <= jmax; ++j) {
+        float a4[4], b4[4];
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          a4[m] = dTf[(i0 + m) * LDF + j];
+          b4[m] = Mf[(k0 + m) * LDF + j];
+        }
+#pragma unroll
+        for (int m = 0; m < 4; ++m)
+#pragma unroll
+          for (int n = 0; n < 4; ++n) acc[m][n] += a4[m] * b4[n];
+      }
+#pragma unroll
+      for (int m = 0; m < 4; ++m)
+        *reinterpret_cast<float4 *>(tmpf + (i0 + m) * 64 + k0) = make_float4(acc[m][0], acc[m][1], acc[m][2], acc[m][3]);
     }
     __syncthreads();
-    // dL = -M^T tmp, strict lower -> dN (into dTf)
-    for (int e = tid; e < 64 * 64; e += kGThreads) {
-      const int aa = e >> 6, kk = e & 63;
-      float s = 0.f;
-      if (kk < aa)
-        for (int i = aa; i < 64; ++i) s -= Mf[i * LDF + aa] * tmpf[i * 64 + kk];
-      dTf[aa * LDF + kk] = s;  // overwrites dM row aa: dM is dead (tmp holds it)
+    // dL = -M^T tmp, strict lower -> dN (into dTf; dM is dead), 4 x 4 per thread
+    {
+      const int a0 = (tid >> 4) * 4, k0 = (tid & 15) * 4;
+      float acc[4][4];
+#pragma unroll
+      for (int m = 0; m < 4; ++m)
+#pragma unroll
+        for (int n = 0; n < 4; ++n) acc[m][n] = 0.f;
+      if (k0 <= a0 + 2)
+        for (int i = a0; i < 64; ++i) {  // M[i][a] = 0 for i < a
+          float m4[4];
+#pragma unroll
+          for (int m = 0; m < 4; ++m) m4[m] = Mf[i * LDF + a0 + m];
+          const float4 t4 = *reinterpret_cast<const float4 *>(tmpf + i * 64 + k0);
+          const float tt[4] = {t4.x, t4.y, t4.z, t4.w};
+#pragma unroll
+          for (int m = 0; m < 4; ++m)
+#pragma unroll
+            for (int n = 0; n < 4; ++n) acc[m][n] += m4[m] * tt[n];
+        }
+      __syncthreads();  // every read of dM (dTf) and tmp is done before dN overwrites dTf
+#pragma unroll
+      for (int m = 0; m < 4; ++m)
+#pragma unroll
+        for (int n = 0; n < 4; ++n) {
+          const int aa = a0 + m, kk = k0 + n;
+          dTf[aa * LDF + kk] = kk < aa ? -acc[m][n] : 0.f;
+        }
     }
     __syncthreads();
     // dA = Diag(beta) dN -> bf16 rows 0..63 of the [dA; dA_q] tile; dbeta (row part)
@@ -837,68 +891,100 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(BwdTcArgs ta) {
       }
       tmem_wait_st();
     }
-    if (!wait_all(&ms.bar[5], ph, a.status, 408)) { abort = true; break; }
+    if (!wait_one(&ms.bar[5], ph, a.status, 408)) { abort = true; break; }
     tc_fence_after();
 
     // ---------------- final elementwise gradients ----------------
+    // hand the prep values from the row-group layout to the channel layout
+    // (lane = key channel, as TMEM rows are) through the now idle tiles
+    float *Gs = reinterpret_cast<float *>(sm + G_A1);              // [64][128] Gam
+    uint32_t *KQs = reinterpret_cast<uint32_t *>(sm + G_B1);       // [64][128] k' | q' << 16
+#pragma unroll
+    for (int rr = 0; rr < 8; ++rr) {
+      const int r = 8 * warp + rr;
+      *reinterpret_cast<float4 *>(Gs + r * D + 4 * lane) = make_float4(P.G[rr][0], P.G[rr][1], P.G[rr][2], P.G[rr][3]);
+      uint32_t kq4[4];
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const float p = prep_p(P, rr, m);
+        kq4[m] = pack_bf16(p * prep_k(P, rr, m), p * prep_q(P, rr, m));
+      }
+      *reinterpret_cast<uint4 *>(KQs + r * D + 4 * lane) = make_uint4(kq4[0], kq4[1], kq4[2], kq4[3]);
+    }
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      uint32_t bits = 0;
+#pragma unroll
+      for (int rr = 0; rr < 8; ++rr) bits |= ((P.pre >> (4 * rr + m)) & 1u) << rr;
+      ms.pbits[warp][4 * lane + m] = (uint8_t)bits;
+    }
+    __syncthreads();
     {
       // thread (c, hf): rows 32 hf .. 32 hf + 31 of key channel c
+      float Gm = 0.f, GC = 0.f;
+      uint32_t pcb = 0;
+#pragma unroll
+      for (int ww = 0; ww < 8; ++ww) {
+        const float t = ms.tot.G[ww][c];
+        if (ww <= 3) Gm += t;
+        GC += t;
+        pcb ^= ms.tot.P[ww][c];
+      }
+      const float pCs = pcb ? -1.f : 1.f;
+      const float eGm = fast_exp(Gm), eCm = fast_exp(GC - Gm);
+      const float dC = pCs * fast_exp(GC);
       float dG[32];
       float gcp = 0.f;
 #pragma unroll
-      for (int b16 = 0; b16 < 2; ++b16) {
-        const uint32_t colo = 32 * hf + 16 * b16;
-        float X1[16], X2[16], Y1[16], dQG[16], dKG[16], dKh[16];
-        tmem_ld16(lanebase + 128 + colo, X1);
-        tmem_ld16(lanebase + 192 + colo, X2);
-        tmem_ld16(lanebase + 320 + colo, Y1);
-        tmem_ld16(lanebase + 256 + colo, dQG);
-        tmem_ld16(lanebase + 64 + colo, dKG);
-        tmem_ld16(lanebase + 384 + colo, dKh);
+      for (int b8 = 0; b8 < 4; ++b8) {
+        const uint32_t colo = 32 * hf + 8 * b8;
+        float X1[8], X2[8], Y1[8], dQG[8], dKG[8], dKh[8], dVv[8];
+        tmem_ld8(lanebase + 128 + colo, X1);
+        tmem_ld8(lanebase + 192 + colo, X2);
+        tmem_ld8(lanebase + 320 + colo, Y1);
+        tmem_ld8(lanebase + 256 + colo, dQG);
+        tmem_ld8(lanebase + 64 + colo, dKG);
+        tmem_ld8(lanebase + 384 + colo, dKh);
+        tmem_ld8(lanebase + 448 + colo, dVv);
         tmem_wait_ld();
+        const uint32_t pb = ms.pbits[(32 * hf + 8 * b8) >> 3][c];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int ii = 16 * b16 + i;
+        for (int i = 0; i < 8; ++i) {
+          const int ii = 8 * b8 + i;
           const int r = 32 * hf + ii;
-          const float p = ((pre >> ii) & 1u) ? -1.f : 1.f;
-          const float kp = p * __uint_as_float(kq[ii] << 16), qp = p * __uint_as_float(kq[ii] & 0xffff0000u);
+          const float Gr = Gs[r * D + c];
+          const uint32_t kqv = KQs[r * D + c];
+          const float kp = bf_lo(kqv), qp = bf_hi(kqv);
+          const float p = ((pb >> i) & 1u) ? -1.f : 1.f;
           float el, er, E, eC;
           if (fast) {
-            el = fast_exp(G[ii] - Gm);
+            el = fast_exp(Gr - Gm);
             er = __frcp_rn(el);
             E = el * eGm;
             eC = er * eCm;
           } else {
             el = 1.f;
             er = 1.f;
-            E = fast_exp(G[ii]);
-            eC = fast_exp(GC - G[ii]);
+            E = fast_exp(Gr);
+            eC = fast_exp(GC - Gr);
           }
           const float x1 = el * X1[i], x2 = el * X2[i], y1 = er * Y1[i];
-          const float KG = kp * E, QG = qp * E, Kh = pCs * kp * eC;
+          const float KGv = kp * E, QGv = qp * E, Kh = pCs * kp * eC;
           const float dkp = x1 + y1 + dKG[i] * E + pCs * dKh[i] * eC;
           const float dqp = x2 + dQG[i] * E;
-          dG[ii] = kp * x1 + qp * x2 - kp * y1 + dKG[i] * KG + dQG[i] * QG - dKh[i] * Kh;
+          dG[ii] = kp * x1 + qp * x2 - kp * y1 + dKG[i] * KGv + dQG[i] * QGv - dKh[i] * Kh;
           gcp += dKh[i] * Kh;
           if (r < len) {
             const size_t off = ((size_t)(tok0 + r) * H + h) * D + c;
             dq[off] = __float2bfloat16_rn(p * dqp);
             dk[off] = __float2bfloat16_rn(p * dkp);
+            dv[off] = __float2bfloat16_rn(dVv[i]);  // lane c is value channel c here
           }
         }
-        // dV^T lanes = value channel, columns = token
-        float dVv[16];
-        tmem_ld16(lanebase + 448 + colo, dVv);
-        tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int j = 32 * hf + 16 * b16 + i;
-          if (j < len) dv[((size_t)(tok0 + j) * H + h) * D + c] = __float2bfloat16_rn(dVv[i]);
-        }
       }
-      ms.gcp[hf][c] = gcp;
+      gcps[hf * 128 + c] = gcp;
       __syncthreads();
-      const float gC = ms.gcp[0][c] + ms.gcp[1][c] + (ms.dd[0][c] + ms.dd[1][c]) * dC;
+      const float gC = gcps[c] + gcps[128 + c] + (ms.dd[0][c] + ms.dd[1][c]) * dC;
       // reverse in-chunk cumsum: the upper half first, then the lower half continues
       if (hf == 1) {
         float acc = gC;
@@ -908,11 +994,11 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(BwdTcArgs ta) {
           const int r = 32 + ii;
           if (r < len) a.dg[((size_t)(tok0 + r) * H + h) * D + c] = acc;
         }
-        ms.acc1[c] = acc;
+        acc1s[c] = acc;
       }
       __syncthreads();
       if (hf == 0) {
-        float acc = ms.acc1[c];
+        float acc = acc1s[c];
 #pragma unroll
         for (int ii = 31; ii >= 0; --ii) {
           acc += dG[ii];
@@ -978,5 +1064,7 @@ cudaError_t tc_backward(const BwdArgs &b, const unsigned char *recs, unsigned ch
 }
 
 size_t tc_bwd_smem_bytes() { return G_MISC + sizeof(GMisc) + 1024; }
+static_assert(G_MISC + sizeof(GMisc) + 1024 <= 232448, "gradient kernel shared memory");
+static_assert(G_XS + 3 * 16 * 16 * 4 <= G_WN + 33792, "inverse scratch inside the N region");
 
 }  // namespace ckda

@@ -60,10 +60,7 @@ struct IntraMisc {
   uint32_t tmem;
   int flag;
   float beta[64];
-  float totG[2][128];
-  uint32_t totP[2][128];
-  float Gm[128], eGm[128], eCm[128], GamC[128];
-  uint32_t pC[128];
+  PrepTot tot;
   float X[3][16][16];
 };
 
@@ -106,7 +103,6 @@ __global__ void __launch_bounds__(kIntraThreads, 2) tc_intra_kernel(TcArgs ta) {
   float *Mf = reinterpret_cast<float *>(sm + I_MF);
   float *fb = ta.fb + (size_t)blockIdx.x * 3 * 64 * D;
 
-  const int c = tid & 127, hf = tid >> 7;
   const int nitems = a.map.n_chunks() * H;
   uint32_t it = 0;
   bool abort = false;
@@ -117,103 +113,98 @@ __global__ void __launch_bounds__(kIntraThreads, 2) tc_intra_kernel(TcArgs ta) {
     a.map.info(cid, seq, tok0, len, jl);
     unsigned char *rec = ta.recs + (size_t)item * REC;
 
-    // ---------------- prep, pass 1: local scans over 32 rows ----------------
-    float G[32];
-    uint32_t kq[32];   // bf16 k (low half) and q (high half) of each row
-    uint32_t neg = 0;  // bit i: sign of row 32*hf + i is negative
-    load_rows(a.g, a.sign, k, q, tok0, len, h, H, c, hf, G, kq, neg);
-    // prefix parity of the sign bits
-    uint32_t par = 0, pre = 0;
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      par ^= (neg >> i) & 1u;
-      pre |= par << i;
-    }
-    ms.totG[hf][c] = G[31];
-    ms.totP[hf][c] = par;
+    // ---------------- prep: row-group layout (rows 8w.., channels 4l..) ----------------
+    Prep P;
+    prep_load(a.g, a.sign, k, q, tok0, len, h, H, warp, lane, P, ms.tot);
     // V tile (MN-major A operand, K = token j, M = value channel)
-    for (int e = tid; e < 64 * 16; e += kIntraThreads) {
-      const int j = e >> 4, cc = e & 15;
-      uint4 val = make_uint4(0, 0, 0, 0);
-      if (j < len)
-        val = *reinterpret_cast<const uint4 *>(v + ((size_t)(tok0 + j) * H + h) * D + cc * 8);
-      *reinterpret_cast<uint4 *>(sm + I_V + mnmaj_off(j, cc * 8, 64)) = val;
+    {
+      uint4 vv[4];
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const int e = tid + kIntraThreads * m, j = e >> 4, cc = e & 15;
+        const int jj = j < len ? j : len - 1;
+        vv[m] = *reinterpret_cast<const uint4 *>(v + ((size_t)(tok0 + jj) * H + h) * D + cc * 8);
+      }
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const int e = tid + kIntraThreads * m, j = e >> 4, cc = e & 15;
+        *reinterpret_cast<uint4 *>(sm + I_V + mnmaj_off(j, cc * 8, 64)) =
+            j < len ? vv[m] : make_uint4(0, 0, 0, 0);
+      }
     }
     if (tid < 64) ms.beta[tid] = tid < len ? __bfloat162float(beta[(size_t)(tok0 + tid) * H + h]) : 0.f;
     __syncthreads();
-
-    // ---------------- carry, reference row, range check ----------------
-    if (hf == 1) {
-      const float cg = ms.totG[0][c];
-      const uint32_t cp = ms.totP[0][c] ? 0xffffffffu : 0u;
-#pragma unroll
-      for (int i = 0; i < 32; ++i) G[i] += cg;
-      pre ^= cp;
-    }
-    const float Gm = ms.totG[0][c];
-    const float GC = ms.totG[0][c] + ms.totG[1][c];
-    const uint32_t pCneg = ms.totP[0][c] ^ ms.totP[1][c];
+    prep_carry(warp, lane, P, ms.tot);
     int bad = 0;
 #pragma unroll
-    for (int i = 0; i < 32; ++i)
-      if (!(fabsf(G[i] - Gm) <= kTau)) bad = 1;
-    const bool fast = !__syncthreads_or(bad);
-    const float eGm = fast_exp(Gm);
-    const float eCm = fast_exp(GC - Gm);
-    const float pCs = pCneg ? -1.f : 1.f;
-    if (hf == 0) {
-      reinterpret_cast<float *>(rec + R5)[c] = pCs * fast_exp(GC);
-      ms.Gm[c] = Gm;
-      ms.GamC[c] = GC;
-      ms.pC[c] = pCneg;
-    }
-
-    // ---------------- prep, pass 2: operand tiles and record tiles ----------------
-    if (fast) {
-      uint32_t qg_pack[16], kh_pack[16];
+    for (int rr = 0; rr < 8; ++rr)
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const int r = 32 * hf + i;
-        const float p = ((pre >> i) & 1u) ? -1.f : 1.f;
-        const float kp = p * __uint_as_float(kq[i] << 16), qp = p * __uint_as_float(kq[i] & 0xffff0000u);
-        const float el = fast_exp(G[i] - Gm);
-        const float er = __frcp_rn(el);
-        const float ql = qp * el, kl = kp * el, kr = kp * er;
-        st_bf16(sm + I_A1, kmaj_off(r, c, 128), ql);
-        st_bf16(sm + I_A1, kmaj_off(64 + r, c, 128), kl);
-        st_bf16(sm + I_B1, kmaj_off(r, c, 64), kr);
-        st_bf16(sm + I_KG, mnmaj_off(r, c, 64), kl * eGm);
-        const float qg = ql * eGm, kh = pCs * kr * eCm;
-        if (i & 1) {
-          qg_pack[i >> 1] |= (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(qg)) << 16;
-          kh_pack[i >> 1] |= (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(kh)) << 16;
-        } else {
-          qg_pack[i >> 1] = __bfloat16_as_ushort(__float2bfloat16_rn(qg));
-          kh_pack[i >> 1] = __bfloat16_as_ushort(__float2bfloat16_rn(kh));
+      for (int m = 0; m < 4; ++m)
+        if (!(fabsf(P.G[rr][m] - P.Gm[m]) <= kTau)) bad = 1;
+    const bool fast = !__syncthreads_or(bad);
+    float eGm[4], eCm[4], pCs[4];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      eGm[m] = fast_exp(P.Gm[m]);
+      eCm[m] = fast_exp(P.GC[m] - P.Gm[m]);
+      pCs[m] = ((P.pC >> m) & 1u) ? -1.f : 1.f;
+    }
+    if (warp == 0)
+      *reinterpret_cast<float4 *>(rec + R5 + 16 * lane) =
+          make_float4(pCs[0] * fast_exp(P.GC[0]), pCs[1] * fast_exp(P.GC[1]), pCs[2] * fast_exp(P.GC[2]),
+                      pCs[3] * fast_exp(P.GC[3]));
+
+    // ---------------- operand tiles and record tiles ----------------
+    {
+      float qg[8][4], kh[8][4];
+#pragma unroll
+      for (int rr = 0; rr < 8; ++rr) {
+        const int r = 8 * warp + rr;
+        float ql[4], kl[4], kr[4], kgv[4];
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          const float p = prep_p(P, rr, m);
+          const float kp = p * prep_k(P, rr, m), qp = p * prep_q(P, rr, m);
+          if (fast) {
+            const float el = fast_exp(P.G[rr][m] - P.Gm[m]);
+            const float er = __frcp_rn(el);
+            ql[m] = qp * el;
+            kl[m] = kp * el;
+            kr[m] = kp * er;
+            kgv[m] = kl[m] * eGm[m];
+            qg[rr][m] = ql[m] * eGm[m];
+            kh[rr][m] = pCs[m] * kr[m] * eCm[m];
+          } else {
+            const float E = fast_exp(P.G[rr][m]);
+            kgv[m] = kp * E;
+            qg[rr][m] = qp * E;
+            kh[rr][m] = pCs[m] * kp * fast_exp(P.GC[m] - P.G[rr][m]);
+            ql[m] = qp;  // kept for the exact pair sums below
+            kl[m] = kp;
+            kr[m] = P.G[rr][m];
+          }
         }
+        if (fast) {
+          st_bf16x4(sm + I_A1, kmaj_off(r, 4 * lane, 128), ql[0], ql[1], ql[2], ql[3]);
+          st_bf16x4(sm + I_A1, kmaj_off(64 + r, 4 * lane, 128), kl[0], kl[1], kl[2], kl[3]);
+          st_bf16x4(sm + I_B1, kmaj_off(r, 4 * lane, 64), kr[0], kr[1], kr[2], kr[3]);
+        } else {
+          *reinterpret_cast<float4 *>(fb + r * D + 4 * lane) = make_float4(kr[0], kr[1], kr[2], kr[3]);
+          *reinterpret_cast<float4 *>(fb + 64 * D + r * D + 4 * lane) = make_float4(kl[0], kl[1], kl[2], kl[3]);
+          *reinterpret_cast<float4 *>(fb + 128 * D + r * D + 4 * lane) = make_float4(ql[0], ql[1], ql[2], ql[3]);
+        }
+        st_bf16x4(sm + I_KG, mnmaj_off(r, 4 * lane, 64), kgv[0], kgv[1], kgv[2], kgv[3]);
       }
-      // QG^T row c (N index 64 + r) and Khat^T row c (K index r): 4 chunks each
+      // QG^T (N index 64 + r) and Khat^T (K index r) of each channel: one 16-byte chunk
 #pragma unroll
       for (int m = 0; m < 4; ++m) {
-        const uint4 vq = make_uint4(qg_pack[4 * m], qg_pack[4 * m + 1], qg_pack[4 * m + 2], qg_pack[4 * m + 3]);
-        const uint4 vk = make_uint4(kh_pack[4 * m], kh_pack[4 * m + 1], kh_pack[4 * m + 2], kh_pack[4 * m + 3]);
-        *reinterpret_cast<uint4 *>(rec + R1 + mnmaj_off(c, 64 + 32 * hf + 8 * m, 128)) = vq;
-        *reinterpret_cast<uint4 *>(rec + R4 + kmaj_off(c, 32 * hf + 8 * m, 128)) = vk;
-      }
-    } else {
-      // exact path: keep Gam, k', q' for the per-pair sums; KG, QG, Khat direct
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const int r = 32 * hf + i;
-        const float p = ((pre >> i) & 1u) ? -1.f : 1.f;
-        const float kp = p * __uint_as_float(kq[i] << 16), qp = p * __uint_as_float(kq[i] & 0xffff0000u);
-        fb[r * D + c] = G[i];
-        fb[64 * D + r * D + c] = kp;
-        fb[128 * D + r * D + c] = qp;
-        const float E = fast_exp(G[i]);
-        st_bf16(sm + I_KG, mnmaj_off(r, c, 64), kp * E);
-        st_bf16(rec, R1 + mnmaj_off(c, 64 + r, 128), qp * E);
-        st_bf16(rec, R4 + kmaj_off(c, r, 128), pCs * kp * fast_exp(GC - G[i]));
+        const int cch = 4 * lane + m;
+        *reinterpret_cast<uint4 *>(rec + R1 + mnmaj_off(cch, 64 + 8 * warp, 128)) =
+            make_uint4(pack_bf16(qg[0][m], qg[1][m]), pack_bf16(qg[2][m], qg[3][m]),
+                       pack_bf16(qg[4][m], qg[5][m]), pack_bf16(qg[6][m], qg[7][m]));
+        *reinterpret_cast<uint4 *>(rec + R4 + kmaj_off(cch, 8 * warp, 128)) =
+            make_uint4(pack_bf16(kh[0][m], kh[1][m]), pack_bf16(kh[2][m], kh[3][m]),
+                       pack_bf16(kh[4][m], kh[5][m]), pack_bf16(kh[6][m], kh[7][m]));
       }
     }
     fence_async_smem();
@@ -232,7 +223,8 @@ __global__ void __launch_bounds__(kIntraThreads, 2) tc_intra_kernel(TcArgs ta) {
         }
         mma_commit(&ms.mbar1);
       }
-      const bool ok = mbar_wait(&ms.mbar1, it & 1, a.status, 101);
+      bool ok = true;
+      if (tid == 0) ok = mbar_wait(&ms.mbar1, it & 1, a.status, 101);
       if (__syncthreads_or(!ok)) { abort = true; break; }
       tc_fence_after();
       const int qd = warp & 3, ch = warp >> 2;
@@ -348,7 +340,8 @@ __global__ void __launch_bounds__(kIntraThreads, 2) tc_intra_kernel(TcArgs ta) {
       mma_commit(&ms.mbar2);
     }
     {
-      const bool ok = mbar_wait(&ms.mbar2, it & 1, a.status, 102);
+      bool ok = true;
+      if (tid == 0) ok = mbar_wait(&ms.mbar2, it & 1, a.status, 102);
       if (__syncthreads_or(!ok)) { abort = true; break; }
     }
     tc_fence_after();
@@ -396,7 +389,7 @@ __global__ void __launch_bounds__(kIntraThreads, 2) tc_intra_kernel(TcArgs ta) {
 // ===========================================================================
 // sequential state kernel
 // ===========================================================================
-constexpr int kStateThreads = 128;
+constexpr int kStateThreads = 256;              // two warps per TMEM lane quadrant
 constexpr uint32_t S_REC0 = 0;
 constexpr uint32_t S_REC1 = REC_PAD;
 constexpr uint32_t S_TS = 2 * REC_PAD;          // S^T bf16, K-major [v][c] 128 x 128
@@ -408,15 +401,25 @@ struct StateMisc {
   uint32_t tmem;
 };
 
+__device__ __forceinline__ bool wait_one(uint64_t *bar, uint32_t phase, DevStatus *st, uint32_t site) {
+  bool ok = true;
+  if (threadIdx.x == 0) ok = mbar_wait(bar, phase, st, site);
+  return !__syncthreads_or(!ok);
+}
+
+// TMEM columns: S^T [0,128); per chunk parity p the MMA3/4 accumulator
+// [(W S)^T | O^T] at 128 + 128 p (so the next chunk's MMA3 can run while the
+// output rows of this chunk are written out).
 __global__ void __launch_bounds__(kStateThreads, 1) tc_state_kernel(TcArgs ta) {
   extern __shared__ unsigned char smem_raw[];
   unsigned char *sm = reinterpret_cast<unsigned char *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   StateMisc &ms = *reinterpret_cast<StateMisc *>(sm + S_MISC);
   const FwdArgs &a = ta.f;
-  const int tid = threadIdx.x, warp = tid >> 5;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int qd = warp & 3, ch = warp >> 2;
   const int h = blockIdx.x, seq = blockIdx.y, H = a.H;
-  const int v = tid;  // value channel = TMEM lane
+  const int v = 32 * qd + lane;  // value channel = TMEM lane
   __nv_bfloat16 *o = (__nv_bfloat16 *)a.o;
 
   int first;
@@ -433,17 +436,27 @@ __global__ void __launch_bounds__(kStateThreads, 1) tc_state_kernel(TcArgs ta) {
     mbar_fence_init();
   }
   if (warp == 0) {
-    tmem_alloc(&ms.tmem, 256);
+    tmem_alloc(&ms.tmem, 512);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = ms.tmem;
-  const uint32_t lanebase = tmem + ((uint32_t)(32 * warp) << 16);
+  const uint32_t lanebase = tmem + ((uint32_t)(32 * qd) << 16);
   unsigned char *recbuf[2] = {sm + S_REC0, sm + S_REC1};
   auto record = [&](int j) -> const unsigned char * {
     return ta.recs + ((size_t)(first + j) * H + h) * REC;
+  };
+  auto issue_mma3 = [&](int j) {
+    tc_fence_after();
+    const uint32_t id = idesc_bf16(128, 128, false, true);
+    const uint32_t sS = smem_u32(sm + S_TS), sR = smem_u32(recbuf[j & 1] + R1);
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk)
+      mma_bf16(tmem + 128 + 128 * (j & 1), sdesc(sS + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+               sdesc(sR + kk * 2048, 16384, 1024), id, kk > 0);
+    mma_commit(&ms.m3);
   };
   if (tid == 0) {
     for (int j = 0; j < 2 && j < nc; ++j) {
@@ -459,7 +472,7 @@ __global__ void __launch_bounds__(kStateThreads, 1) tc_state_kernel(TcArgs ta) {
     if (__syncthreads_or(!ok)) abort = true;
     if (!abort) {
       const float *d0 = reinterpret_cast<const float *>(recbuf[0] + R5);
-      for (int c0 = 0; c0 < D; c0 += 16) {
+      for (int c0 = 64 * ch; c0 < 64 * ch + 64; c0 += 16) {
         float sv[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) sv[i] = a.S0 ? a.S0[sbase + (size_t)(c0 + i) * D + v] : 0.f;
@@ -486,37 +499,21 @@ __global__ void __launch_bounds__(kStateThreads, 1) tc_state_kernel(TcArgs ta) {
   fence_async_smem();
   tc_fence_before();
   __syncthreads();
+  if (!abort && tid == 0 && nc > 0) issue_mma3(0);
 
   for (int j = 0; j < nc && !abort; ++j) {
     const int buf = j & 1;
     unsigned char *rec = recbuf[buf];
+    const uint32_t acc = 128 + 128 * buf;  // [(W S)^T | O^T] of this chunk
     int sq, len, jl;
     int64_t tok0;
     a.map.info(first + j, sq, tok0, len, jl);
-    {
-      const bool ok = mbar_wait(&ms.mrec[buf], (j >> 1) & 1, a.status, 202);
-      if (__syncthreads_or(!ok)) { abort = true; break; }
-    }
-    // MMA3: [(W S)^T | (QG S)^T] = S^T [W^T | QG^T]
-    if (tid == 0) {
-      tc_fence_after();
-      const uint32_t id = idesc_bf16(128, 128, false, true);
-      const uint32_t sS = smem_u32(sm + S_TS), sR = smem_u32(rec + R1);
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk)
-        mma_bf16(tmem + 128, sdesc(sS + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-                 sdesc(sR + kk * 2048, 16384, 1024), id, kk > 0);
-      mma_commit(&ms.m3);
-    }
-    {
-      const bool ok = mbar_wait(&ms.m3, j & 1, a.status, 203);
-      if (__syncthreads_or(!ok)) { abort = true; break; }
-    }
+    if (!wait_one(&ms.m3, j & 1, a.status, 203)) { abort = true; break; }
     tc_fence_after();
-    // U^T = U0^T - (W S)^T  -> bf16 K-major tile [v][s]
-    for (int s0 = 0; s0 < 64; s0 += 16) {
+    // U^T = U0^T - (W S)^T  -> bf16 K-major tile [v][s]; this thread: s in [32 ch, 32 ch + 32)
+    for (int s0 = 32 * ch; s0 < 32 * ch + 32; s0 += 16) {
       float w[16];
-      tmem_ld16(lanebase + 128 + s0, w);
+      tmem_ld16(lanebase + acc + s0, w);
       tmem_wait_ld();
       const uint4 u0a = *reinterpret_cast<const uint4 *>(rec + R2 + kmaj_off(v, s0, 128));
       const uint4 u0b = *reinterpret_cast<const uint4 *>(rec + R2 + kmaj_off(v, s0 + 8, 128));
@@ -545,33 +542,19 @@ __global__ void __launch_bounds__(kStateThreads, 1) tc_state_kernel(TcArgs ta) {
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk) {
         const uint64_t ad = sdesc(sU + kk * 32, 16, 1024);
-        mma_bf16(tmem + 192, ad, sdesc(smem_u32(rec + R3) + kk * 32, 16, 1024), id4, true);
+        mma_bf16(tmem + acc + 64, ad, sdesc(smem_u32(rec + R3) + kk * 32, 16, 1024), id4, true);
         mma_bf16(tmem + 0, ad, sdesc(smem_u32(rec + R4) + kk * 32, 16, 1024), id5, true);
       }
       mma_commit(&ms.m4);
     }
-    {
-      const bool ok = mbar_wait(&ms.m4, j & 1, a.status, 204);
-      if (__syncthreads_or(!ok)) { abort = true; break; }
-    }
+    if (!wait_one(&ms.m4, j & 1, a.status, 204)) { abort = true; break; }
     tc_fence_after();
     // the record buffer is free again: fetch chunk j + 2 into it
     if (tid == 0 && j + 2 < nc) {
       mbar_arrive_expect_tx(&ms.mrec[buf], REC);
       bulk_g2s(rec, record(j + 2), REC, &ms.mrec[buf]);
     }
-    // output rows of this chunk
-    if (ta.write_o) {
-      for (int r0 = 0; r0 < 64; r0 += 16) {
-        float ov[16];
-        tmem_ld16(lanebase + 192 + r0, ov);
-        tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 16; ++i)
-          if (r0 + i < len) o[((size_t)(tok0 + r0 + i) * H + h) * D + v] = __float2bfloat16_rn(ov[i]);
-      }
-    }
-    // next state
+    // next state (this thread: columns c in [64 ch, 64 ch + 64))
     const bool last = (j + 1 == nc);
     const float *dn = nullptr;
     if (!last) {
@@ -579,7 +562,7 @@ __global__ void __launch_bounds__(kStateThreads, 1) tc_state_kernel(TcArgs ta) {
       if (__syncthreads_or(!ok)) { abort = true; break; }
       dn = reinterpret_cast<const float *>(recbuf[buf ^ 1] + R5);
     }
-    for (int c0 = 0; c0 < D; c0 += 16) {
+    for (int c0 = 64 * ch; c0 < 64 * ch + 64; c0 += 16) {
       float sv[16];
       tmem_ld16(lanebase + c0, sv);
       tmem_wait_ld();
@@ -604,13 +587,26 @@ __global__ void __launch_bounds__(kStateThreads, 1) tc_state_kernel(TcArgs ta) {
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
+    if (tid == 0 && !last) issue_mma3(j + 1);
+    // output rows of this chunk (overlaps the next chunk's MMA3); rows [32 ch, 32 ch + 32)
+    if (ta.write_o) {
+      for (int r0 = 32 * ch; r0 < 32 * ch + 32; r0 += 16) {
+        float ov[16];
+        tmem_ld16(lanebase + acc + 64 + r0, ov);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          if (r0 + i < len) o[((size_t)(tok0 + r0 + i) * H + h) * D + v] = __float2bfloat16_rn(ov[i]);
+      }
+    }
+    tc_fence_before();
   }
   if (abort && tid == 0) {
     mma_commit(&ms.mfin);
     mbar_wait(&ms.mfin, 0, a.status, 209);
   }
   __syncthreads();
-  if (warp == 0) tmem_dealloc(tmem, 256);
+  if (warp == 0) tmem_dealloc(tmem, 512);
 }
 
 int g_num_sms = 0;
