@@ -219,7 +219,19 @@ constexpr uint32_t R4 = 57344;   // Khat^T: K-major tile [c][s] (128 x 64)
 constexpr uint32_t R5 = 73728;   // d[128] fp32
 constexpr uint32_t REC = 74240;  // bytes per (chunk, head) record
 
-__device__ __forceinline__ float fast_exp(float x) { return exp2f(x * kLog2e); }
+// 2^x and 1/x with one MUFU instruction each (PTX ex2.approx / rcp.approx);
+// their relative error (~2^-22) is far below the bf16 operand rounding.
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float fast_exp(float x) { return ex2_approx(x * kLog2e); }
 
 __device__ __forceinline__ void st_bf16(unsigned char *base, uint32_t off, float x) {
   *reinterpret_cast<__nv_bfloat16 *>(base + off) = __float2bfloat16_rn(x);

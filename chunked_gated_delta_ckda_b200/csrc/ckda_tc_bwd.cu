@@ -363,7 +363,7 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(BwdTcArgs ta) {
   float *tmpf = reinterpret_cast<float *>(sm + G_KG);  // [64][64]
   float(*Xs)[16][16] = reinterpret_cast<float(*)[16][16]>(sm + G_XS);
   float *gcps = reinterpret_cast<float *>(sm + G_UV);         // [2][128], final epilogue only
-  float *acc1s = gcps + 256;                                  // [128]
+  float *acc1s = gcps + 256;                                  // [2][128]
   float *fb = ta.fb + (size_t)blockIdx.x * 3 * 64 * D;
 
   const int c = tid & 127, hf = tid >> 7;
@@ -430,37 +430,44 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(BwdTcArgs ta) {
     const bool fast = !__syncthreads_or(bad);
 
     // ---------------- operand tiles ----------------
+    if (fast) {
 #pragma unroll
-    for (int rr = 0; rr < 8; ++rr) {
-      const int r = 8 * warp + rr;
-      float ql[4], kl[4], kr[4], kgv[4];
+      for (int rr = 0; rr < 8; ++rr) {
+        const int r = 8 * warp + rr;
+        float ql[4], kl[4], kr[4];
 #pragma unroll
-      for (int m = 0; m < 4; ++m) {
-        const float p = prep_p(P, rr, m);
-        const float kp = p * prep_k(P, rr, m), qp = p * prep_q(P, rr, m);
-        if (fast) {
-          const float el = fast_exp(P.G[rr][m] - P.Gm[m]), er = __frcp_rn(el);
+        for (int m = 0; m < 4; ++m) {
+          const float p = prep_p(P, rr, m);
+          const float kp = p * prep_k(P, rr, m), qp = p * prep_q(P, rr, m);
+          const float el = fast_exp(P.G[rr][m] - P.Gm[m]), er = rcp_approx(el);
           ql[m] = qp * el;
           kl[m] = kp * el;
           kr[m] = kp * er;
-          kgv[m] = kl[m] * fast_exp(P.Gm[m]);
-        } else {
-          ql[m] = qp;
-          kl[m] = kp;
-          kr[m] = P.G[rr][m];
-          kgv[m] = kp * fast_exp(P.G[rr][m]);
         }
-      }
-      if (fast) {
+        const float e0 = fast_exp(P.Gm[0]), e1 = fast_exp(P.Gm[1]), e2 = fast_exp(P.Gm[2]), e3 = fast_exp(P.Gm[3]);
         st_bf16x4(sm + G_A1, kmaj_off(r, 4 * lane, 128), ql[0], ql[1], ql[2], ql[3]);
         st_bf16x4(sm + G_A1, kmaj_off(64 + r, 4 * lane, 128), kl[0], kl[1], kl[2], kl[3]);
         st_bf16x4(sm + G_B1, kmaj_off(r, 4 * lane, 64), kr[0], kr[1], kr[2], kr[3]);
-      } else {
-        *reinterpret_cast<float4 *>(fb + r * D + 4 * lane) = make_float4(kr[0], kr[1], kr[2], kr[3]);
-        *reinterpret_cast<float4 *>(fb + 64 * D + r * D + 4 * lane) = make_float4(kl[0], kl[1], kl[2], kl[3]);
-        *reinterpret_cast<float4 *>(fb + 128 * D + r * D + 4 * lane) = make_float4(ql[0], ql[1], ql[2], ql[3]);
+        st_bf16x4(sm + G_KG, mnmaj_off(r, 4 * lane, 64), kl[0] * e0, kl[1] * e1, kl[2] * e2, kl[3] * e3);
       }
-      st_bf16x4(sm + G_KG, mnmaj_off(r, 4 * lane, 64), kgv[0], kgv[1], kgv[2], kgv[3]);
+    } else {
+#pragma unroll
+      for (int rr = 0; rr < 8; ++rr) {
+        const int r = 8 * warp + rr;
+        float kp4[4], qp4[4], g4[4], kg4[4];
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          const float p = prep_p(P, rr, m);
+          kp4[m] = p * prep_k(P, rr, m);
+          qp4[m] = p * prep_q(P, rr, m);
+          g4[m] = P.G[rr][m];
+          kg4[m] = kp4[m] * fast_exp(g4[m]);
+        }
+        *reinterpret_cast<float4 *>(fb + r * D + 4 * lane) = make_float4(g4[0], g4[1], g4[2], g4[3]);
+        *reinterpret_cast<float4 *>(fb + 64 * D + r * D + 4 * lane) = make_float4(kp4[0], kp4[1], kp4[2], kp4[3]);
+        *reinterpret_cast<float4 *>(fb + 128 * D + r * D + 4 * lane) = make_float4(qp4[0], qp4[1], qp4[2], qp4[3]);
+        st_bf16x4(sm + G_KG, mnmaj_off(r, 4 * lane, 64), kg4[0], kg4[1], kg4[2], kg4[3]);
+      }
     }
     fence_async_smem();
     __syncthreads();
@@ -717,15 +724,15 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(BwdTcArgs ta) {
     }
     tc_fence_before();
     __syncthreads();
-    // dbeta (column part) and dM = dT Diag(beta)
-    if (tid < 64) {
-      const int j = tid;
+    // dbeta (column part): sum_i dT[i][j] M[i][j], four lanes per column
+    {
+      const int j = tid >> 2, part = tid & 3;
       float s = 0.f;
-      for (int i = j; i < 64; ++i) s += dTf[i * LDF + j] * Mf[i * LDF + j];
-      ms.dbc[j] = s;
+      for (int i = j + part; i < 64; i += 4) s += dTf[i * LDF + j] * Mf[i * LDF + j];
+      s += __shfl_xor_sync(0xffffffffu, s, 1);
+      s += __shfl_xor_sync(0xffffffffu, s, 2);
+      if (part == 0) ms.dbc[j] = s;
     }
-    __syncthreads();
-    for (int e = tid; e < 64 * 64; e += kGThreads) dTf[(e >> 6) * LDF + (e & 63)] *= ms.beta[e & 63];
     __syncthreads();
     // tmp = dM M^T  (tmp[i][kk] = sum_{j <= min(i, kk)} dM[i][j] M[kk][j]), 4 x 4 per thread;
     // dM and M are lower triangular, so the extra j of a tile contribute zeros
@@ -740,8 +747,10 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(BwdTcArgs ta) {
       for (int j = 0; j <= jmax; ++j) {
         float a4[4], b4[4];
 #pragma unroll
+        const float bj = ms.beta[j];  // dM = dT Diag(beta), applied on the fly
+#pragma unroll
         for (int m = 0; m < 4; ++m) {
-          a4[m] = dTf[(i0 + m) * LDF + j];
+          a4[m] = dTf[(i0 + m) * LDF + j] * bj;
           b4[m] = Mf[(k0 + m) * LDF + j];
         }
 #pragma unroll
@@ -933,9 +942,9 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(BwdTcArgs ta) {
       const float pCs = pcb ? -1.f : 1.f;
       const float eGm = fast_exp(Gm), eCm = fast_exp(GC - Gm);
       const float dC = pCs * fast_exp(GC);
-      float dG[32];
+      float *dGs = reinterpret_cast<float *>(sm + G_OU);  // [64][128] dL/dGam, idle tile
       float gcp = 0.f;
-#pragma unroll
+#pragma unroll 1
       for (int b8 = 0; b8 < 4; ++b8) {
         const uint32_t colo = 32 * hf + 8 * b8;
         float X1[8], X2[8], Y1[8], dQG[8], dKG[8], dKh[8], dVv[8];
@@ -950,29 +959,22 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(BwdTcArgs ta) {
         const uint32_t pb = ms.pbits[(32 * hf + 8 * b8) >> 3][c];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          const int ii = 8 * b8 + i;
-          const int r = 32 * hf + ii;
+          const int r = 32 * hf + 8 * b8 + i;
           const float Gr = Gs[r * D + c];
           const uint32_t kqv = KQs[r * D + c];
           const float kp = bf_lo(kqv), qp = bf_hi(kqv);
           const float p = ((pb >> i) & 1u) ? -1.f : 1.f;
-          float el, er, E, eC;
-          if (fast) {
-            el = fast_exp(Gr - Gm);
-            er = __frcp_rn(el);
-            E = el * eGm;
-            eC = er * eCm;
-          } else {
-            el = 1.f;
-            er = 1.f;
-            E = fast_exp(Gr);
-            eC = fast_exp(GC - Gr);
-          }
+          // fast path: the pair terms carry the reference-row scaling; exact
+          // path: they are final, and the factors come straight from Gam
+          const float el = fast ? fast_exp(Gr - Gm) : 1.f;
+          const float er = fast ? rcp_approx(el) : 1.f;
+          const float E = fast ? el * eGm : fast_exp(Gr);
+          const float eC = fast ? er * eCm : fast_exp(GC - Gr);
           const float x1 = el * X1[i], x2 = el * X2[i], y1 = er * Y1[i];
           const float KGv = kp * E, QGv = qp * E, Kh = pCs * kp * eC;
           const float dkp = x1 + y1 + dKG[i] * E + pCs * dKh[i] * eC;
           const float dqp = x2 + dQG[i] * E;
-          dG[ii] = kp * x1 + qp * x2 - kp * y1 + dKG[i] * KGv + dQG[i] * QGv - dKh[i] * Kh;
+          dGs[r * D + c] = kp * x1 + qp * x2 - kp * y1 + dKG[i] * KGv + dQG[i] * QGv - dKh[i] * Kh;
           gcp += dKh[i] * Kh;
           if (r < len) {
             const size_t off = ((size_t)(tok0 + r) * H + h) * D + c;
@@ -982,28 +984,21 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(BwdTcArgs ta) {
           }
         }
       }
+      // reverse in-chunk cumsum of dL/dGam (plus the chunk-end terms) -> dg;
+      // both halves at once: the lower half starts from the upper half's total
+      float part = 0.f;
+#pragma unroll 8
+      for (int ii = 0; ii < 32; ++ii) part += dGs[(32 * hf + ii) * D + c];
       gcps[hf * 128 + c] = gcp;
+      acc1s[hf * 128 + c] = part;
       __syncthreads();
       const float gC = gcps[c] + gcps[128 + c] + (ms.dd[0][c] + ms.dd[1][c]) * dC;
-      // reverse in-chunk cumsum: the upper half first, then the lower half continues
-      if (hf == 1) {
-        float acc = gC;
-#pragma unroll
-        for (int ii = 31; ii >= 0; --ii) {
-          acc += dG[ii];
-          const int r = 32 + ii;
-          if (r < len) a.dg[((size_t)(tok0 + r) * H + h) * D + c] = acc;
-        }
-        acc1s[c] = acc;
-      }
-      __syncthreads();
-      if (hf == 0) {
-        float acc = acc1s[c];
-#pragma unroll
-        for (int ii = 31; ii >= 0; --ii) {
-          acc += dG[ii];
-          if (ii < len) a.dg[((size_t)(tok0 + ii) * H + h) * D + c] = acc;
-        }
+      float acc = gC + (hf == 0 ? acc1s[128 + c] : 0.f);
+#pragma unroll 8
+      for (int ii = 31; ii >= 0; --ii) {
+        const int r = 32 * hf + ii;
+        acc += dGs[r * D + c];
+        if (r < len) a.dg[((size_t)(tok0 + r) * H + h) * D + c] = acc;
       }
       if (tid < 64 && tid < len)
         dbeta[(size_t)(tok0 + tid) * H + h] =

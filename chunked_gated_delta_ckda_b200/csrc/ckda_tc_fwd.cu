@@ -157,43 +157,51 @@ __global__ void __launch_bounds__(kIntraThreads, 2) tc_intra_kernel(TcArgs ta) {
     // ---------------- operand tiles and record tiles ----------------
     {
       float qg[8][4], kh[8][4];
+      if (fast) {
 #pragma unroll
-      for (int rr = 0; rr < 8; ++rr) {
-        const int r = 8 * warp + rr;
-        float ql[4], kl[4], kr[4], kgv[4];
+        for (int rr = 0; rr < 8; ++rr) {
+          const int r = 8 * warp + rr;
+          float ql[4], kl[4], kr[4];
 #pragma unroll
-        for (int m = 0; m < 4; ++m) {
-          const float p = prep_p(P, rr, m);
-          const float kp = p * prep_k(P, rr, m), qp = p * prep_q(P, rr, m);
-          if (fast) {
+          for (int m = 0; m < 4; ++m) {
+            const float p = prep_p(P, rr, m);
+            const float kp = p * prep_k(P, rr, m), qp = p * prep_q(P, rr, m);
             const float el = fast_exp(P.G[rr][m] - P.Gm[m]);
-            const float er = __frcp_rn(el);
+            const float er = rcp_approx(el);
             ql[m] = qp * el;
             kl[m] = kp * el;
             kr[m] = kp * er;
-            kgv[m] = kl[m] * eGm[m];
             qg[rr][m] = ql[m] * eGm[m];
             kh[rr][m] = pCs[m] * kr[m] * eCm[m];
-          } else {
-            const float E = fast_exp(P.G[rr][m]);
-            kgv[m] = kp * E;
-            qg[rr][m] = qp * E;
-            kh[rr][m] = pCs[m] * kp * fast_exp(P.GC[m] - P.G[rr][m]);
-            ql[m] = qp;  // kept for the exact pair sums below
-            kl[m] = kp;
-            kr[m] = P.G[rr][m];
           }
-        }
-        if (fast) {
           st_bf16x4(sm + I_A1, kmaj_off(r, 4 * lane, 128), ql[0], ql[1], ql[2], ql[3]);
           st_bf16x4(sm + I_A1, kmaj_off(64 + r, 4 * lane, 128), kl[0], kl[1], kl[2], kl[3]);
           st_bf16x4(sm + I_B1, kmaj_off(r, 4 * lane, 64), kr[0], kr[1], kr[2], kr[3]);
-        } else {
-          *reinterpret_cast<float4 *>(fb + r * D + 4 * lane) = make_float4(kr[0], kr[1], kr[2], kr[3]);
-          *reinterpret_cast<float4 *>(fb + 64 * D + r * D + 4 * lane) = make_float4(kl[0], kl[1], kl[2], kl[3]);
-          *reinterpret_cast<float4 *>(fb + 128 * D + r * D + 4 * lane) = make_float4(ql[0], ql[1], ql[2], ql[3]);
+          st_bf16x4(sm + I_KG, mnmaj_off(r, 4 * lane, 64), kl[0] * eGm[0], kl[1] * eGm[1], kl[2] * eGm[2],
+                    kl[3] * eGm[3]);
         }
-        st_bf16x4(sm + I_KG, mnmaj_off(r, 4 * lane, 64), kgv[0], kgv[1], kgv[2], kgv[3]);
+      } else {
+        // exact path: keep Gam, k', q' for the per-pair sums; KG, QG, Khat directly
+#pragma unroll
+        for (int rr = 0; rr < 8; ++rr) {
+          const int r = 8 * warp + rr;
+          float kp4[4], qp4[4], g4[4], kg4[4];
+#pragma unroll
+          for (int m = 0; m < 4; ++m) {
+            const float p = prep_p(P, rr, m);
+            kp4[m] = p * prep_k(P, rr, m);
+            qp4[m] = p * prep_q(P, rr, m);
+            g4[m] = P.G[rr][m];
+            const float E = fast_exp(g4[m]);
+            kg4[m] = kp4[m] * E;
+            qg[rr][m] = qp4[m] * E;
+            kh[rr][m] = pCs[m] * kp4[m] * fast_exp(P.GC[m] - g4[m]);
+          }
+          *reinterpret_cast<float4 *>(fb + r * D + 4 * lane) = make_float4(g4[0], g4[1], g4[2], g4[3]);
+          *reinterpret_cast<float4 *>(fb + 64 * D + r * D + 4 * lane) = make_float4(kp4[0], kp4[1], kp4[2], kp4[3]);
+          *reinterpret_cast<float4 *>(fb + 128 * D + r * D + 4 * lane) = make_float4(qp4[0], qp4[1], qp4[2], qp4[3]);
+          st_bf16x4(sm + I_KG, mnmaj_off(r, 4 * lane, 64), kg4[0], kg4[1], kg4[2], kg4[3]);
+        }
       }
       // QG^T (N index 64 + r) and Khat^T (K index r) of each channel: one 16-byte chunk
 #pragma unroll
