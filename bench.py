@@ -267,6 +267,105 @@ def run_ours(args, rank, world, local_rank):
     return out, inp
 
 
+def run_secondary(args, rank, world, local_rank):
+    """Secondary workloads (not the headline line): forward only, packed
+    variable-length forward, recurrent decode."""
+    from chunked_gated_delta_ckda_b200 import _abi, api
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    peaks = measured_peaks()
+    clocks = ClockSampler(local_rank)
+    if args.workload == "decode":
+        w = W.DECODE
+        N, H, dk, dv = w.B, w.H, w.dk, w.dv
+        state = W.make_decode_state(w).to(dev)
+        pool = [{k: v.to(dev) for k, v in W.make_decode_step(w, t).items()} for t in range(16)]
+        o = torch.empty(N, H, dv, dtype=w.io_dtype, device=dev)
+        code = api.io_code(w.io_dtype)
+        it = [0]
+
+        def step():
+            x = pool[it[0] % len(pool)]
+            it[0] += 1
+            _abi.ckda_decode_step(N, H, dk, dv, code, x["q"], x["k"], x["v"], x["g"], x["sign"],
+                                  x["beta"], state, o)
+        units, per_unit, unit_name = N * H, DECODE_BYTES_PER_NH, "B per (sequence, head) step"
+        tokens = N
+        metric = "CKDA decode tokens/s (N=256,H=16,d=128,bf16 I/O,fp32 state)"
+        cfg = {"workload": w.name, "N": N, "H": H, "dk": dk, "dv": dv, "io_dtype": "bf16",
+               "state_dtype": "f32", "l2": "state (512 MiB) larger than L2"}
+    elif args.workload == "varlen":
+        w = W.VARLEN
+        inp = W.make_varlen(w)
+        d = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+        T, H, dk, dv = inp["q"].shape[1], w.H, w.dk, w.dv
+        Nd = len(inp["lens"])
+        o = torch.empty(1, T, H, dv, dtype=w.io_dtype, device=dev)
+        ST = torch.empty(Nd, H, dk, dv, dtype=torch.float32, device=dev)
+        ws = api.workspace(_abi.CKDA_OP_VARLEN_FWD, 1, T, H, dk, dv, Nd, device=dev, cache=False)
+        cu = d["cu_seqlens"]
+        mx = max(inp["lens"])
+        code = api.io_code(w.io_dtype)
+
+        def step():
+            _abi.ckda_varlen_fwd(T, Nd, cu, mx, H, dk, dv, code, d["q"], d["k"], d["v"], d["g"],
+                                 d["sign"], d["beta"], None, o, ST, ws)
+        units, per_unit, unit_name = T * H, FWD_BYTES, "B per token-head (fwd)"
+        tokens = T
+        metric = "CKDA varlen fwd tokens/s (65536 packed tokens,H=16,d=128,bf16)"
+        cfg = {"workload": w.name, "total_T": T, "docs": Nd, "H": H, "dk": dk, "dv": dv,
+               "io_dtype": "bf16", "l2": "inputs larger than L2"}
+    else:  # fwd
+        w = W.LAYER_FWD
+        inp = W.make(w)
+        d = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+        B, T, H, dk, dv = w.B, w.T, w.H, w.dk, w.dv
+        o = torch.empty(B, T, H, dv, dtype=w.io_dtype, device=dev)
+        ST = torch.empty(B, H, dk, dv, dtype=torch.float32, device=dev)
+        ws = api.workspace(_abi.CKDA_OP_CHUNK_FWD, B, T, H, dk, dv, device=dev, cache=False)
+        code = api.io_code(w.io_dtype)
+
+        def step():
+            _abi.ckda_chunk_fwd(B, T, H, dk, dv, code, d["q"], d["k"], d["v"], d["g"], d["sign"],
+                                d["beta"], None, o, ST, None, ws)
+        units, per_unit, unit_name = B * T * H, FWD_BYTES, "B per token-head (fwd)"
+        tokens = B * T
+        metric = "CKDA fwd tokens/s (H=16,d=128,T=4096,bf16)"
+        cfg = {"workload": w.name, "B": B, "T": T, "H": H, "dk": dk, "dv": dv, "io_dtype": "bf16",
+               "l2": "inputs larger than L2"}
+    clocks.start()
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    _abi.ckda_profile_reset()
+    _abi.ckda_profile_enable(True)
+    ms = _time_steps(step, args.steps, 0, world)
+    _abi.ckda_profile_enable(False)
+    prof = _abi.ckda_profile_collect()
+    clk = clocks.stop()
+    ms = reduce_max(ms, world)
+    total = sum(t for _, t in prof.values())
+    kernels = {k: {"launches": n, "ms_per_launch": t / n, "share": t / total if total else None}
+               for k, (n, t) in sorted(prof.items(), key=lambda kv: -kv[1][1])}
+    top = max(prof.items(), key=lambda kv: kv[1][1])[0]
+    n, t = prof[top]
+    launches_per_step = n / args.steps
+    alg = per_unit * units / launches_per_step if launches_per_step >= 1 else per_unit * units
+    achieved = alg / (t / n / 1e3) / 1e9
+    step_bytes = per_unit * units
+    out = {"metric": metric, "value": tokens * world / (ms / 1e3), "unit": "tokens/s",
+           "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+           "data": "synthetic", "config": cfg,
+           "roofline": {"bound": "hbm", "kernel": top, "achieved": achieved, "peak": peaks["hbm_gbs"],
+                        "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                        "algorithmic_bytes_per_launch": alg, "per_unit": "%d %s" % (per_unit, unit_name),
+                        "peak_source": peaks["source"]},
+           "step_hbm_frac": step_bytes / (peaks["hbm_gbs"] * 1e9) / (ms / 1e3),
+           "kernels": kernels, "gpu_launches": int(sum(n for n, _ in prof.values())), "clocks": clk}
+    return out
+
+
 def run_e2e(inp, dev, args, world):
     """Same step through the public API from pinned HOST buffers: H2D of the
     inputs and D2H of every output inside the timed region."""
@@ -381,6 +480,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer pass")
+    ap.add_argument("--workload", choices=["fwdbwd", "fwd", "varlen", "decode"], default="fwdbwd",
+                    help="fwdbwd is the headline; the others are secondary measurements")
     ap.add_argument("--batch", type=int, default=0,
                     help="override B (profiling a smaller case; not a bench line)")
     args = ap.parse_args(argv)
@@ -404,6 +505,11 @@ def main(argv=None):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
     try:
+        if args.workload != "fwdbwd":
+            out = run_secondary(args, rank, world, local_rank)
+            if rank == 0:
+                print(json.dumps(out), flush=True)
+            return 0
         out, inp = run_ours(args, rank, world, local_rank)
         if rank == 0:
             if world == 1 and not args.no_cpu_baseline:

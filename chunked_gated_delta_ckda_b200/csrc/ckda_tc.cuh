@@ -395,5 +395,65 @@ __device__ __forceinline__ void st_bf16x4(unsigned char *base, uint32_t off, flo
   *reinterpret_cast<uint2 *>(base + off) = make_uint2(pack_bf16(a, b), pack_bf16(c, d));
 }
 
+// ---------------------------------------------------------------------------
+// M = (I + N)^{-1} for strictly lower N (fp32, row stride LDF), 64 x 64, by
+// 16 x 16 blocks, 256 threads: diagonal blocks by forward substitution (one
+// column per thread), then the block diagonals d = 1, 2, 3:
+//   M_IJ = -M_II sum_{K=J}^{I-1} N_IK M_KJ.
+// Every entry on or below the diagonal is written; the strictly upper 16x16
+// blocks are zeroed (the diagonal blocks carry their own zeros).
+// ---------------------------------------------------------------------------
+constexpr int kLdf = 65;
+__device__ __forceinline__ void inverse64(float *Mf, const float *Nf, float (*Xs)[16][16]) {
+  const int tid = threadIdx.x;
+  if (tid < 64) {
+    const int bI = tid >> 4, j = tid & 15, o = 16 * bI;
+    float xc[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      float s = 0.f;
+#pragma unroll
+      for (int kk = 0; kk < i; ++kk) s += Nf[(o + i) * kLdf + o + kk] * xc[kk];
+      xc[i] = (i == j) ? 1.f : (i < j ? 0.f : -s);
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) Mf[(o + i) * kLdf + o + j] = xc[i];
+  } else {
+    // strictly upper blocks (I < J): 6 blocks of 256
+    for (int e = tid - 64; e < 6 * 256; e += 192) {
+      const int b = e >> 8, aa = (e >> 4) & 15, bb = e & 15;
+      const int I = b < 3 ? 0 : (b < 5 ? 1 : 2);
+      const int J = b < 3 ? b + 1 : (b < 5 ? b - 1 : 3);
+      Mf[(16 * I + aa) * kLdf + 16 * J + bb] = 0.f;
+    }
+  }
+  __syncthreads();
+#pragma unroll 1
+  for (int d = 1; d < 4; ++d) {
+    const int nb = 4 - d;
+    for (int e = tid; e < nb * 256; e += 256) {
+      const int J = e >> 8, I = J + d, aa = (e >> 4) & 15, bb = e & 15;
+      float s = 0.f;
+      for (int K = J; K < I; ++K) {
+        const float *nrow = Nf + (16 * I + aa) * kLdf + 16 * K;
+        const float *mcol = Mf + (16 * K) * kLdf + 16 * J + bb;
+#pragma unroll
+        for (int t = 0; t < 16; ++t) s += nrow[t] * mcol[t * kLdf];
+      }
+      Xs[J][aa][bb] = s;
+    }
+    __syncthreads();
+    for (int e = tid; e < nb * 256; e += 256) {
+      const int J = e >> 8, I = J + d, aa = (e >> 4) & 15, bb = e & 15;
+      const float *mrow = Mf + (16 * I + aa) * kLdf + 16 * I;
+      float s = 0.f;
+#pragma unroll
+      for (int t = 0; t < 16; ++t) s += mrow[t] * Xs[J][t][bb];
+      Mf[(16 * I + aa) * kLdf + 16 * J + bb] = -s;
+    }
+    __syncthreads();
+  }
+}
+
 }  // namespace tc
 }  // namespace ckda

@@ -389,35 +389,33 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(BwdTcArgs ta) {
       bulk_g2s(sm + G_OU + 8192, gdU, 8192, &ms.mdu);
       bulk_g2s(sm + G_OU + 16384 + 8192, gdU + 8192, 8192, &ms.mdu);
     }
+    // every load of the item is in flight before any of them is used:
+    // V and dO rows, the start state S_c (fp32), then the prep rows
+    uint4 vv[4], oo[4];
+    float4 x[16];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const int e = tid + kGThreads * m, j = e >> 4, cc = e & 15;
+      const int jj = j < len ? j : len - 1;
+      const size_t off = ((size_t)(tok0 + jj) * H + h) * D + cc * 8;
+      vv[m] = *reinterpret_cast<const uint4 *>(v + off);
+      oo[m] = *reinterpret_cast<const uint4 *>(dO + off);
+    }
+#pragma unroll
+    for (int m = 0; m < 16; ++m) x[m] = *reinterpret_cast<const float4 *>(Sc + (size_t)(warp + 8 * m) * D + 4 * lane);
     Prep P;  // row-group layout: rows 8 warp .., channels 4 lane ..
     prep_load(a.g, a.sign, k, q, tok0, len, h, H, warp, lane, P, ms.tot);
-    {  // V and dO rows (all loads in flight before the stores)
-      uint4 vv[4], oo[4];
 #pragma unroll
-      for (int m = 0; m < 4; ++m) {
-        const int e = tid + kGThreads * m, j = e >> 4, cc = e & 15;
-        const int jj = j < len ? j : len - 1;
-        const size_t off = ((size_t)(tok0 + jj) * H + h) * D + cc * 8;
-        vv[m] = *reinterpret_cast<const uint4 *>(v + off);
-        oo[m] = *reinterpret_cast<const uint4 *>(dO + off);
-      }
-#pragma unroll
-      for (int m = 0; m < 4; ++m) {
-        const int e = tid + kGThreads * m, j = e >> 4, cc = e & 15;
-        if (j >= len) vv[m] = oo[m] = make_uint4(0, 0, 0, 0);
-        *reinterpret_cast<uint4 *>(sm + G_UV + kmaj_off(64 + j, cc * 8, 128)) = vv[m];
-        *reinterpret_cast<uint4 *>(sm + G_OU + kmaj_off(j, cc * 8, 128)) = oo[m];
-      }
+    for (int m = 0; m < 4; ++m) {
+      const int e = tid + kGThreads * m, j = e >> 4, cc = e & 15;
+      if (j >= len) vv[m] = oo[m] = make_uint4(0, 0, 0, 0);
+      *reinterpret_cast<uint4 *>(sm + G_UV + kmaj_off(64 + j, cc * 8, 128)) = vv[m];
+      *reinterpret_cast<uint4 *>(sm + G_OU + kmaj_off(j, cc * 8, 128)) = oo[m];
     }
-    {  // S_c fp32 rows -> bf16 K-major [c][v]; 16 rows per warp, all loads in flight
-      float4 x[16];
 #pragma unroll
-      for (int m = 0; m < 16; ++m) x[m] = *reinterpret_cast<const float4 *>(Sc + (size_t)(warp + 8 * m) * D + 4 * lane);
-#pragma unroll
-      for (int m = 0; m < 16; ++m)
-        *reinterpret_cast<uint2 *>(sm + G_SC + kmaj_off(warp + 8 * m, 4 * lane, 128)) =
-            make_uint2(pack_bf16(x[m].x, x[m].y), pack_bf16(x[m].z, x[m].w));
-    }
+    for (int m = 0; m < 16; ++m)  // S_c fp32 rows -> bf16 K-major [c][v]
+      *reinterpret_cast<uint2 *>(sm + G_SC + kmaj_off(warp + 8 * m, 4 * lane, 128)) =
+          make_uint2(pack_bf16(x[m].x, x[m].y), pack_bf16(x[m].z, x[m].w));
     if (tid < 64) ms.beta[tid] = tid < len ? __bfloat162float(beta[(size_t)(tok0 + tid) * H + h]) : 0.f;
     __syncthreads();
     prep_carry(warp, lane, P, ms.tot);
@@ -512,40 +510,7 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(BwdTcArgs ta) {
     __syncthreads();
 
     // ---------------- M = (I + N)^{-1} ----------------
-    for (int e = tid; e < 64 * 64; e += kGThreads) Mf[(e >> 6) * LDF + (e & 63)] = 0.f;
-    __syncthreads();
-    if (tid < 64) {
-      const int bI = tid >> 4, j = tid & 15, o = 16 * bI;
-      float xc[16];
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        float s = 0.f;
-#pragma unroll
-        for (int kk = 0; kk < i; ++kk) s += Nf[(o + i) * LDF + o + kk] * xc[kk];
-        xc[i] = (i == j) ? 1.f : (i < j ? 0.f : -s);
-      }
-#pragma unroll
-      for (int i = 0; i < 16; ++i) Mf[(o + i) * LDF + o + j] = xc[i];
-    }
-    __syncthreads();
-    for (int d = 1; d < 4; ++d) {
-      const int nb = 4 - d;
-      for (int e = tid; e < nb * 256; e += kGThreads) {
-        const int J = e >> 8, I = J + d, aa = (e >> 4) & 15, bb = e & 15;
-        float s = 0.f;
-        for (int u = 16 * J; u < 16 * I; ++u) s += Nf[(16 * I + aa) * LDF + u] * Mf[u * LDF + 16 * J + bb];
-        Xs[J][aa][bb] = s;
-      }
-      __syncthreads();
-      for (int e = tid; e < nb * 256; e += kGThreads) {
-        const int J = e >> 8, I = J + d, aa = (e >> 4) & 15, bb = e & 15;
-        float s = 0.f;
-#pragma unroll
-        for (int t = 0; t < 16; ++t) s += Mf[(16 * I + aa) * LDF + 16 * I + t] * Xs[J][t][bb];
-        Mf[(16 * I + aa) * LDF + 16 * J + bb] = -s;
-      }
-      __syncthreads();
-    }
+    inverse64(Mf, Nf, Xs);
     {
       const int r = tid >> 2, j0 = (tid & 3) * 16;
       uint32_t pk[8];

@@ -114,17 +114,18 @@ __global__ void __launch_bounds__(kIntraThreads, 2) tc_intra_kernel(TcArgs ta) {
     unsigned char *rec = ta.recs + (size_t)item * REC;
 
     // ---------------- prep: row-group layout (rows 8w.., channels 4l..) ----------------
+    // V rows are requested first so their latency overlaps the prep loads
+    uint4 vv[4];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const int e = tid + kIntraThreads * m, j = e >> 4, cc = e & 15;
+      const int jj = j < len ? j : len - 1;
+      vv[m] = *reinterpret_cast<const uint4 *>(v + ((size_t)(tok0 + jj) * H + h) * D + cc * 8);
+    }
     Prep P;
     prep_load(a.g, a.sign, k, q, tok0, len, h, H, warp, lane, P, ms.tot);
     // V tile (MN-major A operand, K = token j, M = value channel)
     {
-      uint4 vv[4];
-#pragma unroll
-      for (int m = 0; m < 4; ++m) {
-        const int e = tid + kIntraThreads * m, j = e >> 4, cc = e & 15;
-        const int jj = j < len ? j : len - 1;
-        vv[m] = *reinterpret_cast<const uint4 *>(v + ((size_t)(tok0 + jj) * H + h) * D + cc * 8);
-      }
 #pragma unroll
       for (int m = 0; m < 4; ++m) {
         const int e = tid + kIntraThreads * m, j = e >> 4, cc = e & 15;
@@ -287,40 +288,7 @@ __global__ void __launch_bounds__(kIntraThreads, 2) tc_intra_kernel(TcArgs ta) {
     __syncthreads();
 
     // ---------------- M = (I + N)^{-1}, 16 x 16 blocks ----------------
-    for (int e = tid; e < 64 * 64; e += kIntraThreads) Mf[(e >> 6) * LDF + (e & 63)] = 0.f;
-    __syncthreads();
-    if (tid < 64) {
-      const int bI = tid >> 4, j = tid & 15, o = 16 * bI;
-      float xc[16];
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        float s = 0.f;
-#pragma unroll
-        for (int kk = 0; kk < i; ++kk) s += Nf[(o + i) * LDF + o + kk] * xc[kk];
-        xc[i] = (i == j) ? 1.f : (i < j ? 0.f : -s);
-      }
-#pragma unroll
-      for (int i = 0; i < 16; ++i) Mf[(o + i) * LDF + o + j] = xc[i];
-    }
-    __syncthreads();
-    for (int d = 1; d < 4; ++d) {
-      const int nb = 4 - d;
-      for (int e = tid; e < nb * 256; e += kIntraThreads) {
-        const int J = e >> 8, I = J + d, aa = (e >> 4) & 15, bb = e & 15;
-        float s = 0.f;
-        for (int u = 16 * J; u < 16 * I; ++u) s += Nf[(16 * I + aa) * LDF + u] * Mf[u * LDF + 16 * J + bb];
-        ms.X[J][aa][bb] = s;
-      }
-      __syncthreads();
-      for (int e = tid; e < nb * 256; e += kIntraThreads) {
-        const int J = e >> 8, I = J + d, aa = (e >> 4) & 15, bb = e & 15;
-        float s = 0.f;
-#pragma unroll
-        for (int t = 0; t < 16; ++t) s += Mf[(16 * I + aa) * LDF + 16 * I + t] * ms.X[J][t][bb];
-        Mf[(16 * I + aa) * LDF + 16 * J + bb] = -s;
-      }
-      __syncthreads();
-    }
+    inverse64(Mf, Nf, reinterpret_cast<float(*)[16][16]>(&ms.X[0][0][0]));
     // T = M Diag(beta) -> bf16 K-major B tile [r][j]
     {
       const int r = tid >> 2, j0 = (tid & 3) * 16;
