@@ -5,8 +5,9 @@
                     [--workload fwdbwd|fwd|varlen|decode]
 
 Default workload (the headline): one step = ckda_chunk_fwd (saving chunk
-states) + ckda_chunk_bwd on B=8, H=16, T=4096, dk=dv=128, bf16 I/O, fp32
-gate and state -- the shape of one 1.3B-model token-mixer layer.  Inputs are
+states and its per-chunk results) + ckda_chunk_bwd on B=8, H=16, T=4096,
+dk=dv=128, bf16 I/O, fp32 gate and state -- the shape of one 1.3B-model
+token-mixer layer.  Inputs are
 seeded synthetic tensors (chunked_gated_delta_ckda_b200.workloads), resident
 in HBM when the timed region starts; each step streams ~2 GB, more than L2.
 
@@ -47,6 +48,10 @@ DECODE_BYTES_PER_NH = 131072 + 1666  # state read + write, per-token inputs and 
 
 # Which per-unit figure a kernel's roofline uses (the call it implements).
 KERNEL_UNITS = {
+    "tc_grad": ("bwd", BWD_BYTES, BWD_FLOP),
+    "tc_state_bwd": ("bwd", BWD_BYTES, BWD_FLOP),
+    "tc_intra": ("fwd", FWD_BYTES, FWD_FLOP),
+    "tc_state_fwd": ("fwd", FWD_BYTES, FWD_FLOP),
     "v1_grad": ("bwd", BWD_BYTES, BWD_FLOP),
     "v1_state_bwd": ("bwd", BWD_BYTES, BWD_FLOP),
     "v1_intra": ("fwd", FWD_BYTES, FWD_FLOP),
@@ -170,13 +175,15 @@ def _fwdbwd_setup(inp, dev):
     wsf = api.workspace(_abi.CKDA_OP_CHUNK_FWD, B, T, H, dk, dv, device=dev, cache=False)
     wsb = api.workspace(_abi.CKDA_OP_CHUNK_BWD, B, T, H, dk, dv, device=dev, cache=False)
     code = api.io_code(io)
+    # the forward hands its per-chunk results to the backward (training use)
+    sv = api.saved_buffer(B, T, H, dk, dv, io, dev)
 
     def step():
         _abi.ckda_chunk_fwd(B, T, H, dk, dv, code, d["q"], d["k"], d["v"], d["g"], d["sign"],
-                            d["beta"], None, buf["o"], buf["ST"], buf["cs"], wsf)
+                            d["beta"], None, buf["o"], buf["ST"], buf["cs"], wsf, saved=sv)
         _abi.ckda_chunk_bwd(B, T, H, dk, dv, code, d["q"], d["k"], d["v"], d["g"], d["sign"],
                             d["beta"], None, d["dO"], None, buf["cs"], buf["dq"], buf["dk"],
-                            buf["dv"], buf["dg"], buf["dbeta"], buf["dS0"], wsb)
+                            buf["dv"], buf["dg"], buf["dbeta"], buf["dS0"], wsb, saved=sv)
     return d, buf, step
 
 
@@ -256,10 +263,11 @@ def run_ours(args, rank, world, local_rank):
     out = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-           "dtype": "f32", "data": "synthetic",
+           "dtype": "bf16", "data": "synthetic",
            "config": {"workload": w.name, "B": B, "T": T, "H": H, "dk": w.dk, "dv": w.dv,
                       "io_dtype": "bf16", "gate_dtype": "f32", "state_dtype": "f32",
-                      "step": "ckda_chunk_fwd(save chunk states) + ckda_chunk_bwd",
+                      "contraction": "bf16 tensor-core operands, f32 accumulate",
+                      "step": "ckda_chunk_fwd(save chunk states and per-chunk results) + ckda_chunk_bwd",
                       "global_batch": B * world, "seq_len": T, "parallelism": "dp%d" % world,
                       "l2": "inputs larger than L2 (about 2 GB streamed per step)"},
            "roofline": roof, "step_roofline": step_roof, "kernels": kernels,
@@ -380,6 +388,7 @@ def run_e2e(inp, dev, args, world):
     wsf = api.workspace(_abi.CKDA_OP_CHUNK_FWD, B, T, H, dk, dv, device=dev, cache=False)
     wsb = api.workspace(_abi.CKDA_OP_CHUNK_BWD, B, T, H, dk, dv, device=dev, cache=False)
     code = api.io_code(inp["q"].dtype)
+    sv = api.saved_buffer(B, T, H, dk, dv, inp["q"].dtype, dev)
     h2d = sum(v.numel() * v.element_size() for v in host_in.values())
     d2h = sum(v.numel() * v.element_size() for v in host_out.values())
 
@@ -388,10 +397,10 @@ def run_e2e(inp, dev, args, world):
             dev_in[k].copy_(v, non_blocking=True)
         x = dev_in
         _abi.ckda_chunk_fwd(B, T, H, dk, dv, code, x["q"], x["k"], x["v"], x["g"], x["sign"],
-                            x["beta"], None, buf["o"], buf["ST"], buf["cs"], wsf)
+                            x["beta"], None, buf["o"], buf["ST"], buf["cs"], wsf, saved=sv)
         _abi.ckda_chunk_bwd(B, T, H, dk, dv, code, x["q"], x["k"], x["v"], x["g"], x["sign"],
                             x["beta"], None, x["dO"], None, buf["cs"], buf["dq"], buf["dk"],
-                            buf["dv"], buf["dg"], buf["dbeta"], buf["dS0"], wsb)
+                            buf["dv"], buf["dg"], buf["dbeta"], buf["dS0"], wsb, saved=sv)
         for k, v in host_out.items():
             v.copy_(buf[k], non_blocking=True)
 

@@ -47,8 +47,10 @@ def _load():
         P, I, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
         lib.ckda_workspace_size.argtypes = [I] * 7
         lib.ckda_workspace_size.restype = Z
-        lib.ckda_chunk_fwd.argtypes = [I] * 6 + [P] * 11 + [Z, P]
-        lib.ckda_chunk_bwd.argtypes = [I] * 6 + [P] * 17 + [Z, P]
+        lib.ckda_saved_size.argtypes = [I] * 6
+        lib.ckda_saved_size.restype = Z
+        lib.ckda_chunk_fwd.argtypes = [I] * 6 + [P] * 11 + [Z, P, Z, P]
+        lib.ckda_chunk_bwd.argtypes = [I] * 6 + [P] * 11 + [Z] + [P] * 7 + [Z, P]
         lib.ckda_decode_step.argtypes = [I] * 5 + [P] * 9
         lib.ckda_varlen_fwd.argtypes = [I, I, P, I, I, I, I, I] + [P] * 10 + [Z, P]
         lib.ckda_chunk_fwd_noalloc.argtypes = [I] * 6 + [P] * 11
@@ -113,17 +115,24 @@ def ckda_workspace_size(op, B, T, H, dk, dv, N=0) -> int:
     return int(_load().ckda_workspace_size(op, B, T, H, dk, dv, N))
 
 
+def ckda_saved_size(B, T, H, dk, dv, io_dtype) -> int:
+    return int(_load().ckda_saved_size(B, T, H, dk, dv, io_dtype))
+
+
 def ckda_chunk_fwd(B, T, H, dk, dv, io_dtype, q, k, v, g, sign, beta, S0, o, ST, chunk_states,
-                   ws, ws_bytes=None, stream=None):
+                   ws, ws_bytes=None, stream=None, saved=None, saved_bytes=None):
     _check(_load().ckda_chunk_fwd(B, T, H, dk, dv, io_dtype, _p(q), _p(k), _p(v), _p(g),
                                   _p(sign), _p(beta), _p(S0), _p(o), _p(ST), _p(chunk_states),
+                                  _p(saved), _nbytes(saved, saved_bytes),
                                   _p(ws), _nbytes(ws, ws_bytes), _s(stream)), "ckda_chunk_fwd")
 
 
 def ckda_chunk_bwd(B, T, H, dk, dv, io_dtype, q, k, v, g, sign, beta, S0, dO, dST, chunk_states,
-                   dq, dk_out, dv_out, dg, dbeta, dS0, ws, ws_bytes=None, stream=None):
+                   dq, dk_out, dv_out, dg, dbeta, dS0, ws, ws_bytes=None, stream=None, saved=None,
+                   saved_bytes=None):
     _check(_load().ckda_chunk_bwd(B, T, H, dk, dv, io_dtype, _p(q), _p(k), _p(v), _p(g),
                                   _p(sign), _p(beta), _p(S0), _p(dO), _p(dST), _p(chunk_states),
+                                  _p(saved), _nbytes(saved, saved_bytes),
                                   _p(dq), _p(dk_out), _p(dv_out), _p(dg), _p(dbeta), _p(dS0),
                                   _p(ws), _nbytes(ws, ws_bytes), _s(stream)), "ckda_chunk_bwd")
 

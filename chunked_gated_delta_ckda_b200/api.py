@@ -3,6 +3,8 @@ torch (device memory is torch's job here) and call the library.
 
     o, ST, cs = chunk_fwd(q, k, v, g, sign, beta, S0=None, save_chunk_states=True)
     grads     = chunk_bwd(q, k, v, g, sign, beta, dO, S0=None, dST=None, chunk_states=cs)
+    o, ST, cs, sv = chunk_fwd(..., save_chunk_states=True, save_for_backward=True)
+    grads     = chunk_bwd(..., chunk_states=cs, saved=sv)   # no recomputation
     o         = decode_step(q, k, v, g, sign, beta, state)     # state updated in place
     o, ST     = varlen_fwd(q, k, v, g, sign, beta, cu_seqlens, max_seqlen, S0=None)
 
@@ -54,8 +56,14 @@ def _c(x: Optional[torch.Tensor]) -> Optional[torch.Tensor]:
     return x if x.is_contiguous() else x.contiguous()
 
 
+def saved_buffer(B, T, H, dk, dv, dtype, device) -> Optional[torch.Tensor]:
+    """The forward-to-backward saved buffer (None: this configuration recomputes)."""
+    n = _abi.ckda_saved_size(B, T, H, dk, dv, io_code(dtype))
+    return torch.empty(n, dtype=torch.uint8, device=device) if n > 0 else None
+
+
 def chunk_fwd(q, k, v, g, sign, beta, S0=None, output_final_state=True, save_chunk_states=False,
-              ws=None):
+              ws=None, save_for_backward=False):
     q, k, v, g, sign, beta, S0 = map(_c, (q, k, v, g, sign, beta, S0))
     B, T, H, dk = q.shape
     dv = v.shape[-1]
@@ -67,12 +75,15 @@ def chunk_fwd(q, k, v, g, sign, beta, S0=None, output_final_state=True, save_chu
           if save_chunk_states else None)
     if ws is None:
         ws = workspace(CKDA_OP_CHUNK_FWD, B, T, H, dk, dv, device=q.device)
-    _abi.ckda_chunk_fwd(B, T, H, dk, dv, io, q, k, v, g, sign, beta, S0, o, ST, cs, ws)
+    sv = saved_buffer(B, T, H, dk, dv, q.dtype, q.device) if save_for_backward else None
+    _abi.ckda_chunk_fwd(B, T, H, dk, dv, io, q, k, v, g, sign, beta, S0, o, ST, cs, ws, saved=sv)
+    if save_for_backward:
+        return o, ST, cs, sv
     return o, ST, cs
 
 
 def chunk_bwd(q, k, v, g, sign, beta, dO, S0=None, dST=None, chunk_states=None, need_dS0=True,
-              ws=None):
+              ws=None, saved=None):
     q, k, v, g, sign, beta, dO, S0, dST, chunk_states = map(
         _c, (q, k, v, g, sign, beta, dO, S0, dST, chunk_states))
     B, T, H, dk = q.shape
@@ -87,7 +98,7 @@ def chunk_bwd(q, k, v, g, sign, beta, dO, S0=None, dST=None, chunk_states=None, 
     if ws is None:
         ws = workspace(CKDA_OP_CHUNK_BWD, B, T, H, dk, dv, device=q.device)
     _abi.ckda_chunk_bwd(B, T, H, dk, dv, io, q, k, v, g, sign, beta, S0, dO, dST, chunk_states,
-                        dq, dk_, dv_, dg, dbeta, dS0, ws)
+                        dq, dk_, dv_, dg, dbeta, dS0, ws, saved=saved)
     return dict(dq=dq, dk=dk_, dv=dv_, dg=dg, dbeta=dbeta, dS0=dS0)
 
 

@@ -83,12 +83,34 @@ int check_ws(const void *ws, size_t ws_bytes, size_t need) {
   return CKDA_OK;
 }
 
+// bytes of the forward-to-backward saved buffer; 0: no saved form
+size_t saved_bytes_for(int B, int T, int H, int dk, int dv, int io_dtype);
+
+// The saved buffer, if one is given and the configuration has a saved form;
+// null otherwise.  *rc: CKDA_OK or the argument error.
+const void *saved_or_null(const void *saved, size_t saved_bytes, int B, int T, int H, int dk, int dv,
+                          int io_dtype, int *rc) {
+  *rc = CKDA_OK;
+  const size_t need = saved_bytes_for(B, T, H, dk, dv, io_dtype);
+  if (!saved || need == 0) return nullptr;
+  *rc = check_ws(saved, saved_bytes, need);
+  return *rc == CKDA_OK ? saved : nullptr;
+}
+
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? CKDA_OK : CKDA_ERR_CUDA; }
 
 // bf16 I/O at dk = dv = 128 runs on the tensor cores; other shapes and fp32
 // I/O (whose 1e-4 accuracy target bf16 operands cannot meet) on CUDA cores.
 bool use_tensor_cores(int io_dtype, int dk, int dv) {
   return io_dtype == CKDA_BF16 && dk == 128 && dv == 128;
+}
+
+// The tensor-core path's per-(chunk, head) records are what the forward can
+// save for the backward.
+size_t saved_bytes_for(int B, int T, int H, int dk, int dv, int io_dtype) {
+  if (!use_tensor_cores(io_dtype, dk, dv)) return 0;
+  const int64_t nch = (int64_t)B * ((T + C - 1) / C);
+  return (size_t)nch * H * tc_record_bytes();
 }
 
 #define CKDA_TRY(expr)                          \
@@ -111,14 +133,24 @@ size_t ckda_workspace_size(int op, int B, int T, int H, int dk, int dv, int N) {
   return ws_layout(op, B, T, H, dk, dv, N).total;
 }
 
+size_t ckda_saved_size(int B, int T, int H, int dk, int dv, int io_dtype) {
+  if (check_common(B, T, H, dk, dv, io_dtype) != CKDA_OK) return 0;
+  return saved_bytes_for(B, T, H, dk, dv, io_dtype);
+}
+
 int ckda_chunk_fwd(int B, int T, int H, int dk, int dv, int io_dtype, const void *q,
                    const void *k, const void *v, const float *g, const int8_t *sign,
                    const void *beta, const float *S0, void *o, float *ST, float *chunk_states,
-                   void *ws, size_t ws_bytes, cudaStream_t stream) {
+                   void *saved, size_t saved_bytes, void *ws, size_t ws_bytes,
+                   cudaStream_t stream) {
   CKDA_TRY(check_common(B, T, H, dk, dv, io_dtype));
   const bool empty = (int64_t)B * T == 0;
   if (!empty) CKDA_TRY(check_ptrs({q, k, v, g, sign, beta, o}, {S0, ST, chunk_states}));
   else CKDA_TRY(check_ptrs({}, {S0, ST, chunk_states}));
+  int rc;
+  unsigned char *recs_out = static_cast<unsigned char *>(
+      const_cast<void *>(saved_or_null(saved, saved_bytes, B, T, H, dk, dv, io_dtype, &rc)));
+  CKDA_TRY(rc);
   const WsLayout L = ws_layout(CKDA_OP_CHUNK_FWD, B, T, H, dk, dv, 0);
   CKDA_TRY(check_ws(ws, ws_bytes, L.total));
   char *w = static_cast<char *>(ws);
@@ -135,7 +167,7 @@ int ckda_chunk_fwd(int B, int T, int H, int dk, int dv, int io_dtype, const void
   a.status = reinterpret_cast<DevStatus *>(w);
   const bool bf16 = io_dtype == CKDA_BF16;
   if (use_tensor_cores(io_dtype, dk, dv)) {
-    CKDA_CUDA(tc_forward(a, reinterpret_cast<unsigned char *>(w + L.intra),
+    CKDA_CUDA(tc_forward(a, recs_out ? recs_out : reinterpret_cast<unsigned char *>(w + L.intra),
                          reinterpret_cast<float *>(w + L.fscratch), true, chunk_states, stream));
     return CKDA_OK;
   }
@@ -147,8 +179,9 @@ int ckda_chunk_fwd(int B, int T, int H, int dk, int dv, int io_dtype, const void
 int ckda_chunk_bwd(int B, int T, int H, int dk, int dv, int io_dtype, const void *q,
                    const void *k, const void *v, const float *g, const int8_t *sign,
                    const void *beta, const float *S0, const void *dO, const float *dST,
-                   const float *chunk_states, void *dq, void *dk_out, void *dv_out, float *dg,
-                   void *dbeta, float *dS0, void *ws, size_t ws_bytes, cudaStream_t stream) {
+                   const float *chunk_states, const void *saved, size_t saved_bytes, void *dq,
+                   void *dk_out, void *dv_out, float *dg, void *dbeta, float *dS0, void *ws,
+                   size_t ws_bytes, cudaStream_t stream) {
   CKDA_TRY(check_common(B, T, H, dk, dv, io_dtype));
   const bool empty = (int64_t)B * T == 0;
   if (!empty)
@@ -156,6 +189,10 @@ int ckda_chunk_bwd(int B, int T, int H, int dk, int dv, int io_dtype, const void
                         {S0, dST, chunk_states, dS0}));
   else
     CKDA_TRY(check_ptrs({}, {S0, dST, chunk_states, dS0}));
+  int rc;
+  const unsigned char *recs_in = static_cast<const unsigned char *>(
+      saved_or_null(saved, saved_bytes, B, T, H, dk, dv, io_dtype, &rc));
+  CKDA_TRY(rc);
   const WsLayout L = ws_layout(CKDA_OP_CHUNK_BWD, B, T, H, dk, dv, 0);
   CKDA_TRY(check_ws(ws, ws_bytes, L.total));
   char *w = static_cast<char *>(ws);
@@ -172,11 +209,15 @@ int ckda_chunk_bwd(int B, int T, int H, int dk, int dv, int io_dtype, const void
   f.intra = reinterpret_cast<float *>(w + L.intra);
   f.status = reinterpret_cast<DevStatus *>(w);
   const float *states = chunk_states;
+  const unsigned char *recs =
+      recs_in ? recs_in : reinterpret_cast<const unsigned char *>(w + L.intra);
   if (tcp) {
+    // the intra-chunk records: the forward's when saved, else recomputed here
     float *st = reinterpret_cast<float *>(w + L.states);
-    CKDA_CUDA(tc_forward(f, reinterpret_cast<unsigned char *>(w + L.intra),
-                         reinterpret_cast<float *>(w + L.fscratch), false, st, stream,
-                         /*state_pass=*/states == nullptr));
+    if (!recs_in || !states)
+      CKDA_CUDA(tc_forward(f, const_cast<unsigned char *>(recs),
+                           reinterpret_cast<float *>(w + L.fscratch), false, st, stream,
+                           /*state_pass=*/states == nullptr, /*intra_pass=*/recs_in == nullptr));
     if (!states) states = st;
   } else {
     CKDA_CUDA(v1_intra(f, bf16, reinterpret_cast<float *>(w + L.fscratch), stream));
@@ -198,8 +239,7 @@ int ckda_chunk_bwd(int B, int T, int H, int dk, int dv, int io_dtype, const void
   a.scratch = reinterpret_cast<float *>(w + L.scratch);
   a.status = f.status;
   if (tcp) {
-    CKDA_CUDA(tc_backward(a, reinterpret_cast<unsigned char *>(w + L.intra),
-                          reinterpret_cast<unsigned char *>(w + L.dsend),
+    CKDA_CUDA(tc_backward(a, recs, reinterpret_cast<unsigned char *>(w + L.dsend),
                           reinterpret_cast<unsigned char *>(w + L.du),
                           reinterpret_cast<float *>(w + L.fscratch), stream));
     return CKDA_OK;

@@ -187,8 +187,10 @@ cudaError_t v1_state_fwd(const FwdArgs &a, bool bf16, bool write_o, float *state
 cudaError_t v1_backward(const BwdArgs &a, bool bf16, cudaStream_t s);
 size_t tc_fwd_fallback_floats(int ctas);
 int tc_intra_ctas();
+size_t tc_record_bytes();
 cudaError_t tc_forward(const FwdArgs &f, unsigned char *recs, float *fb, bool write_o,
-                       float *states_out, cudaStream_t s, bool state_pass = true);
+                       float *states_out, cudaStream_t s, bool state_pass = true,
+                       bool intra_pass = true);
 cudaError_t tc_backward(const BwdArgs &b, const unsigned char *recs, unsigned char *dS_tiles,
                         unsigned char *dU_tiles, float *fb, cudaStream_t s);
 cudaError_t decode_step(int N, int H, int dk, int dv, bool bf16, const void *q,

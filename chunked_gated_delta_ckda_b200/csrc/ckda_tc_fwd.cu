@@ -602,10 +602,13 @@ int tc_intra_ctas() {
   return want < kBwdCtas ? want : kBwdCtas;
 }
 
+size_t tc_record_bytes() { return REC; }
+
 // Forward on tensor cores.  recs: n_chunks_bound * H records of REC bytes;
-// fb: tc_fwd_fallback_floats(tc_intra_ctas()) floats.
+// fb: tc_fwd_fallback_floats(tc_intra_ctas()) floats.  intra_pass = false
+// reuses records an earlier call wrote for the same inputs.
 cudaError_t tc_forward(const FwdArgs &f, unsigned char *recs, float *fb, bool write_o,
-                       float *states_out, cudaStream_t s, bool state_pass) {
+                       float *states_out, cudaStream_t s, bool state_pass, bool intra_pass) {
   TcArgs ta;
   ta.f = f;
   ta.recs = recs;
@@ -619,7 +622,7 @@ cudaError_t tc_forward(const FwdArgs &f, unsigned char *recs, float *fb, bool wr
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(tc_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_state);
   if (e != cudaSuccess) return e;
-  {
+  if (intra_pass) {
     ProfScope prof("tc_intra", s);
     tc_intra_kernel<<<tc_intra_ctas(), kIntraThreads, sm_intra, s>>>(ta);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;

@@ -89,6 +89,15 @@ extern "C" {
  * tokens and N = number of sequences.  Returns 0 for invalid arguments. */
 size_t ckda_workspace_size(int op, int B, int T, int H, int dk, int dv, int N);
 
+/* Bytes of the "saved" buffer through which ckda_chunk_fwd can hand its
+ * per-chunk intra-chunk results (the UT-transform products of every
+ * (chunk, head)) to ckda_chunk_bwd, so that the backward does not recompute
+ * them: a memory-for-time trade, like chunk_states.  Returns 0 for shapes
+ * and dtypes that have no saved form (then `saved` is ignored by both calls
+ * and the backward recomputes) and for invalid arguments.  The contents are
+ * opaque; they are valid for the inputs of the forward that wrote them. */
+size_t ckda_saved_size(int B, int T, int H, int dk, int dv, int io_dtype);
+
 /* Chunked forward over B independent sequences of length T.
  *   q, k  [B,T,H,dk] io;  v [B,T,H,dv] io;  g [B,T,H,dk] f32;
  *   sign  [B,T,H,dk] int8;  beta [B,T,H] io
@@ -98,20 +107,27 @@ size_t ckda_workspace_size(int op, int B, int T, int H, int dk, int dv, int N);
  *   chunk_states [B,H,ceil(T/64),dk,dv] f32, nullable: the state at the start
  *         of every 64-token chunk (true frame); pass it to ckda_chunk_bwd to
  *         skip the backward's forward recomputation.
+ *   saved, saved_bytes: nullable; when ckda_saved_size(...) > 0, a 256-byte
+ *         aligned buffer of at least that many bytes (CKDA_ERR_WORKSPACE if
+ *         smaller) that receives the per-chunk results for ckda_chunk_bwd.
  * The algorithm is the chunk-wise (WY / UT-transform) form the second source
  * names: per 64-token chunk a unit-lower-triangular intra-chunk system is
  * inverted, then a sequential pass carries the state across chunks. */
 int ckda_chunk_fwd(int B, int T, int H, int dk, int dv, int io_dtype,
                    const void *q, const void *k, const void *v, const float *g,
                    const int8_t *sign, const void *beta, const float *S0,
-                   void *o, float *ST, float *chunk_states, void *ws,
-                   size_t ws_bytes, cudaStream_t stream);
+                   void *o, float *ST, float *chunk_states, void *saved,
+                   size_t saved_bytes, void *ws, size_t ws_bytes,
+                   cudaStream_t stream);
 
 /* Gradients of L(o, ST) through ckda_chunk_fwd.
  *   dO    [B,T,H,dv] io: dL/do
  *   dST   [B,H,dk,dv] f32, nullable (zero): dL/dST
  *   chunk_states: nullable; the buffer ckda_chunk_fwd filled for the same
  *         inputs (else the forward chunk states are recomputed in ws)
+ *   saved, saved_bytes: nullable; the buffer ckda_chunk_fwd filled for the
+ *         same inputs (else the per-chunk results are recomputed in ws).
+ *         Ignored when ckda_saved_size(...) is 0.
  *   dq, dk_out [B,T,H,dk] io;  dv_out [B,T,H,dv] io;  dg [B,T,H,dk] f32
  *         (dL/d log|alpha|);  dbeta [B,T,H] io;  dS0 [B,H,dk,dv] f32, nullable
  * The sign gets no gradient (piecewise constant); dg is the exact gradient
@@ -121,7 +137,8 @@ int ckda_chunk_bwd(int B, int T, int H, int dk, int dv, int io_dtype,
                    const void *q, const void *k, const void *v, const float *g,
                    const int8_t *sign, const void *beta, const float *S0,
                    const void *dO, const float *dST, const float *chunk_states,
-                   void *dq, void *dk_out, void *dv_out, float *dg, void *dbeta,
+                   const void *saved, size_t saved_bytes, void *dq,
+                   void *dk_out, void *dv_out, float *dg, void *dbeta,
                    float *dS0, void *ws, size_t ws_bytes, cudaStream_t stream);
 
 /* One recurrent step of N*H independent states, in place (the model card's

@@ -37,6 +37,18 @@ def test_workspace_size_rules():
     assert ws(0, 1, 0, 2, 64, 64, 0) > 0         # empty input still has a status block
 
 
+def test_saved_size_rules():
+    sv = _abi.ckda_saved_size
+    one = sv(1, 64, 1, 128, 128, 1)                # one (chunk, head) record
+    assert one > 0 and one % 256 == 0
+    assert sv(8, 4096, 16, 128, 128, 1) == 8 * 64 * 16 * one
+    assert sv(2, 65, 3, 128, 128, 1) == 2 * 2 * 3 * one   # a ragged last chunk has a record
+    assert sv(8, 4096, 16, 128, 128, 0) == 0       # fp32 I/O: the backward recomputes
+    assert sv(8, 4096, 16, 64, 64, 1) == 0         # d = 64: the backward recomputes
+    assert sv(1, 64, 2, 96, 64, 1) == 0            # unsupported dk
+    assert sv(1, 0, 2, 128, 128, 1) == 0           # empty
+
+
 def _raw():
     return _abi.library()
 
@@ -45,23 +57,32 @@ def test_host_validation_without_gpu():
     lib = _raw()
     fake = ctypes.c_void_p(1 << 20)     # never dereferenced: the calls fail validation first
     odd = ctypes.c_void_p((1 << 20) + 4)
-    args = [fake] * 11
+    args = [fake] * 10
+    nosave = [None, 0]
+
+    def fwd(B, T, H, dk, dv, io, a, ws_bytes, saved=nosave):
+        return lib.ckda_chunk_fwd(B, T, H, dk, dv, io, *a, *saved, fake, ws_bytes, None)
+
     # unsupported head size
-    assert lib.ckda_chunk_fwd(1, 64, 2, 96, 64, 0, *args, 1 << 30, None) == 2
+    assert fwd(1, 64, 2, 96, 64, 0, args, 1 << 30) == 2
     # bad io dtype
-    assert lib.ckda_chunk_fwd(1, 64, 2, 64, 64, 5, *args, 1 << 30, None) == 1
+    assert fwd(1, 64, 2, 64, 64, 5, args, 1 << 30) == 1
     # negative sizes
-    assert lib.ckda_chunk_fwd(-1, 64, 2, 64, 64, 0, *args, 1 << 30, None) == 1
+    assert fwd(-1, 64, 2, 64, 64, 0, args, 1 << 30) == 1
     # null required pointer
     a = list(args)
     a[0] = None
-    assert lib.ckda_chunk_fwd(1, 64, 2, 64, 64, 0, *a, 1 << 30, None) == 1
+    assert fwd(1, 64, 2, 64, 64, 0, a, 1 << 30) == 1
     # misaligned tensor
     a = list(args)
     a[1] = odd
-    assert lib.ckda_chunk_fwd(1, 64, 2, 64, 64, 0, *a, 1 << 30, None) == 3
+    assert fwd(1, 64, 2, 64, 64, 0, a, 1 << 30) == 3
     # workspace too small
-    assert lib.ckda_chunk_fwd(1, 64, 2, 64, 64, 0, *args, 16, None) == 4
+    assert fwd(1, 64, 2, 64, 64, 0, args, 16) == 4
+    # saved buffer: too small / misaligned where the configuration has a saved form
+    need = lib.ckda_saved_size(1, 64, 2, 128, 128, 1)
+    assert fwd(1, 64, 2, 128, 128, 1, args, 1 << 30, [fake, need - 1]) == 4
+    assert fwd(1, 64, 2, 128, 128, 1, args, 1 << 30, [ctypes.c_void_p((1 << 20) + 16), need]) == 3
     # decode: unsupported / null
     assert lib.ckda_decode_step(4, 2, 64, 32, 0, *([fake] * 8), None) == 2
     assert lib.ckda_decode_step(4, 2, 64, 64, 0, *([None] * 8), None) == 1
@@ -69,12 +90,18 @@ def test_host_validation_without_gpu():
     v = [fake] * 9
     assert lib.ckda_varlen_fwd(100, 2, fake, 0, 2, 64, 64, 0, *v, fake, 1 << 30, None) == 1
     assert lib.ckda_varlen_fwd(100, -1, fake, 50, 2, 64, 64, 0, *v, fake, 1 << 30, None) == 1
+
+    def bwd(io, b, ws_bytes, saved=nosave):
+        return lib.ckda_chunk_bwd(1, 64, 2, 128, 128, io, *b[:10], *saved, *b[10:], fake, ws_bytes, None)
+
     # backward: missing gradient output
-    b = [fake] * 17
+    b = [fake] * 16
     b[13] = None  # dg
-    assert lib.ckda_chunk_bwd(1, 64, 2, 64, 64, 1, *b, 1 << 30, None) == 1
+    assert bwd(1, b, 1 << 30) == 1
     # backward: workspace too small
     b[13] = fake
-    assert lib.ckda_chunk_bwd(1, 64, 2, 64, 64, 1, *b, 16, None) == 4
+    assert bwd(1, b, 16) == 4
+    # backward: saved buffer too small (bf16, d = 128 has a saved form)
+    assert bwd(1, b, 1 << 30, [fake, 16]) == 4
     # zero-sized decode is a no-op
     assert lib.ckda_decode_step(0, 2, 64, 64, 0, *([None] * 8), None) == 0

@@ -122,6 +122,44 @@ def test_backward_uses_saved_chunk_states():
         check(key, a[key], f64(b[key]), io)
 
 
+@pytest.mark.parametrize("with_cs", [True, False])
+def test_backward_with_saved_forward_results(with_cs):
+    """The forward's saved per-chunk results stand in for the backward's
+    recomputation: same kernel on the same inputs, so the gradients are
+    bit-identical; and they match the oracle."""
+    io = torch.bfloat16
+    inp = random_inputs(2, 300, 2, 128, 128, io, seed=13, gscale=0.3, extreme_p=0.05)
+    d = to_dev(inp)
+    S0, dST = inp["S0"].cuda(), inp["dST"].cuda()
+    o, ST, cs, sv = api.chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["sign"], d["beta"], S0=S0,
+                                  save_chunk_states=True, save_for_backward=True)
+    assert sv is not None and sv.numel() == _abi.ckda_saved_size(2, 300, 2, 128, 128, _abi.CKDA_BF16)
+    args = (d["q"], d["k"], d["v"], d["g"], d["sign"], d["beta"], d["dO"])
+    a = api.chunk_bwd(*args, S0=S0, dST=dST, chunk_states=cs if with_cs else None, saved=sv)
+    b = api.chunk_bwd(*args, S0=S0, dST=dST, chunk_states=cs if with_cs else None)
+    torch.cuda.synchronize()
+    for key in a:
+        assert torch.equal(a[key], b[key]), key
+    ref = oracle_bwd_batched(inp, inp["dO"], S0=inp["S0"], dST=inp["dST"])
+    for key in ("dq", "dk", "dv", "dg", "dbeta", "dS0"):
+        check(key, a[key], ref[key], io)
+
+
+def test_saved_is_ignored_without_a_saved_form():
+    io = torch.float32
+    inp = random_inputs(1, 100, 2, 64, 64, io, seed=14)
+    d = to_dev(inp)
+    o, ST, cs, sv = api.chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["sign"], d["beta"],
+                                  save_chunk_states=True, save_for_backward=True)
+    assert sv is None and _abi.ckda_saved_size(1, 100, 2, 64, 64, _abi.CKDA_F32) == 0
+    junk = torch.empty(4096, dtype=torch.uint8, device="cuda")   # ignored for this configuration
+    got = api.chunk_bwd(d["q"], d["k"], d["v"], d["g"], d["sign"], d["beta"], d["dO"],
+                        chunk_states=cs, saved=junk)
+    ref = oracle_bwd_batched(inp, inp["dO"])
+    for key in ("dq", "dk", "dv", "dg", "dbeta", "dS0"):
+        check(key, got[key], ref[key], io)
+
+
 def test_backward_without_state_inputs():
     io = torch.float32
     inp = random_inputs(1, 100, 2, 64, 64, io, seed=12)
@@ -241,8 +279,10 @@ def test_full_layer_fwd_bwd_sampled_heads():
     w = W.LAYER_FWDBWD
     inp = W.make(w)
     d = to_dev(inp)
-    o, ST, cs = api.chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["sign"], d["beta"], save_chunk_states=True)
-    gr = api.chunk_bwd(d["q"], d["k"], d["v"], d["g"], d["sign"], d["beta"], d["dO"], chunk_states=cs)
+    o, ST, cs, sv = api.chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["sign"], d["beta"],
+                                  save_chunk_states=True, save_for_backward=True)
+    gr = api.chunk_bwd(d["q"], d["k"], d["v"], d["g"], d["sign"], d["beta"], d["dO"], chunk_states=cs,
+                       saved=sv)
     torch.cuda.synchronize()
     for b, h in _sample_heads(w.B, w.H, 3, seed=1):
         sub = {k: inp[k][b:b + 1, :, h:h + 1].contiguous() for k in ("q", "k", "v", "g", "sign", "beta", "dO")}
