@@ -217,7 +217,9 @@ constexpr uint32_t R2 = 32768;   // U0^T: K-major tile [v][s] (128 x 64)
 constexpr uint32_t R3 = 49152;   // A_q: K-major tile [r][s] (64 x 64)
 constexpr uint32_t R4 = 57344;   // Khat^T: K-major tile [c][s] (128 x 64)
 constexpr uint32_t R5 = 73728;   // d[128] fp32
-constexpr uint32_t REC = 74240;  // bytes per (chunk, head) record
+constexpr uint32_t R6 = 74240;   // M = (I + Diag(beta) A)^{-1}: fp32 [64][65] (row stride 65)
+constexpr uint32_t REC_STATE = R6;  // R1 .. R5: the part the sequential state passes read
+constexpr uint32_t REC = 90880;  // bytes per (chunk, head) record
 
 // 2^x and 1/x with one MUFU instruction each (PTX ex2.approx / rcp.approx);
 // their relative error (~2^-22) is far below the bf16 operand rounding.
@@ -287,7 +289,8 @@ __device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8]) {
 // warp w owns chunk rows 8w .. 8w+7, lane l owns key channels 4l .. 4l+3.
 // Every load is a coalesced vector load of a full 128-channel row.
 // ---------------------------------------------------------------------------
-struct PrepTot {  // per-group totals exchanged through shared memory
+// per-group totals exchanged through shared memory (G is accessed as float4)
+struct alignas(16) PrepTot {
   float G[8][128];
   uint8_t P[8][128];
 };

@@ -293,14 +293,17 @@ constexpr uint32_t G_UV = 65536;      // [U; V] K-major 128 x 128
 constexpr uint32_t G_TT = 98304;      // T K-major [r][j] 64 x 64
 constexpr uint32_t G_OU = 106496;     // [dO; dU] K-major 128 x 128
 constexpr uint32_t G_SC = 139264;     // S_c bf16 K-major [c][v]; later dW in rows 64..127
-constexpr uint32_t G_WN = 172032;     // N fp32 | W tile | dS1 tile | [dA; dAq] + dT fp32
+constexpr uint32_t G_WN = 172032;     // W tile | dS1 tile | [dA; dAq] + dT fp32
 constexpr uint32_t G_DT = G_WN + 16384;
 constexpr uint32_t G_MF = 205824;     // M fp32 [64][65]
 constexpr uint32_t G_MISC = 222464;
 constexpr int LDF = 65;
+constexpr uint32_t W_TILE = 16384;              // W^T half of the record's R1 tile
+constexpr uint32_t M_BYTES = 64 * LDF * 4;      // the record's M
+static_assert(M_BYTES == REC - R6, "M is the record's last field");
 
 struct GMisc {
-  uint64_t bar[6], mdu, mds, mfin;
+  uint64_t bar[6], mdu, mds, mfin, mrec;
   uint32_t tmem;
   int pad;
   float beta[64], dbc[64], dbr[2][64];
@@ -308,9 +311,6 @@ struct GMisc {
   uint8_t pbits[8][128];
   float dd[2][128];
 };
-// scratch that lives in tiles idle at the time: inverse blocks in the free
-// tail of the N-matrix region, final-epilogue sums in the [U; V] tile
-constexpr uint32_t G_XS = G_WN + 17408;  // float [3][16][16]
 
 // Completion of MMAs (or of a copy only MMAs consume): one thread polls the
 // mbarrier, the others wait at the CTA barrier (no spinning issue slots).
@@ -344,6 +344,7 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(BwdTcArgs ta) {
     mbar_init(&ms.mdu, 1);
     mbar_init(&ms.mds, 1);
     mbar_init(&ms.mfin, 1);
+    mbar_init(&ms.mrec, 1);
     mbar_fence_init();
   }
   if (warp == 0) {
@@ -357,11 +358,9 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(BwdTcArgs ta) {
   const uint32_t sA1 = smem_u32(sm + G_A1), sB1 = smem_u32(sm + G_B1), sKG = smem_u32(sm + G_KG);
   const uint32_t sUV = smem_u32(sm + G_UV), sTT = smem_u32(sm + G_TT), sOU = smem_u32(sm + G_OU);
   const uint32_t sSC = smem_u32(sm + G_SC), sWN = smem_u32(sm + G_WN);
-  float *Nf = reinterpret_cast<float *>(sm + G_WN);
   float *dTf = reinterpret_cast<float *>(sm + G_DT);
   float *Mf = reinterpret_cast<float *>(sm + G_MF);
   float *tmpf = reinterpret_cast<float *>(sm + G_KG);  // [64][64]
-  float(*Xs)[16][16] = reinterpret_cast<float(*)[16][16]>(sm + G_XS);
   float *gcps = reinterpret_cast<float *>(sm + G_UV);         // [2][128], final epilogue only
   float *acc1s = gcps + 256;                                  // [2][128]
   float *fb = ta.fb + (size_t)blockIdx.x * 3 * 64 * D;
@@ -385,9 +384,15 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(BwdTcArgs ta) {
 
     // ---------------- loads ----------------
     if (tid == 0) {
+      fence_async_smem();  // earlier generic accesses of the destinations come first
       mbar_arrive_expect_tx(&ms.mdu, DU_TILE);
       bulk_g2s(sm + G_OU + 8192, gdU, 8192, &ms.mdu);
       bulk_g2s(sm + G_OU + 16384 + 8192, gdU + 8192, 8192, &ms.mdu);
+      // the forward's W tile and M of this chunk
+      const unsigned char *rec = ta.recs + (size_t)item * REC;
+      mbar_arrive_expect_tx(&ms.mrec, W_TILE + M_BYTES);
+      bulk_g2s(sm + G_WN, rec + R1, W_TILE, &ms.mrec);
+      bulk_g2s(sm + G_MF, rec + R6, M_BYTES, &ms.mrec);
     }
     // every load of the item is in flight before any of them is used:
     // V and dO rows, the start state S_c (fp32), then the prep rows
@@ -470,47 +475,8 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(BwdTcArgs ta) {
     fence_async_smem();
     __syncthreads();
 
-    // ---------------- A (-> N = Diag(beta) A) ----------------
-    if (fast) {
-      if (tid == 0) {
-        tc_fence_after();
-        const uint32_t id = idesc_bf16(128, 64, false, false);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_bf16(tmem, sdesc(sA1 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-                   sdesc(sB1 + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), id, kk > 0);
-        mma_commit(&ms.bar[0]);
-      }
-      if (!wait_one(&ms.bar[0], ph, a.status, 401)) { abort = true; break; }
-      tc_fence_after();
-      if (qd >= 2) {  // lanes 64..127: rows of A
-        const int r = 32 * qd + lane - 64, ch = warp >> 2;
-        float x[16], y[16];
-        tmem_ld16(lanebase + 32 * ch, x);
-        tmem_ld16(lanebase + 32 * ch + 16, y);
-        tmem_wait_ld();
-        const float br = ms.beta[r];
-#pragma unroll
-        for (int jj = 0; jj < 32; ++jj) {
-          const int s = 32 * ch + jj;
-          const float val = jj < 16 ? x[jj] : y[jj - 16];
-          Nf[r * LDF + s] = s < r ? br * val : 0.f;
-        }
-      }
-    } else {
-      for (int e = tid; e < 64 * 64; e += kGThreads) {
-        const int r = e >> 6, s = e & 63;
-        float aa = 0.f;
-        if (s < r)
-          for (int cc = 0; cc < D; ++cc)
-            aa += fb[64 * D + r * D + cc] * fb[64 * D + s * D + cc] * expf(fb[r * D + cc] - fb[s * D + cc]);
-        Nf[r * LDF + s] = s < r ? ms.beta[r] * aa : 0.f;
-      }
-    }
-    __syncthreads();
-
-    // ---------------- M = (I + N)^{-1} ----------------
-    inverse64(Mf, Nf, Xs);
+    // ---------------- T = M Diag(beta) (M from the forward's record) ----------------
+    if (!wait_all(&ms.mrec, ph, a.status, 401)) { abort = true; break; }
     {
       const int r = tid >> 2, j0 = (tid & 3) * 16;
       uint32_t pk[8];
@@ -524,48 +490,27 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(BwdTcArgs ta) {
     fence_async_smem();
     __syncthreads();
 
-    // ---------------- W^T, U0^T ----------------
+    // ---------------- A (kept in TMEM for dbeta), U^T = V^T T^T - (W S)^T ----------------
+    // A's MMA completes before any later commit fires, which covers its reads.
     if (tid == 0) {
       tc_fence_after();
-      const uint32_t id = idesc_bf16(128, 64, true, false);
+      if (fast) {
+        const uint32_t id = idesc_bf16(128, 64, false, false);
 #pragma unroll
-      for (int kk = 0; kk < 4; ++kk) {
-        const uint64_t bd = sdesc(sTT + kk * 32, 16, 1024);
-        mma_bf16(tmem + 64, sdesc(sKG + kk * 2048, 8192, 1024), bd, id, kk > 0);
-        mma_bf16(tmem + 128, sdesc(sUV + 8192 + kk * 2048, 16384, 1024), bd, id, kk > 0);
+        for (int kk = 0; kk < 8; ++kk)
+          mma_bf16(tmem, sdesc(sA1 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                   sdesc(sB1 + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), id, kk > 0);
       }
-      mma_commit(&ms.bar[1]);
-    }
-    if (!wait_one(&ms.bar[1], ph, a.status, 402)) { abort = true; break; }
-    tc_fence_after();
-    {  // W^T -> W tile, MN-major B [K = c][N = r] (over the dead N matrix)
-      const int ch = warp >> 2;
-      float x[16], y[16];
-      tmem_ld16(lanebase + 64 + 32 * ch, x);
-      tmem_ld16(lanebase + 64 + 32 * ch + 16, y);
-      tmem_wait_ld();
-      uint32_t pk[16];
+      const uint32_t idu = idesc_bf16(128, 64, true, false);
 #pragma unroll
-      for (int m = 0; m < 8; ++m) pk[m] = pack_bf16(x[2 * m], x[2 * m + 1]);
-#pragma unroll
-      for (int m = 0; m < 8; ++m) pk[8 + m] = pack_bf16(y[2 * m], y[2 * m + 1]);
-#pragma unroll
-      for (int m = 0; m < 4; ++m)
-        *reinterpret_cast<uint4 *>(sm + G_WN + mnmaj_off(c, 32 * ch + 8 * m, 128)) =
-            make_uint4(pk[4 * m], pk[4 * m + 1], pk[4 * m + 2], pk[4 * m + 3]);
-    }
-    fence_async_smem();
-    tc_fence_before();
-    __syncthreads();
-
-    // ---------------- (W S)^T -> U ----------------
-    if (tid == 0) {
-      tc_fence_after();
-      const uint32_t id = idesc_bf16(128, 64, true, true);
+      for (int kk = 0; kk < 4; ++kk)
+        mma_bf16(tmem + 128, sdesc(sUV + 8192 + kk * 2048, 16384, 1024), sdesc(sTT + kk * 32, 16, 1024), idu,
+                 kk > 0);
+      const uint32_t idw = idesc_bf16(128, 64, true, true) | (1u << 13);  // negate A: subtract
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk)
-        mma_bf16(tmem + 192, sdesc(sSC + kk * 2048, 16384, 1024), sdesc(sWN + kk * 2048, 16384, 1024), id,
-                 kk > 0);
+        mma_bf16(tmem + 128, sdesc(sSC + kk * 2048, 16384, 1024), sdesc(sWN + kk * 2048, 16384, 1024), idw,
+                 true);
       mma_commit(&ms.bar[2]);
     }
     if (!wait_one(&ms.bar[2], ph, a.status, 403)) { abort = true; break; }
@@ -574,16 +519,15 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(BwdTcArgs ta) {
       mbar_arrive_expect_tx(&ms.mds, DS_TILE);
       bulk_g2s(sm + G_WN, gdS, DS_TILE, &ms.mds);
     }
-    {  // U^T = U0^T - (W S)^T ; U rows s (K-major [s][v]) of the [U; V] tile
+    {  // U rows s (K-major [s][v]) of the [U; V] tile
       const int ch = warp >> 2;
 #pragma unroll
       for (int h16 = 0; h16 < 2; ++h16) {
-        float u0[16], ws[16];
-        tmem_ld16(lanebase + 128 + 32 * ch + 16 * h16, u0);
-        tmem_ld16(lanebase + 192 + 32 * ch + 16 * h16, ws);
+        float u[16];
+        tmem_ld16(lanebase + 128 + 32 * ch + 16 * h16, u);
         tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 16; ++i) st_bf16(sm + G_UV, kmaj_off(32 * ch + 16 * h16 + i, c, 128), u0[i] - ws[i]);
+        for (int i = 0; i < 16; ++i) st_bf16(sm + G_UV, kmaj_off(32 * ch + 16 * h16 + i, c, 128), u[i]);
       }
     }
     // dd partial: sum over v of S_c[c][v] * dS1[c][v] (dS1 arrives meanwhile)
@@ -1025,6 +969,5 @@ cudaError_t tc_backward(const BwdArgs &b, const unsigned char *recs, unsigned ch
 
 size_t tc_bwd_smem_bytes() { return G_MISC + sizeof(GMisc) + 1024; }
 static_assert(G_MISC + sizeof(GMisc) + 1024 <= 232448, "gradient kernel shared memory");
-static_assert(G_XS + 3 * 16 * 16 * 4 <= G_WN + 33792, "inverse scratch inside the N region");
 
 }  // namespace ckda

@@ -39,6 +39,7 @@ namespace {
 using namespace tc;
 
 constexpr uint32_t REC_PAD = 74752;  // record slot in shared memory (73 x 1024)
+static_assert(REC_STATE <= REC_PAD, "the state pass's part of a record fits its slot");
 
 // ===========================================================================
 // intra-chunk kernel
@@ -300,6 +301,9 @@ __global__ void __launch_bounds__(kIntraThreads, 2) tc_intra_kernel(TcArgs ta) {
       *reinterpret_cast<uint4 *>(sm + I_T + kmaj_off(r, j0, 64)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
       *reinterpret_cast<uint4 *>(sm + I_T + kmaj_off(r, j0 + 8, 64)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
     }
+    // M itself goes to the record too: the backward starts from it
+    for (int i = tid; i < 64 * LDF / 4; i += kIntraThreads)
+      reinterpret_cast<float4 *>(rec + R6)[i] = reinterpret_cast<const float4 *>(Mf)[i];
     fence_async_smem();
     __syncthreads();
 
@@ -436,8 +440,8 @@ __global__ void __launch_bounds__(kStateThreads, 1) tc_state_kernel(TcArgs ta) {
   };
   if (tid == 0) {
     for (int j = 0; j < 2 && j < nc; ++j) {
-      mbar_arrive_expect_tx(&ms.mrec[j], REC);
-      bulk_g2s(recbuf[j], record(j), REC, &ms.mrec[j]);
+      mbar_arrive_expect_tx(&ms.mrec[j], REC_STATE);
+      bulk_g2s(recbuf[j], record(j), REC_STATE, &ms.mrec[j]);
     }
   }
   bool abort = false;
@@ -527,8 +531,8 @@ __global__ void __launch_bounds__(kStateThreads, 1) tc_state_kernel(TcArgs ta) {
     tc_fence_after();
     // the record buffer is free again: fetch chunk j + 2 into it
     if (tid == 0 && j + 2 < nc) {
-      mbar_arrive_expect_tx(&ms.mrec[buf], REC);
-      bulk_g2s(rec, record(j + 2), REC, &ms.mrec[buf]);
+      mbar_arrive_expect_tx(&ms.mrec[buf], REC_STATE);
+      bulk_g2s(rec, record(j + 2), REC_STATE, &ms.mrec[buf]);
     }
     // next state (this thread: columns c in [64 ch, 64 ch + 64))
     const bool last = (j + 1 == nc);
