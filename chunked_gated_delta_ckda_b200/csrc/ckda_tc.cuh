@@ -3,6 +3,7 @@
 // with bounded waits, bulk async copies.  Inline PTX only (PTX ISA forms).
 #pragma once
 
+#include <cuda.h>  // CUtensorMap (a plain 128-byte descriptor type)
 #include <cuda_bf16.h>
 #include <stdint.h>
 
@@ -10,6 +11,17 @@
 
 namespace ckda {
 namespace tc {
+
+// Tensor maps of the per-token row tensors, viewed as [tokens][H][128]: each
+// TMA box is 64 tokens x one head x 64 channels (bf16, 128-byte swizzle: the
+// K-major SW128 tile layout) or 128 channels (g fp32, sign int8; plain rows).
+// Rows past the last token read as zeros.
+struct RowMaps {
+  CUtensorMap q, k, v, dO, g, sign;
+};
+// host: encode the maps for ntok tokens of H heads (dO may be null)
+cudaError_t make_row_maps(RowMaps &m, const void *q, const void *k, const void *v, const void *dO,
+                          const float *g, const int8_t *sign, int64_t ntok, int H);
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -57,6 +69,17 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t phase, DevStat
 // ---------------------------------------------------------------------------
 // bulk async copy global -> shared (1-D, 16-byte aligned, size % 16 == 0)
 // ---------------------------------------------------------------------------
+// One TMA box of a RowMaps tensor: channels c0.., head h, tokens tok..tok+63.
+// c0 * element size is a multiple of 16 bytes (0 or 64 channels of bf16).
+__device__ __forceinline__ void tma_rows(void *smem_dst, const CUtensorMap *map, int c0, int h, int tok,
+                                         uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, "
+      "%4}], [%5];" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(h), "r"(tok), "r"(smem_u32(bar))
+      : "memory");
+}
+
 __device__ __forceinline__ void bulk_g2s(void *smem_dst, const void *gmem_src, uint32_t bytes,
                                          uint64_t *bar) {
   asm volatile(
@@ -204,6 +227,14 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t *>(&v);
 }
+// x = hi + lo with hi = bf16(x) and lo = bf16(x - hi): a pair of bf16 values
+// that carries ~16 significant bits into a tensor-core product
+__device__ __forceinline__ void split_bf16x2(float a, float b, uint32_t &hi, uint32_t &lo) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  const float2 hf = __bfloat1622float2(h);
+  hi = *reinterpret_cast<const uint32_t *>(&h);
+  lo = pack_bf16(a - hf.x, b - hf.y);
+}
 
 // ---------------------------------------------------------------------------
 // per (chunk, head) record of the intra-chunk kernel (bf16 I/O, dk = dv = 128),
@@ -287,7 +318,7 @@ __device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8]) {
 // ---------------------------------------------------------------------------
 // Chunk preprocessing in the "row-group" thread layout (256 threads):
 // warp w owns chunk rows 8w .. 8w+7, lane l owns key channels 4l .. 4l+3.
-// Every load is a coalesced vector load of a full 128-channel row.
+// Each warp reads whole 128-channel rows of the staged (TMA-loaded) tiles.
 // ---------------------------------------------------------------------------
 // per-group totals exchanged through shared memory (G is accessed as float4)
 struct alignas(16) PrepTot {
@@ -304,47 +335,56 @@ struct Prep {
   uint32_t pC;       // bit m: chunk sign product of channel 4l+m is negative
 };
 
-// Loads the 8 x 4 block of this thread, local scans, writes the group totals.
-__device__ __forceinline__ void prep_load(const float *g, const int8_t *sign, const __nv_bfloat16 *k,
-                                          const __nv_bfloat16 *q, int64_t tok0, int len, int h, int H,
-                                          int w, int l, Prep &P, PrepTot &tot) {
-  float4 gv[8];
-  uint32_t sg[8];
-#pragma unroll
-  for (int rr = 0; rr < 8; ++rr) {
-    const int r = 8 * w + rr;
-    const int rrow = r < len ? r : len - 1;
-    const size_t off = ((size_t)(tok0 + rrow) * H + h) * D + 4 * l;
-    gv[rr] = *reinterpret_cast<const float4 *>(g + off);
-    sg[rr] = *reinterpret_cast<const uint32_t *>(sign + off);
-    const uint2 kv = *reinterpret_cast<const uint2 *>(k + off);
-    const uint2 qv = *reinterpret_cast<const uint2 *>(q + off);
-    P.k2[rr][0] = kv.x; P.k2[rr][1] = kv.y;
-    P.q2[rr][0] = qv.x; P.q2[rr][1] = qv.y;
-  }
+// Staged rows of one chunk-head in shared memory (TMA boxes, see RowMaps):
+// q and k as K-major SW128 tiles of 64 rows (two 64-channel blocks), g as
+// fp32 [64][128], sign as int8 [64][128].  Rows past the chunk's length hold
+// other tokens or zeros; they are masked here.
+constexpr uint32_t kStageQ = 0, kStageK = 16384;  // offsets inside the q|k staging region
+constexpr uint32_t kRowBytesQK = 2 * 16384, kRowBytesG = 32768, kRowBytesSign = 8192;
+
+// Reads the 8 x 4 block of this thread, local scans, writes the group totals.
+__device__ __forceinline__ void prep_load_smem(const unsigned char *sqk, const float *sg, const uint8_t *ss,
+                                               int len, int w, int l, Prep &P, PrepTot &tot) {
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
   uint32_t par = 0, pre = 0;
 #pragma unroll
   for (int rr = 0; rr < 8; ++rr) {
-    const bool valid = 8 * w + rr < len;
-    const float gg[4] = {gv[rr].x, gv[rr].y, gv[rr].z, gv[rr].w};
+    const int r = 8 * w + rr;
+    const bool valid = r < len;
+    const float4 gv = *reinterpret_cast<const float4 *>(sg + r * D + 4 * l);
+    const uint32_t sgn = *reinterpret_cast<const uint32_t *>(ss + r * D + 4 * l);
+    const uint32_t off = kmaj_off(r, 4 * l, 64);
+    const uint2 kv = *reinterpret_cast<const uint2 *>(sqk + kStageK + off);
+    const uint2 qv = *reinterpret_cast<const uint2 *>(sqk + kStageQ + off);
+    P.k2[rr][0] = valid ? kv.x : 0u;
+    P.k2[rr][1] = valid ? kv.y : 0u;
+    P.q2[rr][0] = valid ? qv.x : 0u;
+    P.q2[rr][1] = valid ? qv.y : 0u;
+    const float gg[4] = {gv.x, gv.y, gv.z, gv.w};
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
       acc[m] += valid ? gg[m] : 0.f;
       P.G[rr][m] = acc[m];
-      const bool neg = valid && (int8_t)((sg[rr] >> (8 * m)) & 0xffu) < 0;
+      const bool neg = valid && (int8_t)((sgn >> (8 * m)) & 0xffu) < 0;
       par ^= (neg ? 1u : 0u) << m;
     }
     pre |= par << (4 * rr);
-    if (!valid) {
-      P.k2[rr][0] = P.k2[rr][1] = 0u;
-      P.q2[rr][0] = P.q2[rr][1] = 0u;
-    }
   }
   P.pre = pre;
   *reinterpret_cast<float4 *>(&tot.G[w][4 * l]) = make_float4(acc[0], acc[1], acc[2], acc[3]);
 #pragma unroll
   for (int m = 0; m < 4; ++m) tot.P[w][4 * l + m] = (uint8_t)((par >> m) & 1u);
+}
+
+// Zero rows len..63 of a 64-row, 128-channel K-major SW128 tile (two 8 KiB
+// blocks at `base` and `base + block_stride`): whole 128-byte rows, so the
+// swizzle does not matter.
+__device__ __forceinline__ void zero_tail_rows(unsigned char *base, uint32_t block_stride, int len, int tid,
+                                               int nthreads) {
+  for (int e = tid; e < (64 - len) * 16; e += nthreads) {
+    const int r = len + (e >> 4), ch = e & 15;
+    *reinterpret_cast<uint4 *>(base + (ch >> 3) * block_stride + r * 128 + (ch & 7) * 16) = make_uint4(0, 0, 0, 0);
+  }
 }
 
 // After a barrier: add the carry of the earlier row groups; reference row 31

@@ -33,6 +33,7 @@ constexpr uint32_t DS_TILE = 32768;  // dL/dS_{c+1}: bf16 K-major [c][v], 128 ro
 constexpr uint32_t DU_TILE = 16384;  // dU: bf16 K-major [i][v], 64 rows
 
 struct BwdTcArgs {
+  RowMaps rm;                 // q, k, v, dO, g, sign (gradient kernel)
   BwdArgs b;
   const unsigned char *recs;  // intra-chunk records (forward layout)
   unsigned char *dS_tiles;    // [n_chunks][H] DS_TILE
@@ -288,7 +289,7 @@ __global__ void __launch_bounds__(kSbThreads, 1) tc_state_bwd_kernel(BwdTcArgs t
 constexpr int kGThreads = 256;
 constexpr uint32_t G_A1 = 0;          // [Q~; K~l] K-major 128 x 128
 constexpr uint32_t G_B1 = 32768;      // K~r K-major 64 x 128
-constexpr uint32_t G_KG = 49152;      // KG (== K-major [j][c] 64 rows); later tmp fp32 [64][64]
+constexpr uint32_t G_KG = 49152;      // KG (== K-major [j][c] 64 rows); later dM M^T parts
 constexpr uint32_t G_UV = 65536;      // [U; V] K-major 128 x 128
 constexpr uint32_t G_TT = 98304;      // T K-major [r][j] 64 x 64
 constexpr uint32_t G_OU = 106496;     // [dO; dU] K-major 128 x 128
@@ -298,12 +299,16 @@ constexpr uint32_t G_DT = G_WN + 16384;
 constexpr uint32_t G_MF = 205824;     // M fp32 [64][65]
 constexpr uint32_t G_MISC = 222464;
 constexpr int LDF = 65;
+// bf16 hi / lo parts for the dL = -M^T dM M^T products, in tiles idle by then
+constexpr uint32_t G_DMH = G_UV, G_DML = G_UV + 8192;           // dM, K-major [i][j]
+constexpr uint32_t G_MH = G_UV + 16384, G_ML = G_UV + 24576;    // M, K-major [i][a]
+constexpr uint32_t G_TH = G_KG, G_TL = G_KG + 8192;             // dM M^T, K-major [i][k]
 constexpr uint32_t W_TILE = 16384;              // W^T half of the record's R1 tile
 constexpr uint32_t M_BYTES = 64 * LDF * 4;      // the record's M
 static_assert(M_BYTES == REC - R6, "M is the record's last field");
 
 struct GMisc {
-  uint64_t bar[6], mdu, mds, mfin, mrec;
+  uint64_t bar[6], mdu, mds, mfin, mrec, mld;
   uint32_t tmem;
   int pad;
   float beta[64], dbc[64], dbr[2][64];
@@ -325,7 +330,7 @@ __device__ __forceinline__ bool wait_all(uint64_t *bar, uint32_t phase, DevStatu
   return !__syncthreads_or(!ok);
 }
 
-__global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(BwdTcArgs ta) {
+__global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_constant__ BwdTcArgs ta) {
   extern __shared__ unsigned char smem_raw[];
   unsigned char *sm = reinterpret_cast<unsigned char *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -333,9 +338,7 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(BwdTcArgs ta) {
   const BwdArgs &a = ta.b;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int H = a.H;
-  const __nv_bfloat16 *q = (const __nv_bfloat16 *)a.q, *k = (const __nv_bfloat16 *)a.k;
-  const __nv_bfloat16 *v = (const __nv_bfloat16 *)a.v, *beta = (const __nv_bfloat16 *)a.beta;
-  const __nv_bfloat16 *dO = (const __nv_bfloat16 *)a.dO;
+  const __nv_bfloat16 *beta = (const __nv_bfloat16 *)a.beta;
   __nv_bfloat16 *dq = (__nv_bfloat16 *)a.dq, *dk = (__nv_bfloat16 *)a.dkg;
   __nv_bfloat16 *dv = (__nv_bfloat16 *)a.dvg, *dbeta = (__nv_bfloat16 *)a.dbeta;
 
@@ -345,6 +348,7 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(BwdTcArgs ta) {
     mbar_init(&ms.mds, 1);
     mbar_init(&ms.mfin, 1);
     mbar_init(&ms.mrec, 1);
+    mbar_init(&ms.mld, 1);
     mbar_fence_init();
   }
   if (warp == 0) {
@@ -360,7 +364,6 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(BwdTcArgs ta) {
   const uint32_t sSC = smem_u32(sm + G_SC), sWN = smem_u32(sm + G_WN);
   float *dTf = reinterpret_cast<float *>(sm + G_DT);
   float *Mf = reinterpret_cast<float *>(sm + G_MF);
-  float *tmpf = reinterpret_cast<float *>(sm + G_KG);  // [64][64]
   float *gcps = reinterpret_cast<float *>(sm + G_UV);         // [2][128], final epilogue only
   float *acc1s = gcps + 256;                                  // [2][128]
   float *fb = ta.fb + (size_t)blockIdx.x * 3 * 64 * D;
@@ -394,34 +397,39 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(BwdTcArgs ta) {
       bulk_g2s(sm + G_WN, rec + R1, W_TILE, &ms.mrec);
       bulk_g2s(sm + G_MF, rec + R6, M_BYTES, &ms.mrec);
     }
-    // every load of the item is in flight before any of them is used:
-    // V and dO rows, the start state S_c (fp32), then the prep rows
-    uint4 vv[4], oo[4];
+    // the start state S_c (fp32) through registers; the row tensors by TMA:
+    // q, k staged in A1, g in B1 + KG, sign in TT (the prep consumes them
+    // before those tiles are written), V into rows 64.. of [U; V] and dO into
+    // rows 0..63 of [dO; dU] (K-major SW128 boxes)
     float4 x[16];
 #pragma unroll
-    for (int m = 0; m < 4; ++m) {
-      const int e = tid + kGThreads * m, j = e >> 4, cc = e & 15;
-      const int jj = j < len ? j : len - 1;
-      const size_t off = ((size_t)(tok0 + jj) * H + h) * D + cc * 8;
-      vv[m] = *reinterpret_cast<const uint4 *>(v + off);
-      oo[m] = *reinterpret_cast<const uint4 *>(dO + off);
-    }
-#pragma unroll
     for (int m = 0; m < 16; ++m) x[m] = *reinterpret_cast<const float4 *>(Sc + (size_t)(warp + 8 * m) * D + 4 * lane);
-    Prep P;  // row-group layout: rows 8 warp .., channels 4 lane ..
-    prep_load(a.g, a.sign, k, q, tok0, len, h, H, warp, lane, P, ms.tot);
-#pragma unroll
-    for (int m = 0; m < 4; ++m) {
-      const int e = tid + kGThreads * m, j = e >> 4, cc = e & 15;
-      if (j >= len) vv[m] = oo[m] = make_uint4(0, 0, 0, 0);
-      *reinterpret_cast<uint4 *>(sm + G_UV + kmaj_off(64 + j, cc * 8, 128)) = vv[m];
-      *reinterpret_cast<uint4 *>(sm + G_OU + kmaj_off(j, cc * 8, 128)) = oo[m];
+    if (tid == 0) {
+      mbar_arrive_expect_tx(&ms.mld, kRowBytesQK + kRowBytesG + kRowBytesSign + 2 * 16384);
+      const int t = (int)tok0;
+      tma_rows(sm + G_A1 + kStageQ, &ta.rm.q, 0, h, t, &ms.mld);
+      tma_rows(sm + G_A1 + kStageQ + 8192, &ta.rm.q, 64, h, t, &ms.mld);
+      tma_rows(sm + G_A1 + kStageK, &ta.rm.k, 0, h, t, &ms.mld);
+      tma_rows(sm + G_A1 + kStageK + 8192, &ta.rm.k, 64, h, t, &ms.mld);
+      tma_rows(sm + G_B1, &ta.rm.g, 0, h, t, &ms.mld);
+      tma_rows(sm + G_TT, &ta.rm.sign, 0, h, t, &ms.mld);
+      tma_rows(sm + G_UV + 8192, &ta.rm.v, 0, h, t, &ms.mld);
+      tma_rows(sm + G_UV + 16384 + 8192, &ta.rm.v, 64, h, t, &ms.mld);
+      tma_rows(sm + G_OU, &ta.rm.dO, 0, h, t, &ms.mld);
+      tma_rows(sm + G_OU + 16384, &ta.rm.dO, 64, h, t, &ms.mld);
     }
+    if (tid < 64) ms.beta[tid] = tid < len ? __bfloat162float(beta[(size_t)(tok0 + tid) * H + h]) : 0.f;
 #pragma unroll
     for (int m = 0; m < 16; ++m)  // S_c fp32 rows -> bf16 K-major [c][v]
       *reinterpret_cast<uint2 *>(sm + G_SC + kmaj_off(warp + 8 * m, 4 * lane, 128)) =
           make_uint2(pack_bf16(x[m].x, x[m].y), pack_bf16(x[m].z, x[m].w));
-    if (tid < 64) ms.beta[tid] = tid < len ? __bfloat162float(beta[(size_t)(tok0 + tid) * H + h]) : 0.f;
+    if (!wait_all(&ms.mld, ph, a.status, 400)) { abort = true; break; }
+    Prep P;  // row-group layout: rows 8 warp .., channels 4 lane ..
+    prep_load_smem(sm + G_A1, reinterpret_cast<const float *>(sm + G_B1), sm + G_TT, len, warp, lane, P, ms.tot);
+    if (len < 64) {  // V and dO rows past the chunk
+      zero_tail_rows(sm + G_UV + 8192, 16384, len, tid, kGThreads);
+      zero_tail_rows(sm + G_OU, 16384, len, tid, kGThreads);
+    }
     __syncthreads();
     prep_carry(warp, lane, P, ms.tot);
     int bad = 0;
@@ -618,21 +626,59 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(BwdTcArgs ta) {
         for (int m = 0; m < 4; ++m)
           *reinterpret_cast<uint4 *>(sm + G_WN + kmaj_off(64 + r, 32 * ch + 8 * m, 128)) =
               make_uint4(pk[4 * m], pk[4 * m + 1], pk[4 * m + 2], pk[4 * m + 3]);
-      } else {  // dT rows (masked j <= i) -> fp32
+        // row r of M as bf16 hi + lo parts (K-major [i][a]) for the products below
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          const int a0 = 32 * ch + 8 * m;
+          uint32_t hi[4], lo[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) split_bf16x2(Mf[r * LDF + a0 + 2 * e], Mf[r * LDF + a0 + 2 * e + 1], hi[e], lo[e]);
+          *reinterpret_cast<uint4 *>(sm + G_MH + kmaj_off(r, a0, 64)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+          *reinterpret_cast<uint4 *>(sm + G_ML + kmaj_off(r, a0, 64)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        }
+      } else {  // dT rows (masked j <= i) -> fp32, and dM = dT Diag(beta) as bf16 hi + lo parts
         tmem_ld16(lanebase + 192 + 32 * ch, x);
         tmem_ld16(lanebase + 192 + 32 * ch + 16, y);
         tmem_wait_ld();
         const int i = L - 64;
+        float dm[32];
 #pragma unroll
         for (int jj = 0; jj < 32; ++jj) {
           const int j = 32 * ch + jj;
-          const float val = jj < 16 ? x[jj] : y[jj - 16];
-          dTf[i * LDF + j] = j <= i ? val : 0.f;
+          const float val = j <= i ? (jj < 16 ? x[jj] : y[jj - 16]) : 0.f;
+          dTf[i * LDF + j] = val;
+          dm[jj] = val * ms.beta[j];
+        }
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          uint32_t hi[4], lo[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) split_bf16x2(dm[8 * m + 2 * e], dm[8 * m + 2 * e + 1], hi[e], lo[e]);
+          *reinterpret_cast<uint4 *>(sm + G_DMH + kmaj_off(i, 32 * ch + 8 * m, 64)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+          *reinterpret_cast<uint4 *>(sm + G_DML + kmaj_off(i, 32 * ch + 8 * m, 64)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
         }
       }
     }
+    fence_async_smem();
     tc_fence_before();
     __syncthreads();
+    // tmp = dM M^T on the tensor cores, in three bf16 products of the hi / lo parts
+    // (dM_hi M_hi^T + dM_hi M_lo^T + dM_lo M_hi^T, fp32 accumulate: ~16 significant
+    // bits).  A has 64 meaningful rows; its other 64 (the next tile) fill TMEM
+    // lanes 64..127, which nothing reads.
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t id = idesc_bf16(128, 64, false, false);
+      const uint32_t a2[3] = {smem_u32(sm + G_DMH), smem_u32(sm + G_DMH), smem_u32(sm + G_DML)};
+      const uint32_t b2[3] = {smem_u32(sm + G_MH), smem_u32(sm + G_ML), smem_u32(sm + G_MH)};
+#pragma unroll
+      for (int p = 0; p < 3; ++p)
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_bf16(tmem + 128, sdesc(a2[p] + kk * 32, 16, 1024), sdesc(b2[p] + kk * 32, 16, 1024), id,
+                   p > 0 || kk > 0);
+      mma_commit(&ms.bar[0]);
+    }
     // dbeta (column part): sum_i dT[i][j] M[i][j], four lanes per column
     {
       const int j = tid >> 2, part = tid & 3;
@@ -642,77 +688,72 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(BwdTcArgs ta) {
       s += __shfl_xor_sync(0xffffffffu, s, 2);
       if (part == 0) ms.dbc[j] = s;
     }
-    __syncthreads();
-    // tmp = dM M^T  (tmp[i][kk] = sum_{j <= min(i, kk)} dM[i][j] M[kk][j]), 4 x 4 per thread;
-    // dM and M are lower triangular, so the extra j of a tile contribute zeros
-    {
-      const int i0 = (tid >> 4) * 4, k0 = (tid & 15) * 4;
-      const int jmax = (i0 < k0 ? i0 : k0) + 3;
-      float acc[4][4];
+    if (!wait_one(&ms.bar[0], ph, a.status, 410)) { abort = true; break; }
+    tc_fence_after();
+    if (qd < 2) {  // tmp rows i (lanes 0..63) -> bf16 hi + lo tiles, K-major [i][k]
+      const int i = 32 * qd + lane, ch = warp >> 2;
+      float x[16], y[16];
+      tmem_ld16(lanebase + 128 + 32 * ch, x);
+      tmem_ld16(lanebase + 128 + 32 * ch + 16, y);
+      tmem_wait_ld();
 #pragma unroll
-      for (int m = 0; m < 4; ++m)
+      for (int m = 0; m < 4; ++m) {
+        uint32_t hi[4], lo[4];
 #pragma unroll
-        for (int n = 0; n < 4; ++n) acc[m][n] = 0.f;
-      for (int j = 0; j <= jmax; ++j) {
-        float a4[4], b4[4];
-#pragma unroll
-        const float bj = ms.beta[j];  // dM = dT Diag(beta), applied on the fly
-#pragma unroll
-        for (int m = 0; m < 4; ++m) {
-          a4[m] = dTf[(i0 + m) * LDF + j] * bj;
-          b4[m] = Mf[(k0 + m) * LDF + j];
+        for (int e = 0; e < 4; ++e) {
+          const int jj = 8 * m + 2 * e;
+          split_bf16x2(jj < 16 ? x[jj] : y[jj - 16], jj + 1 < 16 ? x[jj + 1] : y[jj + 1 - 16], hi[e], lo[e]);
         }
+        *reinterpret_cast<uint4 *>(sm + G_TH + kmaj_off(i, 32 * ch + 8 * m, 64)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        *reinterpret_cast<uint4 *>(sm + G_TL + kmaj_off(i, 32 * ch + 8 * m, 64)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+      }
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    // dL = -M^T tmp, same three-product split: A = M^T is the M tile read
+    // MN-major (K = i), B = tmp read MN-major (K = i, N = k); negated A
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t id = idesc_bf16(128, 64, true, true) | (1u << 13);
+      const uint32_t a2[3] = {smem_u32(sm + G_MH), smem_u32(sm + G_MH), smem_u32(sm + G_ML)};
+      const uint32_t b2[3] = {smem_u32(sm + G_TH), smem_u32(sm + G_TL), smem_u32(sm + G_TH)};
 #pragma unroll
-        for (int m = 0; m < 4; ++m)
+      for (int p = 0; p < 3; ++p)
 #pragma unroll
-          for (int n = 0; n < 4; ++n) acc[m][n] += a4[m] * b4[n];
+        for (int kk = 0; kk < 4; ++kk)
+          mma_bf16(tmem + 192, sdesc(a2[p] + kk * 2048, 8192, 1024), sdesc(b2[p] + kk * 2048, 8192, 1024), id,
+                   p > 0 || kk > 0);
+      mma_commit(&ms.bar[1]);
+    }
+    if (!wait_one(&ms.bar[1], ph, a.status, 411)) { abort = true; break; }
+    tc_fence_after();
+    // dN = strict_lower(dL) -> fp32 (for the dbeta row part) and
+    // dA = Diag(beta) dN -> bf16 rows 0..63 of the [dA; dA_q] tile
+    if (qd < 2) {
+      const int r = 32 * qd + lane, ch = warp >> 2;
+      float x[16], y[16];
+      tmem_ld16(lanebase + 192 + 32 * ch, x);
+      tmem_ld16(lanebase + 192 + 32 * ch + 16, y);
+      tmem_wait_ld();
+      const float br = ms.beta[r];
+      uint32_t pk[16];
+#pragma unroll
+      for (int jj = 0; jj < 32; jj += 2) {
+        const int k0 = 32 * ch + jj;
+        const float v0 = k0 < r ? (jj < 16 ? x[jj] : y[jj - 16]) : 0.f;
+        const float v1 = k0 + 1 < r ? (jj + 1 < 16 ? x[jj + 1] : y[jj + 1 - 16]) : 0.f;
+        dTf[r * LDF + k0] = v0;
+        dTf[r * LDF + k0 + 1] = v1;
+        pk[jj >> 1] = pack_bf16(br * v0, br * v1);
       }
 #pragma unroll
       for (int m = 0; m < 4; ++m)
-        *reinterpret_cast<float4 *>(tmpf + (i0 + m) * 64 + k0) = make_float4(acc[m][0], acc[m][1], acc[m][2], acc[m][3]);
+        *reinterpret_cast<uint4 *>(sm + G_WN + kmaj_off(r, 32 * ch + 8 * m, 128)) =
+            make_uint4(pk[4 * m], pk[4 * m + 1], pk[4 * m + 2], pk[4 * m + 3]);
     }
     __syncthreads();
-    // dL = -M^T tmp, strict lower -> dN (into dTf; dM is dead), 4 x 4 per thread
-    {
-      const int a0 = (tid >> 4) * 4, k0 = (tid & 15) * 4;
-      float acc[4][4];
-#pragma unroll
-      for (int m = 0; m < 4; ++m)
-#pragma unroll
-        for (int n = 0; n < 4; ++n) acc[m][n] = 0.f;
-      if (k0 <= a0 + 2)
-        for (int i = a0; i < 64; ++i) {  // M[i][a] = 0 for i < a
-          float m4[4];
-#pragma unroll
-          for (int m = 0; m < 4; ++m) m4[m] = Mf[i * LDF + a0 + m];
-          const float4 t4 = *reinterpret_cast<const float4 *>(tmpf + i * 64 + k0);
-          const float tt[4] = {t4.x, t4.y, t4.z, t4.w};
-#pragma unroll
-          for (int m = 0; m < 4; ++m)
-#pragma unroll
-            for (int n = 0; n < 4; ++n) acc[m][n] += m4[m] * tt[n];
-        }
-      __syncthreads();  // every read of dM (dTf) and tmp is done before dN overwrites dTf
-#pragma unroll
-      for (int m = 0; m < 4; ++m)
-#pragma unroll
-        for (int n = 0; n < 4; ++n) {
-          const int aa = a0 + m, kk = k0 + n;
-          dTf[aa * LDF + kk] = kk < aa ? -acc[m][n] : 0.f;
-        }
-    }
-    __syncthreads();
-    // dA = Diag(beta) dN -> bf16 rows 0..63 of the [dA; dA_q] tile; dbeta (row part)
-    {
-      const int r = tid >> 2, j0 = (tid & 3) * 16;
-      const float br = ms.beta[r];
-      uint32_t pk[8];
-#pragma unroll
-      for (int m = 0; m < 8; ++m)
-        pk[m] = pack_bf16(br * dTf[r * LDF + j0 + 2 * m], br * dTf[r * LDF + j0 + 2 * m + 1]);
-      *reinterpret_cast<uint4 *>(sm + G_WN + kmaj_off(r, j0, 128)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-      *reinterpret_cast<uint4 *>(sm + G_WN + kmaj_off(r, j0 + 8, 128)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-    }
+    // dbeta (row part): sum_{j < r} dN[r][j] A[r][j]
     if (fast) {
       if (qd >= 2) {
         const int r = 32 * qd + lane - 64, ch = warp >> 2;
@@ -940,7 +981,7 @@ int num_sms() {
 // these inputs; dS_tiles / dU_tiles: n_chunks * H tiles of 32 KiB / 16 KiB.
 cudaError_t tc_backward(const BwdArgs &b, const unsigned char *recs, unsigned char *dS_tiles,
                         unsigned char *dU_tiles, float *fb, cudaStream_t s) {
-  BwdTcArgs ta;
+  BwdTcArgs ta{};
   ta.b = b;
   ta.recs = recs;
   ta.dS_tiles = dS_tiles;
@@ -959,6 +1000,8 @@ cudaError_t tc_backward(const BwdArgs &b, const unsigned char *recs, unsigned ch
     tc_state_bwd_kernel<<<dim3(b.H, b.map.n_seq), kSbThreads, sm_sb, s>>>(ta);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
+  e = make_row_maps(ta.rm, b.q, b.k, b.v, b.dO, b.g, b.sign, (int64_t)b.B * b.T, b.H);
+  if (e != cudaSuccess) return e;
   {
     ProfScope prof("tc_grad", s);
     tc_grad_kernel<<<num_sms(), kGThreads, sm_g, s>>>(ta);

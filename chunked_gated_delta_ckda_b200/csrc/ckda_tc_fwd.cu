@@ -57,7 +57,7 @@ constexpr uint32_t I_MF = 16640;      // fp32 M [64][65]  (reuses A1/B1 after MM
 constexpr int LDF = 65;
 
 struct IntraMisc {
-  uint64_t mbar1, mbar2, mfin;
+  uint64_t mbar1, mbar2, mfin, mld;
   uint32_t tmem;
   int flag;
   float beta[64];
@@ -66,6 +66,7 @@ struct IntraMisc {
 };
 
 struct TcArgs {
+  RowMaps rm;           // q, k, v, g, sign (intra-chunk kernel)
   FwdArgs f;
   unsigned char *recs;  // (chunk, head) records
   float *fb;            // per-CTA fallback scratch: Gam, k', q' (3 x 64 x 128 fp32)
@@ -73,7 +74,7 @@ struct TcArgs {
   bool write_o;
 };
 
-__global__ void __launch_bounds__(kIntraThreads, 2) tc_intra_kernel(TcArgs ta) {
+__global__ void __launch_bounds__(kIntraThreads, 2) tc_intra_kernel(const __grid_constant__ TcArgs ta) {
   extern __shared__ unsigned char smem_raw[];
   unsigned char *sm = reinterpret_cast<unsigned char *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -81,13 +82,13 @@ __global__ void __launch_bounds__(kIntraThreads, 2) tc_intra_kernel(TcArgs ta) {
   const FwdArgs &a = ta.f;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int H = a.H;
-  const __nv_bfloat16 *q = (const __nv_bfloat16 *)a.q, *k = (const __nv_bfloat16 *)a.k;
-  const __nv_bfloat16 *v = (const __nv_bfloat16 *)a.v, *beta = (const __nv_bfloat16 *)a.beta;
+  const __nv_bfloat16 *beta = (const __nv_bfloat16 *)a.beta;
 
   if (tid == 0) {
     mbar_init(&ms.mbar1, 1);
     mbar_init(&ms.mbar2, 1);
     mbar_init(&ms.mfin, 1);
+    mbar_init(&ms.mld, 1);
     mbar_fence_init();
   }
   if (warp == 0) {
@@ -114,27 +115,32 @@ __global__ void __launch_bounds__(kIntraThreads, 2) tc_intra_kernel(TcArgs ta) {
     a.map.info(cid, seq, tok0, len, jl);
     unsigned char *rec = ta.recs + (size_t)item * REC;
 
-    // ---------------- prep: row-group layout (rows 8w.., channels 4l..) ----------------
-    // V rows are requested first so their latency overlaps the prep loads
-    uint4 vv[4];
-#pragma unroll
-    for (int m = 0; m < 4; ++m) {
-      const int e = tid + kIntraThreads * m, j = e >> 4, cc = e & 15;
-      const int jj = j < len ? j : len - 1;
-      vv[m] = *reinterpret_cast<const uint4 *>(v + ((size_t)(tok0 + jj) * H + h) * D + cc * 8);
-    }
-    Prep P;
-    prep_load(a.g, a.sign, k, q, tok0, len, h, H, warp, lane, P, ms.tot);
-    // V tile (MN-major A operand, K = token j, M = value channel)
-    {
-#pragma unroll
-      for (int m = 0; m < 4; ++m) {
-        const int e = tid + kIntraThreads * m, j = e >> 4, cc = e & 15;
-        *reinterpret_cast<uint4 *>(sm + I_V + mnmaj_off(j, cc * 8, 64)) =
-            j < len ? vv[m] : make_uint4(0, 0, 0, 0);
-      }
+    // ---------------- loads: one TMA box per 64-row tile, one barrier ----------------
+    // q, k staged in the A1 region, g in B1 + KG, sign in T (each consumed by
+    // the prep before those tiles are written); V straight into its operand
+    // tile (MN-major A, K = token j, M = value channel: the box layout).
+    if (tid == 0) {
+      fence_async_smem();  // earlier generic accesses of these regions come first
+      mbar_arrive_expect_tx(&ms.mld, kRowBytesQK + kRowBytesG + kRowBytesSign + 16384);
+      const int t = (int)tok0;
+      tma_rows(sm + I_A1 + kStageQ, &ta.rm.q, 0, h, t, &ms.mld);
+      tma_rows(sm + I_A1 + kStageQ + 8192, &ta.rm.q, 64, h, t, &ms.mld);
+      tma_rows(sm + I_A1 + kStageK, &ta.rm.k, 0, h, t, &ms.mld);
+      tma_rows(sm + I_A1 + kStageK + 8192, &ta.rm.k, 64, h, t, &ms.mld);
+      tma_rows(sm + I_B1, &ta.rm.g, 0, h, t, &ms.mld);
+      tma_rows(sm + I_T, &ta.rm.sign, 0, h, t, &ms.mld);
+      tma_rows(sm + I_V, &ta.rm.v, 0, h, t, &ms.mld);
+      tma_rows(sm + I_V + 8192, &ta.rm.v, 64, h, t, &ms.mld);
     }
     if (tid < 64) ms.beta[tid] = tid < len ? __bfloat162float(beta[(size_t)(tok0 + tid) * H + h]) : 0.f;
+    {
+      const bool ok = mbar_wait(&ms.mld, it & 1, a.status, 100);
+      if (__syncthreads_or(!ok)) { abort = true; break; }
+    }
+    // ---------------- prep: row-group layout (rows 8w.., channels 4l..) ----------------
+    Prep P;
+    prep_load_smem(sm + I_A1, reinterpret_cast<const float *>(sm + I_B1), sm + I_T, len, warp, lane, P, ms.tot);
+    if (len < 64) zero_tail_rows(sm + I_V, 8192, len, tid, kIntraThreads);  // V rows past the chunk
     __syncthreads();
     prep_carry(warp, lane, P, ms.tot);
     int bad = 0;
@@ -613,7 +619,7 @@ size_t tc_record_bytes() { return REC; }
 // reuses records an earlier call wrote for the same inputs.
 cudaError_t tc_forward(const FwdArgs &f, unsigned char *recs, float *fb, bool write_o,
                        float *states_out, cudaStream_t s, bool state_pass, bool intra_pass) {
-  TcArgs ta;
+  TcArgs ta{};
   ta.f = f;
   ta.recs = recs;
   ta.fb = fb;
@@ -627,6 +633,8 @@ cudaError_t tc_forward(const FwdArgs &f, unsigned char *recs, float *fb, bool wr
   e = cudaFuncSetAttribute(tc_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_state);
   if (e != cudaSuccess) return e;
   if (intra_pass) {
+    e = make_row_maps(ta.rm, f.q, f.k, f.v, nullptr, f.g, f.sign, (int64_t)f.B * f.T, f.H);
+    if (e != cudaSuccess) return e;
     ProfScope prof("tc_intra", s);
     tc_intra_kernel<<<tc_intra_ctas(), kIntraThreads, sm_intra, s>>>(ta);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
