@@ -65,6 +65,12 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t phase, DevStat
   }
   return false;
 }
+// The same wait out of line, for kernels that wait at many sites: one copy
+// of the loop keeps their instruction footprint small (the latency-bound
+// state passes keep the inline form).
+static __device__ __noinline__ bool mbar_wait_ool(uint64_t *bar, uint32_t phase, DevStatus *st, uint32_t site) {
+  return mbar_wait(bar, phase, st, site);
+}
 
 // ---------------------------------------------------------------------------
 // bulk async copy global -> shared (1-D, 16-byte aligned, size % 16 == 0)

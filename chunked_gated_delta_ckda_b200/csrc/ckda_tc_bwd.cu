@@ -286,7 +286,7 @@ __global__ void __launch_bounds__(kSbThreads, 1) tc_state_bwd_kernel(BwdTcArgs t
 // ===========================================================================
 // per-chunk gradient kernel
 // ===========================================================================
-constexpr int kGThreads = 256;
+constexpr int kGThreads = 512;  // 16 warps: four per TMEM lane quadrant
 constexpr uint32_t G_A1 = 0;          // [Q~; K~l] K-major 128 x 128
 constexpr uint32_t G_B1 = 32768;      // K~r K-major 64 x 128
 constexpr uint32_t G_KG = 49152;      // KG (== K-major [j][c] 64 rows); later dM M^T parts
@@ -303,6 +303,9 @@ constexpr int LDF = 65;
 constexpr uint32_t G_DMH = G_UV, G_DML = G_UV + 8192;           // dM, K-major [i][j]
 constexpr uint32_t G_MH = G_UV + 16384, G_ML = G_UV + 24576;    // M, K-major [i][a]
 constexpr uint32_t G_TH = G_KG, G_TL = G_KG + 8192;             // dM M^T, K-major [i][k]
+// final epilogue scratch in the idle [U; V] tile: per-quarter sums, sign bits
+constexpr uint32_t G_FSUM = G_UV;               // float [2][4][128]
+constexpr uint32_t G_PBITS = G_UV + 8192;       // uint8 [8][128]
 constexpr uint32_t W_TILE = 16384;              // W^T half of the record's R1 tile
 constexpr uint32_t M_BYTES = 64 * LDF * 4;      // the record's M
 static_assert(M_BYTES == REC - R6, "M is the record's last field");
@@ -311,23 +314,101 @@ struct GMisc {
   uint64_t bar[6], mdu, mds, mfin, mrec, mld;
   uint32_t tmem;
   int pad;
-  float beta[64], dbc[64], dbr[2][64];
+  float beta[64], dbc[64], dbr[4][64];
   PrepTot tot;
-  uint8_t pbits[8][128];
-  float dd[2][128];
+  float dd[4][128];
 };
 
 // Completion of MMAs (or of a copy only MMAs consume): one thread polls the
 // mbarrier, the others wait at the CTA barrier (no spinning issue slots).
 __device__ __forceinline__ bool wait_one(uint64_t *bar, uint32_t phase, DevStatus *st, uint32_t site) {
   bool ok = true;
-  if (threadIdx.x == 0) ok = mbar_wait(bar, phase, st, site);
+  if (threadIdx.x == 0) ok = mbar_wait_ool(bar, phase, st, site);
   return !__syncthreads_or(!ok);
 }
 // Completion of a copy whose data every thread reads: every thread observes it.
 __device__ __forceinline__ bool wait_all(uint64_t *bar, uint32_t phase, DevStatus *st, uint32_t site) {
-  const bool ok = mbar_wait(bar, phase, st, site);
+  const bool ok = mbar_wait_ool(bar, phase, st, site);
   return !__syncthreads_or(!ok);
+}
+
+// Prep in the 16-warp layout: warp w owns chunk rows 8 (w & 7) .. + 7 and
+// key channels 64 (w >> 3) + 2 lane, + 1 (two per lane); the group totals
+// are the same [8][128] arrays as the 8-warp layout's.
+struct Prep2 {
+  float G[8][2];      // chunk-local inclusive cumsum of g (after the carry)
+  uint32_t k2[8];     // raw bf16 k of the two channels
+  uint32_t q2[8];
+  uint32_t pre;       // bit 2*rr+m: sign product of row 8 rg + rr, channel ch0 + m is negative
+  float Gm[2], GC[2];
+  uint32_t pC;        // bit m: chunk sign product of channel ch0 + m is negative
+};
+__device__ __forceinline__ void prep2_load(const unsigned char *sqk, const float *sg, const uint8_t *ss, int len,
+                                           int rg, int ch0, Prep2 &P, PrepTot &tot) {
+  float acc[2] = {0.f, 0.f};
+  uint32_t par = 0, pre = 0;
+#pragma unroll
+  for (int rr = 0; rr < 8; ++rr) {
+    const int r = 8 * rg + rr;
+    const bool valid = r < len;
+    const float2 gv = *reinterpret_cast<const float2 *>(sg + r * D + ch0);
+    const uint32_t sgn = *reinterpret_cast<const uint16_t *>(ss + r * D + ch0);
+    const uint32_t off = kmaj_off(r, ch0, 64);
+    const uint32_t kv = *reinterpret_cast<const uint32_t *>(sqk + kStageK + off);
+    const uint32_t qv = *reinterpret_cast<const uint32_t *>(sqk + kStageQ + off);
+    P.k2[rr] = valid ? kv : 0u;
+    P.q2[rr] = valid ? qv : 0u;
+    const float gg[2] = {gv.x, gv.y};
+#pragma unroll
+    for (int m = 0; m < 2; ++m) {
+      acc[m] += valid ? gg[m] : 0.f;
+      P.G[rr][m] = acc[m];
+      const bool neg = valid && (int8_t)((sgn >> (8 * m)) & 0xffu) < 0;
+      par ^= (neg ? 1u : 0u) << m;
+    }
+    pre |= par << (2 * rr);
+  }
+  P.pre = pre;
+  *reinterpret_cast<float2 *>(&tot.G[rg][ch0]) = make_float2(acc[0], acc[1]);
+  tot.P[rg][ch0] = (uint8_t)(par & 1u);
+  tot.P[rg][ch0 + 1] = (uint8_t)((par >> 1) & 1u);
+}
+__device__ __forceinline__ void prep2_carry(int rg, int ch0, Prep2 &P, const PrepTot &tot) {
+  float cg[2] = {0.f, 0.f}, gm[2] = {0.f, 0.f}, gc[2] = {0.f, 0.f};
+  uint32_t cp = 0, pc = 0;
+#pragma unroll
+  for (int ww = 0; ww < 8; ++ww) {
+    const float2 t = *reinterpret_cast<const float2 *>(&tot.G[ww][ch0]);
+    const float tt[2] = {t.x, t.y};
+#pragma unroll
+    for (int m = 0; m < 2; ++m) {
+      const uint32_t pb = tot.P[ww][ch0 + m];
+      if (ww < rg) { cg[m] += tt[m]; cp ^= pb << m; }
+      if (ww <= 3) gm[m] += tt[m];
+      gc[m] += tt[m];
+      pc ^= pb << m;
+    }
+  }
+#pragma unroll
+  for (int rr = 0; rr < 8; ++rr)
+#pragma unroll
+    for (int m = 0; m < 2; ++m) P.G[rr][m] += cg[m];
+  uint32_t rep = 0;  // replicate the 2-bit carry parity over the 8 rows
+#pragma unroll
+  for (int rr = 0; rr < 8; ++rr) rep |= cp << (2 * rr);
+  P.pre ^= rep;
+#pragma unroll
+  for (int m = 0; m < 2; ++m) { P.Gm[m] = gm[m]; P.GC[m] = gc[m]; }
+  P.pC = pc;
+}
+__device__ __forceinline__ float prep2_p(const Prep2 &P, int rr, int m) {
+  return ((P.pre >> (2 * rr + m)) & 1u) ? -1.f : 1.f;
+}
+__device__ __forceinline__ float prep2_k(const Prep2 &P, int rr, int m) {
+  return m ? bf_hi(P.k2[rr]) : bf_lo(P.k2[rr]);
+}
+__device__ __forceinline__ float prep2_q(const Prep2 &P, int rr, int m) {
+  return m ? bf_hi(P.q2[rr]) : bf_lo(P.q2[rr]);
 }
 
 __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_constant__ BwdTcArgs ta) {
@@ -364,13 +445,15 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
   const uint32_t sSC = smem_u32(sm + G_SC), sWN = smem_u32(sm + G_WN);
   float *dTf = reinterpret_cast<float *>(sm + G_DT);
   float *Mf = reinterpret_cast<float *>(sm + G_MF);
-  float *gcps = reinterpret_cast<float *>(sm + G_UV);         // [2][128], final epilogue only
-  float *acc1s = gcps + 256;                                  // [2][128]
   float *fb = ta.fb + (size_t)blockIdx.x * 3 * 64 * D;
 
-  const int c = tid & 127, hf = tid >> 7;
-  const int qd = warp & 3;  // TMEM lane quadrant of this warp
+  // TMEM-facing mapping: lane quadrant qd of the accumulator rows, column
+  // quarter cq; c = 32 qd + lane is the accumulator row (channel) of this thread
+  const int qd = warp & 3, cq = warp >> 2;
+  const int c = tid & 127;
   const uint32_t lanebase = tmem + ((uint32_t)(32 * qd) << 16);
+  // prep mapping: row group rg, channels ch0, ch0 + 1
+  const int rg = warp & 7, ch0 = 64 * (warp >> 3) + 2 * lane;
   const int nitems = a.map.n_chunks() * H;
   uint32_t it = 0;
   bool abort = false;
@@ -396,15 +479,9 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
       mbar_arrive_expect_tx(&ms.mrec, W_TILE + M_BYTES);
       bulk_g2s(sm + G_WN, rec + R1, W_TILE, &ms.mrec);
       bulk_g2s(sm + G_MF, rec + R6, M_BYTES, &ms.mrec);
-    }
-    // the start state S_c (fp32) through registers; the row tensors by TMA:
-    // q, k staged in A1, g in B1 + KG, sign in TT (the prep consumes them
-    // before those tiles are written), V into rows 64.. of [U; V] and dO into
-    // rows 0..63 of [dO; dU] (K-major SW128 boxes)
-    float4 x[16];
-#pragma unroll
-    for (int m = 0; m < 16; ++m) x[m] = *reinterpret_cast<const float4 *>(Sc + (size_t)(warp + 8 * m) * D + 4 * lane);
-    if (tid == 0) {
+      // the row tensors: q, k staged in A1, g in B1 + KG, sign in TT (the prep
+      // consumes them before those tiles are written), V into rows 64.. of
+      // [U; V] and dO into rows 0..63 of [dO; dU] (K-major SW128 boxes)
       mbar_arrive_expect_tx(&ms.mld, kRowBytesQK + kRowBytesG + kRowBytesSign + 2 * 16384);
       const int t = (int)tok0;
       tma_rows(sm + G_A1 + kStageQ, &ta.rm.q, 0, h, t, &ms.mld);
@@ -418,66 +495,72 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
       tma_rows(sm + G_OU, &ta.rm.dO, 0, h, t, &ms.mld);
       tma_rows(sm + G_OU + 16384, &ta.rm.dO, 64, h, t, &ms.mld);
     }
-    if (tid < 64) ms.beta[tid] = tid < len ? __bfloat162float(beta[(size_t)(tok0 + tid) * H + h]) : 0.f;
+    // the start state S_c (fp32) through registers -> bf16 K-major [c][v]
+    {
+      float4 x[8];
 #pragma unroll
-    for (int m = 0; m < 16; ++m)  // S_c fp32 rows -> bf16 K-major [c][v]
-      *reinterpret_cast<uint2 *>(sm + G_SC + kmaj_off(warp + 8 * m, 4 * lane, 128)) =
-          make_uint2(pack_bf16(x[m].x, x[m].y), pack_bf16(x[m].z, x[m].w));
+      for (int m = 0; m < 8; ++m) x[m] = *reinterpret_cast<const float4 *>(Sc + (size_t)(warp + 16 * m) * D + 4 * lane);
+      if (tid < 64) ms.beta[tid] = tid < len ? __bfloat162float(beta[(size_t)(tok0 + tid) * H + h]) : 0.f;
+#pragma unroll
+      for (int m = 0; m < 8; ++m)
+        *reinterpret_cast<uint2 *>(sm + G_SC + kmaj_off(warp + 16 * m, 4 * lane, 128)) =
+            make_uint2(pack_bf16(x[m].x, x[m].y), pack_bf16(x[m].z, x[m].w));
+    }
     if (!wait_all(&ms.mld, ph, a.status, 400)) { abort = true; break; }
-    Prep P;  // row-group layout: rows 8 warp .., channels 4 lane ..
-    prep_load_smem(sm + G_A1, reinterpret_cast<const float *>(sm + G_B1), sm + G_TT, len, warp, lane, P, ms.tot);
+    Prep2 P;
+    prep2_load(sm + G_A1, reinterpret_cast<const float *>(sm + G_B1), sm + G_TT, len, rg, ch0, P, ms.tot);
     if (len < 64) {  // V and dO rows past the chunk
       zero_tail_rows(sm + G_UV + 8192, 16384, len, tid, kGThreads);
       zero_tail_rows(sm + G_OU, 16384, len, tid, kGThreads);
     }
     __syncthreads();
-    prep_carry(warp, lane, P, ms.tot);
+    prep2_carry(rg, ch0, P, ms.tot);
     int bad = 0;
 #pragma unroll
     for (int rr = 0; rr < 8; ++rr)
 #pragma unroll
-      for (int m = 0; m < 4; ++m)
+      for (int m = 0; m < 2; ++m)
         if (!(fabsf(P.G[rr][m] - P.Gm[m]) <= kTau)) bad = 1;
     const bool fast = !__syncthreads_or(bad);
 
     // ---------------- operand tiles ----------------
     if (fast) {
+      const float e0 = fast_exp(P.Gm[0]), e1 = fast_exp(P.Gm[1]);
 #pragma unroll
       for (int rr = 0; rr < 8; ++rr) {
-        const int r = 8 * warp + rr;
-        float ql[4], kl[4], kr[4];
+        const int r = 8 * rg + rr;
+        float ql[2], kl[2], kr[2];
 #pragma unroll
-        for (int m = 0; m < 4; ++m) {
-          const float p = prep_p(P, rr, m);
-          const float kp = p * prep_k(P, rr, m), qp = p * prep_q(P, rr, m);
+        for (int m = 0; m < 2; ++m) {
+          const float p = prep2_p(P, rr, m);
+          const float kp = p * prep2_k(P, rr, m), qp = p * prep2_q(P, rr, m);
           const float el = fast_exp(P.G[rr][m] - P.Gm[m]), er = rcp_approx(el);
           ql[m] = qp * el;
           kl[m] = kp * el;
           kr[m] = kp * er;
         }
-        const float e0 = fast_exp(P.Gm[0]), e1 = fast_exp(P.Gm[1]), e2 = fast_exp(P.Gm[2]), e3 = fast_exp(P.Gm[3]);
-        st_bf16x4(sm + G_A1, kmaj_off(r, 4 * lane, 128), ql[0], ql[1], ql[2], ql[3]);
-        st_bf16x4(sm + G_A1, kmaj_off(64 + r, 4 * lane, 128), kl[0], kl[1], kl[2], kl[3]);
-        st_bf16x4(sm + G_B1, kmaj_off(r, 4 * lane, 64), kr[0], kr[1], kr[2], kr[3]);
-        st_bf16x4(sm + G_KG, mnmaj_off(r, 4 * lane, 64), kl[0] * e0, kl[1] * e1, kl[2] * e2, kl[3] * e3);
+        *reinterpret_cast<uint32_t *>(sm + G_A1 + kmaj_off(r, ch0, 128)) = pack_bf16(ql[0], ql[1]);
+        *reinterpret_cast<uint32_t *>(sm + G_A1 + kmaj_off(64 + r, ch0, 128)) = pack_bf16(kl[0], kl[1]);
+        *reinterpret_cast<uint32_t *>(sm + G_B1 + kmaj_off(r, ch0, 64)) = pack_bf16(kr[0], kr[1]);
+        *reinterpret_cast<uint32_t *>(sm + G_KG + mnmaj_off(r, ch0, 64)) = pack_bf16(kl[0] * e0, kl[1] * e1);
       }
     } else {
-#pragma unroll
+#pragma unroll 1
       for (int rr = 0; rr < 8; ++rr) {
-        const int r = 8 * warp + rr;
-        float kp4[4], qp4[4], g4[4], kg4[4];
+        const int r = 8 * rg + rr;
+        float kp2[2], qp2[2], g2[2];
 #pragma unroll
-        for (int m = 0; m < 4; ++m) {
-          const float p = prep_p(P, rr, m);
-          kp4[m] = p * prep_k(P, rr, m);
-          qp4[m] = p * prep_q(P, rr, m);
-          g4[m] = P.G[rr][m];
-          kg4[m] = kp4[m] * fast_exp(g4[m]);
+        for (int m = 0; m < 2; ++m) {
+          const float p = prep2_p(P, rr, m);
+          kp2[m] = p * prep2_k(P, rr, m);
+          qp2[m] = p * prep2_q(P, rr, m);
+          g2[m] = P.G[rr][m];
         }
-        *reinterpret_cast<float4 *>(fb + r * D + 4 * lane) = make_float4(g4[0], g4[1], g4[2], g4[3]);
-        *reinterpret_cast<float4 *>(fb + 64 * D + r * D + 4 * lane) = make_float4(kp4[0], kp4[1], kp4[2], kp4[3]);
-        *reinterpret_cast<float4 *>(fb + 128 * D + r * D + 4 * lane) = make_float4(qp4[0], qp4[1], qp4[2], qp4[3]);
-        st_bf16x4(sm + G_KG, mnmaj_off(r, 4 * lane, 64), kg4[0], kg4[1], kg4[2], kg4[3]);
+        *reinterpret_cast<float2 *>(fb + r * D + ch0) = make_float2(g2[0], g2[1]);
+        *reinterpret_cast<float2 *>(fb + 64 * D + r * D + ch0) = make_float2(kp2[0], kp2[1]);
+        *reinterpret_cast<float2 *>(fb + 128 * D + r * D + ch0) = make_float2(qp2[0], qp2[1]);
+        *reinterpret_cast<uint32_t *>(sm + G_KG + mnmaj_off(r, ch0, 64)) =
+            pack_bf16(kp2[0] * fast_exp(g2[0]), kp2[1] * fast_exp(g2[1]));
       }
     }
     fence_async_smem();
@@ -486,14 +569,13 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
     // ---------------- T = M Diag(beta) (M from the forward's record) ----------------
     if (!wait_all(&ms.mrec, ph, a.status, 401)) { abort = true; break; }
     {
-      const int r = tid >> 2, j0 = (tid & 3) * 16;
-      uint32_t pk[8];
+      const int r = tid >> 3, j0 = (tid & 7) * 8;
+      uint32_t pk[4];
 #pragma unroll
-      for (int m = 0; m < 8; ++m)
+      for (int m = 0; m < 4; ++m)
         pk[m] = pack_bf16(Mf[r * LDF + j0 + 2 * m] * ms.beta[j0 + 2 * m],
                           Mf[r * LDF + j0 + 2 * m + 1] * ms.beta[j0 + 2 * m + 1]);
       *reinterpret_cast<uint4 *>(sm + G_TT + kmaj_off(r, j0, 64)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-      *reinterpret_cast<uint4 *>(sm + G_TT + kmaj_off(r, j0 + 8, 64)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
     }
     fence_async_smem();
     __syncthreads();
@@ -504,18 +586,18 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
       tc_fence_after();
       if (fast) {
         const uint32_t id = idesc_bf16(128, 64, false, false);
-#pragma unroll
+#pragma unroll 1
         for (int kk = 0; kk < 8; ++kk)
           mma_bf16(tmem, sdesc(sA1 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
                    sdesc(sB1 + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), id, kk > 0);
       }
       const uint32_t idu = idesc_bf16(128, 64, true, false);
-#pragma unroll
+#pragma unroll 1
       for (int kk = 0; kk < 4; ++kk)
         mma_bf16(tmem + 128, sdesc(sUV + 8192 + kk * 2048, 16384, 1024), sdesc(sTT + kk * 32, 16, 1024), idu,
                  kk > 0);
       const uint32_t idw = idesc_bf16(128, 64, true, true) | (1u << 13);  // negate A: subtract
-#pragma unroll
+#pragma unroll 1
       for (int kk = 0; kk < 8; ++kk)
         mma_bf16(tmem + 128, sdesc(sSC + kk * 2048, 16384, 1024), sdesc(sWN + kk * 2048, 16384, 1024), idw,
                  true);
@@ -527,30 +609,26 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
       mbar_arrive_expect_tx(&ms.mds, DS_TILE);
       bulk_g2s(sm + G_WN, gdS, DS_TILE, &ms.mds);
     }
-    {  // U rows s (K-major [s][v]) of the [U; V] tile
-      const int ch = warp >> 2;
+    {  // U rows s (K-major [s][v]) of the [U; V] tile: lane = v, columns 16 cq ..
+      float u[16];
+      tmem_ld16(lanebase + 128 + 16 * cq, u);
+      tmem_wait_ld();
 #pragma unroll
-      for (int h16 = 0; h16 < 2; ++h16) {
-        float u[16];
-        tmem_ld16(lanebase + 128 + 32 * ch + 16 * h16, u);
-        tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 16; ++i) st_bf16(sm + G_UV, kmaj_off(32 * ch + 16 * h16 + i, c, 128), u[i]);
-      }
+      for (int i = 0; i < 16; ++i) st_bf16(sm + G_UV, kmaj_off(16 * cq + i, c, 128), u[i]);
     }
     // dd partial: sum over v of S_c[c][v] * dS1[c][v] (dS1 arrives meanwhile)
     if (!wait_all(&ms.mds, ph, a.status, 404)) { abort = true; break; }
     {
       float s = 0.f;
-      for (int vv = 64 * hf; vv < 64 * hf + 64; vv += 8) {
+#pragma unroll
+      for (int vv = 32 * cq; vv < 32 * cq + 32; vv += 8) {
         const uint4 xa = *reinterpret_cast<const uint4 *>(sm + G_SC + kmaj_off(c, vv, 128));
         const uint4 xb = *reinterpret_cast<const uint4 *>(sm + G_WN + kmaj_off(c, vv, 128));
-        const __nv_bfloat16 *pa = reinterpret_cast<const __nv_bfloat16 *>(&xa);
-        const __nv_bfloat16 *pb = reinterpret_cast<const __nv_bfloat16 *>(&xb);
+        const uint32_t wa[4] = {xa.x, xa.y, xa.z, xa.w}, wb[4] = {xb.x, xb.y, xb.z, xb.w};
 #pragma unroll
-        for (int m = 0; m < 8; ++m) s += __bfloat162float(pa[m]) * __bfloat162float(pb[m]);
+        for (int m = 0; m < 4; ++m) s += bf_lo(wa[m]) * bf_lo(wb[m]) + bf_hi(wa[m]) * bf_hi(wb[m]);
       }
-      ms.dd[hf][c] = s;
+      ms.dd[cq][c] = s;
     }
     if (!wait_one(&ms.mdu, ph, a.status, 405)) { abort = true; break; }
     fence_async_smem();
@@ -562,7 +640,7 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
       tc_fence_after();
       const uint32_t id1 = idesc_bf16(128, 128, false, false);
       const uint32_t id2 = idesc_bf16(128, 64, false, false);
-#pragma unroll
+#pragma unroll 1
       for (int kk = 0; kk < 8; ++kk) {
         const uint32_t ko = (kk >> 2) * 16384 + (kk & 3) * 32;
         mma_bf16(tmem + 256, sdesc(sSC + ko, 16, 1024), sdesc(sOU + ko, 16, 1024), id1, kk > 0);
@@ -573,15 +651,11 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
     if (!wait_one(&ms.bar[3], ph, a.status, 406)) { abort = true; break; }
     tc_fence_after();
     {  // dW = -dU S_c^T -> rows 64..127 of the S_c tile (K-major [i][c]); S_c is dead
-      const int ch = warp >> 2;
+      float w[16];
+      tmem_ld16(lanebase + 320 + 16 * cq, w);
+      tmem_wait_ld();
 #pragma unroll
-      for (int h16 = 0; h16 < 2; ++h16) {
-        float w[16];
-        tmem_ld16(lanebase + 320 + 32 * ch + 16 * h16, w);
-        tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 16; ++i) st_bf16(sm + G_SC, kmaj_off(64 + 32 * ch + 16 * h16 + i, c, 128), -w[i]);
-      }
+      for (int i = 0; i < 16; ++i) st_bf16(sm + G_SC, kmaj_off(64 + 16 * cq + i, c, 128), -w[i]);
     }
     fence_async_smem();
     tc_fence_before();
@@ -592,12 +666,12 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
       tc_fence_after();
       const uint32_t id1 = idesc_bf16(128, 128, false, false);
       const uint32_t id2 = idesc_bf16(128, 64, false, false);
-#pragma unroll
+#pragma unroll 1
       for (int kk = 0; kk < 8; ++kk) {
         const uint32_t ko = (kk >> 2) * 16384 + (kk & 3) * 32;
         mma_bf16(tmem + 128, sdesc(sOU + ko, 16, 1024), sdesc(sUV + ko, 16, 1024), id1, kk > 0);
       }
-#pragma unroll
+#pragma unroll 1
       for (int kk = 0; kk < 8; ++kk)
         mma_bf16(tmem + 192, sdesc(sSC + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
                  sdesc(sKG + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), id2, true);
@@ -606,30 +680,24 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
     if (!wait_one(&ms.bar[4], ph, a.status, 407)) { abort = true; break; }
     tc_fence_after();
     {
-      const int ch = warp >> 2;
-      const int L = 32 * qd + lane;
-      float x[16], y[16];
-      if (L < 64) {  // dA_q rows -> bf16 rows 64..127 of the [dA; dA_q] tile
-        tmem_ld16(lanebase + 128 + 32 * ch, x);
-        tmem_ld16(lanebase + 128 + 32 * ch + 16, y);
+      float x[16];
+      if (qd < 2) {  // dA_q rows -> bf16 rows 64..127 of the [dA; dA_q] tile; M rows as hi / lo
+        const int r = c;
+        tmem_ld16(lanebase + 128 + 16 * cq, x);
         tmem_wait_ld();
-        const int r = L;
-        uint32_t pk[16];
+        uint32_t pk[8];
 #pragma unroll
-        for (int jj = 0; jj < 16; ++jj) {
-          const int s0 = 32 * ch + 2 * jj;
-          const float v0 = jj < 8 ? x[2 * jj] : y[2 * jj - 16];
-          const float v1 = jj < 8 ? x[2 * jj + 1] : y[2 * jj + 1 - 16];
-          pk[jj] = pack_bf16(s0 <= r ? v0 : 0.f, s0 + 1 <= r ? v1 : 0.f);
+        for (int jj = 0; jj < 8; ++jj) {
+          const int s0 = 16 * cq + 2 * jj;
+          pk[jj] = pack_bf16(s0 <= r ? x[2 * jj] : 0.f, s0 + 1 <= r ? x[2 * jj + 1] : 0.f);
         }
 #pragma unroll
-        for (int m = 0; m < 4; ++m)
-          *reinterpret_cast<uint4 *>(sm + G_WN + kmaj_off(64 + r, 32 * ch + 8 * m, 128)) =
+        for (int m = 0; m < 2; ++m)
+          *reinterpret_cast<uint4 *>(sm + G_WN + kmaj_off(64 + r, 16 * cq + 8 * m, 128)) =
               make_uint4(pk[4 * m], pk[4 * m + 1], pk[4 * m + 2], pk[4 * m + 3]);
-        // row r of M as bf16 hi + lo parts (K-major [i][a]) for the products below
 #pragma unroll
-        for (int m = 0; m < 4; ++m) {
-          const int a0 = 32 * ch + 8 * m;
+        for (int m = 0; m < 2; ++m) {
+          const int a0 = 16 * cq + 8 * m;
           uint32_t hi[4], lo[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) split_bf16x2(Mf[r * LDF + a0 + 2 * e], Mf[r * LDF + a0 + 2 * e + 1], hi[e], lo[e]);
@@ -637,25 +705,24 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
           *reinterpret_cast<uint4 *>(sm + G_ML + kmaj_off(r, a0, 64)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
         }
       } else {  // dT rows (masked j <= i) -> fp32, and dM = dT Diag(beta) as bf16 hi + lo parts
-        tmem_ld16(lanebase + 192 + 32 * ch, x);
-        tmem_ld16(lanebase + 192 + 32 * ch + 16, y);
+        const int i = c - 64;
+        tmem_ld16(lanebase + 192 + 16 * cq, x);
         tmem_wait_ld();
-        const int i = L - 64;
-        float dm[32];
+        float dm[16];
 #pragma unroll
-        for (int jj = 0; jj < 32; ++jj) {
-          const int j = 32 * ch + jj;
-          const float val = j <= i ? (jj < 16 ? x[jj] : y[jj - 16]) : 0.f;
+        for (int jj = 0; jj < 16; ++jj) {
+          const int j = 16 * cq + jj;
+          const float val = j <= i ? x[jj] : 0.f;
           dTf[i * LDF + j] = val;
           dm[jj] = val * ms.beta[j];
         }
 #pragma unroll
-        for (int m = 0; m < 4; ++m) {
+        for (int m = 0; m < 2; ++m) {
           uint32_t hi[4], lo[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) split_bf16x2(dm[8 * m + 2 * e], dm[8 * m + 2 * e + 1], hi[e], lo[e]);
-          *reinterpret_cast<uint4 *>(sm + G_DMH + kmaj_off(i, 32 * ch + 8 * m, 64)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-          *reinterpret_cast<uint4 *>(sm + G_DML + kmaj_off(i, 32 * ch + 8 * m, 64)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+          *reinterpret_cast<uint4 *>(sm + G_DMH + kmaj_off(i, 16 * cq + 8 * m, 64)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+          *reinterpret_cast<uint4 *>(sm + G_DML + kmaj_off(i, 16 * cq + 8 * m, 64)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
         }
       }
     }
@@ -669,43 +736,39 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
     if (tid == 0) {
       tc_fence_after();
       const uint32_t id = idesc_bf16(128, 64, false, false);
-      const uint32_t a2[3] = {smem_u32(sm + G_DMH), smem_u32(sm + G_DMH), smem_u32(sm + G_DML)};
-      const uint32_t b2[3] = {smem_u32(sm + G_MH), smem_u32(sm + G_ML), smem_u32(sm + G_MH)};
-#pragma unroll
-      for (int p = 0; p < 3; ++p)
-#pragma unroll
+#pragma unroll 1
+      for (int p = 0; p < 3; ++p) {
+        const uint32_t pa = smem_u32(sm + (p == 2 ? G_DML : G_DMH)), pb = smem_u32(sm + (p == 1 ? G_ML : G_MH));
+#pragma unroll 1
         for (int kk = 0; kk < 4; ++kk)
-          mma_bf16(tmem + 128, sdesc(a2[p] + kk * 32, 16, 1024), sdesc(b2[p] + kk * 32, 16, 1024), id,
-                   p > 0 || kk > 0);
+          mma_bf16(tmem + 128, sdesc(pa + kk * 32, 16, 1024), sdesc(pb + kk * 32, 16, 1024), id, p > 0 || kk > 0);
+      }
       mma_commit(&ms.bar[0]);
     }
-    // dbeta (column part): sum_i dT[i][j] M[i][j], four lanes per column
+    // dbeta (column part): sum_i dT[i][j] M[i][j], eight lanes per column
     {
-      const int j = tid >> 2, part = tid & 3;
+      const int j = tid >> 3, part = tid & 7;
       float s = 0.f;
-      for (int i = j + part; i < 64; i += 4) s += dTf[i * LDF + j] * Mf[i * LDF + j];
+      for (int i = j + part; i < 64; i += 8) s += dTf[i * LDF + j] * Mf[i * LDF + j];
       s += __shfl_xor_sync(0xffffffffu, s, 1);
       s += __shfl_xor_sync(0xffffffffu, s, 2);
+      s += __shfl_xor_sync(0xffffffffu, s, 4);
       if (part == 0) ms.dbc[j] = s;
     }
     if (!wait_one(&ms.bar[0], ph, a.status, 410)) { abort = true; break; }
     tc_fence_after();
     if (qd < 2) {  // tmp rows i (lanes 0..63) -> bf16 hi + lo tiles, K-major [i][k]
-      const int i = 32 * qd + lane, ch = warp >> 2;
-      float x[16], y[16];
-      tmem_ld16(lanebase + 128 + 32 * ch, x);
-      tmem_ld16(lanebase + 128 + 32 * ch + 16, y);
+      const int i = c;
+      float x[16];
+      tmem_ld16(lanebase + 128 + 16 * cq, x);
       tmem_wait_ld();
 #pragma unroll
-      for (int m = 0; m < 4; ++m) {
+      for (int m = 0; m < 2; ++m) {
         uint32_t hi[4], lo[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int jj = 8 * m + 2 * e;
-          split_bf16x2(jj < 16 ? x[jj] : y[jj - 16], jj + 1 < 16 ? x[jj + 1] : y[jj + 1 - 16], hi[e], lo[e]);
-        }
-        *reinterpret_cast<uint4 *>(sm + G_TH + kmaj_off(i, 32 * ch + 8 * m, 64)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-        *reinterpret_cast<uint4 *>(sm + G_TL + kmaj_off(i, 32 * ch + 8 * m, 64)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        for (int e = 0; e < 4; ++e) split_bf16x2(x[8 * m + 2 * e], x[8 * m + 2 * e + 1], hi[e], lo[e]);
+        *reinterpret_cast<uint4 *>(sm + G_TH + kmaj_off(i, 16 * cq + 8 * m, 64)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        *reinterpret_cast<uint4 *>(sm + G_TL + kmaj_off(i, 16 * cq + 8 * m, 64)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
       }
     }
     fence_async_smem();
@@ -716,14 +779,14 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
     if (tid == 0) {
       tc_fence_after();
       const uint32_t id = idesc_bf16(128, 64, true, true) | (1u << 13);
-      const uint32_t a2[3] = {smem_u32(sm + G_MH), smem_u32(sm + G_MH), smem_u32(sm + G_ML)};
-      const uint32_t b2[3] = {smem_u32(sm + G_TH), smem_u32(sm + G_TL), smem_u32(sm + G_TH)};
-#pragma unroll
-      for (int p = 0; p < 3; ++p)
-#pragma unroll
+#pragma unroll 1
+      for (int p = 0; p < 3; ++p) {
+        const uint32_t pa = smem_u32(sm + (p == 2 ? G_ML : G_MH)), pb = smem_u32(sm + (p == 1 ? G_TL : G_TH));
+#pragma unroll 1
         for (int kk = 0; kk < 4; ++kk)
-          mma_bf16(tmem + 192, sdesc(a2[p] + kk * 2048, 8192, 1024), sdesc(b2[p] + kk * 2048, 8192, 1024), id,
+          mma_bf16(tmem + 192, sdesc(pa + kk * 2048, 8192, 1024), sdesc(pb + kk * 2048, 8192, 1024), id,
                    p > 0 || kk > 0);
+      }
       mma_commit(&ms.bar[1]);
     }
     if (!wait_one(&ms.bar[1], ph, a.status, 411)) { abort = true; break; }
@@ -731,58 +794,54 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
     // dN = strict_lower(dL) -> fp32 (for the dbeta row part) and
     // dA = Diag(beta) dN -> bf16 rows 0..63 of the [dA; dA_q] tile
     if (qd < 2) {
-      const int r = 32 * qd + lane, ch = warp >> 2;
-      float x[16], y[16];
-      tmem_ld16(lanebase + 192 + 32 * ch, x);
-      tmem_ld16(lanebase + 192 + 32 * ch + 16, y);
+      const int r = c;
+      float x[16];
+      tmem_ld16(lanebase + 192 + 16 * cq, x);
       tmem_wait_ld();
       const float br = ms.beta[r];
-      uint32_t pk[16];
+      uint32_t pk[8];
 #pragma unroll
-      for (int jj = 0; jj < 32; jj += 2) {
-        const int k0 = 32 * ch + jj;
-        const float v0 = k0 < r ? (jj < 16 ? x[jj] : y[jj - 16]) : 0.f;
-        const float v1 = k0 + 1 < r ? (jj + 1 < 16 ? x[jj + 1] : y[jj + 1 - 16]) : 0.f;
-        dTf[r * LDF + k0] = v0;
+      for (int jj = 0; jj < 16; jj += 2) {
+        const int k0 = 16 * cq + jj;
+        const float v0 = k0 < r ? x[jj] : 0.f;
+        const float v1 = k0 + 1 < r ? x[jj + 1] : 0.f;
+        dTf[r * LDF + k0] = v0;  // row stride 65: scalar stores
         dTf[r * LDF + k0 + 1] = v1;
         pk[jj >> 1] = pack_bf16(br * v0, br * v1);
       }
 #pragma unroll
-      for (int m = 0; m < 4; ++m)
-        *reinterpret_cast<uint4 *>(sm + G_WN + kmaj_off(r, 32 * ch + 8 * m, 128)) =
+      for (int m = 0; m < 2; ++m)
+        *reinterpret_cast<uint4 *>(sm + G_WN + kmaj_off(r, 16 * cq + 8 * m, 128)) =
             make_uint4(pk[4 * m], pk[4 * m + 1], pk[4 * m + 2], pk[4 * m + 3]);
     }
     __syncthreads();
     // dbeta (row part): sum_{j < r} dN[r][j] A[r][j]
     if (fast) {
       if (qd >= 2) {
-        const int r = 32 * qd + lane - 64, ch = warp >> 2;
-        float x[16], y[16];
-        tmem_ld16(lanebase + 32 * ch, x);
-        tmem_ld16(lanebase + 32 * ch + 16, y);
+        const int r = c - 64;
+        float x[16];
+        tmem_ld16(lanebase + 16 * cq, x);
         tmem_wait_ld();
         float s = 0.f;
 #pragma unroll
-        for (int jj = 0; jj < 32; ++jj) {
-          const int j = 32 * ch + jj;
-          if (j < r) s += dTf[r * LDF + j] * (jj < 16 ? x[jj] : y[jj - 16]);
+        for (int jj = 0; jj < 16; ++jj) {
+          const int j = 16 * cq + jj;
+          if (j < r) s += dTf[r * LDF + j] * x[jj];
         }
-        ms.dbr[ch][r] = s;
+        ms.dbr[cq][r] = s;
       }
-    } else {
+    } else if (tid < 256) {
       // exact path: recompute the needed A entries from the fallback scratch
-      if (tid < 128) {
-        const int r = tid & 63, ch = tid >> 6;
-        float s = 0.f;
-        for (int j = 32 * ch; j < 32 * ch + 32; ++j) {
-          if (j >= r) break;
-          float aa = 0.f;
-          for (int cc = 0; cc < D; ++cc)
-            aa += fb[64 * D + r * D + cc] * fb[64 * D + j * D + cc] * expf(fb[r * D + cc] - fb[j * D + cc]);
-          s += dTf[r * LDF + j] * aa;
-        }
-        ms.dbr[ch][r] = s;
+      const int r = tid & 63, qq = tid >> 6;
+      float s = 0.f;
+      for (int j = 16 * qq; j < 16 * qq + 16; ++j) {
+        if (j >= r) break;
+        float aa = 0.f;
+        for (int cc = 0; cc < D; ++cc)
+          aa += fb[64 * D + r * D + cc] * fb[64 * D + j * D + cc] * expf(fb[r * D + cc] - fb[j * D + cc]);
+        s += dTf[r * LDF + j] * aa;
       }
+      ms.dbr[qq][r] = s;
     }
     fence_async_smem();
     tc_fence_before();
@@ -792,7 +851,7 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
     if (tid == 0) {
       tc_fence_after();
       const uint32_t idT = idesc_bf16(128, 64, true, true);
-#pragma unroll
+#pragma unroll 1
       for (int kk = 0; kk < 4; ++kk) {
         const uint64_t bd = sdesc(sTT + kk * 2048, 8192, 1024);
         mma_bf16(tmem + 448, sdesc(sOU + 8192 + kk * 2048, 16384, 1024), bd, idT, kk > 0);
@@ -800,15 +859,15 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
       }
       if (fast) {
         const uint32_t idX = idesc_bf16(128, 128, true, false);
-#pragma unroll
+#pragma unroll 1
         for (int kk = 0; kk < 4; ++kk)
           mma_bf16(tmem + 128, sdesc(sB1 + kk * 2048, 8192, 1024), sdesc(sWN + kk * 32, 16, 1024), idX, kk > 0);
         const uint32_t idY = idesc_bf16(128, 64, true, true);
-#pragma unroll
+#pragma unroll 1
         for (int kk = 0; kk < 4; ++kk)
           mma_bf16(tmem + 320, sdesc(sA1 + 8192 + kk * 2048, 16384, 1024), sdesc(sWN + kk * 2048, 8192, 1024),
                    idY, kk > 0);
-#pragma unroll
+#pragma unroll 1
         for (int kk = 0; kk < 4; ++kk)
           mma_bf16(tmem + 320, sdesc(sA1 + kk * 2048, 16384, 1024), sdesc(sWN + 8192 + kk * 2048, 8192, 1024),
                    idY, true);
@@ -817,37 +876,33 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
     }
     if (!fast) {
       // exact pair terms into the TMEM columns the fast path fills:
-      // X1 (128 + r), X2 (192 + r), Y1 (320 + r) of lane c
+      // X1 (128 + r), X2 (192 + r), Y1 (320 + r) of lane c, rows 16 cq ..
       const float *Gc = fb, *kpc = fb + 64 * D, *qpc = fb + 128 * D;
-
       auto dAv = [&](int r, int s) {  // dA (rows 0..63) / dA_q (rows 64..127) from the bf16 tile
         return __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(sm + G_WN + kmaj_off(r, s, 128)));
       };
-
-      for (int b16 = 0; b16 < 2; ++b16) {
-        float x1[16], x2[16], y1[16];
-        for (int i = 0; i < 16; ++i) {
-          const int r = 32 * hf + 16 * b16 + i;
-          const float gr = Gc[r * D + c];
-          float a1 = 0.f, a2 = 0.f, b1 = 0.f;
-          for (int s = 0; s <= r; ++s) {
-            const float e = expf(gr - Gc[s * D + c]) * kpc[s * D + c];
-            a1 += dAv(r, s) * e;
-            a2 += dAv(64 + r, s) * e;
-          }
-          for (int t = r; t < 64; ++t) {
-            const float e = expf(Gc[t * D + c] - gr);
-            b1 += (dAv(t, r) * kpc[t * D + c] + dAv(64 + t, r) * qpc[t * D + c]) * e;
-          }
-          x1[i] = a1;
-          x2[i] = a2;
-          y1[i] = b1;
+      float x1[16], x2[16], y1[16];
+#pragma unroll 1
+      for (int i = 0; i < 16; ++i) {
+        const int r = 16 * cq + i;
+        const float gr = Gc[r * D + c];
+        float a1 = 0.f, a2 = 0.f, b1 = 0.f;
+        for (int s = 0; s <= r; ++s) {
+          const float e = expf(gr - Gc[s * D + c]) * kpc[s * D + c];
+          a1 += dAv(r, s) * e;
+          a2 += dAv(64 + r, s) * e;
         }
-        const uint32_t colo = 32 * hf + 16 * b16;
-        tmem_st16(lanebase + 128 + colo, x1);
-        tmem_st16(lanebase + 192 + colo, x2);
-        tmem_st16(lanebase + 320 + colo, y1);
+        for (int t = r; t < 64; ++t) {
+          const float e = expf(Gc[t * D + c] - gr);
+          b1 += (dAv(t, r) * kpc[t * D + c] + dAv(64 + t, r) * qpc[t * D + c]) * e;
+        }
+        x1[i] = a1;
+        x2[i] = a2;
+        y1[i] = b1;
       }
+      tmem_st16(lanebase + 128 + 16 * cq, x1);
+      tmem_st16(lanebase + 192 + 16 * cq, x2);
+      tmem_st16(lanebase + 320 + 16 * cq, y1);
       tmem_wait_st();
     }
     if (!wait_one(&ms.bar[5], ph, a.status, 408)) { abort = true; break; }
@@ -858,28 +913,30 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
     // (lane = key channel, as TMEM rows are) through the now idle tiles
     float *Gs = reinterpret_cast<float *>(sm + G_A1);              // [64][128] Gam
     uint32_t *KQs = reinterpret_cast<uint32_t *>(sm + G_B1);       // [64][128] k' | q' << 16
+    uint8_t *pbits = sm + G_PBITS;                                 // [8][128] row-group sign bits
+    float *qsum = reinterpret_cast<float *>(sm + G_FSUM);          // [2][4][128]
 #pragma unroll
     for (int rr = 0; rr < 8; ++rr) {
-      const int r = 8 * warp + rr;
-      *reinterpret_cast<float4 *>(Gs + r * D + 4 * lane) = make_float4(P.G[rr][0], P.G[rr][1], P.G[rr][2], P.G[rr][3]);
-      uint32_t kq4[4];
+      const int r = 8 * rg + rr;
+      *reinterpret_cast<float2 *>(Gs + r * D + ch0) = make_float2(P.G[rr][0], P.G[rr][1]);
+      uint32_t kq2[2];
 #pragma unroll
-      for (int m = 0; m < 4; ++m) {
-        const float p = prep_p(P, rr, m);
-        kq4[m] = pack_bf16(p * prep_k(P, rr, m), p * prep_q(P, rr, m));
+      for (int m = 0; m < 2; ++m) {
+        const float p = prep2_p(P, rr, m);
+        kq2[m] = pack_bf16(p * prep2_k(P, rr, m), p * prep2_q(P, rr, m));
       }
-      *reinterpret_cast<uint4 *>(KQs + r * D + 4 * lane) = make_uint4(kq4[0], kq4[1], kq4[2], kq4[3]);
+      *reinterpret_cast<uint2 *>(KQs + r * D + ch0) = make_uint2(kq2[0], kq2[1]);
     }
 #pragma unroll
-    for (int m = 0; m < 4; ++m) {
+    for (int m = 0; m < 2; ++m) {
       uint32_t bits = 0;
 #pragma unroll
-      for (int rr = 0; rr < 8; ++rr) bits |= ((P.pre >> (4 * rr + m)) & 1u) << rr;
-      ms.pbits[warp][4 * lane + m] = (uint8_t)bits;
+      for (int rr = 0; rr < 8; ++rr) bits |= ((P.pre >> (2 * rr + m)) & 1u) << rr;
+      pbits[rg * D + ch0 + m] = (uint8_t)bits;
     }
     __syncthreads();
     {
-      // thread (c, hf): rows 32 hf .. 32 hf + 31 of key channel c
+      // thread (c, cq): rows 16 cq .. 16 cq + 15 of key channel c
       float Gm = 0.f, GC = 0.f;
       uint32_t pcb = 0;
 #pragma unroll
@@ -895,21 +952,23 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
       float *dGs = reinterpret_cast<float *>(sm + G_OU);  // [64][128] dL/dGam, idle tile
       float gcp = 0.f;
 #pragma unroll 1
-      for (int b8 = 0; b8 < 4; ++b8) {
-        const uint32_t colo = 32 * hf + 8 * b8;
+      for (int b8 = 0; b8 < 2; ++b8) {
+        const int r0 = 16 * cq + 8 * b8;
         float X1[8], X2[8], Y1[8], dQG[8], dKG[8], dKh[8], dVv[8];
-        tmem_ld8(lanebase + 128 + colo, X1);
-        tmem_ld8(lanebase + 192 + colo, X2);
-        tmem_ld8(lanebase + 320 + colo, Y1);
-        tmem_ld8(lanebase + 256 + colo, dQG);
-        tmem_ld8(lanebase + 64 + colo, dKG);
-        tmem_ld8(lanebase + 384 + colo, dKh);
-        tmem_ld8(lanebase + 448 + colo, dVv);
+        tmem_ld8(lanebase + 128 + r0, X1);
+        tmem_ld8(lanebase + 192 + r0, X2);
+        tmem_ld8(lanebase + 320 + r0, Y1);
+        tmem_ld8(lanebase + 256 + r0, dQG);
+        tmem_ld8(lanebase + 64 + r0, dKG);
+        tmem_ld8(lanebase + 384 + r0, dKh);
+        tmem_ld8(lanebase + 448 + r0, dVv);
         tmem_wait_ld();
-        const uint32_t pb = ms.pbits[(32 * hf + 8 * b8) >> 3][c];
+        const uint32_t pb = pbits[(r0 >> 3) * D + c];
+        const size_t off0 = ((size_t)(tok0 + r0) * H + h) * D + c;
+        const size_t rstride = (size_t)H * D;
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          const int r = 32 * hf + 8 * b8 + i;
+          const int r = r0 + i;
           const float Gr = Gs[r * D + c];
           const uint32_t kqv = KQs[r * D + c];
           const float kp = bf_lo(kqv), qp = bf_hi(kqv);
@@ -927,7 +986,7 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
           dGs[r * D + c] = kp * x1 + qp * x2 - kp * y1 + dKG[i] * KGv + dQG[i] * QGv - dKh[i] * Kh;
           gcp += dKh[i] * Kh;
           if (r < len) {
-            const size_t off = ((size_t)(tok0 + r) * H + h) * D + c;
+            const size_t off = off0 + i * rstride;
             dq[off] = __float2bfloat16_rn(p * dqp);
             dk[off] = __float2bfloat16_rn(p * dkp);
             dv[off] = __float2bfloat16_rn(dVv[i]);  // lane c is value channel c here
@@ -935,24 +994,30 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
         }
       }
       // reverse in-chunk cumsum of dL/dGam (plus the chunk-end terms) -> dg;
-      // both halves at once: the lower half starts from the upper half's total
+      // the four quarters at once: each starts from the totals of the later ones
       float part = 0.f;
-#pragma unroll 8
-      for (int ii = 0; ii < 32; ++ii) part += dGs[(32 * hf + ii) * D + c];
-      gcps[hf * 128 + c] = gcp;
-      acc1s[hf * 128 + c] = part;
+#pragma unroll
+      for (int ii = 0; ii < 16; ++ii) part += dGs[(16 * cq + ii) * D + c];
+      qsum[cq * D + c] = gcp;
+      qsum[4 * D + cq * D + c] = part;
       __syncthreads();
-      const float gC = gcps[c] + gcps[128 + c] + (ms.dd[0][c] + ms.dd[1][c]) * dC;
-      float acc = gC + (hf == 0 ? acc1s[128 + c] : 0.f);
-#pragma unroll 8
-      for (int ii = 31; ii >= 0; --ii) {
-        const int r = 32 * hf + ii;
+      float gC = 0.f, later = 0.f, ddc = 0.f;
+#pragma unroll
+      for (int q2 = 0; q2 < 4; ++q2) {
+        gC += qsum[q2 * D + c];
+        ddc += ms.dd[q2][c];
+        if (q2 > cq) later += qsum[4 * D + q2 * D + c];
+      }
+      float acc = gC + ddc * dC + later;
+#pragma unroll
+      for (int ii = 15; ii >= 0; --ii) {
+        const int r = 16 * cq + ii;
         acc += dGs[r * D + c];
         if (r < len) a.dg[((size_t)(tok0 + r) * H + h) * D + c] = acc;
       }
       if (tid < 64 && tid < len)
-        dbeta[(size_t)(tok0 + tid) * H + h] =
-            __float2bfloat16_rn(ms.dbc[tid] + ms.dbr[0][tid] + ms.dbr[1][tid]);
+        dbeta[(size_t)(tok0 + tid) * H + h] = __float2bfloat16_rn(
+            ms.dbc[tid] + ms.dbr[0][tid] + ms.dbr[1][tid] + ms.dbr[2][tid] + ms.dbr[3][tid]);
     }
     tc_fence_before();
     __syncthreads();

@@ -134,7 +134,7 @@ __global__ void __launch_bounds__(kIntraThreads, 2) tc_intra_kernel(const __grid
     }
     if (tid < 64) ms.beta[tid] = tid < len ? __bfloat162float(beta[(size_t)(tok0 + tid) * H + h]) : 0.f;
     {
-      const bool ok = mbar_wait(&ms.mld, it & 1, a.status, 100);
+      const bool ok = mbar_wait_ool(&ms.mld, it & 1, a.status, 100);
       if (__syncthreads_or(!ok)) { abort = true; break; }
     }
     // ---------------- prep: row-group layout (rows 8w.., channels 4l..) ----------------
@@ -240,7 +240,7 @@ __global__ void __launch_bounds__(kIntraThreads, 2) tc_intra_kernel(const __grid
         mma_commit(&ms.mbar1);
       }
       bool ok = true;
-      if (tid == 0) ok = mbar_wait(&ms.mbar1, it & 1, a.status, 101);
+      if (tid == 0) ok = mbar_wait_ool(&ms.mbar1, it & 1, a.status, 101);
       if (__syncthreads_or(!ok)) { abort = true; break; }
       tc_fence_after();
       const int qd = warp & 3, ch = warp >> 2;
@@ -327,7 +327,7 @@ __global__ void __launch_bounds__(kIntraThreads, 2) tc_intra_kernel(const __grid
     }
     {
       bool ok = true;
-      if (tid == 0) ok = mbar_wait(&ms.mbar2, it & 1, a.status, 102);
+      if (tid == 0) ok = mbar_wait_ool(&ms.mbar2, it & 1, a.status, 102);
       if (__syncthreads_or(!ok)) { abort = true; break; }
     }
     tc_fence_after();
@@ -366,7 +366,7 @@ __global__ void __launch_bounds__(kIntraThreads, 2) tc_intra_kernel(const __grid
   // wind down: make sure no MMA is still writing TMEM before freeing it
   if (abort && tid == 0) {
     mma_commit(&ms.mfin);
-    mbar_wait(&ms.mfin, 0, a.status, 109);
+    mbar_wait_ool(&ms.mfin, 0, a.status, 109);
   }
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, 256);
