@@ -4,8 +4,8 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload fwdbwd|fwd|varlen|decode]
 
-Default workload (the headline): one step = ckda_chunk_fwd (saving chunk
-states and its per-chunk results) + ckda_chunk_bwd on B=8, H=16, T=4096,
+Default workload (the headline): one step = ckda_chunk_fwd (saving its
+per-chunk results for the backward) + ckda_chunk_bwd on B=8, H=16, T=4096,
 dk=dv=128, bf16 I/O, fp32 gate and state -- the shape of one 1.3B-model
 token-mixer layer.  Inputs are
 seeded synthetic tensors (chunked_gated_delta_ckda_b200.workloads), resident
@@ -175,14 +175,17 @@ def _fwdbwd_setup(inp, dev):
     wsf = api.workspace(_abi.CKDA_OP_CHUNK_FWD, B, T, H, dk, dv, device=dev, cache=False)
     wsb = api.workspace(_abi.CKDA_OP_CHUNK_BWD, B, T, H, dk, dv, device=dev, cache=False)
     code = api.io_code(io)
-    # the forward hands its per-chunk results to the backward (training use)
+    # the forward hands its per-chunk results (intra-chunk products and the
+    # chunk-start states) to the backward (training use); fp32 chunk states
+    # are only materialised where there is no saved form
     sv = api.saved_buffer(B, T, H, dk, dv, io, dev)
+    cs = None if sv is not None else buf["cs"]
 
     def step():
         _abi.ckda_chunk_fwd(B, T, H, dk, dv, code, d["q"], d["k"], d["v"], d["g"], d["sign"],
-                            d["beta"], None, buf["o"], buf["ST"], buf["cs"], wsf, saved=sv)
+                            d["beta"], None, buf["o"], buf["ST"], cs, wsf, saved=sv)
         _abi.ckda_chunk_bwd(B, T, H, dk, dv, code, d["q"], d["k"], d["v"], d["g"], d["sign"],
-                            d["beta"], None, d["dO"], None, buf["cs"], buf["dq"], buf["dk"],
+                            d["beta"], None, d["dO"], None, cs, buf["dq"], buf["dk"],
                             buf["dv"], buf["dg"], buf["dbeta"], buf["dS0"], wsb, saved=sv)
     return d, buf, step
 
@@ -267,7 +270,7 @@ def run_ours(args, rank, world, local_rank):
            "config": {"workload": w.name, "B": B, "T": T, "H": H, "dk": w.dk, "dv": w.dv,
                       "io_dtype": "bf16", "gate_dtype": "f32", "state_dtype": "f32",
                       "contraction": "bf16 tensor-core operands, f32 accumulate",
-                      "step": "ckda_chunk_fwd(save chunk states and per-chunk results) + ckda_chunk_bwd",
+                      "step": "ckda_chunk_fwd(saved buffer for the backward) + ckda_chunk_bwd(saved)",
                       "global_batch": B * world, "seq_len": T, "parallelism": "dp%d" % world,
                       "l2": "inputs larger than L2 (about 2 GB streamed per step)"},
            "roofline": roof, "step_roofline": step_roof, "kernels": kernels,
@@ -389,6 +392,7 @@ def run_e2e(inp, dev, args, world):
     wsb = api.workspace(_abi.CKDA_OP_CHUNK_BWD, B, T, H, dk, dv, device=dev, cache=False)
     code = api.io_code(inp["q"].dtype)
     sv = api.saved_buffer(B, T, H, dk, dv, inp["q"].dtype, dev)
+    cs = None if sv is not None else buf["cs"]
     h2d = sum(v.numel() * v.element_size() for v in host_in.values())
     d2h = sum(v.numel() * v.element_size() for v in host_out.values())
 
@@ -397,9 +401,9 @@ def run_e2e(inp, dev, args, world):
             dev_in[k].copy_(v, non_blocking=True)
         x = dev_in
         _abi.ckda_chunk_fwd(B, T, H, dk, dv, code, x["q"], x["k"], x["v"], x["g"], x["sign"],
-                            x["beta"], None, buf["o"], buf["ST"], buf["cs"], wsf, saved=sv)
+                            x["beta"], None, buf["o"], buf["ST"], cs, wsf, saved=sv)
         _abi.ckda_chunk_bwd(B, T, H, dk, dv, code, x["q"], x["k"], x["v"], x["g"], x["sign"],
-                            x["beta"], None, x["dO"], None, buf["cs"], buf["dq"], buf["dk"],
+                            x["beta"], None, x["dO"], None, cs, buf["dq"], buf["dk"],
                             buf["dv"], buf["dg"], buf["dbeta"], buf["dS0"], wsb, saved=sv)
         for k, v in host_out.items():
             v.copy_(buf[k], non_blocking=True)

@@ -167,8 +167,10 @@ int ckda_chunk_fwd(int B, int T, int H, int dk, int dv, int io_dtype, const void
   a.status = reinterpret_cast<DevStatus *>(w);
   const bool bf16 = io_dtype == CKDA_BF16;
   if (use_tensor_cores(io_dtype, dk, dv)) {
+    // with a saved buffer the state pass also stores each chunk-start state there
     CKDA_CUDA(tc_forward(a, recs_out ? recs_out : reinterpret_cast<unsigned char *>(w + L.intra),
-                         reinterpret_cast<float *>(w + L.fscratch), true, chunk_states, stream));
+                         reinterpret_cast<float *>(w + L.fscratch), true, chunk_states, stream,
+                         /*state_pass=*/true, /*intra_pass=*/true, /*state_tiles=*/recs_out != nullptr));
     return CKDA_OK;
   }
   CKDA_CUDA(v1_intra(a, bf16, reinterpret_cast<float *>(w + L.fscratch), stream));
@@ -211,15 +213,15 @@ int ckda_chunk_bwd(int B, int T, int H, int dk, int dv, int io_dtype, const void
   const float *states = chunk_states;
   const unsigned char *recs =
       recs_in ? recs_in : reinterpret_cast<const unsigned char *>(w + L.intra);
-  if (tcp) {
-    // the intra-chunk records: the forward's when saved, else recomputed here
-    float *st = reinterpret_cast<float *>(w + L.states);
-    if (!recs_in || !states)
-      CKDA_CUDA(tc_forward(f, const_cast<unsigned char *>(recs),
-                           reinterpret_cast<float *>(w + L.fscratch), false, st, stream,
-                           /*state_pass=*/states == nullptr, /*intra_pass=*/recs_in == nullptr));
-    if (!states) states = st;
-  } else {
+  if (tcp && !recs_in) {
+    // no saved buffer: recompute the records here.  Their chunk-start state
+    // tiles come from the caller's fp32 chunk states when given, else from a
+    // recomputed state pass.
+    unsigned char *rw = const_cast<unsigned char *>(recs);
+    CKDA_CUDA(tc_forward(f, rw, reinterpret_cast<float *>(w + L.fscratch), false, nullptr, stream,
+                         /*state_pass=*/states == nullptr, /*intra_pass=*/true, /*state_tiles=*/true));
+    if (states) CKDA_CUDA(tc_state_tiles(states, rw, B, H, f.map.NC, stream));
+  } else if (!tcp) {
     CKDA_CUDA(v1_intra(f, bf16, reinterpret_cast<float *>(w + L.fscratch), stream));
     if (!states) {
       float *st = reinterpret_cast<float *>(w + L.states);

@@ -190,7 +190,10 @@ int tc_intra_ctas();
 size_t tc_record_bytes();
 cudaError_t tc_forward(const FwdArgs &f, unsigned char *recs, float *fb, bool write_o,
                        float *states_out, cudaStream_t s, bool state_pass = true,
-                       bool intra_pass = true);
+                       bool intra_pass = true, bool state_tiles = false);
+// bf16 chunk-start state tiles of the records from fp32 chunk states [B,H,NC,128,128]
+cudaError_t tc_state_tiles(const float *chunk_states, unsigned char *recs, int B, int H, int NC,
+                           cudaStream_t s);
 cudaError_t tc_backward(const BwdArgs &b, const unsigned char *recs, unsigned char *dS_tiles,
                         unsigned char *dU_tiles, float *fb, cudaStream_t s);
 cudaError_t decode_step(int N, int H, int dk, int dv, bool bf16, const void *q,

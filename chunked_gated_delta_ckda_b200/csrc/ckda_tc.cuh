@@ -65,6 +65,27 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t phase, DevStat
   }
   return false;
 }
+// Plain arrive (release): for hand-offs between warp groups of one CTA.
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+// Barrier over `nthreads` threads (a warp group) with id `id` (1..15), and
+// its OR-reduction form: every thread of the group gets the OR of `v`.
+__device__ __forceinline__ void group_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+__device__ __forceinline__ bool group_sync_or(int id, int nthreads, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 q, %1, 0;\n\t"
+      "bar.red.or.pred p, %2, %3, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v), "r"(id), "r"(nthreads)
+      : "memory");
+  return r != 0;
+}
 // The same wait out of line, for kernels that wait at many sites: one copy
 // of the loop keeps their instruction footprint small (the latency-bound
 // state passes keep the inline form).
@@ -75,6 +96,20 @@ static __device__ __noinline__ bool mbar_wait_ool(uint64_t *bar, uint32_t phase,
 // ---------------------------------------------------------------------------
 // bulk async copy global -> shared (1-D, 16-byte aligned, size % 16 == 0)
 // ---------------------------------------------------------------------------
+// Bulk async copy shared -> global (1-D, both 16-byte aligned, size % 16 ==
+// 0), tracked by the issuing thread's bulk groups: commit, then wait until
+// the source may be overwritten (.read) or the data is written.
+__device__ __forceinline__ void bulk_s2g(void *gmem_dst, const void *smem_src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gmem_dst),
+               "r"(smem_u32(smem_src)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read_all() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 // One TMA box of a RowMaps tensor: channels c0.., head h, tokens tok..tok+63.
 // c0 * element size is a multiple of 16 bytes (0 or 64 channels of bf16).
 __device__ __forceinline__ void tma_rows(void *smem_dst, const CUtensorMap *map, int c0, int h, int tok,
@@ -255,8 +290,10 @@ constexpr uint32_t R3 = 49152;   // A_q: K-major tile [r][s] (64 x 64)
 constexpr uint32_t R4 = 57344;   // Khat^T: K-major tile [c][s] (128 x 64)
 constexpr uint32_t R5 = 73728;   // d[128] fp32
 constexpr uint32_t R6 = 74240;   // M = (I + Diag(beta) A)^{-1}: fp32 [64][65] (row stride 65)
+constexpr uint32_t R7 = 90880;   // S_c^T bf16, K-major [v][c] 128 x 128: the chunk-start state
+                                 // (written by the state pass, read by the backward)
 constexpr uint32_t REC_STATE = R6;  // R1 .. R5: the part the sequential state passes read
-constexpr uint32_t REC = 90880;  // bytes per (chunk, head) record
+constexpr uint32_t REC = 123648;    // bytes per (chunk, head) record
 
 // 2^x and 1/x with one MUFU instruction each (PTX ex2.approx / rcp.approx);
 // their relative error (~2^-22) is far below the bf16 operand rounding.

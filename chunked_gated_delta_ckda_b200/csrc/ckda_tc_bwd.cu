@@ -29,7 +29,7 @@ namespace {
 using namespace tc;
 
 // bytes of the per-(chunk, head) tiles the reverse pass hands to the gradient kernel
-constexpr uint32_t DS_TILE = 32768;  // dL/dS_{c+1}: bf16 K-major [c][v], 128 rows
+constexpr uint32_t DS_TILE = 32768;  // dL/dS_{c+1}, transposed: bf16 K-major [v][c], 128 rows
 constexpr uint32_t DU_TILE = 16384;  // dU: bf16 K-major [i][v], 64 rows
 
 struct BwdTcArgs {
@@ -60,7 +60,8 @@ constexpr uint32_t SB_O0 = 2 * RB_SIZE;        // dO tile K-major [r][v], 64 row
 constexpr uint32_t SB_O1 = SB_O0 + 16384;
 constexpr uint32_t SB_DS = SB_O1 + 16384;      // dS^T bf16 K-major [v][c], 128 rows
 constexpr uint32_t SB_DU = SB_DS + 32768;      // dU^T bf16 K-major [v][s], 128 rows x 64
-constexpr uint32_t SB_MISC = SB_DU + 16384;
+constexpr uint32_t SB_DUG = SB_DU + 16384;     // dU bf16 K-major [s][v] 64 rows: the dU tile out
+constexpr uint32_t SB_MISC = SB_DUG + 16384;
 
 struct SbMisc {
   uint64_t mrec[2], mu, ms, mfin;
@@ -124,11 +125,11 @@ __global__ void __launch_bounds__(kSbThreads, 1) tc_state_bwd_kernel(BwdTcArgs t
     }
     cp_async_commit();
   };
-  // dL/dS_{c+1} snapshot of chunk j from the fp32 values of dS^T row v
-  auto snapshot = [&](int j, int c0, const float (&sv)[16]) {
-    unsigned char *dst = ta.dS_tiles + ((size_t)(first + j) * H + h) * DS_TILE;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) st_bf16(dst, kmaj_off(c0 + i, v, 128), sv[i]);
+  // dL/dS_{c+1} snapshot of chunk j: the bf16 dS^T operand tile as it stands
+  // (one bulk store by thread 0, after the tile's writers have synchronised)
+  auto snapshot = [&](int j) {
+    bulk_s2g(ta.dS_tiles + ((size_t)(first + j) * H + h) * DS_TILE, sm + SB_DS, DS_TILE);
+    bulk_commit();
   };
 
   if (tid == 0 && nc > 0) {
@@ -146,7 +147,6 @@ __global__ void __launch_bounds__(kSbThreads, 1) tc_state_bwd_kernel(BwdTcArgs t
         for (int i = 0; i < 16; ++i) a.dS0[sbase + (size_t)(c0 + i) * D + v] = sv[i];
       continue;
     }
-    snapshot(nc - 1, c0, sv);
     uint32_t pk[8];
 #pragma unroll
     for (int m = 0; m < 8; ++m) pk[m] = pack_bf16(sv[2 * m], sv[2 * m + 1]);
@@ -158,6 +158,7 @@ __global__ void __launch_bounds__(kSbThreads, 1) tc_state_bwd_kernel(BwdTcArgs t
   fence_async_smem();
   tc_fence_before();
   __syncthreads();
+  if (tid == 0 && nc > 0) snapshot(nc - 1);
 
   bool abort = false;
   for (int s = 0; s < nc && !abort; ++s) {
@@ -208,13 +209,15 @@ __global__ void __launch_bounds__(kSbThreads, 1) tc_state_bwd_kernel(BwdTcArgs t
     }
     {
       bool ok = true;
-      if (tid == 0) ok = mbar_wait(&ms.mu, s & 1, a.status, 302);
+      if (tid == 0) {
+        ok = mbar_wait(&ms.mu, s & 1, a.status, 302);
+        bulk_wait_read_all();  // the previous dU tile has left its staging tile
+      }
       if (__syncthreads_or(!ok)) { abort = true; break; }
     }
     tc_fence_after();
     // dU^T -> bf16 operand tile and the dU tile of this chunk
     {
-      unsigned char *gdu = ta.dU_tiles + ((size_t)(first + j) * H + h) * DU_TILE;
       for (int s0 = 32 * ch; s0 < 32 * ch + 32; s0 += 16) {
         float w[16];
         tmem_ld16(lanebase + 128 + s0, w);
@@ -225,12 +228,16 @@ __global__ void __launch_bounds__(kSbThreads, 1) tc_state_bwd_kernel(BwdTcArgs t
         *reinterpret_cast<uint4 *>(sm + SB_DU + kmaj_off(v, s0, 128)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
         *reinterpret_cast<uint4 *>(sm + SB_DU + kmaj_off(v, s0 + 8, 128)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) st_bf16(gdu, kmaj_off(s0 + i, v, 64), w[i]);
+        for (int i = 0; i < 16; ++i) st_bf16(sm + SB_DUG, kmaj_off(s0 + i, v, 64), w[i]);
       }
     }
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
+    if (tid == 0) {
+      bulk_s2g(ta.dU_tiles + ((size_t)(first + j) * H + h) * DU_TILE, sm + SB_DUG, DU_TILE);
+      bulk_commit();
+    }
     // dS^T += dO^T QG - dU^T W
     if (tid == 0) {
       tc_fence_after();
@@ -248,7 +255,10 @@ __global__ void __launch_bounds__(kSbThreads, 1) tc_state_bwd_kernel(BwdTcArgs t
     }
     {
       bool ok = true;
-      if (tid == 0) ok = mbar_wait(&ms.ms, s & 1, a.status, 303);
+      if (tid == 0) {
+        ok = mbar_wait(&ms.ms, s & 1, a.status, 303);
+        bulk_wait_read_all();  // the last snapshot has left the dS^T tile
+      }
       if (__syncthreads_or(!ok)) { abort = true; break; }
     }
     tc_fence_after();
@@ -263,7 +273,6 @@ __global__ void __launch_bounds__(kSbThreads, 1) tc_state_bwd_kernel(BwdTcArgs t
           for (int i = 0; i < 16; ++i) a.dS0[sbase + (size_t)(c0 + i) * D + v] = sv[i];
         continue;
       }
-      snapshot(j - 1, c0, sv);
       uint32_t pk[8];
 #pragma unroll
       for (int m = 0; m < 8; ++m) pk[m] = pack_bf16(sv[2 * m], sv[2 * m + 1]);
@@ -273,8 +282,10 @@ __global__ void __launch_bounds__(kSbThreads, 1) tc_state_bwd_kernel(BwdTcArgs t
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
+    if (tid == 0 && j > 0) snapshot(j - 1);
   }
   cp_async_wait_all();
+  if (tid == 0) bulk_wait_all();  // every tile written before the kernel ends
   if (abort && tid == 0) {
     mma_commit(&ms.mfin);
     mbar_wait(&ms.mfin, 0, a.status, 309);
@@ -293,7 +304,7 @@ constexpr uint32_t G_KG = 49152;      // KG (== K-major [j][c] 64 rows); later d
 constexpr uint32_t G_UV = 65536;      // [U; V] K-major 128 x 128
 constexpr uint32_t G_TT = 98304;      // T K-major [r][j] 64 x 64
 constexpr uint32_t G_OU = 106496;     // [dO; dU] K-major 128 x 128
-constexpr uint32_t G_SC = 139264;     // S_c bf16 K-major [c][v]; later dW in rows 64..127
+constexpr uint32_t G_SC = 139264;     // S_c^T bf16 K-major [v][c]; later dW in rows 64..127
 constexpr uint32_t G_WN = 172032;     // W tile | dS1 tile | [dA; dAq] + dT fp32
 constexpr uint32_t G_DT = G_WN + 16384;
 constexpr uint32_t G_MF = 205824;     // M fp32 [64][65]
@@ -307,16 +318,17 @@ constexpr uint32_t G_TH = G_KG, G_TL = G_KG + 8192;             // dM M^T, K-maj
 constexpr uint32_t G_FSUM = G_UV;               // float [2][4][128]
 constexpr uint32_t G_PBITS = G_UV + 8192;       // uint8 [8][128]
 constexpr uint32_t W_TILE = 16384;              // W^T half of the record's R1 tile
+constexpr uint32_t S_TILE = 32768;              // the record's S_c^T (bf16 K-major [v][c])
 constexpr uint32_t M_BYTES = 64 * LDF * 4;      // the record's M
-static_assert(M_BYTES == REC - R6, "M is the record's last field");
+static_assert(M_BYTES == R7 - R6 && S_TILE == REC - R7, "record layout");
 
 struct GMisc {
-  uint64_t bar[6], mdu, mds, mfin, mrec, mld;
+  uint64_t bar[7], mdu, mds, mfin, mrec, mld;
   uint32_t tmem;
   int pad;
   float beta[64], dbc[64], dbr[4][64];
   PrepTot tot;
-  float dd[4][128];
+  float dd[128];
 };
 
 // Completion of MMAs (or of a copy only MMAs consume): one thread polls the
@@ -424,7 +436,7 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
   __nv_bfloat16 *dv = (__nv_bfloat16 *)a.dvg, *dbeta = (__nv_bfloat16 *)a.dbeta;
 
   if (tid == 0) {
-    for (int i = 0; i < 6; ++i) mbar_init(&ms.bar[i], 1);
+    for (int i = 0; i < 7; ++i) mbar_init(&ms.bar[i], 1);
     mbar_init(&ms.mdu, 1);
     mbar_init(&ms.mds, 1);
     mbar_init(&ms.mfin, 1);
@@ -463,8 +475,6 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
     int seq, len, jl;
     int64_t tok0;
     a.map.info(cid, seq, tok0, len, jl);
-    const size_t sidx = (((size_t)seq * H + h) * a.map.NC + jl) * D * D;
-    const float *Sc = a.states + sidx;
     const unsigned char *gdS = ta.dS_tiles + (size_t)item * DS_TILE;
     const unsigned char *gdU = ta.dU_tiles + (size_t)item * DU_TILE;
 
@@ -474,11 +484,12 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
       mbar_arrive_expect_tx(&ms.mdu, DU_TILE);
       bulk_g2s(sm + G_OU + 8192, gdU, 8192, &ms.mdu);
       bulk_g2s(sm + G_OU + 16384 + 8192, gdU + 8192, 8192, &ms.mdu);
-      // the forward's W tile and M of this chunk
+      // the forward's W tile, M and chunk-start state S_c^T of this chunk
       const unsigned char *rec = ta.recs + (size_t)item * REC;
-      mbar_arrive_expect_tx(&ms.mrec, W_TILE + M_BYTES);
+      mbar_arrive_expect_tx(&ms.mrec, W_TILE + M_BYTES + S_TILE);
       bulk_g2s(sm + G_WN, rec + R1, W_TILE, &ms.mrec);
       bulk_g2s(sm + G_MF, rec + R6, M_BYTES, &ms.mrec);
+      bulk_g2s(sm + G_SC, rec + R7, S_TILE, &ms.mrec);
       // the row tensors: q, k staged in A1, g in B1 + KG, sign in TT (the prep
       // consumes them before those tiles are written), V into rows 64.. of
       // [U; V] and dO into rows 0..63 of [dO; dU] (K-major SW128 boxes)
@@ -495,17 +506,7 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
       tma_rows(sm + G_OU, &ta.rm.dO, 0, h, t, &ms.mld);
       tma_rows(sm + G_OU + 16384, &ta.rm.dO, 64, h, t, &ms.mld);
     }
-    // the start state S_c (fp32) through registers -> bf16 K-major [c][v]
-    {
-      float4 x[8];
-#pragma unroll
-      for (int m = 0; m < 8; ++m) x[m] = *reinterpret_cast<const float4 *>(Sc + (size_t)(warp + 16 * m) * D + 4 * lane);
-      if (tid < 64) ms.beta[tid] = tid < len ? __bfloat162float(beta[(size_t)(tok0 + tid) * H + h]) : 0.f;
-#pragma unroll
-      for (int m = 0; m < 8; ++m)
-        *reinterpret_cast<uint2 *>(sm + G_SC + kmaj_off(warp + 16 * m, 4 * lane, 128)) =
-            make_uint2(pack_bf16(x[m].x, x[m].y), pack_bf16(x[m].z, x[m].w));
-    }
+    if (tid < 64) ms.beta[tid] = tid < len ? __bfloat162float(beta[(size_t)(tok0 + tid) * H + h]) : 0.f;
     if (!wait_all(&ms.mld, ph, a.status, 400)) { abort = true; break; }
     Prep2 P;
     prep2_load(sm + G_A1, reinterpret_cast<const float *>(sm + G_B1), sm + G_TT, len, rg, ch0, P, ms.tot);
@@ -596,11 +597,11 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
       for (int kk = 0; kk < 4; ++kk)
         mma_bf16(tmem + 128, sdesc(sUV + 8192 + kk * 2048, 16384, 1024), sdesc(sTT + kk * 32, 16, 1024), idu,
                  kk > 0);
-      const uint32_t idw = idesc_bf16(128, 64, true, true) | (1u << 13);  // negate A: subtract
+      const uint32_t idw = idesc_bf16(128, 64, false, true) | (1u << 13);  // negate A: subtract
 #pragma unroll 1
       for (int kk = 0; kk < 8; ++kk)
-        mma_bf16(tmem + 128, sdesc(sSC + kk * 2048, 16384, 1024), sdesc(sWN + kk * 2048, 16384, 1024), idw,
-                 true);
+        mma_bf16(tmem + 128, sdesc(sSC + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                 sdesc(sWN + kk * 2048, 16384, 1024), idw, true);
       mma_commit(&ms.bar[2]);
     }
     if (!wait_one(&ms.bar[2], ph, a.status, 403)) { abort = true; break; }
@@ -616,19 +617,33 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
 #pragma unroll
       for (int i = 0; i < 16; ++i) st_bf16(sm + G_UV, kmaj_off(16 * cq + i, c, 128), u[i]);
     }
-    // dd partial: sum over v of S_c[c][v] * dS1[c][v] (dS1 arrives meanwhile)
-    if (!wait_all(&ms.mds, ph, a.status, 404)) { abort = true; break; }
-    {
-      float s = 0.f;
+    // dd[c] = sum over v of S_c[c][v] dS1[c][v]: the diagonal of S_c dS1^T, one
+    // MMA from the two transposed tiles (both read MN-major, K = v) into TMEM
+    // columns [256, 384), free until the next products
+    if (!wait_one(&ms.mds, ph, a.status, 404)) { abort = true; break; }
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t id = idesc_bf16(128, 128, true, true);
+#pragma unroll 1
+      for (int kk = 0; kk < 8; ++kk)
+        mma_bf16(tmem + 256, sdesc(sSC + kk * 2048, 16384, 1024), sdesc(sWN + kk * 2048, 16384, 1024), id,
+                 kk > 0);
+      mma_commit(&ms.bar[6]);
+    }
+    if (!wait_one(&ms.bar[6], ph, a.status, 412)) { abort = true; break; }
+    tc_fence_after();
+    if (cq == 0) {
+      float x[16], y[16];
+      tmem_ld16(lanebase + 256 + 32 * qd, x);
+      tmem_ld16(lanebase + 256 + 32 * qd + 16, y);
+      tmem_wait_ld();
+      float dg = 0.f;
 #pragma unroll
-      for (int vv = 32 * cq; vv < 32 * cq + 32; vv += 8) {
-        const uint4 xa = *reinterpret_cast<const uint4 *>(sm + G_SC + kmaj_off(c, vv, 128));
-        const uint4 xb = *reinterpret_cast<const uint4 *>(sm + G_WN + kmaj_off(c, vv, 128));
-        const uint32_t wa[4] = {xa.x, xa.y, xa.z, xa.w}, wb[4] = {xb.x, xb.y, xb.z, xb.w};
-#pragma unroll
-        for (int m = 0; m < 4; ++m) s += bf_lo(wa[m]) * bf_lo(wb[m]) + bf_hi(wa[m]) * bf_hi(wb[m]);
+      for (int k = 0; k < 16; ++k) {
+        dg = (k == lane) ? x[k] : dg;
+        dg = (k + 16 == lane) ? y[k] : dg;
       }
-      ms.dd[cq][c] = s;
+      ms.dd[c] = dg;
     }
     if (!wait_one(&ms.mdu, ph, a.status, 405)) { abort = true; break; }
     fence_async_smem();
@@ -638,13 +653,13 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
     // ---------------- [dQG^T | S dU^T], dKhat^T ----------------
     if (tid == 0) {
       tc_fence_after();
-      const uint32_t id1 = idesc_bf16(128, 128, false, false);
-      const uint32_t id2 = idesc_bf16(128, 64, false, false);
+      const uint32_t id1 = idesc_bf16(128, 128, true, false);  // S_c read MN-major (K = v)
+      const uint32_t id2 = idesc_bf16(128, 64, true, false);   // dS1 read MN-major (K = v)
 #pragma unroll 1
       for (int kk = 0; kk < 8; ++kk) {
         const uint32_t ko = (kk >> 2) * 16384 + (kk & 3) * 32;
-        mma_bf16(tmem + 256, sdesc(sSC + ko, 16, 1024), sdesc(sOU + ko, 16, 1024), id1, kk > 0);
-        mma_bf16(tmem + 384, sdesc(sWN + ko, 16, 1024), sdesc(sUV + ko, 16, 1024), id2, kk > 0);
+        mma_bf16(tmem + 256, sdesc(sSC + kk * 2048, 16384, 1024), sdesc(sOU + ko, 16, 1024), id1, kk > 0);
+        mma_bf16(tmem + 384, sdesc(sWN + kk * 2048, 16384, 1024), sdesc(sUV + ko, 16, 1024), id2, kk > 0);
       }
       mma_commit(&ms.bar[3]);
     }
@@ -1001,11 +1016,12 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
       qsum[cq * D + c] = gcp;
       qsum[4 * D + cq * D + c] = part;
       __syncthreads();
-      float gC = 0.f, later = 0.f, ddc = 0.f;
+      float gC = 0.f, later = 0.f;
+      const float ddc = ms.dd[c];
 #pragma unroll
       for (int q2 = 0; q2 < 4; ++q2) {
         gC += qsum[q2 * D + c];
-        ddc += ms.dd[q2][c];
+
         if (q2 > cq) later += qsum[4 * D + q2 * D + c];
       }
       float acc = gC + ddc * dC + later;
@@ -1028,6 +1044,25 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
   }
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, 512);
+}
+
+// bf16 S^T tile (K-major [v][c], 128-byte swizzle) of one fp32 chunk state
+// [c][v] per CTA: the record field the gradient kernel reads, for callers
+// that hand over fp32 chunk states instead of the forward's saved buffer.
+__global__ void __launch_bounds__(256) tc_state_tiles_kernel(const float *cs, unsigned char *recs, int H,
+                                                             int NC) {
+  const int item = blockIdx.x;  // (sequence * NC + chunk) * H + head
+  const int h = item % H, cid = item / H, b = cid / NC, j = cid % NC;
+  const float *src = cs + (((size_t)b * H + h) * NC + j) * D * D;
+  unsigned char *dst = recs + (size_t)item * REC + R7;
+  const int v = threadIdx.x & 127, half = threadIdx.x >> 7;
+#pragma unroll 2
+  for (int c0 = 64 * half; c0 < 64 * half + 64; c0 += 8) {
+    uint32_t pk[4];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) pk[m] = pack_bf16(src[(size_t)(c0 + 2 * m) * D + v], src[(size_t)(c0 + 2 * m + 1) * D + v]);
+    *reinterpret_cast<uint4 *>(dst + kmaj_off(v, c0, 128)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+  }
 }
 
 int g_sms = 0;
@@ -1073,6 +1108,15 @@ cudaError_t tc_backward(const BwdArgs &b, const unsigned char *recs, unsigned ch
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   return cudaSuccess;
+}
+
+cudaError_t tc_state_tiles(const float *chunk_states, unsigned char *recs, int B, int H, int NC,
+                           cudaStream_t s) {
+  const int64_t items = (int64_t)B * NC * H;
+  if (items == 0) return cudaSuccess;
+  ProfScope prof("tc_state_tiles", s);
+  tc_state_tiles_kernel<<<(unsigned)items, 256, 0, s>>>(chunk_states, recs, H, NC);
+  return cudaGetLastError();
 }
 
 size_t tc_bwd_smem_bytes() { return G_MISC + sizeof(GMisc) + 1024; }

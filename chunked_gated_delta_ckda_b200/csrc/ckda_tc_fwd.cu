@@ -72,6 +72,7 @@ struct TcArgs {
   float *fb;            // per-CTA fallback scratch: Gam, k', q' (3 x 64 x 128 fp32)
   float *states_out;    // chunk-start states (batched only) or null
   bool write_o;
+  bool state_tiles;     // the state pass also stores each chunk-start state (bf16) in its record
 };
 
 __global__ void __launch_bounds__(kIntraThreads, 2) tc_intra_kernel(const __grid_constant__ TcArgs ta) {
@@ -375,7 +376,8 @@ __global__ void __launch_bounds__(kIntraThreads, 2) tc_intra_kernel(const __grid
 // ===========================================================================
 // sequential state kernel
 // ===========================================================================
-constexpr int kStateThreads = 256;              // two warps per TMEM lane quadrant
+constexpr int kStateThreads = 512;   // two warp groups of 256 (two warps per TMEM lane quadrant each)
+constexpr int kGroup = 256;
 constexpr uint32_t S_REC0 = 0;
 constexpr uint32_t S_REC1 = REC_PAD;
 constexpr uint32_t S_TS = 2 * REC_PAD;          // S^T bf16, K-major [v][c] 128 x 128
@@ -383,19 +385,20 @@ constexpr uint32_t S_TU = S_TS + 32768;         // U^T bf16, K-major [v][s] 128 
 constexpr uint32_t S_MISC = S_TU + 16384;
 
 struct StateMisc {
-  uint64_t mrec[2], m3, m4, mfin;
+  uint64_t mrec[2], m3, m4, mfin, sready, sdone;
   uint32_t tmem;
 };
 
-__device__ __forceinline__ bool wait_one(uint64_t *bar, uint32_t phase, DevStatus *st, uint32_t site) {
-  bool ok = true;
-  if (threadIdx.x == 0) ok = mbar_wait(bar, phase, st, site);
-  return !__syncthreads_or(!ok);
-}
-
 // TMEM columns: S^T [0,128); per chunk parity p the MMA3/4 accumulator
-// [(W S)^T | O^T] at 128 + 128 p (so the next chunk's MMA3 can run while the
-// output rows of this chunk are written out).
+// [(W S)^T | O^T] at 128 + 128 p.
+//
+// Two warp groups.  Group A (warps 0-7) runs the chain that carries the
+// state: U^T from MMA3, MMA4/5, the bf16 copy of the new state, the next
+// MMA3.  Group B (warps 8-15) takes what is off that chain: it writes the
+// chunk states out, scales S^T by the next chunk's decay in TMEM (needed only
+// by the next MMA5) and writes the chunk's output rows.  They hand off through
+// two mbarriers, one arrive per warp: sready (A: S_{j+1} and O_j are in TMEM)
+// and sdone (B: S^T is scaled and O_j has been read).
 __global__ void __launch_bounds__(kStateThreads, 1) tc_state_kernel(TcArgs ta) {
   extern __shared__ unsigned char smem_raw[];
   unsigned char *sm = reinterpret_cast<unsigned char *>(
@@ -403,7 +406,9 @@ __global__ void __launch_bounds__(kStateThreads, 1) tc_state_kernel(TcArgs ta) {
   StateMisc &ms = *reinterpret_cast<StateMisc *>(sm + S_MISC);
   const FwdArgs &a = ta.f;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int qd = warp & 3, ch = warp >> 2;
+  const bool grpA = tid < kGroup;
+  const int gt = tid & (kGroup - 1);
+  const int qd = warp & 3, ch = (warp >> 2) & 1;
   const int h = blockIdx.x, seq = blockIdx.y, H = a.H;
   const int v = 32 * qd + lane;  // value channel = TMEM lane
   __nv_bfloat16 *o = (__nv_bfloat16 *)a.o;
@@ -419,6 +424,8 @@ __global__ void __launch_bounds__(kStateThreads, 1) tc_state_kernel(TcArgs ta) {
     mbar_init(&ms.m3, 1);
     mbar_init(&ms.m4, 1);
     mbar_init(&ms.mfin, 1);
+    mbar_init(&ms.sready, kGroup / 32);
+    mbar_init(&ms.sdone, kGroup / 32);
     mbar_fence_init();
   }
   if (warp == 0) {
@@ -451,12 +458,12 @@ __global__ void __launch_bounds__(kStateThreads, 1) tc_state_kernel(TcArgs ta) {
     }
   }
   bool abort = false;
-  // initial state: S^T row v = column v of S0; bf16 copy and Diag(d_0)-scaled fp32
+  // initial state (group A): S^T row v = column v of S0; bf16 copy and Diag(d_0)-scaled fp32
   {
     bool ok = true;
-    if (nc > 0) ok = mbar_wait(&ms.mrec[0], 0, a.status, 201);
+    if (grpA && nc > 0) ok = mbar_wait(&ms.mrec[0], 0, a.status, 201);
     if (__syncthreads_or(!ok)) abort = true;
-    if (!abort) {
+    if (!abort && grpA) {
       const float *d0 = reinterpret_cast<const float *>(recbuf[0] + R5);
       for (int c0 = 64 * ch; c0 < 64 * ch + 64; c0 += 16) {
         float sv[16];
@@ -485,108 +492,155 @@ __global__ void __launch_bounds__(kStateThreads, 1) tc_state_kernel(TcArgs ta) {
   fence_async_smem();
   tc_fence_before();
   __syncthreads();
-  if (!abort && tid == 0 && nc > 0) issue_mma3(0);
-
-  for (int j = 0; j < nc && !abort; ++j) {
-    const int buf = j & 1;
-    unsigned char *rec = recbuf[buf];
-    const uint32_t acc = 128 + 128 * buf;  // [(W S)^T | O^T] of this chunk
-    int sq, len, jl;
-    int64_t tok0;
-    a.map.info(first + j, sq, tok0, len, jl);
-    if (!wait_one(&ms.m3, j & 1, a.status, 203)) { abort = true; break; }
-    tc_fence_after();
-    // U^T = U0^T - (W S)^T  -> bf16 K-major tile [v][s]; this thread: s in [32 ch, 32 ch + 32)
-    for (int s0 = 32 * ch; s0 < 32 * ch + 32; s0 += 16) {
-      float w[16];
-      tmem_ld16(lanebase + acc + s0, w);
-      tmem_wait_ld();
-      const uint4 u0a = *reinterpret_cast<const uint4 *>(rec + R2 + kmaj_off(v, s0, 128));
-      const uint4 u0b = *reinterpret_cast<const uint4 *>(rec + R2 + kmaj_off(v, s0 + 8, 128));
-      const __nv_bfloat16 *ua = reinterpret_cast<const __nv_bfloat16 *>(&u0a);
-      const __nv_bfloat16 *ub = reinterpret_cast<const __nv_bfloat16 *>(&u0b);
-      uint32_t pk[8];
-#pragma unroll
-      for (int m = 0; m < 4; ++m)
-        pk[m] = pack_bf16(__bfloat162float(ua[2 * m]) - w[2 * m], __bfloat162float(ua[2 * m + 1]) - w[2 * m + 1]);
-#pragma unroll
-      for (int m = 0; m < 4; ++m)
-        pk[4 + m] = pack_bf16(__bfloat162float(ub[2 * m]) - w[8 + 2 * m],
-                              __bfloat162float(ub[2 * m + 1]) - w[8 + 2 * m + 1]);
-      *reinterpret_cast<uint4 *>(sm + S_TU + kmaj_off(v, s0, 128)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-      *reinterpret_cast<uint4 *>(sm + S_TU + kmaj_off(v, s0 + 8, 128)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+  if (!abort && tid == 0 && nc > 0) {
+    issue_mma3(0);
+    if (ta.state_tiles) {  // S_0 for the backward
+      bulk_s2g(const_cast<unsigned char *>(record(0)) + R7, sm + S_TS, 32768);
+      bulk_commit();
     }
-    fence_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    // MMA4: O^T += U^T A_q^T ; MMA5: S^T += U^T Khat
-    if (tid == 0) {
-      tc_fence_after();
-      const uint32_t sU = smem_u32(sm + S_TU);
-      const uint32_t id4 = idesc_bf16(128, 64, false, false);
-      const uint32_t id5 = idesc_bf16(128, 128, false, false);
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk) {
-        const uint64_t ad = sdesc(sU + kk * 32, 16, 1024);
-        mma_bf16(tmem + acc + 64, ad, sdesc(smem_u32(rec + R3) + kk * 32, 16, 1024), id4, true);
-        mma_bf16(tmem + 0, ad, sdesc(smem_u32(rec + R4) + kk * 32, 16, 1024), id5, true);
-      }
-      mma_commit(&ms.m4);
-    }
-    if (!wait_one(&ms.m4, j & 1, a.status, 204)) { abort = true; break; }
-    tc_fence_after();
-    // the record buffer is free again: fetch chunk j + 2 into it
-    if (tid == 0 && j + 2 < nc) {
-      mbar_arrive_expect_tx(&ms.mrec[buf], REC_STATE);
-      bulk_g2s(rec, record(j + 2), REC_STATE, &ms.mrec[buf]);
-    }
-    // next state (this thread: columns c in [64 ch, 64 ch + 64))
-    const bool last = (j + 1 == nc);
-    const float *dn = nullptr;
-    if (!last) {
-      const bool ok = mbar_wait(&ms.mrec[buf ^ 1], ((j + 1) >> 1) & 1, a.status, 205);
-      if (__syncthreads_or(!ok)) { abort = true; break; }
-      dn = reinterpret_cast<const float *>(recbuf[buf ^ 1] + R5);
-    }
-    for (int c0 = 64 * ch; c0 < 64 * ch + 64; c0 += 16) {
-      float sv[16];
-      tmem_ld16(lanebase + c0, sv);
-      tmem_wait_ld();
-      if (last) {
-        if (a.ST)
-          for (int i = 0; i < 16; ++i) a.ST[sbase + (size_t)(c0 + i) * D + v] = sv[i];
-        continue;
-      }
-      if (ta.states_out)
-        for (int i = 0; i < 16; ++i)
-          ta.states_out[(((size_t)seq * H + h) * NCb + j + 1) * D * D + (size_t)(c0 + i) * D + v] = sv[i];
-      uint32_t pk[8];
-#pragma unroll
-      for (int m = 0; m < 8; ++m) pk[m] = pack_bf16(sv[2 * m], sv[2 * m + 1]);
-      *reinterpret_cast<uint4 *>(sm + S_TS + kmaj_off(v, c0, 128)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-      *reinterpret_cast<uint4 *>(sm + S_TS + kmaj_off(v, c0 + 8, 128)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-#pragma unroll
-      for (int i = 0; i < 16; ++i) sv[i] *= dn[c0 + i];
-      tmem_st16(lanebase + c0, sv);
-    }
-    tmem_wait_st();
-    fence_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    if (tid == 0 && !last) issue_mma3(j + 1);
-    // output rows of this chunk (overlaps the next chunk's MMA3); rows [32 ch, 32 ch + 32)
-    if (ta.write_o) {
-      for (int r0 = 32 * ch; r0 < 32 * ch + 32; r0 += 16) {
-        float ov[16];
-        tmem_ld16(lanebase + acc + 64 + r0, ov);
-        tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 16; ++i)
-          if (r0 + i < len) o[((size_t)(tok0 + r0 + i) * H + h) * D + v] = __float2bfloat16_rn(ov[i]);
-      }
-    }
-    tc_fence_before();
   }
+
+  if (grpA) {
+    // one thread polls, the group meets at its own barrier (id 1)
+    auto wait_a = [&](uint64_t *bar, uint32_t phase, uint32_t site, bool ok_in) -> bool {
+      bool ok = ok_in;
+      if (gt == 0 && ok) ok = mbar_wait(bar, phase, a.status, site);
+      return !group_sync_or(1, kGroup, !ok);
+    };
+    for (int j = 0; j < nc && !abort; ++j) {
+      const int buf = j & 1;
+      unsigned char *rec = recbuf[buf];
+      const uint32_t acc = 128 + 128 * buf;  // [(W S)^T | O^T] of this chunk
+      if (!wait_a(&ms.m3, j & 1, 203, true)) { abort = true; break; }
+      tc_fence_after();
+      // U^T = U0^T - (W S)^T  -> bf16 K-major tile [v][s]; this thread: s in [32 ch, 32 ch + 32)
+      for (int s0 = 32 * ch; s0 < 32 * ch + 32; s0 += 16) {
+        float w[16];
+        tmem_ld16(lanebase + acc + s0, w);
+        tmem_wait_ld();
+        const uint4 u0a = *reinterpret_cast<const uint4 *>(rec + R2 + kmaj_off(v, s0, 128));
+        const uint4 u0b = *reinterpret_cast<const uint4 *>(rec + R2 + kmaj_off(v, s0 + 8, 128));
+        const __nv_bfloat16 *ua = reinterpret_cast<const __nv_bfloat16 *>(&u0a);
+        const __nv_bfloat16 *ub = reinterpret_cast<const __nv_bfloat16 *>(&u0b);
+        uint32_t pk[8];
+#pragma unroll
+        for (int m = 0; m < 4; ++m)
+          pk[m] = pack_bf16(__bfloat162float(ua[2 * m]) - w[2 * m], __bfloat162float(ua[2 * m + 1]) - w[2 * m + 1]);
+#pragma unroll
+        for (int m = 0; m < 4; ++m)
+          pk[4 + m] = pack_bf16(__bfloat162float(ub[2 * m]) - w[8 + 2 * m],
+                                __bfloat162float(ub[2 * m + 1]) - w[8 + 2 * m + 1]);
+        *reinterpret_cast<uint4 *>(sm + S_TU + kmaj_off(v, s0, 128)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        *reinterpret_cast<uint4 *>(sm + S_TU + kmaj_off(v, s0 + 8, 128)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+      }
+      fence_async_smem();
+      tc_fence_before();
+      group_sync(1, kGroup);
+      // MMA4: O^T += U^T A_q^T ; MMA5: S^T += U^T Khat (S^T scaled by group B first)
+      bool ok = true;
+      if (gt == 0) {
+        if (j > 0) ok = mbar_wait(&ms.sdone, (j - 1) & 1, a.status, 206);
+        if (ok) {
+          tc_fence_after();
+          const uint32_t sU = smem_u32(sm + S_TU);
+          const uint32_t id4 = idesc_bf16(128, 64, false, false);
+          const uint32_t id5 = idesc_bf16(128, 128, false, false);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t ad = sdesc(sU + kk * 32, 16, 1024);
+            mma_bf16(tmem + acc + 64, ad, sdesc(smem_u32(rec + R3) + kk * 32, 16, 1024), id4, true);
+            mma_bf16(tmem + 0, ad, sdesc(smem_u32(rec + R4) + kk * 32, 16, 1024), id5, true);
+          }
+          mma_commit(&ms.m4);
+        }
+      }
+      if (gt == 0) bulk_wait_read_all();  // the last state tile has left S_TS
+      if (!wait_a(&ms.m4, j & 1, 204, ok)) { abort = true; break; }
+      tc_fence_after();
+      // the record buffer is free again: fetch chunk j + 2 into it
+      if (gt == 0 && j + 2 < nc) {
+        mbar_arrive_expect_tx(&ms.mrec[buf], REC_STATE);
+        bulk_g2s(rec, record(j + 2), REC_STATE, &ms.mrec[buf]);
+      }
+      if (j + 1 < nc) {
+        // bf16 copy of S_{j+1} for the next MMA3 (columns c in [64 ch, 64 ch + 64))
+        for (int c0 = 64 * ch; c0 < 64 * ch + 64; c0 += 16) {
+          float sv[16];
+          tmem_ld16(lanebase + c0, sv);
+          tmem_wait_ld();
+          uint32_t pk[8];
+#pragma unroll
+          for (int m = 0; m < 8; ++m) pk[m] = pack_bf16(sv[2 * m], sv[2 * m + 1]);
+          *reinterpret_cast<uint4 *>(sm + S_TS + kmaj_off(v, c0, 128)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          *reinterpret_cast<uint4 *>(sm + S_TS + kmaj_off(v, c0 + 8, 128)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        }
+        fence_async_smem();
+        tc_fence_before();
+        if (!wait_a(&ms.mrec[buf ^ 1], ((j + 1) >> 1) & 1, 205, true)) { abort = true; break; }
+        if (gt == 0) {
+          issue_mma3(j + 1);
+          if (ta.state_tiles) {  // S_{j+1} for the backward
+            bulk_s2g(const_cast<unsigned char *>(record(j + 1)) + R7, sm + S_TS, 32768);
+            bulk_commit();
+          }
+        }
+      }
+      // S_{j+1} and O_j are in TMEM: hand them to group B
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ms.sready);
+    }
+  } else {
+    for (int j = 0; j < nc && !abort; ++j) {
+      const int buf = j & 1;
+      const uint32_t acc = 128 + 128 * buf;
+      int sq, len, jl;
+      int64_t tok0;
+      a.map.info(first + j, sq, tok0, len, jl);
+      const bool last = (j + 1 == nc);
+      bool ok = mbar_wait(&ms.sready, j & 1, a.status, 207);
+      if (ok && !last) ok = mbar_wait(&ms.mrec[buf ^ 1], ((j + 1) >> 1) & 1, a.status, 208);
+      if (group_sync_or(2, kGroup, !ok)) { abort = true; break; }
+      tc_fence_after();
+      // output rows of this chunk, rows [32 ch, 32 ch + 32): read now (MMA3 of
+      // chunk j + 2 reuses these columns once sdone is signalled), stored below
+      float ov[16], ow[16];
+      if (ta.write_o) {
+        tmem_ld16(lanebase + acc + 64 + 32 * ch, ov);
+        tmem_ld16(lanebase + acc + 64 + 32 * ch + 16, ow);
+      }
+      // S_{j+1}: chunk state out (or the final state), then Diag(d_{j+1}) S^T in place
+      const float *dn = last ? nullptr : reinterpret_cast<const float *>(recbuf[buf ^ 1] + R5);
+      for (int c0 = 64 * ch; c0 < 64 * ch + 64; c0 += 16) {
+        float sv[16];
+        tmem_ld16(lanebase + c0, sv);
+        tmem_wait_ld();
+        if (last) {
+          if (a.ST)
+            for (int i = 0; i < 16; ++i) a.ST[sbase + (size_t)(c0 + i) * D + v] = sv[i];
+          continue;
+        }
+        if (ta.states_out)
+          for (int i = 0; i < 16; ++i)
+            ta.states_out[(((size_t)seq * H + h) * NCb + j + 1) * D * D + (size_t)(c0 + i) * D + v] = sv[i];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) sv[i] *= dn[c0 + i];
+        tmem_st16(lanebase + c0, sv);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ms.sdone);
+      if (ta.write_o) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          if (32 * ch + i < len)
+            o[((size_t)(tok0 + 32 * ch + i) * H + h) * D + v] = __float2bfloat16_rn(i < 16 ? ov[i] : ow[i - 16]);
+      }
+    }
+  }
+  if (tid == 0) bulk_wait_all();  // every state tile written before the kernel ends
+  __syncthreads();
   if (abort && tid == 0) {
     mma_commit(&ms.mfin);
     mbar_wait(&ms.mfin, 0, a.status, 209);
@@ -618,13 +672,15 @@ size_t tc_record_bytes() { return REC; }
 // fb: tc_fwd_fallback_floats(tc_intra_ctas()) floats.  intra_pass = false
 // reuses records an earlier call wrote for the same inputs.
 cudaError_t tc_forward(const FwdArgs &f, unsigned char *recs, float *fb, bool write_o,
-                       float *states_out, cudaStream_t s, bool state_pass, bool intra_pass) {
+                       float *states_out, cudaStream_t s, bool state_pass, bool intra_pass,
+                       bool state_tiles) {
   TcArgs ta{};
   ta.f = f;
   ta.recs = recs;
   ta.fb = fb;
   ta.states_out = states_out;
   ta.write_o = write_o;
+  ta.state_tiles = state_tiles;
   const size_t sm_intra = I_MISC + sizeof(IntraMisc) + 1024;
   const size_t sm_state = S_MISC + sizeof(StateMisc) + 1024;
   cudaError_t e = cudaFuncSetAttribute(tc_intra_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,

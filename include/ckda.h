@@ -90,9 +90,9 @@ extern "C" {
 size_t ckda_workspace_size(int op, int B, int T, int H, int dk, int dv, int N);
 
 /* Bytes of the "saved" buffer through which ckda_chunk_fwd can hand its
- * per-chunk intra-chunk results (the UT-transform products of every
- * (chunk, head)) to ckda_chunk_bwd, so that the backward does not recompute
- * them: a memory-for-time trade, like chunk_states.  Returns 0 for shapes
+ * per-chunk results (the UT-transform products of every (chunk, head) and
+ * the chunk-start states, bf16) to ckda_chunk_bwd, so that the backward
+ * recomputes nothing and needs no chunk_states: a memory-for-time trade.  Returns 0 for shapes
  * and dtypes that have no saved form (then `saved` is ignored by both calls
  * and the backward recomputes) and for invalid arguments.  The contents are
  * opaque; they are valid for the inputs of the forward that wrote them. */
@@ -127,7 +127,8 @@ int ckda_chunk_fwd(int B, int T, int H, int dk, int dv, int io_dtype,
  *         inputs (else the forward chunk states are recomputed in ws)
  *   saved, saved_bytes: nullable; the buffer ckda_chunk_fwd filled for the
  *         same inputs (else the per-chunk results are recomputed in ws).
- *         Ignored when ckda_saved_size(...) is 0.
+ *         When given, chunk_states is not read.  Ignored when
+ *         ckda_saved_size(...) is 0.
  *   dq, dk_out [B,T,H,dk] io;  dv_out [B,T,H,dv] io;  dg [B,T,H,dk] f32
  *         (dL/d log|alpha|);  dbeta [B,T,H] io;  dS0 [B,H,dk,dv] f32, nullable
  * The sign gets no gradient (piecewise constant); dg is the exact gradient
