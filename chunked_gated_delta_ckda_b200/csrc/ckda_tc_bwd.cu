@@ -314,9 +314,9 @@ constexpr int LDF = 65;
 constexpr uint32_t G_DMH = G_UV, G_DML = G_UV + 8192;           // dM, K-major [i][j]
 constexpr uint32_t G_MH = G_UV + 16384, G_ML = G_UV + 24576;    // M, K-major [i][a]
 constexpr uint32_t G_TH = G_KG, G_TL = G_KG + 8192;             // dM M^T, K-major [i][k]
-// final epilogue scratch in the idle [U; V] tile: per-quarter sums, sign bits
+// final epilogue scratch in the idle [U; V] tile (rows 0..63 of block 0;
+// the next item's V lands in rows 64..): per-quarter sums
 constexpr uint32_t G_FSUM = G_UV;               // float [2][4][128]
-constexpr uint32_t G_PBITS = G_UV + 8192;       // uint8 [8][128]
 constexpr uint32_t W_TILE = 16384;              // W^T half of the record's R1 tile
 constexpr uint32_t S_TILE = 32768;              // the record's S_c^T (bf16 K-major [v][c])
 constexpr uint32_t M_BYTES = 64 * LDF * 4;      // the record's M
@@ -327,7 +327,8 @@ struct GMisc {
   uint32_t tmem;
   int pad;
   float beta[64], dbc[64], dbr[4][64];
-  PrepTot tot;
+  float qt[4][128];    // per-quarter totals of g (prep)
+  uint8_t qp[4][128];  // per-quarter sign parities (prep)
   float dd[128];
 };
 
@@ -344,83 +345,60 @@ __device__ __forceinline__ bool wait_all(uint64_t *bar, uint32_t phase, DevStatu
   return !__syncthreads_or(!ok);
 }
 
-// Prep in the 16-warp layout: warp w owns chunk rows 8 (w & 7) .. + 7 and
-// key channels 64 (w >> 3) + 2 lane, + 1 (two per lane); the group totals
-// are the same [8][128] arrays as the 8-warp layout's.
-struct Prep2 {
-  float G[8][2];      // chunk-local inclusive cumsum of g (after the carry)
-  uint32_t k2[8];     // raw bf16 k of the two channels
-  uint32_t q2[8];
-  uint32_t pre;       // bit 2*rr+m: sign product of row 8 rg + rr, channel ch0 + m is negative
-  float Gm[2], GC[2];
-  uint32_t pC;        // bit m: chunk sign product of channel ch0 + m is negative
+// Prep in the channel layout: thread (c = tid & 127, cq = tid >> 7) owns key
+// channel c -- the TMEM lane its warp reads -- for chunk rows 16 cq .. 16 cq + 15,
+// so the prep values meet the accumulators of the final epilogue in registers.
+struct PrepC {
+  float G[16];      // chunk-local inclusive cumsum of g (after the carry)
+  uint32_t kq[16];  // raw bf16 k (low half) and q (high half)
+  uint32_t pre;     // bit i: sign product of row 16 cq + i is negative
+  float Gm, GC;     // Gam at the reference row 31 and at the chunk end
+  uint32_t pC;      // the chunk's sign product is negative
 };
-__device__ __forceinline__ void prep2_load(const unsigned char *sqk, const float *sg, const uint8_t *ss, int len,
-                                           int rg, int ch0, Prep2 &P, PrepTot &tot) {
-  float acc[2] = {0.f, 0.f};
+// Reads the staged rows (q, k K-major SW128 tiles, g fp32 [64][128], sign
+// int8 [64][128]), scans the 16 rows, writes the quarter totals.
+__device__ __forceinline__ void prepc_load(const unsigned char *sqk, const float *sg, const uint8_t *ss, int len,
+                                           int c, int cq, PrepC &P, float *qt, uint8_t *qp) {
+  float acc = 0.f;
   uint32_t par = 0, pre = 0;
 #pragma unroll
-  for (int rr = 0; rr < 8; ++rr) {
-    const int r = 8 * rg + rr;
+  for (int i = 0; i < 16; ++i) {
+    const int r = 16 * cq + i;
     const bool valid = r < len;
-    const float2 gv = *reinterpret_cast<const float2 *>(sg + r * D + ch0);
-    const uint32_t sgn = *reinterpret_cast<const uint16_t *>(ss + r * D + ch0);
-    const uint32_t off = kmaj_off(r, ch0, 64);
-    const uint32_t kv = *reinterpret_cast<const uint32_t *>(sqk + kStageK + off);
-    const uint32_t qv = *reinterpret_cast<const uint32_t *>(sqk + kStageQ + off);
-    P.k2[rr] = valid ? kv : 0u;
-    P.q2[rr] = valid ? qv : 0u;
-    const float gg[2] = {gv.x, gv.y};
-#pragma unroll
-    for (int m = 0; m < 2; ++m) {
-      acc[m] += valid ? gg[m] : 0.f;
-      P.G[rr][m] = acc[m];
-      const bool neg = valid && (int8_t)((sgn >> (8 * m)) & 0xffu) < 0;
-      par ^= (neg ? 1u : 0u) << m;
-    }
-    pre |= par << (2 * rr);
+    const float g = sg[r * D + c];
+    const int8_t sgn = (int8_t)ss[r * D + c];
+    const uint32_t off = kmaj_off(r, c, 64);
+    const uint32_t kb = *reinterpret_cast<const uint16_t *>(sqk + kStageK + off);
+    const uint32_t qb = *reinterpret_cast<const uint16_t *>(sqk + kStageQ + off);
+    P.kq[i] = valid ? (kb | (qb << 16)) : 0u;
+    acc += valid ? g : 0.f;
+    P.G[i] = acc;
+    par ^= (valid && sgn < 0) ? 1u : 0u;
+    pre |= par << i;
   }
   P.pre = pre;
-  *reinterpret_cast<float2 *>(&tot.G[rg][ch0]) = make_float2(acc[0], acc[1]);
-  tot.P[rg][ch0] = (uint8_t)(par & 1u);
-  tot.P[rg][ch0 + 1] = (uint8_t)((par >> 1) & 1u);
+  qt[cq * D + c] = acc;
+  qp[cq * D + c] = (uint8_t)par;
 }
-__device__ __forceinline__ void prep2_carry(int rg, int ch0, Prep2 &P, const PrepTot &tot) {
-  float cg[2] = {0.f, 0.f}, gm[2] = {0.f, 0.f}, gc[2] = {0.f, 0.f};
+// After a barrier: carry of the earlier quarters, reference row 31, chunk totals.
+__device__ __forceinline__ void prepc_carry(int c, int cq, PrepC &P, const float *qt, const uint8_t *qp) {
+  float cg = 0.f, gm = 0.f, gc = 0.f;
   uint32_t cp = 0, pc = 0;
 #pragma unroll
-  for (int ww = 0; ww < 8; ++ww) {
-    const float2 t = *reinterpret_cast<const float2 *>(&tot.G[ww][ch0]);
-    const float tt[2] = {t.x, t.y};
-#pragma unroll
-    for (int m = 0; m < 2; ++m) {
-      const uint32_t pb = tot.P[ww][ch0 + m];
-      if (ww < rg) { cg[m] += tt[m]; cp ^= pb << m; }
-      if (ww <= 3) gm[m] += tt[m];
-      gc[m] += tt[m];
-      pc ^= pb << m;
-    }
+  for (int q = 0; q < 4; ++q) {
+    const float t = qt[q * D + c];
+    const uint32_t b = qp[q * D + c];
+    if (q < cq) { cg += t; cp ^= b; }
+    if (q <= 1) gm += t;
+    gc += t;
+    pc ^= b;
   }
 #pragma unroll
-  for (int rr = 0; rr < 8; ++rr)
-#pragma unroll
-    for (int m = 0; m < 2; ++m) P.G[rr][m] += cg[m];
-  uint32_t rep = 0;  // replicate the 2-bit carry parity over the 8 rows
-#pragma unroll
-  for (int rr = 0; rr < 8; ++rr) rep |= cp << (2 * rr);
-  P.pre ^= rep;
-#pragma unroll
-  for (int m = 0; m < 2; ++m) { P.Gm[m] = gm[m]; P.GC[m] = gc[m]; }
+  for (int i = 0; i < 16; ++i) P.G[i] += cg;
+  if (cp) P.pre ^= 0xffffu;
+  P.Gm = gm;
+  P.GC = gc;
   P.pC = pc;
-}
-__device__ __forceinline__ float prep2_p(const Prep2 &P, int rr, int m) {
-  return ((P.pre >> (2 * rr + m)) & 1u) ? -1.f : 1.f;
-}
-__device__ __forceinline__ float prep2_k(const Prep2 &P, int rr, int m) {
-  return m ? bf_hi(P.k2[rr]) : bf_lo(P.k2[rr]);
-}
-__device__ __forceinline__ float prep2_q(const Prep2 &P, int rr, int m) {
-  return m ? bf_hi(P.q2[rr]) : bf_lo(P.q2[rr]);
 }
 
 __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_constant__ BwdTcArgs ta) {
@@ -460,13 +438,51 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
   float *fb = ta.fb + (size_t)blockIdx.x * 3 * 64 * D;
 
   // TMEM-facing mapping: lane quadrant qd of the accumulator rows, column
-  // quarter cq; c = 32 qd + lane is the accumulator row (channel) of this thread
+  // quarter cq; c = 32 qd + lane is the accumulator row (channel) of this
+  // thread, and the key channel of its prep (rows 16 cq .. 16 cq + 15)
   const int qd = warp & 3, cq = warp >> 2;
   const int c = tid & 127;
   const uint32_t lanebase = tmem + ((uint32_t)(32 * qd) << 16);
-  // prep mapping: row group rg, channels ch0, ch0 + 1
-  const int rg = warp & 7, ch0 = 64 * (warp >> 3) + 2 * lane;
   const int nitems = a.map.n_chunks() * H;
+
+  // Every load of one item: the reverse pass's dU tile, the forward's W tile,
+  // M and S_c^T, and the row tensors (q, k staged in A1, g in B1 + KG, sign in
+  // TT -- the prep consumes them before those tiles are written -- V into
+  // rows 64.. of [U; V] and dO into rows 0..63 of [dO; dU], K-major SW128
+  // boxes).  Issued by thread 0 once the previous item's last readers of
+  // these regions are done (its phase E), so they overlap its final epilogue.
+  // thread 0's count of issued load sets (each completes mld, mrec and mdu
+  // once) and of the completions it has seen: an abort drains the rest
+  uint32_t n_issued = 0, n_mld = 0, n_mrec = 0, n_mdu = 0;
+  auto issue_loads = [&](int itm) {
+    ++n_issued;
+    int sq_, len_, jl_;
+    int64_t tk_;
+    a.map.info(itm / H, sq_, tk_, len_, jl_);
+    const int hh = itm % H, t = (int)tk_;
+    fence_async_smem();  // earlier generic accesses of the destinations come first
+    const unsigned char *gdU = ta.dU_tiles + (size_t)itm * DU_TILE;
+    mbar_arrive_expect_tx(&ms.mdu, DU_TILE);
+    bulk_g2s(sm + G_OU + 8192, gdU, 8192, &ms.mdu);
+    bulk_g2s(sm + G_OU + 16384 + 8192, gdU + 8192, 8192, &ms.mdu);
+    const unsigned char *rec = ta.recs + (size_t)itm * REC;
+    mbar_arrive_expect_tx(&ms.mrec, W_TILE + M_BYTES + S_TILE);
+    bulk_g2s(sm + G_WN, rec + R1, W_TILE, &ms.mrec);
+    bulk_g2s(sm + G_MF, rec + R6, M_BYTES, &ms.mrec);
+    bulk_g2s(sm + G_SC, rec + R7, S_TILE, &ms.mrec);
+    mbar_arrive_expect_tx(&ms.mld, kRowBytesQK + kRowBytesG + kRowBytesSign + 2 * 16384);
+    tma_rows(sm + G_A1 + kStageQ, &ta.rm.q, 0, hh, t, &ms.mld);
+    tma_rows(sm + G_A1 + kStageQ + 8192, &ta.rm.q, 64, hh, t, &ms.mld);
+    tma_rows(sm + G_A1 + kStageK, &ta.rm.k, 0, hh, t, &ms.mld);
+    tma_rows(sm + G_A1 + kStageK + 8192, &ta.rm.k, 64, hh, t, &ms.mld);
+    tma_rows(sm + G_B1, &ta.rm.g, 0, hh, t, &ms.mld);
+    tma_rows(sm + G_TT, &ta.rm.sign, 0, hh, t, &ms.mld);
+    tma_rows(sm + G_UV + 8192, &ta.rm.v, 0, hh, t, &ms.mld);
+    tma_rows(sm + G_UV + 16384 + 8192, &ta.rm.v, 64, hh, t, &ms.mld);
+    tma_rows(sm + G_OU, &ta.rm.dO, 0, hh, t, &ms.mld);
+    tma_rows(sm + G_OU + 16384, &ta.rm.dO, 64, hh, t, &ms.mld);
+  };
+
   uint32_t it = 0;
   bool abort = false;
   for (int item = blockIdx.x; item < nitems && !abort; item += gridDim.x, ++it) {
@@ -476,92 +492,52 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
     int64_t tok0;
     a.map.info(cid, seq, tok0, len, jl);
     const unsigned char *gdS = ta.dS_tiles + (size_t)item * DS_TILE;
-    const unsigned char *gdU = ta.dU_tiles + (size_t)item * DU_TILE;
 
     // ---------------- loads ----------------
-    if (tid == 0) {
-      fence_async_smem();  // earlier generic accesses of the destinations come first
-      mbar_arrive_expect_tx(&ms.mdu, DU_TILE);
-      bulk_g2s(sm + G_OU + 8192, gdU, 8192, &ms.mdu);
-      bulk_g2s(sm + G_OU + 16384 + 8192, gdU + 8192, 8192, &ms.mdu);
-      // the forward's W tile, M and chunk-start state S_c^T of this chunk
-      const unsigned char *rec = ta.recs + (size_t)item * REC;
-      mbar_arrive_expect_tx(&ms.mrec, W_TILE + M_BYTES + S_TILE);
-      bulk_g2s(sm + G_WN, rec + R1, W_TILE, &ms.mrec);
-      bulk_g2s(sm + G_MF, rec + R6, M_BYTES, &ms.mrec);
-      bulk_g2s(sm + G_SC, rec + R7, S_TILE, &ms.mrec);
-      // the row tensors: q, k staged in A1, g in B1 + KG, sign in TT (the prep
-      // consumes them before those tiles are written), V into rows 64.. of
-      // [U; V] and dO into rows 0..63 of [dO; dU] (K-major SW128 boxes)
-      mbar_arrive_expect_tx(&ms.mld, kRowBytesQK + kRowBytesG + kRowBytesSign + 2 * 16384);
-      const int t = (int)tok0;
-      tma_rows(sm + G_A1 + kStageQ, &ta.rm.q, 0, h, t, &ms.mld);
-      tma_rows(sm + G_A1 + kStageQ + 8192, &ta.rm.q, 64, h, t, &ms.mld);
-      tma_rows(sm + G_A1 + kStageK, &ta.rm.k, 0, h, t, &ms.mld);
-      tma_rows(sm + G_A1 + kStageK + 8192, &ta.rm.k, 64, h, t, &ms.mld);
-      tma_rows(sm + G_B1, &ta.rm.g, 0, h, t, &ms.mld);
-      tma_rows(sm + G_TT, &ta.rm.sign, 0, h, t, &ms.mld);
-      tma_rows(sm + G_UV + 8192, &ta.rm.v, 0, h, t, &ms.mld);
-      tma_rows(sm + G_UV + 16384 + 8192, &ta.rm.v, 64, h, t, &ms.mld);
-      tma_rows(sm + G_OU, &ta.rm.dO, 0, h, t, &ms.mld);
-      tma_rows(sm + G_OU + 16384, &ta.rm.dO, 64, h, t, &ms.mld);
-    }
+    if (tid == 0 && it == 0) issue_loads(item);  // later items: issued during the previous one
     if (tid < 64) ms.beta[tid] = tid < len ? __bfloat162float(beta[(size_t)(tok0 + tid) * H + h]) : 0.f;
     if (!wait_all(&ms.mld, ph, a.status, 400)) { abort = true; break; }
-    Prep2 P;
-    prep2_load(sm + G_A1, reinterpret_cast<const float *>(sm + G_B1), sm + G_TT, len, rg, ch0, P, ms.tot);
+    ++n_mld;
+    PrepC P;
+    prepc_load(sm + G_A1, reinterpret_cast<const float *>(sm + G_B1), sm + G_TT, len, c, cq, P, &ms.qt[0][0],
+               &ms.qp[0][0]);
     if (len < 64) {  // V and dO rows past the chunk
       zero_tail_rows(sm + G_UV + 8192, 16384, len, tid, kGThreads);
       zero_tail_rows(sm + G_OU, 16384, len, tid, kGThreads);
     }
     __syncthreads();
-    prep2_carry(rg, ch0, P, ms.tot);
+    prepc_carry(c, cq, P, &ms.qt[0][0], &ms.qp[0][0]);
     int bad = 0;
 #pragma unroll
-    for (int rr = 0; rr < 8; ++rr)
-#pragma unroll
-      for (int m = 0; m < 2; ++m)
-        if (!(fabsf(P.G[rr][m] - P.Gm[m]) <= kTau)) bad = 1;
+    for (int i = 0; i < 16; ++i)
+      if (!(fabsf(P.G[i] - P.Gm) <= kTau)) bad = 1;
     const bool fast = !__syncthreads_or(bad);
 
     // ---------------- operand tiles ----------------
+    // the stores of a warp cover 32 consecutive channels of one row
     if (fast) {
-      const float e0 = fast_exp(P.Gm[0]), e1 = fast_exp(P.Gm[1]);
+      const float eGm = fast_exp(P.Gm);
 #pragma unroll
-      for (int rr = 0; rr < 8; ++rr) {
-        const int r = 8 * rg + rr;
-        float ql[2], kl[2], kr[2];
-#pragma unroll
-        for (int m = 0; m < 2; ++m) {
-          const float p = prep2_p(P, rr, m);
-          const float kp = p * prep2_k(P, rr, m), qp = p * prep2_q(P, rr, m);
-          const float el = fast_exp(P.G[rr][m] - P.Gm[m]), er = rcp_approx(el);
-          ql[m] = qp * el;
-          kl[m] = kp * el;
-          kr[m] = kp * er;
-        }
-        *reinterpret_cast<uint32_t *>(sm + G_A1 + kmaj_off(r, ch0, 128)) = pack_bf16(ql[0], ql[1]);
-        *reinterpret_cast<uint32_t *>(sm + G_A1 + kmaj_off(64 + r, ch0, 128)) = pack_bf16(kl[0], kl[1]);
-        *reinterpret_cast<uint32_t *>(sm + G_B1 + kmaj_off(r, ch0, 64)) = pack_bf16(kr[0], kr[1]);
-        *reinterpret_cast<uint32_t *>(sm + G_KG + mnmaj_off(r, ch0, 64)) = pack_bf16(kl[0] * e0, kl[1] * e1);
+      for (int i = 0; i < 16; ++i) {
+        const int r = 16 * cq + i;
+        const float p = ((P.pre >> i) & 1u) ? -1.f : 1.f;
+        const float kp = p * bf_lo(P.kq[i]), qp = p * bf_hi(P.kq[i]);
+        const float el = fast_exp(P.G[i] - P.Gm), er = rcp_approx(el);
+        st_bf16(sm + G_A1, kmaj_off(r, c, 128), qp * el);
+        st_bf16(sm + G_A1, kmaj_off(64 + r, c, 128), kp * el);
+        st_bf16(sm + G_B1, kmaj_off(r, c, 64), kp * er);
+        st_bf16(sm + G_KG, mnmaj_off(r, c, 64), kp * el * eGm);
       }
     } else {
 #pragma unroll 1
-      for (int rr = 0; rr < 8; ++rr) {
-        const int r = 8 * rg + rr;
-        float kp2[2], qp2[2], g2[2];
-#pragma unroll
-        for (int m = 0; m < 2; ++m) {
-          const float p = prep2_p(P, rr, m);
-          kp2[m] = p * prep2_k(P, rr, m);
-          qp2[m] = p * prep2_q(P, rr, m);
-          g2[m] = P.G[rr][m];
-        }
-        *reinterpret_cast<float2 *>(fb + r * D + ch0) = make_float2(g2[0], g2[1]);
-        *reinterpret_cast<float2 *>(fb + 64 * D + r * D + ch0) = make_float2(kp2[0], kp2[1]);
-        *reinterpret_cast<float2 *>(fb + 128 * D + r * D + ch0) = make_float2(qp2[0], qp2[1]);
-        *reinterpret_cast<uint32_t *>(sm + G_KG + mnmaj_off(r, ch0, 64)) =
-            pack_bf16(kp2[0] * fast_exp(g2[0]), kp2[1] * fast_exp(g2[1]));
+      for (int i = 0; i < 16; ++i) {
+        const int r = 16 * cq + i;
+        const float p = ((P.pre >> i) & 1u) ? -1.f : 1.f;
+        const float kp = p * bf_lo(P.kq[i]), qp = p * bf_hi(P.kq[i]);
+        fb[r * D + c] = P.G[i];
+        fb[64 * D + r * D + c] = kp;
+        fb[128 * D + r * D + c] = qp;
+        st_bf16(sm + G_KG, mnmaj_off(r, c, 64), kp * fast_exp(P.G[i]));
       }
     }
     fence_async_smem();
@@ -569,6 +545,7 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
 
     // ---------------- T = M Diag(beta) (M from the forward's record) ----------------
     if (!wait_all(&ms.mrec, ph, a.status, 401)) { abort = true; break; }
+    ++n_mrec;
     {
       const int r = tid >> 3, j0 = (tid & 7) * 8;
       uint32_t pk[4];
@@ -646,6 +623,7 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
       ms.dd[c] = dg;
     }
     if (!wait_one(&ms.mdu, ph, a.status, 405)) { abort = true; break; }
+    ++n_mdu;
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -922,51 +900,22 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
     }
     if (!wait_one(&ms.bar[5], ph, a.status, 408)) { abort = true; break; }
     tc_fence_after();
+    // every shared-memory tile is idle now: the next item's loads overlap the
+    // final epilogue (TMEM, registers and the quarter sums only)
+    if (tid == 0 && item + (int)gridDim.x < nitems) issue_loads(item + gridDim.x);
 
     // ---------------- final elementwise gradients ----------------
-    // hand the prep values from the row-group layout to the channel layout
-    // (lane = key channel, as TMEM rows are) through the now idle tiles
-    float *Gs = reinterpret_cast<float *>(sm + G_A1);              // [64][128] Gam
-    uint32_t *KQs = reinterpret_cast<uint32_t *>(sm + G_B1);       // [64][128] k' | q' << 16
-    uint8_t *pbits = sm + G_PBITS;                                 // [8][128] row-group sign bits
-    float *qsum = reinterpret_cast<float *>(sm + G_FSUM);          // [2][4][128]
-#pragma unroll
-    for (int rr = 0; rr < 8; ++rr) {
-      const int r = 8 * rg + rr;
-      *reinterpret_cast<float2 *>(Gs + r * D + ch0) = make_float2(P.G[rr][0], P.G[rr][1]);
-      uint32_t kq2[2];
-#pragma unroll
-      for (int m = 0; m < 2; ++m) {
-        const float p = prep2_p(P, rr, m);
-        kq2[m] = pack_bf16(p * prep2_k(P, rr, m), p * prep2_q(P, rr, m));
-      }
-      *reinterpret_cast<uint2 *>(KQs + r * D + ch0) = make_uint2(kq2[0], kq2[1]);
-    }
-#pragma unroll
-    for (int m = 0; m < 2; ++m) {
-      uint32_t bits = 0;
-#pragma unroll
-      for (int rr = 0; rr < 8; ++rr) bits |= ((P.pre >> (2 * rr + m)) & 1u) << rr;
-      pbits[rg * D + ch0 + m] = (uint8_t)bits;
-    }
-    __syncthreads();
+    // thread (c, cq): rows 16 cq .. 16 cq + 15 of key channel c, prep values
+    // and accumulators both at hand; dL/dGam stays in registers
     {
-      // thread (c, cq): rows 16 cq .. 16 cq + 15 of key channel c
-      float Gm = 0.f, GC = 0.f;
-      uint32_t pcb = 0;
-#pragma unroll
-      for (int ww = 0; ww < 8; ++ww) {
-        const float t = ms.tot.G[ww][c];
-        if (ww <= 3) Gm += t;
-        GC += t;
-        pcb ^= ms.tot.P[ww][c];
-      }
-      const float pCs = pcb ? -1.f : 1.f;
-      const float eGm = fast_exp(Gm), eCm = fast_exp(GC - Gm);
-      const float dC = pCs * fast_exp(GC);
-      float *dGs = reinterpret_cast<float *>(sm + G_OU);  // [64][128] dL/dGam, idle tile
+      float *qsum = reinterpret_cast<float *>(sm + G_FSUM);  // [2][4][128]
+      const float pCs = P.pC ? -1.f : 1.f;
+      const float eGm = fast_exp(P.Gm), eCm = fast_exp(P.GC - P.Gm);
+      const float dC = pCs * fast_exp(P.GC);
+      const size_t rstride = (size_t)H * D;
+      float dgs[16];
       float gcp = 0.f;
-#pragma unroll 1
+#pragma unroll
       for (int b8 = 0; b8 < 2; ++b8) {
         const int r0 = 16 * cq + 8 * b8;
         float X1[8], X2[8], Y1[8], dQG[8], dKG[8], dKh[8], dVv[8];
@@ -978,27 +927,24 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
         tmem_ld8(lanebase + 384 + r0, dKh);
         tmem_ld8(lanebase + 448 + r0, dVv);
         tmem_wait_ld();
-        const uint32_t pb = pbits[(r0 >> 3) * D + c];
         const size_t off0 = ((size_t)(tok0 + r0) * H + h) * D + c;
-        const size_t rstride = (size_t)H * D;
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          const int r = r0 + i;
-          const float Gr = Gs[r * D + c];
-          const uint32_t kqv = KQs[r * D + c];
-          const float kp = bf_lo(kqv), qp = bf_hi(kqv);
-          const float p = ((pb >> i) & 1u) ? -1.f : 1.f;
+          const int ii = 8 * b8 + i, r = r0 + i;
+          const float Gr = P.G[ii];
+          const float p = ((P.pre >> ii) & 1u) ? -1.f : 1.f;
+          const float kp = p * bf_lo(P.kq[ii]), qp = p * bf_hi(P.kq[ii]);
           // fast path: the pair terms carry the reference-row scaling; exact
           // path: they are final, and the factors come straight from Gam
-          const float el = fast ? fast_exp(Gr - Gm) : 1.f;
+          const float el = fast ? fast_exp(Gr - P.Gm) : 1.f;
           const float er = fast ? rcp_approx(el) : 1.f;
           const float E = fast ? el * eGm : fast_exp(Gr);
-          const float eC = fast ? er * eCm : fast_exp(GC - Gr);
+          const float eC = fast ? er * eCm : fast_exp(P.GC - Gr);
           const float x1 = el * X1[i], x2 = el * X2[i], y1 = er * Y1[i];
           const float KGv = kp * E, QGv = qp * E, Kh = pCs * kp * eC;
           const float dkp = x1 + y1 + dKG[i] * E + pCs * dKh[i] * eC;
           const float dqp = x2 + dQG[i] * E;
-          dGs[r * D + c] = kp * x1 + qp * x2 - kp * y1 + dKG[i] * KGv + dQG[i] * QGv - dKh[i] * Kh;
+          dgs[ii] = kp * x1 + qp * x2 - kp * y1 + dKG[i] * KGv + dQG[i] * QGv - dKh[i] * Kh;
           gcp += dKh[i] * Kh;
           if (r < len) {
             const size_t off = off0 + i * rstride;
@@ -1012,7 +958,7 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
       // the four quarters at once: each starts from the totals of the later ones
       float part = 0.f;
 #pragma unroll
-      for (int ii = 0; ii < 16; ++ii) part += dGs[(16 * cq + ii) * D + c];
+      for (int ii = 0; ii < 16; ++ii) part += dgs[ii];
       qsum[cq * D + c] = gcp;
       qsum[4 * D + cq * D + c] = part;
       __syncthreads();
@@ -1021,14 +967,13 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
 #pragma unroll
       for (int q2 = 0; q2 < 4; ++q2) {
         gC += qsum[q2 * D + c];
-
         if (q2 > cq) later += qsum[4 * D + q2 * D + c];
       }
       float acc = gC + ddc * dC + later;
 #pragma unroll
       for (int ii = 15; ii >= 0; --ii) {
         const int r = 16 * cq + ii;
-        acc += dGs[r * D + c];
+        acc += dgs[ii];
         if (r < len) a.dg[((size_t)(tok0 + r) * H + h) * D + c] = acc;
       }
       if (tid < 64 && tid < len)
@@ -1041,6 +986,10 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
   if (abort && tid == 0) {
     mma_commit(&ms.mfin);
     mbar_wait(&ms.mfin, 0, a.status, 409);
+    // copies still landing in shared memory finish before the CTA leaves
+    for (; n_mld < n_issued; ++n_mld) mbar_wait(&ms.mld, n_mld & 1, a.status, 413);
+    for (; n_mrec < n_issued; ++n_mrec) mbar_wait(&ms.mrec, n_mrec & 1, a.status, 414);
+    for (; n_mdu < n_issued; ++n_mdu) mbar_wait(&ms.mdu, n_mdu & 1, a.status, 415);
   }
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, 512);
