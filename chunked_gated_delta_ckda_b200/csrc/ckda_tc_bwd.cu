@@ -52,7 +52,8 @@ __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wai
 // ===========================================================================
 // reverse state pass
 // ===========================================================================
-constexpr int kSbThreads = 256;  // two warps per TMEM lane quadrant
+constexpr int kSbThreads = 512;  // two warp groups of 256 (two warps per TMEM lane quadrant each)
+constexpr int kSbGroup = 256;
 constexpr uint32_t RB_SIZE = 58368;            // compact record: R1 | R3 | R4 | R5
 constexpr uint32_t RB_R1 = 0, RB_R3 = 32768, RB_R4 = 40960, RB_R5 = 57344;
 constexpr uint32_t SB_RB0 = 0, SB_RB1 = RB_SIZE;
@@ -64,10 +65,20 @@ constexpr uint32_t SB_DUG = SB_DU + 16384;     // dU bf16 K-major [s][v] 64 rows
 constexpr uint32_t SB_MISC = SB_DUG + 16384;
 
 struct SbMisc {
-  uint64_t mrec[2], mu, ms, mfin;
+  uint64_t mrec[2], mu, ms, mfin, dsready, scaled, dudone;
   uint32_t tmem;
 };
 
+// TMEM: dS^T fp32 [0,128) (lanes = value channel); dU^T of step s at
+// 128 + 64 (s & 1).
+//
+// Two warp groups.  Group A (warps 0-7) carries the reverse recurrence: the
+// dU MMA, the bf16 dU^T operand, the dS MMA, the bf16 dS^T operand (and the
+// dL/dS snapshot by bulk store).  Group B (warps 8-15) does what the next
+// MMA only needs done in time: dS^T <- dS^T Diag(d_j) in TMEM before the dS
+// MMA of step s, and the dU tile out (staged transposed, bulk stored).
+// Hand-offs (one arrive per warp): dsready (A: dS^T has been read), scaled
+// (B: dS^T is scaled), dudone (B: the dU^T buffer has been read).
 __global__ void __launch_bounds__(kSbThreads, 1) tc_state_bwd_kernel(BwdTcArgs ta) {
   extern __shared__ unsigned char smem_raw[];
   unsigned char *sm = reinterpret_cast<unsigned char *>(
@@ -75,7 +86,9 @@ __global__ void __launch_bounds__(kSbThreads, 1) tc_state_bwd_kernel(BwdTcArgs t
   SbMisc &ms = *reinterpret_cast<SbMisc *>(sm + SB_MISC);
   const BwdArgs &a = ta.b;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int qd = warp & 3, ch = warp >> 2;
+  const bool grpA = tid < kSbGroup;
+  const int gt = tid & (kSbGroup - 1);
+  const int qd = warp & 3, ch = (warp >> 2) & 1;
   const int h = blockIdx.x, seq = blockIdx.y, H = a.H;
   const int v = 32 * qd + lane;
   const __nv_bfloat16 *dO = (const __nv_bfloat16 *)a.dO;
@@ -89,6 +102,9 @@ __global__ void __launch_bounds__(kSbThreads, 1) tc_state_bwd_kernel(BwdTcArgs t
     mbar_init(&ms.mu, 1);
     mbar_init(&ms.ms, 1);
     mbar_init(&ms.mfin, 1);
+    mbar_init(&ms.dsready, kSbGroup / 32);
+    mbar_init(&ms.scaled, kSbGroup / 32);
+    mbar_init(&ms.dudone, kSbGroup / 32);
     mbar_fence_init();
   }
   if (warp == 0) {
@@ -112,13 +128,13 @@ __global__ void __launch_bounds__(kSbThreads, 1) tc_state_bwd_kernel(BwdTcArgs t
     bulk_g2s(dst + RB_R1, src + R1, 32768, &ms.mrec[s & 1]);
     bulk_g2s(dst + RB_R3, src + R3, 25088, &ms.mrec[s & 1]);
   };
-  auto issue_dO = [&](int s) {
+  auto issue_dO = [&](int s) {  // group A
     const int j = nc - 1 - s;
     int sq, len, jl;
     int64_t tok0;
     a.map.info(first + j, sq, tok0, len, jl);
     unsigned char *dst = ob[s & 1];
-    for (int e = tid; e < 64 * 16; e += kSbThreads) {
+    for (int e = gt; e < 64 * 16; e += kSbGroup) {
       const int r = e >> 4, cc = e & 15;
       const int rr = r < len ? r : 0;
       cp_async16(dst + kmaj_off(r, cc * 8, 64), dO + ((size_t)(tok0 + rr) * H + h) * D + cc * 8, r < len);
@@ -126,7 +142,7 @@ __global__ void __launch_bounds__(kSbThreads, 1) tc_state_bwd_kernel(BwdTcArgs t
     cp_async_commit();
   };
   // dL/dS_{c+1} snapshot of chunk j: the bf16 dS^T operand tile as it stands
-  // (one bulk store by thread 0, after the tile's writers have synchronised)
+  // (one bulk store by group A's first thread, after the tile's writers have synchronised)
   auto snapshot = [&](int j) {
     bulk_s2g(ta.dS_tiles + ((size_t)(first + j) * H + h) * DS_TILE, sm + SB_DS, DS_TILE);
     bulk_commit();
@@ -136,139 +152,14 @@ __global__ void __launch_bounds__(kSbThreads, 1) tc_state_bwd_kernel(BwdTcArgs t
     issue_record(0);
     if (nc > 1) issue_record(1);
   }
-  if (nc > 0) issue_dO(0);
-  // dS_T (true frame) -> dS^T rows; bf16 copy for the MMA, fp32 in TMEM
-  for (int c0 = 64 * ch; c0 < 64 * ch + 64; c0 += 16) {
-    float sv[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) sv[i] = a.dST ? a.dST[sbase + (size_t)(c0 + i) * D + v] : 0.f;
-    if (nc == 0) {
-      if (a.dS0)
-        for (int i = 0; i < 16; ++i) a.dS0[sbase + (size_t)(c0 + i) * D + v] = sv[i];
-      continue;
-    }
-    uint32_t pk[8];
-#pragma unroll
-    for (int m = 0; m < 8; ++m) pk[m] = pack_bf16(sv[2 * m], sv[2 * m + 1]);
-    *reinterpret_cast<uint4 *>(sm + SB_DS + kmaj_off(v, c0, 128)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-    *reinterpret_cast<uint4 *>(sm + SB_DS + kmaj_off(v, c0 + 8, 128)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-    tmem_st16(lanebase + c0, sv);
-  }
-  tmem_wait_st();
-  fence_async_smem();
-  tc_fence_before();
-  __syncthreads();
-  if (tid == 0 && nc > 0) snapshot(nc - 1);
-
-  bool abort = false;
-  for (int s = 0; s < nc && !abort; ++s) {
-    const int j = nc - 1 - s;
-    const int b = s & 1;
-    unsigned char *rec = rb[b];
-    unsigned char *ot = ob[b];
-    int sq, len, jl;
-    int64_t tok0;
-    a.map.info(first + j, sq, tok0, len, jl);
-    if (s + 1 < nc) issue_dO(s + 1);  // prefetch next dO into the other buffer
-    {
-      // dO of this step landed (all but the group just committed)
-      if (s + 1 < nc) asm volatile("cp.async.wait_group 1;" ::: "memory");
-      else cp_async_wait_all();
-      fence_async_smem();
-      const bool ok = mbar_wait(&ms.mrec[b], (s >> 1) & 1, a.status, 301);
-      if (__syncthreads_or(!ok)) { abort = true; break; }
-    }
-    // dU^T = dO^T A_q + dS1^T Khat^T
-    if (tid == 0) {
-      tc_fence_after();
-      const uint32_t sO = smem_u32(ot), sRec = smem_u32(rec), sDS = smem_u32(sm + SB_DS);
-      const uint32_t id1 = idesc_bf16(128, 64, true, true);
-      const uint32_t id2 = idesc_bf16(128, 64, false, true);
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk)
-        mma_bf16(tmem + 128, sdesc(sO + kk * 2048, 8192, 1024), sdesc(sRec + RB_R3 + kk * 2048, 8192, 1024),
-                 id1, kk > 0);
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk)
-        mma_bf16(tmem + 128, sdesc(sDS + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-                 sdesc(sRec + RB_R4 + kk * 2048, 8192, 1024), id2, true);
-      mma_commit(&ms.mu);
-    }
-    // meanwhile: dS^T <- dS^T Diag(d_j)
-    {
-      const float *dj = reinterpret_cast<const float *>(rec + RB_R5);
-      for (int c0 = 64 * ch; c0 < 64 * ch + 64; c0 += 16) {
-        float sv[16];
-        tmem_ld16(lanebase + c0, sv);
-        tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 16; ++i) sv[i] *= dj[c0 + i];
-        tmem_st16(lanebase + c0, sv);
-      }
-      tmem_wait_st();
-    }
-    {
-      bool ok = true;
-      if (tid == 0) {
-        ok = mbar_wait(&ms.mu, s & 1, a.status, 302);
-        bulk_wait_read_all();  // the previous dU tile has left its staging tile
-      }
-      if (__syncthreads_or(!ok)) { abort = true; break; }
-    }
-    tc_fence_after();
-    // dU^T -> bf16 operand tile and the dU tile of this chunk
-    {
-      for (int s0 = 32 * ch; s0 < 32 * ch + 32; s0 += 16) {
-        float w[16];
-        tmem_ld16(lanebase + 128 + s0, w);
-        tmem_wait_ld();
-        uint32_t pk[8];
-#pragma unroll
-        for (int m = 0; m < 8; ++m) pk[m] = pack_bf16(w[2 * m], w[2 * m + 1]);
-        *reinterpret_cast<uint4 *>(sm + SB_DU + kmaj_off(v, s0, 128)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-        *reinterpret_cast<uint4 *>(sm + SB_DU + kmaj_off(v, s0 + 8, 128)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) st_bf16(sm + SB_DUG, kmaj_off(s0 + i, v, 64), w[i]);
-      }
-    }
-    fence_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    if (tid == 0) {
-      bulk_s2g(ta.dU_tiles + ((size_t)(first + j) * H + h) * DU_TILE, sm + SB_DUG, DU_TILE);
-      bulk_commit();
-    }
-    // dS^T += dO^T QG - dU^T W
-    if (tid == 0) {
-      tc_fence_after();
-      const uint32_t sO = smem_u32(ot), sRec = smem_u32(rec), sDU = smem_u32(sm + SB_DU);
-      const uint32_t id1 = idesc_bf16(128, 128, true, false);
-      const uint32_t id2 = idesc_bf16(128, 128, false, false) | (1u << 13);  // negate A
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk)
-        mma_bf16(tmem, sdesc(sO + kk * 2048, 8192, 1024), sdesc(sRec + RB_R1 + 16384 + kk * 32, 16, 1024),
-                 id1, true);
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk)
-        mma_bf16(tmem, sdesc(sDU + kk * 32, 16, 1024), sdesc(sRec + RB_R1 + kk * 32, 16, 1024), id2, true);
-      mma_commit(&ms.ms);
-    }
-    {
-      bool ok = true;
-      if (tid == 0) {
-        ok = mbar_wait(&ms.ms, s & 1, a.status, 303);
-        bulk_wait_read_all();  // the last snapshot has left the dS^T tile
-      }
-      if (__syncthreads_or(!ok)) { abort = true; break; }
-    }
-    tc_fence_after();
-    if (tid == 0 && s + 2 < nc) issue_record(s + 2);
-    // dS at the start of chunk j: next step's operand, snapshot of chunk j-1, or dS0
+  if (grpA) {
+    if (nc > 0) issue_dO(0);
+    // dS_T (true frame) -> dS^T rows; bf16 copy for the MMA, fp32 in TMEM
     for (int c0 = 64 * ch; c0 < 64 * ch + 64; c0 += 16) {
       float sv[16];
-      tmem_ld16(lanebase + c0, sv);
-      tmem_wait_ld();
-      if (j == 0) {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) sv[i] = a.dST ? a.dST[sbase + (size_t)(c0 + i) * D + v] : 0.f;
+      if (nc == 0) {
         if (a.dS0)
           for (int i = 0; i < 16; ++i) a.dS0[sbase + (size_t)(c0 + i) * D + v] = sv[i];
         continue;
@@ -278,14 +169,176 @@ __global__ void __launch_bounds__(kSbThreads, 1) tc_state_bwd_kernel(BwdTcArgs t
       for (int m = 0; m < 8; ++m) pk[m] = pack_bf16(sv[2 * m], sv[2 * m + 1]);
       *reinterpret_cast<uint4 *>(sm + SB_DS + kmaj_off(v, c0, 128)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
       *reinterpret_cast<uint4 *>(sm + SB_DS + kmaj_off(v, c0 + 8, 128)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+      tmem_st16(lanebase + c0, sv);
     }
-    fence_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    if (tid == 0 && j > 0) snapshot(j - 1);
+    tmem_wait_st();
   }
-  cp_async_wait_all();
-  if (tid == 0) bulk_wait_all();  // every tile written before the kernel ends
+  fence_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  if (tid == 0 && nc > 0) snapshot(nc - 1);
+  if (grpA && nc > 0) {  // dS^T is in place: group B may scale it for step 0
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&ms.dsready);
+  }
+
+  bool abort = false;
+  if (grpA) {
+    auto wait_a = [&](uint64_t *bar, uint32_t phase, uint32_t site, bool ok_in) -> bool {
+      bool ok = ok_in;
+      if (gt == 0 && ok) ok = mbar_wait(bar, phase, a.status, site);
+      return !group_sync_or(1, kSbGroup, !ok);
+    };
+    for (int s = 0; s < nc && !abort; ++s) {
+      const int j = nc - 1 - s;
+      const int b = s & 1;
+      unsigned char *rec = rb[b];
+      unsigned char *ot = ob[b];
+      const uint32_t du = 128 + 64 * b;  // dU^T buffer of this step
+      if (s + 1 < nc) issue_dO(s + 1);  // prefetch next dO into the other buffer
+      // dO of this step landed (all but the group just committed)
+      if (s + 1 < nc) asm volatile("cp.async.wait_group 1;" ::: "memory");
+      else cp_async_wait_all();
+      fence_async_smem();
+      if (!wait_a(&ms.mrec[b], (s >> 1) & 1, 301, true)) { abort = true; break; }
+      // dU^T = dO^T A_q + dS1^T Khat^T
+      bool ok = true;
+      if (gt == 0) {
+        // group B has read the dU^T of step s - 1 (waiting for that completion
+        // rather than the one for step s - 2, whose buffer this step reuses,
+        // keeps the parity wait unambiguous: B cannot run two steps ahead)
+        if (s >= 1) ok = mbar_wait(&ms.dudone, (s - 1) & 1, a.status, 304);
+        if (ok) {
+          tc_fence_after();
+          const uint32_t sO = smem_u32(ot), sRec = smem_u32(rec), sDS = smem_u32(sm + SB_DS);
+          const uint32_t id1 = idesc_bf16(128, 64, true, true);
+          const uint32_t id2 = idesc_bf16(128, 64, false, true);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_bf16(tmem + du, sdesc(sO + kk * 2048, 8192, 1024), sdesc(sRec + RB_R3 + kk * 2048, 8192, 1024),
+                     id1, kk > 0);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_bf16(tmem + du, sdesc(sDS + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                     sdesc(sRec + RB_R4 + kk * 2048, 8192, 1024), id2, true);
+          mma_commit(&ms.mu);
+        }
+      }
+      if (!wait_a(&ms.mu, s & 1, 302, ok)) { abort = true; break; }
+      tc_fence_after();
+      // dU^T -> bf16 operand tile (group B writes the dU tile out)
+      for (int s0 = 32 * ch; s0 < 32 * ch + 32; s0 += 16) {
+        float w[16];
+        tmem_ld16(lanebase + du + s0, w);
+        tmem_wait_ld();
+        uint32_t pk[8];
+#pragma unroll
+        for (int m = 0; m < 8; ++m) pk[m] = pack_bf16(w[2 * m], w[2 * m + 1]);
+        *reinterpret_cast<uint4 *>(sm + SB_DU + kmaj_off(v, s0, 128)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        *reinterpret_cast<uint4 *>(sm + SB_DU + kmaj_off(v, s0 + 8, 128)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+      }
+      fence_async_smem();
+      tc_fence_before();
+      group_sync(1, kSbGroup);
+      // dS^T += dO^T QG - dU^T W  (dS^T scaled by group B first)
+      ok = true;
+      if (gt == 0) {
+        ok = mbar_wait(&ms.scaled, s & 1, a.status, 305);
+        if (ok) {
+          tc_fence_after();
+          const uint32_t sO = smem_u32(ot), sRec = smem_u32(rec), sDU = smem_u32(sm + SB_DU);
+          const uint32_t id1 = idesc_bf16(128, 128, true, false);
+          const uint32_t id2 = idesc_bf16(128, 128, false, false) | (1u << 13);  // negate A
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_bf16(tmem, sdesc(sO + kk * 2048, 8192, 1024), sdesc(sRec + RB_R1 + 16384 + kk * 32, 16, 1024),
+                     id1, true);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_bf16(tmem, sdesc(sDU + kk * 32, 16, 1024), sdesc(sRec + RB_R1 + kk * 32, 16, 1024), id2, true);
+          mma_commit(&ms.ms);
+        }
+        bulk_wait_read_all();  // the last snapshot has left the dS^T tile
+      }
+      if (!wait_a(&ms.ms, s & 1, 303, ok)) { abort = true; break; }
+      tc_fence_after();
+      if (gt == 0 && s + 2 < nc) issue_record(s + 2);
+      // dS at the start of chunk j: next step's operand, snapshot of chunk j-1, or dS0
+      for (int c0 = 64 * ch; c0 < 64 * ch + 64; c0 += 16) {
+        float sv[16];
+        tmem_ld16(lanebase + c0, sv);
+        tmem_wait_ld();
+        if (j == 0) {
+          if (a.dS0)
+            for (int i = 0; i < 16; ++i) a.dS0[sbase + (size_t)(c0 + i) * D + v] = sv[i];
+          continue;
+        }
+        uint32_t pk[8];
+#pragma unroll
+        for (int m = 0; m < 8; ++m) pk[m] = pack_bf16(sv[2 * m], sv[2 * m + 1]);
+        *reinterpret_cast<uint4 *>(sm + SB_DS + kmaj_off(v, c0, 128)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        *reinterpret_cast<uint4 *>(sm + SB_DS + kmaj_off(v, c0 + 8, 128)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+      }
+      fence_async_smem();
+      tc_fence_before();
+      group_sync(1, kSbGroup);
+      if (gt == 0 && j > 0) snapshot(j - 1);
+      if (j > 0) {  // dS^T has been read: group B may scale it for the next step
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ms.dsready);
+      }
+    }
+    cp_async_wait_all();
+  } else {
+    for (int s = 0; s < nc && !abort; ++s) {
+      const int b = s & 1;
+      const uint32_t du = 128 + 64 * b;
+      // dS^T <- dS^T Diag(d_j) once group A has read it
+      bool ok = mbar_wait(&ms.dsready, s & 1, a.status, 306);
+      if (ok) ok = mbar_wait(&ms.mrec[b], (s >> 1) & 1, a.status, 307);
+      if (group_sync_or(2, kSbGroup, !ok)) { abort = true; break; }
+      tc_fence_after();
+      {
+        const float *dj = reinterpret_cast<const float *>(rb[b] + RB_R5);
+        for (int c0 = 64 * ch; c0 < 64 * ch + 64; c0 += 16) {
+          float sv[16];
+          tmem_ld16(lanebase + c0, sv);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) sv[i] *= dj[c0 + i];
+          tmem_st16(lanebase + c0, sv);
+        }
+        tmem_wait_st();
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ms.scaled);
+      // the dU tile of this chunk, staged transposed ([s][v]) and bulk stored
+      ok = mbar_wait(&ms.mu, s & 1, a.status, 308);
+      if (gt == 0) bulk_wait_read_all();  // the previous dU tile has left the staging tile
+      if (group_sync_or(2, kSbGroup, !ok)) { abort = true; break; }
+      tc_fence_after();
+      for (int s0 = 32 * ch; s0 < 32 * ch + 32; s0 += 16) {
+        float w[16];
+        tmem_ld16(lanebase + du + s0, w);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) st_bf16(sm + SB_DUG, kmaj_off(s0 + i, v, 64), w[i]);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ms.dudone);
+      fence_async_smem();
+      group_sync(2, kSbGroup);
+      if (gt == 0) {
+        const int j = nc - 1 - s;
+        bulk_s2g(ta.dU_tiles + ((size_t)(first + j) * H + h) * DU_TILE, sm + SB_DUG, DU_TILE);
+        bulk_commit();
+      }
+    }
+  }
+  if (gt == 0) bulk_wait_all();  // every tile written before the kernel ends
+  __syncthreads();
   if (abort && tid == 0) {
     mma_commit(&ms.mfin);
     mbar_wait(&ms.mfin, 0, a.status, 309);
