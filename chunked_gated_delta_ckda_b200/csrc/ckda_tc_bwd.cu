@@ -502,38 +502,47 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
   // M and S_c^T, and the row tensors (q, k staged in A1, g in B1 + KG, sign in
   // TT -- the prep consumes them before those tiles are written -- V into
   // rows 64.. of [U; V] and dO into rows 0..63 of [dO; dU], K-major SW128
-  // boxes).  Issued by thread 0 once the previous item's last readers of
-  // these regions are done (its phase E), so they overlap its final epilogue.
+  // boxes).  Issued once the previous item's last readers of these regions
+  // are done (its phase E), so they overlap its final epilogue.
   // thread 0's count of issued load sets (each completes mld, mrec and mdu
   // once) and of the completions it has seen: an abort drains the rest
   uint32_t n_issued = 0, n_mld = 0, n_mrec = 0, n_mdu = 0;
+  // The copies are spread over lane 0 of warps 0..3 (each copy instruction
+  // takes a while to issue); warp 0 posts every byte count with its arrive,
+  // so the others only add copies (a transiently negative transaction count
+  // is allowed; the phase needs warp 0's arrive to complete).
   auto issue_loads = [&](int itm) {
-    ++n_issued;
     int sq_, len_, jl_;
     int64_t tk_;
     a.map.info(itm / H, sq_, tk_, len_, jl_);
     const int hh = itm % H, t = (int)tk_;
     fence_async_smem();  // earlier generic accesses of the destinations come first
-    const unsigned char *gdU = ta.dU_tiles + (size_t)itm * DU_TILE;
-    mbar_arrive_expect_tx(&ms.mdu, DU_TILE);
-    bulk_g2s(sm + G_OU + 8192, gdU, 8192, &ms.mdu);
-    bulk_g2s(sm + G_OU + 16384 + 8192, gdU + 8192, 8192, &ms.mdu);
-    const unsigned char *rec = ta.recs + (size_t)itm * REC;
-    mbar_arrive_expect_tx(&ms.mrec, W_TILE + M_BYTES + S_TILE);
-    bulk_g2s(sm + G_WN, rec + R1, W_TILE, &ms.mrec);
-    bulk_g2s(sm + G_MF, rec + R6, M_BYTES, &ms.mrec);
-    bulk_g2s(sm + G_SC, rec + R7, S_TILE, &ms.mrec);
-    mbar_arrive_expect_tx(&ms.mld, kRowBytesQK + kRowBytesG + kRowBytesSign + 2 * 16384);
-    tma_rows(sm + G_A1 + kStageQ, &ta.rm.q, 0, hh, t, &ms.mld);
-    tma_rows(sm + G_A1 + kStageQ + 8192, &ta.rm.q, 64, hh, t, &ms.mld);
-    tma_rows(sm + G_A1 + kStageK, &ta.rm.k, 0, hh, t, &ms.mld);
-    tma_rows(sm + G_A1 + kStageK + 8192, &ta.rm.k, 64, hh, t, &ms.mld);
-    tma_rows(sm + G_B1, &ta.rm.g, 0, hh, t, &ms.mld);
-    tma_rows(sm + G_TT, &ta.rm.sign, 0, hh, t, &ms.mld);
-    tma_rows(sm + G_UV + 8192, &ta.rm.v, 0, hh, t, &ms.mld);
-    tma_rows(sm + G_UV + 16384 + 8192, &ta.rm.v, 64, hh, t, &ms.mld);
-    tma_rows(sm + G_OU, &ta.rm.dO, 0, hh, t, &ms.mld);
-    tma_rows(sm + G_OU + 16384, &ta.rm.dO, 64, hh, t, &ms.mld);
+    if (warp == 0) {
+      ++n_issued;
+      const unsigned char *gdU = ta.dU_tiles + (size_t)itm * DU_TILE;
+      mbar_arrive_expect_tx(&ms.mdu, DU_TILE);
+      mbar_arrive_expect_tx(&ms.mrec, W_TILE + M_BYTES + S_TILE);
+      mbar_arrive_expect_tx(&ms.mld, kRowBytesQK + kRowBytesG + kRowBytesSign + 2 * 16384);
+      bulk_g2s(sm + G_OU + 8192, gdU, 8192, &ms.mdu);
+      bulk_g2s(sm + G_OU + 16384 + 8192, gdU + 8192, 8192, &ms.mdu);
+      const unsigned char *rec = ta.recs + (size_t)itm * REC;
+      bulk_g2s(sm + G_WN, rec + R1, W_TILE, &ms.mrec);
+      bulk_g2s(sm + G_MF, rec + R6, M_BYTES, &ms.mrec);
+      bulk_g2s(sm + G_SC, rec + R7, S_TILE, &ms.mrec);
+    } else if (warp == 1) {
+      tma_rows(sm + G_A1 + kStageQ, &ta.rm.q, 0, hh, t, &ms.mld);
+      tma_rows(sm + G_A1 + kStageQ + 8192, &ta.rm.q, 64, hh, t, &ms.mld);
+      tma_rows(sm + G_A1 + kStageK, &ta.rm.k, 0, hh, t, &ms.mld);
+      tma_rows(sm + G_A1 + kStageK + 8192, &ta.rm.k, 64, hh, t, &ms.mld);
+    } else if (warp == 2) {
+      tma_rows(sm + G_B1, &ta.rm.g, 0, hh, t, &ms.mld);
+      tma_rows(sm + G_TT, &ta.rm.sign, 0, hh, t, &ms.mld);
+      tma_rows(sm + G_UV + 8192, &ta.rm.v, 0, hh, t, &ms.mld);
+      tma_rows(sm + G_UV + 16384 + 8192, &ta.rm.v, 64, hh, t, &ms.mld);
+    } else {
+      tma_rows(sm + G_OU, &ta.rm.dO, 0, hh, t, &ms.mld);
+      tma_rows(sm + G_OU + 16384, &ta.rm.dO, 64, hh, t, &ms.mld);
+    }
   };
 
   uint32_t it = 0;
@@ -547,7 +556,7 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
     const unsigned char *gdS = ta.dS_tiles + (size_t)item * DS_TILE;
 
     // ---------------- loads ----------------
-    if (tid == 0 && it == 0) issue_loads(item);  // later items: issued during the previous one
+    if (lane == 0 && warp < 4 && it == 0) issue_loads(item);  // later items: during the previous one
     if (tid < 64) ms.beta[tid] = tid < len ? __bfloat162float(beta[(size_t)(tok0 + tid) * H + h]) : 0.f;
     if (!wait_all(&ms.mld, ph, a.status, 400)) { abort = true; break; }
     ++n_mld;
@@ -955,7 +964,7 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
     tc_fence_after();
     // every shared-memory tile is idle now: the next item's loads overlap the
     // final epilogue (TMEM, registers and the quarter sums only)
-    if (tid == 0 && item + (int)gridDim.x < nitems) issue_loads(item + gridDim.x);
+    if (lane == 0 && warp < 4 && item + (int)gridDim.x < nitems) issue_loads(item + gridDim.x);
 
     // ---------------- final elementwise gradients ----------------
     // thread (c, cq): rows 16 cq .. 16 cq + 15 of key channel c, prep values

@@ -120,18 +120,25 @@ __global__ void __launch_bounds__(kIntraThreads, 2) tc_intra_kernel(const __grid
     // q, k staged in the A1 region, g in B1 + KG, sign in T (each consumed by
     // the prep before those tiles are written); V straight into its operand
     // tile (MN-major A, K = token j, M = value channel: the box layout).
-    if (tid == 0) {
+    // (issued from lane 0 of four warps; warp 0 posts the byte count with its
+    // arrive, so the phase cannot complete before every copy has landed)
+    if (lane == 0 && warp < 4) {
       fence_async_smem();  // earlier generic accesses of these regions come first
-      mbar_arrive_expect_tx(&ms.mld, kRowBytesQK + kRowBytesG + kRowBytesSign + 16384);
       const int t = (int)tok0;
-      tma_rows(sm + I_A1 + kStageQ, &ta.rm.q, 0, h, t, &ms.mld);
-      tma_rows(sm + I_A1 + kStageQ + 8192, &ta.rm.q, 64, h, t, &ms.mld);
-      tma_rows(sm + I_A1 + kStageK, &ta.rm.k, 0, h, t, &ms.mld);
-      tma_rows(sm + I_A1 + kStageK + 8192, &ta.rm.k, 64, h, t, &ms.mld);
-      tma_rows(sm + I_B1, &ta.rm.g, 0, h, t, &ms.mld);
-      tma_rows(sm + I_T, &ta.rm.sign, 0, h, t, &ms.mld);
-      tma_rows(sm + I_V, &ta.rm.v, 0, h, t, &ms.mld);
-      tma_rows(sm + I_V + 8192, &ta.rm.v, 64, h, t, &ms.mld);
+      if (warp == 0) {
+        mbar_arrive_expect_tx(&ms.mld, kRowBytesQK + kRowBytesG + kRowBytesSign + 16384);
+        tma_rows(sm + I_A1 + kStageQ, &ta.rm.q, 0, h, t, &ms.mld);
+        tma_rows(sm + I_A1 + kStageQ + 8192, &ta.rm.q, 64, h, t, &ms.mld);
+      } else if (warp == 1) {
+        tma_rows(sm + I_A1 + kStageK, &ta.rm.k, 0, h, t, &ms.mld);
+        tma_rows(sm + I_A1 + kStageK + 8192, &ta.rm.k, 64, h, t, &ms.mld);
+      } else if (warp == 2) {
+        tma_rows(sm + I_B1, &ta.rm.g, 0, h, t, &ms.mld);
+        tma_rows(sm + I_T, &ta.rm.sign, 0, h, t, &ms.mld);
+      } else {
+        tma_rows(sm + I_V, &ta.rm.v, 0, h, t, &ms.mld);
+        tma_rows(sm + I_V + 8192, &ta.rm.v, 64, h, t, &ms.mld);
+      }
     }
     if (tid < 64) ms.beta[tid] = tid < len ? __bfloat162float(beta[(size_t)(tok0 + tid) * H + h]) : 0.f;
     {
