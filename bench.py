@@ -60,10 +60,13 @@ KERNEL_UNITS = {
     "decode": ("decode", DECODE_BYTES_PER_NH, 0),
 }
 
-# DRAM traffic per launch measured by ncu (dram__bytes_read.sum +
-# dram__bytes_write.sum) for the kernel as it stands, keyed by kernel and
-# workload; None until captured for the current kernel version.
-NCU_TRAFFIC = {}
+# DRAM traffic measured by ncu (dram__bytes_read.sum + dram__bytes_write.sum)
+# for the kernel as it stands, per chunk-head, keyed by kernel and workload:
+# captured on a B=2 launch (inputs still larger than L2), traffic being
+# proportional to the chunk-heads a launch processes (profiles/).
+NCU_TRAFFIC = {
+    ("tc_grad", "layer_fwdbwd_bf16"): (453896192 + 146766080) / (2 * 64 * 16),
+}
 
 
 # ---------------------------------------------------------------------------
@@ -251,7 +254,8 @@ def run_ours(args, rank, world, local_rank):
         achieved = alg_bytes / (t / n / 1e3) / 1e9
         roof = {"bound": "hbm", "kernel": top, "achieved": achieved, "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
-                "traffic": NCU_TRAFFIC.get((top, w.name)),
+                "traffic": (NCU_TRAFFIC[(top, w.name)] * B * ((T + 63) // 64) * H
+                            if (top, w.name) in NCU_TRAFFIC else None),
                 "algorithmic_bytes_per_launch": alg_bytes, "per_unit": "%d B per token-head (%s)" % (bytes_per, unit),
                 "peak_source": peaks["source"]}
     # whole step against both roofs
@@ -304,7 +308,7 @@ def run_secondary(args, rank, world, local_rank):
         tokens = N
         metric = "CKDA decode tokens/s (N=256,H=16,d=128,bf16 I/O,fp32 state)"
         cfg = {"workload": w.name, "N": N, "H": H, "dk": dk, "dv": dv, "io_dtype": "bf16",
-               "state_dtype": "f32", "l2": "state (512 MiB) larger than L2"}
+               "state_dtype": "f32", "l2": "state (256 MiB) larger than L2"}
     elif args.workload == "varlen":
         w = W.VARLEN
         inp = W.make_varlen(w)
