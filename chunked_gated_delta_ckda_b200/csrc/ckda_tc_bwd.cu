@@ -695,12 +695,21 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
       tc_fence_after();
       const uint32_t id1 = idesc_bf16(128, 128, true, false);  // S_c read MN-major (K = v)
       const uint32_t id2 = idesc_bf16(128, 64, true, false);   // dS1 read MN-major (K = v)
+      const uint32_t id3 = idesc_bf16(128, 128, false, false);
 #pragma unroll 1
       for (int kk = 0; kk < 8; ++kk) {
         const uint32_t ko = (kk >> 2) * 16384 + (kk & 3) * 32;
         mma_bf16(tmem + 256, sdesc(sSC + kk * 2048, 16384, 1024), sdesc(sOU + ko, 16, 1024), id1, kk > 0);
         mma_bf16(tmem + 384, sdesc(sWN + kk * 2048, 16384, 1024), sdesc(sUV + ko, 16, 1024), id2, kk > 0);
+        // D7, first part: [dO; dU][U; V]^T (needs neither dW nor the epilogue below)
+        mma_bf16(tmem + 128, sdesc(sOU + ko, 16, 1024), sdesc(sUV + ko, 16, 1024), id3, kk > 0);
       }
+      // dV^T = dU^T T^T (T and dU are in place)
+      const uint32_t idT = idesc_bf16(128, 64, true, true);
+#pragma unroll 1
+      for (int kk = 0; kk < 4; ++kk)
+        mma_bf16(tmem + 448, sdesc(sOU + 8192 + kk * 2048, 16384, 1024), sdesc(sTT + kk * 2048, 8192, 1024), idT,
+                 kk > 0);
       mma_commit(&ms.bar[3]);
     }
     if (!wait_one(&ms.bar[3], ph, a.status, 406)) { abort = true; break; }
@@ -716,20 +725,20 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
     tc_fence_before();
     __syncthreads();
 
-    // ---------------- D7 = [dO; dU][U; V]^T + [.; dW] KG^T ----------------
+    // ---------------- D7 = [dO; dU][U; V]^T + [.; dW] KG^T (second part), dKG^T ----------------
     if (tid == 0) {
       tc_fence_after();
-      const uint32_t id1 = idesc_bf16(128, 128, false, false);
       const uint32_t id2 = idesc_bf16(128, 64, false, false);
-#pragma unroll 1
-      for (int kk = 0; kk < 8; ++kk) {
-        const uint32_t ko = (kk >> 2) * 16384 + (kk & 3) * 32;
-        mma_bf16(tmem + 128, sdesc(sOU + ko, 16, 1024), sdesc(sUV + ko, 16, 1024), id1, kk > 0);
-      }
 #pragma unroll 1
       for (int kk = 0; kk < 8; ++kk)
         mma_bf16(tmem + 192, sdesc(sSC + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
                  sdesc(sKG + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), id2, true);
+      // dKG^T = dW^T T^T (dW just written)
+      const uint32_t idT = idesc_bf16(128, 64, true, true);
+#pragma unroll 1
+      for (int kk = 0; kk < 4; ++kk)
+        mma_bf16(tmem + 64, sdesc(sSC + 8192 + kk * 2048, 16384, 1024), sdesc(sTT + kk * 2048, 8192, 1024), idT,
+                 kk > 0);
       mma_commit(&ms.bar[4]);
     }
     if (!wait_one(&ms.bar[4], ph, a.status, 407)) { abort = true; break; }
@@ -902,16 +911,9 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
     tc_fence_before();
     __syncthreads();
 
-    // ---------------- dV^T, dKG^T, X^T, Y^T ----------------
+    // ---------------- X^T, Y^T (dV^T and dKG^T were issued earlier) ----------------
     if (tid == 0) {
       tc_fence_after();
-      const uint32_t idT = idesc_bf16(128, 64, true, true);
-#pragma unroll 1
-      for (int kk = 0; kk < 4; ++kk) {
-        const uint64_t bd = sdesc(sTT + kk * 2048, 8192, 1024);
-        mma_bf16(tmem + 448, sdesc(sOU + 8192 + kk * 2048, 16384, 1024), bd, idT, kk > 0);
-        mma_bf16(tmem + 64, sdesc(sSC + 8192 + kk * 2048, 16384, 1024), bd, idT, kk > 0);
-      }
       if (fast) {
         const uint32_t idX = idesc_bf16(128, 128, true, false);
 #pragma unroll 1

@@ -122,13 +122,14 @@ def test_backward_uses_saved_chunk_states():
         check(key, a[key], f64(b[key]), io)
 
 
-@pytest.mark.parametrize("with_cs", [True, False])
-def test_backward_with_saved_forward_results(with_cs):
+@pytest.mark.parametrize("with_cs,gscale", [(True, 0.3), (False, 0.3), (False, 3.0)])
+def test_backward_with_saved_forward_results(with_cs, gscale):
     """The forward's saved per-chunk results stand in for the backward's
     recomputation: same kernel on the same inputs, so the gradients are
-    bit-identical; and they match the oracle."""
+    bit-identical; and they match the oracle (gscale 3: chunks on the exact
+    per-pair path)."""
     io = torch.bfloat16
-    inp = random_inputs(2, 300, 2, 128, 128, io, seed=13, gscale=0.3, extreme_p=0.05)
+    inp = random_inputs(2, 300, 2, 128, 128, io, seed=13, gscale=gscale, extreme_p=0.05)
     d = to_dev(inp)
     S0, dST = inp["S0"].cuda(), inp["dST"].cuda()
     o, ST, cs, sv = api.chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["sign"], d["beta"], S0=S0,
