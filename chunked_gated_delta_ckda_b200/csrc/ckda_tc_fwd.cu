@@ -54,6 +54,10 @@ constexpr uint32_t I_T = 81920;       // T          K-major 64 x 64         8 Ki
 constexpr uint32_t I_MISC = 90112;    // small arrays
 constexpr uint32_t I_NF = 0;          // fp32 N [64][65]  (reuses A1 after MMA1)
 constexpr uint32_t I_MF = 16640;      // fp32 M [64][65]  (reuses A1/B1 after MMA1)
+// record tiles staged in shared memory and written out by bulk copies
+constexpr uint32_t I_AQS = 34816;     // A_q, K-major [r][s] 64 x 64 (in B1, free after MMA1)
+constexpr uint32_t I_WS = I_KG;       // W^T, MN-major [c][r]  (KG, free after MMA2)
+constexpr uint32_t I_US = I_V;        // U0^T, K-major [v][s]   (V, free after MMA2)
 constexpr int LDF = 65;
 
 struct IntraMisc {
@@ -269,11 +273,16 @@ __global__ void __launch_bounds__(kIntraThreads, 2) tc_intra_kernel(const __grid
         }
 #pragma unroll
         for (int m = 0; m < 4; ++m)
-          *reinterpret_cast<uint4 *>(rec + R3 + kmaj_off(r, 32 * ch + 8 * m, 64)) =
+          *reinterpret_cast<uint4 *>(sm + I_AQS + kmaj_off(r, 32 * ch + 8 * m, 64)) =
               make_uint4(pk[4 * m], pk[4 * m + 1], pk[4 * m + 2], pk[4 * m + 3]);
       }
+      fence_async_smem();
       tc_fence_before();
       __syncthreads();  // all TMEM reads of MMA1's accumulator done before A1 is reused
+      if (tid == 0) {
+        bulk_s2g(rec + R3, sm + I_AQS, 8192);
+        bulk_commit();
+      }
       if (L >= 64) {
         const int r = L - 64;
         const float br = ms.beta[r];
@@ -297,7 +306,13 @@ __global__ void __launch_bounds__(kIntraThreads, 2) tc_intra_kernel(const __grid
             aq += fb[128 * D + r * D + cc] * ks;
           }
         Nf[r * LDF + s] = s < r ? ms.beta[r] * aa : 0.f;
-        st_bf16(rec, R3 + kmaj_off(r, s, 64), s <= r ? aq : 0.f);
+        st_bf16(sm + I_AQS, kmaj_off(r, s, 64), s <= r ? aq : 0.f);
+      }
+      fence_async_smem();
+      __syncthreads();
+      if (tid == 0) {
+        bulk_s2g(rec + R3, sm + I_AQS, 8192);
+        bulk_commit();
       }
     }
     __syncthreads();
@@ -315,11 +330,12 @@ __global__ void __launch_bounds__(kIntraThreads, 2) tc_intra_kernel(const __grid
       *reinterpret_cast<uint4 *>(sm + I_T + kmaj_off(r, j0, 64)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
       *reinterpret_cast<uint4 *>(sm + I_T + kmaj_off(r, j0 + 8, 64)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
     }
-    // M itself goes to the record too: the backward starts from it
-    for (int i = tid; i < 64 * LDF / 4; i += kIntraThreads)
-      reinterpret_cast<float4 *>(rec + R6)[i] = reinterpret_cast<const float4 *>(Mf)[i];
     fence_async_smem();
     __syncthreads();
+    if (tid == 0) {  // M itself goes to the record too: the backward starts from it
+      bulk_s2g(rec + R6, Mf, 64 * LDF * 4);
+      bulk_commit();
+    }
 
     // ---------------- W^T = KG^T T^T, U0^T = V^T T^T ----------------
     if (tid == 0) {
@@ -354,7 +370,7 @@ __global__ void __launch_bounds__(kIntraThreads, 2) tc_intra_kernel(const __grid
       for (int j = 0; j < 8; ++j) pk[8 + j] = pack_bf16(y[2 * j], y[2 * j + 1]);
 #pragma unroll
       for (int m = 0; m < 4; ++m)
-        *reinterpret_cast<uint4 *>(rec + R1 + mnmaj_off(L, 32 * ch + 8 * m, 128)) =
+        *reinterpret_cast<uint4 *>(sm + I_WS + mnmaj_off(L, 32 * ch + 8 * m, 128)) =
             make_uint4(pk[4 * m], pk[4 * m + 1], pk[4 * m + 2], pk[4 * m + 3]);
       tmem_ld16(lanebase + 128 + 32 * ch, x);
       tmem_ld16(lanebase + 128 + 32 * ch + 16, y);
@@ -365,12 +381,23 @@ __global__ void __launch_bounds__(kIntraThreads, 2) tc_intra_kernel(const __grid
       for (int j = 0; j < 8; ++j) pk[8 + j] = pack_bf16(y[2 * j], y[2 * j + 1]);
 #pragma unroll
       for (int m = 0; m < 4; ++m)
-        *reinterpret_cast<uint4 *>(rec + R2 + kmaj_off(L, 32 * ch + 8 * m, 128)) =
+        *reinterpret_cast<uint4 *>(sm + I_US + kmaj_off(L, 32 * ch + 8 * m, 128)) =
             make_uint4(pk[4 * m], pk[4 * m + 1], pk[4 * m + 2], pk[4 * m + 3]);
     }
+    fence_async_smem();
     tc_fence_before();
     __syncthreads();
+    if (tid == 0) {
+      // W^T and U0^T out; every staged tile has left shared memory before the
+      // next item's loads land there
+      bulk_s2g(rec + R1, sm + I_WS, 16384);
+      bulk_s2g(rec + R2, sm + I_US, 16384);
+      bulk_commit();
+      bulk_wait_read_all();
+    }
+    __syncthreads();
   }
+  if (tid == 0) bulk_wait_all();  // every record tile written before the kernel ends
   // wind down: make sure no MMA is still writing TMEM before freeing it
   if (abort && tid == 0) {
     mma_commit(&ms.mfin);
