@@ -218,6 +218,13 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo_bytes, ui
   return d;
 }
 
+// The same descriptor for the tile `byte_off` bytes further on (a multiple of
+// 16): only the 14-bit start-address field moves, and shared-memory
+// addresses stay below 2^18, so the add never carries out of it.  Lets one
+// thread issue a run of MMAs with one add per operand instead of rebuilding
+// each 64-bit descriptor.
+__device__ __forceinline__ uint64_t sdesc_off(uint64_t d, uint32_t byte_off) { return d + (byte_off >> 4); }
+
 // byte offset of element (row, col) inside a K-major SW128 tile whose rows
 // are `rows` long groups of 64 columns (col may exceed 63: next 64-col block)
 __host__ __device__ __forceinline__ uint32_t kmaj_off(int row, int col, int rows) {

@@ -215,12 +215,12 @@ __global__ void __launch_bounds__(kSbThreads, 1) tc_state_bwd_kernel(BwdTcArgs t
           const uint32_t id2 = idesc_bf16(128, 64, false, true);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            mma_bf16(tmem + du, sdesc(sO + kk * 2048, 8192, 1024), sdesc(sRec + RB_R3 + kk * 2048, 8192, 1024),
+            mma_bf16(tmem + du, sdesc_off(sdesc(sO, 8192, 1024), kk * 2048), sdesc_off(sdesc(sRec + RB_R3, 8192, 1024), kk * 2048),
                      id1, kk > 0);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            mma_bf16(tmem + du, sdesc(sDS + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-                     sdesc(sRec + RB_R4 + kk * 2048, 8192, 1024), id2, true);
+            mma_bf16(tmem + du, sdesc_off(sdesc(sDS, 16, 1024), (kk >> 2) * 16384 + (kk & 3) * 32),
+                     sdesc_off(sdesc(sRec + RB_R4, 8192, 1024), kk * 2048), id2, true);
           mma_commit(&ms.mu);
         }
       }
@@ -251,11 +251,11 @@ __global__ void __launch_bounds__(kSbThreads, 1) tc_state_bwd_kernel(BwdTcArgs t
           const uint32_t id2 = idesc_bf16(128, 128, false, false) | (1u << 13);  // negate A
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            mma_bf16(tmem, sdesc(sO + kk * 2048, 8192, 1024), sdesc(sRec + RB_R1 + 16384 + kk * 32, 16, 1024),
+            mma_bf16(tmem, sdesc_off(sdesc(sO, 8192, 1024), kk * 2048), sdesc_off(sdesc(sRec + RB_R1 + 16384, 16, 1024), kk * 32),
                      id1, true);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            mma_bf16(tmem, sdesc(sDU + kk * 32, 16, 1024), sdesc(sRec + RB_R1 + kk * 32, 16, 1024), id2, true);
+            mma_bf16(tmem, sdesc_off(sdesc(sDU, 16, 1024), kk * 32), sdesc_off(sdesc(sRec + RB_R1, 16, 1024), kk * 32), id2, true);
           mma_commit(&ms.ms);
         }
         bulk_wait_read_all();  // the last snapshot has left the dS^T tile
@@ -626,21 +626,21 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
       tc_fence_after();
       if (fast) {
         const uint32_t id = idesc_bf16(128, 64, false, false);
-#pragma unroll 1
+#pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_bf16(tmem, sdesc(sA1 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-                   sdesc(sB1 + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), id, kk > 0);
+          mma_bf16(tmem, sdesc_off(sdesc(sA1, 16, 1024), (kk >> 2) * 16384 + (kk & 3) * 32),
+                   sdesc_off(sdesc(sB1, 16, 1024), (kk >> 2) * 8192 + (kk & 3) * 32), id, kk > 0);
       }
       const uint32_t idu = idesc_bf16(128, 64, true, false);
-#pragma unroll 1
+#pragma unroll
       for (int kk = 0; kk < 4; ++kk)
-        mma_bf16(tmem + 128, sdesc(sUV + 8192 + kk * 2048, 16384, 1024), sdesc(sTT + kk * 32, 16, 1024), idu,
+        mma_bf16(tmem + 128, sdesc_off(sdesc(sUV + 8192, 16384, 1024), kk * 2048), sdesc_off(sdesc(sTT, 16, 1024), kk * 32), idu,
                  kk > 0);
       const uint32_t idw = idesc_bf16(128, 64, false, true) | (1u << 13);  // negate A: subtract
-#pragma unroll 1
+#pragma unroll
       for (int kk = 0; kk < 8; ++kk)
-        mma_bf16(tmem + 128, sdesc(sSC + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-                 sdesc(sWN + kk * 2048, 16384, 1024), idw, true);
+        mma_bf16(tmem + 128, sdesc_off(sdesc(sSC, 16, 1024), (kk >> 2) * 16384 + (kk & 3) * 32),
+                 sdesc_off(sdesc(sWN, 16384, 1024), kk * 2048), idw, true);
       mma_commit(&ms.bar[2]);
     }
     if (!wait_one(&ms.bar[2], ph, a.status, 403)) { abort = true; break; }
@@ -663,9 +663,9 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
     if (tid == 0) {
       tc_fence_after();
       const uint32_t id = idesc_bf16(128, 128, true, true);
-#pragma unroll 1
+#pragma unroll
       for (int kk = 0; kk < 8; ++kk)
-        mma_bf16(tmem + 256, sdesc(sSC + kk * 2048, 16384, 1024), sdesc(sWN + kk * 2048, 16384, 1024), id,
+        mma_bf16(tmem + 256, sdesc_off(sdesc(sSC, 16384, 1024), kk * 2048), sdesc_off(sdesc(sWN, 16384, 1024), kk * 2048), id,
                  kk > 0);
       mma_commit(&ms.bar[6]);
     }
@@ -696,19 +696,19 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
       const uint32_t id1 = idesc_bf16(128, 128, true, false);  // S_c read MN-major (K = v)
       const uint32_t id2 = idesc_bf16(128, 64, true, false);   // dS1 read MN-major (K = v)
       const uint32_t id3 = idesc_bf16(128, 128, false, false);
-#pragma unroll 1
+#pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
         const uint32_t ko = (kk >> 2) * 16384 + (kk & 3) * 32;
-        mma_bf16(tmem + 256, sdesc(sSC + kk * 2048, 16384, 1024), sdesc(sOU + ko, 16, 1024), id1, kk > 0);
-        mma_bf16(tmem + 384, sdesc(sWN + kk * 2048, 16384, 1024), sdesc(sUV + ko, 16, 1024), id2, kk > 0);
+        mma_bf16(tmem + 256, sdesc_off(sdesc(sSC, 16384, 1024), kk * 2048), sdesc_off(sdesc(sOU, 16, 1024), ko), id1, kk > 0);
+        mma_bf16(tmem + 384, sdesc_off(sdesc(sWN, 16384, 1024), kk * 2048), sdesc_off(sdesc(sUV, 16, 1024), ko), id2, kk > 0);
         // D7, first part: [dO; dU][U; V]^T (needs neither dW nor the epilogue below)
-        mma_bf16(tmem + 128, sdesc(sOU + ko, 16, 1024), sdesc(sUV + ko, 16, 1024), id3, kk > 0);
+        mma_bf16(tmem + 128, sdesc_off(sdesc(sOU, 16, 1024), ko), sdesc_off(sdesc(sUV, 16, 1024), ko), id3, kk > 0);
       }
       // dV^T = dU^T T^T (T and dU are in place)
       const uint32_t idT = idesc_bf16(128, 64, true, true);
-#pragma unroll 1
+#pragma unroll
       for (int kk = 0; kk < 4; ++kk)
-        mma_bf16(tmem + 448, sdesc(sOU + 8192 + kk * 2048, 16384, 1024), sdesc(sTT + kk * 2048, 8192, 1024), idT,
+        mma_bf16(tmem + 448, sdesc_off(sdesc(sOU + 8192, 16384, 1024), kk * 2048), sdesc_off(sdesc(sTT, 8192, 1024), kk * 2048), idT,
                  kk > 0);
       mma_commit(&ms.bar[3]);
     }
@@ -729,15 +729,15 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
     if (tid == 0) {
       tc_fence_after();
       const uint32_t id2 = idesc_bf16(128, 64, false, false);
-#pragma unroll 1
+#pragma unroll
       for (int kk = 0; kk < 8; ++kk)
-        mma_bf16(tmem + 192, sdesc(sSC + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-                 sdesc(sKG + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), id2, true);
+        mma_bf16(tmem + 192, sdesc_off(sdesc(sSC, 16, 1024), (kk >> 2) * 16384 + (kk & 3) * 32),
+                 sdesc_off(sdesc(sKG, 16, 1024), (kk >> 2) * 8192 + (kk & 3) * 32), id2, true);
       // dKG^T = dW^T T^T (dW just written)
       const uint32_t idT = idesc_bf16(128, 64, true, true);
-#pragma unroll 1
+#pragma unroll
       for (int kk = 0; kk < 4; ++kk)
-        mma_bf16(tmem + 64, sdesc(sSC + 8192 + kk * 2048, 16384, 1024), sdesc(sTT + kk * 2048, 8192, 1024), idT,
+        mma_bf16(tmem + 64, sdesc_off(sdesc(sSC + 8192, 16384, 1024), kk * 2048), sdesc_off(sdesc(sTT, 8192, 1024), kk * 2048), idT,
                  kk > 0);
       mma_commit(&ms.bar[4]);
     }
@@ -800,12 +800,12 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
     if (tid == 0) {
       tc_fence_after();
       const uint32_t id = idesc_bf16(128, 64, false, false);
-#pragma unroll 1
+#pragma unroll
       for (int p = 0; p < 3; ++p) {
         const uint32_t pa = smem_u32(sm + (p == 2 ? G_DML : G_DMH)), pb = smem_u32(sm + (p == 1 ? G_ML : G_MH));
-#pragma unroll 1
+#pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_bf16(tmem + 128, sdesc(pa + kk * 32, 16, 1024), sdesc(pb + kk * 32, 16, 1024), id, p > 0 || kk > 0);
+          mma_bf16(tmem + 128, sdesc_off(sdesc(pa, 16, 1024), kk * 32), sdesc_off(sdesc(pb, 16, 1024), kk * 32), id, p > 0 || kk > 0);
       }
       mma_commit(&ms.bar[0]);
     }
@@ -843,12 +843,12 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
     if (tid == 0) {
       tc_fence_after();
       const uint32_t id = idesc_bf16(128, 64, true, true) | (1u << 13);
-#pragma unroll 1
+#pragma unroll
       for (int p = 0; p < 3; ++p) {
         const uint32_t pa = smem_u32(sm + (p == 2 ? G_ML : G_MH)), pb = smem_u32(sm + (p == 1 ? G_TL : G_TH));
-#pragma unroll 1
+#pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_bf16(tmem + 192, sdesc(pa + kk * 2048, 8192, 1024), sdesc(pb + kk * 2048, 8192, 1024), id,
+          mma_bf16(tmem + 192, sdesc_off(sdesc(pa, 8192, 1024), kk * 2048), sdesc_off(sdesc(pb, 8192, 1024), kk * 2048), id,
                    p > 0 || kk > 0);
       }
       mma_commit(&ms.bar[1]);
@@ -916,17 +916,17 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
       tc_fence_after();
       if (fast) {
         const uint32_t idX = idesc_bf16(128, 128, true, false);
-#pragma unroll 1
+#pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_bf16(tmem + 128, sdesc(sB1 + kk * 2048, 8192, 1024), sdesc(sWN + kk * 32, 16, 1024), idX, kk > 0);
+          mma_bf16(tmem + 128, sdesc_off(sdesc(sB1, 8192, 1024), kk * 2048), sdesc_off(sdesc(sWN, 16, 1024), kk * 32), idX, kk > 0);
         const uint32_t idY = idesc_bf16(128, 64, true, true);
-#pragma unroll 1
+#pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_bf16(tmem + 320, sdesc(sA1 + 8192 + kk * 2048, 16384, 1024), sdesc(sWN + kk * 2048, 8192, 1024),
+          mma_bf16(tmem + 320, sdesc_off(sdesc(sA1 + 8192, 16384, 1024), kk * 2048), sdesc_off(sdesc(sWN, 8192, 1024), kk * 2048),
                    idY, kk > 0);
-#pragma unroll 1
+#pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_bf16(tmem + 320, sdesc(sA1 + kk * 2048, 16384, 1024), sdesc(sWN + 8192 + kk * 2048, 8192, 1024),
+          mma_bf16(tmem + 320, sdesc_off(sdesc(sA1, 16384, 1024), kk * 2048), sdesc_off(sdesc(sWN + 8192, 8192, 1024), kk * 2048),
                    idY, true);
       }
       mma_commit(&ms.bar[5]);

@@ -245,8 +245,8 @@ __global__ void __launch_bounds__(kIntraThreads, 2) tc_intra_kernel(const __grid
         const uint32_t id = idesc_bf16(128, 64, false, false);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t ad = sdesc(sA1 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-          const uint64_t bd = sdesc(sB1 + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024);
+          const uint64_t ad = sdesc_off(sdesc(sA1, 16, 1024), (kk >> 2) * 16384 + (kk & 3) * 32);
+          const uint64_t bd = sdesc_off(sdesc(sB1, 16, 1024), (kk >> 2) * 8192 + (kk & 3) * 32);
           mma_bf16(tmem, ad, bd, id, kk > 0);
         }
         mma_commit(&ms.mbar1);
@@ -343,9 +343,9 @@ __global__ void __launch_bounds__(kIntraThreads, 2) tc_intra_kernel(const __grid
       const uint32_t id = idesc_bf16(128, 64, true, false);
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk) {
-        const uint64_t bd = sdesc(sT + kk * 32, 16, 1024);
-        mma_bf16(tmem + 64, sdesc(sKG + kk * 2048, 8192, 1024), bd, id, kk > 0);
-        mma_bf16(tmem + 128, sdesc(sV + kk * 2048, 8192, 1024), bd, id, kk > 0);
+        const uint64_t bd = sdesc_off(sdesc(sT, 16, 1024), kk * 32);
+        mma_bf16(tmem + 64, sdesc_off(sdesc(sKG, 8192, 1024), kk * 2048), bd, id, kk > 0);
+        mma_bf16(tmem + 128, sdesc_off(sdesc(sV, 8192, 1024), kk * 2048), bd, id, kk > 0);
       }
       mma_commit(&ms.mbar2);
     }
@@ -481,8 +481,8 @@ __global__ void __launch_bounds__(kStateThreads, 1) tc_state_kernel(TcArgs ta) {
     const uint32_t sS = smem_u32(sm + S_TS), sR = smem_u32(recbuf[j & 1] + R1);
 #pragma unroll
     for (int kk = 0; kk < 8; ++kk)
-      mma_bf16(tmem + 128 + 128 * (j & 1), sdesc(sS + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-               sdesc(sR + kk * 2048, 16384, 1024), id, kk > 0);
+      mma_bf16(tmem + 128 + 128 * (j & 1), sdesc_off(sdesc(sS, 16, 1024), (kk >> 2) * 16384 + (kk & 3) * 32),
+               sdesc_off(sdesc(sR, 16384, 1024), kk * 2048), id, kk > 0);
     mma_commit(&ms.m3);
   };
   if (tid == 0) {
@@ -581,9 +581,9 @@ __global__ void __launch_bounds__(kStateThreads, 1) tc_state_kernel(TcArgs ta) {
           const uint32_t id5 = idesc_bf16(128, 128, false, false);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t ad = sdesc(sU + kk * 32, 16, 1024);
-            mma_bf16(tmem + acc + 64, ad, sdesc(smem_u32(rec + R3) + kk * 32, 16, 1024), id4, true);
-            mma_bf16(tmem + 0, ad, sdesc(smem_u32(rec + R4) + kk * 32, 16, 1024), id5, true);
+            const uint64_t ad = sdesc_off(sdesc(sU, 16, 1024), kk * 32);
+            mma_bf16(tmem + acc + 64, ad, sdesc_off(sdesc(smem_u32(rec + R3), 16, 1024), kk * 32), id4, true);
+            mma_bf16(tmem + 0, ad, sdesc_off(sdesc(smem_u32(rec + R4), 16, 1024), kk * 32), id5, true);
           }
           mma_commit(&ms.m4);
         }
