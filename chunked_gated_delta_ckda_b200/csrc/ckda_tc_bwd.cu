@@ -467,10 +467,14 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
   __nv_bfloat16 *dv = (__nv_bfloat16 *)a.dvg, *dbeta = (__nv_bfloat16 *)a.dbeta;
 
   if (tid == 0) {
-    for (int i = 0; i < 7; ++i) mbar_init(&ms.bar[i], 1);
+    // MMA groups that do not share an accumulator are issued by lane 0 of up
+    // to three warps (a tcgen05.mma takes tens of ns to issue): each such
+    // barrier counts one commit per issuing thread
+    const uint32_t issuers[7] = {1, 1, 2, 3, 2, 2, 1};
+    for (int i = 0; i < 7; ++i) mbar_init(&ms.bar[i], issuers[i]);
     mbar_init(&ms.mdu, 1);
     mbar_init(&ms.mds, 1);
-    mbar_init(&ms.mfin, 1);
+    mbar_init(&ms.mfin, 3);
     mbar_init(&ms.mrec, 1);
     mbar_init(&ms.mld, 1);
     mbar_fence_init();
@@ -621,8 +625,7 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
     __syncthreads();
 
     // ---------------- A (kept in TMEM for dbeta), U^T = V^T T^T - (W S)^T ----------------
-    // A's MMA completes before any later commit fires, which covers its reads.
-    if (tid == 0) {
+    if (tid == 32) {  // A, by a second thread (its commit is part of this phase)
       tc_fence_after();
       if (fast) {
         const uint32_t id = idesc_bf16(128, 64, false, false);
@@ -631,6 +634,10 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
           mma_bf16(tmem, sdesc_off(sdesc(sA1, 16, 1024), (kk >> 2) * 16384 + (kk & 3) * 32),
                    sdesc_off(sdesc(sB1, 16, 1024), (kk >> 2) * 8192 + (kk & 3) * 32), id, kk > 0);
       }
+      mma_commit(&ms.bar[2]);
+    }
+    if (tid == 0) {
+      tc_fence_after();
       const uint32_t idu = idesc_bf16(128, 64, true, false);
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)
@@ -691,25 +698,38 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
     __syncthreads();
 
     // ---------------- [dQG^T | S dU^T], dKhat^T ----------------
+    // (three independent groups, three issuing threads)
     if (tid == 0) {
       tc_fence_after();
       const uint32_t id1 = idesc_bf16(128, 128, true, false);  // S_c read MN-major (K = v)
-      const uint32_t id2 = idesc_bf16(128, 64, true, false);   // dS1 read MN-major (K = v)
-      const uint32_t id3 = idesc_bf16(128, 128, false, false);
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const uint32_t ko = (kk >> 2) * 16384 + (kk & 3) * 32;
-        mma_bf16(tmem + 256, sdesc_off(sdesc(sSC, 16384, 1024), kk * 2048), sdesc_off(sdesc(sOU, 16, 1024), ko), id1, kk > 0);
-        mma_bf16(tmem + 384, sdesc_off(sdesc(sWN, 16384, 1024), kk * 2048), sdesc_off(sdesc(sUV, 16, 1024), ko), id2, kk > 0);
-        // D7, first part: [dO; dU][U; V]^T (needs neither dW nor the epilogue below)
-        mma_bf16(tmem + 128, sdesc_off(sdesc(sOU, 16, 1024), ko), sdesc_off(sdesc(sUV, 16, 1024), ko), id3, kk > 0);
-      }
+      for (int kk = 0; kk < 8; ++kk)
+        mma_bf16(tmem + 256, sdesc_off(sdesc(sSC, 16384, 1024), kk * 2048),
+                 sdesc_off(sdesc(sOU, 16, 1024), (kk >> 2) * 16384 + (kk & 3) * 32), id1, kk > 0);
+      mma_commit(&ms.bar[3]);
+    } else if (tid == 32) {
+      tc_fence_after();
+      const uint32_t id2 = idesc_bf16(128, 64, true, false);   // dS1 read MN-major (K = v)
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk)
+        mma_bf16(tmem + 384, sdesc_off(sdesc(sWN, 16384, 1024), kk * 2048),
+                 sdesc_off(sdesc(sUV, 16, 1024), (kk >> 2) * 16384 + (kk & 3) * 32), id2, kk > 0);
       // dV^T = dU^T T^T (T and dU are in place)
       const uint32_t idT = idesc_bf16(128, 64, true, true);
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)
-        mma_bf16(tmem + 448, sdesc_off(sdesc(sOU + 8192, 16384, 1024), kk * 2048), sdesc_off(sdesc(sTT, 8192, 1024), kk * 2048), idT,
-                 kk > 0);
+        mma_bf16(tmem + 448, sdesc_off(sdesc(sOU + 8192, 16384, 1024), kk * 2048),
+                 sdesc_off(sdesc(sTT, 8192, 1024), kk * 2048), idT, kk > 0);
+      mma_commit(&ms.bar[3]);
+    } else if (tid == 64) {
+      tc_fence_after();
+      // D7, first part: [dO; dU][U; V]^T (needs neither dW nor the epilogue below)
+      const uint32_t id3 = idesc_bf16(128, 128, false, false);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t ko = (kk >> 2) * 16384 + (kk & 3) * 32;
+        mma_bf16(tmem + 128, sdesc_off(sdesc(sOU, 16, 1024), ko), sdesc_off(sdesc(sUV, 16, 1024), ko), id3, kk > 0);
+      }
       mma_commit(&ms.bar[3]);
     }
     if (!wait_one(&ms.bar[3], ph, a.status, 406)) { abort = true; break; }
@@ -733,6 +753,9 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
       for (int kk = 0; kk < 8; ++kk)
         mma_bf16(tmem + 192, sdesc_off(sdesc(sSC, 16, 1024), (kk >> 2) * 16384 + (kk & 3) * 32),
                  sdesc_off(sdesc(sKG, 16, 1024), (kk >> 2) * 8192 + (kk & 3) * 32), id2, true);
+      mma_commit(&ms.bar[4]);
+    } else if (tid == 32) {
+      tc_fence_after();
       // dKG^T = dW^T T^T (dW just written)
       const uint32_t idT = idesc_bf16(128, 64, true, true);
 #pragma unroll
@@ -919,6 +942,11 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
           mma_bf16(tmem + 128, sdesc_off(sdesc(sB1, 8192, 1024), kk * 2048), sdesc_off(sdesc(sWN, 16, 1024), kk * 32), idX, kk > 0);
+      }
+      mma_commit(&ms.bar[5]);
+    } else if (tid == 32) {
+      tc_fence_after();
+      if (fast) {
         const uint32_t idY = idesc_bf16(128, 64, true, true);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
@@ -1047,6 +1075,7 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
     tc_fence_before();
     __syncthreads();
   }
+  if (abort && (tid == 32 || tid == 64)) mma_commit(&ms.mfin);
   if (abort && tid == 0) {
     mma_commit(&ms.mfin);
     mbar_wait(&ms.mfin, 0, a.status, 409);
