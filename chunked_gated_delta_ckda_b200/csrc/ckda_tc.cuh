@@ -104,6 +104,10 @@ __device__ __forceinline__ void bulk_s2g(void *gmem_dst, const void *smem_src, u
                "r"(smem_u32(smem_src)), "r"(bytes)
                : "memory");
 }
+// L2 prefetch of a 16-byte aligned range (size % 16 == 0), fire and forget.
+__device__ __forceinline__ void prefetch_l2(const void *p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_read_all() {
   asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");

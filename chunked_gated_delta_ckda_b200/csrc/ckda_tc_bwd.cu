@@ -20,6 +20,7 @@
 // in TMEM, lanes = value channel) writes per chunk the dL/dS_{c+1} and dU
 // tiles; tc_grad_kernel (persistent, one CTA per SM) does everything else.
 #include <cmath>
+#include <type_traits>
 
 #include "ckda_tc.cuh"
 
@@ -533,6 +534,8 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
       bulk_g2s(sm + G_WN, rec + R1, W_TILE, &ms.mrec);
       bulk_g2s(sm + G_MF, rec + R6, M_BYTES, &ms.mrec);
       bulk_g2s(sm + G_SC, rec + R7, S_TILE, &ms.mrec);
+      // the reverse pass's dS tile is copied in mid-item: have it in L2 by then
+      prefetch_l2(ta.dS_tiles + (size_t)itm * DS_TILE, DS_TILE);
     } else if (warp == 1) {
       tma_rows(sm + G_A1 + kStageQ, &ta.rm.q, 0, hh, t, &ms.mld);
       tma_rows(sm + G_A1 + kStageQ + 8192, &ta.rm.q, 64, hh, t, &ms.mld);
@@ -561,7 +564,9 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
 
     // ---------------- loads ----------------
     if (lane == 0 && warp < 4 && it == 0) issue_loads(item);  // later items: during the previous one
-    if (tid < 64) ms.beta[tid] = tid < len ? __bfloat162float(beta[(size_t)(tok0 + tid) * H + h]) : 0.f;
+    // beta rows: loaded here for the first item, during the previous item's
+    // final epilogue for the others
+    if (it == 0 && tid < 64) ms.beta[tid] = tid < len ? __bfloat162float(beta[(size_t)(tok0 + tid) * H + h]) : 0.f;
     if (!wait_all(&ms.mld, ph, a.status, 400)) { abort = true; break; }
     ++n_mld;
     PrepC P;
@@ -1005,8 +1010,21 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
       const float eGm = fast_exp(P.Gm), eCm = fast_exp(P.GC - P.Gm);
       const float dC = pCs * fast_exp(P.GC);
       const size_t rstride = (size_t)H * D;
+      // the next item's beta, requested now and stored after the loop below
+      float beta_next = 0.f;
+      const int nxt = item + gridDim.x;
+      if (tid < 64 && nxt < nitems) {
+        int sq_, len_, jl_;
+        int64_t tk_;
+        a.map.info(nxt / H, sq_, tk_, len_, jl_);
+        if (tid < len_) beta_next = __bfloat162float(beta[(size_t)(tk_ + tid) * H + nxt % H]);
+      }
       float dgs[16];
       float gcp = 0.f;
+      // fast path: the pair terms carry the reference-row scaling; exact path:
+      // they are final, and the factors come straight from Gam
+      auto rows = [&](auto fast_c) {
+        constexpr bool kFast = decltype(fast_c)::value;
 #pragma unroll
       for (int b8 = 0; b8 < 2; ++b8) {
         const int r0 = 16 * cq + 8 * b8;
@@ -1026,12 +1044,10 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
           const float Gr = P.G[ii];
           const float p = ((P.pre >> ii) & 1u) ? -1.f : 1.f;
           const float kp = p * bf_lo(P.kq[ii]), qp = p * bf_hi(P.kq[ii]);
-          // fast path: the pair terms carry the reference-row scaling; exact
-          // path: they are final, and the factors come straight from Gam
-          const float el = fast ? fast_exp(Gr - P.Gm) : 1.f;
-          const float er = fast ? rcp_approx(el) : 1.f;
-          const float E = fast ? el * eGm : fast_exp(Gr);
-          const float eC = fast ? er * eCm : fast_exp(P.GC - Gr);
+          const float el = kFast ? fast_exp(Gr - P.Gm) : 1.f;
+          const float er = kFast ? rcp_approx(el) : 1.f;
+          const float E = kFast ? el * eGm : fast_exp(Gr);
+          const float eC = kFast ? er * eCm : fast_exp(P.GC - Gr);
           const float x1 = el * X1[i], x2 = el * X2[i], y1 = er * Y1[i];
           const float KGv = kp * E, QGv = qp * E, Kh = pCs * kp * eC;
           const float dkp = x1 + y1 + dKG[i] * E + pCs * dKh[i] * eC;
@@ -1046,6 +1062,10 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
           }
         }
       }
+      };
+      if (fast) rows(std::true_type{});
+      else rows(std::false_type{});
+      if (tid < 64) ms.beta[tid] = beta_next;  // this item's beta is no longer read
       // reverse in-chunk cumsum of dL/dGam (plus the chunk-end terms) -> dg;
       // the four quarters at once: each starts from the totals of the later ones
       float part = 0.f;
