@@ -91,8 +91,8 @@ __global__ void __launch_bounds__(kIntraThreads, 2) tc_intra_kernel(const __grid
 
   if (tid == 0) {
     mbar_init(&ms.mbar1, 1);
-    mbar_init(&ms.mbar2, 1);
-    mbar_init(&ms.mfin, 1);
+    mbar_init(&ms.mbar2, 2);  // W^T and U0^T are issued by two threads
+    mbar_init(&ms.mfin, 2);
     mbar_init(&ms.mld, 1);
     mbar_fence_init();
   }
@@ -338,15 +338,14 @@ __global__ void __launch_bounds__(kIntraThreads, 2) tc_intra_kernel(const __grid
     }
 
     // ---------------- W^T = KG^T T^T, U0^T = V^T T^T ----------------
-    if (tid == 0) {
+    if (tid == 0 || tid == 32) {
       tc_fence_after();
       const uint32_t id = idesc_bf16(128, 64, true, false);
+      const uint32_t dst = tid == 0 ? 64 : 128;
+      const uint64_t ad = tid == 0 ? sdesc(sKG, 8192, 1024) : sdesc(sV, 8192, 1024);
 #pragma unroll
-      for (int kk = 0; kk < 4; ++kk) {
-        const uint64_t bd = sdesc_off(sdesc(sT, 16, 1024), kk * 32);
-        mma_bf16(tmem + 64, sdesc_off(sdesc(sKG, 8192, 1024), kk * 2048), bd, id, kk > 0);
-        mma_bf16(tmem + 128, sdesc_off(sdesc(sV, 8192, 1024), kk * 2048), bd, id, kk > 0);
-      }
+      for (int kk = 0; kk < 4; ++kk)
+        mma_bf16(tmem + dst, sdesc_off(ad, kk * 2048), sdesc_off(sdesc(sT, 16, 1024), kk * 32), id, kk > 0);
       mma_commit(&ms.mbar2);
     }
     {
@@ -399,6 +398,7 @@ __global__ void __launch_bounds__(kIntraThreads, 2) tc_intra_kernel(const __grid
   }
   if (tid == 0) bulk_wait_all();  // every record tile written before the kernel ends
   // wind down: make sure no MMA is still writing TMEM before freeing it
+  if (abort && tid == 32) mma_commit(&ms.mfin);
   if (abort && tid == 0) {
     mma_commit(&ms.mfin);
     mbar_wait_ool(&ms.mfin, 0, a.status, 109);
@@ -456,8 +456,8 @@ __global__ void __launch_bounds__(kStateThreads, 1) tc_state_kernel(TcArgs ta) {
     mbar_init(&ms.mrec[0], 1);
     mbar_init(&ms.mrec[1], 1);
     mbar_init(&ms.m3, 1);
-    mbar_init(&ms.m4, 1);
-    mbar_init(&ms.mfin, 1);
+    mbar_init(&ms.m4, 2);  // MMA4 and MMA5 are issued by two threads
+    mbar_init(&ms.mfin, 2);
     mbar_init(&ms.sready, kGroup / 32);
     mbar_init(&ms.sdone, kGroup / 32);
     mbar_fence_init();
@@ -570,23 +570,29 @@ __global__ void __launch_bounds__(kStateThreads, 1) tc_state_kernel(TcArgs ta) {
       fence_async_smem();
       tc_fence_before();
       group_sync(1, kGroup);
-      // MMA4: O^T += U^T A_q^T ; MMA5: S^T += U^T Khat (S^T scaled by group B first)
+      // MMA4: O^T += U^T A_q^T (second thread, at once); MMA5: S^T += U^T Khat
+      // (this group's first thread, once group B has scaled S^T)
       bool ok = true;
+      if (gt == 32) {
+        tc_fence_after();
+        const uint32_t id4 = idesc_bf16(128, 64, false, false);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_bf16(tmem + acc + 64, sdesc_off(sdesc(smem_u32(sm + S_TU), 16, 1024), kk * 32),
+                   sdesc_off(sdesc(smem_u32(rec + R3), 16, 1024), kk * 32), id4, true);
+        mma_commit(&ms.m4);
+      }
       if (gt == 0) {
         if (j > 0) ok = mbar_wait(&ms.sdone, (j - 1) & 1, a.status, 206);
         if (ok) {
           tc_fence_after();
-          const uint32_t sU = smem_u32(sm + S_TU);
-          const uint32_t id4 = idesc_bf16(128, 64, false, false);
           const uint32_t id5 = idesc_bf16(128, 128, false, false);
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t ad = sdesc_off(sdesc(sU, 16, 1024), kk * 32);
-            mma_bf16(tmem + acc + 64, ad, sdesc_off(sdesc(smem_u32(rec + R3), 16, 1024), kk * 32), id4, true);
-            mma_bf16(tmem + 0, ad, sdesc_off(sdesc(smem_u32(rec + R4), 16, 1024), kk * 32), id5, true);
-          }
-          mma_commit(&ms.m4);
+          for (int kk = 0; kk < 4; ++kk)
+            mma_bf16(tmem + 0, sdesc_off(sdesc(smem_u32(sm + S_TU), 16, 1024), kk * 32),
+                     sdesc_off(sdesc(smem_u32(rec + R4), 16, 1024), kk * 32), id5, true);
         }
+        mma_commit(&ms.m4);  // also on failure: the other arrival must not wait on a missing one
       }
       if (gt == 0) bulk_wait_read_all();  // the last state tile has left S_TS
       if (!wait_a(&ms.m4, j & 1, 204, ok)) { abort = true; break; }
@@ -675,6 +681,7 @@ __global__ void __launch_bounds__(kStateThreads, 1) tc_state_kernel(TcArgs ta) {
   }
   if (tid == 0) bulk_wait_all();  // every state tile written before the kernel ends
   __syncthreads();
+  if (abort && tid == 32) mma_commit(&ms.mfin);
   if (abort && tid == 0) {
     mma_commit(&ms.mfin);
     mbar_wait(&ms.mfin, 0, a.status, 209);
