@@ -35,6 +35,7 @@ import torch  # noqa: E402
 from chunked_gated_delta_ckda_b200 import workloads as W  # noqa: E402
 
 METRIC = "CKDA fwd+bwd tokens/s (H=16,d=128,T=4096,bf16); % tensor/HBM roofline"
+METRIC_KDA = "KDA (gate sign +1) fwd+bwd tokens/s (H=16,d=128,T=4096,bf16), same kernels"
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 
@@ -162,9 +163,11 @@ class ClockSampler:
 # our implementation
 # ---------------------------------------------------------------------------
 
-def _fwdbwd_setup(inp, dev):
+def _fwdbwd_setup(inp, dev, kda=False):
     from chunked_gated_delta_ckda_b200 import _abi, api
     d = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+    if kda:  # standard KDA: no sign tensor (every gate sign +1)
+        d["sign"] = None
     B, T, H, dk = d["q"].shape
     dv = d["v"].shape[-1]
     NC = (T + 63) // 64
@@ -224,7 +227,8 @@ def run_ours(args, rank, world, local_rank):
     inp = W.make(w)
     B, T, H = w.B, w.T, w.H
     tokens = B * T
-    d, buf, step = _fwdbwd_setup(inp, dev)
+    kda = args.workload == "kda"
+    d, buf, step = _fwdbwd_setup(inp, dev, kda=kda)
 
     clocks = ClockSampler(local_rank)
     clocks.start()
@@ -265,9 +269,9 @@ def run_ours(args, rank, world, local_rank):
                  "tensor_frac": t_tc / ms_max, "binding_frac": max(t_hbm, t_tc) / ms_max}
 
     # end to end through the public API with host buffers
-    e2e = None if args.no_e2e else run_e2e(inp, dev, args, world)
+    e2e = None if (args.no_e2e or kda) else run_e2e(inp, dev, args, world)
 
-    out = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+    out = {"metric": METRIC_KDA if kda else METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
            "dtype": "bf16", "data": "synthetic",
@@ -276,7 +280,8 @@ def run_ours(args, rank, world, local_rank):
                       "contraction": "bf16 tensor-core operands, f32 accumulate",
                       "step": "ckda_chunk_fwd(saved buffer for the backward) + ckda_chunk_bwd(saved)",
                       "global_batch": B * world, "seq_len": T, "parallelism": "dp%d" % world,
-                      "l2": "inputs larger than L2 (about 2 GB streamed per step)"},
+                      "l2": "inputs larger than L2 (about 2 GB streamed per step)",
+                      "gate_sign": "none: every sign +1 (standard KDA)" if kda else "int8 +-1 (CKDA)"},
            "roofline": roof, "step_roofline": step_roof, "kernels": kernels,
            "gpu_launches": int(sum(n for n, _ in prof.values())), "clocks": clk, "e2e": e2e}
     return out, inp
@@ -382,41 +387,78 @@ def run_secondary(args, rank, world, local_rank):
 
 
 def run_e2e(inp, dev, args, world):
-    """Same step through the public API from pinned HOST buffers: H2D of the
-    inputs and D2H of every output inside the timed region."""
+    """Same step through the public API from pinned HOST buffers: every step
+    uploads its inputs and downloads every output inside the timed region.
+    Steps are pipelined the way a training input pipeline runs: the next
+    step's inputs upload (one copy engine) and the previous step's outputs
+    download (the other) while the current step computes; two device buffer
+    sets alternate, ordered by CUDA events."""
     from chunked_gated_delta_ckda_b200 import _abi, api
-    host_in = {k: inp[k].pin_memory() for k in ("q", "k", "v", "g", "sign", "beta", "dO")}
-    dev_in = {k: torch.empty_like(v, device=dev) for k, v in host_in.items()}
+    names_in = ("q", "k", "v", "g", "sign", "beta", "dO")
+    host_in = {k: inp[k].pin_memory() for k in names_in}
     B, T, H, dk = inp["q"].shape
     dv = inp["v"].shape[-1]
-    d, buf, _ = _fwdbwd_setup({**inp}, dev)
-    host_out = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True)
-                for k, v in buf.items() if k not in ("cs",)}
+    code = api.io_code(inp["q"].dtype)
     wsf = api.workspace(_abi.CKDA_OP_CHUNK_FWD, B, T, H, dk, dv, device=dev, cache=False)
     wsb = api.workspace(_abi.CKDA_OP_CHUNK_BWD, B, T, H, dk, dv, device=dev, cache=False)
-    code = api.io_code(inp["q"].dtype)
     sv = api.saved_buffer(B, T, H, dk, dv, inp["q"].dtype, dev)
-    cs = None if sv is not None else buf["cs"]
+    sets = []
+    for _ in range(2):
+        _, buf, _ = _fwdbwd_setup({**inp}, dev)
+        sets.append(dict(dev_in={k: torch.empty_like(v, device=dev) for k, v in host_in.items()}, buf=buf,
+                         host_out={k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True)
+                                   for k, v in buf.items() if k != "cs"},
+                         in_ready=torch.cuda.Event(), comp_done=torch.cuda.Event(),
+                         out_done=torch.cuda.Event()))
     h2d = sum(v.numel() * v.element_size() for v in host_in.values())
-    d2h = sum(v.numel() * v.element_size() for v in host_out.values())
+    d2h = sum(v.numel() * v.element_size() for v in sets[0]["host_out"].values())
+    s_in, s_comp, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
 
-    def step():
-        for k, v in host_in.items():
-            dev_in[k].copy_(v, non_blocking=True)
-        x = dev_in
+    def issue(i):
+        S = sets[i % 2]
+        x, buf = S["dev_in"], S["buf"]
+        cs = None if sv is not None else buf["cs"]
+        s_in.wait_event(S["comp_done"])  # this set's inputs were last read two steps ago
+        with torch.cuda.stream(s_in):
+            for k, v in host_in.items():
+                x[k].copy_(v, non_blocking=True)
+        S["in_ready"].record(s_in)
+        s_comp.wait_event(S["in_ready"])
+        s_comp.wait_event(S["out_done"])  # this set's outputs have been downloaded
         _abi.ckda_chunk_fwd(B, T, H, dk, dv, code, x["q"], x["k"], x["v"], x["g"], x["sign"],
-                            x["beta"], None, buf["o"], buf["ST"], cs, wsf, saved=sv)
+                            x["beta"], None, buf["o"], buf["ST"], cs, wsf, saved=sv, stream=s_comp)
         _abi.ckda_chunk_bwd(B, T, H, dk, dv, code, x["q"], x["k"], x["v"], x["g"], x["sign"],
                             x["beta"], None, x["dO"], None, cs, buf["dq"], buf["dk"],
-                            buf["dv"], buf["dg"], buf["dbeta"], buf["dS0"], wsb, saved=sv)
-        for k, v in host_out.items():
-            v.copy_(buf[k], non_blocking=True)
+                            buf["dv"], buf["dg"], buf["dbeta"], buf["dS0"], wsb, saved=sv,
+                            stream=s_comp)
+        S["comp_done"].record(s_comp)
+        s_out.wait_event(S["comp_done"])
+        with torch.cuda.stream(s_out):
+            for k, v in S["host_out"].items():
+                v.copy_(buf[k], non_blocking=True)
+        S["out_done"].record(s_out)
 
+    import torch.distributed as dist
     steps = max(1, min(args.steps, 10))
-    ms = _time_steps(step, steps, max(1, min(args.warmup, 3)), world)
-    ms = reduce_max(ms, world)
+    for i in range(max(1, min(args.warmup, 3))):
+        issue(i)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(s_in)
+    s_comp.wait_event(t0)
+    s_out.wait_event(t0)
+    for i in range(steps):
+        issue(i)
+    s_out.wait_event(sets[(steps - 1) % 2]["out_done"])
+    t1.record(s_out)
+    torch.cuda.synchronize(dev)
+    ms = reduce_max(t0.elapsed_time(t1) / steps, world)
     return {"value": aggregate(B * T, world, ms), "unit": "tokens/s", "ms_per_step": ms,
-            "steps": steps, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+            "steps": steps, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "pipelined": "upload of step i+1 and download of step i-1 overlap step i's kernels"}
 
 
 # ---------------------------------------------------------------------------
@@ -497,7 +539,7 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer pass")
-    ap.add_argument("--workload", choices=["fwdbwd", "fwd", "varlen", "decode"], default="fwdbwd",
+    ap.add_argument("--workload", choices=["fwdbwd", "kda", "fwd", "varlen", "decode"], default="fwdbwd",
                     help="fwdbwd is the headline; the others are secondary measurements")
     ap.add_argument("--batch", type=int, default=0,
                     help="override B (profiling a smaller case; not a bench line)")
@@ -522,14 +564,14 @@ def main(argv=None):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
     try:
-        if args.workload != "fwdbwd":
+        if args.workload not in ("fwdbwd", "kda"):
             out = run_secondary(args, rank, world, local_rank)
             if rank == 0:
                 print(json.dumps(out), flush=True)
             return 0
         out, inp = run_ours(args, rank, world, local_rank)
         if rank == 0:
-            if world == 1 and not args.no_cpu_baseline:
+            if world == 1 and not args.no_cpu_baseline and args.workload == "fwdbwd":
                 out["cpu_baseline"] = cpu_baseline(inp, W.LAYER_FWDBWD.H)
             print(json.dumps(out), flush=True)
     finally:

@@ -9,8 +9,9 @@ torch (device memory is torch's job here) and call the library.
     o, ST     = varlen_fwd(q, k, v, g, sign, beta, cu_seqlens, max_seqlen, S0=None)
 
 Shapes and dtypes are those of include/ckda.h: q, k, g, sign [B,T,H,dk]; v
-[B,T,H,dv]; beta [B,T,H]; g fp32; sign int8; q, k, v, beta either fp32 or
-bf16 (all the same); states fp32 [B,H,dk,dv].
+[B,T,H,dv]; beta [B,T,H]; g fp32; sign int8 (None: every sign +1, standard
+KDA); q, k, v, beta either fp32 or bf16 (all the same); states fp32
+[B,H,dk,dv].
 """
 from __future__ import annotations
 

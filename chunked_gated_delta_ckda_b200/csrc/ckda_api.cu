@@ -145,8 +145,8 @@ int ckda_chunk_fwd(int B, int T, int H, int dk, int dv, int io_dtype, const void
                    cudaStream_t stream) {
   CKDA_TRY(check_common(B, T, H, dk, dv, io_dtype));
   const bool empty = (int64_t)B * T == 0;
-  if (!empty) CKDA_TRY(check_ptrs({q, k, v, g, sign, beta, o}, {S0, ST, chunk_states}));
-  else CKDA_TRY(check_ptrs({}, {S0, ST, chunk_states}));
+  if (!empty) CKDA_TRY(check_ptrs({q, k, v, g, beta, o}, {sign, S0, ST, chunk_states}));
+  else CKDA_TRY(check_ptrs({}, {sign, S0, ST, chunk_states}));
   int rc;
   unsigned char *recs_out = static_cast<unsigned char *>(
       const_cast<void *>(saved_or_null(saved, saved_bytes, B, T, H, dk, dv, io_dtype, &rc)));
@@ -187,8 +187,8 @@ int ckda_chunk_bwd(int B, int T, int H, int dk, int dv, int io_dtype, const void
   CKDA_TRY(check_common(B, T, H, dk, dv, io_dtype));
   const bool empty = (int64_t)B * T == 0;
   if (!empty)
-    CKDA_TRY(check_ptrs({q, k, v, g, sign, beta, dO, dq, dk_out, dv_out, dg, dbeta},
-                        {S0, dST, chunk_states, dS0}));
+    CKDA_TRY(check_ptrs({q, k, v, g, beta, dO, dq, dk_out, dv_out, dg, dbeta},
+                        {sign, S0, dST, chunk_states, dS0}));
   else
     CKDA_TRY(check_ptrs({}, {S0, dST, chunk_states, dS0}));
   int rc;
@@ -255,7 +255,7 @@ int ckda_decode_step(int N, int H, int dk, int dv, int io_dtype, const void *q, 
                      float *state, void *o, cudaStream_t stream) {
   CKDA_TRY(check_common(N, 1, H, dk, dv, io_dtype));
   if (N == 0) return CKDA_OK;
-  CKDA_TRY(check_ptrs({q, k, v, g, sign, beta, state, o}, {}));
+  CKDA_TRY(check_ptrs({q, k, v, g, beta, state, o}, {sign}));
   return cuda_status(decode_step(N, H, dk, dv, io_dtype == CKDA_BF16, q, k, v, g, sign, beta,
                                  state, o, stream));
 }
@@ -269,8 +269,8 @@ int ckda_varlen_fwd(int total_T, int N, const int32_t *cu_seqlens, int max_seqle
   if (N == 0) return total_T == 0 ? CKDA_OK : CKDA_ERR_INVALID_ARG;
   if (!cu_seqlens) return CKDA_ERR_INVALID_ARG;
   if (total_T > 0 && (max_seqlen < 1 || max_seqlen > total_T)) return CKDA_ERR_INVALID_ARG;
-  if (total_T > 0) CKDA_TRY(check_ptrs({q, k, v, g, sign, beta, o}, {S0, ST}));
-  else CKDA_TRY(check_ptrs({}, {S0, ST}));
+  if (total_T > 0) CKDA_TRY(check_ptrs({q, k, v, g, beta, o}, {sign, S0, ST}));
+  else CKDA_TRY(check_ptrs({}, {sign, S0, ST}));
   if ((reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) != 0) return CKDA_ERR_ALIGNMENT;
   const WsLayout L = ws_layout(CKDA_OP_VARLEN_FWD, 1, total_T, H, dk, dv, N);
   CKDA_TRY(check_ws(ws, ws_bytes, L.total));

@@ -51,7 +51,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(const IO *__restric
     s_k[i] = kk;
     s_q[i] = qq;
     const float a = expf(g[nh * DK + i]);
-    s_a[i] = sign[nh * DK + i] < 0 ? -a : a;
+    s_a[i] = (sign && sign[nh * DK + i] < 0) ? -a : a;  // no sign tensor: all +1 (KDA)
     kq += kk * qq;
   }
 #pragma unroll

@@ -71,7 +71,7 @@ extern "C" int ckda_chunk_fwd_noalloc(int B, int T, int H, int dk, int dv, int i
   if ((int64_t)B * T > INT32_MAX / 2 || need > (size_t)CKDA_NOALLOC_SCRATCH_BYTES)
     return CKDA_ERR_NOALLOC_CAPACITY;
   if ((int64_t)B * T > 0) {
-    const void *req[] = {q, k, v, g, sign, beta, o};
+    const void *req[] = {q, k, v, g, beta, o};  // sign may be null (all +1)
     for (const void *p : req)
       if (!p) return CKDA_ERR_INVALID_ARG;
     for (const void *p : req)

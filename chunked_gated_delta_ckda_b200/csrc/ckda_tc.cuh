@@ -15,7 +15,8 @@ namespace tc {
 // Tensor maps of the per-token row tensors, viewed as [tokens][H][128]: each
 // TMA box is 64 tokens x one head x 64 channels (bf16, 128-byte swizzle: the
 // K-major SW128 tile layout) or 128 channels (g fp32, sign int8; plain rows).
-// Rows past the last token read as zeros.
+// Rows past the last token read as zeros.  Without a sign tensor (standard
+// KDA, every sign +1) the sign map stays empty and is never used.
 struct RowMaps {
   CUtensorMap q, k, v, dO, g, sign;
 };
@@ -391,8 +392,9 @@ struct Prep {
 
 // Staged rows of one chunk-head in shared memory (TMA boxes, see RowMaps):
 // q and k as K-major SW128 tiles of 64 rows (two 64-channel blocks), g as
-// fp32 [64][128], sign as int8 [64][128].  Rows past the chunk's length hold
-// other tokens or zeros; they are masked here.
+// fp32 [64][128], sign as int8 [64][128] (null: no sign tensor, all +1).
+// Rows past the chunk's length hold other tokens or zeros; they are masked
+// here.
 constexpr uint32_t kStageQ = 0, kStageK = 16384;  // offsets inside the q|k staging region
 constexpr uint32_t kRowBytesQK = 2 * 16384, kRowBytesG = 32768, kRowBytesSign = 8192;
 
@@ -406,7 +408,7 @@ __device__ __forceinline__ void prep_load_smem(const unsigned char *sqk, const f
     const int r = 8 * w + rr;
     const bool valid = r < len;
     const float4 gv = *reinterpret_cast<const float4 *>(sg + r * D + 4 * l);
-    const uint32_t sgn = *reinterpret_cast<const uint32_t *>(ss + r * D + 4 * l);
+    const uint32_t sgn = ss ? *reinterpret_cast<const uint32_t *>(ss + r * D + 4 * l) : 0u;
     const uint32_t off = kmaj_off(r, 4 * l, 64);
     const uint2 kv = *reinterpret_cast<const uint2 *>(sqk + kStageK + off);
     const uint2 qv = *reinterpret_cast<const uint2 *>(sqk + kStageQ + off);

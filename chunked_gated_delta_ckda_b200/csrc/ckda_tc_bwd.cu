@@ -420,7 +420,7 @@ __device__ __forceinline__ void prepc_load(const unsigned char *sqk, const float
     const int r = 16 * cq + i;
     const bool valid = r < len;
     const float g = sg[r * D + c];
-    const int8_t sgn = (int8_t)ss[r * D + c];
+    const int8_t sgn = ss ? (int8_t)ss[r * D + c] : (int8_t)1;
     const uint32_t off = kmaj_off(r, c, 64);
     const uint32_t kb = *reinterpret_cast<const uint16_t *>(sqk + kStageK + off);
     const uint32_t qb = *reinterpret_cast<const uint16_t *>(sqk + kStageQ + off);
@@ -527,7 +527,7 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
       const unsigned char *gdU = ta.dU_tiles + (size_t)itm * DU_TILE;
       mbar_arrive_expect_tx(&ms.mdu, DU_TILE);
       mbar_arrive_expect_tx(&ms.mrec, W_TILE + M_BYTES + S_TILE);
-      mbar_arrive_expect_tx(&ms.mld, kRowBytesQK + kRowBytesG + kRowBytesSign + 2 * 16384);
+      mbar_arrive_expect_tx(&ms.mld, kRowBytesQK + kRowBytesG + (a.sign ? kRowBytesSign : 0) + 2 * 16384);
       bulk_g2s(sm + G_OU + 8192, gdU, 8192, &ms.mdu);
       bulk_g2s(sm + G_OU + 16384 + 8192, gdU + 8192, 8192, &ms.mdu);
       const unsigned char *rec = ta.recs + (size_t)itm * REC;
@@ -543,7 +543,7 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
       tma_rows(sm + G_A1 + kStageK + 8192, &ta.rm.k, 64, hh, t, &ms.mld);
     } else if (warp == 2) {
       tma_rows(sm + G_B1, &ta.rm.g, 0, hh, t, &ms.mld);
-      tma_rows(sm + G_TT, &ta.rm.sign, 0, hh, t, &ms.mld);
+      if (a.sign) tma_rows(sm + G_TT, &ta.rm.sign, 0, hh, t, &ms.mld);
       tma_rows(sm + G_UV + 8192, &ta.rm.v, 0, hh, t, &ms.mld);
       tma_rows(sm + G_UV + 16384 + 8192, &ta.rm.v, 64, hh, t, &ms.mld);
     } else {
@@ -570,8 +570,8 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
     if (!wait_all(&ms.mld, ph, a.status, 400)) { abort = true; break; }
     ++n_mld;
     PrepC P;
-    prepc_load(sm + G_A1, reinterpret_cast<const float *>(sm + G_B1), sm + G_TT, len, c, cq, P, &ms.qt[0][0],
-               &ms.qp[0][0]);
+    prepc_load(sm + G_A1, reinterpret_cast<const float *>(sm + G_B1), a.sign ? sm + G_TT : nullptr, len, c, cq,
+               P, &ms.qt[0][0], &ms.qp[0][0]);
     if (len < 64) {  // V and dO rows past the chunk
       zero_tail_rows(sm + G_UV + 8192, 16384, len, tid, kGThreads);
       zero_tail_rows(sm + G_OU, 16384, len, tid, kGThreads);

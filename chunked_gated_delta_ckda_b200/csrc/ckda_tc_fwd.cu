@@ -130,7 +130,7 @@ __global__ void __launch_bounds__(kIntraThreads, 2) tc_intra_kernel(const __grid
       fence_async_smem();  // earlier generic accesses of these regions come first
       const int t = (int)tok0;
       if (warp == 0) {
-        mbar_arrive_expect_tx(&ms.mld, kRowBytesQK + kRowBytesG + kRowBytesSign + 16384);
+        mbar_arrive_expect_tx(&ms.mld, kRowBytesQK + kRowBytesG + (a.sign ? kRowBytesSign : 0) + 16384);
         tma_rows(sm + I_A1 + kStageQ, &ta.rm.q, 0, h, t, &ms.mld);
         tma_rows(sm + I_A1 + kStageQ + 8192, &ta.rm.q, 64, h, t, &ms.mld);
       } else if (warp == 1) {
@@ -138,7 +138,7 @@ __global__ void __launch_bounds__(kIntraThreads, 2) tc_intra_kernel(const __grid
         tma_rows(sm + I_A1 + kStageK + 8192, &ta.rm.k, 64, h, t, &ms.mld);
       } else if (warp == 2) {
         tma_rows(sm + I_B1, &ta.rm.g, 0, h, t, &ms.mld);
-        tma_rows(sm + I_T, &ta.rm.sign, 0, h, t, &ms.mld);
+        if (a.sign) tma_rows(sm + I_T, &ta.rm.sign, 0, h, t, &ms.mld);
       } else {
         tma_rows(sm + I_V, &ta.rm.v, 0, h, t, &ms.mld);
         tma_rows(sm + I_V + 8192, &ta.rm.v, 64, h, t, &ms.mld);
@@ -151,7 +151,8 @@ __global__ void __launch_bounds__(kIntraThreads, 2) tc_intra_kernel(const __grid
     }
     // ---------------- prep: row-group layout (rows 8w.., channels 4l..) ----------------
     Prep P;
-    prep_load_smem(sm + I_A1, reinterpret_cast<const float *>(sm + I_B1), sm + I_T, len, warp, lane, P, ms.tot);
+    prep_load_smem(sm + I_A1, reinterpret_cast<const float *>(sm + I_B1), a.sign ? sm + I_T : nullptr, len, warp,
+                   lane, P, ms.tot);
     if (len < 64) zero_tail_rows(sm + I_V, 8192, len, tid, kIntraThreads);  // V rows past the chunk
     __syncthreads();
     prep_carry(warp, lane, P, ms.tot);

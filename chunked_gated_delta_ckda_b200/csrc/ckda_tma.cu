@@ -54,6 +54,7 @@ cudaError_t make_row_maps(RowMaps &m, const void *q, const void *k, const void *
   if (dO && (e = encode(&m.dO, dO, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ntok, H, 64, true)) != cudaSuccess)
     return e;
   if ((e = encode(&m.g, g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, ntok, H, D, false)) != cudaSuccess) return e;
+  if (!sign) return cudaSuccess;  // all +1: no sign rows to load
   return encode(&m.sign, sign, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, ntok, H, D, false);
 }
 

@@ -85,7 +85,7 @@ __device__ void load_chunk(const IO *q, const IO *k, const IO *v, const float *g
       if (r < len) {
         const size_t off = ((size_t)(tok0 + r) * H + h) * dk + c;
         G += g[off];
-        if (sign[off] < 0) Pp = -Pp;
+        if (sign && sign[off] < 0) Pp = -Pp;  // no sign tensor: all +1 (KDA)
         kv = ld_io(k, off);
         qv = ld_io(q, off);
       }

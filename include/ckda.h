@@ -27,7 +27,8 @@
  *             in the backward, to dO, dq, dk, dv and dbeta.  g, dg and every
  *             state (S0, ST, chunk_states, dST, dS0, the decode state) are fp32.
  *             sign is int8 holding +1 or -1 (any other value: undefined
- *             output).  g = log|alpha| should be <= 0; the library computes
+ *             output); a null sign pointer means every sign is +1, i.e.
+ *             standard KDA (the same kernels without the sign loads).  g = log|alpha| should be <= 0; the library computes
  *             exactly what it is given, and very negative g (a gate near 0) is
  *             supported.
  *  Shapes     dk, dv in {64, 128}; any T >= 0; the chunk length is 64.

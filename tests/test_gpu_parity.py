@@ -161,6 +161,49 @@ def test_saved_is_ignored_without_a_saved_form():
         check(key, got[key], ref[key], io)
 
 
+@pytest.mark.parametrize("io,d", [(torch.bfloat16, 128), (torch.float32, 64)])
+def test_kda_mode_without_sign_tensor(io, d):
+    """A null sign pointer is standard KDA (every gate sign +1): forward with
+    the saved buffer, backward, decode and packed documents match the oracle
+    run with an all-ones sign tensor."""
+    inp = random_inputs(2, 150, 2, d, d, io, seed=21 + d, extreme_p=0.05)
+    inp["sign"] = torch.ones_like(inp["sign"])
+    x = to_dev(inp)
+    S0, dST = inp["S0"].cuda(), inp["dST"].cuda()
+    o, ST, cs, sv = api.chunk_fwd(x["q"], x["k"], x["v"], x["g"], None, x["beta"], S0=S0,
+                                  save_chunk_states=True, save_for_backward=True)
+    gr = api.chunk_bwd(x["q"], x["k"], x["v"], x["g"], None, x["beta"], x["dO"], S0=S0, dST=dST,
+                       chunk_states=cs, saved=sv)
+    torch.cuda.synchronize()
+    o_ref, ST_ref, _ = oracle_fwd_batched(inp, S0=inp["S0"])
+    check("o", o, o_ref, io)
+    check("ST", ST, ST_ref, io)
+    ref = oracle_bwd_batched(inp, inp["dO"], S0=inp["S0"], dST=inp["dST"])
+    for key in ("dq", "dk", "dv", "dg", "dbeta", "dS0"):
+        check(key, gr[key], ref[key], io)
+    # packed documents (the two batch rows as two documents)
+    cu = torch.tensor([0, 150, 300], dtype=torch.int32, device="cuda")
+    P = lambda t: t.reshape(1, -1, *t.shape[2:]).contiguous()
+    ov, STv = api.varlen_fwd(P(x["q"]), P(x["k"]), P(x["v"]), P(x["g"]), None, P(x["beta"]), cu, 150, S0=S0)
+    torch.cuda.synchronize()
+    check("o (packed)", ov.reshape(o.shape), o_ref, io)
+    check("ST (packed)", STv, ST_ref, io)
+    # one decode step from the final state
+    st = ST.clone()
+    y = random_inputs(3, 1, 2, d, d, io, seed=31 + d)
+    y = {k: (v[:, 0] if k in ("q", "k", "v", "g", "sign", "beta") else v) for k, v in y.items()}
+    y["sign"] = torch.ones_like(y["sign"])
+    yd = to_dev(y)
+    st3 = st[:1].expand(3, -1, -1, -1).contiguous()
+    st_ref = f64(st3)
+    od = api.decode_step(yd["q"], yd["k"], yd["v"], yd["g"], None, yd["beta"], st3)
+    torch.cuda.synchronize()
+    od_ref, st_ref = oracle.decode(f64(y["q"]), f64(y["k"]), f64(y["v"]), f64(y["g"]), y["sign"].numpy(),
+                                   f64(y["beta"]), st_ref)
+    check("o (decode)", od, od_ref, io)
+    check("state (decode)", st3, st_ref, io)
+
+
 def test_backward_without_state_inputs():
     io = torch.float32
     inp = random_inputs(1, 100, 2, 64, 64, io, seed=12)
