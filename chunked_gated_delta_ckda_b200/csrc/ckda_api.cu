@@ -32,6 +32,10 @@ WsLayout ws_layout(int op, int B, int T, int H, int dk, int dv, int N) {
   off += align256((size_t)nch * H * L.intra_stride * sizeof(float));
   L.fscratch = off;
   off += align256(v1_fwd_scratch_floats(dk, dv) * sizeof(float));
+  if (!packed) {
+    L.seg = off;
+    off += align256(tc_seg_ws_bytes());
+  }
   if (op == CKDA_OP_CHUNK_BWD) {
     const size_t st = (size_t)B * H * NC * dk * dv * sizeof(float);
     L.states = off;
@@ -170,7 +174,8 @@ int ckda_chunk_fwd(int B, int T, int H, int dk, int dv, int io_dtype, const void
     // with a saved buffer the state pass also stores each chunk-start state there
     CKDA_CUDA(tc_forward(a, recs_out ? recs_out : reinterpret_cast<unsigned char *>(w + L.intra),
                          reinterpret_cast<float *>(w + L.fscratch), true, chunk_states, stream,
-                         /*state_pass=*/true, /*intra_pass=*/true, /*state_tiles=*/recs_out != nullptr));
+                         /*state_pass=*/true, /*intra_pass=*/true, /*state_tiles=*/recs_out != nullptr,
+                         reinterpret_cast<float *>(w + L.seg)));
     return CKDA_OK;
   }
   CKDA_CUDA(v1_intra(a, bf16, reinterpret_cast<float *>(w + L.fscratch), stream));
@@ -219,7 +224,8 @@ int ckda_chunk_bwd(int B, int T, int H, int dk, int dv, int io_dtype, const void
     // recomputed state pass.
     unsigned char *rw = const_cast<unsigned char *>(recs);
     CKDA_CUDA(tc_forward(f, rw, reinterpret_cast<float *>(w + L.fscratch), false, nullptr, stream,
-                         /*state_pass=*/states == nullptr, /*intra_pass=*/true, /*state_tiles=*/true));
+                         /*state_pass=*/states == nullptr, /*intra_pass=*/true, /*state_tiles=*/true,
+                         reinterpret_cast<float *>(w + L.seg)));
     if (states) CKDA_CUDA(tc_state_tiles(states, rw, B, H, f.map.NC, stream));
   } else if (!tcp) {
     CKDA_CUDA(v1_intra(f, bf16, reinterpret_cast<float *>(w + L.fscratch), stream));

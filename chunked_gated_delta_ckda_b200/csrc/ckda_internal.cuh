@@ -96,6 +96,7 @@ struct WsLayout {
   size_t du = 0;         // bwd: dL/dU per (chunk, head) [C, dv]
   size_t fscratch = 0;   // per-CTA scratch of the intra-chunk kernel
   size_t scratch = 0;    // bwd: per-CTA scratch of the per-chunk gradient kernel
+  size_t seg = 0;        // segment maps, their scan (long sequences; tensor-core path)
   size_t total = 0;
   size_t intra_stride = 0;  // floats per (chunk, head)
   int n_chunks_bound = 0;
@@ -190,7 +191,9 @@ int tc_intra_ctas();
 size_t tc_record_bytes();
 cudaError_t tc_forward(const FwdArgs &f, unsigned char *recs, float *fb, bool write_o,
                        float *states_out, cudaStream_t s, bool state_pass = true,
-                       bool intra_pass = true, bool state_tiles = false);
+                       bool intra_pass = true, bool state_tiles = false, float *seg_ws = nullptr);
+int tc_seg_count(int B, int H, int NC);  // segments per sequence of the long-sequence scan (0: off)
+size_t tc_seg_ws_bytes();                // workspace of the long-sequence scan
 // bf16 chunk-start state tiles of the records from fp32 chunk states [B,H,NC,128,128]
 cudaError_t tc_state_tiles(const float *chunk_states, unsigned char *recs, int B, int H, int NC,
                            cudaStream_t s);

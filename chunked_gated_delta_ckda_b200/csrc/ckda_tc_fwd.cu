@@ -77,6 +77,12 @@ struct TcArgs {
   float *states_out;    // chunk-start states (batched only) or null
   bool write_o;
   bool state_tiles;     // the state pass also stores each chunk-start state (bf16) in its record
+  // segment mode (long sequences, few of them): the chunks of a sequence are
+  // split into seg_count segments of seg_len chunks; blockIdx.y = seq *
+  // seg_count + segment in the segment kernels and the state pass
+  int seg_len, seg_count;
+  float *seg_M, *seg_b;  // per segment: its affine map S -> M S + b (fp32 [128][128] each)
+  float *seg_S0;         // per segment: its start state (fp32 [128][128])
 };
 
 __global__ void __launch_bounds__(kIntraThreads, 2) tc_intra_kernel(const __grid_constant__ TcArgs ta) {
@@ -444,13 +450,32 @@ __global__ void __launch_bounds__(kStateThreads, 1) tc_state_kernel(TcArgs ta) {
   const bool grpA = tid < kGroup;
   const int gt = tid & (kGroup - 1);
   const int qd = warp & 3, ch = (warp >> 2) & 1;
-  const int h = blockIdx.x, seq = blockIdx.y, H = a.H;
+  const int h = blockIdx.x, H = a.H;
   const int v = 32 * qd + lane;  // value channel = TMEM lane
   __nv_bfloat16 *o = (__nv_bfloat16 *)a.o;
 
+  // this CTA's chunks: a whole sequence, or one segment of it (whose start
+  // state comes from the segment scan; only the last segment has the final state)
+  int seq = blockIdx.y, j0 = 0;
   int first;
-  const int nc = a.map.seq_chunks(seq, first);
-  const size_t sbase = ((size_t)seq * H + h) * D * D;
+  int nc = 0;
+  const float *S0p;
+  bool last_seg = true;
+  if (ta.seg_len > 0) {
+    seq = blockIdx.y / ta.seg_count;
+    const int sg = blockIdx.y % ta.seg_count;
+    nc = a.map.seq_chunks(seq, first);
+    j0 = sg * ta.seg_len;
+    nc = nc - j0 < ta.seg_len ? nc - j0 : ta.seg_len;
+    if (nc < 0) nc = 0;
+    first += j0;
+    S0p = ta.seg_S0 + ((size_t)blockIdx.y * H + h) * D * D;
+    last_seg = sg == ta.seg_count - 1;
+  } else {
+    nc = a.map.seq_chunks(seq, first);
+    S0p = a.S0 ? a.S0 + ((size_t)seq * H + h) * D * D : nullptr;
+  }
+  float *STp = (a.ST && last_seg) ? a.ST + ((size_t)seq * H + h) * D * D : nullptr;
   const int NCb = a.map.NC;
 
   if (tid == 0) {
@@ -503,15 +528,15 @@ __global__ void __launch_bounds__(kStateThreads, 1) tc_state_kernel(TcArgs ta) {
       for (int c0 = 64 * ch; c0 < 64 * ch + 64; c0 += 16) {
         float sv[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) sv[i] = a.S0 ? a.S0[sbase + (size_t)(c0 + i) * D + v] : 0.f;
+        for (int i = 0; i < 16; ++i) sv[i] = S0p ? S0p[(size_t)(c0 + i) * D + v] : 0.f;
         if (nc == 0) {
-          if (a.ST)
-            for (int i = 0; i < 16; ++i) a.ST[sbase + (size_t)(c0 + i) * D + v] = sv[i];
+          if (STp)
+            for (int i = 0; i < 16; ++i) STp[(size_t)(c0 + i) * D + v] = sv[i];
           continue;
         }
         if (ta.states_out)
           for (int i = 0; i < 16; ++i)
-            ta.states_out[(((size_t)seq * H + h) * NCb + 0) * D * D + (size_t)(c0 + i) * D + v] = sv[i];
+            ta.states_out[(((size_t)seq * H + h) * NCb + j0) * D * D + (size_t)(c0 + i) * D + v] = sv[i];
         uint32_t pk[8];
 #pragma unroll
         for (int m = 0; m < 8; ++m) pk[m] = pack_bf16(sv[2 * m], sv[2 * m + 1]);
@@ -657,13 +682,13 @@ __global__ void __launch_bounds__(kStateThreads, 1) tc_state_kernel(TcArgs ta) {
         tmem_ld16(lanebase + c0, sv);
         tmem_wait_ld();
         if (last) {
-          if (a.ST)
-            for (int i = 0; i < 16; ++i) a.ST[sbase + (size_t)(c0 + i) * D + v] = sv[i];
+          if (STp)
+            for (int i = 0; i < 16; ++i) STp[(size_t)(c0 + i) * D + v] = sv[i];
           continue;
         }
         if (ta.states_out)
           for (int i = 0; i < 16; ++i)
-            ta.states_out[(((size_t)seq * H + h) * NCb + j + 1) * D * D + (size_t)(c0 + i) * D + v] = sv[i];
+            ta.states_out[(((size_t)seq * H + h) * NCb + j0 + j + 1) * D * D + (size_t)(c0 + i) * D + v] = sv[i];
 #pragma unroll
         for (int i = 0; i < 16; ++i) sv[i] *= dn[c0 + i];
         tmem_st16(lanebase + c0, sv);
@@ -691,6 +716,285 @@ __global__ void __launch_bounds__(kStateThreads, 1) tc_state_kernel(TcArgs ta) {
   if (warp == 0) tmem_dealloc(tmem, 512);
 }
 
+// ===========================================================================
+// segment scan for long sequences (few (sequence, head) pairs, many chunks)
+// ===========================================================================
+// A chunk maps the state affinely: S' = A S + B with A = Diag(d) - Khat^T W
+// and B = Khat^T U0.  The chunks of a sequence are split into segments:
+// (1) tc_segmap_kernel composes each segment's map S -> M S + b in parallel,
+//     by running the chunk recurrence on the state [I | 0] (dk x (dk + dv));
+// (2) tc_segscan_kernel walks the segments in order (fp32) for their start
+//     states;
+// (3) the state pass runs every segment from its start state, in parallel.
+constexpr int kSegThreads = 256;
+constexpr uint32_t SG_RSZ = 50176;                 // compact record slot: W^T | U0^T | Khat^T, d
+constexpr uint32_t SG_W = 0, SG_U0 = 16384, SG_KH = 32768, SG_D = 49152;
+constexpr uint32_t SG_R0 = 0, SG_R1 = SG_RSZ;
+constexpr uint32_t SG_S1 = 2 * SG_RSZ;             // bf16 M^T part, K-major [j][c] 128 x 128
+constexpr uint32_t SG_S2 = SG_S1 + 32768;          // bf16 b^T part, K-major [v][c]
+constexpr uint32_t SG_U1 = SG_S2 + 32768;          // bf16 U^T of the M part, K-major [j][s]
+constexpr uint32_t SG_U2 = SG_U1 + 16384;          // bf16 U^T of the b part
+constexpr uint32_t SG_MISC = SG_U2 + 16384;
+
+struct SegMisc {
+  uint64_t mrec[2], ma, mb, mfin;
+  uint32_t tmem;
+};
+
+// TMEM: M^T [0,128), b^T [128,256), (W M)^T [256,320), (W b)^T [320,384).
+__global__ void __launch_bounds__(kSegThreads, 1) tc_segmap_kernel(TcArgs ta) {
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char *sm = reinterpret_cast<unsigned char *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  SegMisc &ms = *reinterpret_cast<SegMisc *>(sm + SG_MISC);
+  const FwdArgs &a = ta.f;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int qd = warp & 3, ch = warp >> 2;
+  const int h = blockIdx.x, H = a.H;
+  const int seq = blockIdx.y / ta.seg_count, sg = blockIdx.y % ta.seg_count;
+  const int j = 32 * qd + lane;  // TMEM lane: input index of the map
+  int first;
+  int nc = a.map.seq_chunks(seq, first);
+  const int j0 = sg * ta.seg_len;
+  nc = nc - j0 < ta.seg_len ? nc - j0 : ta.seg_len;
+  if (nc < 0) nc = 0;
+  first += j0;
+
+  if (tid == 0) {
+    mbar_init(&ms.mrec[0], 1);
+    mbar_init(&ms.mrec[1], 1);
+    mbar_init(&ms.ma, 1);
+    mbar_init(&ms.mb, 1);
+    mbar_init(&ms.mfin, 1);
+    mbar_fence_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(&ms.tmem, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ms.tmem;
+  const uint32_t lanebase = tmem + ((uint32_t)(32 * qd) << 16);
+  unsigned char *rb[2] = {sm + SG_R0, sm + SG_R1};
+  auto fetch = [&](int i) {  // record of the segment's chunk i into slot i & 1
+    const unsigned char *src = ta.recs + ((size_t)(first + i) * H + h) * REC;
+    unsigned char *dst = rb[i & 1];
+    mbar_arrive_expect_tx(&ms.mrec[i & 1], 16384 + 16384 + 16896);
+    bulk_g2s(dst + SG_W, src + R1, 16384, &ms.mrec[i & 1]);
+    bulk_g2s(dst + SG_U0, src + R2, 16384, &ms.mrec[i & 1]);
+    bulk_g2s(dst + SG_KH, src + R4, 16896, &ms.mrec[i & 1]);  // Khat^T and d
+  };
+  if (tid == 0) {
+    for (int i = 0; i < 2 && i < nc; ++i) fetch(i);
+  }
+  // start: M^T = I, b^T = 0 (fp32 in TMEM, bf16 operand copies); columns [64 ch, 64 ch + 64)
+  for (int c0 = 64 * ch; c0 < 64 * ch + 64; c0 += 16) {
+    float e[16], z[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      e[i] = (c0 + i == j) ? 1.f : 0.f;
+      z[i] = 0.f;
+    }
+    tmem_st16(lanebase + c0, e);
+    tmem_st16(lanebase + 128 + c0, z);
+    uint32_t pk[8];
+#pragma unroll
+    for (int m = 0; m < 8; ++m) pk[m] = pack_bf16(e[2 * m], e[2 * m + 1]);
+    *reinterpret_cast<uint4 *>(sm + SG_S1 + kmaj_off(j, c0, 128)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+    *reinterpret_cast<uint4 *>(sm + SG_S1 + kmaj_off(j, c0 + 8, 128)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+    *reinterpret_cast<uint4 *>(sm + SG_S2 + kmaj_off(j, c0, 128)) = make_uint4(0, 0, 0, 0);
+    *reinterpret_cast<uint4 *>(sm + SG_S2 + kmaj_off(j, c0 + 8, 128)) = make_uint4(0, 0, 0, 0);
+  }
+  tmem_wait_st();
+  fence_async_smem();
+  tc_fence_before();
+  __syncthreads();
+
+  bool abort = false;
+  for (int i = 0; i < nc && !abort; ++i) {
+    unsigned char *rec = rb[i & 1];
+    {
+      bool ok = true;
+      if (tid == 0) ok = mbar_wait_ool(&ms.mrec[i & 1], (i >> 1) & 1, a.status, 221);
+      if (__syncthreads_or(!ok)) { abort = true; break; }
+    }
+    // (W X)^T = X^T W^T for both parts (N = 64, K = c)
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t id = idesc_bf16(128, 64, false, true);
+      const uint64_t bw = sdesc(smem_u32(rec + SG_W), 16384, 1024);
+      const uint64_t a1 = sdesc(smem_u32(sm + SG_S1), 16, 1024), a2 = sdesc(smem_u32(sm + SG_S2), 16, 1024);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t ko = (kk >> 2) * 16384 + (kk & 3) * 32;
+        mma_bf16(tmem + 256, sdesc_off(a1, ko), sdesc_off(bw, kk * 2048), id, kk > 0);
+        mma_bf16(tmem + 320, sdesc_off(a2, ko), sdesc_off(bw, kk * 2048), id, kk > 0);
+      }
+      mma_commit(&ms.ma);
+    }
+    {
+      bool ok = true;
+      if (tid == 0) ok = mbar_wait_ool(&ms.ma, i & 1, a.status, 222);
+      if (__syncthreads_or(!ok)) { abort = true; break; }
+    }
+    tc_fence_after();
+    // U^T = -(W M)^T and U0^T - (W b)^T -> bf16 tiles; columns s in [32 ch, 32 ch + 32)
+    for (int s0 = 32 * ch; s0 < 32 * ch + 32; s0 += 16) {
+      float w1[16], w2[16];
+      tmem_ld16(lanebase + 256 + s0, w1);
+      tmem_ld16(lanebase + 320 + s0, w2);
+      tmem_wait_ld();
+      const uint4 ua = *reinterpret_cast<const uint4 *>(rec + SG_U0 + kmaj_off(j, s0, 128));
+      const uint4 ub = *reinterpret_cast<const uint4 *>(rec + SG_U0 + kmaj_off(j, s0 + 8, 128));
+      const uint32_t u0[8] = {ua.x, ua.y, ua.z, ua.w, ub.x, ub.y, ub.z, ub.w};
+      uint32_t p1[8], p2[8];
+#pragma unroll
+      for (int m = 0; m < 8; ++m) {
+        p1[m] = pack_bf16(-w1[2 * m], -w1[2 * m + 1]);
+        p2[m] = pack_bf16(bf_lo(u0[m]) - w2[2 * m], bf_hi(u0[m]) - w2[2 * m + 1]);
+      }
+      *reinterpret_cast<uint4 *>(sm + SG_U1 + kmaj_off(j, s0, 128)) = make_uint4(p1[0], p1[1], p1[2], p1[3]);
+      *reinterpret_cast<uint4 *>(sm + SG_U1 + kmaj_off(j, s0 + 8, 128)) = make_uint4(p1[4], p1[5], p1[6], p1[7]);
+      *reinterpret_cast<uint4 *>(sm + SG_U2 + kmaj_off(j, s0, 128)) = make_uint4(p2[0], p2[1], p2[2], p2[3]);
+      *reinterpret_cast<uint4 *>(sm + SG_U2 + kmaj_off(j, s0 + 8, 128)) = make_uint4(p2[4], p2[5], p2[6], p2[7]);
+    }
+    // X^T <- X^T Diag(d) in TMEM (both parts); columns c in [64 ch, 64 ch + 64)
+    {
+      const float *dj = reinterpret_cast<const float *>(rec + SG_D);
+      for (int c0 = 64 * ch; c0 < 64 * ch + 64; c0 += 16) {
+        float x1[16], x2[16];
+        tmem_ld16(lanebase + c0, x1);
+        tmem_ld16(lanebase + 128 + c0, x2);
+        tmem_wait_ld();
+#pragma unroll
+        for (int m = 0; m < 16; ++m) {
+          x1[m] *= dj[c0 + m];
+          x2[m] *= dj[c0 + m];
+        }
+        tmem_st16(lanebase + c0, x1);
+        tmem_st16(lanebase + 128 + c0, x2);
+      }
+      tmem_wait_st();
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    // X^T += U^T Khat (N = 128 over c, K = s)
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t id = idesc_bf16(128, 128, false, false);
+      const uint64_t bk = sdesc(smem_u32(rec + SG_KH), 16, 1024);
+      const uint64_t u1 = sdesc(smem_u32(sm + SG_U1), 16, 1024), u2 = sdesc(smem_u32(sm + SG_U2), 16, 1024);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        mma_bf16(tmem + 0, sdesc_off(u1, kk * 32), sdesc_off(bk, kk * 32), id, true);
+        mma_bf16(tmem + 128, sdesc_off(u2, kk * 32), sdesc_off(bk, kk * 32), id, true);
+      }
+      mma_commit(&ms.mb);
+    }
+    {
+      bool ok = true;
+      if (tid == 0) ok = mbar_wait_ool(&ms.mb, i & 1, a.status, 223);
+      if (__syncthreads_or(!ok)) { abort = true; break; }
+    }
+    tc_fence_after();
+    if (tid == 0 && i + 2 < nc) fetch(i + 2);  // this slot's record is consumed
+    if (i + 1 < nc) {  // bf16 operand copies of the new M^T, b^T
+      for (int c0 = 64 * ch; c0 < 64 * ch + 64; c0 += 16) {
+        float x1[16], x2[16];
+        tmem_ld16(lanebase + c0, x1);
+        tmem_ld16(lanebase + 128 + c0, x2);
+        tmem_wait_ld();
+        uint32_t p1[8], p2[8];
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+          p1[m] = pack_bf16(x1[2 * m], x1[2 * m + 1]);
+          p2[m] = pack_bf16(x2[2 * m], x2[2 * m + 1]);
+        }
+        *reinterpret_cast<uint4 *>(sm + SG_S1 + kmaj_off(j, c0, 128)) = make_uint4(p1[0], p1[1], p1[2], p1[3]);
+        *reinterpret_cast<uint4 *>(sm + SG_S1 + kmaj_off(j, c0 + 8, 128)) = make_uint4(p1[4], p1[5], p1[6], p1[7]);
+        *reinterpret_cast<uint4 *>(sm + SG_S2 + kmaj_off(j, c0, 128)) = make_uint4(p2[0], p2[1], p2[2], p2[3]);
+        *reinterpret_cast<uint4 *>(sm + SG_S2 + kmaj_off(j, c0 + 8, 128)) = make_uint4(p2[4], p2[5], p2[6], p2[7]);
+      }
+      fence_async_smem();
+    }
+    tc_fence_before();
+    __syncthreads();
+  }
+  if (!abort) {  // the map: M[c][j] = M^T[j][c], b[c][v] = b^T[v][c] (fp32, row-major)
+    float *Mo = ta.seg_M + ((size_t)blockIdx.y * H + h) * D * D;
+    float *bo = ta.seg_b + ((size_t)blockIdx.y * H + h) * D * D;
+    for (int c0 = 64 * ch; c0 < 64 * ch + 64; c0 += 16) {
+      float x1[16], x2[16];
+      tmem_ld16(lanebase + c0, x1);
+      tmem_ld16(lanebase + 128 + c0, x2);
+      tmem_wait_ld();
+#pragma unroll
+      for (int m = 0; m < 16; ++m) {
+        Mo[(size_t)(c0 + m) * D + j] = x1[m];
+        bo[(size_t)(c0 + m) * D + j] = x2[m];
+      }
+    }
+  }
+  if (abort && tid == 0) {
+    mma_commit(&ms.mfin);
+    mbar_wait(&ms.mfin, 0, a.status, 229);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, 512);
+}
+
+// The segments of one (sequence, head) in order, fp32 on CUDA cores:
+// start(0) = S0 (or 0), start(g + 1) = M_g start(g) + b_g.
+constexpr int kScanThreads = 256;
+__global__ void __launch_bounds__(kScanThreads, 1) tc_segscan_kernel(TcArgs ta) {
+  extern __shared__ unsigned char smem_raw[];
+  float *S = reinterpret_cast<float *>(smem_raw);  // [128][128] current start state
+  float *M = S + D * D;                            // [128][128] this segment's M
+  const FwdArgs &a = ta.f;
+  const int tid = threadIdx.x, h = blockIdx.x, seq = blockIdx.y, H = a.H, G = ta.seg_count;
+  const float *S0 = a.S0 ? a.S0 + ((size_t)seq * H + h) * D * D : nullptr;
+  for (int e = tid; e < D * D / 4; e += kScanThreads)
+    reinterpret_cast<float4 *>(S)[e] = S0 ? reinterpret_cast<const float4 *>(S0)[e] : make_float4(0.f, 0.f, 0.f, 0.f);
+  __syncthreads();
+  // thread: row c = tid / 2, columns v in [64 (tid % 2), + 64)
+  const int c = tid >> 1, v0 = 64 * (tid & 1);
+  for (int g = 0; g < G; ++g) {
+    const size_t sidx = ((size_t)(seq * G + g) * H + h) * D * D;
+    float4 *out = reinterpret_cast<float4 *>(ta.seg_S0 + sidx);
+    for (int e = tid; e < D * D / 4; e += kScanThreads) out[e] = reinterpret_cast<const float4 *>(S)[e];
+    if (g + 1 == G) break;
+    const float4 *Mg = reinterpret_cast<const float4 *>(ta.seg_M + sidx);
+    for (int e = tid; e < D * D / 4; e += kScanThreads) reinterpret_cast<float4 *>(M)[e] = Mg[e];
+    __syncthreads();
+    float acc[64];
+    const float *bg = ta.seg_b + sidx + (size_t)c * D + v0;
+#pragma unroll
+    for (int m = 0; m < 64; ++m) acc[m] = bg[m];
+#pragma unroll 4
+    for (int jj = 0; jj < D; ++jj) {
+      const float mcj = M[c * D + jj];
+      const float4 *srow = reinterpret_cast<const float4 *>(S + jj * D + v0);
+#pragma unroll
+      for (int m4 = 0; m4 < 16; ++m4) {
+        const float4 x = srow[m4];
+        acc[4 * m4] += mcj * x.x;
+        acc[4 * m4 + 1] += mcj * x.y;
+        acc[4 * m4 + 2] += mcj * x.z;
+        acc[4 * m4 + 3] += mcj * x.w;
+      }
+    }
+    __syncthreads();  // every read of S and M is done
+#pragma unroll
+    for (int m4 = 0; m4 < 16; ++m4)
+      reinterpret_cast<float4 *>(S + c * D + v0)[m4] = make_float4(acc[4 * m4], acc[4 * m4 + 1], acc[4 * m4 + 2], acc[4 * m4 + 3]);
+    __syncthreads();
+  }
+}
+
 int g_num_sms = 0;
 
 }  // namespace
@@ -713,9 +1017,29 @@ size_t tc_record_bytes() { return REC; }
 // Forward on tensor cores.  recs: n_chunks_bound * H records of REC bytes;
 // fb: tc_fwd_fallback_floats(tc_intra_ctas()) floats.  intra_pass = false
 // reuses records an earlier call wrote for the same inputs.
+// Segments per sequence for the segment scan: only for batched calls whose
+// (sequence, head) pairs fill at most half the SMs and whose sequences are
+// long (>= 32 chunks); at least 16 chunks per segment, at most one wave of
+// CTAs.  0: run the plain sequential state pass.
+int tc_seg_count(int B, int H, int NC) {
+  (void)tc_intra_ctas();  // SM count
+  const int sms = g_num_sms > 0 ? g_num_sms : 148;
+  const int pairs = B * H;
+  if (pairs <= 0 || 2 * pairs > sms || NC < 32) return 0;
+  int G = sms / pairs;
+  if (G > NC / 16) G = NC / 16;
+  if (G < 2) return 0;
+  const int L = (NC + G - 1) / G;
+  return (NC + L - 1) / L;
+}
+size_t tc_seg_ws_bytes() {
+  (void)tc_intra_ctas();  // SM count
+  return (size_t)3 * (g_num_sms > 0 ? g_num_sms : 148) * D * D * sizeof(float);
+}
+
 cudaError_t tc_forward(const FwdArgs &f, unsigned char *recs, float *fb, bool write_o,
                        float *states_out, cudaStream_t s, bool state_pass, bool intra_pass,
-                       bool state_tiles) {
+                       bool state_tiles, float *seg_ws) {
   TcArgs ta{};
   ta.f = f;
   ta.recs = recs;
@@ -738,6 +1062,36 @@ cudaError_t tc_forward(const FwdArgs &f, unsigned char *recs, float *fb, bool wr
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   if (state_pass && f.map.n_seq > 0) {
+    const int G = (seg_ws && !f.map.table) ? tc_seg_count(f.B, f.H, f.map.NC) : 0;
+    if (G >= 2) {  // long sequences: segment maps, their scan, then every segment at once
+      ta.seg_count = G;
+      ta.seg_len = (f.map.NC + G - 1) / G;
+      const size_t per = (size_t)f.B * G * f.H * D * D;
+      ta.seg_M = seg_ws;
+      ta.seg_b = seg_ws + per;
+      ta.seg_S0 = seg_ws + 2 * per;
+      const size_t sm_map = SG_MISC + sizeof(SegMisc) + 1024, sm_scan = 2 * D * D * sizeof(float);
+      if ((e = cudaFuncSetAttribute(tc_segmap_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)sm_map)) != cudaSuccess)
+        return e;
+      if ((e = cudaFuncSetAttribute(tc_segscan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)sm_scan)) != cudaSuccess)
+        return e;
+      {
+        ProfScope prof("tc_segmap", s);
+        tc_segmap_kernel<<<dim3(f.H, f.B * G), kSegThreads, sm_map, s>>>(ta);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+      }
+      {
+        ProfScope prof("tc_segscan", s);
+        tc_segscan_kernel<<<dim3(f.H, f.B), kScanThreads, sm_scan, s>>>(ta);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+      }
+      ProfScope prof(write_o ? "tc_state_fwd" : "tc_state_fwd_recompute", s);
+      tc_state_kernel<<<dim3(f.H, f.B * G), kStateThreads, sm_state, s>>>(ta);
+      if ((e = cudaGetLastError()) != cudaSuccess) return e;
+      return cudaSuccess;
+    }
     ProfScope prof(write_o ? "tc_state_fwd" : "tc_state_fwd_recompute", s);
     tc_state_kernel<<<dim3(f.H, f.map.n_seq), kStateThreads, sm_state, s>>>(ta);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;

@@ -204,6 +204,28 @@ def test_kda_mode_without_sign_tensor(io, d):
     check("state (decode)", st3, st_ref, io)
 
 
+@pytest.mark.parametrize("B,H", [(1, 2), (2, 1)])
+def test_long_sequence_segment_scan(B, H):
+    """Few (sequence, head) pairs and many chunks take the segment scan (the
+    sequence's chunks split into segments whose affine maps are composed in
+    parallel, scanned, and re-run): T = 64 * 48 + 17 gives three segments of
+    at most 17 chunks.  Forward with start state, chunk states and final
+    state, and the backward's recomputed state pass, against the oracle."""
+    io = torch.bfloat16
+    T = 64 * 48 + 17
+    inp = random_inputs(B, T, H, 128, 128, io, seed=41 + B, gscale=0.05, extreme_p=0.05)
+    o, ST, cs = _fwd(inp, S0=inp["S0"], chunk_states=True)
+    o_ref, ST_ref, cs_ref = oracle_fwd_batched(inp, S0=inp["S0"], chunk=64)
+    check("o", o, o_ref, io)
+    check("ST", ST, ST_ref, io)
+    NC = (T + 63) // 64
+    check("chunk states", cs, cs_ref.reshape(B, NC, H, 128, 128).transpose(0, 2, 1, 3, 4), io)
+    got = _bwd(inp, inp["S0"], inp["dST"])
+    ref = oracle_bwd_batched(inp, inp["dO"], S0=inp["S0"], dST=inp["dST"])
+    for key in ("dq", "dk", "dv", "dg", "dbeta", "dS0"):
+        check(key, got[key], ref[key], io)
+
+
 def test_backward_without_state_inputs():
     io = torch.float32
     inp = random_inputs(1, 100, 2, 64, 64, io, seed=12)
