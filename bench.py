@@ -2,7 +2,7 @@
 """Benchmark of the CKDA recurrence library on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload fwdbwd|fwd|varlen|decode]
+                    [--workload fwdbwd|kda|fwd|varlen|long|decode]
 
 Default workload (the headline): one step = ckda_chunk_fwd (saving its
 per-chunk results for the backward) + ckda_chunk_bwd on B=8, H=16, T=4096,
@@ -335,6 +335,25 @@ def run_secondary(args, rank, world, local_rank):
         metric = "CKDA varlen fwd tokens/s (65536 packed tokens,H=16,d=128,bf16)"
         cfg = {"workload": w.name, "total_T": T, "docs": Nd, "H": H, "dk": dk, "dv": dv,
                "io_dtype": "bf16", "l2": "inputs larger than L2"}
+    elif args.workload == "long":
+        w = W.LONG
+        inp = W.make(w)
+        d = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+        B, T, H, dk, dv = w.B, w.T, w.H, w.dk, w.dv
+        o = torch.empty(B, T, H, dv, dtype=w.io_dtype, device=dev)
+        ST = torch.empty(B, H, dk, dv, dtype=torch.float32, device=dev)
+        ws = api.workspace(_abi.CKDA_OP_CHUNK_FWD, B, T, H, dk, dv, device=dev, cache=False)
+        code = api.io_code(w.io_dtype)
+        S0 = d["S0"].float().contiguous()
+
+        def step():
+            _abi.ckda_chunk_fwd(B, T, H, dk, dv, code, d["q"], d["k"], d["v"], d["g"], d["sign"],
+                                d["beta"], S0, o, ST, None, ws)
+        units, per_unit, unit_name = B * T * H, FWD_BYTES, "B per token-head (fwd)"
+        tokens = B * T
+        metric = "CKDA long-sequence fwd tokens/s (B=1,T=65536,H=16,d=128,bf16)"
+        cfg = {"workload": w.name, "B": B, "T": T, "H": H, "dk": dk, "dv": dv, "io_dtype": "bf16",
+               "S0": True, "l2": "inputs larger than L2"}
     else:  # fwd
         w = W.LAYER_FWD
         inp = W.make(w)
@@ -539,7 +558,7 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer pass")
-    ap.add_argument("--workload", choices=["fwdbwd", "kda", "fwd", "varlen", "decode"], default="fwdbwd",
+    ap.add_argument("--workload", choices=["fwdbwd", "kda", "fwd", "varlen", "long", "decode"], default="fwdbwd",
                     help="fwdbwd is the headline; the others are secondary measurements")
     ap.add_argument("--batch", type=int, default=0,
                     help="override B (profiling a smaller case; not a bench line)")

@@ -923,7 +923,7 @@ __global__ void __launch_bounds__(kSegThreads, 1) tc_segmap_kernel(TcArgs ta) {
     tc_fence_before();
     __syncthreads();
   }
-  if (!abort) {  // the map: M[c][j] = M^T[j][c], b[c][v] = b^T[v][c] (fp32, row-major)
+  if (!abort) {  // the map, fp32: M^T [j][c] as held, b[c][v] = b^T[v][c] (row-major)
     float *Mo = ta.seg_M + ((size_t)blockIdx.y * H + h) * D * D;
     float *bo = ta.seg_b + ((size_t)blockIdx.y * H + h) * D * D;
     for (int c0 = 64 * ch; c0 < 64 * ch + 64; c0 += 16) {
@@ -931,11 +931,11 @@ __global__ void __launch_bounds__(kSegThreads, 1) tc_segmap_kernel(TcArgs ta) {
       tmem_ld16(lanebase + c0, x1);
       tmem_ld16(lanebase + 128 + c0, x2);
       tmem_wait_ld();
+      float4 *mrow = reinterpret_cast<float4 *>(Mo + (size_t)j * D + c0);
 #pragma unroll
-      for (int m = 0; m < 16; ++m) {
-        Mo[(size_t)(c0 + m) * D + j] = x1[m];
-        bo[(size_t)(c0 + m) * D + j] = x2[m];
-      }
+      for (int m = 0; m < 4; ++m) mrow[m] = make_float4(x1[4 * m], x1[4 * m + 1], x1[4 * m + 2], x1[4 * m + 3]);
+#pragma unroll
+      for (int m = 0; m < 16; ++m) bo[(size_t)(c0 + m) * D + j] = x2[m];
     }
   }
   if (abort && tid == 0) {
@@ -948,50 +948,85 @@ __global__ void __launch_bounds__(kSegThreads, 1) tc_segmap_kernel(TcArgs ta) {
 }
 
 // The segments of one (sequence, head) in order, fp32 on CUDA cores:
-// start(0) = S0 (or 0), start(g + 1) = M_g start(g) + b_g.
+// start(0) = S0 (or 0), start(g + 1) = M_g start(g) + b_g.  The value columns
+// are independent, so a CTA takes a slice of VC of them (blockIdx.z); a
+// thread holds a 4 x (VC / 8) block of the slice in registers.  M_g^T
+// (64 KB) is double-buffered in shared memory by bulk copies.
 constexpr int kScanThreads = 256;
+template <int VC>
 __global__ void __launch_bounds__(kScanThreads, 1) tc_segscan_kernel(TcArgs ta) {
+  constexpr int NV = VC / 8;  // columns per thread
   extern __shared__ unsigned char smem_raw[];
-  float *S = reinterpret_cast<float *>(smem_raw);  // [128][128] current start state
-  float *M = S + D * D;                            // [128][128] this segment's M
+  unsigned char *sm = reinterpret_cast<unsigned char *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~(uintptr_t)127);
+  float *Mt = reinterpret_cast<float *>(sm);         // [2][128][128] M_g^T
+  float *Ss = Mt + 2 * D * D;                         // [128][VC] current start state, this slice
+  uint64_t *mfull = reinterpret_cast<uint64_t *>(Ss + D * VC);
   const FwdArgs &a = ta.f;
   const int tid = threadIdx.x, h = blockIdx.x, seq = blockIdx.y, H = a.H, G = ta.seg_count;
-  const float *S0 = a.S0 ? a.S0 + ((size_t)seq * H + h) * D * D : nullptr;
-  for (int e = tid; e < D * D / 4; e += kScanThreads)
-    reinterpret_cast<float4 *>(S)[e] = S0 ? reinterpret_cast<const float4 *>(S0)[e] : make_float4(0.f, 0.f, 0.f, 0.f);
+  const int tv = tid & 7, tc = tid >> 3;
+  const int c0 = 4 * tc, vl = NV * tv, vg = VC * blockIdx.z + vl;  // rows c0..c0+3; local/global column
+  if (tid == 0) {
+    mbar_init(&mfull[0], 1);
+    mbar_init(&mfull[1], 1);
+    mbar_fence_init();
+  }
   __syncthreads();
-  // thread: row c = tid / 2, columns v in [64 (tid % 2), + 64)
-  const int c = tid >> 1, v0 = 64 * (tid & 1);
+  auto fetch = [&](int g) {  // M_g^T into buffer g & 1
+    const size_t sidx = ((size_t)(seq * G + g) * H + h) * D * D;
+    mbar_arrive_expect_tx(&mfull[g & 1], D * D * 4);
+    bulk_g2s(Mt + (g & 1) * D * D, ta.seg_M + sidx, D * D * 4, &mfull[g & 1]);
+  };
+  if (tid == 0 && G > 1) fetch(0);
+  float st[4][NV];
+  const float *S0 = a.S0 ? a.S0 + ((size_t)seq * H + h) * D * D : nullptr;
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int k = 0; k < NV; ++k) st[i][k] = S0 ? S0[(size_t)(c0 + i) * D + vg + k] : 0.f;
   for (int g = 0; g < G; ++g) {
     const size_t sidx = ((size_t)(seq * G + g) * H + h) * D * D;
-    float4 *out = reinterpret_cast<float4 *>(ta.seg_S0 + sidx);
-    for (int e = tid; e < D * D / 4; e += kScanThreads) out[e] = reinterpret_cast<const float4 *>(S)[e];
-    if (g + 1 == G) break;
-    const float4 *Mg = reinterpret_cast<const float4 *>(ta.seg_M + sidx);
-    for (int e = tid; e < D * D / 4; e += kScanThreads) reinterpret_cast<float4 *>(M)[e] = Mg[e];
-    __syncthreads();
-    float acc[64];
-    const float *bg = ta.seg_b + sidx + (size_t)c * D + v0;
+    float *out = ta.seg_S0 + sidx;
 #pragma unroll
-    for (int m = 0; m < 64; ++m) acc[m] = bg[m];
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int k = 0; k < NV; ++k) out[(size_t)(c0 + i) * D + vg + k] = st[i][k];
+    if (g + 1 == G) break;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int k = 0; k < NV; ++k) Ss[(c0 + i) * VC + vl + k] = st[i][k];
+    if (tid == 0 && g + 1 < G - 1) fetch(g + 1);  // its buffer was released by the last step's barrier
+    const float *bg = ta.seg_b + sidx;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int k = 0; k < NV; ++k) st[i][k] = bg[(size_t)(c0 + i) * D + vg + k];
+    bool ok = true;
+    if (tid == 0) ok = mbar_wait_ool(&mfull[g & 1], (g >> 1) & 1, a.status, 231);
+    if (__syncthreads_or(!ok)) {  // gave up: let the copy into the other buffer land first
+      if (tid == 0 && g + 1 < G - 1) mbar_wait_ool(&mfull[(g + 1) & 1], ((g + 1) >> 1) & 1, a.status, 232);
+      return;
+    }
+    const float *Mb = Mt + (g & 1) * D * D;
 #pragma unroll 4
     for (int jj = 0; jj < D; ++jj) {
-      const float mcj = M[c * D + jj];
-      const float4 *srow = reinterpret_cast<const float4 *>(S + jj * D + v0);
-#pragma unroll
-      for (int m4 = 0; m4 < 16; ++m4) {
-        const float4 x = srow[m4];
-        acc[4 * m4] += mcj * x.x;
-        acc[4 * m4 + 1] += mcj * x.y;
-        acc[4 * m4 + 2] += mcj * x.z;
-        acc[4 * m4 + 3] += mcj * x.w;
+      const float4 m = *reinterpret_cast<const float4 *>(Mb + jj * D + c0);
+      float sv[NV];
+      if constexpr (NV == 4) {
+        const float4 x = *reinterpret_cast<const float4 *>(Ss + jj * VC + vl);
+        sv[0] = x.x; sv[1] = x.y; sv[2] = x.z; sv[3] = x.w;
+      } else {
+        const float2 x = *reinterpret_cast<const float2 *>(Ss + jj * VC + vl);
+        sv[0] = x.x; sv[1] = x.y;
       }
-    }
-    __syncthreads();  // every read of S and M is done
+      const float mv[4] = {m.x, m.y, m.z, m.w};
 #pragma unroll
-    for (int m4 = 0; m4 < 16; ++m4)
-      reinterpret_cast<float4 *>(S + c * D + v0)[m4] = make_float4(acc[4 * m4], acc[4 * m4 + 1], acc[4 * m4 + 2], acc[4 * m4 + 3]);
-    __syncthreads();
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int k = 0; k < NV; ++k) st[i][k] = fmaf(mv[i], sv[k], st[i][k]);
+    }
+    __syncthreads();  // every read of Ss and of this M buffer is done
   }
 }
 
@@ -1020,7 +1055,8 @@ size_t tc_record_bytes() { return REC; }
 // Segments per sequence for the segment scan: only for batched calls whose
 // (sequence, head) pairs fill at most half the SMs and whose sequences are
 // long (>= 32 chunks); at least 16 chunks per segment, at most one wave of
-// CTAs.  0: run the plain sequential state pass.
+// CTAs, and only where the estimate below says it pays.  0: run the plain
+// sequential state pass.
 int tc_seg_count(int B, int H, int NC) {
   (void)tc_intra_ctas();  // SM count
   const int sms = g_num_sms > 0 ? g_num_sms : 148;
@@ -1030,7 +1066,11 @@ int tc_seg_count(int B, int H, int NC) {
   if (G > NC / 16) G = NC / 16;
   if (G < 2) return 0;
   const int L = (NC + G - 1) / G;
-  return (NC + L - 1) / L;
+  G = (NC + L - 1) / L;
+  // the maps and the segments' state passes each take about L chunk steps,
+  // the scan about one per segment: keep it only where that beats NC steps
+  if (2 * L + G + 4 > NC) return 0;
+  return G;
 }
 size_t tc_seg_ws_bytes() {
   (void)tc_intra_ctas();  // SM count
@@ -1070,12 +1110,16 @@ cudaError_t tc_forward(const FwdArgs &f, unsigned char *recs, float *fb, bool wr
       ta.seg_M = seg_ws;
       ta.seg_b = seg_ws + per;
       ta.seg_S0 = seg_ws + 2 * per;
-      const size_t sm_map = SG_MISC + sizeof(SegMisc) + 1024, sm_scan = 2 * D * D * sizeof(float);
+      // value-column slices of the scan: 8 (16 columns) while the CTAs fit on the SMs, else 4
+      const int split = 8 * f.B * f.H <= g_num_sms ? 8 : 4;
+      const size_t sm_map = SG_MISC + sizeof(SegMisc) + 1024;
+      const size_t sm_scan = 128 + (2 * D * D + D * (D / split)) * sizeof(float) + 2 * sizeof(uint64_t);
       if ((e = cudaFuncSetAttribute(tc_segmap_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     (int)sm_map)) != cudaSuccess)
         return e;
-      if ((e = cudaFuncSetAttribute(tc_segscan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    (int)sm_scan)) != cudaSuccess)
+      auto scan = split == 8 ? tc_segscan_kernel<16> : tc_segscan_kernel<32>;
+      if ((e = cudaFuncSetAttribute(scan, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_scan)) !=
+          cudaSuccess)
         return e;
       {
         ProfScope prof("tc_segmap", s);
@@ -1084,7 +1128,7 @@ cudaError_t tc_forward(const FwdArgs &f, unsigned char *recs, float *fb, bool wr
       }
       {
         ProfScope prof("tc_segscan", s);
-        tc_segscan_kernel<<<dim3(f.H, f.B), kScanThreads, sm_scan, s>>>(ta);
+        scan<<<dim3(f.H, f.B, split), kScanThreads, sm_scan, s>>>(ta);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
       }
       ProfScope prof(write_o ? "tc_state_fwd" : "tc_state_fwd_recompute", s);

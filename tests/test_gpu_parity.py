@@ -226,6 +226,21 @@ def test_long_sequence_segment_scan(B, H):
         check(key, got[key], ref[key], io)
 
 
+def test_long_sequence_segment_scan_many_pairs():
+    """20 (sequence, head) pairs over 64 chunks: four segments of 16 chunks,
+    the scan split into four value-column slices per pair.  Forward chunk
+    states and final state against the oracle."""
+    io = torch.bfloat16
+    B, H, T = 2, 10, 64 * 63 + 9
+    inp = random_inputs(B, T, H, 128, 128, io, seed=47, gscale=0.05, extreme_p=0.05)
+    o, ST, cs = _fwd(inp, S0=inp["S0"], chunk_states=True)
+    o_ref, ST_ref, cs_ref = oracle_fwd_batched(inp, S0=inp["S0"], chunk=64)
+    check("o", o, o_ref, io)
+    check("ST", ST, ST_ref, io)
+    NC = (T + 63) // 64
+    check("chunk states", cs, cs_ref.reshape(B, NC, H, 128, 128).transpose(0, 2, 1, 3, 4), io)
+
+
 def test_backward_without_state_inputs():
     io = torch.float32
     inp = random_inputs(1, 100, 2, 64, 64, io, seed=12)
