@@ -2,7 +2,7 @@
 """Benchmark of the CKDA recurrence library on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload fwdbwd|kda|fwd|varlen|long|decode]
+                    [--workload fwdbwd|kda|fwd|varlen|long|decode|decode_multi]
 
 Default workload (the headline): one step = ckda_chunk_fwd (saving its
 per-chunk results for the backward) + ckda_chunk_bwd on B=8, H=16, T=4096,
@@ -314,6 +314,27 @@ def run_secondary(args, rank, world, local_rank):
         metric = "CKDA decode tokens/s (N=256,H=16,d=128,bf16 I/O,fp32 state)"
         cfg = {"workload": w.name, "N": N, "H": H, "dk": dk, "dv": dv, "io_dtype": "bf16",
                "state_dtype": "f32", "l2": "state (256 MiB) larger than L2"}
+    elif args.workload == "decode_multi":
+        w = W.DECODE_MULTI
+        N, K, H, dk, dv = w.B, w.T, w.H, w.dk, w.dv
+        pool = W.make_decode_pool(w).to(dev)
+        calls = [{k: v.to(dev) for k, v in W.make_decode_multi(w, c).items()} for c in range(8)]
+        o = torch.empty(N, K, H, dv, dtype=w.io_dtype, device=dev)
+        code = api.io_code(w.io_dtype)
+        it = [0]
+
+        def step():
+            x = calls[it[0] % len(calls)]
+            it[0] += 1
+            _abi.ckda_decode_multi(N, K, H, dk, dv, code, x["q"], x["k"], x["v"], x["g"], x["sign"], x["beta"],
+                                   None, x["slots"], pool.shape[0], pool, True, o)
+        units, per_unit, unit_name = N * H, DECODE_BYTES_PER_NH + (K - 1) * FWD_BYTES, \
+            "B per (sequence, head) call of %d tokens" % K
+        tokens = N * K
+        metric = "CKDA multi-token decode tokens/s (N=256,K=4,H=16,d=128,bf16 I/O,fp32 state pool)"
+        cfg = {"workload": w.name, "N": N, "K": K, "H": H, "dk": dk, "dv": dv, "io_dtype": "bf16",
+               "state_dtype": "f32", "n_slots": pool.shape[0],
+               "l2": "touched states (256 MiB) larger than L2"}
     elif args.workload == "varlen":
         w = W.VARLEN
         inp = W.make_varlen(w)
@@ -558,7 +579,7 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer pass")
-    ap.add_argument("--workload", choices=["fwdbwd", "kda", "fwd", "varlen", "long", "decode"], default="fwdbwd",
+    ap.add_argument("--workload", choices=["fwdbwd", "kda", "fwd", "varlen", "long", "decode", "decode_multi"], default="fwdbwd",
                     help="fwdbwd is the headline; the others are secondary measurements")
     ap.add_argument("--batch", type=int, default=0,
                     help="override B (profiling a smaller case; not a bench line)")

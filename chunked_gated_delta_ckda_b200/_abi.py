@@ -52,6 +52,7 @@ def _load():
         lib.ckda_chunk_fwd.argtypes = [I] * 6 + [P] * 11 + [Z, P, Z, P]
         lib.ckda_chunk_bwd.argtypes = [I] * 6 + [P] * 11 + [Z] + [P] * 7 + [Z, P]
         lib.ckda_decode_step.argtypes = [I] * 5 + [P] * 9
+        lib.ckda_decode_multi.argtypes = [I] * 6 + [P] * 8 + [I, P, I, P, P]
         lib.ckda_varlen_fwd.argtypes = [I, I, P, I, I, I, I, I] + [P] * 10 + [Z, P]
         lib.ckda_chunk_fwd_noalloc.argtypes = [I] * 6 + [P] * 11
         lib.ckda_check_device_status.argtypes = [P, P]
@@ -64,7 +65,7 @@ def _load():
                                          ctypes.POINTER(ctypes.c_double)]
         lib.ckda_profile_reset.argtypes = []
         lib.ckda_profile_reset.restype = None
-        for f in ("ckda_chunk_fwd", "ckda_chunk_bwd", "ckda_decode_step", "ckda_varlen_fwd",
+        for f in ("ckda_chunk_fwd", "ckda_chunk_bwd", "ckda_decode_step", "ckda_decode_multi", "ckda_varlen_fwd",
                   "ckda_chunk_fwd_noalloc", "ckda_check_device_status", "ckda_version", "ckda_profile_enable",
                   "ckda_profile_collect", "ckda_profile_get"):
             getattr(lib, f).restype = I
@@ -140,6 +141,13 @@ def ckda_chunk_bwd(B, T, H, dk, dv, io_dtype, q, k, v, g, sign, beta, S0, dO, dS
 def ckda_decode_step(N, H, dk, dv, io_dtype, q, k, v, g, sign, beta, state, o, stream=None):
     _check(_load().ckda_decode_step(N, H, dk, dv, io_dtype, _p(q), _p(k), _p(v), _p(g), _p(sign),
                                     _p(beta), _p(state), _p(o), _s(stream)), "ckda_decode_step")
+
+
+def ckda_decode_multi(N, K, H, dk, dv, io_dtype, q, k, v, g, sign, beta, n_tokens, slots, n_slots, state,
+                      write_state, o, stream=None):
+    _check(_load().ckda_decode_multi(N, K, H, dk, dv, io_dtype, _p(q), _p(k), _p(v), _p(g), _p(sign),
+                                     _p(beta), _p(n_tokens), _p(slots), n_slots, _p(state),
+                                     1 if write_state else 0, _p(o), _s(stream)), "ckda_decode_multi")
 
 
 def ckda_varlen_fwd(total_T, N, cu_seqlens, max_seqlen, H, dk, dv, io_dtype, q, k, v, g, sign,

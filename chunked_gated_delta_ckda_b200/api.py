@@ -6,6 +6,8 @@ torch (device memory is torch's job here) and call the library.
     o, ST, cs, sv = chunk_fwd(..., save_chunk_states=True, save_for_backward=True)
     grads     = chunk_bwd(..., chunk_states=cs, saved=sv)   # no recomputation
     o         = decode_step(q, k, v, g, sign, beta, state)     # state updated in place
+    o         = decode_multi(q, k, v, g, sign, beta, pool, slots=None, n_tokens=None,
+                             write_state=True)                 # K tokens per sequence
     o, ST     = varlen_fwd(q, k, v, g, sign, beta, cu_seqlens, max_seqlen, S0=None)
 
 Shapes and dtypes are those of include/ckda.h: q, k, g, sign [B,T,H,dk]; v
@@ -112,6 +114,26 @@ def decode_step(q, k, v, g, sign, beta, state, o=None):
     if o is None:
         o = torch.empty(N, H, dv, dtype=q.dtype, device=q.device)
     _abi.ckda_decode_step(N, H, dk, dv, io_code(q.dtype), q, k, v, g, sign, beta, state, o)
+    return o
+
+
+def decode_multi(q, k, v, g, sign, beta, pool, slots=None, n_tokens=None, write_state=True, o=None,
+                 want_o=True):
+    """K steps per sequence: q, k, g, sign [N,K,H,dk]; v [N,K,H,dv]; beta [N,K,H];
+    pool [n_slots,H,dk,dv] fp32 (updated in place when write_state);
+    slots / n_tokens: int32 [N] on the device, or None (slot n / all K)."""
+    q, k, v, g, sign, beta, slots, n_tokens = map(_c, (q, k, v, g, sign, beta, slots, n_tokens))
+    if not pool.is_contiguous() or pool.dtype != torch.float32:
+        raise ValueError("pool must be a contiguous float32 tensor")
+    for t in (slots, n_tokens):
+        if t is not None and t.dtype != torch.int32:
+            raise TypeError("slots and n_tokens must be int32")
+    N, K, H, dk = q.shape
+    dv = v.shape[-1]
+    if o is None and want_o:
+        o = torch.empty(N, K, H, dv, dtype=q.dtype, device=q.device)
+    _abi.ckda_decode_multi(N, K, H, dk, dv, io_code(q.dtype), q, k, v, g, sign, beta, n_tokens, slots,
+                           pool.shape[0], pool, write_state, o)
     return o
 
 

@@ -266,6 +266,21 @@ int ckda_decode_step(int N, int H, int dk, int dv, int io_dtype, const void *q, 
                                  state, o, stream));
 }
 
+int ckda_decode_multi(int N, int K, int H, int dk, int dv, int io_dtype, const void *q, const void *k,
+                      const void *v, const float *g, const int8_t *sign, const void *beta,
+                      const int32_t *n_tokens, const int32_t *slots, int n_slots, float *state,
+                      int write_state, void *o, cudaStream_t stream) {
+  CKDA_TRY(check_common(N, K, H, dk, dv, io_dtype));
+  if (n_slots < 0 || (write_state != 0 && write_state != 1)) return CKDA_ERR_INVALID_ARG;
+  if (!slots && n_slots < N) return CKDA_ERR_INVALID_ARG;
+  if (N == 0 || K == 0) return CKDA_OK;
+  CKDA_TRY(check_ptrs({q, k, v, g, beta, state}, {sign, o}));
+  if ((reinterpret_cast<uintptr_t>(n_tokens) & 3u) != 0 || (reinterpret_cast<uintptr_t>(slots) & 3u) != 0)
+    return CKDA_ERR_ALIGNMENT;
+  return cuda_status(decode_multi(N, K, H, dk, dv, io_dtype == CKDA_BF16, q, k, v, g, sign, beta, n_tokens,
+                                  slots, n_slots, state, write_state == 1, o, stream));
+}
+
 int ckda_varlen_fwd(int total_T, int N, const int32_t *cu_seqlens, int max_seqlen, int H,
                     int dk, int dv, int io_dtype, const void *q, const void *k, const void *v,
                     const float *g, const int8_t *sign, const void *beta, const float *S0,

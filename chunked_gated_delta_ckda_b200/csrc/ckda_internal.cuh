@@ -202,5 +202,9 @@ cudaError_t tc_backward(const BwdArgs &b, const unsigned char *recs, unsigned ch
 cudaError_t decode_step(int N, int H, int dk, int dv, bool bf16, const void *q,
                         const void *k, const void *v, const float *g, const int8_t *sign,
                         const void *beta, float *state, void *o, cudaStream_t s);
+cudaError_t decode_multi(int N, int K, int H, int dk, int dv, bool bf16, const void *q, const void *k,
+                         const void *v, const float *g, const int8_t *sign, const void *beta,
+                         const int32_t *n_tokens, const int32_t *slots, int n_slots, float *state,
+                         bool write_state, void *o, cudaStream_t s);
 
 }  // namespace ckda

@@ -73,6 +73,13 @@ DECODE = Workload("decode_bf16", B=256, H=16, T=1, dk=128, dv=128, io_dtype=torc
                   seed=4, with_S0=True, decode_steps=512,
                   note="recurrent decode, 512 consecutive one-token steps")
 
+# Multi-token decode on a slot pool: 256 live sequences placed at random in a
+# pool of 512 states, 4 tokens each per call (a speculative-decoding verify
+# width; every call commits all 4).
+DECODE_MULTI = Workload("decode_multi_bf16", B=256, T=4, H=16, dk=128, dv=128, io_dtype=torch.bfloat16,
+                        seed=5, with_S0=True, decode_steps=64, extra={"n_slots": 512},
+                        note="4 tokens per sequence per call, states in a 512-slot pool")
+
 
 def _gen(seed: int) -> torch.Generator:
     gen = torch.Generator(device="cpu")
@@ -178,3 +185,19 @@ def make_decode_step(w: Workload = DECODE, step: int = 0, N: Optional[int] = Non
     H = w.H if H is None else H
     gen = _gen(w.seed * 1_000_003 + 7919 * (step + 1))
     return draw((N,), H, w.dk, w.dv, w.io_dtype, gen, w.g_floor, w.extreme_p)
+
+
+def make_decode_multi(w: Workload = DECODE_MULTI, call: int = 0) -> dict:
+    """Per-token inputs [N, K, H, d] of multi-token decode call ``call``
+    (independently seeded per call) and the slot table: a fixed random
+    placement of the N sequences in the pool."""
+    N, K = w.B, w.T
+    gen = _gen(w.seed * 1_000_003 + 7919 * (call + 1))
+    out = draw((N, K), w.H, w.dk, w.dv, w.io_dtype, gen, w.g_floor, w.extreme_p)
+    out["slots"] = torch.randperm(w.extra["n_slots"], generator=_gen(w.seed))[:N].to(torch.int32)
+    return out
+
+
+def make_decode_pool(w: Workload = DECODE_MULTI) -> torch.Tensor:
+    """The state pool [n_slots, H, dk, dv], N(0, 0.1^2)."""
+    return 0.1 * torch.randn(w.extra["n_slots"], w.H, w.dk, w.dv, generator=_gen(w.seed + 1))

@@ -153,6 +153,33 @@ int ckda_decode_step(int N, int H, int dk, int dv, int io_dtype, const void *q,
                      const int8_t *sign, const void *beta, float *state,
                      void *o, cudaStream_t stream);
 
+/* Up to K recurrent steps per sequence in one pass over its state: batched
+ * multi-token decode, and the verify / commit halves of speculative decoding
+ * (the model card's "purely recurrent" inference form; each step is the one
+ * of ckda_decode_step).  States live in a pool addressed through a slot table
+ * (continuous batching: a sequence's state stays in its slot while the batch
+ * around it changes).
+ *   q, k [N,K,H,dk] io;  v [N,K,H,dv] io;  g [N,K,H,dk] f32;  sign [N,K,H,dk]
+ *         int8, nullable (all +1: KDA);  beta [N,K,H] io.  Token t of
+ *         sequence n is row (n, t), in order.
+ *   n_tokens [N] int32 DEVICE, nullable (all K): steps taken by sequence n;
+ *         values are clamped to [0, K].
+ *   slots [N] int32 DEVICE, nullable (slot n, needs n_slots >= N): the pool
+ *         slot of sequence n; a slot < 0 or >= n_slots skips the sequence
+ *         (its o rows are zero and no state is touched).  Two sequences must
+ *         not name the same slot when write_state is 1.
+ *   state [n_slots,H,dk,dv] f32, the pool (true frame).
+ *   write_state: 1 writes the state after the n_tokens steps back into the
+ *         slot; 0 leaves the pool untouched (verify: outputs only).
+ *   o [N,K,H,dv] io, nullable: rows t >= n_tokens[n] are zero.
+ * No workspace. */
+int ckda_decode_multi(int N, int K, int H, int dk, int dv, int io_dtype,
+                      const void *q, const void *k, const void *v,
+                      const float *g, const int8_t *sign, const void *beta,
+                      const int32_t *n_tokens, const int32_t *slots, int n_slots,
+                      float *state, int write_state, void *o,
+                      cudaStream_t stream);
+
 /* Chunked forward over N packed documents (training packs documents back to
  * back; the state restarts at each boundary).
  *   cu_seqlens [N+1] int32 DEVICE: cu[0] = 0, non-decreasing, cu[N] = total_T

@@ -157,6 +157,43 @@ def decode(q, k, v, g, sign, beta, state, nthreads=0):
     return o, st
 
 
+def decode_multi(q, k, v, g, sign, beta, pool, n_tokens=None, slots=None, write_state=True,
+                 nthreads=0):
+    """Up to K recurrent steps per sequence on states held in a slot pool
+    ("openeurollm/complex-kda-1.3B-100B" model card: purely recurrent
+    inference, one token at a time), written as repeated ``decode`` steps.
+
+    q, k, g, sign: [N,K,H,dk]; v: [N,K,H,dv]; beta: [N,K,H]; pool:
+    [n_slots,H,dk,dv].  Sequence n starts from pool[slots[n]] (slot n when
+    slots is None) and takes n_tokens[n] steps (clamped to [0, K]; K when
+    None); a slot outside [0, n_slots) skips the sequence.  Returns (o
+    [N,K,H,dv], with zero rows for the steps not taken; the pool after the
+    steps when write_state, else an unchanged copy)."""
+    q, k, v, g, beta = map(_f64, (q, k, v, g, beta))
+    N, K, H, dk = q.shape
+    dv = v.shape[-1]
+    sign = np.ones((N, K, H, dk), dtype=np.int8) if sign is None else _sign(sign)
+    pool = np.array(pool, dtype=np.float64, copy=True, order="C")
+    n_slots = pool.shape[0]
+    nt = np.full(N, K, dtype=np.int64) if n_tokens is None else np.clip(np.asarray(n_tokens, np.int64), 0, K)
+    sl = np.arange(N, dtype=np.int64) if slots is None else np.asarray(slots, np.int64)
+    live = np.array([n for n in range(N) if 0 <= sl[n] < n_slots], dtype=np.int64)
+    o = np.zeros((N, K, H, dv))
+    st = pool[sl[live]] if len(live) else np.zeros((0, H, dk, dv))
+    for t in range(K):
+        act = np.nonzero(nt[live] > t)[0]
+        if len(act) == 0:
+            break
+        seqs = live[act]
+        ot, new = decode(q[seqs, t], k[seqs, t], v[seqs, t], g[seqs, t], sign[seqs, t], beta[seqs, t],
+                         st[act], nthreads=nthreads)
+        o[seqs, t] = ot
+        st[act] = new
+    if write_state and len(live):
+        pool[sl[live]] = st
+    return o, pool
+
+
 def batched_cu_seqlens(B: int, T: int) -> np.ndarray:
     """Offsets of B back-to-back sequences of length T ([B,T,...] == [B*T,...])."""
     return np.arange(B + 1, dtype=np.int64) * T

@@ -105,3 +105,18 @@ def test_host_validation_without_gpu():
     assert bwd(1, b, 1 << 30, [fake, 16]) == 4
     # zero-sized decode is a no-op
     assert lib.ckda_decode_step(0, 2, 64, 64, 0, *([None] * 8), None) == 0
+
+    def multi(N=4, K=3, dk=64, dv=64, io=0, ptrs=None, n_tokens=None, slots=None, n_slots=4, write=1):
+        p = [fake] * 6 if ptrs is None else ptrs
+        return lib.ckda_decode_multi(N, K, 2, dk, dv, io, *p, n_tokens, slots, n_slots, fake, write, fake, None)
+
+    assert multi(N=-1) == 1 and multi(K=-1) == 1
+    assert multi(dk=96) == 2
+    assert multi(io=7) == 1
+    assert multi(write=2) == 1
+    assert multi(n_slots=3) == 1                      # identity slots need n_slots >= N
+    assert multi(n_slots=-1, slots=fake) == 1
+    assert multi(ptrs=[None] + [fake] * 5) == 1       # q missing
+    assert multi(ptrs=[fake, odd] + [fake] * 4) == 3  # k misaligned
+    assert multi(n_tokens=ctypes.c_void_p((1 << 20) + 2)) == 3
+    assert multi(N=0) == 0 and multi(K=0) == 0        # nothing to do

@@ -330,6 +330,88 @@ def test_decode_steps(io, dk, dv):
         check("state[%d]" % t, st_dev, st_ref, io)
 
 
+@pytest.mark.parametrize("io", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("dk,dv", [(128, 128), (64, 128), (128, 64), (64, 64)])
+@pytest.mark.parametrize("K", [1, 3, 8])
+def test_decode_multi_pool(io, dk, dv, K):
+    """Several steps per sequence on a slot pool: permuted slots, skipped
+    sequences (slot -1 and slot n_slots), ragged step counts (0 .. K, one
+    clamped from above), no sign tensor on one case; verify (no write-back)
+    then commit, against the oracle."""
+    N, H, n_slots = 6, 3, 9
+    x = random_inputs(N, K, H, dk, dv, io, seed=7 * K + dk + dv)
+    pool = 0.1 * torch.randn(n_slots, H, dk, dv, generator=torch.Generator().manual_seed(K + dk))
+    slots = torch.tensor([4, 0, -1, 8, 2, 9], dtype=torch.int32)
+    n_tok = torch.tensor([K, 0, K, 1, K + 5, max(K - 1, 0)], dtype=torch.int32)
+    sign = None if (K == 3 and dk == 64) else x["sign"]
+    d = to_dev(x)
+    sg = None if sign is None else d["sign"]
+    args = (d["q"], d["k"], d["v"], d["g"], sg, d["beta"])
+    P = lambda t: f64(t)
+    oargs = (P(x["q"]), P(x["k"]), P(x["v"]), P(x["g"]), None if sign is None else sign.numpy(), P(x["beta"]))
+    dev_pool = pool.cuda()
+    o_ver = api.decode_multi(*args, dev_pool, slots=slots.cuda(), n_tokens=None, write_state=False)
+    torch.cuda.synchronize()
+    assert torch.equal(dev_pool.cpu(), pool)  # verify leaves the pool untouched
+    ref_o, _ = oracle.decode_multi(*oargs, P(pool), n_tokens=None, slots=slots.numpy(), write_state=False)
+    check("o (verify)", o_ver, ref_o, io)
+    o_com = api.decode_multi(*args, dev_pool, slots=slots.cuda(), n_tokens=n_tok.cuda(), write_state=True)
+    torch.cuda.synchronize()
+    ref_o, ref_pool = oracle.decode_multi(*oargs, P(pool), n_tokens=n_tok.numpy(), slots=slots.numpy())
+    check("o (commit)", o_com, ref_o, io)
+    check("pool", dev_pool, ref_pool, io)
+    untouched = [s for s in range(n_slots) if s not in (4, 8, 2)]
+    assert torch.equal(dev_pool.cpu()[untouched], pool[untouched])
+
+
+@pytest.mark.parametrize("io,d", [(torch.bfloat16, 128), (torch.float32, 64)])
+def test_decode_multi_many_items_per_cta(io, d):
+    """More (sequence, head, column slice) items than resident CTAs, so every
+    CTA walks several items and prefetches the next one's state: skipped and
+    zero-step sequences interleaved, ragged step counts, a permuted pool."""
+    N, K, H, n_slots = 160, 3, 4, 200
+    x = random_inputs(N, K, H, d, d, io, seed=91 + d)
+    gen = torch.Generator().manual_seed(d)
+    pool = 0.1 * torch.randn(n_slots, H, d, d, generator=gen)
+    slots = torch.randperm(n_slots, generator=gen)[:N].to(torch.int32)
+    slots[torch.rand(N, generator=gen) < 0.1] = -1
+    n_tok = torch.randint(0, K + 1, (N,), generator=gen, dtype=torch.int32)
+    d_ = to_dev(x)
+    dev_pool = pool.cuda()
+    o = api.decode_multi(d_["q"], d_["k"], d_["v"], d_["g"], d_["sign"], d_["beta"], dev_pool, slots=slots.cuda(),
+                         n_tokens=n_tok.cuda())
+    torch.cuda.synchronize()
+    ref_o, ref_pool = oracle.decode_multi(f64(x["q"]), f64(x["k"]), f64(x["v"]), f64(x["g"]), x["sign"].numpy(),
+                                          f64(x["beta"]), f64(pool), n_tokens=n_tok.numpy(), slots=slots.numpy())
+    check("o", o, ref_o, io)
+    check("pool", dev_pool, ref_pool, io)
+
+
+def test_decode_multi_matches_decode_steps():
+    """K steps in one call against K single-step calls (the existing decode
+    kernel) on the same states: both against the oracle, and close to each
+    other."""
+    io, N, K, H, dk, dv = torch.bfloat16, 4, 5, 2, 128, 128
+    x = random_inputs(N, K, H, dk, dv, io, seed=77)
+    state = 0.1 * torch.randn(N, H, dk, dv, generator=torch.Generator().manual_seed(5))
+    d = to_dev(x)
+    a = state.cuda()
+    o_multi = api.decode_multi(d["q"], d["k"], d["v"], d["g"], d["sign"], d["beta"], a)
+    b = state.cuda()
+    outs = []
+    for t in range(K):
+        outs.append(api.decode_step(*(d[n][:, t].contiguous() for n in ("q", "k", "v", "g", "sign", "beta")), b))
+    torch.cuda.synchronize()
+    o_steps = torch.stack(outs, 1)
+    ref_o, ref_pool = oracle.decode_multi(f64(x["q"]), f64(x["k"]), f64(x["v"]), f64(x["g"]), x["sign"].numpy(),
+                                          f64(x["beta"]), f64(state))
+    check("o (multi)", o_multi, ref_o, io)
+    check("o (steps)", o_steps, ref_o, io)
+    check("state (multi)", a, ref_pool, io)
+    check("state (steps)", b, ref_pool, io)
+    assert (a - b).abs().max().item() < 1e-4
+
+
 def test_decode_continues_chunked_final_state():
     """States cross the ABI in the true frame: decode after a chunked forward
     equals one forward over the concatenation."""

@@ -354,6 +354,62 @@ def test_decode_steps_equal_forward():
     np.testing.assert_array_equal(st, ST)
 
 
+def test_decode_multi_equals_forward_per_sequence():
+    """Several steps per sequence from pooled, permuted slots with ragged step
+    counts: each sequence's outputs and final state are the token forward's
+    over its first n_tokens tokens from its slot's state (state
+    continuation), untouched slots stay bitwise, skipped sequences give zeros."""
+    N, K, H, dk, dv, n_slots = 5, 4, 2, 5, 3, 8
+    q, k, v, g, sign, beta = rand_inputs(RNG, N * K, H, dk, dv)
+    shp = lambda x: x.reshape(N, K, *x.shape[1:])
+    q, k, v, g, sign, beta = map(shp, (q, k, v, g, sign, beta))
+    pool = RNG.standard_normal((n_slots, H, dk, dv))
+    slots = np.array([6, 1, -1, 3, 8])      # -1 and 8 (= n_slots) are skipped
+    n_tok = np.array([4, 0, 2, 9, 1])       # 9 is clamped to K
+    o, new = oracle.decode_multi(q, k, v, g, sign, beta, pool, n_tokens=n_tok, slots=slots)
+    for n in range(N):
+        s = slots[n]
+        if not 0 <= s < n_slots:
+            assert np.all(o[n] == 0)
+            continue
+        L = min(int(n_tok[n]), K)
+        if L:
+            on, Sn, _ = oracle.fwd([0, L], q[n, :L], k[n, :L], v[n, :L], g[n, :L], sign[n, :L], beta[n, :L],
+                                   S0=pool[s:s + 1])
+            np.testing.assert_array_equal(o[n, :L], on)
+            np.testing.assert_array_equal(new[s], Sn[0])
+        else:
+            np.testing.assert_array_equal(new[s], pool[s])
+        assert np.all(o[n, L:] == 0)
+    for s in set(range(n_slots)) - {6, 1, 3}:
+        np.testing.assert_array_equal(new[s], pool[s])
+    # verify (no write-back): same outputs, pool unchanged
+    o2, same = oracle.decode_multi(q, k, v, g, sign, beta, pool, n_tokens=n_tok, slots=slots,
+                                   write_state=False)
+    np.testing.assert_array_equal(o2, o)
+    np.testing.assert_array_equal(same, pool)
+
+
+def test_decode_multi_commit_after_verify():
+    """Speculative decoding: verifying K draft tokens and then committing the
+    first a of them leaves the state the forward over those a tokens gives."""
+    N, K, H, dk, dv = 3, 5, 1, 4, 4
+    q, k, v, g, sign, beta = rand_inputs(RNG, N * K, H, dk, dv)
+    shp = lambda x: x.reshape(N, K, *x.shape[1:])
+    q, k, v, g, sign, beta = map(shp, (q, k, v, g, sign, beta))
+    pool = RNG.standard_normal((N, H, dk, dv))
+    o_ver, _ = oracle.decode_multi(q, k, v, g, sign, beta, pool, write_state=False)
+    acc = np.array([2, 5, 0])
+    o_com, new = oracle.decode_multi(q, k, v, g, sign, beta, pool, n_tokens=acc)
+    for n in range(N):
+        np.testing.assert_array_equal(o_com[n, :acc[n]], o_ver[n, :acc[n]])
+        ref = pool[n:n + 1]
+        if acc[n]:
+            _, ref, _ = oracle.fwd([0, acc[n]], q[n, :acc[n]], k[n, :acc[n]], v[n, :acc[n]], g[n, :acc[n]],
+                                   sign[n, :acc[n]], beta[n, :acc[n]], S0=pool[n:n + 1])
+        np.testing.assert_array_equal(new[n], ref[0])
+
+
 # ---------------------------------------------------------------------------
 # gradients against central finite differences of the oracle's forward
 # ---------------------------------------------------------------------------

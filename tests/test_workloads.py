@@ -51,3 +51,13 @@ def test_decode_steps_independent():
     b = W.make_decode_step(W.DECODE, step=3, N=4, H=2)
     c = W.make_decode_step(W.DECODE, step=4, N=4, H=2)
     assert torch.equal(a["q"], b["q"]) and not torch.equal(a["q"], c["q"])
+
+
+def test_decode_multi_slots_are_distinct_and_in_pool():
+    w = W.DECODE_MULTI
+    x = W.make_decode_multi(w, call=2)
+    assert x["q"].shape == (w.B, w.T, w.H, w.dk) and x["beta"].shape == (w.B, w.T, w.H)
+    s = x["slots"]
+    assert s.dtype == torch.int32 and len(set(s.tolist())) == w.B
+    assert int(s.min()) >= 0 and int(s.max()) < w.extra["n_slots"]
+    assert torch.equal(s, W.make_decode_multi(w, call=3)["slots"])   # placement fixed across calls
