@@ -197,3 +197,6 @@ def decode_multi(q, k, v, g, sign, beta, pool, n_tokens=None, slots=None, write_
 def batched_cu_seqlens(B: int, T: int) -> np.ndarray:
     """Offsets of B back-to-back sequences of length T ([B,T,...] == [B*T,...])."""
     return np.arange(B + 1, dtype=np.int64) * T
+
+
+from .prologue import prologue_bwd, prologue_fwd  # noqa: E402,F401  (the token-mixer prologue)
