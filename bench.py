@@ -2,7 +2,7 @@
 """Benchmark of the CKDA recurrence library on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload fwdbwd|kda|fwd|varlen|long|decode|decode_multi]
+                    [--workload fwdbwd|kda|fwd|varlen|long|decode|decode_multi|prologue]
 
 Default workload (the headline): one step = ckda_chunk_fwd (saving its
 per-chunk results for the backward) + ckda_chunk_bwd on B=8, H=16, T=4096,
@@ -46,6 +46,11 @@ FALLBACK_BF16_TFLOPS = 1590.0
 FWD_FLOP, FWD_BYTES = 139264, 1666
 BWD_FLOP, BWD_BYTES = 278528, 2948
 DECODE_BYTES_PER_NH = 131072 + 1666  # state read + write, per-token inputs and output
+# prologue per token-head (bf16 I/O, fp32 gate): forward reads xq, xk, xv 768 +
+# a 512 + b 2, writes q, k, v 768 + g 512 + sign 128 + beta 2; backward reads
+# the forward's inputs 1282 and dq, dk, dv 768 + dg 512 + dbeta 2, writes
+# dxq, dxk, dxv 768 + da 512 + db 2 (the taps' gradients are per channel)
+PROLOGUE_FWD_BYTES, PROLOGUE_BWD_BYTES = 2692, 3846
 
 # Which per-unit figure a kernel's roofline uses (the call it implements).
 KERNEL_UNITS = {
@@ -295,6 +300,7 @@ def run_secondary(args, rank, world, local_rank):
     torch.cuda.set_device(dev)
     peaks = measured_peaks()
     clocks = ClockSampler(local_rank)
+    kernel_bytes = {}
     if args.workload == "decode":
         w = W.DECODE
         N, H, dk, dv = w.B, w.H, w.dk, w.dv
@@ -335,6 +341,31 @@ def run_secondary(args, rank, world, local_rank):
         cfg = {"workload": w.name, "N": N, "K": K, "H": H, "dk": dk, "dv": dv, "io_dtype": "bf16",
                "state_dtype": "f32", "n_slots": pool.shape[0],
                "l2": "touched states (256 MiB) larger than L2"}
+    elif args.workload == "prologue":
+        w = W.LAYER_FWDBWD
+        x = {k: v.to(dev) for k, v in W.make_prologue(w).items()}
+        B, T, H, dk, dv = w.B, w.T, w.H, w.dk, w.dv
+        code = api.io_code(w.io_dtype)
+        e = lambda t, dt=None: torch.empty_like(t, dtype=dt) if dt else torch.empty_like(t)
+        outs = dict(q=e(x["xq"]), k=e(x["xk"]), v=e(x["xv"]), g=e(x["a"]), sign=e(x["a"], torch.int8),
+                    beta=e(x["b"]))
+        grads = dict(dxq=e(x["xq"]), dxk=e(x["xk"]), dxv=e(x["xv"]), dwq=e(x["wq"]), dwk=e(x["wk"]),
+                     dwv=e(x["wv"]), da=e(x["a"]), db=e(x["b"]))
+        args_in = (x["xq"], x["xk"], x["xv"], x["wq"], x["wk"], x["wv"], x["a"], x["b"], -5.0)
+
+        def step():
+            _abi.ckda_prologue_fwd(B, T, H, dk, dv, code, *args_in, outs["q"], outs["k"], outs["v"], outs["g"],
+                                   outs["sign"], outs["beta"])
+            _abi.ckda_prologue_bwd(B, T, H, dk, dv, code, *args_in, x["dq"], x["dk"], x["dv"], x["dg"], x["dbeta"],
+                                   grads["dxq"], grads["dxk"], grads["dxv"], grads["dwq"], grads["dwk"],
+                                   grads["dwv"], grads["da"], grads["db"])
+        units, per_unit, unit_name = B * T * H, PROLOGUE_FWD_BYTES + PROLOGUE_BWD_BYTES, \
+            "B per token-head (prologue fwd + bwd)"
+        kernel_bytes = {"prologue_fwd": PROLOGUE_FWD_BYTES, "prologue_bwd": PROLOGUE_BWD_BYTES}
+        tokens = B * T
+        metric = "CKDA prologue fwd+bwd tokens/s (short conv + q/k L2 norm + signed gate + beta; B=8,T=4096,H=16,d=128,bf16)"
+        cfg = {"workload": "prologue_" + w.name, "B": B, "T": T, "H": H, "dk": dk, "dv": dv, "io_dtype": "bf16",
+               "g_floor": -5.0, "l2": "inputs larger than L2"}
     elif args.workload == "varlen":
         w = W.VARLEN
         inp = W.make_varlen(w)
@@ -410,9 +441,12 @@ def run_secondary(args, rank, world, local_rank):
     top = max(prof.items(), key=lambda kv: kv[1][1])[0]
     n, t = prof[top]
     launches_per_step = n / args.steps
+    step_bytes = per_unit * units
+    if top in kernel_bytes:  # a step of several different kernels: the top one's own bytes
+        per_unit, unit_name = kernel_bytes[top], "B per token-head (%s)" % top
+        launches_per_step = 1
     alg = per_unit * units / launches_per_step if launches_per_step >= 1 else per_unit * units
     achieved = alg / (t / n / 1e3) / 1e9
-    step_bytes = per_unit * units
     out = {"metric": metric, "value": tokens * world / (ms / 1e3), "unit": "tokens/s",
            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
@@ -579,7 +613,7 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer pass")
-    ap.add_argument("--workload", choices=["fwdbwd", "kda", "fwd", "varlen", "long", "decode", "decode_multi"], default="fwdbwd",
+    ap.add_argument("--workload", choices=["fwdbwd", "kda", "fwd", "varlen", "long", "decode", "decode_multi", "prologue"], default="fwdbwd",
                     help="fwdbwd is the headline; the others are secondary measurements")
     ap.add_argument("--batch", type=int, default=0,
                     help="override B (profiling a smaller case; not a bench line)")

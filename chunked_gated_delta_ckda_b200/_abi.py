@@ -53,6 +53,9 @@ def _load():
         lib.ckda_chunk_bwd.argtypes = [I] * 6 + [P] * 11 + [Z] + [P] * 7 + [Z, P]
         lib.ckda_decode_step.argtypes = [I] * 5 + [P] * 9
         lib.ckda_decode_multi.argtypes = [I] * 6 + [P] * 8 + [I, P, I, P, P]
+        F = ctypes.c_float
+        lib.ckda_prologue_fwd.argtypes = [I] * 6 + [P] * 8 + [F] + [P] * 7
+        lib.ckda_prologue_bwd.argtypes = [I] * 6 + [P] * 8 + [F] + [P] * 14
         lib.ckda_varlen_fwd.argtypes = [I, I, P, I, I, I, I, I] + [P] * 10 + [Z, P]
         lib.ckda_chunk_fwd_noalloc.argtypes = [I] * 6 + [P] * 11
         lib.ckda_check_device_status.argtypes = [P, P]
@@ -66,6 +69,7 @@ def _load():
         lib.ckda_profile_reset.argtypes = []
         lib.ckda_profile_reset.restype = None
         for f in ("ckda_chunk_fwd", "ckda_chunk_bwd", "ckda_decode_step", "ckda_decode_multi", "ckda_varlen_fwd",
+                  "ckda_prologue_fwd", "ckda_prologue_bwd",
                   "ckda_chunk_fwd_noalloc", "ckda_check_device_status", "ckda_version", "ckda_profile_enable",
                   "ckda_profile_collect", "ckda_profile_get"):
             getattr(lib, f).restype = I
@@ -148,6 +152,21 @@ def ckda_decode_multi(N, K, H, dk, dv, io_dtype, q, k, v, g, sign, beta, n_token
     _check(_load().ckda_decode_multi(N, K, H, dk, dv, io_dtype, _p(q), _p(k), _p(v), _p(g), _p(sign),
                                      _p(beta), _p(n_tokens), _p(slots), n_slots, _p(state),
                                      1 if write_state else 0, _p(o), _s(stream)), "ckda_decode_multi")
+
+
+def ckda_prologue_fwd(B, T, H, dk, dv, io_dtype, xq, xk, xv, wq, wk, wv, a, b, g_floor, q, k, v, g, sign, beta,
+                      stream=None):
+    _check(_load().ckda_prologue_fwd(B, T, H, dk, dv, io_dtype, _p(xq), _p(xk), _p(xv), _p(wq), _p(wk), _p(wv),
+                                     _p(a), _p(b), float(g_floor), _p(q), _p(k), _p(v), _p(g), _p(sign), _p(beta),
+                                     _s(stream)), "ckda_prologue_fwd")
+
+
+def ckda_prologue_bwd(B, T, H, dk, dv, io_dtype, xq, xk, xv, wq, wk, wv, a, b, g_floor, dq, dk_in, dv_in, dg, dbeta,
+                      dxq, dxk, dxv, dwq, dwk, dwv, da, db, stream=None):
+    _check(_load().ckda_prologue_bwd(B, T, H, dk, dv, io_dtype, _p(xq), _p(xk), _p(xv), _p(wq), _p(wk), _p(wv),
+                                     _p(a), _p(b), float(g_floor), _p(dq), _p(dk_in), _p(dv_in), _p(dg), _p(dbeta),
+                                     _p(dxq), _p(dxk), _p(dxv), _p(dwq), _p(dwk), _p(dwv), _p(da), _p(db),
+                                     _s(stream)), "ckda_prologue_bwd")
 
 
 def ckda_varlen_fwd(total_T, N, cu_seqlens, max_seqlen, H, dk, dv, io_dtype, q, k, v, g, sign,

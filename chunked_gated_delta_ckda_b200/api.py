@@ -9,6 +9,8 @@ torch (device memory is torch's job here) and call the library.
     o         = decode_multi(q, k, v, g, sign, beta, pool, slots=None, n_tokens=None,
                              write_state=True)                 # K tokens per sequence
     o, ST     = varlen_fwd(q, k, v, g, sign, beta, cu_seqlens, max_seqlen, S0=None)
+    x         = prologue_fwd(xq, xk, xv, wq, wk, wv, a, b, g_floor=-5.0)   # q, k, v, g, sign, beta
+    grads     = prologue_bwd(xq, xk, xv, wq, wk, wv, a, b, dq, dk, dv, dg, dbeta, g_floor=-5.0)
 
 Shapes and dtypes are those of include/ckda.h: q, k, g, sign [B,T,H,dk]; v
 [B,T,H,dv]; beta [B,T,H]; g fp32; sign int8 (None: every sign +1, standard
@@ -135,6 +137,36 @@ def decode_multi(q, k, v, g, sign, beta, pool, slots=None, n_tokens=None, write_
     _abi.ckda_decode_multi(N, K, H, dk, dv, io_code(q.dtype), q, k, v, g, sign, beta, n_tokens, slots,
                            pool.shape[0], pool, write_state, o)
     return o
+
+
+def prologue_fwd(xq, xk, xv, wq, wk, wv, a, b, g_floor=-5.0):
+    """Projections [B,T,H,d] (io dtype), conv taps [H*d, 4] fp32, gate
+    pre-activation a [B,T,H,dk] fp32, b [B,T,H] -> dict q, k, v, g, sign, beta
+    (the inputs of chunk_fwd)."""
+    xq, xk, xv, wq, wk, wv, a, b = map(_c, (xq, xk, xv, wq, wk, wv, a, b))
+    B, T, H, dk = xq.shape
+    dv = xv.shape[-1]
+    out = dict(q=torch.empty_like(xq), k=torch.empty_like(xk), v=torch.empty_like(xv),
+               g=torch.empty(B, T, H, dk, dtype=torch.float32, device=xq.device),
+               sign=torch.empty(B, T, H, dk, dtype=torch.int8, device=xq.device), beta=torch.empty_like(b))
+    _abi.ckda_prologue_fwd(B, T, H, dk, dv, io_code(xq.dtype), xq, xk, xv, wq, wk, wv, a, b, g_floor,
+                           out["q"], out["k"], out["v"], out["g"], out["sign"], out["beta"])
+    return out
+
+
+def prologue_bwd(xq, xk, xv, wq, wk, wv, a, b, dq, dk, dv, dg, dbeta, g_floor=-5.0):
+    """Gradients of prologue_fwd's inputs: dict dxq, dxk, dxv, dwq, dwk, dwv, da, db."""
+    xq, xk, xv, wq, wk, wv, a, b, dq, dk, dv, dg, dbeta = map(
+        _c, (xq, xk, xv, wq, wk, wv, a, b, dq, dk, dv, dg, dbeta))
+    B, T, H, dk_ = xq.shape
+    dv_ = xv.shape[-1]
+    out = dict(dxq=torch.empty_like(xq), dxk=torch.empty_like(xk), dxv=torch.empty_like(xv),
+               dwq=torch.empty_like(wq), dwk=torch.empty_like(wk), dwv=torch.empty_like(wv),
+               da=torch.empty_like(a), db=torch.empty_like(b))
+    _abi.ckda_prologue_bwd(B, T, H, dk_, dv_, io_code(xq.dtype), xq, xk, xv, wq, wk, wv, a, b, g_floor,
+                           dq, dk, dv, dg, dbeta, out["dxq"], out["dxk"], out["dxv"], out["dwq"], out["dwk"],
+                           out["dwv"], out["da"], out["db"])
+    return out
 
 
 def varlen_fwd(q, k, v, g, sign, beta, cu_seqlens, max_seqlen, S0=None, output_final_state=True,

@@ -207,4 +207,21 @@ cudaError_t decode_multi(int N, int K, int H, int dk, int dv, bool bf16, const v
                          const int32_t *n_tokens, const int32_t *slots, int n_slots, float *state,
                          bool write_state, void *o, cudaStream_t s);
 
+// token-mixer prologue (forward, or backward when `backward`)
+struct PrologueLaunch {
+  int B, T, H, dk, dv;
+  bool bf16, backward;
+  float g_floor;
+  const void *xq, *xk, *xv, *b;
+  const float *wq, *wk, *wv, *a;
+  void *q, *k, *v, *beta;
+  float *g;
+  int8_t *sign;
+  const void *dq, *dk_in, *dv_in, *dbeta;
+  const float *dg;
+  void *dxq, *dxk, *dxv, *db;
+  float *dwq, *dwk, *dwv, *da;
+};
+cudaError_t prologue(const PrologueLaunch &p, cudaStream_t s);
+
 }  // namespace ckda

@@ -201,3 +201,20 @@ def make_decode_multi(w: Workload = DECODE_MULTI, call: int = 0) -> dict:
 def make_decode_pool(w: Workload = DECODE_MULTI) -> torch.Tensor:
     """The state pool [n_slots, H, dk, dv], N(0, 0.1^2)."""
     return 0.1 * torch.randn(w.extra["n_slots"], w.H, w.dk, w.dv, generator=_gen(w.seed + 1))
+
+
+def make_prologue(w: Workload = LAYER_FWDBWD, B: Optional[int] = None) -> dict:
+    """Inputs of the token-mixer prologue at a layer's shape: projections
+    xq, xk, xv ~ N(0, 1) in the I/O dtype, conv taps ~ N(0, 0.5^2) fp32
+    [H*d, 4], gate pre-activation a ~ N(0, 1.5^2) fp32, beta pre-activation
+    b ~ N(0, 2^2); and the upstream gradients dq, dk, dv, dbeta ~ N(0, 1)
+    (I/O dtype), dg ~ N(0, 1) fp32."""
+    B = w.B if B is None else B
+    T, H, dk, dv, io = w.T, w.H, w.dk, w.dv, w.io_dtype
+    gen = _gen(w.seed * 7 + 11)
+    r = lambda *shape: torch.randn(*shape, generator=gen)
+    return dict(xq=r(B, T, H, dk).to(io), xk=r(B, T, H, dk).to(io), xv=r(B, T, H, dv).to(io),
+                wq=0.5 * r(H * dk, 4), wk=0.5 * r(H * dk, 4), wv=0.5 * r(H * dv, 4),
+                a=1.5 * r(B, T, H, dk), b=(2.0 * r(B, T, H)).to(io),
+                dq=r(B, T, H, dk).to(io), dk=r(B, T, H, dk).to(io), dv=r(B, T, H, dv).to(io),
+                dg=r(B, T, H, dk), dbeta=r(B, T, H).to(io))

@@ -180,6 +180,51 @@ int ckda_decode_multi(int N, int K, int H, int dk, int dv, int io_dtype,
                       float *state, int write_state, void *o,
                       cudaStream_t stream);
 
+/* ---- token-mixer prologue --------------------------------------------------
+ * The recurrence's inputs from the per-token projections of a layer (the
+ * model card's architecture: a short convolution of width 4 ahead of the
+ * recurrence; the paper's section 3 "CKDA": beta in [0, 2] and a signed gate
+ * in [-1, 1] carried as log-magnitude and sign).  The pages leave the gate's
+ * parameterisation, floor and backward convention to an appendix they do not
+ * contain; this library's reading:
+ *   q, k, v = SiLU(y), y[t,c] = sum_j w[c][j] x[t-3+j, c]  (causal depthwise
+ *             conv of width 4, tap 3 on the current token, zero history at
+ *             each sequence start: every batch row is its own sequence)
+ *   q, k   /= sqrt(sum over the head's dk channels of the square + 1e-6)
+ *   alpha   = tanh(a);  g = max(log|alpha|, g_floor);  sign = alpha < 0 ? -1 : +1
+ *   beta    = 2 sigmoid(b)
+ *   xq, xk [B,T,H,dk] io;  xv [B,T,H,dv] io;  wq, wk [H*dk, 4] f32;
+ *   wv [H*dv, 4] f32 (row h*d + c holds channel c of head h's four taps);
+ *   a [B,T,H,dk] f32 (gate pre-activation);  b [B,T,H] io;
+ *   g_floor: finite and <= 0 (e.g. -5), else CKDA_ERR_INVALID_ARG.
+ *   Outputs q, k [B,T,H,dk] io;  v [B,T,H,dv] io;  g [B,T,H,dk] f32;
+ *   sign [B,T,H,dk] int8;  beta [B,T,H] io: the inputs of ckda_chunk_fwd.
+ * B and H at most 65535.  No workspace. */
+int ckda_prologue_fwd(int B, int T, int H, int dk, int dv, int io_dtype,
+                      const void *xq, const void *xk, const void *xv,
+                      const float *wq, const float *wk, const float *wv,
+                      const float *a, const void *b, float g_floor, void *q,
+                      void *k, void *v, float *g, int8_t *sign, void *beta,
+                      cudaStream_t stream);
+
+/* Backward of ckda_prologue_fwd (same inputs) from the gradients of its
+ * outputs (dq, dk_in [B,T,H,dk] io;  dv_in [B,T,H,dv] io;  dg [B,T,H,dk]
+ * f32;  dbeta [B,T,H] io -- what ckda_chunk_bwd returns).  Exact gradients of
+ * the formulas above; the sign gets none; where the floor is active g gets
+ * none through a.
+ *   dxq, dxk [B,T,H,dk] io;  dxv [B,T,H,dv] io;  da [B,T,H,dk] f32;
+ *   db [B,T,H] io;  dwq, dwk [H*dk, 4] f32;  dwv [H*dv, 4] f32.
+ * dw* are overwritten: cleared on the stream, then summed over the tokens
+ * with float atomics (the order of the partial sums is not fixed). */
+int ckda_prologue_bwd(int B, int T, int H, int dk, int dv, int io_dtype,
+                      const void *xq, const void *xk, const void *xv,
+                      const float *wq, const float *wk, const float *wv,
+                      const float *a, const void *b, float g_floor,
+                      const void *dq, const void *dk_in, const void *dv_in,
+                      const float *dg, const void *dbeta, void *dxq, void *dxk,
+                      void *dxv, float *dwq, float *dwk, float *dwv, float *da,
+                      void *db, cudaStream_t stream);
+
 /* Chunked forward over N packed documents (training packs documents back to
  * back; the state restarts at each boundary).
  *   cu_seqlens [N+1] int32 DEVICE: cu[0] = 0, non-decreasing, cu[N] = total_T
