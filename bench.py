@@ -343,8 +343,8 @@ def run_secondary(args, rank, world, local_rank):
                "l2": "touched states (256 MiB) larger than L2"}
     elif args.workload == "prologue":
         w = W.LAYER_FWDBWD
-        x = {k: v.to(dev) for k, v in W.make_prologue(w).items()}
-        B, T, H, dk, dv = w.B, w.T, w.H, w.dk, w.dv
+        x = {k: v.to(dev) for k, v in W.make_prologue(w, B=args.batch or None).items()}
+        B, T, H, dk, dv = x["xq"].shape[0], w.T, w.H, w.dk, w.dv
         code = api.io_code(w.io_dtype)
         e = lambda t, dt=None: torch.empty_like(t, dtype=dt) if dt else torch.empty_like(t)
         outs = dict(q=e(x["xq"]), k=e(x["xk"]), v=e(x["xv"]), g=e(x["a"]), sign=e(x["a"], torch.int8),
