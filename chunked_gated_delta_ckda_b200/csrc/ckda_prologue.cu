@@ -46,6 +46,20 @@ struct PrologueArgs {
 // about -88, where the exponential overflows)
 __device__ __forceinline__ float sigm(float y) { return __fdividef(1.f, 1.f + __expf(-y)); }
 
+// tanh from the fast exponential, written from the identities
+//   tanh|x| = (1 - e) / (1 + e),  e = exp(-2|x|)          (|x| >= 0.05)
+//   tanh x  = x - x^3/3 + 2 x^5/15 - ...  (Taylor series)  (|x| <  0.05, where
+//             1 - e would cancel; the first omitted term, 17 x^7/315, is
+//             below 1e-9 of the value there)
+// both evaluated (no divergence), the sign restored at the end
+__device__ __forceinline__ float tanh_fast(float x) {
+  const float t = fabsf(x), t2 = t * t;
+  const float e = __expf(-2.f * t);
+  const float big = __fdividef(1.f - e, 1.f + e);
+  const float small = t * (1.f - t2 * (1.f / 3.f) + t2 * t2 * (2.f / 15.f));
+  return copysignf(t < 0.05f ? small : big, x);
+}
+
 // Sums of 16 values over the CTA's 128 threads; every thread gets all 16
 // totals.  In the warp, a halving exchange (8 + 4 + 2 + 1 + 1 shuffles)
 // leaves lane pair (2m, 2m + 1) with the warp total of value
@@ -80,13 +94,14 @@ __device__ __forceinline__ void block_sum16(float (&x)[16], float (*red)[kPrThre
 
 // Forward: 8 tokens per reduction (q and k sums of squares).
 constexpr int kFwdG = 8;
-template <typename IO>
-__global__ void __launch_bounds__(kPrThreads) prologue_fwd_kernel(const PrologueArgs a) {
+template <typename IO, int DK, int DV>
+__global__ void __launch_bounds__(kPrThreads, 6) prologue_fwd_kernel(const PrologueArgs a) {
   __shared__ __align__(16) float red[2][kPrThreads / 32][16];
   const int c = threadIdx.x, h = blockIdx.y, sq = blockIdx.z;
-  const int T = a.T, H = a.H, dk = a.dk, dv = a.dv;
+  const int T = a.T, H = a.H;
+  constexpr int dk = DK, dv = DV;
   const int t0 = blockIdx.x * kPrTok, t1 = min(t0 + kPrTok, T);
-  const bool kc = c < dk, vc = c < dv;
+  const bool kc = DK == kPrThreads || c < DK, vc = DV == kPrThreads || c < DV;  // (compile-time true at 128)
   const IO *xq = (const IO *)a.xq, *xk = (const IO *)a.xk, *xv = (const IO *)a.xv;
   float wq[4], wk[4], wv[4];
 #pragma unroll
@@ -139,7 +154,7 @@ __global__ void __launch_bounds__(kPrThreads) prologue_fwd_kernel(const Prologue
       s[2 * i + 1] = nk[i] * nk[i];
       if (live && vc) st_io((IO *)a.v, row * dv + c, yv * sigm(yv));
       if (live && kc) {
-        const float al = tanhf(la[i]);
+        const float al = tanh_fast(la[i]);
         a.g[row * dk + c] = fmaxf(__logf(fabsf(al)), a.g_floor);
         a.sign[row * dk + c] = al < 0.f ? -1 : 1;
       }
@@ -164,14 +179,15 @@ __global__ void __launch_bounds__(kPrThreads) prologue_fwd_kernel(const Prologue
 // Backward: 4 tokens per reduction (|n|^2 and n . dn for q and k); the run's
 // tokens plus a three-token halo (dx of token s needs dy of s .. s + 3).
 constexpr int kBwdG = 4;
-template <typename IO>
-__global__ void __launch_bounds__(kPrThreads) prologue_bwd_kernel(const PrologueArgs a) {
+template <typename IO, int DK, int DV>
+__global__ void __launch_bounds__(kPrThreads, 4) prologue_bwd_kernel(const PrologueArgs a) {
   __shared__ __align__(16) float red[2][kPrThreads / 32][16];
   const int c = threadIdx.x, h = blockIdx.y, sq = blockIdx.z;
-  const int T = a.T, H = a.H, dk = a.dk, dv = a.dv;
+  const int T = a.T, H = a.H;
+  constexpr int dk = DK, dv = DV;
   const int t0 = blockIdx.x * kPrTok, t1 = min(t0 + kPrTok, T);
   const int tend = min(t0 + kPrTok + 3, T);
-  const bool kc = c < dk, vc = c < dv;
+  const bool kc = DK == kPrThreads || c < DK, vc = DV == kPrThreads || c < DV;  // (compile-time true at 128)
   const IO *xq = (const IO *)a.xq, *xk = (const IO *)a.xk, *xv = (const IO *)a.xv;
   const IO *gq = (const IO *)a.dq, *gk = (const IO *)a.dk_in, *gv = (const IO *)a.dv_in;
   float wq[4], wk[4], wv[4];
@@ -237,7 +253,7 @@ __global__ void __launch_bounds__(kPrThreads) prologue_bwd_kernel(const Prologue
       s[4 * i + 2] = nq * dqt[i];
       s[4 * i + 3] = nk * dkt[i];
       if (live && t < t1 && kc) {  // gate: the floor's clamp passes no gradient
-        const float al = tanhf(la[i]);
+        const float al = tanh_fast(la[i]);
         const bool open = __logf(fabsf(al)) > a.g_floor;
         a.da[row * dk + c] = open ? __fdividef(lg[i] * (1.f - al * al), al) : 0.f;
       }
@@ -309,15 +325,23 @@ cudaError_t prologue(const PrologueLaunch &p, cudaStream_t s) {
   a.dwq = p.dwq; a.dwk = p.dwk; a.dwv = p.dwv; a.da = p.da;
   if ((size_t)p.B * p.T * p.H == 0) return cudaSuccess;
   const dim3 grid((p.T + kPrTok - 1) / kPrTok, p.H, p.B);
-  if (p.backward) {
-    ProfScope prof("prologue_bwd", s);
-    if (p.bf16) prologue_bwd_kernel<__nv_bfloat16><<<grid, kPrThreads, 0, s>>>(a);
-    else prologue_bwd_kernel<float><<<grid, kPrThreads, 0, s>>>(a);
-    return cudaGetLastError();
-  }
-  ProfScope prof("prologue_fwd", s);
-  if (p.bf16) prologue_fwd_kernel<__nv_bfloat16><<<grid, kPrThreads, 0, s>>>(a);
-  else prologue_fwd_kernel<float><<<grid, kPrThreads, 0, s>>>(a);
+  ProfScope prof(p.backward ? "prologue_bwd" : "prologue_fwd", s);
+#define CKDA_PRO_LAUNCH(IO, K, V)                                                   \
+  do {                                                                              \
+    if (p.backward) prologue_bwd_kernel<IO, K, V><<<grid, kPrThreads, 0, s>>>(a);  \
+    else prologue_fwd_kernel<IO, K, V><<<grid, kPrThreads, 0, s>>>(a);             \
+  } while (0)
+#define CKDA_PRO_DIMS(IO)                                   \
+  do {                                                      \
+    if (p.dk == 128 && p.dv == 128) CKDA_PRO_LAUNCH(IO, 128, 128); \
+    else if (p.dk == 128) CKDA_PRO_LAUNCH(IO, 128, 64);    \
+    else if (p.dv == 128) CKDA_PRO_LAUNCH(IO, 64, 128);    \
+    else CKDA_PRO_LAUNCH(IO, 64, 64);                      \
+  } while (0)
+  if (p.bf16) CKDA_PRO_DIMS(__nv_bfloat16);
+  else CKDA_PRO_DIMS(float);
+#undef CKDA_PRO_DIMS
+#undef CKDA_PRO_LAUNCH
   return cudaGetLastError();
 }
 
