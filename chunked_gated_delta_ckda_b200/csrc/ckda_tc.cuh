@@ -498,7 +498,9 @@ __device__ __forceinline__ void st_bf16x4(unsigned char *base, uint32_t off, flo
 // M = (I + N)^{-1} for strictly lower N (fp32, row stride LDF), 64 x 64, by
 // 16 x 16 blocks, 256 threads: diagonal blocks by forward substitution (one
 // column per thread), then the block diagonals d = 1, 2, 3:
-//   M_IJ = -M_II sum_{K=J}^{I-1} N_IK M_KJ.
+//   M_IJ = -M_II sum_{K=J}^{I-1} N_IK M_KJ,
+// two passes per diagonal (the inner sum into Xs, then the product with
+// M_II), each output block in 2 x 2 register tiles.
 // Every entry on or below the diagonal is written; the strictly upper 16x16
 // blocks are zeroed (the diagonal blocks carry their own zeros).
 // ---------------------------------------------------------------------------
@@ -527,28 +529,38 @@ __device__ __forceinline__ void inverse64(float *Mf, const float *Nf, float (*Xs
     }
   }
   __syncthreads();
+  // each thread a 2 x 2 block of outputs (rows aa, aa + 1, columns bb, bb + 1):
+  // two loads of N and two of M feed four products
 #pragma unroll 1
   for (int d = 1; d < 4; ++d) {
     const int nb = 4 - d;
-    for (int e = tid; e < nb * 256; e += 256) {
-      const int J = e >> 8, I = J + d, aa = (e >> 4) & 15, bb = e & 15;
-      float s = 0.f;
+    for (int e = tid; e < nb * 64; e += 256) {
+      const int J = e >> 6, I = J + d, aa = ((e >> 3) & 7) * 2, bb = (e & 7) * 2;
+      float s00 = 0.f, s01 = 0.f, s10 = 0.f, s11 = 0.f;
       for (int K = J; K < I; ++K) {
-        const float *nrow = Nf + (16 * I + aa) * kLdf + 16 * K;
-        const float *mcol = Mf + (16 * K) * kLdf + 16 * J + bb;
+        const float *n0 = Nf + (16 * I + aa) * kLdf + 16 * K, *n1 = n0 + kLdf;
+        const float *mc = Mf + (16 * K) * kLdf + 16 * J + bb;
 #pragma unroll
-        for (int t = 0; t < 16; ++t) s += nrow[t] * mcol[t * kLdf];
+        for (int t = 0; t < 16; ++t) {
+          const float a0 = n0[t], a1 = n1[t], b0 = mc[t * kLdf], b1 = mc[t * kLdf + 1];
+          s00 += a0 * b0; s01 += a0 * b1; s10 += a1 * b0; s11 += a1 * b1;
+        }
       }
-      Xs[J][aa][bb] = s;
+      Xs[J][aa][bb] = s00; Xs[J][aa][bb + 1] = s01;
+      Xs[J][aa + 1][bb] = s10; Xs[J][aa + 1][bb + 1] = s11;
     }
     __syncthreads();
-    for (int e = tid; e < nb * 256; e += 256) {
-      const int J = e >> 8, I = J + d, aa = (e >> 4) & 15, bb = e & 15;
-      const float *mrow = Mf + (16 * I + aa) * kLdf + 16 * I;
-      float s = 0.f;
+    for (int e = tid; e < nb * 64; e += 256) {
+      const int J = e >> 6, I = J + d, aa = ((e >> 3) & 7) * 2, bb = (e & 7) * 2;
+      const float *m0 = Mf + (16 * I + aa) * kLdf + 16 * I, *m1 = m0 + kLdf;
+      float s00 = 0.f, s01 = 0.f, s10 = 0.f, s11 = 0.f;
 #pragma unroll
-      for (int t = 0; t < 16; ++t) s += mrow[t] * Xs[J][t][bb];
-      Mf[(16 * I + aa) * kLdf + 16 * J + bb] = -s;
+      for (int t = 0; t < 16; ++t) {
+        const float a0 = m0[t], a1 = m1[t], b0 = Xs[J][t][bb], b1 = Xs[J][t][bb + 1];
+        s00 += a0 * b0; s01 += a0 * b1; s10 += a1 * b0; s11 += a1 * b1;
+      }
+      float *o0 = Mf + (16 * I + aa) * kLdf + 16 * J + bb, *o1 = o0 + kLdf;
+      o0[0] = -s00; o0[1] = -s01; o1[0] = -s10; o1[1] = -s11;
     }
     __syncthreads();
   }
