@@ -71,7 +71,7 @@ KERNEL_UNITS = {
 # captured on a B=2 launch (inputs still larger than L2), traffic being
 # proportional to the chunk-heads a launch processes (profiles/).
 NCU_TRAFFIC = {
-    ("tc_grad", "layer_fwdbwd_bf16"): (454207744 + 148805888) / (2 * 64 * 16),
+    ("tc_grad", "layer_fwdbwd_bf16"): (454119168 + 152589312) / (2 * 64 * 16),
 }
 
 
