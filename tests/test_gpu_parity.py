@@ -560,3 +560,54 @@ def test_prologue_feeds_the_recurrence():
     o_ref, ST_ref, _ = oracle_fwd_batched(cpu)
     check("o", o, o_ref, io)
     check("ST", ST, ST_ref, io)
+
+
+def test_full_decode_multi_sampled():
+    """The benchmark's multi-token decode (256 sequences x 4 tokens, H=16,
+    d=128, 512-slot pool) in its launch configuration, checked on sampled
+    sequences (all heads) and on the slots nothing touched."""
+    w = W.DECODE_MULTI
+    x = W.make_decode_multi(w, call=0)
+    pool = W.make_decode_pool(w)
+    dpool = pool.cuda()
+    d = to_dev(x)
+    o = api.decode_multi(d["q"], d["k"], d["v"], d["g"], d["sign"], d["beta"], dpool, slots=d["slots"])
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(4)
+    seqs = sorted(rng.choice(w.B, 3, replace=False).tolist())
+    sub = lambda t: t[seqs]
+    slots = x["slots"][seqs].numpy()
+    ref_o, ref_pool = oracle.decode_multi(f64(sub(x["q"])), f64(sub(x["k"])), f64(sub(x["v"])), f64(sub(x["g"])),
+                                          sub(x["sign"]).numpy(), f64(sub(x["beta"])), f64(pool), slots=slots)
+    check("o (sampled sequences)", o[seqs], ref_o, w.io_dtype)
+    check("pool (their slots)", dpool[torch.from_numpy(slots).long().cuda()], ref_pool[slots], w.io_dtype)
+    live = set(x["slots"].tolist())
+    idle = [s for s in range(pool.shape[0]) if s not in live][:8]
+    assert torch.equal(dpool[idle].cpu(), pool[idle])
+
+
+def test_full_prologue_sampled_heads():
+    """The benchmark's prologue (B=8, T=4096, H=16, d=128, bf16) forward and
+    backward, checked on sampled heads over the whole batch (the conv taps'
+    gradients sum over every token of a head)."""
+    w = W.LAYER_FWDBWD
+    x = W.make_prologue(w)
+    d = to_dev(x)
+    names = ("xq", "xk", "xv", "wq", "wk", "wv", "a", "b")
+    p = api.prologue_fwd(*(d[n] for n in names), g_floor=-5.0)
+    gr = api.prologue_bwd(*(d[n] for n in names), d["dq"], d["dk"], d["dv"], d["dg"], d["dbeta"], g_floor=-5.0)
+    torch.cuda.synchronize()
+    for h in (3, 11):
+        hs = slice(h, h + 1)
+        X = {n: f64(x[n][:, :, hs]) for n in ("xq", "xk", "xv", "a", "b")}
+        X.update({n: f64(x[n][h * 128:(h + 1) * 128]) for n in ("wq", "wk", "wv")})
+        up = {n: f64(x[n][:, :, hs]) for n in ("dq", "dk", "dv", "dg", "dbeta")}
+        ref = oracle.prologue_fwd(**X, g_floor=-5.0)
+        for n in ("q", "k", "v", "g", "beta"):
+            check("%s[h=%d]" % (n, h), p[n][:, :, hs], ref[n], w.io_dtype)
+        assert torch.equal(p["sign"][:, :, hs].cpu(), torch.from_numpy(ref["sign"]))
+        rg = oracle.prologue_bwd(**X, **up, g_floor=-5.0)
+        for n in ("dxq", "dxk", "dxv", "da", "db"):
+            check("%s[h=%d]" % (n, h), gr[n][:, :, hs], rg[n], w.io_dtype)
+        for n in ("dwq", "dwk", "dwv"):
+            check("%s[h=%d]" % (n, h), gr[n][h * 128:(h + 1) * 128], rg[n], w.io_dtype)
