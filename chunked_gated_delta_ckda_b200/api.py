@@ -61,6 +61,40 @@ def _c(x: Optional[torch.Tensor]) -> Optional[torch.Tensor]:
     return x if x.is_contiguous() else x.contiguous()
 
 
+def _expect(name, t, shape, dtype=None, optional=False):
+    """Shape (and dtype) check of one argument: the library reads exactly the
+    bytes the sizes imply, so a mismatch must stop here."""
+    if t is None:
+        if optional:
+            return
+        raise ValueError("%s is required" % name)
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError("%s must have shape %s, got %s" % (name, tuple(shape), tuple(t.shape)))
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError("%s must be %s, got %s" % (name, dtype, t.dtype))
+
+
+def _expect_io(io_dtype, **named):
+    for name, t in named.items():
+        if t is not None and t.dtype != io_dtype:
+            raise TypeError("%s must be %s like q, got %s" % (name, io_dtype, t.dtype))
+
+
+def _recurrence_inputs(q, k, v, g, sign, beta, lead):
+    """q, k, g, sign [*lead, H, dk]; v [*lead, H, dv]; beta [*lead, H]."""
+    if q.dim() != len(lead) + 2:
+        raise ValueError("q must have shape %s + (H, dk), got %s" % (tuple(lead), tuple(q.shape)))
+    H, dk = q.shape[-2], q.shape[-1]
+    dv = v.shape[-1]
+    io_code(q.dtype)
+    _expect("k", k, (*lead, H, dk), q.dtype)
+    _expect("v", v, (*lead, H, dv), q.dtype)
+    _expect("g", g, (*lead, H, dk), torch.float32)
+    _expect("sign", sign, (*lead, H, dk), torch.int8, optional=True)
+    _expect("beta", beta, (*lead, H), q.dtype)
+    return H, dk, dv
+
+
 def saved_buffer(B, T, H, dk, dv, dtype, device) -> Optional[torch.Tensor]:
     """The forward-to-backward saved buffer (None: this configuration recomputes)."""
     n = _abi.ckda_saved_size(B, T, H, dk, dv, io_code(dtype))
@@ -69,9 +103,10 @@ def saved_buffer(B, T, H, dk, dv, dtype, device) -> Optional[torch.Tensor]:
 
 def chunk_fwd(q, k, v, g, sign, beta, S0=None, output_final_state=True, save_chunk_states=False,
               ws=None, save_for_backward=False):
+    B, T = q.shape[:2]
+    H, dk, dv = _recurrence_inputs(q, k, v, g, sign, beta, (B, T))
+    _expect("S0", S0, (B, H, dk, dv), torch.float32, optional=True)
     q, k, v, g, sign, beta, S0 = map(_c, (q, k, v, g, sign, beta, S0))
-    B, T, H, dk = q.shape
-    dv = v.shape[-1]
     io = io_code(q.dtype)
     o = torch.empty(B, T, H, dv, dtype=q.dtype, device=q.device)
     ST = torch.empty(B, H, dk, dv, dtype=torch.float32, device=q.device) if output_final_state else None
@@ -89,10 +124,16 @@ def chunk_fwd(q, k, v, g, sign, beta, S0=None, output_final_state=True, save_chu
 
 def chunk_bwd(q, k, v, g, sign, beta, dO, S0=None, dST=None, chunk_states=None, need_dS0=True,
               ws=None, saved=None):
-    q, k, v, g, sign, beta, dO, S0, dST, chunk_states = map(
-        _c, (q, k, v, g, sign, beta, dO, S0, dST, chunk_states))
-    B, T, H, dk = q.shape
-    dv = v.shape[-1]
+    B, T = q.shape[:2]
+    H, dk, dv = _recurrence_inputs(q, k, v, g, sign, beta, (B, T))
+    _expect("dO", dO, (B, T, H, dv), q.dtype)
+    _expect("S0", S0, (B, H, dk, dv), torch.float32, optional=True)
+    _expect("dST", dST, (B, H, dk, dv), torch.float32, optional=True)
+    _expect("chunk_states", chunk_states, (B, H, (T + 63) // 64, dk, dv), torch.float32, optional=True)
+    if saved is not None and saved.dtype != torch.uint8:
+        raise TypeError("saved must be the uint8 buffer chunk_fwd returned")
+    q, k, v, g, sign, beta, dO, S0, dST, chunk_states, saved = map(
+        _c, (q, k, v, g, sign, beta, dO, S0, dST, chunk_states, saved))
     io = io_code(q.dtype)
     dq = torch.empty_like(q)
     dk_ = torch.empty_like(k)
@@ -108,11 +149,13 @@ def chunk_bwd(q, k, v, g, sign, beta, dO, S0=None, dST=None, chunk_states=None, 
 
 
 def decode_step(q, k, v, g, sign, beta, state, o=None):
-    q, k, v, g, sign, beta = map(_c, (q, k, v, g, sign, beta))
-    if not state.is_contiguous() or state.dtype != torch.float32:
-        raise ValueError("state must be a contiguous float32 tensor (updated in place)")
-    N, H, dk = q.shape
-    dv = v.shape[-1]
+    N = q.shape[0]
+    H, dk, dv = _recurrence_inputs(q, k, v, g, sign, beta, (N,))
+    _expect("state", state, (N, H, dk, dv), torch.float32)
+    _expect("o", o, (N, H, dv), q.dtype, optional=True)
+    q, k, v, g, sign, beta, o = map(_c, (q, k, v, g, sign, beta, o))
+    if not state.is_cuda or not state.is_contiguous():
+        raise ValueError("state must be a contiguous CUDA tensor (updated in place)")
     if o is None:
         o = torch.empty(N, H, dv, dtype=q.dtype, device=q.device)
     _abi.ckda_decode_step(N, H, dk, dv, io_code(q.dtype), q, k, v, g, sign, beta, state, o)
@@ -124,14 +167,17 @@ def decode_multi(q, k, v, g, sign, beta, pool, slots=None, n_tokens=None, write_
     """K steps per sequence: q, k, g, sign [N,K,H,dk]; v [N,K,H,dv]; beta [N,K,H];
     pool [n_slots,H,dk,dv] fp32 (updated in place when write_state);
     slots / n_tokens: int32 [N] on the device, or None (slot n / all K)."""
-    q, k, v, g, sign, beta, slots, n_tokens = map(_c, (q, k, v, g, sign, beta, slots, n_tokens))
-    if not pool.is_contiguous() or pool.dtype != torch.float32:
-        raise ValueError("pool must be a contiguous float32 tensor")
-    for t in (slots, n_tokens):
-        if t is not None and t.dtype != torch.int32:
-            raise TypeError("slots and n_tokens must be int32")
-    N, K, H, dk = q.shape
-    dv = v.shape[-1]
+    N, K = q.shape[:2]
+    H, dk, dv = _recurrence_inputs(q, k, v, g, sign, beta, (N, K))
+    if pool.dim() != 4:
+        raise ValueError("pool must have shape (n_slots, H, dk, dv), got %s" % (tuple(pool.shape),))
+    _expect("pool", pool, (pool.shape[0], H, dk, dv), torch.float32)
+    _expect("slots", slots, (N,), torch.int32, optional=True)
+    _expect("n_tokens", n_tokens, (N,), torch.int32, optional=True)
+    _expect("o", o, (N, K, H, dv), q.dtype, optional=True)
+    q, k, v, g, sign, beta, slots, n_tokens, o = map(_c, (q, k, v, g, sign, beta, slots, n_tokens, o))
+    if not pool.is_cuda or not pool.is_contiguous():
+        raise ValueError("pool must be a contiguous CUDA tensor (updated in place)")
     if o is None and want_o:
         o = torch.empty(N, K, H, dv, dtype=q.dtype, device=q.device)
     _abi.ckda_decode_multi(N, K, H, dk, dv, io_code(q.dtype), q, k, v, g, sign, beta, n_tokens, slots,
@@ -139,13 +185,28 @@ def decode_multi(q, k, v, g, sign, beta, pool, slots=None, n_tokens=None, write_
     return o
 
 
+def _prologue_shapes(xq, xk, xv, wq, wk, wv, a, b):
+    if xq.dim() != 4:
+        raise ValueError("xq must have shape (B, T, H, dk), got %s" % (tuple(xq.shape),))
+    B, T, H, dk = xq.shape
+    dv = xv.shape[-1]
+    io_code(xq.dtype)
+    _expect("xk", xk, (B, T, H, dk), xq.dtype)
+    _expect("xv", xv, (B, T, H, dv), xq.dtype)
+    _expect("wq", wq, (H * dk, 4), torch.float32)
+    _expect("wk", wk, (H * dk, 4), torch.float32)
+    _expect("wv", wv, (H * dv, 4), torch.float32)
+    _expect("a", a, (B, T, H, dk), torch.float32)
+    _expect("b", b, (B, T, H), xq.dtype)
+    return B, T, H, dk, dv
+
+
 def prologue_fwd(xq, xk, xv, wq, wk, wv, a, b, g_floor=-5.0):
     """Projections [B,T,H,d] (io dtype), conv taps [H*d, 4] fp32, gate
     pre-activation a [B,T,H,dk] fp32, b [B,T,H] -> dict q, k, v, g, sign, beta
     (the inputs of chunk_fwd)."""
+    B, T, H, dk, dv = _prologue_shapes(xq, xk, xv, wq, wk, wv, a, b)
     xq, xk, xv, wq, wk, wv, a, b = map(_c, (xq, xk, xv, wq, wk, wv, a, b))
-    B, T, H, dk = xq.shape
-    dv = xv.shape[-1]
     out = dict(q=torch.empty_like(xq), k=torch.empty_like(xk), v=torch.empty_like(xv),
                g=torch.empty(B, T, H, dk, dtype=torch.float32, device=xq.device),
                sign=torch.empty(B, T, H, dk, dtype=torch.int8, device=xq.device), beta=torch.empty_like(b))
@@ -156,10 +217,14 @@ def prologue_fwd(xq, xk, xv, wq, wk, wv, a, b, g_floor=-5.0):
 
 def prologue_bwd(xq, xk, xv, wq, wk, wv, a, b, dq, dk, dv, dg, dbeta, g_floor=-5.0):
     """Gradients of prologue_fwd's inputs: dict dxq, dxk, dxv, dwq, dwk, dwv, da, db."""
+    B, T, H, dk_, dv_ = _prologue_shapes(xq, xk, xv, wq, wk, wv, a, b)
+    _expect("dq", dq, (B, T, H, dk_), xq.dtype)
+    _expect("dk", dk, (B, T, H, dk_), xq.dtype)
+    _expect("dv", dv, (B, T, H, dv_), xq.dtype)
+    _expect("dg", dg, (B, T, H, dk_), torch.float32)
+    _expect("dbeta", dbeta, (B, T, H), xq.dtype)
     xq, xk, xv, wq, wk, wv, a, b, dq, dk, dv, dg, dbeta = map(
         _c, (xq, xk, xv, wq, wk, wv, a, b, dq, dk, dv, dg, dbeta))
-    B, T, H, dk_ = xq.shape
-    dv_ = xv.shape[-1]
     out = dict(dxq=torch.empty_like(xq), dxk=torch.empty_like(xk), dxv=torch.empty_like(xv),
                dwq=torch.empty_like(wq), dwk=torch.empty_like(wk), dwv=torch.empty_like(wv),
                da=torch.empty_like(a), db=torch.empty_like(b))
@@ -171,12 +236,15 @@ def prologue_bwd(xq, xk, xv, wq, wk, wv, a, b, dq, dk, dv, dg, dbeta, g_floor=-5
 
 def varlen_fwd(q, k, v, g, sign, beta, cu_seqlens, max_seqlen, S0=None, output_final_state=True,
                ws=None):
-    q, k, v, g, sign, beta, S0, cu_seqlens = map(_c, (q, k, v, g, sign, beta, S0, cu_seqlens))
-    if cu_seqlens.dtype != torch.int32:
-        raise TypeError("cu_seqlens must be int32")
-    _, T, H, dk = q.shape
-    dv = v.shape[-1]
+    if q.dim() != 4 or q.shape[0] != 1:
+        raise ValueError("packed q must have shape (1, total_T, H, dk), got %s" % (tuple(q.shape),))
+    T = q.shape[1]
+    H, dk, dv = _recurrence_inputs(q, k, v, g, sign, beta, (1, T))
+    if cu_seqlens.dim() != 1 or cu_seqlens.dtype != torch.int32:
+        raise TypeError("cu_seqlens must be a 1-D int32 tensor")
     N = cu_seqlens.numel() - 1
+    _expect("S0", S0, (N, H, dk, dv), torch.float32, optional=True)
+    q, k, v, g, sign, beta, S0, cu_seqlens = map(_c, (q, k, v, g, sign, beta, S0, cu_seqlens))
     o = torch.empty(1, T, H, dv, dtype=q.dtype, device=q.device)
     ST = torch.empty(N, H, dk, dv, dtype=torch.float32, device=q.device) if output_final_state else None
     if ws is None:
