@@ -556,6 +556,50 @@ def oracle_fwdbwd_sample(inp, pairs, nthreads):
     return time.perf_counter() - t0
 
 
+def oracle_fwd_sample(inp, pairs, nthreads):
+    """Oracle forward over the sampled (batch, head) sequences."""
+    import numpy as np
+    import oracle
+    T = inp["q"].shape[1]
+    P = lambda x, b, h: x[b, :, h:h + 1].to(torch.float64).numpy()
+    cat = lambda key: np.concatenate([P(inp[key], b, h) for b, h in pairs], axis=0)
+    sg = np.concatenate([inp["sign"][b, :, h:h + 1].numpy() for b, h in pairs], axis=0)
+    cu = np.arange(len(pairs) + 1, dtype=np.int64) * T
+    q, k, v, g, beta = (cat(x) for x in ("q", "k", "v", "g", "beta"))
+    t0 = time.perf_counter()
+    oracle.fwd(cu, q, k, v, g, sg, beta, nthreads=nthreads)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline_secondary(workload):
+    """The oracle on the host cores for the forward and decode workloads
+    (bounded samples, the same seeded inputs)."""
+    import oracle
+    cores = oracle.default_threads()
+    if workload == "fwd":
+        w = W.LAYER_FWD
+        inp = W.make(w)
+        n_pairs = max(8, min(128, 16 * cores))
+        pairs = [(i % w.B, (i * 7) % w.H) for i in range(n_pairs)]
+        threads = min(cores, n_pairs)
+        dt = oracle_fwd_sample(inp, pairs, threads)
+        return {"value": n_pairs * w.T / w.H / dt, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                "sample": "%d of %d (batch, head) sequences of %d tokens, forward, fp64, %d threads, %.1f s"
+                          % (n_pairs, w.B * w.H, w.T, threads, dt)}
+    w = W.DECODE  # decode: consecutive steps of every (sequence, head) state
+    x = W.make_decode_step(w, 0)
+    st = W.make_decode_state(w).to(torch.float64).numpy()
+    f = lambda t: t.to(torch.float64).numpy()
+    args = (f(x["q"]), f(x["k"]), f(x["v"]), f(x["g"]), x["sign"].numpy(), f(x["beta"]))
+    steps, t0 = 0, time.perf_counter()
+    while steps < 2 or (time.perf_counter() - t0 < 5.0 and steps < 64):
+        _, st = oracle.decode(*args, st, nthreads=cores)
+        steps += 1
+    dt = time.perf_counter() - t0
+    return {"value": steps * w.B / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": "%d steps of all %d x %d states, fp64, %d threads, %.1f s" % (steps, w.B, w.H, cores, dt)}
+
+
 def cpu_baseline(inp, H, n_pairs=None):
     import oracle
     cores = oracle.default_threads()
@@ -641,6 +685,8 @@ def main(argv=None):
         if args.workload not in ("fwdbwd", "kda"):
             out = run_secondary(args, rank, world, local_rank)
             if rank == 0:
+                if world == 1 and not args.no_cpu_baseline and args.workload in ("fwd", "decode"):
+                    out["cpu_baseline"] = cpu_baseline_secondary(args.workload)
                 print(json.dumps(out), flush=True)
             return 0
         out, inp = run_ours(args, rank, world, local_rank)
