@@ -52,8 +52,8 @@ def test_conv_restarts_at_each_sequence():
     x = _inputs(2, 9, 1, 4, 4)
     r = oracle.prologue_fwd(**x)
     solo = oracle.prologue_fwd(**{k: (v[1:2] if v.ndim >= 3 else v) for k, v in x.items()})
-    for name in ("q", "k", "v"):
-        np.testing.assert_array_equal(r[name][1:2], solo[name])
+    for name in ("q", "k", "v"):  # (reductions may be ordered differently for another batch size)
+        np.testing.assert_allclose(r[name][1:2], solo[name], rtol=1e-14, atol=1e-15)
 
 
 def test_single_tap_reduces_to_pointwise():
