@@ -2,7 +2,7 @@
 """Benchmark of the CKDA recurrence library on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload fwdbwd|kda|fwd|varlen|long|decode|decode_multi|prologue]
+                    [--workload fwdbwd|kda|fwd|varlen|long|long_fwdbwd|decode|decode_multi|prologue]
 
 Default workload (the headline): one step = ckda_chunk_fwd (saving its
 per-chunk results for the backward) + ckda_chunk_bwd on B=8, H=16, T=4096,
@@ -36,6 +36,7 @@ from chunked_gated_delta_ckda_b200 import workloads as W  # noqa: E402
 
 METRIC = "CKDA fwd+bwd tokens/s (H=16,d=128,T=4096,bf16); % tensor/HBM roofline"
 METRIC_KDA = "KDA (gate sign +1) fwd+bwd tokens/s (H=16,d=128,T=4096,bf16), same kernels"
+METRIC_LONG = "CKDA long-sequence fwd+bwd tokens/s (B=1,T=65536,H=16,d=128,bf16, with S0)"
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 
@@ -192,11 +193,13 @@ def _fwdbwd_setup(inp, dev, kda=False):
     sv = api.saved_buffer(B, T, H, dk, dv, io, dev)
     cs = None if sv is not None else buf["cs"]
 
+    S0 = d.get("S0")  # (the long-sequence workload starts from a state)
+
     def step():
         _abi.ckda_chunk_fwd(B, T, H, dk, dv, code, d["q"], d["k"], d["v"], d["g"], d["sign"],
-                            d["beta"], None, buf["o"], buf["ST"], cs, wsf, saved=sv)
+                            d["beta"], S0, buf["o"], buf["ST"], cs, wsf, saved=sv)
         _abi.ckda_chunk_bwd(B, T, H, dk, dv, code, d["q"], d["k"], d["v"], d["g"], d["sign"],
-                            d["beta"], None, d["dO"], None, cs, buf["dq"], buf["dk"],
+                            d["beta"], S0, d["dO"], None, cs, buf["dq"], buf["dk"],
                             buf["dv"], buf["dg"], buf["dbeta"], buf["dS0"], wsb, saved=sv)
     return d, buf, step
 
@@ -226,7 +229,9 @@ def run_ours(args, rank, world, local_rank):
     from chunked_gated_delta_ckda_b200 import _abi
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    wl = W.LAYER_FWDBWD
+    long_seq = args.workload == "long_fwdbwd"
+    wl = W.Workload(**{**W.LONG.__dict__, "name": "long_fwdbwd_bf16", "with_dO": True}) if long_seq \
+        else W.LAYER_FWDBWD
     w = W.Workload(**{**wl.__dict__, "seed": rank_seed(wl.seed, rank),
                       "B": args.batch or wl.B})
     inp = W.make(w)
@@ -274,9 +279,10 @@ def run_ours(args, rank, world, local_rank):
                  "tensor_frac": t_tc / ms_max, "binding_frac": max(t_hbm, t_tc) / ms_max}
 
     # end to end through the public API with host buffers
-    e2e = None if (args.no_e2e or kda) else run_e2e(inp, dev, args, world)
+    e2e = None if (args.no_e2e or kda or long_seq) else run_e2e(inp, dev, args, world)
 
-    out = {"metric": METRIC_KDA if kda else METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+    metric = METRIC_KDA if kda else (METRIC_LONG if long_seq else METRIC)
+    out = {"metric": metric, "value": value, "unit": "tokens/s", "n_gpus": world,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
            "dtype": "bf16", "data": "synthetic",
@@ -285,7 +291,8 @@ def run_ours(args, rank, world, local_rank):
                       "contraction": "bf16 tensor-core operands, f32 accumulate",
                       "step": "ckda_chunk_fwd(saved buffer for the backward) + ckda_chunk_bwd(saved)",
                       "global_batch": B * world, "seq_len": T, "parallelism": "dp%d" % world,
-                      "l2": "inputs larger than L2 (about 2 GB streamed per step)",
+                      "l2": "inputs larger than L2 (about %.1f GB streamed per step)"
+                            % ((FWD_BYTES + BWD_BYTES) * B * T * H / 1e9),
                       "gate_sign": "none: every sign +1 (standard KDA)" if kda else "int8 +-1 (CKDA)"},
            "roofline": roof, "step_roofline": step_roof, "kernels": kernels,
            "gpu_launches": int(sum(n for n, _ in prof.values())), "clocks": clk, "e2e": e2e}
@@ -657,7 +664,7 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer pass")
-    ap.add_argument("--workload", choices=["fwdbwd", "kda", "fwd", "varlen", "long", "decode", "decode_multi", "prologue"], default="fwdbwd",
+    ap.add_argument("--workload", choices=["fwdbwd", "kda", "fwd", "varlen", "long", "long_fwdbwd", "decode", "decode_multi", "prologue"], default="fwdbwd",
                     help="fwdbwd is the headline; the others are secondary measurements")
     ap.add_argument("--batch", type=int, default=0,
                     help="override B (profiling a smaller case; not a bench line)")
@@ -682,7 +689,7 @@ def main(argv=None):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
     try:
-        if args.workload not in ("fwdbwd", "kda"):
+        if args.workload not in ("fwdbwd", "kda", "long_fwdbwd"):
             out = run_secondary(args, rank, world, local_rank)
             if rank == 0:
                 if world == 1 and not args.no_cpu_baseline and args.workload in ("fwd", "decode"):

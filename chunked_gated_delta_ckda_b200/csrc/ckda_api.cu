@@ -249,7 +249,8 @@ int ckda_chunk_bwd(int B, int T, int H, int dk, int dv, int io_dtype, const void
   if (tcp) {
     CKDA_CUDA(tc_backward(a, recs, reinterpret_cast<unsigned char *>(w + L.dsend),
                           reinterpret_cast<unsigned char *>(w + L.du),
-                          reinterpret_cast<float *>(w + L.fscratch), stream));
+                          reinterpret_cast<float *>(w + L.fscratch), stream,
+                          reinterpret_cast<float *>(w + L.seg)));
     return CKDA_OK;
   }
   CKDA_CUDA(v1_backward(a, bf16, stream));

@@ -194,11 +194,19 @@ cudaError_t tc_forward(const FwdArgs &f, unsigned char *recs, float *fb, bool wr
                        bool intra_pass = true, bool state_tiles = false, float *seg_ws = nullptr);
 int tc_seg_count(int B, int H, int NC);  // segments per sequence of the long-sequence scan (0: off)
 size_t tc_seg_ws_bytes();                // workspace of the long-sequence scan
+int tc_seg_count_bwd(int B, int H, int NC);  // segments of the long-sequence backward (0: off)
+// the segments' maps M_g as rows [c][j] (and their offsets) from the records
+cudaError_t tc_seg_maps_rows(const FwdArgs &f, const unsigned char *recs, int G, float *seg_M, float *seg_b,
+                             cudaStream_t s);
+// adjoint states at each segment's end, from the last segment down:
+// end(G-1) = X0 (or 0), end(g-1) = M_g^T end(g) + e_g
+cudaError_t tc_seg_scan_reverse(const FwdArgs &f, int G, const float *seg_M, const float *seg_e, const float *X0,
+                                float *seg_ends, cudaStream_t s);
 // bf16 chunk-start state tiles of the records from fp32 chunk states [B,H,NC,128,128]
 cudaError_t tc_state_tiles(const float *chunk_states, unsigned char *recs, int B, int H, int NC,
                            cudaStream_t s);
 cudaError_t tc_backward(const BwdArgs &b, const unsigned char *recs, unsigned char *dS_tiles,
-                        unsigned char *dU_tiles, float *fb, cudaStream_t s);
+                        unsigned char *dU_tiles, float *fb, cudaStream_t s, float *seg_ws = nullptr);
 cudaError_t decode_step(int N, int H, int dk, int dv, bool bf16, const void *q,
                         const void *k, const void *v, const float *g, const int8_t *sign,
                         const void *beta, float *state, void *o, cudaStream_t s);

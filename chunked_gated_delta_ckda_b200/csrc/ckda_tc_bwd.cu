@@ -40,6 +40,12 @@ struct BwdTcArgs {
   unsigned char *dS_tiles;    // [n_chunks][H] DS_TILE
   unsigned char *dU_tiles;    // [n_chunks][H] DU_TILE
   float *fb;                  // per-CTA fallback scratch (3 x 64 x 128 fp32)
+  // segment mode of the reverse pass (long sequences): blockIdx.y = seq *
+  // seg_count + segment, each CTA walks one segment of seg_len chunks
+  int seg_len, seg_count;
+  const float *seg_in;  // adjoint state at each segment's end, fp32 [128][128] (null: zero)
+  float *seg_out;       // adjoint state at each segment's start (null: dS0 for the first segment)
+  bool no_tiles;        // provisional pass: no dS / dU tiles
 };
 
 __device__ __forceinline__ void cp_async16(void *smem_dst, const void *gsrc, bool valid) {
@@ -90,12 +96,29 @@ __global__ void __launch_bounds__(kSbThreads, 1) tc_state_bwd_kernel(BwdTcArgs t
   const bool grpA = tid < kSbGroup;
   const int gt = tid & (kSbGroup - 1);
   const int qd = warp & 3, ch = (warp >> 2) & 1;
-  const int h = blockIdx.x, seq = blockIdx.y, H = a.H;
+  const int h = blockIdx.x, H = a.H;
   const int v = 32 * qd + lane;
   const __nv_bfloat16 *dO = (const __nv_bfloat16 *)a.dO;
-  int first;
-  const int nc = a.map.seq_chunks(seq, first);
-  const size_t sbase = ((size_t)seq * H + h) * D * D;
+  // this CTA's chunks: a whole sequence, or one segment of it; the adjoint
+  // state it starts from (the range's end) and where the range's start state goes
+  int seq = blockIdx.y, first, nc;
+  const float *X0;
+  float *Xout;
+  if (ta.seg_len > 0) {
+    seq = blockIdx.y / ta.seg_count;
+    const int sg = blockIdx.y % ta.seg_count, j0 = sg * ta.seg_len;
+    nc = a.map.seq_chunks(seq, first);
+    nc = nc - j0 < ta.seg_len ? nc - j0 : ta.seg_len;
+    if (nc < 0) nc = 0;
+    first += j0;
+    const size_t own = ((size_t)blockIdx.y * H + h) * D * D;
+    X0 = ta.seg_in ? ta.seg_in + own : nullptr;
+    Xout = ta.seg_out ? ta.seg_out + own : ((sg == 0 && a.dS0) ? a.dS0 + ((size_t)seq * H + h) * D * D : nullptr);
+  } else {
+    nc = a.map.seq_chunks(seq, first);
+    X0 = a.dST ? a.dST + ((size_t)seq * H + h) * D * D : nullptr;
+    Xout = a.dS0 ? a.dS0 + ((size_t)seq * H + h) * D * D : nullptr;
+  }
 
   if (tid == 0) {
     mbar_init(&ms.mrec[0], 1);
@@ -145,6 +168,7 @@ __global__ void __launch_bounds__(kSbThreads, 1) tc_state_bwd_kernel(BwdTcArgs t
   // dL/dS_{c+1} snapshot of chunk j: the bf16 dS^T operand tile as it stands
   // (one bulk store by group A's first thread, after the tile's writers have synchronised)
   auto snapshot = [&](int j) {
+    if (ta.no_tiles) return;
     bulk_s2g(ta.dS_tiles + ((size_t)(first + j) * H + h) * DS_TILE, sm + SB_DS, DS_TILE);
     bulk_commit();
   };
@@ -159,10 +183,10 @@ __global__ void __launch_bounds__(kSbThreads, 1) tc_state_bwd_kernel(BwdTcArgs t
     for (int c0 = 64 * ch; c0 < 64 * ch + 64; c0 += 16) {
       float sv[16];
 #pragma unroll
-      for (int i = 0; i < 16; ++i) sv[i] = a.dST ? a.dST[sbase + (size_t)(c0 + i) * D + v] : 0.f;
+      for (int i = 0; i < 16; ++i) sv[i] = X0 ? X0[(size_t)(c0 + i) * D + v] : 0.f;
       if (nc == 0) {
-        if (a.dS0)
-          for (int i = 0; i < 16; ++i) a.dS0[sbase + (size_t)(c0 + i) * D + v] = sv[i];
+        if (Xout)
+          for (int i = 0; i < 16; ++i) Xout[(size_t)(c0 + i) * D + v] = sv[i];
         continue;
       }
       uint32_t pk[8];
@@ -270,8 +294,8 @@ __global__ void __launch_bounds__(kSbThreads, 1) tc_state_bwd_kernel(BwdTcArgs t
         tmem_ld16(lanebase + c0, sv);
         tmem_wait_ld();
         if (j == 0) {
-          if (a.dS0)
-            for (int i = 0; i < 16; ++i) a.dS0[sbase + (size_t)(c0 + i) * D + v] = sv[i];
+          if (Xout)
+            for (int i = 0; i < 16; ++i) Xout[(size_t)(c0 + i) * D + v] = sv[i];
           continue;
         }
         uint32_t pk[8];
@@ -331,7 +355,7 @@ __global__ void __launch_bounds__(kSbThreads, 1) tc_state_bwd_kernel(BwdTcArgs t
       if (lane == 0) mbar_arrive(&ms.dudone);
       fence_async_smem();
       group_sync(2, kSbGroup);
-      if (gt == 0) {
+      if (gt == 0 && !ta.no_tiles) {
         const int j = nc - 1 - s;
         bulk_s2g(ta.dU_tiles + ((size_t)(first + j) * H + h) * DU_TILE, sm + SB_DUG, DU_TILE);
         bulk_commit();
@@ -1142,7 +1166,7 @@ int num_sms() {
 // Backward on tensor cores.  recs: records of tc_forward's intra kernel for
 // these inputs; dS_tiles / dU_tiles: n_chunks * H tiles of 32 KiB / 16 KiB.
 cudaError_t tc_backward(const BwdArgs &b, const unsigned char *recs, unsigned char *dS_tiles,
-                        unsigned char *dU_tiles, float *fb, cudaStream_t s) {
+                        unsigned char *dU_tiles, float *fb, cudaStream_t s, float *seg_ws) {
   BwdTcArgs ta{};
   ta.b = b;
   ta.recs = recs;
@@ -1157,7 +1181,38 @@ cudaError_t tc_backward(const BwdArgs &b, const unsigned char *recs, unsigned ch
   e = cudaFuncSetAttribute(tc_grad_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_g);
   if (e != cudaSuccess) return e;
   if (b.map.n_seq == 0) return cudaSuccess;
-  {
+  const int G = (seg_ws && !b.map.table) ? tc_seg_count_bwd(b.B, b.H, b.map.NC) : 0;
+  if (G >= 2) {
+    // long sequences: dS at a segment's start = M_g^T (dS at its end) + e_g, with
+    // M_g the forward map of the segment's chunks and e_g the reverse pass from
+    // zero; the segments' maps, their provisional passes, the reverse scan, then
+    // every segment's pass from its true end state
+    FwdArgs f{};
+    f.B = b.B; f.T = b.T; f.H = b.H; f.dk = b.dk; f.dv = b.dv;
+    f.map = b.map;
+    f.status = b.status;
+    const size_t per = (size_t)b.B * G * b.H * D * D;
+    float *segM = seg_ws, *sege = seg_ws + per, *segE = seg_ws + 2 * per;
+    if ((e = tc_seg_maps_rows(f, recs, G, segM, sege, s)) != cudaSuccess) return e;
+    ta.seg_count = G;
+    ta.seg_len = (b.map.NC + G - 1) / G;
+    ta.seg_in = nullptr;
+    ta.seg_out = sege;
+    ta.no_tiles = true;
+    {
+      ProfScope prof("tc_state_bwd_provisional", s);
+      tc_state_bwd_kernel<<<dim3(b.H, b.B * G), kSbThreads, sm_sb, s>>>(ta);
+      if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    if ((e = tc_seg_scan_reverse(f, G, segM, sege, b.dST, segE, s)) != cudaSuccess) return e;
+    ta.seg_in = segE;
+    ta.seg_out = nullptr;
+    ta.no_tiles = false;
+    ProfScope prof("tc_state_bwd", s);
+    tc_state_bwd_kernel<<<dim3(b.H, b.B * G), kSbThreads, sm_sb, s>>>(ta);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    ta.seg_len = 0;
+  } else {
     ProfScope prof("tc_state_bwd", s);
     tc_state_bwd_kernel<<<dim3(b.H, b.map.n_seq), kSbThreads, sm_sb, s>>>(ta);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;

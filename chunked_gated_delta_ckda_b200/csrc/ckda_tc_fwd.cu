@@ -83,6 +83,9 @@ struct TcArgs {
   int seg_len, seg_count;
   float *seg_M, *seg_b;  // per segment: its affine map S -> M S + b (fp32 [128][128] each)
   float *seg_S0;         // per segment: its start state (fp32 [128][128])
+  bool seg_M_rows;       // the map kernel writes M itself ([c][j]) instead of M^T ([j][c])
+  bool seg_reverse;      // the scan runs from the last segment down (adjoint states)
+  const float *seg_X0;   // the scan's first state (null: zero)
 };
 
 __global__ void __launch_bounds__(kIntraThreads, 2) tc_intra_kernel(const __grid_constant__ TcArgs ta) {
@@ -931,9 +934,14 @@ __global__ void __launch_bounds__(kSegThreads, 1) tc_segmap_kernel(TcArgs ta) {
       tmem_ld16(lanebase + c0, x1);
       tmem_ld16(lanebase + 128 + c0, x2);
       tmem_wait_ld();
-      float4 *mrow = reinterpret_cast<float4 *>(Mo + (size_t)j * D + c0);
+      if (ta.seg_M_rows) {  // M[c][j]: a warp writes 32 consecutive j of each row c
 #pragma unroll
-      for (int m = 0; m < 4; ++m) mrow[m] = make_float4(x1[4 * m], x1[4 * m + 1], x1[4 * m + 2], x1[4 * m + 3]);
+        for (int m = 0; m < 16; ++m) Mo[(size_t)(c0 + m) * D + j] = x1[m];
+      } else {
+        float4 *mrow = reinterpret_cast<float4 *>(Mo + (size_t)j * D + c0);
+#pragma unroll
+        for (int m = 0; m < 4; ++m) mrow[m] = make_float4(x1[4 * m], x1[4 * m + 1], x1[4 * m + 2], x1[4 * m + 3]);
+      }
 #pragma unroll
       for (int m = 0; m < 16; ++m) bo[(size_t)(c0 + m) * D + j] = x2[m];
     }
@@ -948,7 +956,11 @@ __global__ void __launch_bounds__(kSegThreads, 1) tc_segmap_kernel(TcArgs ta) {
 }
 
 // The segments of one (sequence, head) in order, fp32 on CUDA cores:
-// start(0) = S0 (or 0), start(g + 1) = M_g start(g) + b_g.  The value columns
+// start(0) = S0 (or 0), start(g + 1) = M_g start(g) + b_g; or, reversed (the
+// backward's adjoint states, with the maps' rows M_g^T and the adjoint
+// offsets e_g): end(G - 1) = dS_T (or 0), end(g - 1) = M_g^T end(g) + e_g.
+// The kernel reads a table T_g (M_g^T for the forward, M_g for the reverse)
+// and forms out[c][v] = sum_k T_g[k][c] X[k][v] + b_g[c][v].  The value columns
 // are independent, so a CTA takes a slice of VC of them (blockIdx.z); a
 // thread holds a 4 x (VC / 8) block of the slice in registers.  M_g^T
 // (64 KB) is double-buffered in shared memory by bulk copies.
@@ -972,20 +984,22 @@ __global__ void __launch_bounds__(kScanThreads, 1) tc_segscan_kernel(TcArgs ta) 
     mbar_fence_init();
   }
   __syncthreads();
-  auto fetch = [&](int g) {  // M_g^T into buffer g & 1
-    const size_t sidx = ((size_t)(seq * G + g) * H + h) * D * D;
-    mbar_arrive_expect_tx(&mfull[g & 1], D * D * 4);
-    bulk_g2s(Mt + (g & 1) * D * D, ta.seg_M + sidx, D * D * 4, &mfull[g & 1]);
+  // step i handles segment g(i): i in order, or from the last one down
+  auto seg_of = [&](int i) { return ta.seg_reverse ? G - 1 - i : i; };
+  auto fetch = [&](int i) {  // the table of step i into buffer i & 1
+    const size_t sidx = ((size_t)(seq * G + seg_of(i)) * H + h) * D * D;
+    mbar_arrive_expect_tx(&mfull[i & 1], D * D * 4);
+    bulk_g2s(Mt + (i & 1) * D * D, ta.seg_M + sidx, D * D * 4, &mfull[i & 1]);
   };
   if (tid == 0 && G > 1) fetch(0);
   float st[4][NV];
-  const float *S0 = a.S0 ? a.S0 + ((size_t)seq * H + h) * D * D : nullptr;
+  const float *S0 = ta.seg_X0 ? ta.seg_X0 + ((size_t)seq * H + h) * D * D : nullptr;
 #pragma unroll
   for (int i = 0; i < 4; ++i)
 #pragma unroll
     for (int k = 0; k < NV; ++k) st[i][k] = S0 ? S0[(size_t)(c0 + i) * D + vg + k] : 0.f;
-  for (int g = 0; g < G; ++g) {
-    const size_t sidx = ((size_t)(seq * G + g) * H + h) * D * D;
+  for (int g = 0; g < G; ++g) {  // (g counts steps; the segment is seg_of(g))
+    const size_t sidx = ((size_t)(seq * G + seg_of(g)) * H + h) * D * D;
     float *out = ta.seg_S0 + sidx;
 #pragma unroll
     for (int i = 0; i < 4; ++i)
@@ -1049,6 +1063,27 @@ int tc_intra_ctas() {
 
 size_t tc_record_bytes() { return REC; }
 
+// The segment kernels' launches (the segment fields of ta are set).
+static cudaError_t launch_segmap(const TcArgs &ta, cudaStream_t s) {
+  const size_t sm_map = SG_MISC + sizeof(SegMisc) + 1024;
+  cudaError_t e = cudaFuncSetAttribute(tc_segmap_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_map);
+  if (e != cudaSuccess) return e;
+  ProfScope prof("tc_segmap", s);
+  tc_segmap_kernel<<<dim3(ta.f.H, ta.f.B * ta.seg_count), kSegThreads, sm_map, s>>>(ta);
+  return cudaGetLastError();
+}
+static cudaError_t launch_segscan(const TcArgs &ta, cudaStream_t s) {
+  // value-column slices of the scan: 8 (16 columns) while the CTAs fit on the SMs, else 4
+  const int split = 8 * ta.f.B * ta.f.H <= g_num_sms ? 8 : 4;
+  const size_t sm_scan = 128 + (2 * D * D + D * (D / split)) * sizeof(float) + 2 * sizeof(uint64_t);
+  auto scan = split == 8 ? tc_segscan_kernel<16> : tc_segscan_kernel<32>;
+  cudaError_t e = cudaFuncSetAttribute(scan, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_scan);
+  if (e != cudaSuccess) return e;
+  ProfScope prof("tc_segscan", s);
+  scan<<<dim3(ta.f.H, ta.f.B, split), kScanThreads, sm_scan, s>>>(ta);
+  return cudaGetLastError();
+}
+
 // Forward on tensor cores.  recs: n_chunks_bound * H records of REC bytes;
 // fb: tc_fwd_fallback_floats(tc_intra_ctas()) floats.  intra_pass = false
 // reuses records an earlier call wrote for the same inputs.
@@ -1110,27 +1145,9 @@ cudaError_t tc_forward(const FwdArgs &f, unsigned char *recs, float *fb, bool wr
       ta.seg_M = seg_ws;
       ta.seg_b = seg_ws + per;
       ta.seg_S0 = seg_ws + 2 * per;
-      // value-column slices of the scan: 8 (16 columns) while the CTAs fit on the SMs, else 4
-      const int split = 8 * f.B * f.H <= g_num_sms ? 8 : 4;
-      const size_t sm_map = SG_MISC + sizeof(SegMisc) + 1024;
-      const size_t sm_scan = 128 + (2 * D * D + D * (D / split)) * sizeof(float) + 2 * sizeof(uint64_t);
-      if ((e = cudaFuncSetAttribute(tc_segmap_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    (int)sm_map)) != cudaSuccess)
-        return e;
-      auto scan = split == 8 ? tc_segscan_kernel<16> : tc_segscan_kernel<32>;
-      if ((e = cudaFuncSetAttribute(scan, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_scan)) !=
-          cudaSuccess)
-        return e;
-      {
-        ProfScope prof("tc_segmap", s);
-        tc_segmap_kernel<<<dim3(f.H, f.B * G), kSegThreads, sm_map, s>>>(ta);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
-      }
-      {
-        ProfScope prof("tc_segscan", s);
-        scan<<<dim3(f.H, f.B, split), kScanThreads, sm_scan, s>>>(ta);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
-      }
+      ta.seg_X0 = f.S0;
+      if ((e = launch_segmap(ta, s)) != cudaSuccess) return e;
+      if ((e = launch_segscan(ta, s)) != cudaSuccess) return e;
       ProfScope prof(write_o ? "tc_state_fwd" : "tc_state_fwd_recompute", s);
       tc_state_kernel<<<dim3(f.H, f.B * G), kStateThreads, sm_state, s>>>(ta);
       if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -1141,6 +1158,44 @@ cudaError_t tc_forward(const FwdArgs &f, unsigned char *recs, float *fb, bool wr
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   return cudaSuccess;
+}
+
+// Segments of the long-sequence backward: the same split as the forward's
+// (tc_seg_count) but only where three passes of L chunks (the maps, the
+// reverse pass from zero, the reverse pass from the scanned states) and the
+// scan beat one pass of NC chunks.
+int tc_seg_count_bwd(int B, int H, int NC) {
+  const int G = tc_seg_count(B, H, NC);
+  if (G < 2) return 0;
+  const int L = (NC + G - 1) / G;
+  return 3 * L + G + 8 < NC ? G : 0;
+}
+
+cudaError_t tc_seg_maps_rows(const FwdArgs &f, const unsigned char *recs, int G, float *seg_M, float *seg_b,
+                             cudaStream_t s) {
+  TcArgs ta{};
+  ta.f = f;
+  ta.recs = const_cast<unsigned char *>(recs);
+  ta.seg_count = G;
+  ta.seg_len = (f.map.NC + G - 1) / G;
+  ta.seg_M = seg_M;
+  ta.seg_b = seg_b;
+  ta.seg_M_rows = true;
+  return launch_segmap(ta, s);
+}
+
+cudaError_t tc_seg_scan_reverse(const FwdArgs &f, int G, const float *seg_M, const float *seg_e, const float *X0,
+                                float *seg_ends, cudaStream_t s) {
+  TcArgs ta{};
+  ta.f = f;
+  ta.seg_count = G;
+  ta.seg_len = (f.map.NC + G - 1) / G;
+  ta.seg_M = const_cast<float *>(seg_M);
+  ta.seg_b = const_cast<float *>(seg_e);
+  ta.seg_S0 = seg_ends;
+  ta.seg_reverse = true;
+  ta.seg_X0 = X0;
+  return launch_segscan(ta, s);
 }
 
 }  // namespace ckda

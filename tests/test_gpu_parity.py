@@ -226,6 +226,27 @@ def test_long_sequence_segment_scan(B, H):
         check(key, got[key], ref[key], io)
 
 
+@pytest.mark.parametrize("B,H,use_saved", [(1, 2, True), (2, 1, False)])
+def test_long_sequence_backward_segments(B, H, use_saved):
+    """Few pairs over 151 chunks: the backward also splits the sequence into
+    segments (the maps M_g, a provisional reverse pass per segment from zero,
+    the reverse scan of the adjoint states, then every segment from its true
+    end).  Gradients with S0 and dS_T against the oracle; the saved-buffer
+    and recomputing paths."""
+    io = torch.bfloat16
+    T = 64 * 150 + 33
+    inp = random_inputs(B, T, H, 128, 128, io, seed=61 + B, gscale=0.05, extreme_p=0.05)
+    d = to_dev(inp)
+    S0, dST = inp["S0"].cuda(), inp["dST"].cuda()
+    r = api.chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["sign"], d["beta"], S0=S0, save_for_backward=use_saved)
+    got = api.chunk_bwd(d["q"], d["k"], d["v"], d["g"], d["sign"], d["beta"], d["dO"], S0=S0, dST=dST,
+                        saved=r[3] if use_saved else None)
+    torch.cuda.synchronize()
+    ref = oracle_bwd_batched(inp, inp["dO"], S0=inp["S0"], dST=inp["dST"])
+    for key in ("dq", "dk", "dv", "dg", "dbeta", "dS0"):
+        check(key, got[key], ref[key], io)
+
+
 def test_long_sequence_segment_scan_many_pairs():
     """20 (sequence, head) pairs over 64 chunks: four segments of 16 chunks,
     the scan split into four value-column slices per pair.  Forward chunk
