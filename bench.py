@@ -125,6 +125,8 @@ class ClockSampler:
         self.proc = None
         self.path = None
         self.dev = device_index
+        self.base = 0
+        self.extended = False
 
     def start(self):
         try:
@@ -134,10 +136,36 @@ class ClockSampler:
             os.close(fd)
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", sel, "--query-gpu=" + self.FIELDS,
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            t0 = time.time()  # the sampler is running before anything is timed
+            while self.count() < 1 and time.time() - t0 < 3.0 and self.proc.poll() is None:
+                time.sleep(0.01)
         except Exception:
             self.proc = None
+
+    def count(self) -> int:
+        try:
+            with open(self.path) as f:
+                return sum(1 for _ in f)
+        except Exception:
+            return 0
+
+    def mark(self):
+        """The timed region starts: samples before it are not reported."""
+        self.base = self.count()
+
+    def keep_loaded(self, step, min_samples=3, max_s=1.5):
+        """A timed region shorter than the sampling interval yields too few
+        samples: run the same (untimed) step until min_samples have been taken
+        since mark(), for at most max_s seconds."""
+        if self.proc is None:
+            return
+        t0 = time.time()
+        while self.count() - self.base < min_samples and time.time() - t0 < max_s:
+            step()
+            torch.cuda.synchronize()
+            self.extended = True
 
     def stop(self) -> dict:
         if self.proc is None:
@@ -149,9 +177,9 @@ class ClockSampler:
             self.proc.kill()
         rows = []
         with open(self.path) as f:
-            for line in f:
+            for n, line in enumerate(f):
                 parts = [p.strip() for p in line.split(",")]
-                if len(parts) == 7:
+                if n >= self.base and len(parts) == 7:
                     rows.append(parts)
         os.unlink(self.path)
         if not rows:
@@ -162,7 +190,9 @@ class ClockSampler:
         reasons = sorted({names[i] for r in rows for i in range(4) if r[3 + i] == "Active"})
         return {"sm_mhz": statistics.median(sm) if sm else None,
                 "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
-                "samples": len(rows)}
+                "samples": len(rows),
+                "window": ("the timed region and the identical untimed steps right after it"
+                           if self.extended else "the timed region")}
 
 
 # ---------------------------------------------------------------------------
@@ -247,9 +277,11 @@ def run_ours(args, rank, world, local_rank):
         step()
     torch.cuda.synchronize()
     _abi.ckda_profile_enable(True)
+    clocks.mark()
     ms = _time_steps(step, args.steps, 0, world)
     _abi.ckda_profile_enable(False)
     prof = _abi.ckda_profile_collect()
+    clocks.keep_loaded(step)
     clk = clocks.stop()
     ms_max = reduce_max(ms, world)
     value = aggregate(tokens, world, ms_max)
@@ -437,9 +469,11 @@ def run_secondary(args, rank, world, local_rank):
     torch.cuda.synchronize()
     _abi.ckda_profile_reset()
     _abi.ckda_profile_enable(True)
+    clocks.mark()
     ms = _time_steps(step, args.steps, 0, world)
     _abi.ckda_profile_enable(False)
     prof = _abi.ckda_profile_collect()
+    clocks.keep_loaded(step)
     clk = clocks.stop()
     ms = reduce_max(ms, world)
     total = sum(t for _, t in prof.values())
