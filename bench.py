@@ -665,7 +665,7 @@ def run_reference(args, rank, world):
     w = W.LAYER_FWDBWD
     inp = W.make(w)
     cores = oracle.default_threads()
-    n_pairs = max(2, min(8, cores))
+    n_pairs = max(2, min(32, cores))  # one sequence per host thread: every core busy
     pairs = [(i % w.B, (i * 5) % w.H) for i in range(n_pairs)]
     threads = min(cores, n_pairs)
     for _ in range(args.warmup):
