@@ -2,7 +2,8 @@
 """Benchmark of the CKDA recurrence library on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload fwdbwd|kda|fwd|varlen|long|long_fwdbwd|decode|decode_multi|prologue]
+                    [--workload fwdbwd|kda|fwd|varlen|varlen_fwdbwd|long|long_fwdbwd|
+                                decode|decode_multi|prologue]
 
 Default workload (the headline): one step = ckda_chunk_fwd (saving its
 per-chunk results for the backward) + ckda_chunk_bwd on B=8, H=16, T=4096,
@@ -405,7 +406,7 @@ def run_secondary(args, rank, world, local_rank):
         metric = "CKDA prologue fwd+bwd tokens/s (short conv + q/k L2 norm + signed gate + beta; B=8,T=4096,H=16,d=128,bf16)"
         cfg = {"workload": "prologue_" + w.name, "B": B, "T": T, "H": H, "dk": dk, "dv": dv, "io_dtype": "bf16",
                "g_floor": -5.0, "l2": "inputs larger than L2"}
-    elif args.workload == "varlen":
+    elif args.workload in ("varlen", "varlen_fwdbwd"):
         w = W.VARLEN
         inp = W.make_varlen(w)
         d = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
@@ -426,6 +427,23 @@ def run_secondary(args, rank, world, local_rank):
         metric = "CKDA varlen fwd tokens/s (65536 packed tokens,H=16,d=128,bf16)"
         cfg = {"workload": w.name, "total_T": T, "docs": Nd, "H": H, "dk": dk, "dv": dv,
                "io_dtype": "bf16", "l2": "inputs larger than L2"}
+        if args.workload == "varlen_fwdbwd":  # the packed training step: forward then backward
+            gen = torch.Generator().manual_seed(w.seed + 100)
+            dO = torch.randn(1, T, H, dv, generator=gen).to(w.io_dtype).to(dev)
+            gb = dict(dq=torch.empty_like(d["q"]), dk=torch.empty_like(d["k"]), dv=torch.empty_like(d["v"]),
+                      dg=torch.empty_like(d["g"]), dbeta=torch.empty_like(d["beta"]))
+            wsb = api.workspace(_abi.CKDA_OP_VARLEN_BWD, 1, T, H, dk, dv, Nd, device=dev, cache=False)
+            fwd_step = step
+
+            def step():
+                fwd_step()
+                _abi.ckda_varlen_bwd(T, Nd, cu, mx, H, dk, dv, code, d["q"], d["k"], d["v"], d["g"],
+                                     d["sign"], d["beta"], None, dO, None, gb["dq"], gb["dk"], gb["dv"],
+                                     gb["dg"], gb["dbeta"], None, wsb)
+            per_unit, unit_name = FWD_BYTES + BWD_BYTES, "B per token-head (fwd + bwd)"
+            kernel_bytes = {"tc_grad": BWD_BYTES, "tc_intra": FWD_BYTES}
+            metric = "CKDA varlen fwd+bwd tokens/s (65536 packed tokens,H=16,d=128,bf16)"
+            cfg["workload"] = "varlen_fwdbwd_bf16"
     elif args.workload == "long":
         w = W.LONG
         inp = W.make(w)
@@ -698,7 +716,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer pass")
-    ap.add_argument("--workload", choices=["fwdbwd", "kda", "fwd", "varlen", "long", "long_fwdbwd", "decode", "decode_multi", "prologue"], default="fwdbwd",
+    ap.add_argument("--workload", choices=["fwdbwd", "kda", "fwd", "varlen", "varlen_fwdbwd", "long", "long_fwdbwd", "decode",
+                             "decode_multi", "prologue"], default="fwdbwd",
                     help="fwdbwd is the headline; the others are secondary measurements")
     ap.add_argument("--batch", type=int, default=0,
                     help="override B (profiling a smaller case; not a bench line)")

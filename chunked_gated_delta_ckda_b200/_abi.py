@@ -22,6 +22,7 @@ CKDA_BF16 = 1
 CKDA_OP_CHUNK_FWD = 0
 CKDA_OP_CHUNK_BWD = 1
 CKDA_OP_VARLEN_FWD = 2
+CKDA_OP_VARLEN_BWD = 3
 CKDA_CHUNK = 64
 
 STATUS = {0: "CKDA_OK", 1: "CKDA_ERR_INVALID_ARG", 2: "CKDA_ERR_UNSUPPORTED",
@@ -57,6 +58,7 @@ def _load():
         lib.ckda_prologue_fwd.argtypes = [I] * 6 + [P] * 8 + [F] + [P] * 7
         lib.ckda_prologue_bwd.argtypes = [I] * 6 + [P] * 8 + [F] + [P] * 14
         lib.ckda_varlen_fwd.argtypes = [I, I, P, I, I, I, I, I] + [P] * 10 + [Z, P]
+        lib.ckda_varlen_bwd.argtypes = [I, I, P, I, I, I, I, I] + [P] * 16 + [Z, P]
         lib.ckda_chunk_fwd_noalloc.argtypes = [I] * 6 + [P] * 11
         lib.ckda_check_device_status.argtypes = [P, P]
         lib.ckda_status_string.argtypes = [I]
@@ -69,7 +71,7 @@ def _load():
         lib.ckda_profile_reset.argtypes = []
         lib.ckda_profile_reset.restype = None
         for f in ("ckda_chunk_fwd", "ckda_chunk_bwd", "ckda_decode_step", "ckda_decode_multi", "ckda_varlen_fwd",
-                  "ckda_prologue_fwd", "ckda_prologue_bwd",
+                  "ckda_prologue_fwd", "ckda_prologue_bwd", "ckda_varlen_bwd",
                   "ckda_chunk_fwd_noalloc", "ckda_check_device_status", "ckda_version", "ckda_profile_enable",
                   "ckda_profile_collect", "ckda_profile_get"):
             getattr(lib, f).restype = I
@@ -152,6 +154,14 @@ def ckda_decode_multi(N, K, H, dk, dv, io_dtype, q, k, v, g, sign, beta, n_token
     _check(_load().ckda_decode_multi(N, K, H, dk, dv, io_dtype, _p(q), _p(k), _p(v), _p(g), _p(sign),
                                      _p(beta), _p(n_tokens), _p(slots), n_slots, _p(state),
                                      1 if write_state else 0, _p(o), _s(stream)), "ckda_decode_multi")
+
+
+def ckda_varlen_bwd(total_T, N, cu_seqlens, max_seqlen, H, dk, dv, io_dtype, q, k, v, g, sign, beta, S0, dO,
+                    dST, dq, dk_out, dv_out, dg, dbeta, dS0, ws, ws_bytes=None, stream=None):
+    _check(_load().ckda_varlen_bwd(total_T, N, _p(cu_seqlens), max_seqlen, H, dk, dv, io_dtype, _p(q), _p(k),
+                                   _p(v), _p(g), _p(sign), _p(beta), _p(S0), _p(dO), _p(dST), _p(dq), _p(dk_out),
+                                   _p(dv_out), _p(dg), _p(dbeta), _p(dS0), _p(ws), _nbytes(ws, ws_bytes),
+                                   _s(stream)), "ckda_varlen_bwd")
 
 
 def ckda_prologue_fwd(B, T, H, dk, dv, io_dtype, xq, xk, xv, wq, wk, wv, a, b, g_floor, q, k, v, g, sign, beta,

@@ -9,6 +9,7 @@ torch (device memory is torch's job here) and call the library.
     o         = decode_multi(q, k, v, g, sign, beta, pool, slots=None, n_tokens=None,
                              write_state=True)                 # K tokens per sequence
     o, ST     = varlen_fwd(q, k, v, g, sign, beta, cu_seqlens, max_seqlen, S0=None)
+    grads     = varlen_bwd(q, k, v, g, sign, beta, dO, cu_seqlens, max_seqlen, S0=None, dST=None)
     x         = prologue_fwd(xq, xk, xv, wq, wk, wv, a, b, g_floor=-5.0)   # q, k, v, g, sign, beta
     grads     = prologue_bwd(xq, xk, xv, wq, wk, wv, a, b, dq, dk, dv, dg, dbeta, g_floor=-5.0)
 
@@ -24,7 +25,8 @@ from typing import Optional
 import torch
 
 from . import _abi
-from ._abi import CKDA_BF16, CKDA_F32, CKDA_OP_CHUNK_BWD, CKDA_OP_CHUNK_FWD, CKDA_OP_VARLEN_FWD
+from ._abi import (CKDA_BF16, CKDA_F32, CKDA_OP_CHUNK_BWD, CKDA_OP_CHUNK_FWD, CKDA_OP_VARLEN_BWD,
+                   CKDA_OP_VARLEN_FWD)
 
 _ws_cache: dict = {}
 
@@ -252,3 +254,27 @@ def varlen_fwd(q, k, v, g, sign, beta, cu_seqlens, max_seqlen, S0=None, output_f
     _abi.ckda_varlen_fwd(T, N, cu_seqlens, int(max_seqlen), H, dk, dv, io_code(q.dtype), q, k, v,
                          g, sign, beta, S0, o, ST, ws)
     return o, ST
+
+
+def varlen_bwd(q, k, v, g, sign, beta, dO, cu_seqlens, max_seqlen, S0=None, dST=None, need_dS0=True, ws=None):
+    """Gradients of varlen_fwd: dict dq, dk, dv, dg, dbeta, dS0 ([N,H,dk,dv] or None)."""
+    if q.dim() != 4 or q.shape[0] != 1:
+        raise ValueError("packed q must have shape (1, total_T, H, dk), got %s" % (tuple(q.shape),))
+    T = q.shape[1]
+    H, dk, dv = _recurrence_inputs(q, k, v, g, sign, beta, (1, T))
+    if cu_seqlens.dim() != 1 or cu_seqlens.dtype != torch.int32:
+        raise TypeError("cu_seqlens must be a 1-D int32 tensor")
+    N = cu_seqlens.numel() - 1
+    _expect("dO", dO, (1, T, H, dv), q.dtype)
+    _expect("S0", S0, (N, H, dk, dv), torch.float32, optional=True)
+    _expect("dST", dST, (N, H, dk, dv), torch.float32, optional=True)
+    q, k, v, g, sign, beta, dO, S0, dST, cu_seqlens = map(
+        _c, (q, k, v, g, sign, beta, dO, S0, dST, cu_seqlens))
+    out = dict(dq=torch.empty_like(q), dk=torch.empty_like(k), dv=torch.empty_like(v), dg=torch.empty_like(g),
+               dbeta=torch.empty_like(beta),
+               dS0=torch.empty(N, H, dk, dv, dtype=torch.float32, device=q.device) if need_dS0 else None)
+    if ws is None:
+        ws = workspace(CKDA_OP_VARLEN_BWD, 1, T, H, dk, dv, N, device=q.device)
+    _abi.ckda_varlen_bwd(T, N, cu_seqlens, int(max_seqlen), H, dk, dv, io_code(q.dtype), q, k, v, g, sign, beta,
+                         S0, dO, dST, out["dq"], out["dk"], out["dv"], out["dg"], out["dbeta"], out["dS0"], ws)
+    return out

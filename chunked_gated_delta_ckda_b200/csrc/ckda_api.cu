@@ -9,7 +9,7 @@ namespace ckda {
 
 WsLayout ws_layout(int op, int B, int T, int H, int dk, int dv, int N) {
   WsLayout L;
-  const bool packed = (op == CKDA_OP_VARLEN_FWD);
+  const bool packed = (op == CKDA_OP_VARLEN_FWD || op == CKDA_OP_VARLEN_BWD);
   int64_t nch;
   int NC = 0;
   if (packed) {
@@ -36,8 +36,8 @@ WsLayout ws_layout(int op, int B, int T, int H, int dk, int dv, int N) {
     L.seg = off;
     off += align256(tc_seg_ws_bytes());
   }
-  if (op == CKDA_OP_CHUNK_BWD) {
-    const size_t st = (size_t)B * H * NC * dk * dv * sizeof(float);
+  if (op == CKDA_OP_CHUNK_BWD || op == CKDA_OP_VARLEN_BWD) {
+    const size_t st = (size_t)(packed ? nch : (int64_t)B * NC) * H * dk * dv * sizeof(float);
     L.states = off;
     off += align256(st);
     L.dsend = off;
@@ -129,8 +129,8 @@ size_t saved_bytes_for(int B, int T, int H, int dk, int dv, int io_dtype) {
 extern "C" {
 
 size_t ckda_workspace_size(int op, int B, int T, int H, int dk, int dv, int N) {
-  if (op < CKDA_OP_CHUNK_FWD || op > CKDA_OP_VARLEN_FWD) return 0;
-  if (op == CKDA_OP_VARLEN_FWD) {
+  if (op < CKDA_OP_CHUNK_FWD || op > CKDA_OP_VARLEN_BWD) return 0;
+  if (op == CKDA_OP_VARLEN_FWD || op == CKDA_OP_VARLEN_BWD) {
     if (B != 1 || N < 0) return 0;
   }
   if (check_common(B, T, H, dk, dv, CKDA_F32) != CKDA_OK) return 0;
@@ -368,6 +368,74 @@ int ckda_varlen_fwd(int total_T, int N, const int32_t *cu_seqlens, int max_seqle
   }
   CKDA_CUDA(v1_intra(a, bf16, reinterpret_cast<float *>(w + L.fscratch), stream));
   CKDA_CUDA(v1_state_fwd(a, bf16, true, nullptr, stream));
+  return CKDA_OK;
+}
+
+int ckda_varlen_bwd(int total_T, int N, const int32_t *cu_seqlens, int max_seqlen, int H, int dk, int dv,
+                    int io_dtype, const void *q, const void *k, const void *v, const float *g,
+                    const int8_t *sign, const void *beta, const float *S0, const void *dO, const float *dST,
+                    void *dq, void *dk_out, void *dv_out, float *dg, void *dbeta, float *dS0, void *ws,
+                    size_t ws_bytes, cudaStream_t stream) {
+  CKDA_TRY(check_common(1, total_T, H, dk, dv, io_dtype));
+  if (N < 0) return CKDA_ERR_INVALID_ARG;
+  if (N == 0) return total_T == 0 ? CKDA_OK : CKDA_ERR_INVALID_ARG;
+  if (!cu_seqlens) return CKDA_ERR_INVALID_ARG;
+  if (total_T > 0 && (max_seqlen < 1 || max_seqlen > total_T)) return CKDA_ERR_INVALID_ARG;
+  if (total_T > 0)
+    CKDA_TRY(check_ptrs({q, k, v, g, beta, dO, dq, dk_out, dv_out, dg, dbeta}, {sign, S0, dST, dS0}));
+  else
+    CKDA_TRY(check_ptrs({}, {sign, S0, dST, dS0}));
+  if ((reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) != 0) return CKDA_ERR_ALIGNMENT;
+  const WsLayout L = ws_layout(CKDA_OP_VARLEN_BWD, 1, total_T, H, dk, dv, N);
+  CKDA_TRY(check_ws(ws, ws_bytes, L.total));
+  char *w = static_cast<char *>(ws);
+  CKDA_CUDA(cudaMemsetAsync(w, 0, sizeof(DevStatus), stream));
+  FwdArgs f{};
+  f.B = 1; f.T = total_T; f.H = H; f.dk = dk; f.dv = dv;
+  f.q = q; f.k = k; f.v = v; f.beta = beta; f.g = g; f.sign = sign; f.S0 = S0;
+  f.map.table = reinterpret_cast<const int32_t *>(w + L.table);
+  f.map.seq_first = reinterpret_cast<const int32_t *>(w + L.seq_first);
+  f.map.status = reinterpret_cast<const DevStatus *>(w);
+  f.map.T = total_T;
+  f.map.NC = 0;
+  f.map.n_seq = N;
+  f.map.n_chunks_bound = L.n_chunks_bound;
+  f.intra = reinterpret_cast<float *>(w + L.intra);
+  f.status = reinterpret_cast<DevStatus *>(w);
+  CKDA_CUDA(build_chunk_table(cu_seqlens, N, total_T, total_T > 0 ? max_seqlen : 0, L.n_chunks_bound,
+                              reinterpret_cast<int32_t *>(w + L.table), reinterpret_cast<int32_t *>(w + L.seq_first),
+                              reinterpret_cast<DevStatus *>(w), stream));
+  const bool bf16 = io_dtype == CKDA_BF16;
+  const bool tcp = use_tensor_cores(io_dtype, dk, dv);
+  const float *states = nullptr;
+  unsigned char *recs = reinterpret_cast<unsigned char *>(w + L.intra);
+  if (tcp) {  // records with their bf16 chunk-start states, recomputed
+    CKDA_CUDA(tc_forward(f, recs, reinterpret_cast<float *>(w + L.fscratch), false, nullptr, stream,
+                         /*state_pass=*/true, /*intra_pass=*/true, /*state_tiles=*/true, nullptr));
+  } else {
+    CKDA_CUDA(v1_intra(f, bf16, reinterpret_cast<float *>(w + L.fscratch), stream));
+    float *st = reinterpret_cast<float *>(w + L.states);
+    CKDA_CUDA(v1_state_fwd(f, bf16, false, st, stream));
+    states = st;
+  }
+  BwdArgs a{};
+  a.B = 1; a.T = total_T; a.H = H; a.dk = dk; a.dv = dv;
+  a.q = q; a.k = k; a.v = v; a.beta = beta; a.dO = dO; a.g = g; a.sign = sign;
+  a.S0 = S0; a.dST = dST; a.states = states;
+  a.dq = dq; a.dkg = dk_out; a.dvg = dv_out; a.dbeta = dbeta; a.dg = dg; a.dS0 = dS0;
+  a.map = f.map;
+  a.intra = f.intra;
+  a.dsend = reinterpret_cast<float *>(w + L.dsend);
+  a.du = reinterpret_cast<float *>(w + L.du);
+  a.scratch = reinterpret_cast<float *>(w + L.scratch);
+  a.status = f.status;
+  if (tcp) {
+    CKDA_CUDA(tc_backward(a, recs, reinterpret_cast<unsigned char *>(w + L.dsend),
+                          reinterpret_cast<unsigned char *>(w + L.du),
+                          reinterpret_cast<float *>(w + L.fscratch), stream, nullptr));
+    return CKDA_OK;
+  }
+  CKDA_CUDA(v1_backward(a, bf16, stream));
   return CKDA_OK;
 }
 

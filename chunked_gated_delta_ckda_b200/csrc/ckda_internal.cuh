@@ -71,6 +71,11 @@ struct ChunkMap {
       len = rem < C ? rem : C;
     }
   }
+  // slot of a per-(chunk, head) state in a chunk-state buffer: [B][H][NC]
+  // (batched: the layout callers see) or [chunk id][H] (packed)
+  __device__ __forceinline__ size_t state_slot(int seq, int h, int H, int j, int cid) const {
+    return packed() ? (size_t)cid * H + h : ((size_t)seq * H + h) * NC + j;
+  }
   __device__ __forceinline__ int seq_chunks(int seq, int &first) const {
     if (packed()) {
       first = seq_first[seq];

@@ -279,7 +279,7 @@ __global__ void __launch_bounds__(NT) state_fwd_kernel(FwdArgs a, bool write_o,
     a.map.info(cid, sq, tok0, len, jl);
     const IntraPtrs in = intra_ptrs(a.intra + ((size_t)cid * H + h) * intra_floats(dk, dv), dk, dv);
     if (states_out) {
-      float *dst = states_out + (((size_t)seq * H + h) * a.map.NC + jc) * dk * dv;
+      float *dst = states_out + a.map.state_slot(seq, h, H, jc, cid) * dk * dv;
       for (int idx = threadIdx.x; idx < dk * DVS; idx += blockDim.x)
         dst[(size_t)(idx / DVS) * dv + c0 + idx % DVS] = S[idx];
     }
@@ -338,7 +338,7 @@ __global__ void __launch_bounds__(NT) state_bwd_kernel(BwdArgs a) {
     int64_t tok0;
     a.map.info(cid, sq, tok0, len, jl);
     const IntraPtrs in = intra_ptrs(a.intra + ((size_t)cid * H + h) * intra_floats(dk, dv), dk, dv);
-    float *dst = a.dsend + (((size_t)seq * H + h) * a.map.NC + jc) * dk * dv;
+    float *dst = a.dsend + a.map.state_slot(seq, h, H, jc, cid) * dk * dv;
     for (int idx = threadIdx.x; idx < dk * DVS; idx += blockDim.x)
       dst[(size_t)(idx / DVS) * dv + c0 + idx % DVS] = dS[idx];
     for (int idx = threadIdx.x; idx < C * DVS; idx += blockDim.x) {
@@ -428,7 +428,7 @@ __global__ void __launch_bounds__(NT) grad_kernel(BwdArgs a) {
     int64_t tok0;
     a.map.info(cid, seq, tok0, len, jl);
     const bool fast = intra_core<IO>(q, k, v, a.g, a.sign, beta, tok0, len, h, H, dk, dv, b);
-    const size_t sidx = (((size_t)seq * H + h) * a.map.NC + jl) * dk * dv;
+    const size_t sidx = a.map.state_slot(seq, h, H, jl, cid) * dk * dv;
     const float *Sc = a.states + sidx;
     const float *dS1 = a.dsend + sidx;
     const float *duw = a.du + ((size_t)cid * H + h) * C * dv;

@@ -82,12 +82,14 @@ extern "C" {
 #define CKDA_OP_CHUNK_FWD 0
 #define CKDA_OP_CHUNK_BWD 1
 #define CKDA_OP_VARLEN_FWD 2
+#define CKDA_OP_VARLEN_BWD 3
 
 #define CKDA_CHUNK 64
 
 /* Workspace bytes an operation needs.  For CKDA_OP_CHUNK_FWD / _BWD pass the
- * batched shape (N ignored); for CKDA_OP_VARLEN_FWD pass B = 1, T = total
- * tokens and N = number of sequences.  Returns 0 for invalid arguments. */
+ * batched shape (N ignored); for CKDA_OP_VARLEN_FWD / _BWD pass B = 1,
+ * T = total tokens and N = number of sequences.  Returns 0 for invalid
+ * arguments. */
 size_t ckda_workspace_size(int op, int B, int T, int H, int dk, int dv, int N);
 
 /* Bytes of the "saved" buffer through which ckda_chunk_fwd can hand its
@@ -241,6 +243,23 @@ int ckda_varlen_fwd(int total_T, int N, const int32_t *cu_seqlens,
                     const int8_t *sign, const void *beta, const float *S0,
                     void *o, float *ST, void *ws, size_t ws_bytes,
                     cudaStream_t stream);
+
+/* Backward of ckda_varlen_fwd: gradients over N packed documents (training
+ * on packed documents).  Arguments as ckda_varlen_fwd plus
+ *   dO [1,total_T,H,dv] io;  dST [N,H,dk,dv] f32, nullable: per-document
+ *   gradient of the final states;  dq, dk_out [1,total_T,H,dk] io;
+ *   dv_out [1,total_T,H,dv] io;  dg [1,total_T,H,dk] f32;  dbeta
+ *   [1,total_T,H] io;  dS0 [N,H,dk,dv] f32, nullable.
+ * The per-chunk forward results are recomputed in the workspace
+ * (ckda_workspace_size(CKDA_OP_VARLEN_BWD, 1, total_T, H, dk, dv, N) bytes).
+ * Malformed cu_seqlens are reported as for the forward. */
+int ckda_varlen_bwd(int total_T, int N, const int32_t *cu_seqlens,
+                    int max_seqlen, int H, int dk, int dv, int io_dtype,
+                    const void *q, const void *k, const void *v, const float *g,
+                    const int8_t *sign, const void *beta, const float *S0,
+                    const void *dO, const float *dST, void *dq, void *dk_out,
+                    void *dv_out, float *dg, void *dbeta, float *dS0, void *ws,
+                    size_t ws_bytes, cudaStream_t stream);
 
 /* ---- chunked forward without any allocation --------------------------------
  * The pages have no counterpart to this call; it serves callers that cannot

@@ -34,6 +34,8 @@ def test_workspace_size_rules():
     assert ws(0, 1, 100, 2, 96, 64, 0) == 0      # unsupported dk
     assert ws(2, 2, 100, 2, 64, 64, 3) == 0      # packed call needs B == 1
     assert ws(7, 1, 100, 2, 64, 64, 0) == 0      # unknown op
+    assert ws(3, 1, 65536, 16, 128, 128, 44) > ws(2, 1, 65536, 16, 128, 128, 44)  # packed backward
+    assert ws(3, 2, 100, 2, 64, 64, 3) == 0      # packed backward needs B == 1
     assert ws(0, 1, 0, 2, 64, 64, 0) > 0         # empty input still has a status block
 
 
@@ -90,6 +92,11 @@ def test_host_validation_without_gpu():
     v = [fake] * 9
     assert lib.ckda_varlen_fwd(100, 2, fake, 0, 2, 64, 64, 0, *v, fake, 1 << 30, None) == 1
     assert lib.ckda_varlen_fwd(100, -1, fake, 50, 2, 64, 64, 0, *v, fake, 1 << 30, None) == 1
+    vb = [fake] * 15
+    assert lib.ckda_varlen_bwd(100, 2, fake, 0, 2, 64, 64, 0, *vb, fake, 1 << 30, None) == 1   # max_seqlen
+    assert lib.ckda_varlen_bwd(100, 2, None, 50, 2, 64, 64, 0, *vb, fake, 1 << 30, None) == 1  # cu_seqlens
+    assert lib.ckda_varlen_bwd(100, 2, fake, 50, 2, 64, 64, 0, *vb, fake, 16, None) == 4       # workspace
+    assert lib.ckda_varlen_bwd(0, 0, fake, 0, 2, 64, 64, 0, *vb, fake, 1 << 30, None) == 0     # nothing to do
 
     def bwd(io, b, ws_bytes, saved=nosave):
         return lib.ckda_chunk_bwd(1, 64, 2, 128, 128, io, *b[:10], *saved, *b[10:], fake, ws_bytes, None)

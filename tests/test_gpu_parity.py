@@ -632,3 +632,56 @@ def test_full_prologue_sampled_heads():
             check("%s[h=%d]" % (n, h), gr[n][:, :, hs], rg[n], w.io_dtype)
         for n in ("dwq", "dwk", "dwv"):
             check("%s[h=%d]" % (n, h), gr[n][h * 128:(h + 1) * 128], rg[n], w.io_dtype)
+
+
+# ---------------------------------------------------------------------------
+# packed documents: backward
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("io,d", [(torch.bfloat16, 128), (torch.float32, 64)])
+@pytest.mark.parametrize("lens", [[200, 1, 64, 0, 130], [64 * 5 + 3], [0, 65, 0]])
+def test_varlen_backward(io, d, lens):
+    """Gradients over packed documents (ragged, a one-token document, empty
+    documents), with per-document initial states and final-state gradients,
+    on the tensor-core (bf16, d=128) and CUDA-core (fp32, d=64) paths."""
+    T, H, N = int(sum(lens)), 2, len(lens)
+    inp = random_inputs(1, T, H, d, d, io, seed=T + d, gscale=0.05, extreme_p=0.05)
+    gen = torch.Generator().manual_seed(T + 7)
+    S0 = 0.1 * torch.randn(N, H, d, d, generator=gen)
+    dST = torch.randn(N, H, d, d, generator=gen)
+    cu = torch.tensor(np.concatenate([[0], np.cumsum(lens)]), dtype=torch.int32)
+    x = to_dev(inp)
+    got = api.varlen_bwd(x["q"], x["k"], x["v"], x["g"], x["sign"], x["beta"], x["dO"], cu.cuda(),
+                         max(max(lens), 1), S0=S0.cuda(), dST=dST.cuda())
+    torch.cuda.synchronize()
+    P = lambda t: f64(t[0])
+    ref = oracle.bwd(cu.numpy().astype(np.int64), P(inp["q"]), P(inp["k"]), P(inp["v"]), P(inp["g"]),
+                     inp["sign"][0].numpy(), P(inp["beta"]), P(inp["dO"]), S0=f64(S0), dST=f64(dST))
+    for key in ("dq", "dk", "dv", "dg", "dbeta"):
+        check(key, got[key][0], ref[key], io)
+    check("dS0", got["dS0"], ref["dS0"], io)
+
+
+def test_full_varlen_backward_sampled():
+    """The packed-document workload (65536 tokens, geometric document
+    lengths, H=16, d=128, bf16) through the backward, checked on sampled
+    documents and heads."""
+    w = W.VARLEN
+    inp = W.make_varlen(w)
+    d = to_dev(inp)
+    cu = inp["cu_seqlens"]
+    gen = torch.Generator().manual_seed(9)
+    dO = torch.randn(inp["q"].shape[:3] + (w.dv,), generator=gen).to(w.io_dtype)
+    got = api.varlen_bwd(d["q"], d["k"], d["v"], d["g"], d["sign"], d["beta"], dO.cuda(), cu.cuda(),
+                         max(inp["lens"]))
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(5)
+    for i in rng.choice(len(inp["lens"]), 3, replace=False):
+        a, b = int(cu[i]), int(cu[i + 1])
+        h = int(rng.integers(0, w.H))
+        sl = lambda x: f64(x[0, a:b, h:h + 1])
+        ref = oracle.bwd([0, b - a], sl(inp["q"]), sl(inp["k"]), sl(inp["v"]), sl(inp["g"]),
+                         inp["sign"][0, a:b, h:h + 1].numpy(), sl(inp["beta"]), sl(dO))
+        for key in ("dq", "dk", "dv", "dg", "dbeta"):
+            check("%s[doc %d]" % (key, i), got[key][0, a:b, h:h + 1], ref[key], w.io_dtype)
+        check("dS0[doc %d]" % i, got["dS0"][i:i + 1, h:h + 1], ref["dS0"], w.io_dtype)
