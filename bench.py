@@ -433,13 +433,16 @@ def run_secondary(args, rank, world, local_rank):
             gb = dict(dq=torch.empty_like(d["q"]), dk=torch.empty_like(d["k"]), dv=torch.empty_like(d["v"]),
                       dg=torch.empty_like(d["g"]), dbeta=torch.empty_like(d["beta"]))
             wsb = api.workspace(_abi.CKDA_OP_VARLEN_BWD, 1, T, H, dk, dv, Nd, device=dev, cache=False)
-            fwd_step = step
+            # the forward hands its per-chunk results to the backward (as in the headline step)
+            n_sv = _abi.ckda_varlen_saved_size(T, Nd, H, dk, dv, code)
+            sv = torch.empty(n_sv, dtype=torch.uint8, device=dev) if n_sv > 0 else None
 
             def step():
-                fwd_step()
+                _abi.ckda_varlen_fwd(T, Nd, cu, mx, H, dk, dv, code, d["q"], d["k"], d["v"], d["g"],
+                                     d["sign"], d["beta"], None, o, ST, ws, saved=sv)
                 _abi.ckda_varlen_bwd(T, Nd, cu, mx, H, dk, dv, code, d["q"], d["k"], d["v"], d["g"],
                                      d["sign"], d["beta"], None, dO, None, gb["dq"], gb["dk"], gb["dv"],
-                                     gb["dg"], gb["dbeta"], None, wsb)
+                                     gb["dg"], gb["dbeta"], None, wsb, saved=sv)
             per_unit, unit_name = FWD_BYTES + BWD_BYTES, "B per token-head (fwd + bwd)"
             kernel_bytes = {"tc_grad": BWD_BYTES, "tc_intra": FWD_BYTES}
             metric = "CKDA varlen fwd+bwd tokens/s (65536 packed tokens,H=16,d=128,bf16)"

@@ -57,8 +57,10 @@ def _load():
         F = ctypes.c_float
         lib.ckda_prologue_fwd.argtypes = [I] * 6 + [P] * 8 + [F] + [P] * 7
         lib.ckda_prologue_bwd.argtypes = [I] * 6 + [P] * 8 + [F] + [P] * 14
-        lib.ckda_varlen_fwd.argtypes = [I, I, P, I, I, I, I, I] + [P] * 10 + [Z, P]
-        lib.ckda_varlen_bwd.argtypes = [I, I, P, I, I, I, I, I] + [P] * 16 + [Z, P]
+        lib.ckda_varlen_fwd.argtypes = [I, I, P, I, I, I, I, I] + [P] * 9 + [P, Z] + [P, Z, P]
+        lib.ckda_varlen_bwd.argtypes = [I, I, P, I, I, I, I, I] + [P] * 9 + [P, Z] + [P] * 7 + [Z, P]
+        lib.ckda_varlen_saved_size.argtypes = [I] * 6
+        lib.ckda_varlen_saved_size.restype = Z
         lib.ckda_chunk_fwd_noalloc.argtypes = [I] * 6 + [P] * 11
         lib.ckda_check_device_status.argtypes = [P, P]
         lib.ckda_status_string.argtypes = [I]
@@ -157,9 +159,11 @@ def ckda_decode_multi(N, K, H, dk, dv, io_dtype, q, k, v, g, sign, beta, n_token
 
 
 def ckda_varlen_bwd(total_T, N, cu_seqlens, max_seqlen, H, dk, dv, io_dtype, q, k, v, g, sign, beta, S0, dO,
-                    dST, dq, dk_out, dv_out, dg, dbeta, dS0, ws, ws_bytes=None, stream=None):
+                    dST, dq, dk_out, dv_out, dg, dbeta, dS0, ws, ws_bytes=None, stream=None, saved=None,
+                    saved_bytes=None):
     _check(_load().ckda_varlen_bwd(total_T, N, _p(cu_seqlens), max_seqlen, H, dk, dv, io_dtype, _p(q), _p(k),
-                                   _p(v), _p(g), _p(sign), _p(beta), _p(S0), _p(dO), _p(dST), _p(dq), _p(dk_out),
+                                   _p(v), _p(g), _p(sign), _p(beta), _p(S0), _p(dO), _p(dST), _p(saved),
+                                   _nbytes(saved, saved_bytes), _p(dq), _p(dk_out),
                                    _p(dv_out), _p(dg), _p(dbeta), _p(dS0), _p(ws), _nbytes(ws, ws_bytes),
                                    _s(stream)), "ckda_varlen_bwd")
 
@@ -180,11 +184,16 @@ def ckda_prologue_bwd(B, T, H, dk, dv, io_dtype, xq, xk, xv, wq, wk, wv, a, b, g
 
 
 def ckda_varlen_fwd(total_T, N, cu_seqlens, max_seqlen, H, dk, dv, io_dtype, q, k, v, g, sign,
-                    beta, S0, o, ST, ws, ws_bytes=None, stream=None):
+                    beta, S0, o, ST, ws, ws_bytes=None, stream=None, saved=None, saved_bytes=None):
     _check(_load().ckda_varlen_fwd(total_T, N, _p(cu_seqlens), max_seqlen, H, dk, dv, io_dtype,
                                    _p(q), _p(k), _p(v), _p(g), _p(sign), _p(beta), _p(S0), _p(o),
-                                   _p(ST), _p(ws), _nbytes(ws, ws_bytes), _s(stream)),
+                                   _p(ST), _p(saved), _nbytes(saved, saved_bytes), _p(ws),
+                                   _nbytes(ws, ws_bytes), _s(stream)),
            "ckda_varlen_fwd")
+
+
+def ckda_varlen_saved_size(total_T, N, H, dk, dv, io_dtype):
+    return int(_load().ckda_varlen_saved_size(total_T, N, H, dk, dv, io_dtype))
 
 
 def ckda_chunk_fwd_noalloc(B, T, H, dk, dv, io_dtype, q, k, v, g, sign, beta, S0, o, ST,

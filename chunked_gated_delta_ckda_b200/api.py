@@ -237,7 +237,10 @@ def prologue_bwd(xq, xk, xv, wq, wk, wv, a, b, dq, dk, dv, dg, dbeta, g_floor=-5
 
 
 def varlen_fwd(q, k, v, g, sign, beta, cu_seqlens, max_seqlen, S0=None, output_final_state=True,
-               ws=None):
+               ws=None, save_for_backward=False):
+    """Packed documents: o [1,T,H,dv], ST [N,H,dk,dv] (or None); with
+    save_for_backward also the saved buffer for varlen_bwd (None where the
+    configuration has no saved form)."""
     if q.dim() != 4 or q.shape[0] != 1:
         raise ValueError("packed q must have shape (1, total_T, H, dk), got %s" % (tuple(q.shape),))
     T = q.shape[1]
@@ -251,13 +254,22 @@ def varlen_fwd(q, k, v, g, sign, beta, cu_seqlens, max_seqlen, S0=None, output_f
     ST = torch.empty(N, H, dk, dv, dtype=torch.float32, device=q.device) if output_final_state else None
     if ws is None:
         ws = workspace(CKDA_OP_VARLEN_FWD, 1, T, H, dk, dv, N, device=q.device)
+    sv = None
+    if save_for_backward:
+        n = _abi.ckda_varlen_saved_size(T, N, H, dk, dv, io_code(q.dtype))
+        sv = torch.empty(n, dtype=torch.uint8, device=q.device) if n > 0 else None
     _abi.ckda_varlen_fwd(T, N, cu_seqlens, int(max_seqlen), H, dk, dv, io_code(q.dtype), q, k, v,
-                         g, sign, beta, S0, o, ST, ws)
+                         g, sign, beta, S0, o, ST, ws, saved=sv)
+    if save_for_backward:
+        return o, ST, sv
     return o, ST
 
 
-def varlen_bwd(q, k, v, g, sign, beta, dO, cu_seqlens, max_seqlen, S0=None, dST=None, need_dS0=True, ws=None):
-    """Gradients of varlen_fwd: dict dq, dk, dv, dg, dbeta, dS0 ([N,H,dk,dv] or None)."""
+def varlen_bwd(q, k, v, g, sign, beta, dO, cu_seqlens, max_seqlen, S0=None, dST=None, need_dS0=True, ws=None,
+               saved=None):
+    """Gradients of varlen_fwd: dict dq, dk, dv, dg, dbeta, dS0 ([N,H,dk,dv] or
+    None).  saved: the buffer varlen_fwd(save_for_backward=True) returned for
+    the same inputs (else the per-chunk results are recomputed)."""
     if q.dim() != 4 or q.shape[0] != 1:
         raise ValueError("packed q must have shape (1, total_T, H, dk), got %s" % (tuple(q.shape),))
     T = q.shape[1]
@@ -268,13 +280,16 @@ def varlen_bwd(q, k, v, g, sign, beta, dO, cu_seqlens, max_seqlen, S0=None, dST=
     _expect("dO", dO, (1, T, H, dv), q.dtype)
     _expect("S0", S0, (N, H, dk, dv), torch.float32, optional=True)
     _expect("dST", dST, (N, H, dk, dv), torch.float32, optional=True)
-    q, k, v, g, sign, beta, dO, S0, dST, cu_seqlens = map(
-        _c, (q, k, v, g, sign, beta, dO, S0, dST, cu_seqlens))
+    if saved is not None and saved.dtype != torch.uint8:
+        raise TypeError("saved must be the uint8 buffer varlen_fwd returned")
+    q, k, v, g, sign, beta, dO, S0, dST, cu_seqlens, saved = map(
+        _c, (q, k, v, g, sign, beta, dO, S0, dST, cu_seqlens, saved))
     out = dict(dq=torch.empty_like(q), dk=torch.empty_like(k), dv=torch.empty_like(v), dg=torch.empty_like(g),
                dbeta=torch.empty_like(beta),
                dS0=torch.empty(N, H, dk, dv, dtype=torch.float32, device=q.device) if need_dS0 else None)
     if ws is None:
         ws = workspace(CKDA_OP_VARLEN_BWD, 1, T, H, dk, dv, N, device=q.device)
     _abi.ckda_varlen_bwd(T, N, cu_seqlens, int(max_seqlen), H, dk, dv, io_code(q.dtype), q, k, v, g, sign, beta,
-                         S0, dO, dST, out["dq"], out["dk"], out["dv"], out["dg"], out["dbeta"], out["dS0"], ws)
+                         S0, dO, dST, out["dq"], out["dk"], out["dv"], out["dg"], out["dbeta"], out["dS0"], ws,
+                         saved=saved)
     return out

@@ -117,6 +117,12 @@ size_t saved_bytes_for(int B, int T, int H, int dk, int dv, int io_dtype) {
   return (size_t)nch * H * tc_record_bytes();
 }
 
+// packed documents: one record per (chunk, head) of the chunk bound
+size_t packed_saved_bytes_for(int total_T, int N, int H, int dk, int dv, int io_dtype) {
+  if (!use_tensor_cores(io_dtype, dk, dv) || total_T <= 0) return 0;
+  return (size_t)ws_layout(CKDA_OP_VARLEN_FWD, 1, total_T, H, dk, dv, N).n_chunks_bound * H * tc_record_bytes();
+}
+
 #define CKDA_TRY(expr)                          \
   do {                                          \
     int _rc = (expr);                           \
@@ -140,6 +146,11 @@ size_t ckda_workspace_size(int op, int B, int T, int H, int dk, int dv, int N) {
 size_t ckda_saved_size(int B, int T, int H, int dk, int dv, int io_dtype) {
   if (check_common(B, T, H, dk, dv, io_dtype) != CKDA_OK) return 0;
   return saved_bytes_for(B, T, H, dk, dv, io_dtype);
+}
+
+size_t ckda_varlen_saved_size(int total_T, int N, int H, int dk, int dv, int io_dtype) {
+  if (check_common(1, total_T, H, dk, dv, io_dtype) != CKDA_OK || N < 0) return 0;
+  return packed_saved_bytes_for(total_T, N, H, dk, dv, io_dtype);
 }
 
 int ckda_chunk_fwd(int B, int T, int H, int dk, int dv, int io_dtype, const void *q,
@@ -330,7 +341,8 @@ int ckda_prologue_bwd(int B, int T, int H, int dk, int dv, int io_dtype, const v
 int ckda_varlen_fwd(int total_T, int N, const int32_t *cu_seqlens, int max_seqlen, int H,
                     int dk, int dv, int io_dtype, const void *q, const void *k, const void *v,
                     const float *g, const int8_t *sign, const void *beta, const float *S0,
-                    void *o, float *ST, void *ws, size_t ws_bytes, cudaStream_t stream) {
+                    void *o, float *ST, void *saved, size_t saved_bytes, void *ws, size_t ws_bytes,
+                    cudaStream_t stream) {
   CKDA_TRY(check_common(1, total_T, H, dk, dv, io_dtype));
   if (N < 0) return CKDA_ERR_INVALID_ARG;
   if (N == 0) return total_T == 0 ? CKDA_OK : CKDA_ERR_INVALID_ARG;
@@ -339,6 +351,14 @@ int ckda_varlen_fwd(int total_T, int N, const int32_t *cu_seqlens, int max_seqle
   if (total_T > 0) CKDA_TRY(check_ptrs({q, k, v, g, beta, o}, {sign, S0, ST}));
   else CKDA_TRY(check_ptrs({}, {sign, S0, ST}));
   if ((reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) != 0) return CKDA_ERR_ALIGNMENT;
+  unsigned char *recs_out = nullptr;  // the records for ckda_varlen_bwd, if asked for
+  {
+    const size_t need = packed_saved_bytes_for(total_T, N, H, dk, dv, io_dtype);
+    if (saved && need > 0) {
+      CKDA_TRY(check_ws(saved, saved_bytes, need));
+      recs_out = static_cast<unsigned char *>(saved);
+    }
+  }
   const WsLayout L = ws_layout(CKDA_OP_VARLEN_FWD, 1, total_T, H, dk, dv, N);
   CKDA_TRY(check_ws(ws, ws_bytes, L.total));
   char *w = static_cast<char *>(ws);
@@ -362,8 +382,9 @@ int ckda_varlen_fwd(int total_T, int N, const int32_t *cu_seqlens, int max_seqle
                               reinterpret_cast<DevStatus *>(w), stream));
   const bool bf16 = io_dtype == CKDA_BF16;
   if (use_tensor_cores(io_dtype, dk, dv)) {
-    CKDA_CUDA(tc_forward(a, reinterpret_cast<unsigned char *>(w + L.intra),
-                         reinterpret_cast<float *>(w + L.fscratch), true, nullptr, stream));
+    CKDA_CUDA(tc_forward(a, recs_out ? recs_out : reinterpret_cast<unsigned char *>(w + L.intra),
+                         reinterpret_cast<float *>(w + L.fscratch), true, nullptr, stream,
+                         /*state_pass=*/true, /*intra_pass=*/true, /*state_tiles=*/recs_out != nullptr));
     return CKDA_OK;
   }
   CKDA_CUDA(v1_intra(a, bf16, reinterpret_cast<float *>(w + L.fscratch), stream));
@@ -374,8 +395,8 @@ int ckda_varlen_fwd(int total_T, int N, const int32_t *cu_seqlens, int max_seqle
 int ckda_varlen_bwd(int total_T, int N, const int32_t *cu_seqlens, int max_seqlen, int H, int dk, int dv,
                     int io_dtype, const void *q, const void *k, const void *v, const float *g,
                     const int8_t *sign, const void *beta, const float *S0, const void *dO, const float *dST,
-                    void *dq, void *dk_out, void *dv_out, float *dg, void *dbeta, float *dS0, void *ws,
-                    size_t ws_bytes, cudaStream_t stream) {
+                    const void *saved, size_t saved_bytes, void *dq, void *dk_out, void *dv_out, float *dg,
+                    void *dbeta, float *dS0, void *ws, size_t ws_bytes, cudaStream_t stream) {
   CKDA_TRY(check_common(1, total_T, H, dk, dv, io_dtype));
   if (N < 0) return CKDA_ERR_INVALID_ARG;
   if (N == 0) return total_T == 0 ? CKDA_OK : CKDA_ERR_INVALID_ARG;
@@ -386,6 +407,14 @@ int ckda_varlen_bwd(int total_T, int N, const int32_t *cu_seqlens, int max_seqle
   else
     CKDA_TRY(check_ptrs({}, {sign, S0, dST, dS0}));
   if ((reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) != 0) return CKDA_ERR_ALIGNMENT;
+  const unsigned char *recs_in = nullptr;  // the forward's records, if handed over
+  {
+    const size_t need = packed_saved_bytes_for(total_T, N, H, dk, dv, io_dtype);
+    if (saved && need > 0) {
+      CKDA_TRY(check_ws(saved, saved_bytes, need));
+      recs_in = static_cast<const unsigned char *>(saved);
+    }
+  }
   const WsLayout L = ws_layout(CKDA_OP_VARLEN_BWD, 1, total_T, H, dk, dv, N);
   CKDA_TRY(check_ws(ws, ws_bytes, L.total));
   char *w = static_cast<char *>(ws);
@@ -408,11 +437,11 @@ int ckda_varlen_bwd(int total_T, int N, const int32_t *cu_seqlens, int max_seqle
   const bool bf16 = io_dtype == CKDA_BF16;
   const bool tcp = use_tensor_cores(io_dtype, dk, dv);
   const float *states = nullptr;
-  unsigned char *recs = reinterpret_cast<unsigned char *>(w + L.intra);
-  if (tcp) {  // records with their bf16 chunk-start states, recomputed
-    CKDA_CUDA(tc_forward(f, recs, reinterpret_cast<float *>(w + L.fscratch), false, nullptr, stream,
-                         /*state_pass=*/true, /*intra_pass=*/true, /*state_tiles=*/true, nullptr));
-  } else {
+  const unsigned char *recs = recs_in ? recs_in : reinterpret_cast<const unsigned char *>(w + L.intra);
+  if (tcp && !recs_in) {  // records with their bf16 chunk-start states, recomputed
+    CKDA_CUDA(tc_forward(f, const_cast<unsigned char *>(recs), reinterpret_cast<float *>(w + L.fscratch), false,
+                         nullptr, stream, /*state_pass=*/true, /*intra_pass=*/true, /*state_tiles=*/true, nullptr));
+  } else if (!tcp) {
     CKDA_CUDA(v1_intra(f, bf16, reinterpret_cast<float *>(w + L.fscratch), stream));
     float *st = reinterpret_cast<float *>(w + L.states);
     CKDA_CUDA(v1_state_fwd(f, bf16, false, st, stream));

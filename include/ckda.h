@@ -234,6 +234,9 @@ int ckda_prologue_bwd(int B, int T, int H, int dk, int dv, int io_dtype,
  *         a document longer than it is reported as CKDA_ERR_DEVICE_ARG
  *   q, k [1,total_T,H,dk] ... as ckda_chunk_fwd with B = 1, T = total_T
  *   S0, ST [N,H,dk,dv] f32, nullable: per-document initial / final states
+ *   saved, saved_bytes: nullable; when ckda_varlen_saved_size(...) > 0, a
+ *         256-byte aligned buffer of at least that many bytes that receives
+ *         the per-chunk results for ckda_varlen_bwd (as for ckda_chunk_fwd)
  * Chunks restart at each document start; a document's last chunk may be
  * partial.  Malformed cu_seqlens are detected on the device
  * (CKDA_ERR_DEVICE_ARG via ckda_check_device_status; no output is written). */
@@ -241,24 +244,34 @@ int ckda_varlen_fwd(int total_T, int N, const int32_t *cu_seqlens,
                     int max_seqlen, int H, int dk, int dv, int io_dtype,
                     const void *q, const void *k, const void *v, const float *g,
                     const int8_t *sign, const void *beta, const float *S0,
-                    void *o, float *ST, void *ws, size_t ws_bytes,
-                    cudaStream_t stream);
+                    void *o, float *ST, void *saved, size_t saved_bytes,
+                    void *ws, size_t ws_bytes, cudaStream_t stream);
+
+/* Bytes of the packed forward's saved buffer (0: no saved form for this
+ * configuration, or invalid arguments); the packed counterpart of
+ * ckda_saved_size. */
+size_t ckda_varlen_saved_size(int total_T, int N, int H, int dk, int dv,
+                              int io_dtype);
 
 /* Backward of ckda_varlen_fwd: gradients over N packed documents (training
  * on packed documents).  Arguments as ckda_varlen_fwd plus
  *   dO [1,total_T,H,dv] io;  dST [N,H,dk,dv] f32, nullable: per-document
- *   gradient of the final states;  dq, dk_out [1,total_T,H,dk] io;
+ *   gradient of the final states;  saved, saved_bytes: nullable, the buffer
+ *   ckda_varlen_fwd filled for the same inputs (and the same cu_seqlens and
+ *   max_seqlen), else the per-chunk results are recomputed in ws;
+ *   dq, dk_out [1,total_T,H,dk] io;
  *   dv_out [1,total_T,H,dv] io;  dg [1,total_T,H,dk] f32;  dbeta
  *   [1,total_T,H] io;  dS0 [N,H,dk,dv] f32, nullable.
- * The per-chunk forward results are recomputed in the workspace
- * (ckda_workspace_size(CKDA_OP_VARLEN_BWD, 1, total_T, H, dk, dv, N) bytes).
+ * Workspace: ckda_workspace_size(CKDA_OP_VARLEN_BWD, 1, total_T, H, dk, dv,
+ * N) bytes.
  * Malformed cu_seqlens are reported as for the forward. */
 int ckda_varlen_bwd(int total_T, int N, const int32_t *cu_seqlens,
                     int max_seqlen, int H, int dk, int dv, int io_dtype,
                     const void *q, const void *k, const void *v, const float *g,
                     const int8_t *sign, const void *beta, const float *S0,
-                    const void *dO, const float *dST, void *dq, void *dk_out,
-                    void *dv_out, float *dg, void *dbeta, float *dS0, void *ws,
+                    const void *dO, const float *dST, const void *saved,
+                    size_t saved_bytes, void *dq, void *dk_out, void *dv_out,
+                    float *dg, void *dbeta, float *dS0, void *ws,
                     size_t ws_bytes, cudaStream_t stream);
 
 /* ---- chunked forward without any allocation --------------------------------

@@ -90,9 +90,12 @@ def test_host_validation_without_gpu():
     assert lib.ckda_decode_step(4, 2, 64, 64, 0, *([None] * 8), None) == 1
     # packed: bad max_seqlen, N < 0
     v = [fake] * 9
-    assert lib.ckda_varlen_fwd(100, 2, fake, 0, 2, 64, 64, 0, *v, fake, 1 << 30, None) == 1
-    assert lib.ckda_varlen_fwd(100, -1, fake, 50, 2, 64, 64, 0, *v, fake, 1 << 30, None) == 1
-    vb = [fake] * 15
+    assert lib.ckda_varlen_fwd(100, 2, fake, 0, 2, 64, 64, 0, *v, None, 0, fake, 1 << 30, None) == 1
+    assert lib.ckda_varlen_fwd(100, -1, fake, 50, 2, 64, 64, 0, *v, None, 0, fake, 1 << 30, None) == 1
+    need = lib.ckda_varlen_saved_size(100, 2, 2, 128, 128, 1)
+    assert need > 0 and lib.ckda_varlen_saved_size(100, 2, 2, 64, 64, 0) == 0
+    assert lib.ckda_varlen_fwd(100, 2, fake, 50, 2, 128, 128, 1, *v, fake, need - 1, fake, 1 << 30, None) == 4
+    vb = [fake] * 9 + [None, 0] + [fake] * 6
     assert lib.ckda_varlen_bwd(100, 2, fake, 0, 2, 64, 64, 0, *vb, fake, 1 << 30, None) == 1   # max_seqlen
     assert lib.ckda_varlen_bwd(100, 2, None, 50, 2, 64, 64, 0, *vb, fake, 1 << 30, None) == 1  # cu_seqlens
     assert lib.ckda_varlen_bwd(100, 2, fake, 50, 2, 64, 64, 0, *vb, fake, 16, None) == 4       # workspace

@@ -662,6 +662,34 @@ def test_varlen_backward(io, d, lens):
     check("dS0", got["dS0"], ref["dS0"], io)
 
 
+def test_varlen_backward_with_saved_forward_results():
+    """The packed forward's saved per-chunk results stand in for the packed
+    backward's recomputation: bit-identical gradients, and the oracle's."""
+    io, H, d = torch.bfloat16, 2, 128
+    lens = [150, 0, 64, 77]
+    T, N = int(sum(lens)), len(lens)
+    inp = random_inputs(1, T, H, d, d, io, seed=71, gscale=0.3, extreme_p=0.05)
+    gen = torch.Generator().manual_seed(72)
+    S0 = (0.1 * torch.randn(N, H, d, d, generator=gen)).cuda()
+    dST = torch.randn(N, H, d, d, generator=gen).cuda()
+    cu = torch.tensor(np.concatenate([[0], np.cumsum(lens)]), dtype=torch.int32).cuda()
+    x = to_dev(inp)
+    args = (x["q"], x["k"], x["v"], x["g"], x["sign"], x["beta"])
+    o, ST, sv = api.varlen_fwd(*args, cu, max(lens), S0=S0, save_for_backward=True)
+    assert sv is not None and sv.numel() == _abi.ckda_varlen_saved_size(T, N, H, d, d, _abi.CKDA_BF16)
+    a = api.varlen_bwd(*args, x["dO"], cu, max(lens), S0=S0, dST=dST, saved=sv)
+    b = api.varlen_bwd(*args, x["dO"], cu, max(lens), S0=S0, dST=dST)
+    torch.cuda.synchronize()
+    for key in a:
+        assert torch.equal(a[key], b[key]), key
+    P = lambda t: f64(t[0])
+    ref = oracle.bwd(cu.cpu().numpy().astype(np.int64), P(inp["q"]), P(inp["k"]), P(inp["v"]), P(inp["g"]),
+                     inp["sign"][0].numpy(), P(inp["beta"]), P(inp["dO"]), S0=f64(S0.cpu()), dST=f64(dST.cpu()))
+    for key in ("dq", "dk", "dv", "dg", "dbeta"):
+        check(key, a[key][0], ref[key], io)
+    check("dS0", a["dS0"], ref["dS0"], io)
+
+
 def test_full_varlen_backward_sampled():
     """The packed-document workload (65536 tokens, geometric document
     lengths, H=16, d=128, bf16) through the backward, checked on sampled
