@@ -9,7 +9,9 @@ torch (device memory is torch's job here) and call the library.
     o         = decode_multi(q, k, v, g, sign, beta, pool, slots=None, n_tokens=None,
                              write_state=True)                 # K tokens per sequence
     o, ST     = varlen_fwd(q, k, v, g, sign, beta, cu_seqlens, max_seqlen, S0=None)
-    grads     = varlen_bwd(q, k, v, g, sign, beta, dO, cu_seqlens, max_seqlen, S0=None, dST=None)
+    o, ST, sv = varlen_fwd(..., save_for_backward=True)
+    grads     = varlen_bwd(q, k, v, g, sign, beta, dO, cu_seqlens, max_seqlen, S0=None, dST=None,
+                           saved=sv)                           # packed documents
     x         = prologue_fwd(xq, xk, xv, wq, wk, wv, a, b, g_floor=-5.0)   # q, k, v, g, sign, beta
     grads     = prologue_bwd(xq, xk, xv, wq, wk, wv, a, b, dq, dk, dv, dg, dbeta, g_floor=-5.0)
 
