@@ -55,8 +55,8 @@ def _load():
         lib.ckda_decode_step.argtypes = [I] * 5 + [P] * 9
         lib.ckda_decode_multi.argtypes = [I] * 6 + [P] * 8 + [I, P, I, P, P]
         F = ctypes.c_float
-        lib.ckda_prologue_fwd.argtypes = [I] * 6 + [P] * 8 + [F] + [P] * 7
-        lib.ckda_prologue_bwd.argtypes = [I] * 6 + [P] * 8 + [F] + [P] * 14
+        lib.ckda_prologue_fwd.argtypes = [I] * 6 + [P] * 8 + [F, P, I] + [P] * 7
+        lib.ckda_prologue_bwd.argtypes = [I] * 6 + [P] * 8 + [F, P, I] + [P] * 14
         lib.ckda_varlen_fwd.argtypes = [I, I, P, I, I, I, I, I] + [P] * 9 + [P, Z] + [P, Z, P]
         lib.ckda_varlen_bwd.argtypes = [I, I, P, I, I, I, I, I] + [P] * 9 + [P, Z] + [P] * 7 + [Z, P]
         lib.ckda_varlen_saved_size.argtypes = [I] * 6
@@ -169,16 +169,16 @@ def ckda_varlen_bwd(total_T, N, cu_seqlens, max_seqlen, H, dk, dv, io_dtype, q, 
 
 
 def ckda_prologue_fwd(B, T, H, dk, dv, io_dtype, xq, xk, xv, wq, wk, wv, a, b, g_floor, q, k, v, g, sign, beta,
-                      stream=None):
+                      stream=None, cu_seqlens=None, N=0):
     _check(_load().ckda_prologue_fwd(B, T, H, dk, dv, io_dtype, _p(xq), _p(xk), _p(xv), _p(wq), _p(wk), _p(wv),
-                                     _p(a), _p(b), float(g_floor), _p(q), _p(k), _p(v), _p(g), _p(sign), _p(beta),
+                                     _p(a), _p(b), float(g_floor), _p(cu_seqlens), int(N), _p(q), _p(k), _p(v), _p(g), _p(sign), _p(beta),
                                      _s(stream)), "ckda_prologue_fwd")
 
 
 def ckda_prologue_bwd(B, T, H, dk, dv, io_dtype, xq, xk, xv, wq, wk, wv, a, b, g_floor, dq, dk_in, dv_in, dg, dbeta,
-                      dxq, dxk, dxv, dwq, dwk, dwv, da, db, stream=None):
+                      dxq, dxk, dxv, dwq, dwk, dwv, da, db, stream=None, cu_seqlens=None, N=0):
     _check(_load().ckda_prologue_bwd(B, T, H, dk, dv, io_dtype, _p(xq), _p(xk), _p(xv), _p(wq), _p(wk), _p(wv),
-                                     _p(a), _p(b), float(g_floor), _p(dq), _p(dk_in), _p(dv_in), _p(dg), _p(dbeta),
+                                     _p(a), _p(b), float(g_floor), _p(cu_seqlens), int(N), _p(dq), _p(dk_in), _p(dv_in), _p(dg), _p(dbeta),
                                      _p(dxq), _p(dxk), _p(dxv), _p(dwq), _p(dwk), _p(dwv), _p(da), _p(db),
                                      _s(stream)), "ckda_prologue_bwd")
 

@@ -205,23 +205,40 @@ def _prologue_shapes(xq, xk, xv, wq, wk, wv, a, b):
     return B, T, H, dk, dv
 
 
-def prologue_fwd(xq, xk, xv, wq, wk, wv, a, b, g_floor=-5.0):
+def _prologue_docs(B, cu_seqlens):
+    """Packed documents' offsets for the prologue: (tensor, N), or (None, 0)."""
+    if cu_seqlens is None:
+        return None, 0
+    if cu_seqlens.dim() != 1 or cu_seqlens.dtype != torch.int32 or cu_seqlens.numel() < 2:
+        raise TypeError("cu_seqlens must be a 1-D int32 tensor of N + 1 >= 2 offsets")
+    if B != 1:
+        raise ValueError("packed documents (cu_seqlens) take a batch of one row, got B=%d" % B)
+    return _c(cu_seqlens), cu_seqlens.numel() - 1
+
+
+def prologue_fwd(xq, xk, xv, wq, wk, wv, a, b, g_floor=-5.0, cu_seqlens=None):
     """Projections [B,T,H,d] (io dtype), conv taps [H*d, 4] fp32, gate
     pre-activation a [B,T,H,dk] fp32, b [B,T,H] -> dict q, k, v, g, sign, beta
-    (the inputs of chunk_fwd)."""
+    (the inputs of chunk_fwd).  With cu_seqlens (int32 [N+1], B = 1) the
+    convolution's history restarts at each packed document's first token
+    (the inputs of varlen_fwd)."""
     B, T, H, dk, dv = _prologue_shapes(xq, xk, xv, wq, wk, wv, a, b)
+    cu, N = _prologue_docs(B, cu_seqlens)
     xq, xk, xv, wq, wk, wv, a, b = map(_c, (xq, xk, xv, wq, wk, wv, a, b))
     out = dict(q=torch.empty_like(xq), k=torch.empty_like(xk), v=torch.empty_like(xv),
                g=torch.empty(B, T, H, dk, dtype=torch.float32, device=xq.device),
                sign=torch.empty(B, T, H, dk, dtype=torch.int8, device=xq.device), beta=torch.empty_like(b))
     _abi.ckda_prologue_fwd(B, T, H, dk, dv, io_code(xq.dtype), xq, xk, xv, wq, wk, wv, a, b, g_floor,
-                           out["q"], out["k"], out["v"], out["g"], out["sign"], out["beta"])
+                           out["q"], out["k"], out["v"], out["g"], out["sign"], out["beta"],
+                           cu_seqlens=cu, N=N)
     return out
 
 
-def prologue_bwd(xq, xk, xv, wq, wk, wv, a, b, dq, dk, dv, dg, dbeta, g_floor=-5.0):
-    """Gradients of prologue_fwd's inputs: dict dxq, dxk, dxv, dwq, dwk, dwv, da, db."""
+def prologue_bwd(xq, xk, xv, wq, wk, wv, a, b, dq, dk, dv, dg, dbeta, g_floor=-5.0, cu_seqlens=None):
+    """Gradients of prologue_fwd's inputs (same g_floor and cu_seqlens):
+    dict dxq, dxk, dxv, dwq, dwk, dwv, da, db."""
     B, T, H, dk_, dv_ = _prologue_shapes(xq, xk, xv, wq, wk, wv, a, b)
+    cu, N = _prologue_docs(B, cu_seqlens)
     _expect("dq", dq, (B, T, H, dk_), xq.dtype)
     _expect("dk", dk, (B, T, H, dk_), xq.dtype)
     _expect("dv", dv, (B, T, H, dv_), xq.dtype)
@@ -234,7 +251,7 @@ def prologue_bwd(xq, xk, xv, wq, wk, wv, a, b, dq, dk, dv, dg, dbeta, g_floor=-5
                da=torch.empty_like(a), db=torch.empty_like(b))
     _abi.ckda_prologue_bwd(B, T, H, dk_, dv_, io_code(xq.dtype), xq, xk, xv, wq, wk, wv, a, b, g_floor,
                            dq, dk, dv, dg, dbeta, out["dxq"], out["dxk"], out["dxv"], out["dwq"], out["dwk"],
-                           out["dwv"], out["da"], out["db"])
+                           out["dwv"], out["da"], out["db"], cu_seqlens=cu, N=N)
     return out
 
 

@@ -293,18 +293,23 @@ int ckda_decode_multi(int N, int K, int H, int dk, int dv, int io_dtype, const v
                                   slots, n_slots, state, write_state == 1, o, stream));
 }
 
-static int prologue_common(int B, int T, int H, int dk, int dv, int io_dtype, float g_floor) {
+static int prologue_common(int B, int T, int H, int dk, int dv, int io_dtype, float g_floor,
+                           const int32_t *cu_seqlens, int N) {
   CKDA_TRY(check_common(B, T, H, dk, dv, io_dtype));
   if (!(g_floor <= 0.f) || !isfinite(g_floor)) return CKDA_ERR_INVALID_ARG;
+  if (cu_seqlens) {
+    if (B != 1 || N < 1) return CKDA_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) != 0) return CKDA_ERR_ALIGNMENT;
+  }
   if (B > 65535 || H > 65535) return CKDA_ERR_UNSUPPORTED;
   return CKDA_OK;
 }
 
 int ckda_prologue_fwd(int B, int T, int H, int dk, int dv, int io_dtype, const void *xq, const void *xk,
                       const void *xv, const float *wq, const float *wk, const float *wv, const float *a,
-                      const void *b, float g_floor, void *q, void *k, void *v, float *g, int8_t *sign,
-                      void *beta, cudaStream_t stream) {
-  CKDA_TRY(prologue_common(B, T, H, dk, dv, io_dtype, g_floor));
+                      const void *b, float g_floor, const int32_t *cu_seqlens, int N, void *q, void *k,
+                      void *v, float *g, int8_t *sign, void *beta, cudaStream_t stream) {
+  CKDA_TRY(prologue_common(B, T, H, dk, dv, io_dtype, g_floor, cu_seqlens, N));
   if ((int64_t)B * T == 0) return CKDA_OK;
   CKDA_TRY(check_ptrs({xq, xk, xv, wq, wk, wv, a, b, q, k, v, g, sign, beta}, {}));
   PrologueLaunch p{};
@@ -312,15 +317,17 @@ int ckda_prologue_fwd(int B, int T, int H, int dk, int dv, int io_dtype, const v
   p.g_floor = g_floor;
   p.xq = xq; p.xk = xk; p.xv = xv; p.b = b; p.wq = wq; p.wk = wk; p.wv = wv; p.a = a;
   p.q = q; p.k = k; p.v = v; p.g = g; p.sign = sign; p.beta = beta;
+  p.cu = cu_seqlens; p.N = N;
   return cuda_status(prologue(p, stream));
 }
 
 int ckda_prologue_bwd(int B, int T, int H, int dk, int dv, int io_dtype, const void *xq, const void *xk,
                       const void *xv, const float *wq, const float *wk, const float *wv, const float *a,
-                      const void *b, float g_floor, const void *dq, const void *dk_in, const void *dv_in,
-                      const float *dg, const void *dbeta, void *dxq, void *dxk, void *dxv, float *dwq,
-                      float *dwk, float *dwv, float *da, void *db, cudaStream_t stream) {
-  CKDA_TRY(prologue_common(B, T, H, dk, dv, io_dtype, g_floor));
+                      const void *b, float g_floor, const int32_t *cu_seqlens, int N, const void *dq,
+                      const void *dk_in, const void *dv_in, const float *dg, const void *dbeta, void *dxq,
+                      void *dxk, void *dxv, float *dwq, float *dwk, float *dwv, float *da, void *db,
+                      cudaStream_t stream) {
+  CKDA_TRY(prologue_common(B, T, H, dk, dv, io_dtype, g_floor, cu_seqlens, N));
   CKDA_TRY(check_ptrs({wq, wk, wv, dwq, dwk, dwv}, {}));
   if ((int64_t)B * T > 0)
     CKDA_TRY(check_ptrs({xq, xk, xv, a, b, dq, dk_in, dv_in, dg, dbeta, dxq, dxk, dxv, da, db}, {}));
@@ -335,6 +342,7 @@ int ckda_prologue_bwd(int B, int T, int H, int dk, int dv, int io_dtype, const v
   p.xq = xq; p.xk = xk; p.xv = xv; p.b = b; p.wq = wq; p.wk = wk; p.wv = wv; p.a = a;
   p.dq = dq; p.dk_in = dk_in; p.dv_in = dv_in; p.dg = dg; p.dbeta = dbeta;
   p.dxq = dxq; p.dxk = dxk; p.dxv = dxv; p.db = db; p.dwq = dwq; p.dwk = dwk; p.dwv = dwv; p.da = da;
+  p.cu = cu_seqlens; p.N = N;
   return cuda_status(prologue(p, stream));
 }
 

@@ -234,6 +234,8 @@ struct PrologueLaunch {
   const float *dg;
   void *dxq, *dxk, *dxv, *db;
   float *dwq, *dwk, *dwv, *da;
+  const int32_t *cu;  // packed documents (null: batch rows)
+  int N;
 };
 cudaError_t prologue(const PrologueLaunch &p, cudaStream_t s);
 

@@ -40,7 +40,27 @@ struct PrologueArgs {
   const float *dg;
   void *dxq, *dxk, *dxv, *db;  // backward outputs
   float *dwq, *dwk, *dwv, *da;
+  const int32_t *cu;  // packed documents: [N + 1] offsets (null: every batch row is a sequence)
+  int N;
 };
+
+// First token of the document of each token t0 - 3 + e, e < n (0 when every
+// batch row is its own sequence): the convolution's history stops there.
+__device__ __forceinline__ void doc_starts(const PrologueArgs &a, int t0, int n, int *s_ds) {
+  for (int e = threadIdx.x; e < n; e += kPrThreads) {
+    const int t = t0 - 3 + e;
+    int start = 0;
+    if (a.cu && t >= 0 && t < a.T) {  // the last i with cu[i] <= t
+      int lo = 0, hi = a.N;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (a.cu[mid] <= t) lo = mid; else hi = mid - 1;
+      }
+      start = a.cu[lo];
+    }
+    s_ds[e] = start;
+  }
+}
 
 // sigmoid with the fast exponential and division (a few ulp; 0 for y below
 // about -88, where the exponential overflows)
@@ -94,15 +114,21 @@ __device__ __forceinline__ void block_sum16(float (&x)[16], float (*red)[kPrThre
 
 // Forward: 8 tokens per reduction (q and k sums of squares).
 constexpr int kFwdG = 8;
-template <typename IO, int DK, int DV>
+// PACKED: documents packed in one row (a.cu); otherwise the masks are not compiled.
+template <typename IO, int DK, int DV, bool PACKED>
 __global__ void __launch_bounds__(kPrThreads, 6) prologue_fwd_kernel(const PrologueArgs a) {
   __shared__ __align__(16) float red[2][kPrThreads / 32][16];
+  __shared__ int s_ds[PACKED ? kPrTok + 8 : 1];
   const int c = threadIdx.x, h = blockIdx.y, sq = blockIdx.z;
   const int T = a.T, H = a.H;
   constexpr int dk = DK, dv = DV;
   const int t0 = blockIdx.x * kPrTok, t1 = min(t0 + kPrTok, T);
   const bool kc = DK == kPrThreads || c < DK, vc = DV == kPrThreads || c < DV;  // (compile-time true at 128)
   const IO *xq = (const IO *)a.xq, *xk = (const IO *)a.xk, *xv = (const IO *)a.xv;
+  if constexpr (PACKED) {
+    doc_starts(a, t0, kPrTok + 3, s_ds);
+    __syncthreads();
+  }
   float wq[4], wk[4], wv[4];
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
@@ -142,9 +168,13 @@ __global__ void __launch_bounds__(kPrThreads, 6) prologue_fwd_kernel(const Prolo
       const bool live = t < t1;
       const size_t row = ((size_t)sq * T + (live ? t : tb)) * H + h;
       const float xqt = lq[i], xkt = lk[i], xvt = lv[i];
-      const float yq = wq[0] * hq[0] + wq[1] * hq[1] + wq[2] * hq[2] + wq[3] * xqt;
-      const float yk = wk[0] * hk[0] + wk[1] * hk[1] + wk[2] * hk[2] + wk[3] * xkt;
-      const float yv = wv[0] * hv[0] + wv[1] * hv[1] + wv[2] * hv[2] + wv[3] * xvt;
+      // history of token t stops at its document's first token
+      const int ds = PACKED ? s_ds[(live ? t : tb) - t0 + 3] : 0;
+      const float m3 = !PACKED || t - 3 >= ds ? 1.f : 0.f, m2 = !PACKED || t - 2 >= ds ? 1.f : 0.f,
+                  m1 = !PACKED || t - 1 >= ds ? 1.f : 0.f;
+      const float yq = wq[0] * m3 * hq[0] + wq[1] * m2 * hq[1] + wq[2] * m1 * hq[2] + wq[3] * xqt;
+      const float yk = wk[0] * m3 * hk[0] + wk[1] * m2 * hk[1] + wk[2] * m1 * hk[2] + wk[3] * xkt;
+      const float yv = wv[0] * m3 * hv[0] + wv[1] * m2 * hv[1] + wv[2] * m1 * hv[2] + wv[3] * xvt;
       hq[0] = hq[1]; hq[1] = hq[2]; hq[2] = xqt;
       hk[0] = hk[1]; hk[1] = hk[2]; hk[2] = xkt;
       hv[0] = hv[1]; hv[1] = hv[2]; hv[2] = xvt;
@@ -179,14 +209,21 @@ __global__ void __launch_bounds__(kPrThreads, 6) prologue_fwd_kernel(const Prolo
 // Backward: 4 tokens per reduction (|n|^2 and n . dn for q and k); the run's
 // tokens plus a three-token halo (dx of token s needs dy of s .. s + 3).
 constexpr int kBwdG = 4;
-template <typename IO, int DK, int DV>
+template <typename IO, int DK, int DV, bool PACKED>
 __global__ void __launch_bounds__(kPrThreads, 4) prologue_bwd_kernel(const PrologueArgs a) {
   __shared__ __align__(16) float red[2][kPrThreads / 32][16];
+  __shared__ int s_ds[PACKED ? kPrTok + 8 : 1];
   const int c = threadIdx.x, h = blockIdx.y, sq = blockIdx.z;
   const int T = a.T, H = a.H;
   constexpr int dk = DK, dv = DV;
   const int t0 = blockIdx.x * kPrTok, t1 = min(t0 + kPrTok, T);
   const int tend = min(t0 + kPrTok + 3, T);
+  if constexpr (PACKED) {
+    doc_starts(a, t0, kPrTok + 6, s_ds);
+    __syncthreads();
+  }
+  // first token of t's document, t in [t0 - 3, t0 + kPrTok + 3) (0 unpacked)
+  auto ds_of = [&](int t) { return PACKED ? s_ds[t - t0 + 3] : 0; };
   const bool kc = DK == kPrThreads || c < DK, vc = DV == kPrThreads || c < DV;  // (compile-time true at 128)
   const IO *xq = (const IO *)a.xq, *xk = (const IO *)a.xk, *xv = (const IO *)a.xv;
   const IO *gq = (const IO *)a.dq, *gk = (const IO *)a.dk_in, *gv = (const IO *)a.dv_in;
@@ -240,9 +277,12 @@ __global__ void __launch_bounds__(kPrThreads, 4) prologue_bwd_kernel(const Prolo
       const size_t row = ((size_t)sq * T + (live ? t : t0)) * H + h;
       const float xqt = xwq[3 + i], xkt = xwk[3 + i], xvt = xwv[3 + i];
       const float dvt = ldv[i];
-      yq[i] = wq[0] * xwq[i] + wq[1] * xwq[i + 1] + wq[2] * xwq[i + 2] + wq[3] * xqt;
-      yk[i] = wk[0] * xwk[i] + wk[1] * xwk[i + 1] + wk[2] * xwk[i + 2] + wk[3] * xkt;
-      const float yv = wv[0] * xwv[i] + wv[1] * xwv[i + 1] + wv[2] * xwv[i + 2] + wv[3] * xvt;
+      const int ds = live ? ds_of(t) : 0;
+      const float m3 = !PACKED || t - 3 >= ds ? 1.f : 0.f, m2 = !PACKED || t - 2 >= ds ? 1.f : 0.f,
+                  m1 = !PACKED || t - 1 >= ds ? 1.f : 0.f;
+      yq[i] = wq[0] * m3 * xwq[i] + wq[1] * m2 * xwq[i + 1] + wq[2] * m1 * xwq[i + 2] + wq[3] * xqt;
+      yk[i] = wk[0] * m3 * xwk[i] + wk[1] * m2 * xwk[i + 1] + wk[2] * m1 * xwk[i + 2] + wk[3] * xkt;
+      const float yv = wv[0] * m3 * xwv[i] + wv[1] * m2 * xwv[i + 1] + wv[2] * m1 * xwv[i + 2] + wv[3] * xvt;
       pq[i] = sigm(yq[i]);
       pk[i] = sigm(yk[i]);
       const float pv = sigm(yv);
@@ -270,19 +310,29 @@ __global__ void __launch_bounds__(kPrThreads, 4) prologue_bwd_kernel(const Prolo
       const float dyk = live ? (rk * dkt[i] - rk * rk * rk * s[4 * i + 3] * nk) * (pk[i] * (1.f + yk[i] * (1.f - pk[i]))) : 0.f;
       const int so = t - 3;  // dx of token t - 3 is complete
       if (so >= t0 && so < t1) {
+        // token so + k reads x_so only inside so's document (so >= its first token)
+        const float n1 = !PACKED || so >= ds_of(so + 1) ? 1.f : 0.f;
+        const float n2 = !PACKED || so >= ds_of(so + 2) ? 1.f : 0.f;
+        const float n3 = !PACKED || (t < T && so >= ds_of(t)) ? 1.f : 0.f;
         const size_t row = ((size_t)sq * T + so) * H + h;
         if (kc) {
-          st_io((IO *)a.dxq, row * dk + c, wq[3] * eq[0] + wq[2] * eq[1] + wq[1] * eq[2] + wq[0] * dyq);
-          st_io((IO *)a.dxk, row * dk + c, wk[3] * ek[0] + wk[2] * ek[1] + wk[1] * ek[2] + wk[0] * dyk);
+          st_io((IO *)a.dxq, row * dk + c,
+                wq[3] * eq[0] + wq[2] * n1 * eq[1] + wq[1] * n2 * eq[2] + wq[0] * n3 * dyq);
+          st_io((IO *)a.dxk, row * dk + c,
+                wk[3] * ek[0] + wk[2] * n1 * ek[1] + wk[1] * n2 * ek[2] + wk[0] * n3 * dyk);
         }
-        if (vc) st_io((IO *)a.dxv, row * dv + c, wv[3] * ev[0] + wv[2] * ev[1] + wv[1] * ev[2] + wv[0] * dyv[i]);
+        if (vc)
+          st_io((IO *)a.dxv, row * dv + c,
+                wv[3] * ev[0] + wv[2] * n1 * ev[1] + wv[1] * n2 * ev[2] + wv[0] * n3 * dyv[i]);
       }
-      if (t < t1) {  // the taps' sums over this run's tokens: dy_t x_{t-3+j}
+      if (t < t1) {  // the taps' sums over this run's tokens: dy_t x_{t-3+j} (inside t's document)
+        const int ds = ds_of(t);
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          sq4[j] += dyq * xwq[i + j];
-          sk4[j] += dyk * xwk[i + j];
-          sv4[j] += dyv[i] * xwv[i + j];
+          const float mj = (!PACKED || j == 3 || t - 3 + j >= ds) ? 1.f : 0.f;
+          sq4[j] += mj * dyq * xwq[i + j];
+          sk4[j] += mj * dyk * xwk[i + j];
+          sv4[j] += mj * dyv[i] * xwv[i + j];
         }
       }
       eq[0] = eq[1]; eq[1] = eq[2]; eq[2] = dyq;
@@ -323,13 +373,19 @@ cudaError_t prologue(const PrologueLaunch &p, cudaStream_t s) {
   a.dq = p.dq; a.dk_in = p.dk_in; a.dv_in = p.dv_in; a.dbeta = p.dbeta; a.dg = p.dg;
   a.dxq = p.dxq; a.dxk = p.dxk; a.dxv = p.dxv; a.db = p.db;
   a.dwq = p.dwq; a.dwk = p.dwk; a.dwv = p.dwv; a.da = p.da;
+  a.cu = p.cu; a.N = p.N;
   if ((size_t)p.B * p.T * p.H == 0) return cudaSuccess;
   const dim3 grid((p.T + kPrTok - 1) / kPrTok, p.H, p.B);
   ProfScope prof(p.backward ? "prologue_bwd" : "prologue_fwd", s);
 #define CKDA_PRO_LAUNCH(IO, K, V)                                                   \
   do {                                                                              \
-    if (p.backward) prologue_bwd_kernel<IO, K, V><<<grid, kPrThreads, 0, s>>>(a);  \
-    else prologue_fwd_kernel<IO, K, V><<<grid, kPrThreads, 0, s>>>(a);             \
+    if (p.backward) {                                                               \
+      if (a.cu) prologue_bwd_kernel<IO, K, V, true><<<grid, kPrThreads, 0, s>>>(a); \
+      else prologue_bwd_kernel<IO, K, V, false><<<grid, kPrThreads, 0, s>>>(a);     \
+    } else {                                                                        \
+      if (a.cu) prologue_fwd_kernel<IO, K, V, true><<<grid, kPrThreads, 0, s>>>(a); \
+      else prologue_fwd_kernel<IO, K, V, false><<<grid, kPrThreads, 0, s>>>(a);     \
+    }                                                                               \
   } while (0)
 #define CKDA_PRO_DIMS(IO)                                   \
   do {                                                      \

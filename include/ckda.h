@@ -199,17 +199,26 @@ int ckda_decode_multi(int N, int K, int H, int dk, int dv, int io_dtype,
  *   wv [H*dv, 4] f32 (row h*d + c holds channel c of head h's four taps);
  *   a [B,T,H,dk] f32 (gate pre-activation);  b [B,T,H] io;
  *   g_floor: finite and <= 0 (e.g. -5), else CKDA_ERR_INVALID_ARG.
+ *   cu_seqlens: null (every batch row is one sequence), or [N+1] int32
+ *             DEVICE offsets of N documents packed in one row (B = 1, else
+ *             CKDA_ERR_INVALID_ARG; 4-byte aligned; N >= 1): the history
+ *             restarts at each document's first token, as ckda_varlen_fwd's
+ *             recurrence does.  Its offsets are not checked here (the varlen
+ *             calls do): malformed ones give unspecified values, never an
+ *             access outside the buffers.
  *   Outputs q, k [B,T,H,dk] io;  v [B,T,H,dv] io;  g [B,T,H,dk] f32;
- *   sign [B,T,H,dk] int8;  beta [B,T,H] io: the inputs of ckda_chunk_fwd.
+ *   sign [B,T,H,dk] int8;  beta [B,T,H] io: the inputs of ckda_chunk_fwd
+ *   (of ckda_varlen_fwd with cu_seqlens).
  * B and H at most 65535.  No workspace. */
 int ckda_prologue_fwd(int B, int T, int H, int dk, int dv, int io_dtype,
                       const void *xq, const void *xk, const void *xv,
                       const float *wq, const float *wk, const float *wv,
-                      const float *a, const void *b, float g_floor, void *q,
+                      const float *a, const void *b, float g_floor,
+                      const int32_t *cu_seqlens, int N, void *q,
                       void *k, void *v, float *g, int8_t *sign, void *beta,
                       cudaStream_t stream);
 
-/* Backward of ckda_prologue_fwd (same inputs) from the gradients of its
+/* Backward of ckda_prologue_fwd (same inputs, cu_seqlens and N included) from the gradients of its
  * outputs (dq, dk_in [B,T,H,dk] io;  dv_in [B,T,H,dv] io;  dg [B,T,H,dk]
  * f32;  dbeta [B,T,H] io -- what ckda_chunk_bwd returns).  Exact gradients of
  * the formulas above; the sign gets none; where the floor is active g gets
@@ -222,6 +231,7 @@ int ckda_prologue_bwd(int B, int T, int H, int dk, int dv, int io_dtype,
                       const void *xq, const void *xk, const void *xv,
                       const float *wq, const float *wk, const float *wv,
                       const float *a, const void *b, float g_floor,
+                      const int32_t *cu_seqlens, int N,
                       const void *dq, const void *dk_in, const void *dv_in,
                       const float *dg, const void *dbeta, void *dxq, void *dxk,
                       void *dxv, float *dwq, float *dwk, float *dwv, float *da,

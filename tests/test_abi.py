@@ -132,14 +132,19 @@ def test_host_validation_without_gpu():
     assert multi(N=0) == 0 and multi(K=0) == 0        # nothing to do
 
     F = ctypes.c_float
-    pf = lambda B=1, T=8, dk=64, io=0, floor=-5.0, ptrs=None: lib.ckda_prologue_fwd(
-        B, T, 2, dk, 64, io, *([fake] * 8 if ptrs is None else ptrs), F(floor), *([fake] * 6), None)
+    pf = lambda B=1, T=8, dk=64, io=0, floor=-5.0, ptrs=None, cu=None, n=0: lib.ckda_prologue_fwd(
+        B, T, 2, dk, 64, io, *([fake] * 8 if ptrs is None else ptrs), F(floor), cu, n, *([fake] * 6), None)
     assert pf(B=-1) == 1 and pf(io=3) == 1 and pf(dk=32) == 2
     assert pf(floor=0.5) == 1 and pf(floor=float("-inf")) == 1 and pf(floor=float("nan")) == 1
     assert pf(B=70000) == 2                          # grid limit on B and H
     assert pf(ptrs=[fake] * 7 + [None]) == 1         # b missing
     assert pf(ptrs=[odd] + [fake] * 7) == 3
     assert pf(T=0) == 0                              # empty: nothing to do
-    pb = lambda dw=fake, floor=-5.0: lib.ckda_prologue_bwd(
-        1, 8, 2, 64, 64, 0, *([fake] * 8), F(floor), *([fake] * 5), fake, fake, fake, dw, fake, fake, fake, fake, None)
+    assert pf(B=2, cu=fake, n=2) == 1                # packed documents take one row
+    assert pf(cu=fake, n=0) == 1                     # ... and at least one document
+    assert pf(cu=ctypes.c_void_p((1 << 20) + 2), n=2) == 3
+    pb = lambda dw=fake, floor=-5.0, B=1, cu=None, n=0: lib.ckda_prologue_bwd(
+        B, 8, 2, 64, 64, 0, *([fake] * 8), F(floor), cu, n, *([fake] * 5), fake, fake, fake, dw, fake, fake, fake,
+        fake, None)
     assert pb(dw=None) == 1 and pb(floor=1.0) == 1
+    assert pb(B=2, cu=fake, n=1) == 1 and pb(cu=fake, n=-1) == 1

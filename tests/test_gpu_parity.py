@@ -569,6 +569,15 @@ def test_prologue_forward_backward(io, B, T, H, dk, dv, g_floor):
         check(n, gr[n], rg[n], io)
 
 
+def _oracle_prologue_stored(x, io, cu=None):
+    """The oracle's prologue outputs as the boundary stores them (q, k, v,
+    beta in the I/O dtype, g in fp32): the recurrence oracle's inputs."""
+    r = oracle.prologue_fwd(**{n: f64(t) for n, t in x.items()}, g_floor=-5.0, cu_seqlens=cu)
+    st = {n: torch.from_numpy(r[n]).to(io) for n in ("q", "k", "v", "beta")}
+    st.update(g=torch.from_numpy(r["g"]).float(), sign=torch.from_numpy(r["sign"]))
+    return st
+
+
 def test_prologue_feeds_the_recurrence():
     """prologue -> chunked forward equals the oracle's prologue -> recurrence."""
     io, B, T, H, d = torch.bfloat16, 1, 150, 2, 128
@@ -577,9 +586,60 @@ def test_prologue_feeds_the_recurrence():
     p = api.prologue_fwd(dx["xq"], dx["xk"], dx["xv"], dx["wq"], dx["wk"], dx["wv"], dx["a"], dx["b"], g_floor=-5.0)
     o, ST, _ = api.chunk_fwd(p["q"], p["k"], p["v"], p["g"], p["sign"], p["beta"])
     torch.cuda.synchronize()
-    cpu = {n: t.cpu() for n, t in p.items()}
-    o_ref, ST_ref, _ = oracle_fwd_batched(cpu)
+    o_ref, ST_ref, _ = oracle_fwd_batched(_oracle_prologue_stored(x, io))
     check("o", o, o_ref, io)
+    check("ST", ST, ST_ref, io)
+
+
+@pytest.mark.parametrize("io", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("lens,dk,dv", [([1, 2, 0, 58, 3, 2, 64, 3, 67], 64, 128),
+                                        ([61, 4, 1, 1, 1, 62, 70], 128, 64), ([130], 128, 128)])
+def test_prologue_packed_documents(io, lens, dk, dv):
+    """Documents packed in one row (cu_seqlens): the conv history restarts at
+    every document start, forward and backward, against the oracle (documents
+    of one to three tokens, an empty one, starts just before, at and after
+    the kernels' 64-token run edges)."""
+    T, H, g_floor = int(sum(lens)), 2, -5.0
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    x, up = _prologue_inputs(1, T, H, dk, dv, io, seed=T + dk)
+    d = to_dev({**x, **up})
+    names = ("xq", "xk", "xv", "wq", "wk", "wv", "a", "b")
+    dcu = torch.from_numpy(cu).cuda()
+    got = api.prologue_fwd(*(d[n] for n in names), g_floor=g_floor, cu_seqlens=dcu)
+    gr = api.prologue_bwd(*(d[n] for n in names), d["dq"], d["dk"], d["dv"], d["dg"], d["dbeta"],
+                          g_floor=g_floor, cu_seqlens=dcu)
+    torch.cuda.synchronize()
+    X = {n: f64(t) for n, t in x.items()}
+    ref = oracle.prologue_fwd(**X, g_floor=g_floor, cu_seqlens=cu)
+    for n in ("q", "k", "v", "g", "beta"):
+        check(n, got[n], ref[n], io)
+    assert torch.equal(got["sign"].cpu(), torch.from_numpy(ref["sign"]))
+    rg = oracle.prologue_bwd(**X, **{n: f64(t) for n, t in up.items()}, g_floor=g_floor, cu_seqlens=cu)
+    for n in ("dxq", "dxk", "dxv", "dwq", "dwk", "dwv", "da", "db"):
+        check(n, gr[n], rg[n], io)
+    if len(lens) == 1:  # one document: the same kernels' arithmetic as the unpacked row
+        plain = api.prologue_fwd(*(d[n] for n in names), g_floor=g_floor)
+        for n in ("q", "k", "v", "g", "sign", "beta"):
+            assert torch.equal(plain[n], got[n]), n
+
+
+def test_prologue_packed_feeds_varlen():
+    """Packed prologue -> packed recurrence equals the oracle's per-document
+    prologue -> recurrence."""
+    io, H, d, lens = torch.bfloat16, 2, 128, [37, 2, 90, 64]
+    T = sum(lens)
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    x, _ = _prologue_inputs(1, T, H, d, d, io, seed=9)
+    dx = to_dev(x)
+    p = api.prologue_fwd(*(dx[n] for n in ("xq", "xk", "xv", "wq", "wk", "wv", "a", "b")), g_floor=-5.0,
+                         cu_seqlens=torch.from_numpy(cu).cuda())
+    o, ST = api.varlen_fwd(p["q"], p["k"], p["v"], p["g"], p["sign"], p["beta"], torch.from_numpy(cu).cuda(),
+                           max(lens))
+    torch.cuda.synchronize()
+    r = _oracle_prologue_stored(x, io, cu)
+    P = lambda n: f64(r[n][0])
+    o_ref, ST_ref, _ = oracle.fwd(cu.astype(np.int64), P("q"), P("k"), P("v"), P("g"), r["sign"][0].numpy(), P("beta"))
+    check("o", o[0], o_ref, io)
     check("ST", ST, ST_ref, io)
 
 

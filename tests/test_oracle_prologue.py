@@ -122,3 +122,69 @@ def test_gradients_central_differences(g_floor):
         clamped = np.log(np.abs(np.tanh(x["a"]))) < g_floor
         assert clamped.sum() > 3
         assert np.all(grads["da"][clamped] == 0.0)
+
+
+def test_packed_documents_equal_batch_rows():
+    """Three documents of equal length packed in one row give what three
+    batch rows give: outputs, input gradients, and the taps' gradients (sums
+    over every token either way)."""
+    rng = np.random.default_rng(11)
+    x = _inputs(3, 5, 2, 3, 2, rng=rng)
+    up = dict(dq=rng.standard_normal((3, 5, 2, 3)), dk=rng.standard_normal((3, 5, 2, 3)),
+              dv=rng.standard_normal((3, 5, 2, 2)), dg=rng.standard_normal((3, 5, 2, 3)),
+              dbeta=rng.standard_normal((3, 5, 2)))
+    row = lambda v: v.reshape((1, -1) + v.shape[2:])
+    px = {k: (row(v) if k[0] != "w" else v) for k, v in x.items()}
+    pu = {k: row(v) for k, v in up.items()}
+    cu = [0, 5, 10, 15]
+    r, pr = oracle.prologue_fwd(**x), oracle.prologue_fwd(**px, cu_seqlens=cu)
+    for n in ("q", "k", "v", "g", "beta", "sign"):
+        np.testing.assert_allclose(pr[n], row(r[n]), rtol=1e-14, atol=1e-15, err_msg=n)
+    g, pg = oracle.prologue_bwd(**x, **up), oracle.prologue_bwd(**px, **pu, cu_seqlens=cu)
+    for n in ("dxq", "dxk", "dxv", "da", "db"):
+        np.testing.assert_allclose(pg[n], row(g[n]), rtol=1e-13, atol=1e-14, err_msg=n)
+    for n in ("dwq", "dwk", "dwv"):
+        np.testing.assert_allclose(pg[n], g[n], rtol=1e-12, atol=1e-13, err_msg=n)
+
+
+def test_packed_ragged_documents_match_numpy_convolve():
+    """Ragged documents (one shorter than the window, one empty): numpy's
+    convolution restarted at each document start."""
+    rng = np.random.default_rng(12)
+    cu = [0, 2, 2, 9, 13]
+    x = _inputs(1, 13, 2, 3, 4, rng=rng)
+    r = oracle.prologue_fwd(**x, cu_seqlens=cu)
+    want = np.concatenate([_np_conv(x["xv"][:, s:e], x["wv"]) for s, e in zip(cu, cu[1:]) if e > s], axis=1)
+    np.testing.assert_allclose(r["v"], _silu(want), rtol=1e-13, atol=1e-14)
+    with pytest.raises(ValueError):
+        oracle.prologue_fwd(**x, cu_seqlens=[0, 5, 4, 13])
+    with pytest.raises(ValueError):
+        oracle.prologue_fwd(**x, cu_seqlens=[0, 12])
+
+
+def test_packed_gradients_central_differences():
+    """Input and tap gradients of a packed row (a two-token document, an
+    empty one, a five-token one) against central differences."""
+    rng = np.random.default_rng(13)
+    cu = [0, 2, 2, 7]
+    x = _inputs(1, 7, 1, 2, 2, rng=rng, ascale=1.0)
+    up = dict(dq=rng.standard_normal((1, 7, 1, 2)), dk=rng.standard_normal((1, 7, 1, 2)),
+              dv=rng.standard_normal((1, 7, 1, 2)), dg=rng.standard_normal((1, 7, 1, 2)),
+              dbeta=rng.standard_normal((1, 7, 1)))
+
+    def loss(inp):
+        r = oracle.prologue_fwd(**inp, cu_seqlens=cu)
+        return sum(float(np.sum(r[n] * up["d" + n])) for n in ("q", "k", "v", "g", "beta"))
+
+    grads = oracle.prologue_bwd(**x, **up, cu_seqlens=cu)
+    eps = 1e-6
+    for name in ("xq", "xk", "xv", "wq", "wk", "wv"):
+        gr = grads["d" + name]
+        fd = np.zeros_like(gr)
+        for idx in np.ndindex(x[name].shape):
+            xp = {k: v.copy() for k, v in x.items()}
+            xm = {k: v.copy() for k, v in x.items()}
+            xp[name][idx] += eps
+            xm[name][idx] -= eps
+            fd[idx] = (loss(xp) - loss(xm)) / (2 * eps)
+        np.testing.assert_allclose(gr, fd, rtol=1e-5, atol=1e-7, err_msg=name)

@@ -24,6 +24,9 @@ MUTATIONS = {
     "history_across_sequences": (
         "torch.cat([torch.zeros_like(x[:, :shift]), x[:, :T - shift]], dim=1)",
         "torch.cat([torch.roll(x, 1, 0)[:, T - shift:], x[:, :T - shift]], dim=1)"),
+    "history_across_documents": (
+        "return torch.cat([_conv_silu(x[:, s:e], w) for s, e in docs], dim=1)",
+        "return _conv_silu(x, w)"),
     "gradient_through_floor": (
         "g = torch.clamp(torch.log(torch.abs(alpha)), min=g_floor)",
         "lg = torch.log(torch.abs(alpha))\n    g = torch.clamp(lg, min=g_floor).detach() + "
@@ -33,6 +36,7 @@ MUTATIONS = {
 # cheap pins first; the finite-difference sweep last
 PINS = [pins.test_short_conv_silu_matches_numpy_convolve, pins.test_conv_restarts_at_each_sequence,
         pins.test_single_tap_reduces_to_pointwise, pins.test_signed_gate_closed_forms,
+        pins.test_packed_documents_equal_batch_rows, pins.test_packed_ragged_documents_match_numpy_convolve,
         lambda: pins.test_gradients_central_differences(-1.0)]
 
 
