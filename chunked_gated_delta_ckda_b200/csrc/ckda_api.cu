@@ -70,6 +70,12 @@ int check_common(int B, int T, int H, int dk, int dv, int io_dtype) {
   return CKDA_OK;
 }
 
+// sequences (B or N) and heads index grid dimensions limited to 65535
+int check_grid(int B, int H, int N) {
+  if (B > 65535 || H > 65535 || N > 65535) return CKDA_ERR_UNSUPPORTED;
+  return CKDA_OK;
+}
+
 int check_ptrs(std::initializer_list<const void *> required,
                std::initializer_list<const void *> optional) {
   for (const void *p : required)
@@ -139,17 +145,18 @@ size_t ckda_workspace_size(int op, int B, int T, int H, int dk, int dv, int N) {
   if (op == CKDA_OP_VARLEN_FWD || op == CKDA_OP_VARLEN_BWD) {
     if (B != 1 || N < 0) return 0;
   }
-  if (check_common(B, T, H, dk, dv, CKDA_F32) != CKDA_OK) return 0;
+  if (check_common(B, T, H, dk, dv, CKDA_F32) != CKDA_OK || check_grid(B, H, N) != CKDA_OK) return 0;
   return ws_layout(op, B, T, H, dk, dv, N).total;
 }
 
 size_t ckda_saved_size(int B, int T, int H, int dk, int dv, int io_dtype) {
-  if (check_common(B, T, H, dk, dv, io_dtype) != CKDA_OK) return 0;
+  if (check_common(B, T, H, dk, dv, io_dtype) != CKDA_OK || check_grid(B, H, 0) != CKDA_OK) return 0;
   return saved_bytes_for(B, T, H, dk, dv, io_dtype);
 }
 
 size_t ckda_varlen_saved_size(int total_T, int N, int H, int dk, int dv, int io_dtype) {
-  if (check_common(1, total_T, H, dk, dv, io_dtype) != CKDA_OK || N < 0) return 0;
+  if (check_common(1, total_T, H, dk, dv, io_dtype) != CKDA_OK || N < 0 || check_grid(1, H, N) != CKDA_OK)
+    return 0;
   return packed_saved_bytes_for(total_T, N, H, dk, dv, io_dtype);
 }
 
@@ -159,6 +166,7 @@ int ckda_chunk_fwd(int B, int T, int H, int dk, int dv, int io_dtype, const void
                    void *saved, size_t saved_bytes, void *ws, size_t ws_bytes,
                    cudaStream_t stream) {
   CKDA_TRY(check_common(B, T, H, dk, dv, io_dtype));
+  CKDA_TRY(check_grid(B, H, 0));
   const bool empty = (int64_t)B * T == 0;
   if (!empty) CKDA_TRY(check_ptrs({q, k, v, g, beta, o}, {sign, S0, ST, chunk_states}));
   else CKDA_TRY(check_ptrs({}, {sign, S0, ST, chunk_states}));
@@ -201,6 +209,7 @@ int ckda_chunk_bwd(int B, int T, int H, int dk, int dv, int io_dtype, const void
                    void *dk_out, void *dv_out, float *dg, void *dbeta, float *dS0, void *ws,
                    size_t ws_bytes, cudaStream_t stream) {
   CKDA_TRY(check_common(B, T, H, dk, dv, io_dtype));
+  CKDA_TRY(check_grid(B, H, 0));
   const bool empty = (int64_t)B * T == 0;
   if (!empty)
     CKDA_TRY(check_ptrs({q, k, v, g, beta, dO, dq, dk_out, dv_out, dg, dbeta},
@@ -301,8 +310,7 @@ static int prologue_common(int B, int T, int H, int dk, int dv, int io_dtype, fl
     if (B != 1 || N < 1) return CKDA_ERR_INVALID_ARG;
     if ((reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) != 0) return CKDA_ERR_ALIGNMENT;
   }
-  if (B > 65535 || H > 65535) return CKDA_ERR_UNSUPPORTED;
-  return CKDA_OK;
+  return check_grid(B, H, 0);
 }
 
 int ckda_prologue_fwd(int B, int T, int H, int dk, int dv, int io_dtype, const void *xq, const void *xk,
@@ -353,6 +361,7 @@ int ckda_varlen_fwd(int total_T, int N, const int32_t *cu_seqlens, int max_seqle
                     cudaStream_t stream) {
   CKDA_TRY(check_common(1, total_T, H, dk, dv, io_dtype));
   if (N < 0) return CKDA_ERR_INVALID_ARG;
+  CKDA_TRY(check_grid(1, H, N));
   if (N == 0) return total_T == 0 ? CKDA_OK : CKDA_ERR_INVALID_ARG;
   if (!cu_seqlens) return CKDA_ERR_INVALID_ARG;
   if (total_T > 0 && (max_seqlen < 1 || max_seqlen > total_T)) return CKDA_ERR_INVALID_ARG;
@@ -407,6 +416,7 @@ int ckda_varlen_bwd(int total_T, int N, const int32_t *cu_seqlens, int max_seqle
                     void *dbeta, float *dS0, void *ws, size_t ws_bytes, cudaStream_t stream) {
   CKDA_TRY(check_common(1, total_T, H, dk, dv, io_dtype));
   if (N < 0) return CKDA_ERR_INVALID_ARG;
+  CKDA_TRY(check_grid(1, H, N));
   if (N == 0) return total_T == 0 ? CKDA_OK : CKDA_ERR_INVALID_ARG;
   if (!cu_seqlens) return CKDA_ERR_INVALID_ARG;
   if (total_T > 0 && (max_seqlen < 1 || max_seqlen > total_T)) return CKDA_ERR_INVALID_ARG;
@@ -491,7 +501,8 @@ const char *ckda_status_string(int status) {
   switch (status) {
     case CKDA_OK: return "ok";
     case CKDA_ERR_INVALID_ARG: return "invalid argument (null pointer, negative size or bad enum)";
-    case CKDA_ERR_UNSUPPORTED: return "unsupported shape (dk and dv must be 64 or 128)";
+    case CKDA_ERR_UNSUPPORTED:
+      return "unsupported shape (dk, dv in {64, 128}; B, H, N at most 65535; B*T below 2^30)";
     case CKDA_ERR_ALIGNMENT: return "misaligned pointer (tensors 16-byte, workspace 256-byte)";
     case CKDA_ERR_WORKSPACE: return "workspace missing or smaller than ckda_workspace_size()";
     case CKDA_ERR_CUDA: return "CUDA launch or runtime error";

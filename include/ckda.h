@@ -70,7 +70,8 @@ extern "C" {
 /* status codes */
 #define CKDA_OK 0
 #define CKDA_ERR_INVALID_ARG 1 /* null required pointer, negative size, bad enum  */
-#define CKDA_ERR_UNSUPPORTED 2 /* dk or dv outside {64, 128}                       */
+#define CKDA_ERR_UNSUPPORTED 2 /* dk or dv outside {64, 128}; B, H or N above 65535;
+                                  B*T (total_T) at or above 2^30                   */
 #define CKDA_ERR_ALIGNMENT 3   /* a pointer breaks the alignment rule above        */
 #define CKDA_ERR_WORKSPACE 4   /* ws null or smaller than ckda_workspace_size()    */
 #define CKDA_ERR_CUDA 5        /* a kernel launch or runtime call failed           */

@@ -81,6 +81,11 @@ def test_host_validation_without_gpu():
     assert fwd(1, 64, 2, 64, 64, 0, a, 1 << 30) == 3
     # workspace too small
     assert fwd(1, 64, 2, 64, 64, 0, args, 16) == 4
+    # sequences and heads index grid dimensions: at most 65535 each
+    assert fwd(70000, 1, 2, 64, 64, 0, args, 1 << 30) == 2
+    assert fwd(1, 64, 70000, 64, 64, 0, args, 1 << 30) == 2
+    assert lib.ckda_workspace_size(0, 70000, 1, 2, 64, 64, 0) == 0
+    assert lib.ckda_workspace_size(2, 1, 100000, 2, 64, 64, 70000) == 0
     # saved buffer: too small / misaligned where the configuration has a saved form
     need = lib.ckda_saved_size(1, 64, 2, 128, 128, 1)
     assert fwd(1, 64, 2, 128, 128, 1, args, 1 << 30, [fake, need - 1]) == 4
@@ -92,6 +97,7 @@ def test_host_validation_without_gpu():
     v = [fake] * 9
     assert lib.ckda_varlen_fwd(100, 2, fake, 0, 2, 64, 64, 0, *v, None, 0, fake, 1 << 30, None) == 1
     assert lib.ckda_varlen_fwd(100, -1, fake, 50, 2, 64, 64, 0, *v, None, 0, fake, 1 << 30, None) == 1
+    assert lib.ckda_varlen_fwd(100000, 70000, fake, 50, 2, 64, 64, 0, *v, None, 0, fake, 1 << 30, None) == 2
     need = lib.ckda_varlen_saved_size(100, 2, 2, 128, 128, 1)
     assert need > 0 and lib.ckda_varlen_saved_size(100, 2, 2, 64, 64, 0) == 0
     assert lib.ckda_varlen_fwd(100, 2, fake, 50, 2, 128, 128, 1, *v, fake, need - 1, fake, 1 << 30, None) == 4
