@@ -281,6 +281,7 @@ int ckda_decode_step(int N, int H, int dk, int dv, int io_dtype, const void *q, 
                      const void *v, const float *g, const int8_t *sign, const void *beta,
                      float *state, void *o, cudaStream_t stream) {
   CKDA_TRY(check_common(N, 1, H, dk, dv, io_dtype));
+  if ((int64_t)N * H > INT32_MAX / 4) return CKDA_ERR_UNSUPPORTED;  // one CTA per (n, h)
   if (N == 0) return CKDA_OK;
   CKDA_TRY(check_ptrs({q, k, v, g, beta, state, o}, {sign}));
   return cuda_status(decode_step(N, H, dk, dv, io_dtype == CKDA_BF16, q, k, v, g, sign, beta,
@@ -292,6 +293,7 @@ int ckda_decode_multi(int N, int K, int H, int dk, int dv, int io_dtype, const v
                       const int32_t *n_tokens, const int32_t *slots, int n_slots, float *state,
                       int write_state, void *o, cudaStream_t stream) {
   CKDA_TRY(check_common(N, K, H, dk, dv, io_dtype));
+  if ((int64_t)N * H > INT32_MAX / 4) return CKDA_ERR_UNSUPPORTED;  // up to 4 CTAs per (n, h)
   if (n_slots < 0 || (write_state != 0 && write_state != 1)) return CKDA_ERR_INVALID_ARG;
   if (!slots && n_slots < N) return CKDA_ERR_INVALID_ARG;
   if (N == 0 || K == 0) return CKDA_OK;

@@ -136,6 +136,8 @@ def test_host_validation_without_gpu():
     assert multi(ptrs=[fake, odd] + [fake] * 4) == 3  # k misaligned
     assert multi(n_tokens=ctypes.c_void_p((1 << 20) + 2)) == 3
     assert multi(N=0) == 0 and multi(K=0) == 0        # nothing to do
+    assert multi(N=1 << 29, K=1, n_slots=1 << 29) == 2  # grid: N * H CTAs
+    assert lib.ckda_decode_step(1 << 29, 4, 64, 64, 0, *([fake] * 8), None) == 2
 
     F = ctypes.c_float
     pf = lambda B=1, T=8, dk=64, io=0, floor=-5.0, ptrs=None, cu=None, n=0: lib.ckda_prologue_fwd(
