@@ -63,6 +63,7 @@ def _load():
         lib.ckda_varlen_saved_size.restype = Z
         lib.ckda_chunk_fwd_noalloc.argtypes = [I] * 6 + [P] * 11
         lib.ckda_check_device_status.argtypes = [P, P]
+        lib.ckda_selftest_bounded_wait.argtypes = [P, Z, ctypes.c_uint32, P]
         lib.ckda_status_string.argtypes = [I]
         lib.ckda_status_string.restype = ctypes.c_char_p
         lib.ckda_version.argtypes = []
@@ -74,7 +75,8 @@ def _load():
         lib.ckda_profile_reset.restype = None
         for f in ("ckda_chunk_fwd", "ckda_chunk_bwd", "ckda_decode_step", "ckda_decode_multi", "ckda_varlen_fwd",
                   "ckda_prologue_fwd", "ckda_prologue_bwd", "ckda_varlen_bwd",
-                  "ckda_chunk_fwd_noalloc", "ckda_check_device_status", "ckda_version", "ckda_profile_enable",
+                  "ckda_chunk_fwd_noalloc", "ckda_check_device_status", "ckda_selftest_bounded_wait",
+                  "ckda_version", "ckda_profile_enable",
                   "ckda_profile_collect", "ckda_profile_get"):
             getattr(lib, f).restype = I
         _lib = lib
@@ -208,6 +210,14 @@ def ckda_chunk_fwd_noalloc(B, T, H, dk, dv, io_dtype, q, k, v, g, sign, beta, S0
 def ckda_check_device_status(ws, stream=None) -> int:
     """Device-side status of the last call that used ``ws`` (syncs the stream)."""
     return int(_load().ckda_check_device_status(_p(ws), _s(stream)))
+
+
+def ckda_selftest_bounded_wait(ws, polls, stream=None):
+    """Failure-detection self-test: a bounded wait on a barrier nothing
+    arrives at gives up after ``polls`` polls and records the time-out in
+    ``ws``'s status word (read it with ckda_check_device_status)."""
+    _check(_load().ckda_selftest_bounded_wait(_p(ws), _nbytes(ws, None), int(polls), _s(stream)),
+           "ckda_selftest_bounded_wait")
 
 
 def ckda_status_string(status: int) -> str:

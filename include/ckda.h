@@ -321,6 +321,18 @@ int ckda_check_device_status(const void *ws, cudaStream_t stream);
 /* Static message for a status code. */
 const char *ckda_status_string(int status);
 
+/* Failure-detection self-test (not part of the recurrence).  Clears the
+ * status word at the head of `ws` (at least 256 bytes, 256-byte aligned,
+ * device memory), then launches one warp whose thread 0 waits, with the
+ * library's bounded mbarrier wait limited to `polls` polls (the kernels use
+ * 2^26), on a barrier that nothing arrives at.  The wait gives up, records
+ * the time-out (status flag bit 0; detail word = site 900) and the kernel
+ * returns, leaving the context usable: ckda_check_device_status(ws) then
+ * returns CKDA_ERR_TIMEOUT.  Errors: null ws CKDA_ERR_INVALID_ARG, smaller
+ * than 256 bytes CKDA_ERR_WORKSPACE, misaligned CKDA_ERR_ALIGNMENT. */
+int ckda_selftest_bounded_wait(void *ws, size_t ws_bytes, uint32_t polls,
+                               cudaStream_t stream);
+
 /* ---- optional per-kernel timing (host side, off by default) -------------
  * Not part of the recurrence: a measurement aid.  While enabled, every kernel
  * launch of the library is bracketed by a pair of CUDA events recorded on the

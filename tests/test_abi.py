@@ -137,6 +137,10 @@ def test_host_validation_without_gpu():
     assert multi(n_tokens=ctypes.c_void_p((1 << 20) + 2)) == 3
     assert multi(N=0) == 0 and multi(K=0) == 0        # nothing to do
     assert multi(N=1 << 29, K=1, n_slots=1 << 29) == 2  # grid: N * H CTAs
+    # failure-detection self-test: workspace checks come before the launch
+    assert lib.ckda_selftest_bounded_wait(None, 256, 1, None) == 1
+    assert lib.ckda_selftest_bounded_wait(fake, 255, 1, None) == 4
+    assert lib.ckda_selftest_bounded_wait(ctypes.c_void_p((1 << 20) + 16), 256, 1, None) == 3
     assert lib.ckda_decode_step(1 << 29, 4, 64, 64, 0, *([fake] * 8), None) == 2
 
     F = ctypes.c_float
