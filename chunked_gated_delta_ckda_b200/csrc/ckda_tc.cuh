@@ -55,9 +55,13 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t phase) {
   return ok != 0;
 }
 // Bounded wait: gives up after `limit` polls, records the failure in the
-// device status word and returns false (the caller then winds down).
+// device status word and returns false (the caller then winds down).  A poll
+// that finds the phase incomplete suspends the thread for about 4 us on B200
+// (measured), so the default gives up after about 4 s; every wait of these
+// kernels completes within microseconds.
+constexpr uint32_t kWaitPolls = 1u << 20;
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t phase, DevStatus *st,
-                                          uint32_t site, uint32_t limit = 1u << 26) {
+                                          uint32_t site, uint32_t limit = kWaitPolls) {
   for (uint32_t i = 0; i < limit; ++i)
     if (mbar_try_wait(bar, phase)) return true;
   if (st) {

@@ -325,7 +325,7 @@ const char *ckda_status_string(int status);
  * status word at the head of `ws` (at least 256 bytes, 256-byte aligned,
  * device memory), then launches one warp whose thread 0 waits, with the
  * library's bounded mbarrier wait limited to `polls` polls (the kernels use
- * 2^26), on a barrier that nothing arrives at.  The wait gives up, records
+ * 2^20, about 4 s), on a barrier that nothing arrives at.  The wait gives up, records
  * the time-out (status flag bit 0; detail word = site 900) and the kernel
  * returns, leaving the context usable: ckda_check_device_status(ws) then
  * returns CKDA_ERR_TIMEOUT.  Errors: null ws CKDA_ERR_INVALID_ARG, smaller
