@@ -123,3 +123,65 @@ def bwd(q, k, v, g, sign, beta, S0, dO, dST, C=64):
         dkk[sl] = x["p"] * dkp
         dbeta[sl] = db
     return dict(dq=dq, dk=dkk, dv=dvv, dg=dg, dbeta=dbeta, dS0=dS)
+
+
+def fwd_u_chain(q, k, v, g, sign, beta, S0, C=64):
+    """The forward with the chunk-to-chunk dependence carried by U instead of
+    S (a reordering for the sequential pass, not yet what the kernels run):
+
+        U_{j+1} = U0_{j+1} - (W_{j+1} Diag(d_j)) S_j - (W_{j+1} Khat_j^T) U_j
+
+    since S_{j+1} = Diag(d_j) S_j + Khat_j^T U_j.  Step j+1's U needs S_j,
+    not S_{j+1}: the S update runs one step behind, off the U chain, whose
+    only product per step is the 64 x 64 one R_{j+1} U_j."""
+    T = q.shape[0]
+    xs = [chunk_intra(q[c0:c0 + C], k[c0:c0 + C], v[c0:c0 + C], g[c0:c0 + C], sign[c0:c0 + C],
+                      beta[c0:c0 + C]) for c0 in range(0, T, C)]
+    o = np.zeros((T, v.shape[1]))
+    S = S0.copy()
+    U = xs[0]["U0"] - xs[0]["W"] @ S
+    for j, x in enumerate(xs):
+        sl = slice(j * C, min(j * C + C, T))
+        o[sl] = x["QG"] @ S + x["Aq"] @ U
+        if j + 1 < len(xs):
+            nx = xs[j + 1]
+            P = nx["W"] * x["d"][None, :]          # W_{j+1} Diag(d_j), off the chain
+            R = nx["W"] @ x["Khat"].T               # W_{j+1} Khat_j^T, 64 x 64, off the chain
+            U_next = nx["U0"] - P @ S - R @ U
+        S = x["d"][:, None] * S + x["Khat"].T @ U
+        if j + 1 < len(xs):
+            U = U_next
+    return o, S
+
+
+def bwd_du_chain(q, k, v, g, sign, beta, S0, dO, dST, C=64):
+    """The reverse state pass with the dependence carried by dU (the
+    counterpart of fwd_u_chain): with dS_j = Diag(d_j) dS_{j+1} +
+    QG_j^T dO_j - W_j^T dU_j,
+
+        dU_{j-1} = [A_q_{j-1}^T dO_{j-1} + Khat_{j-1} QG_j^T dO_j]
+                   + (Khat_{j-1} Diag(d_j)) dS_{j+1} - (Khat_{j-1} W_j^T) dU_j.
+
+    Returns the per-chunk dU and the chunk-end state gradients dS_{j+1},
+    and dS_0, as the reverse pass does."""
+    T = q.shape[0]
+    xs = [chunk_intra(q[c0:c0 + C], k[c0:c0 + C], v[c0:c0 + C], g[c0:c0 + C], sign[c0:c0 + C],
+                      beta[c0:c0 + C]) for c0 in range(0, T, C)]
+    n = len(xs)
+    dOs = [dO[j * C:min(j * C + C, T)] for j in range(n)]
+    dUs, dSend = [None] * n, [None] * n
+    dS = dST.copy()                                   # dS_{n}
+    dU = xs[-1]["Aq"].T @ dOs[-1] + xs[-1]["Khat"] @ dS
+    for j in range(n - 1, -1, -1):
+        x = xs[j]
+        dUs[j], dSend[j] = dU, dS
+        if j > 0:
+            px = xs[j - 1]
+            Y = px["Khat"] * x["d"][None, :]          # Khat_{j-1} Diag(d_j), off the chain
+            Z = px["Khat"] @ x["W"].T                 # Khat_{j-1} W_j^T, 64 x 64, off the chain
+            base = px["Aq"].T @ dOs[j - 1] + px["Khat"] @ (x["QG"].T @ dOs[j])
+            dU_prev = base + Y @ dS - Z @ dU
+        dS = x["d"][:, None] * dS + x["QG"].T @ dOs[j] - x["W"].T @ dU
+        if j > 0:
+            dU = dU_prev
+    return dUs, dSend, dS
