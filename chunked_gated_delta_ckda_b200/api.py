@@ -14,6 +14,7 @@ torch (device memory is torch's job here) and call the library.
                            saved=sv)                           # packed documents
     x         = prologue_fwd(xq, xk, xv, wq, wk, wv, a, b, g_floor=-5.0)   # q, k, v, g, sign, beta
     grads     = prologue_bwd(xq, xk, xv, wq, wk, wv, a, b, dq, dk, dv, dg, dbeta, g_floor=-5.0)
+    x         = prologue_fwd(..., cu_seqlens=cu)       # packed documents (B = 1): no history across them
 
 Shapes and dtypes are those of include/ckda.h: q, k, g, sign [B,T,H,dk]; v
 [B,T,H,dv]; beta [B,T,H]; g fp32; sign int8 (None: every sign +1, standard
