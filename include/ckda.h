@@ -28,8 +28,9 @@
  *             state (S0, ST, chunk_states, dST, dS0, the decode state) are fp32.
  *             sign is int8 holding +1 or -1 (any other value: undefined
  *             output); a null sign pointer means every sign is +1, i.e.
- *             standard KDA (the same kernels without the sign loads).  g = log|alpha| should be <= 0; the library computes
- *             exactly what it is given, and very negative g (a gate near 0) is
+ *             standard KDA (the same kernels without the sign loads).
+ *             g = log|alpha| should be <= 0; the library computes exactly
+ *             what it is given, and very negative g (a gate near 0) is
  *             supported.
  *  Shapes     dk, dv in {64, 128}; any T >= 0; the chunk length is 64.
  *  States     Every state crossing this ABI is in the true (signed) frame, so
@@ -96,7 +97,8 @@ size_t ckda_workspace_size(int op, int B, int T, int H, int dk, int dv, int N);
 /* Bytes of the "saved" buffer through which ckda_chunk_fwd can hand its
  * per-chunk results (the UT-transform products of every (chunk, head) and
  * the chunk-start states, bf16) to ckda_chunk_bwd, so that the backward
- * recomputes nothing and needs no chunk_states: a memory-for-time trade.  Returns 0 for shapes
+ * recomputes nothing and needs no chunk_states: a memory-for-time trade.
+ * Returns 0 for shapes
  * and dtypes that have no saved form (then `saved` is ignored by both calls
  * and the backward recomputes) and for invalid arguments.  The contents are
  * opaque; they are valid for the inputs of the forward that wrote them. */
