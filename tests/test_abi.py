@@ -2,8 +2,6 @@
 and its host-side argument checks answer without touching a GPU."""
 import ctypes
 
-import pytest
-
 from chunked_gated_delta_ckda_b200 import _abi
 
 P = None

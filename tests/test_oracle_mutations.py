@@ -3,7 +3,6 @@ the pins of test_oracle_pins.py catch every one of them."""
 import os
 import subprocess
 import sys
-import tempfile
 
 import pytest
 
