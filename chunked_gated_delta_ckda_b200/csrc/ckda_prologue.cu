@@ -8,6 +8,7 @@
 // The gate's exact parameterisation and its floor live in an appendix the
 // pages do not contain; these are the readings, stated once in ckda.h:
 //   q, k, v = SiLU(causal depthwise conv of width 4), zero history per sequence
+//             (per document when documents are packed in one row)
 //   q, k   /= sqrt(sum over the head's channels of the square + 1e-6)
 //   alpha   = tanh(a):  g = max(log|alpha|, g_floor),  sign = alpha < 0 ? -1 : +1
 //   beta    = 2 sigmoid(b)
@@ -18,7 +19,8 @@
 // registers, so every input element is read once (plus a three-token halo).
 // The L2 norms need reductions over the head's channels: batched over 8
 // tokens (forward) or 4 (backward) per barrier, so each batch's loads are in
-// flight together.  HBM-bound.
+// flight together.  Its roof is HBM; as measured it is bound by instruction
+// issue (about a third of the HBM roof backward, under half forward).
 #include "ckda_internal.cuh"
 
 namespace ckda {
