@@ -23,6 +23,7 @@ KDA); q, k, v, beta either fp32 or bf16 (all the same); states fp32
 """
 from __future__ import annotations
 
+import functools
 from typing import Optional
 
 import torch
@@ -56,6 +57,27 @@ def workspace(op: int, B: int, T: int, H: int, dk: int, dv: int, N: int = 0,
     if cache:
         _ws_cache[key] = ws
     return ws
+
+
+def _cuda_devices(args, kwargs) -> set:
+    """The devices of the CUDA tensors among a call's arguments."""
+    return {t.device for t in (*args, *kwargs.values()) if getattr(t, "is_cuda", False)}
+
+
+def _one_device(fn):
+    """Every CUDA tensor of the call on one device, made current for the call:
+    the library launches on the current device and torch's current stream, and
+    a pointer into another GPU's memory must never reach its kernels."""
+    @functools.wraps(fn)
+    def call(*args, **kwargs):
+        devices = _cuda_devices(args, kwargs)
+        if len(devices) > 1:
+            raise ValueError("all tensors must be on one CUDA device, got %s" % sorted(map(str, devices)))
+        if not devices:
+            return fn(*args, **kwargs)  # (the argument checks reject it)
+        with torch.cuda.device(devices.pop()):
+            return fn(*args, **kwargs)
+    return call
 
 
 def _c(x: Optional[torch.Tensor]) -> Optional[torch.Tensor]:
@@ -106,6 +128,7 @@ def saved_buffer(B, T, H, dk, dv, dtype, device) -> Optional[torch.Tensor]:
     return torch.empty(n, dtype=torch.uint8, device=device) if n > 0 else None
 
 
+@_one_device
 def chunk_fwd(q, k, v, g, sign, beta, S0=None, output_final_state=True, save_chunk_states=False,
               ws=None, save_for_backward=False):
     B, T = q.shape[:2]
@@ -127,6 +150,7 @@ def chunk_fwd(q, k, v, g, sign, beta, S0=None, output_final_state=True, save_chu
     return o, ST, cs
 
 
+@_one_device
 def chunk_bwd(q, k, v, g, sign, beta, dO, S0=None, dST=None, chunk_states=None, need_dS0=True,
               ws=None, saved=None):
     B, T = q.shape[:2]
@@ -153,6 +177,7 @@ def chunk_bwd(q, k, v, g, sign, beta, dO, S0=None, dST=None, chunk_states=None, 
     return dict(dq=dq, dk=dk_, dv=dv_, dg=dg, dbeta=dbeta, dS0=dS0)
 
 
+@_one_device
 def decode_step(q, k, v, g, sign, beta, state, o=None):
     N = q.shape[0]
     H, dk, dv = _recurrence_inputs(q, k, v, g, sign, beta, (N,))
@@ -167,6 +192,7 @@ def decode_step(q, k, v, g, sign, beta, state, o=None):
     return o
 
 
+@_one_device
 def decode_multi(q, k, v, g, sign, beta, pool, slots=None, n_tokens=None, write_state=True, o=None,
                  want_o=True):
     """K steps per sequence: q, k, g, sign [N,K,H,dk]; v [N,K,H,dv]; beta [N,K,H];
@@ -217,6 +243,7 @@ def _prologue_docs(B, cu_seqlens):
     return _c(cu_seqlens), cu_seqlens.numel() - 1
 
 
+@_one_device
 def prologue_fwd(xq, xk, xv, wq, wk, wv, a, b, g_floor=-5.0, cu_seqlens=None):
     """Projections [B,T,H,d] (io dtype), conv taps [H*d, 4] fp32, gate
     pre-activation a [B,T,H,dk] fp32, b [B,T,H] -> dict q, k, v, g, sign, beta
@@ -235,6 +262,7 @@ def prologue_fwd(xq, xk, xv, wq, wk, wv, a, b, g_floor=-5.0, cu_seqlens=None):
     return out
 
 
+@_one_device
 def prologue_bwd(xq, xk, xv, wq, wk, wv, a, b, dq, dk, dv, dg, dbeta, g_floor=-5.0, cu_seqlens=None):
     """Gradients of prologue_fwd's inputs (same g_floor and cu_seqlens):
     dict dxq, dxk, dxv, dwq, dwk, dwv, da, db."""
@@ -256,6 +284,7 @@ def prologue_bwd(xq, xk, xv, wq, wk, wv, a, b, dq, dk, dv, dg, dbeta, g_floor=-5
     return out
 
 
+@_one_device
 def varlen_fwd(q, k, v, g, sign, beta, cu_seqlens, max_seqlen, S0=None, output_final_state=True,
                ws=None, save_for_backward=False):
     """Packed documents: o [1,T,H,dv], ST [N,H,dk,dv] (or None); with
@@ -285,6 +314,7 @@ def varlen_fwd(q, k, v, g, sign, beta, cu_seqlens, max_seqlen, S0=None, output_f
     return o, ST
 
 
+@_one_device
 def varlen_bwd(q, k, v, g, sign, beta, dO, cu_seqlens, max_seqlen, S0=None, dST=None, need_dS0=True, ws=None,
                saved=None):
     """Gradients of varlen_fwd: dict dq, dk, dv, dg, dbeta, dS0 ([N,H,dk,dv] or

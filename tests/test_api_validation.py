@@ -76,3 +76,24 @@ def test_prologue_arguments_checked():
         api.prologue_fwd(**bad)
     with pytest.raises(ValueError, match="CUDA"):
         api.prologue_fwd(**x)
+
+
+def test_tensors_on_two_devices_are_refused():
+    """A pointer into another GPU's memory must never reach the kernels: the
+    calls refuse CUDA tensors on more than one device before anything else
+    (stand-ins for tensors on cuda:0 and cuda:1; no GPU is touched)."""
+    from types import SimpleNamespace
+    on = lambda i: SimpleNamespace(is_cuda=True, device=torch.device("cuda", i))
+    assert api._cuda_devices((on(0), None, 3, torch.zeros(1)), {"S0": on(0)}) == {torch.device("cuda", 0)}
+    assert len(api._cuda_devices((on(0),), {"S0": on(1)})) == 2
+    seen = []
+    guarded = api._one_device(lambda *a, **k: seen.append(1))
+    with pytest.raises(ValueError, match="one CUDA device"):
+        guarded(on(0), on(1))
+    with pytest.raises(ValueError, match="one CUDA device"):
+        guarded(on(0), ws=on(1))
+    guarded(torch.zeros(1), None)  # host tensors only: passed through (the argument checks refuse them)
+    assert seen == [1]
+    for fn in (api.chunk_fwd, api.chunk_bwd, api.decode_step, api.decode_multi, api.varlen_fwd, api.varlen_bwd,
+               api.prologue_fwd, api.prologue_bwd):
+        assert getattr(fn, "__wrapped__", None) is not None, fn.__name__
