@@ -201,7 +201,9 @@ def ckda_varlen_saved_size(total_T, N, H, dk, dv, io_dtype):
 def ckda_chunk_fwd_noalloc(B, T, H, dk, dv, io_dtype, q, k, v, g, sign, beta, S0, o, ST,
                            chunk_states, stream=None):
     """ckda_chunk_fwd without a workspace: the library's fixed scratch array
-    is used instead (for callers that cannot allocate device memory)."""
+    is used instead (for callers that cannot allocate device memory).  Every
+    pointer must be on the current device and `stream` must belong to it
+    (api.chunk_fwd_noalloc makes the tensors' device current)."""
     _check(_load().ckda_chunk_fwd_noalloc(B, T, H, dk, dv, io_dtype, _p(q), _p(k), _p(v), _p(g),
                                           _p(sign), _p(beta), _p(S0), _p(o), _p(ST),
                                           _p(chunk_states), _s(stream)), "ckda_chunk_fwd_noalloc")

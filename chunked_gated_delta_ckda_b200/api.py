@@ -151,6 +151,24 @@ def chunk_fwd(q, k, v, g, sign, beta, S0=None, output_final_state=True, save_chu
 
 
 @_one_device
+def chunk_fwd_noalloc(q, k, v, g, sign, beta, S0=None, output_final_state=True, save_chunk_states=False):
+    """chunk_fwd for callers that cannot allocate device scratch: the library's
+    fixed scratch array stands in for the workspace (the outputs are still
+    allocated here).  Runs with the tensors' device current and on its current
+    stream, as the C call requires."""
+    B, T = q.shape[:2]
+    H, dk, dv = _recurrence_inputs(q, k, v, g, sign, beta, (B, T))
+    _expect("S0", S0, (B, H, dk, dv), torch.float32, optional=True)
+    q, k, v, g, sign, beta, S0 = map(_c, (q, k, v, g, sign, beta, S0))
+    o = torch.empty(B, T, H, dv, dtype=q.dtype, device=q.device)
+    ST = torch.empty(B, H, dk, dv, dtype=torch.float32, device=q.device) if output_final_state else None
+    cs = (torch.empty(B, H, (T + 63) // 64, dk, dv, dtype=torch.float32, device=q.device)
+          if save_chunk_states else None)
+    _abi.ckda_chunk_fwd_noalloc(B, T, H, dk, dv, io_code(q.dtype), q, k, v, g, sign, beta, S0, o, ST, cs)
+    return o, ST, cs
+
+
+@_one_device
 def chunk_bwd(q, k, v, g, sign, beta, dO, S0=None, dST=None, chunk_states=None, need_dS0=True,
               ws=None, saved=None):
     B, T = q.shape[:2]

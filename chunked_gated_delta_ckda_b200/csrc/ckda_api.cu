@@ -57,35 +57,7 @@ using namespace ckda;
 
 namespace {
 
-bool a16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool a256(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 255u) == 0; }
-bool dim_ok(int d) { return d == 64 || d == 128; }
-
-int check_common(int B, int T, int H, int dk, int dv, int io_dtype) {
-  if (B < 0 || T < 0 || H < 1) return CKDA_ERR_INVALID_ARG;
-  if (io_dtype != CKDA_F32 && io_dtype != CKDA_BF16) return CKDA_ERR_INVALID_ARG;
-  if (!dim_ok(dk) || !dim_ok(dv)) return CKDA_ERR_UNSUPPORTED;
-  // index arithmetic is 64-bit; chunk ids and token offsets are 32-bit
-  if ((int64_t)B * T > INT32_MAX / 2) return CKDA_ERR_UNSUPPORTED;
-  return CKDA_OK;
-}
-
-// sequences (B or N) and heads index grid dimensions limited to 65535
-int check_grid(int B, int H, int N) {
-  if (B > 65535 || H > 65535 || N > 65535) return CKDA_ERR_UNSUPPORTED;
-  return CKDA_OK;
-}
-
-int check_ptrs(std::initializer_list<const void *> required,
-               std::initializer_list<const void *> optional) {
-  for (const void *p : required)
-    if (!p) return CKDA_ERR_INVALID_ARG;
-  for (const void *p : required)
-    if (!a16(p)) return CKDA_ERR_ALIGNMENT;
-  for (const void *p : optional)
-    if (p && !a16(p)) return CKDA_ERR_ALIGNMENT;
-  return CKDA_OK;
-}
 
 int check_ws(const void *ws, size_t ws_bytes, size_t need) {
   if (!ws || ws_bytes < need) return CKDA_ERR_WORKSPACE;

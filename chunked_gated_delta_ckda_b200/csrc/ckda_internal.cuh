@@ -6,6 +6,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <initializer_list>
+
 #include "ckda.h"
 
 namespace ckda {
@@ -133,6 +135,40 @@ __host__ __device__ inline size_t bwd_scratch_floats(int dk, int dv) {
 constexpr int kBwdCtas = 296;  // persistent CTAs of the per-chunk gradient kernel
 
 WsLayout ws_layout(int op, int B, int T, int H, int dk, int dv, int N);
+
+// --------------------------------------------------------------------------
+// Host-side argument checks shared by the entry points (run before anything
+// is enqueued)
+// --------------------------------------------------------------------------
+inline bool a16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// sizes, dtype code and head dimensions
+inline int check_common(int B, int T, int H, int dk, int dv, int io_dtype) {
+  if (B < 0 || T < 0 || H < 1) return CKDA_ERR_INVALID_ARG;
+  if (io_dtype != CKDA_F32 && io_dtype != CKDA_BF16) return CKDA_ERR_INVALID_ARG;
+  if ((dk != 64 && dk != 128) || (dv != 64 && dv != 128)) return CKDA_ERR_UNSUPPORTED;
+  // index arithmetic is 64-bit; chunk ids and token offsets are 32-bit
+  if ((int64_t)B * T > INT32_MAX / 2) return CKDA_ERR_UNSUPPORTED;
+  return CKDA_OK;
+}
+
+// sequences (B or N) and heads index grid dimensions limited to 65535
+inline int check_grid(int B, int H, int N) {
+  if (B > 65535 || H > 65535 || N > 65535) return CKDA_ERR_UNSUPPORTED;
+  return CKDA_OK;
+}
+
+// required pointers non-null and 16-byte aligned; optional ones aligned when given
+inline int check_ptrs(std::initializer_list<const void *> required,
+                      std::initializer_list<const void *> optional) {
+  for (const void *p : required)
+    if (!p) return CKDA_ERR_INVALID_ARG;
+  for (const void *p : required)
+    if (!a16(p)) return CKDA_ERR_ALIGNMENT;
+  for (const void *p : optional)
+    if (p && !a16(p)) return CKDA_ERR_ALIGNMENT;
+  return CKDA_OK;
+}
 
 // --------------------------------------------------------------------------
 // Parameter blocks

@@ -49,44 +49,42 @@ int scratch_address(void **out) {
   return CKDA_OK;
 }
 
-bool a16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
 }  // namespace
 
 using namespace ckda;
+
+#define NOALLOC_TRY(expr)              \
+  do {                                 \
+    const int _rc = (expr);            \
+    if (_rc != CKDA_OK) return _rc;    \
+  } while (0)
 
 extern "C" int ckda_chunk_fwd_noalloc(int B, int T, int H, int dk, int dv, int io_dtype,
                                       const void *q, const void *k, const void *v,
                                       const float *g, const int8_t *sign, const void *beta,
                                       const float *S0, void *o, float *ST,
                                       float *chunk_states, cudaStream_t stream) {
-  if (B < 0 || T < 0 || H < 1) return CKDA_ERR_INVALID_ARG;
-  if (io_dtype != CKDA_F32 && io_dtype != CKDA_BF16) return CKDA_ERR_INVALID_ARG;
-  if ((dk != 64 && dk != 128) || (dv != 64 && dv != 128)) return CKDA_ERR_UNSUPPORTED;
-  // capacity: status block, per-CTA intra scratch, one record per (chunk, head)
+  // the same argument checks as ckda_chunk_fwd, before any size is derived
+  NOALLOC_TRY(check_common(B, T, H, dk, dv, io_dtype));
+  NOALLOC_TRY(check_grid(B, H, 0));
+  if ((int64_t)B * T > 0) NOALLOC_TRY(check_ptrs({q, k, v, g, beta, o}, {sign, S0, ST, chunk_states}));
+  else NOALLOC_TRY(check_ptrs({}, {sign, S0, ST, chunk_states}));
+  // capacity: per-CTA intra scratch, one record per (chunk, head).  The kernels
+  // this call runs have no bounded waits and no device-checked inputs, so it
+  // keeps no device status block.
   const int NC = (T + C - 1) / C;
   const size_t slabs = align256(v1_fwd_scratch_floats_per_cta(dk, dv) * kNoAllocCtas * sizeof(float));
   const size_t records = align256((size_t)B * NC * H * intra_floats(dk, dv) * sizeof(float));
-  const size_t need = align256(sizeof(DevStatus)) + slabs + records;
-  if ((int64_t)B * T > INT32_MAX / 2 || need > (size_t)CKDA_NOALLOC_SCRATCH_BYTES)
-    return CKDA_ERR_NOALLOC_CAPACITY;
-  if ((int64_t)B * T > 0) {
-    const void *req[] = {q, k, v, g, beta, o};  // sign may be null (all +1)
-    for (const void *p : req)
-      if (!p) return CKDA_ERR_INVALID_ARG;
-    for (const void *p : req)
-      if (!a16(p)) return CKDA_ERR_ALIGNMENT;
-  }
-  const void *opt[] = {S0, ST, chunk_states};
-  for (const void *p : opt)
-    if (p && !a16(p)) return CKDA_ERR_ALIGNMENT;
+  if (slabs + records > (size_t)CKDA_NOALLOC_SCRATCH_BYTES) return CKDA_ERR_NOALLOC_CAPACITY;
+  // the scratch address is that of the current device: the stream must belong to it
+  int dev = -1, sdev = -2;
+  if (cudaGetDevice(&dev) != cudaSuccess) return CKDA_ERR_CUDA;
+  if (cudaStreamGetDevice(stream, &sdev) != cudaSuccess) return CKDA_ERR_INVALID_ARG;
+  if (sdev != dev) return CKDA_ERR_INVALID_ARG;
 
   void *base = nullptr;
-  const int rc = scratch_address(&base);
-  if (rc != CKDA_OK) return rc;
+  NOALLOC_TRY(scratch_address(&base));
   char *w = static_cast<char *>(base);
-  // the status block must start at zero; everything else is written before it is read
-  if (cudaMemsetAsync(w, 0, sizeof(DevStatus), stream) != cudaSuccess) return CKDA_ERR_CUDA;
   FwdArgs a{};
   a.B = B; a.T = T; a.H = H; a.dk = dk; a.dv = dv;
   a.q = q; a.k = k; a.v = v; a.beta = beta; a.g = g; a.sign = sign;
@@ -95,9 +93,9 @@ extern "C" int ckda_chunk_fwd_noalloc(int B, int T, int H, int dk, int dv, int i
   a.map.NC = NC;
   a.map.n_seq = B;
   a.map.n_chunks_bound = B * NC;
-  a.status = reinterpret_cast<DevStatus *>(w);
-  float *slab = reinterpret_cast<float *>(w + align256(sizeof(DevStatus)));
-  a.intra = reinterpret_cast<float *>(w + align256(sizeof(DevStatus)) + slabs);
+  a.status = nullptr;
+  float *slab = reinterpret_cast<float *>(w);
+  a.intra = reinterpret_cast<float *>(w + slabs);
   const bool bf16 = io_dtype == CKDA_BF16;
   if (v1_intra_on_ctas(a, bf16, slab, kNoAllocCtas, stream) != cudaSuccess) return CKDA_ERR_CUDA;
   if (v1_state_fwd(a, bf16, true, chunk_states, stream) != cudaSuccess) return CKDA_ERR_CUDA;

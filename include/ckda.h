@@ -298,16 +298,24 @@ int ckda_varlen_bwd(int total_T, int N, const int32_t *cu_seqlens,
  * workspace: scratch comes from one fixed array of CKDA_NOALLOC_SCRATCH_BYTES
  * that the library holds on every GPU that loads it, until the process exits.
  * Nothing is allocated or freed by the call.
- *  - Capacity: one 148 KiB record per (64-token chunk, head) at dk = dv = 128
- *    (72 KiB at 64) plus ~4.7 MiB of fixed scratch must fit: e.g. 194
- *    chunk-heads at d = 128 (B=1, T=4096, H=3).  Larger problems return
- *    CKDA_ERR_NOALLOC_CAPACITY before anything is enqueued.
+ *  - Capacity: the records, one per (64-token chunk, head) -- 147 968 B
+ *    (about 144.5 KiB) at dk = dv = 128, 82 176 B at dk = dv = 64 -- plus
+ *    the intra-chunk kernel's fixed scratch (16 CTAs; 4 718 592 B, 4.5 MiB,
+ *    at d = 128) must fit: at most 194 chunk-heads at d = 128 (e.g. B=1,
+ *    T=4096, H=3, or B=2, T=6208, H=1), 379 at d = 64.  Larger problems
+ *    return CKDA_ERR_NOALLOC_CAPACITY; like every argument error, before
+ *    anything is enqueued.
+ *  - Every pointer must be on the device that is current at the call, and
+ *    `stream` must belong to that device (CKDA_ERR_INVALID_ARG otherwise):
+ *    the scratch array used is the current device's.
  *  - The first call on a device looks up the array's device address
  *    (cudaGetSymbolAddress) with that device current; make that first call
  *    before any stream capture starts.
  *  - Every call uses the same array, which keeps the previous call's
  *    contents; calls whose work may overlap on the GPU (other streams, other
- *    host threads) race on it and must be serialised by the caller. */
+ *    host threads) race on it and must be serialised by the caller.
+ *  - The kernels it runs have no bounded waits and no device-checked inputs:
+ *    there is no device-side status to read for this call. */
 #define CKDA_NOALLOC_SCRATCH_BYTES (32u << 20)
 int ckda_chunk_fwd_noalloc(int B, int T, int H, int dk, int dv, int io_dtype,
                            const void *q, const void *k, const void *v,

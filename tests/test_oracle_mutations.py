@@ -27,6 +27,12 @@ MUTATIONS = {
     "bwd_dbeta_residual": ("db += Gk[j] * r[j];", "db += Gk[j] * v[j];"),
     "bwd_output_term": ("G[i * dv + j] += q[i] * dO[j];", "G[i * dv + j] += q[i] * dO[j] * 0.5;"),
     "bwd_dq_prev_state": ("s += Snew[i * dv + j] * dO[j];", "s += Sprev[i * dv + j] * dO[j];"),
+    "chunk_state_late_snapshot": ("if (p->chunk_states && (t - t0) % p->chunk == 0) {\n"
+                                  "            int64_t c = p->chunk_off[n] + (t - t0) / p->chunk;",
+                                  "if (p->chunk_states && (t - t0 + 1) % p->chunk == 0) {\n"
+                                  "            int64_t c = p->chunk_off[n] + (t - t0 + 1) / p->chunk - 1;"),
+    "chunk_state_sequence_offset": ("int64_t c = p->chunk_off[n] + (t - t0) / p->chunk;",
+                                    "int64_t c = p->chunk_off[n > 0 ? n - 1 : 0] + (t - t0) / p->chunk;"),
     "bwd_checkpoint_off_by_one": ("memcpy(seg, ckpt + s * sz, sizeof(double) * sz);",
                                   "memcpy(seg, ckpt + (s > 0 ? s - 1 : 0) * sz, sizeof(double) * sz);"),
 }

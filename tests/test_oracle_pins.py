@@ -326,6 +326,34 @@ def test_packed_sequences_reset_state():
     assert c == len(cs)
 
 
+def test_chunk_states_are_prefix_final_states():
+    """chunk_states[c] is the state before token j*chunk of its sequence: the
+    final state of the forward over that sequence's first j*chunk tokens (the
+    initial state itself for j = 0), at the global chunk index that counts the
+    earlier sequences' ceil(len / chunk) chunks first."""
+    lens = [37, 16, 1, 50]
+    cu = np.concatenate([[0], np.cumsum(lens)])
+    H, dk, dv, chunk = 2, 4, 3, 16
+    q, k, v, g, sign, beta = rand_inputs(RNG, int(cu[-1]), H, dk, dv)
+    S0 = RNG.standard_normal((len(lens), H, dk, dv))
+    _, _, cs = oracle.fwd(cu, q, k, v, g, sign, beta, S0=S0, chunk=chunk)
+    c = 0
+    for i, L in enumerate(lens):
+        a = cu[i]
+        for j in range((L + chunk - 1) // chunk):
+            n = j * chunk
+            if n == 0:
+                want = S0[i]
+            else:
+                sl = slice(a, a + n)
+                _, want, _ = oracle.fwd([0, n], q[sl], k[sl], v[sl], g[sl], sign[sl], beta[sl],
+                                        S0=S0[i:i + 1])
+                want = want[0]
+            np.testing.assert_array_equal(cs[c], want)
+            c += 1
+    assert c == len(cs)
+
+
 def test_state_continuation():
     T1, T2, H, dk, dv = 37, 50, 2, 4, 6
     q, k, v, g, sign, beta = rand_inputs(RNG, T1 + T2, H, dk, dv)
