@@ -12,6 +12,13 @@ token-mixer layer.  Inputs are
 seeded synthetic tensors (chunked_gated_delta_ckda_b200.workloads), resident
 in HBM when the timed region starts; each step streams ~2 GB, more than L2.
 
+At N=1 the default run also times every secondary workload (decode,
+multi-token decode, packed documents, the long sequence, forward only, KDA,
+the prologue) with fewer steps and its own clock record, in the line's
+"secondary" object (--no-secondary: headline only).  Every value is timed
+with the library's per-launch profiling off; per-kernel times come from a
+separate pass of identical steps.
+
 Prints ONE JSON line (rank 0).  Under torchrun each rank runs its own batch
 (weak scaling, no collective on the data path); ``value`` = tokens of all
 ranks / the slowest rank's device time.
@@ -40,6 +47,7 @@ METRIC_KDA = "KDA (gate sign +1) fwd+bwd tokens/s (H=16,d=128,T=4096,bf16), same
 METRIC_LONG = "CKDA long-sequence fwd+bwd tokens/s (B=1,T=65536,H=16,d=128,bf16, with S0)"
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
+NOMINAL_HBM_GBS = 8000.0  # B200 HBM3e, nominal
 
 # Algorithmic work per token per head (chunk 64, dk = dv = 128; causal masks
 # counted at half; recomputation and padding excluded):
@@ -258,6 +266,20 @@ def _time_steps(step, steps, warmup, world):
     return a.elapsed_time(b) / steps
 
 
+def _profile_pass(step, steps, world):
+    """Per-kernel live times: `steps` identical steps with the library's
+    per-launch CUDA events on (the launch stream's own events).  Returns the
+    per-kernel (launches, total ms) and this pass's ms per step."""
+    from chunked_gated_delta_ckda_b200 import _abi
+    _abi.ckda_profile_reset()
+    _abi.ckda_profile_enable(True)
+    try:
+        ms = _time_steps(step, steps, 0, world)
+    finally:
+        _abi.ckda_profile_enable(False)
+    return _abi.ckda_profile_collect(), ms
+
+
 def run_ours(args, rank, world, local_rank):
     from chunked_gated_delta_ckda_b200 import _abi
     dev = torch.device("cuda", local_rank)
@@ -275,19 +297,19 @@ def run_ours(args, rank, world, local_rank):
 
     clocks = ClockSampler(local_rank)
     clocks.start()
-    _abi.ckda_profile_reset()
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
-    _abi.ckda_profile_enable(True)
+    # the headline: library profiling off, nothing but the step's own launches
     clocks.mark()
     ms = _time_steps(step, args.steps, 0, world)
-    _abi.ckda_profile_enable(False)
-    prof = _abi.ckda_profile_collect()
     clocks.keep_loaded(step)
     clk = clocks.stop()
     ms_max = reduce_max(ms, world)
     value = aggregate(tokens, world, ms_max)
+    # per-kernel breakdown: a separate pass of the same number of identical
+    # steps with a CUDA event pair recorded around every launch
+    prof, ms_prof = _profile_pass(step, args.steps, world)
 
     # dominant kernel, timed live with CUDA events on the launch stream
     peaks = measured_peaks()
@@ -330,6 +352,9 @@ def run_ours(args, rank, world, local_rank):
                             % ((FWD_BYTES + BWD_BYTES) * B * T * H / 1e9),
                       "gate_sign": "none: every sign +1 (standard KDA)" if kda else "int8 +-1 (CKDA)"},
            "roofline": roof, "step_roofline": step_roof, "kernels": kernels,
+           "kernel_times": ("from a separate pass of %d identical steps with a CUDA event pair around every "
+                            "launch (%.4f ms per step there); the headline value is timed without them"
+                            % (args.steps, ms_prof)),
            "gpu_launches": int(sum(n for n, _ in prof.values())), "clocks": clk, "e2e": e2e}
     return out, inp
 
@@ -490,15 +515,12 @@ def run_secondary(args, rank, world, local_rank):
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
-    _abi.ckda_profile_reset()
-    _abi.ckda_profile_enable(True)
     clocks.mark()
-    ms = _time_steps(step, args.steps, 0, world)
-    _abi.ckda_profile_enable(False)
-    prof = _abi.ckda_profile_collect()
+    ms = _time_steps(step, args.steps, 0, world)  # library profiling off
     clocks.keep_loaded(step)
     clk = clocks.stop()
     ms = reduce_max(ms, world)
+    prof, ms_prof = _profile_pass(step, args.steps, world)
     total = sum(t for _, t in prof.values())
     kernels = {k: {"launches": n, "ms_per_launch": t / n, "share": t / total if total else None}
                for k, (n, t) in sorted(prof.items(), key=lambda kv: -kv[1][1])}
@@ -520,8 +542,51 @@ def run_secondary(args, rank, world, local_rank):
                         "algorithmic_bytes_per_launch": alg, "per_unit": "%d %s" % (per_unit, unit_name),
                         "peak_source": peaks["source"]},
            "step_hbm_frac": step_bytes / (peaks["hbm_gbs"] * 1e9) / (ms / 1e3),
-           "kernels": kernels, "gpu_launches": int(sum(n for n, _ in prof.values())), "clocks": clk}
+           "kernels": kernels,
+           "kernel_times": ("from a separate pass of %d identical steps with a CUDA event pair around every "
+                            "launch (%.4f ms per step there); the value is timed without them" % (args.steps, ms_prof)),
+           "gpu_launches": int(sum(n for n, _ in prof.values())), "clocks": clk}
+    if args.workload == "decode":  # the step against the nominal HBM figure too
+        out["step_hbm_frac_nominal"] = step_bytes / (NOMINAL_HBM_GBS * 1e9) / (ms / 1e3)
+        out["step_achieved_gbs"] = step_bytes / (ms / 1e3) / 1e9
     return out
+
+
+# Secondary workloads measured in the default run (after the headline), each
+# with its own clock record: name -> (steps, warm-up) caps
+SECONDARY = (("decode", 64), ("decode_multi", 32), ("varlen", 20), ("varlen_fwdbwd", 10), ("long", 10),
+             ("long_fwdbwd", 6), ("fwd", 20), ("kda", 10), ("prologue", 10))
+
+
+def secondary_suite(args, rank, world, local_rank):
+    """Every secondary workload, timed as its own --workload run would time it
+    (fewer steps), condensed to the figures a reader compares."""
+    res = {}
+    for name, steps in SECONDARY:
+        sub = argparse.Namespace(**{**vars(args), "workload": name, "steps": steps, "warmup": 3, "batch": 0,
+                                    "no_e2e": True})
+        try:
+            if name in ("long_fwdbwd", "kda"):
+                line, _ = run_ours(sub, rank, world, local_rank)
+            else:
+                line = run_secondary(sub, rank, world, local_rank)
+        except Exception as e:  # reported, never fatal to the headline line
+            res[name] = {"error": "%s: %s" % (type(e).__name__, e)}
+            continue
+        r = line.get("roofline") or {}
+        keep = {"metric": line["metric"], "value": line["value"], "unit": line["unit"],
+                "ms_per_step": line["ms_per_step"], "steps": steps, "warmup": 3,
+                "top_kernel": r.get("kernel"), "top_kernel_hbm_frac": r.get("frac"),
+                "top_kernel_achieved_gbs": r.get("achieved"), "clocks": line.get("clocks"),
+                "config": line.get("config")}
+        for key in ("step_hbm_frac", "step_hbm_frac_nominal", "step_achieved_gbs"):
+            if key in line:
+                keep[key] = line[key]
+        if "step_roofline" in line:
+            keep["step_hbm_frac"] = line["step_roofline"]["hbm_frac"]
+        res[name] = keep
+        torch.cuda.empty_cache()
+    return res
 
 
 def run_e2e(inp, dev, args, world):
@@ -724,6 +789,8 @@ def main(argv=None):
     ap.add_argument("--workload", choices=["fwdbwd", "kda", "fwd", "varlen", "varlen_fwdbwd", "long", "long_fwdbwd", "decode",
                              "decode_multi", "prologue"], default="fwdbwd",
                     help="fwdbwd is the headline; the others are secondary measurements")
+    ap.add_argument("--no-secondary", action="store_true",
+                    help="headline only: skip the secondary workloads of the default run")
     ap.add_argument("--batch", type=int, default=0,
                     help="override B (profiling a smaller case; not a bench line)")
     args = ap.parse_args(argv)
@@ -755,6 +822,8 @@ def main(argv=None):
                 print(json.dumps(out), flush=True)
             return 0
         out, inp = run_ours(args, rank, world, local_rank)
+        if world == 1 and args.workload == "fwdbwd" and not args.no_secondary:
+            out["secondary"] = secondary_suite(args, rank, world, local_rank)
         if rank == 0:
             if world == 1 and not args.no_cpu_baseline and args.workload == "fwdbwd":
                 out["cpu_baseline"] = cpu_baseline(inp, W.LAYER_FWDBWD.H)

@@ -531,6 +531,28 @@ def test_full_decode_steps():
     check("state", st_dev, st_ref, w.io_dtype)
 
 
+def test_decode_chain_512_steps():
+    """The recurrent-decode workload's chain length: 512 consecutive single-token
+    calls on fp32 states resident on the device (8 sequences x 16 heads, d=128,
+    bf16 I/O, the decode workload's input generators and N(0, 0.1^2) states),
+    o checked at every step and the state after the last, against the oracle
+    carrying its own fp64 state through the same 512 steps."""
+    w = W.DECODE
+    N, steps = 8, 512
+    state = W.make_decode_state(w, N=N)
+    st_dev = state.cuda()
+    st_ref = f64(state)
+    for t in range(steps):
+        x = W.make_decode_step(w, t, N=N)
+        d = to_dev(x)
+        o = api.decode_step(d["q"], d["k"], d["v"], d["g"], d["sign"], d["beta"], st_dev)
+        o_ref, st_ref = oracle.decode(f64(x["q"]), f64(x["k"]), f64(x["v"]), f64(x["g"]),
+                                      x["sign"].numpy(), f64(x["beta"]), st_ref)
+        torch.cuda.synchronize()
+        check("o[%d]" % t, o, o_ref, w.io_dtype)
+    check("state after %d steps" % steps, st_dev, st_ref, w.io_dtype)
+
+
 # ---------------------------------------------------------------------------
 # token-mixer prologue
 # ---------------------------------------------------------------------------
