@@ -48,6 +48,23 @@ struct BwdTcArgs {
   bool no_tiles;        // provisional pass: no dS / dU tiles
 };
 
+__device__ __forceinline__ void tmem_ld4(uint32_t taddr, float (&v)[4]) {
+  uint32_t r[4];
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(taddr));
+#pragma unroll
+  for (int i = 0; i < 4; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void tmem_st4(uint32_t taddr, const float (&v)[4]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1,%2,%3,%4};" ::"r"(taddr), "r"(__float_as_uint(v[0])),
+               "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])), "r"(__float_as_uint(v[3]))
+               : "memory");
+}
+// one 32-bit column per lane (the whole warp executes it)
+__device__ __forceinline__ void tmem_st1(uint32_t taddr, float v) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(__float_as_uint(v)) : "memory");
+}
 __device__ __forceinline__ void cp_async16(void *smem_dst, const void *gsrc, bool valid) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(smem_dst)), "l"(gsrc),
                "r"(valid ? 16 : 0)
@@ -407,7 +424,7 @@ struct GMisc {
   float beta[64], dbc[64], dbr[4][64];
   float qt[4][128];    // per-quarter totals of g (prep)
   uint8_t qp[4][128];  // per-quarter sign parities (prep)
-  float dd[128];
+  float ddp[8][128];  // partial diag(S_c dS1^T) per eighth of the value channels
 };
 
 // Completion of MMAs (or of a copy only MMAs consume): one thread polls the
@@ -495,7 +512,7 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
     // MMA groups that do not share an accumulator are issued by lane 0 of up
     // to three warps (a tcgen05.mma takes tens of ns to issue): each such
     // barrier counts one commit per issuing thread
-    const uint32_t issuers[7] = {1, 1, 2, 3, 2, 2, 1};
+    const uint32_t issuers[7] = {1, 1, 2, 3, 2, 2, 1};  // (bar[6] is unused)
     for (int i = 0; i < 7; ++i) mbar_init(&ms.bar[i], issuers[i]);
     mbar_init(&ms.mdu, 1);
     mbar_init(&ms.mds, 1);
@@ -536,43 +553,56 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
   // thread 0's count of issued load sets (each completes mld, mrec and mdu
   // once) and of the completions it has seen: an abort drains the rest
   uint32_t n_issued = 0, n_mld = 0, n_mrec = 0, n_mdu = 0;
-  // The copies are spread over lane 0 of warps 0..3 (each copy instruction
-  // takes a while to issue); warp 0 posts every byte count with its arrive,
-  // so the others only add copies (a transiently negative transaction count
-  // is allowed; the phase needs warp 0's arrive to complete).
+  // The copies are spread over lane 0 of all sixteen warps, one each (a copy
+  // instruction takes about 0.1 us to issue, and every warp has the same
+  // share of the final epilogue they overlap); warp 0 posts every byte count
+  // with its arrive, so the others only add copies (a transiently negative
+  // transaction count is allowed; the phase needs warp 0's arrive to complete).
+  // The three byte counts of a load set: posted by thread 0, early (once the
+  // current item's phases of the three barriers have completed) so that the
+  // copy issue at the end of an item is short; a set whose counts were posted
+  // but whose copies were never issued is not waited for on a wind-down.
+  bool posted = false;
+  auto post_bytes = [&]() {
+    mbar_arrive_expect_tx(&ms.mdu, DU_TILE);
+    mbar_arrive_expect_tx(&ms.mrec, W_TILE + M_BYTES + S_TILE);
+    mbar_arrive_expect_tx(&ms.mld, kRowBytesQK + kRowBytesG + (a.sign ? kRowBytesSign : 0) + 2 * 16384);
+  };
   auto issue_loads = [&](int itm) {
     int sq_, len_, jl_;
     int64_t tk_;
     a.map.info(itm / H, sq_, tk_, len_, jl_);
     const int hh = itm % H, t = (int)tk_;
     fence_async_smem();  // earlier generic accesses of the destinations come first
-    if (warp == 0) {
-      ++n_issued;
-      const unsigned char *gdU = ta.dU_tiles + (size_t)itm * DU_TILE;
-      mbar_arrive_expect_tx(&ms.mdu, DU_TILE);
-      mbar_arrive_expect_tx(&ms.mrec, W_TILE + M_BYTES + S_TILE);
-      mbar_arrive_expect_tx(&ms.mld, kRowBytesQK + kRowBytesG + (a.sign ? kRowBytesSign : 0) + 2 * 16384);
-      bulk_g2s(sm + G_OU + 8192, gdU, 8192, &ms.mdu);
-      bulk_g2s(sm + G_OU + 16384 + 8192, gdU + 8192, 8192, &ms.mdu);
-      const unsigned char *rec = ta.recs + (size_t)itm * REC;
-      bulk_g2s(sm + G_WN, rec + R1, W_TILE, &ms.mrec);
-      bulk_g2s(sm + G_MF, rec + R6, M_BYTES, &ms.mrec);
-      bulk_g2s(sm + G_SC, rec + R7, S_TILE, &ms.mrec);
-      // the reverse pass's dS tile is copied in mid-item: have it in L2 by then
-      prefetch_l2(ta.dS_tiles + (size_t)itm * DS_TILE, DS_TILE);
-    } else if (warp == 1) {
-      tma_rows(sm + G_A1 + kStageQ, &ta.rm.q, 0, hh, t, &ms.mld);
-      tma_rows(sm + G_A1 + kStageQ + 8192, &ta.rm.q, 64, hh, t, &ms.mld);
-      tma_rows(sm + G_A1 + kStageK, &ta.rm.k, 0, hh, t, &ms.mld);
-      tma_rows(sm + G_A1 + kStageK + 8192, &ta.rm.k, 64, hh, t, &ms.mld);
-    } else if (warp == 2) {
-      tma_rows(sm + G_B1, &ta.rm.g, 0, hh, t, &ms.mld);
-      if (a.sign) tma_rows(sm + G_TT, &ta.rm.sign, 0, hh, t, &ms.mld);
-      tma_rows(sm + G_UV + 8192, &ta.rm.v, 0, hh, t, &ms.mld);
-      tma_rows(sm + G_UV + 16384 + 8192, &ta.rm.v, 64, hh, t, &ms.mld);
-    } else {
-      tma_rows(sm + G_OU, &ta.rm.dO, 0, hh, t, &ms.mld);
-      tma_rows(sm + G_OU + 16384, &ta.rm.dO, 64, hh, t, &ms.mld);
+    const unsigned char *gdU = ta.dU_tiles + (size_t)itm * DU_TILE;
+    const unsigned char *rec = ta.recs + (size_t)itm * REC;
+    switch (warp) {
+      case 0:
+        ++n_issued;
+        if (!posted) post_bytes();
+        posted = false;
+        bulk_g2s(sm + G_OU + 8192, gdU, 8192, &ms.mdu);
+        break;
+      case 1: bulk_g2s(sm + G_OU + 16384 + 8192, gdU + 8192, 8192, &ms.mdu); break;
+      case 2: bulk_g2s(sm + G_WN, rec + R1, W_TILE, &ms.mrec); break;
+      case 3: bulk_g2s(sm + G_MF, rec + R6, M_BYTES, &ms.mrec); break;
+      case 4: bulk_g2s(sm + G_SC, rec + R7, S_TILE, &ms.mrec); break;
+      case 5: tma_rows(sm + G_A1 + kStageQ, &ta.rm.q, 0, hh, t, &ms.mld); break;
+      case 6: tma_rows(sm + G_A1 + kStageQ + 8192, &ta.rm.q, 64, hh, t, &ms.mld); break;
+      case 7: tma_rows(sm + G_A1 + kStageK, &ta.rm.k, 0, hh, t, &ms.mld); break;
+      case 8: tma_rows(sm + G_A1 + kStageK + 8192, &ta.rm.k, 64, hh, t, &ms.mld); break;
+      case 9: tma_rows(sm + G_B1, &ta.rm.g, 0, hh, t, &ms.mld); break;
+      case 10:
+        if (a.sign) tma_rows(sm + G_TT, &ta.rm.sign, 0, hh, t, &ms.mld);
+        break;
+      case 11: tma_rows(sm + G_UV + 8192, &ta.rm.v, 0, hh, t, &ms.mld); break;
+      case 12: tma_rows(sm + G_UV + 16384 + 8192, &ta.rm.v, 64, hh, t, &ms.mld); break;
+      case 13: tma_rows(sm + G_OU, &ta.rm.dO, 0, hh, t, &ms.mld); break;
+      case 14: tma_rows(sm + G_OU + 16384, &ta.rm.dO, 64, hh, t, &ms.mld); break;
+      default:
+        // the reverse pass's dS tile is copied in mid-item: have it in L2 by then
+        prefetch_l2(ta.dS_tiles + (size_t)itm * DS_TILE, DS_TILE);
+        break;
     }
   };
 
@@ -587,7 +617,7 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
     const unsigned char *gdS = ta.dS_tiles + (size_t)item * DS_TILE;
 
     // ---------------- loads ----------------
-    if (lane == 0 && warp < 4 && it == 0) issue_loads(item);  // later items: during the previous one
+    if (lane == 0 && it == 0) issue_loads(item);  // later items: during the previous one
     // beta rows: loaded here for the first item, during the previous item's
     // final epilogue for the others
     if (it == 0 && tid < 64) ms.beta[tid] = tid < len ? __bfloat162float(beta[(size_t)(tok0 + tid) * H + h]) : 0.f;
@@ -624,7 +654,9 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
         st_bf16(sm + G_KG, mnmaj_off(r, c, 64), kp * el * eGm);
       }
     } else {
-#pragma unroll 1
+      // (unrolled: the prep arrays must stay in registers, which a runtime
+      // index into them would prevent)
+#pragma unroll
       for (int i = 0; i < 16; ++i) {
         const int r = 16 * cq + i;
         const float p = ((P.pre >> i) & 1u) ? -1.f : 1.f;
@@ -692,42 +724,20 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
 #pragma unroll
       for (int i = 0; i < 16; ++i) st_bf16(sm + G_UV, kmaj_off(16 * cq + i, c, 128), u[i]);
     }
-    // dd[c] = sum over v of S_c[c][v] dS1[c][v]: the diagonal of S_c dS1^T, one
-    // MMA from the two transposed tiles (both read MN-major, K = v) into TMEM
-    // columns [256, 384), free until the next products
-    if (!wait_one(&ms.mds, ph, a.status, 404)) { abort = true; break; }
-    if (tid == 0) {
-      tc_fence_after();
-      const uint32_t id = idesc_bf16(128, 128, true, true);
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk)
-        mma_bf16(tmem + 256, sdesc_off(sdesc(sSC, 16384, 1024), kk * 2048), sdesc_off(sdesc(sWN, 16384, 1024), kk * 2048), id,
-                 kk > 0);
-      mma_commit(&ms.bar[6]);
-    }
-    if (!wait_one(&ms.bar[6], ph, a.status, 412)) { abort = true; break; }
-    tc_fence_after();
-    if (cq == 0) {
-      float x[16], y[16];
-      tmem_ld16(lanebase + 256 + 32 * qd, x);
-      tmem_ld16(lanebase + 256 + 32 * qd + 16, y);
-      tmem_wait_ld();
-      float dg = 0.f;
-#pragma unroll
-      for (int k = 0; k < 16; ++k) {
-        dg = (k == lane) ? x[k] : dg;
-        dg = (k + 16 == lane) ? y[k] : dg;
-      }
-      ms.dd[c] = dg;
-    }
     if (!wait_one(&ms.mdu, ph, a.status, 405)) { abort = true; break; }
     ++n_mdu;
+    // the item's phases of mld, mrec and mdu are complete: post the next set's counts
+    if (tid == 0 && item + (int)gridDim.x < nitems) {
+      post_bytes();
+      posted = true;
+    }
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
 
-    // ---------------- [dQG^T | S dU^T], dKhat^T ----------------
-    // (three independent groups, three issuing threads)
+    // ---------------- [dQG^T | S dU^T], dV^T, D7 part 1; then dKhat^T ----------------
+    // (three independent groups, three issuing threads; dKhat^T, the one product
+    // that needs the reverse pass's dS tile, is issued once that tile is in)
     if (tid == 0) {
       tc_fence_after();
       const uint32_t id1 = idesc_bf16(128, 128, true, false);  // S_c read MN-major (K = v)
@@ -738,18 +748,13 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
       mma_commit(&ms.bar[3]);
     } else if (tid == 32) {
       tc_fence_after();
-      const uint32_t id2 = idesc_bf16(128, 64, true, false);   // dS1 read MN-major (K = v)
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk)
-        mma_bf16(tmem + 384, sdesc_off(sdesc(sWN, 16384, 1024), kk * 2048),
-                 sdesc_off(sdesc(sUV, 16, 1024), (kk >> 2) * 16384 + (kk & 3) * 32), id2, kk > 0);
       // dV^T = dU^T T^T (T and dU are in place)
       const uint32_t idT = idesc_bf16(128, 64, true, true);
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)
         mma_bf16(tmem + 448, sdesc_off(sdesc(sOU + 8192, 16384, 1024), kk * 2048),
                  sdesc_off(sdesc(sTT, 8192, 1024), kk * 2048), idT, kk > 0);
-      mma_commit(&ms.bar[3]);
+      // (its commit follows dKhat^T below: one arrival per issuing thread)
     } else if (tid == 64) {
       tc_fence_after();
       // D7, first part: [dO; dU][U; V]^T (needs neither dW nor the epilogue below)
@@ -760,6 +765,33 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
         mma_bf16(tmem + 128, sdesc_off(sdesc(sOU, 16, 1024), ko), sdesc_off(sdesc(sUV, 16, 1024), ko), id3, kk > 0);
       }
       mma_commit(&ms.bar[3]);
+    }
+    // the dS_{c+1} tile is in place (every thread reads it): dKhat^T = dS1^T U^T
+    // on the tensor cores, and meanwhile dd = diag(S_c dS1^T) on the CUDA cores
+    if (!wait_all(&ms.mds, ph, a.status, 404)) { abort = true; break; }
+    if (tid == 32) {
+      tc_fence_after();
+      const uint32_t id2 = idesc_bf16(128, 64, true, false);  // dS1 read MN-major (K = v)
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk)
+        mma_bf16(tmem + 384, sdesc_off(sdesc(sWN, 16384, 1024), kk * 2048),
+                 sdesc_off(sdesc(sUV, 16, 1024), (kk >> 2) * 16384 + (kk & 3) * 32), id2, kk > 0);
+      mma_commit(&ms.bar[3]);
+    }
+    {  // dd[c] = sum over v of S_c[c][v] dS1[c][v] (both tiles K-major [v][c]): this
+      // thread takes channels 2 cp, 2 cp + 1 (one 32-bit word per row) over an
+      // eighth of the v; the eighths are summed in the epilogue
+      const int cp = tid & 63, vg = tid >> 6;
+      float a0 = 0.f, a1 = 0.f;
+#pragma unroll 8
+      for (int v = 16 * vg; v < 16 * vg + 16; ++v) {
+        const uint32_t off = kmaj_off(v, 2 * cp, 128);
+        const float2 sv = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(sm + G_SC + off));
+        const float2 dv2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(sm + G_WN + off));
+        a0 = fmaf(sv.x, dv2.x, a0);
+        a1 = fmaf(sv.y, dv2.y, a1);
+      }
+      *reinterpret_cast<float2 *>(&ms.ddp[vg][2 * cp]) = make_float2(a0, a1);
     }
     if (!wait_one(&ms.bar[3], ph, a.status, 406)) { abort = true; break; }
     tc_fence_after();
@@ -995,7 +1027,8 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
       auto dAv = [&](int r, int s) {  // dA (rows 0..63) / dA_q (rows 64..127) from the bf16 tile
         return __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(sm + G_WN + kmaj_off(r, s, 128)));
       };
-      float x1[16], x2[16], y1[16];
+      // one column per row into TMEM (no register arrays: this rare path must
+      // not raise the register pressure of the common one)
 #pragma unroll 1
       for (int i = 0; i < 16; ++i) {
         const int r = 16 * cq + i;
@@ -1010,20 +1043,17 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
           const float e = expf(Gc[t * D + c] - gr);
           b1 += (dAv(t, r) * kpc[t * D + c] + dAv(64 + t, r) * qpc[t * D + c]) * e;
         }
-        x1[i] = a1;
-        x2[i] = a2;
-        y1[i] = b1;
+        tmem_st1(lanebase + 128 + r, a1);
+        tmem_st1(lanebase + 192 + r, a2);
+        tmem_st1(lanebase + 320 + r, b1);
       }
-      tmem_st16(lanebase + 128 + 16 * cq, x1);
-      tmem_st16(lanebase + 192 + 16 * cq, x2);
-      tmem_st16(lanebase + 320 + 16 * cq, y1);
       tmem_wait_st();
     }
     if (!wait_one(&ms.bar[5], ph, a.status, 408)) { abort = true; break; }
     tc_fence_after();
     // every shared-memory tile is idle now: the next item's loads overlap the
     // final epilogue (TMEM, registers and the quarter sums only)
-    if (lane == 0 && warp < 4 && item + (int)gridDim.x < nitems) issue_loads(item + gridDim.x);
+    if (lane == 0 && item + (int)gridDim.x < nitems) issue_loads(item + gridDim.x);
 
     // ---------------- final elementwise gradients ----------------
     // thread (c, cq): rows 16 cq .. 16 cq + 15 of key channel c, prep values
@@ -1043,48 +1073,81 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
         a.map.info(nxt / H, sq_, tk_, len_, jl_);
         if (tid < len_) beta_next = __bfloat162float(beta[(size_t)(tk_ + tid) * H + nxt % H]);
       }
-      float dgs[16];
-      float gcp = 0.f;
+      float gcp = 0.f, part = 0.f;
       // fast path: the pair terms carry the reference-row scaling; exact path:
       // they are final, and the factors come straight from Gam
       auto rows = [&](auto fast_c) {
         constexpr bool kFast = decltype(fast_c)::value;
 #pragma unroll
-      for (int b8 = 0; b8 < 2; ++b8) {
-        const int r0 = 16 * cq + 8 * b8;
-        float X1[8], X2[8], Y1[8], dQG[8], dKG[8], dKh[8], dVv[8];
-        tmem_ld8(lanebase + 128 + r0, X1);
-        tmem_ld8(lanebase + 192 + r0, X2);
-        tmem_ld8(lanebase + 320 + r0, Y1);
-        tmem_ld8(lanebase + 256 + r0, dQG);
-        tmem_ld8(lanebase + 64 + r0, dKG);
-        tmem_ld8(lanebase + 384 + r0, dKh);
-        tmem_ld8(lanebase + 448 + r0, dVv);
+      // four batches of four rows: seven 4-column loads per batch keep the
+      // accumulators of one batch and the prep values within the registers
+      for (int b4 = 0; b4 < 4; ++b4) {
+        const int r0 = 16 * cq + 4 * b4;
+        float X1[4], X2[4], Y1[4], dQG[4], dKG[4], dKh[4], dVv[4];
+        tmem_ld4(lanebase + 128 + r0, X1);
+        tmem_ld4(lanebase + 192 + r0, X2);
+        tmem_ld4(lanebase + 320 + r0, Y1);
+        tmem_ld4(lanebase + 256 + r0, dQG);
+        tmem_ld4(lanebase + 64 + r0, dKG);
+        tmem_ld4(lanebase + 384 + r0, dKh);
+        tmem_ld4(lanebase + 448 + r0, dVv);
         tmem_wait_ld();
         const size_t off0 = ((size_t)(tok0 + r0) * H + h) * D + c;
+        float dg4[4];  // dL/dGam of the batch's rows: parked in TMEM columns [0, 64) (A is dead)
+        // two rows at a time in packed fp32x2 arithmetic (sm_100 FFMA2 / FMUL2)
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int ii = 8 * b8 + i, r = r0 + i;
-          const float Gr = P.G[ii];
-          const float p = ((P.pre >> ii) & 1u) ? -1.f : 1.f;
-          const float kp = p * bf_lo(P.kq[ii]), qp = p * bf_hi(P.kq[ii]);
-          const float el = kFast ? fast_exp(Gr - P.Gm) : 1.f;
-          const float er = kFast ? rcp_approx(el) : 1.f;
-          const float E = kFast ? el * eGm : fast_exp(Gr);
-          const float eC = kFast ? er * eCm : fast_exp(P.GC - Gr);
-          const float x1 = el * X1[i], x2 = el * X2[i], y1 = er * Y1[i];
-          const float KGv = kp * E, QGv = qp * E, Kh = pCs * kp * eC;
-          const float dkp = x1 + y1 + dKG[i] * E + pCs * dKh[i] * eC;
-          const float dqp = x2 + dQG[i] * E;
-          dgs[ii] = kp * x1 + qp * x2 - kp * y1 + dKG[i] * KGv + dQG[i] * QGv - dKh[i] * Kh;
-          gcp += dKh[i] * Kh;
+        for (int i = 0; i < 4; i += 2) {
+          const int ii = 4 * b4 + i, r = r0 + i;
+          const float2 p2 = make_float2(((P.pre >> ii) & 1u) ? -1.f : 1.f, ((P.pre >> (ii + 1)) & 1u) ? -1.f : 1.f);
+          const float2 kp = __fmul2_rn(p2, make_float2(bf_lo(P.kq[ii]), bf_lo(P.kq[ii + 1])));
+          const float2 qp = __fmul2_rn(p2, make_float2(bf_hi(P.kq[ii]), bf_hi(P.kq[ii + 1])));
+          float2 el, er, E, eC;
+          if (kFast) {
+            el = make_float2(fast_exp(P.G[ii] - P.Gm), fast_exp(P.G[ii + 1] - P.Gm));
+            er = make_float2(rcp_approx(el.x), rcp_approx(el.y));
+            E = __fmul2_rn(el, make_float2(eGm, eGm));
+            eC = __fmul2_rn(er, make_float2(eCm, eCm));
+          } else {
+            el = er = make_float2(1.f, 1.f);
+            E = make_float2(fast_exp(P.G[ii]), fast_exp(P.G[ii + 1]));
+            eC = make_float2(fast_exp(P.GC - P.G[ii]), fast_exp(P.GC - P.G[ii + 1]));
+          }
+          const float2 x1 = __fmul2_rn(el, make_float2(X1[i], X1[i + 1]));
+          const float2 x2 = __fmul2_rn(el, make_float2(X2[i], X2[i + 1]));
+          const float2 y1 = __fmul2_rn(er, make_float2(Y1[i], Y1[i + 1]));
+          const float2 dKG2 = make_float2(dKG[i], dKG[i + 1]), dQG2 = make_float2(dQG[i], dQG[i + 1]);
+          const float2 dKh2 = make_float2(dKh[i], dKh[i + 1]);
+          const float2 Kh = __fmul2_rn(__fmul2_rn(make_float2(pCs, pCs), kp), eC);   // Khat
+          const float2 khd = __fmul2_rn(dKh2, Kh);                                     // dKhat . Khat
+          // dk' = x1 + y1 + dKG E + pC dKhat eC;  dq' = x2 + dQG E
+          const float2 dkp = __ffma2_rn(make_float2(pCs, pCs), __fmul2_rn(dKh2, eC), __ffma2_rn(dKG2, E, __fadd2_rn(x1, y1)));
+          const float2 dqp = __ffma2_rn(dQG2, E, x2);
+          // dL/dGam: k' x1 + q' x2 - k' y1 + dKG KG + dQG QG - dKhat Khat
+          float2 dgv = __fmul2_rn(kp, __fadd2_rn(x1, make_float2(-y1.x, -y1.y)));
+          dgv = __ffma2_rn(qp, x2, dgv);
+          dgv = __ffma2_rn(__fmul2_rn(dKG2, kp), E, dgv);
+          dgv = __ffma2_rn(__fmul2_rn(dQG2, qp), E, dgv);
+          dgv = __fadd2_rn(dgv, make_float2(-khd.x, -khd.y));
+          dg4[i] = dgv.x;
+          dg4[i + 1] = dgv.y;
+          part += dgv.x + dgv.y;
+          gcp += khd.x + khd.y;
+          const float2 oq = __fmul2_rn(p2, dqp), ok = __fmul2_rn(p2, dkp);
+          const __nv_bfloat162 bq = __floats2bfloat162_rn(oq.x, oq.y), bk = __floats2bfloat162_rn(ok.x, ok.y);
+          const __nv_bfloat162 bv = __floats2bfloat162_rn(dVv[i], dVv[i + 1]);  // lane c is value channel c here
+          const size_t off = off0 + i * rstride;
           if (r < len) {
-            const size_t off = off0 + i * rstride;
-            dq[off] = __float2bfloat16_rn(p * dqp);
-            dk[off] = __float2bfloat16_rn(p * dkp);
-            dv[off] = __float2bfloat16_rn(dVv[i]);  // lane c is value channel c here
+            dq[off] = __low2bfloat16(bq);
+            dk[off] = __low2bfloat16(bk);
+            dv[off] = __low2bfloat16(bv);
+          }
+          if (r + 1 < len) {
+            dq[off + rstride] = __high2bfloat16(bq);
+            dk[off + rstride] = __high2bfloat16(bk);
+            dv[off + rstride] = __high2bfloat16(bv);
           }
         }
+        tmem_st4(lanebase + 16 * cq + 4 * b4, dg4);
       }
       };
       if (fast) rows(std::true_type{});
@@ -1092,20 +1155,23 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
       if (tid < 64) ms.beta[tid] = beta_next;  // this item's beta is no longer read
       // reverse in-chunk cumsum of dL/dGam (plus the chunk-end terms) -> dg;
       // the four quarters at once: each starts from the totals of the later ones
-      float part = 0.f;
-#pragma unroll
-      for (int ii = 0; ii < 16; ++ii) part += dgs[ii];
       qsum[cq * D + c] = gcp;
       qsum[4 * D + cq * D + c] = part;
       __syncthreads();
       float gC = 0.f, later = 0.f;
-      const float ddc = ms.dd[c];
+      float ddc = 0.f;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) ddc += ms.ddp[e][c];
 #pragma unroll
       for (int q2 = 0; q2 < 4; ++q2) {
         gC += qsum[q2 * D + c];
         if (q2 > cq) later += qsum[4 * D + q2 * D + c];
       }
       float acc = gC + ddc * dC + later;
+      float dgs[16];
+      tmem_wait_st();
+      tmem_ld16(lanebase + 16 * cq, dgs);
+      tmem_wait_ld();
 #pragma unroll
       for (int ii = 15; ii >= 0; --ii) {
         const int r = 16 * cq + ii;
@@ -1181,6 +1247,9 @@ cudaError_t tc_backward(const BwdArgs &b, const unsigned char *recs, unsigned ch
   e = cudaFuncSetAttribute(tc_grad_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_g);
   if (e != cudaSuccess) return e;
   if (b.map.n_seq == 0) return cudaSuccess;
+  // the row tensors' TMA maps (dO for the reverse pass; all of them for the gradient kernel)
+  e = make_row_maps(ta.rm, b.q, b.k, b.v, b.dO, b.g, b.sign, (int64_t)b.B * b.T, b.H);
+  if (e != cudaSuccess) return e;
   const int G = (seg_ws && !b.map.table) ? tc_seg_count_bwd(b.B, b.H, b.map.NC) : 0;
   if (G >= 2) {
     // long sequences: dS at a segment's start = M_g^T (dS at its end) + e_g, with
@@ -1217,8 +1286,6 @@ cudaError_t tc_backward(const BwdArgs &b, const unsigned char *recs, unsigned ch
     tc_state_bwd_kernel<<<dim3(b.H, b.map.n_seq), kSbThreads, sm_sb, s>>>(ta);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
-  e = make_row_maps(ta.rm, b.q, b.k, b.v, b.dO, b.g, b.sign, (int64_t)b.B * b.T, b.H);
-  if (e != cudaSuccess) return e;
   {
     ProfScope prof("tc_grad", s);
     tc_grad_kernel<<<num_sms(), kGThreads, sm_g, s>>>(ta);
