@@ -553,57 +553,74 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
   // thread 0's count of issued load sets (each completes mld, mrec and mdu
   // once) and of the completions it has seen: an abort drains the rest
   uint32_t n_issued = 0, n_mld = 0, n_mrec = 0, n_mdu = 0;
-  // The copies are spread over lane 0 of all sixteen warps, one each (a copy
-  // instruction takes about 0.1 us to issue, and every warp has the same
-  // share of the final epilogue they overlap); warp 0 posts every byte count
-  // with its arrive, so the others only add copies (a transiently negative
-  // transaction count is allowed; the phase needs warp 0's arrive to complete).
-  // The three byte counts of a load set: posted by thread 0, early (once the
-  // current item's phases of the three barriers have completed) so that the
-  // copy issue at the end of an item is short; a set whose counts were posted
-  // but whose copies were never issued is not waited for on a wind-down.
+  // The next item's copies go out in five stages, each as soon as the regions
+  // it fills are no longer read by the current item, so that the loads spread
+  // over the item instead of piling up at its end:
+  //   0 (after the third MMA group): dU and dO into [dO; dU]; the dS tile into L2
+  //   1 (after the fourth):          S_c^T into the S tile, sign into T
+  //   2 (after the dM M^T products): M
+  //   3 (after dL):                  V into rows 64.. of [U; V]
+  //   4 (after X, Y):                q, k into A1, g into B1 + KG, the W tile
+  // One copy per warp (lane 0) within a stage.  The three byte counts of the
+  // set are posted by thread 0 once the current item's phases of mld, mrec and
+  // mdu have completed; a transiently negative transaction count is allowed
+  // (a phase also needs that arrive).  `staged` counts the stages issued for
+  // the pending set; a wind-down issues the rest first, so that every phase
+  // it waits for completes.
   bool posted = false;
+  int staged = 0, pending_item = -1;
   auto post_bytes = [&]() {
     mbar_arrive_expect_tx(&ms.mdu, DU_TILE);
     mbar_arrive_expect_tx(&ms.mrec, W_TILE + M_BYTES + S_TILE);
     mbar_arrive_expect_tx(&ms.mld, kRowBytesQK + kRowBytesG + (a.sign ? kRowBytesSign : 0) + 2 * 16384);
   };
-  auto issue_loads = [&](int itm) {
+  // copy `w` of stage `st` for item itm (w < number of copies of the stage)
+  auto stage_copy = [&](int st, int w, int itm) {
     int sq_, len_, jl_;
     int64_t tk_;
     a.map.info(itm / H, sq_, tk_, len_, jl_);
     const int hh = itm % H, t = (int)tk_;
-    fence_async_smem();  // earlier generic accesses of the destinations come first
     const unsigned char *gdU = ta.dU_tiles + (size_t)itm * DU_TILE;
     const unsigned char *rec = ta.recs + (size_t)itm * REC;
-    switch (warp) {
-      case 0:
-        ++n_issued;
-        if (!posted) post_bytes();
-        posted = false;
-        bulk_g2s(sm + G_OU + 8192, gdU, 8192, &ms.mdu);
-        break;
-      case 1: bulk_g2s(sm + G_OU + 16384 + 8192, gdU + 8192, 8192, &ms.mdu); break;
-      case 2: bulk_g2s(sm + G_WN, rec + R1, W_TILE, &ms.mrec); break;
-      case 3: bulk_g2s(sm + G_MF, rec + R6, M_BYTES, &ms.mrec); break;
-      case 4: bulk_g2s(sm + G_SC, rec + R7, S_TILE, &ms.mrec); break;
-      case 5: tma_rows(sm + G_A1 + kStageQ, &ta.rm.q, 0, hh, t, &ms.mld); break;
-      case 6: tma_rows(sm + G_A1 + kStageQ + 8192, &ta.rm.q, 64, hh, t, &ms.mld); break;
-      case 7: tma_rows(sm + G_A1 + kStageK, &ta.rm.k, 0, hh, t, &ms.mld); break;
-      case 8: tma_rows(sm + G_A1 + kStageK + 8192, &ta.rm.k, 64, hh, t, &ms.mld); break;
-      case 9: tma_rows(sm + G_B1, &ta.rm.g, 0, hh, t, &ms.mld); break;
-      case 10:
-        if (a.sign) tma_rows(sm + G_TT, &ta.rm.sign, 0, hh, t, &ms.mld);
-        break;
-      case 11: tma_rows(sm + G_UV + 8192, &ta.rm.v, 0, hh, t, &ms.mld); break;
-      case 12: tma_rows(sm + G_UV + 16384 + 8192, &ta.rm.v, 64, hh, t, &ms.mld); break;
-      case 13: tma_rows(sm + G_OU, &ta.rm.dO, 0, hh, t, &ms.mld); break;
-      case 14: tma_rows(sm + G_OU + 16384, &ta.rm.dO, 64, hh, t, &ms.mld); break;
-      default:
-        // the reverse pass's dS tile is copied in mid-item: have it in L2 by then
-        prefetch_l2(ta.dS_tiles + (size_t)itm * DS_TILE, DS_TILE);
-        break;
+    fence_async_smem();  // earlier generic accesses of the destinations come first
+    if (st == 0) {
+      if (w == 0) bulk_g2s(sm + G_OU + 8192, gdU, 8192, &ms.mdu);
+      else if (w == 1) bulk_g2s(sm + G_OU + 16384 + 8192, gdU + 8192, 8192, &ms.mdu);
+      else if (w == 2) tma_rows(sm + G_OU, &ta.rm.dO, 0, hh, t, &ms.mld);
+      else if (w == 3) tma_rows(sm + G_OU + 16384, &ta.rm.dO, 64, hh, t, &ms.mld);
+      else prefetch_l2(ta.dS_tiles + (size_t)itm * DS_TILE, DS_TILE);  // copied in mid-item
+    } else if (st == 1) {
+      if (w == 0) bulk_g2s(sm + G_SC, rec + R7, S_TILE, &ms.mrec);
+      else if (a.sign) tma_rows(sm + G_TT, &ta.rm.sign, 0, hh, t, &ms.mld);
+    } else if (st == 2) {
+      bulk_g2s(sm + G_MF, rec + R6, M_BYTES, &ms.mrec);
+    } else if (st == 3) {
+      tma_rows(sm + G_UV + 8192 + 8192 * w * 2, &ta.rm.v, 64 * w, hh, t, &ms.mld);
+    } else {
+      if (w == 0) bulk_g2s(sm + G_WN, rec + R1, W_TILE, &ms.mrec);
+      else if (w <= 2) tma_rows(sm + G_A1 + kStageQ + 8192 * (w - 1), &ta.rm.q, 64 * (w - 1), hh, t, &ms.mld);
+      else if (w <= 4) tma_rows(sm + G_A1 + kStageK + 8192 * (w - 3), &ta.rm.k, 64 * (w - 3), hh, t, &ms.mld);
+      else tma_rows(sm + G_B1, &ta.rm.g, 0, hh, t, &ms.mld);
     }
+  };
+  constexpr int kStageCopies[5] = {5, 2, 1, 2, 6};
+  // stage st of the next item's set, issued by lane 0 of the first warps
+  auto issue_stage = [&](int st, int itm) {
+    if (tid == 0 && st == 0 && !posted) {  // (the first item: counts not posted yet)
+      post_bytes();
+      posted = true;
+      pending_item = itm;
+    }
+    if (lane == 0 && warp < kStageCopies[st]) stage_copy(st, warp, itm);
+    staged = st + 1;
+    if (st == 4) {
+      if (tid == 0) ++n_issued;
+      posted = false;
+      staged = 0;
+    }
+  };
+  auto issue_loads = [&](int itm) {  // every stage at once (the first item)
+    for (int st = 0; st < 5; ++st) issue_stage(st, itm);
   };
 
   uint32_t it = 0;
@@ -611,13 +628,15 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
   for (int item = blockIdx.x; item < nitems && !abort; item += gridDim.x, ++it) {
     const uint32_t ph = it & 1;
     const int cid = item / H, h = item % H;
+    const int next_item = item + (int)gridDim.x;
+    const bool has_next = next_item < nitems;
     int seq, len, jl;
     int64_t tok0;
     a.map.info(cid, seq, tok0, len, jl);
     const unsigned char *gdS = ta.dS_tiles + (size_t)item * DS_TILE;
 
     // ---------------- loads ----------------
-    if (lane == 0 && it == 0) issue_loads(item);  // later items: during the previous one
+    if (it == 0) issue_loads(item);  // later items: during the previous one
     // beta rows: loaded here for the first item, during the previous item's
     // final epilogue for the others
     if (it == 0 && tid < 64) ms.beta[tid] = tid < len ? __bfloat162float(beta[(size_t)(tok0 + tid) * H + h]) : 0.f;
@@ -727,9 +746,10 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
     if (!wait_one(&ms.mdu, ph, a.status, 405)) { abort = true; break; }
     ++n_mdu;
     // the item's phases of mld, mrec and mdu are complete: post the next set's counts
-    if (tid == 0 && item + (int)gridDim.x < nitems) {
+    if (tid == 0 && has_next) {
       post_bytes();
       posted = true;
+      pending_item = next_item;
     }
     fence_async_smem();
     tc_fence_before();
@@ -795,6 +815,7 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
     }
     if (!wait_one(&ms.bar[3], ph, a.status, 406)) { abort = true; break; }
     tc_fence_after();
+    if (has_next) issue_stage(0, next_item);
     {  // dW = -dU S_c^T -> rows 64..127 of the S_c tile (K-major [i][c]); S_c is dead
       float w[16];
       tmem_ld16(lanebase + 320 + 16 * cq, w);
@@ -827,6 +848,7 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
     }
     if (!wait_one(&ms.bar[4], ph, a.status, 407)) { abort = true; break; }
     tc_fence_after();
+    if (has_next) issue_stage(1, next_item);
     {
       float x[16];
       if (qd < 2) {  // dA_q rows -> bf16 rows 64..127 of the [dA; dA_q] tile; M rows as hi / lo
@@ -905,6 +927,7 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
     }
     if (!wait_one(&ms.bar[0], ph, a.status, 410)) { abort = true; break; }
     tc_fence_after();
+    if (has_next) issue_stage(2, next_item);  // (M was last read by the dbeta column sums above)
     if (qd < 2) {  // tmp rows i (lanes 0..63) -> bf16 hi + lo tiles, K-major [i][k]
       const int i = c;
       float x[16];
@@ -939,6 +962,7 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
     }
     if (!wait_one(&ms.bar[1], ph, a.status, 411)) { abort = true; break; }
     tc_fence_after();
+    if (has_next) issue_stage(3, next_item);
     // dN = strict_lower(dL) -> fp32 (for the dbeta row part) and
     // dA = Diag(beta) dN -> bf16 rows 0..63 of the [dA; dA_q] tile
     if (qd < 2) {
@@ -1053,7 +1077,7 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
     tc_fence_after();
     // every shared-memory tile is idle now: the next item's loads overlap the
     // final epilogue (TMEM, registers and the quarter sums only)
-    if (lane == 0 && item + (int)gridDim.x < nitems) issue_loads(item + gridDim.x);
+    if (has_next) issue_stage(4, next_item);
 
     // ---------------- final elementwise gradients ----------------
     // thread (c, cq): rows 16 cq .. 16 cq + 15 of key channel c, prep values
@@ -1189,6 +1213,13 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
   if (abort && tid == 0) {
     mma_commit(&ms.mfin);
     mbar_wait(&ms.mfin, 0, a.status, 409);
+    // a set whose counts are posted: issue the copies not issued yet, so that
+    // its phases complete, then count it
+    if (posted) {
+      for (int st = staged; st < 5; ++st)
+        for (int w = 0; w < kStageCopies[st]; ++w) stage_copy(st, w, pending_item);
+      ++n_issued;
+    }
     // copies still landing in shared memory finish before the CTA leaves
     for (; n_mld < n_issued; ++n_mld) mbar_wait(&ms.mld, n_mld & 1, a.status, 413);
     for (; n_mrec < n_issued; ++n_mrec) mbar_wait(&ms.mrec, n_mrec & 1, a.status, 414);

@@ -66,7 +66,7 @@ struct IntraMisc {
   uint64_t mbar1, mbar2, mfin, mld;
   uint32_t tmem;
   int flag;
-  float beta[2][64];  // this item's beta rows at [it & 1], the next item's at the other
+  float beta[64];
   PrepTot tot;
 };
 static_assert(I_XS >= I_AQS + 8192 && I_XS + 3 * 16 * 16 * 4 <= I_KG, "inverse scratch in the dead part of B1");
@@ -124,8 +124,6 @@ __global__ void __launch_bounds__(kIntraThreads, 2) tc_intra_kernel(const __grid
   const int nitems = a.map.n_chunks() * H;
   uint32_t it = 0;
   bool abort = false;
-  // next item's row copies: 0 none pending, 1 q, k, sign issued, 2 all issued
-  int ld_pending = 0, pend_item = -1;
   for (int item = blockIdx.x; item < nitems && !abort; item += gridDim.x, ++it) {
     const int cid = item / H, h = item % H;
     int seq, len, jl;
@@ -139,9 +137,7 @@ __global__ void __launch_bounds__(kIntraThreads, 2) tc_intra_kernel(const __grid
     // tile (MN-major A, K = token j, M = value channel: the box layout).
     // (issued from lane 0 of four warps; warp 0 posts the byte count with its
     // arrive, so the phase cannot complete before every copy has landed)
-    // (issued here for the first item only: for every later one, during the
-    // previous item, as soon as each destination is free)
-    if (it == 0 && lane == 0 && warp < 4) {
+    if (lane == 0 && warp < 4) {
       fence_async_smem();  // earlier generic accesses of these regions come first
       const int t = (int)tok0;
       if (warp == 0) {
@@ -159,12 +155,10 @@ __global__ void __launch_bounds__(kIntraThreads, 2) tc_intra_kernel(const __grid
         tma_rows(sm + I_V + 8192, &ta.rm.v, 64, h, t, &ms.mld);
       }
     }
-    float *bcur = ms.beta[it & 1];
-    if (it == 0 && tid < 64) bcur[tid] = tid < len ? __bfloat162float(beta[(size_t)(tok0 + tid) * H + h]) : 0.f;
+    if (tid < 64) ms.beta[tid] = tid < len ? __bfloat162float(beta[(size_t)(tok0 + tid) * H + h]) : 0.f;
     {
       const bool ok = mbar_wait_ool(&ms.mld, it & 1, a.status, 100);
       if (__syncthreads_or(!ok)) { abort = true; break; }
-      ld_pending = 0;
     }
     // ---------------- prep: row-group layout (rows 8w.., channels 4l..) ----------------
     Prep P;
@@ -305,7 +299,7 @@ __global__ void __launch_bounds__(kIntraThreads, 2) tc_intra_kernel(const __grid
       }
       if (L >= 64) {
         const int r = L - 64;
-        const float br = bcur[r];
+        const float br = ms.beta[r];
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
           const int s = 32 * ch + j;
@@ -329,7 +323,7 @@ __global__ void __launch_bounds__(kIntraThreads, 2) tc_intra_kernel(const __grid
             aa += fb[64 * D + r * D + cc] * ks;
             aq += fb[128 * D + r * D + cc] * ks;
           }
-        Nf[r * LDF + s] = s < r ? bcur[r] * aa : 0.f;
+        Nf[r * LDF + s] = s < r ? ms.beta[r] * aa : 0.f;
         st_bf16(sm + I_AQS, kmaj_off(r, s, 64), s <= r ? aq : 0.f);
       }
       fence_async_smem();
@@ -349,8 +343,8 @@ __global__ void __launch_bounds__(kIntraThreads, 2) tc_intra_kernel(const __grid
       uint32_t pk[8];
 #pragma unroll
       for (int m = 0; m < 8; ++m)
-        pk[m] = pack_bf16(Mf[r * LDF + j0 + 2 * m] * bcur[j0 + 2 * m],
-                          Mf[r * LDF + j0 + 2 * m + 1] * bcur[j0 + 2 * m + 1]);
+        pk[m] = pack_bf16(Mf[r * LDF + j0 + 2 * m] * ms.beta[j0 + 2 * m],
+                          Mf[r * LDF + j0 + 2 * m + 1] * ms.beta[j0 + 2 * m + 1]);
       *reinterpret_cast<uint4 *>(sm + I_T + kmaj_off(r, j0, 64)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
       *reinterpret_cast<uint4 *>(sm + I_T + kmaj_off(r, j0 + 8, 64)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
     }
@@ -373,43 +367,11 @@ __global__ void __launch_bounds__(kIntraThreads, 2) tc_intra_kernel(const __grid
       mma_commit(&ms.mbar2);
     }
     {
-      // The next item's rows: its beta into the other beta buffer now (warps 0
-      // and 1, while MMA2 runs); q, k (A1) and sign (T) once MMA2 is done --
-      // A1, B1 and T are dead once this thread's stores of A_q, M and QG^T have
-      // read them -- and g (B1 + KG) and V at the end, once W^T and U0^T have
-      // left KG and V.
-      if (tid < 64 && item + (int)gridDim.x < nitems) {
-        const int nx = item + (int)gridDim.x;
-        int sq_, ln_, jl_;
-        int64_t tk_;
-        a.map.info(nx / H, sq_, tk_, ln_, jl_);
-        ms.beta[(it + 1) & 1][tid] = tid < ln_ ? __bfloat162float(beta[(size_t)(tk_ + tid) * H + nx % H]) : 0.f;
-      }
       bool ok = true;
       if (tid == 0) ok = mbar_wait_ool(&ms.mbar2, it & 1, a.status, 102);
       if (__syncthreads_or(!ok)) { abort = true; break; }
     }
     tc_fence_after();
-    const int nxt = item + (int)gridDim.x;
-    const bool has_next = nxt < nitems;
-    if (has_next && tid == 0) {
-      int sq_, nlen, jl_;
-      int64_t tk_;
-      a.map.info(nxt / H, sq_, tk_, nlen, jl_);
-      const int nh = nxt % H, ntk = (int)tk_;
-      bulk_wait_read_all();
-      fence_async_smem();
-      mbar_arrive_expect_tx(&ms.mld, kRowBytesQK + kRowBytesG + (a.sign ? kRowBytesSign : 0) + 16384);
-      tma_rows(sm + I_A1 + kStageQ, &ta.rm.q, 0, nh, ntk, &ms.mld);
-      tma_rows(sm + I_A1 + kStageQ + 8192, &ta.rm.q, 64, nh, ntk, &ms.mld);
-      tma_rows(sm + I_A1 + kStageK, &ta.rm.k, 0, nh, ntk, &ms.mld);
-      tma_rows(sm + I_A1 + kStageK + 8192, &ta.rm.k, 64, nh, ntk, &ms.mld);
-      if (a.sign) tma_rows(sm + I_T, &ta.rm.sign, 0, nh, ntk, &ms.mld);
-    }
-    if (has_next) {
-      ld_pending = 1;
-      pend_item = nxt;
-    }
     {
       const int qd = warp & 3, ch = warp >> 2;
       const int L = 32 * qd + lane;  // c for W^T, v for U0^T
@@ -449,39 +411,15 @@ __global__ void __launch_bounds__(kIntraThreads, 2) tc_intra_kernel(const __grid
       bulk_s2g(rec + R2, sm + I_US, 16384);
       bulk_commit();
       bulk_wait_read_all();
-      if (has_next) {  // KG and V are free: the next item's g and V
-        int sq_, nlen, jl_;
-        int64_t tk_;
-        a.map.info(nxt / H, sq_, tk_, nlen, jl_);
-        const int nh = nxt % H, ntk = (int)tk_;
-        fence_async_smem();
-        tma_rows(sm + I_B1, &ta.rm.g, 0, nh, ntk, &ms.mld);
-        tma_rows(sm + I_V, &ta.rm.v, 0, nh, ntk, &ms.mld);
-        tma_rows(sm + I_V + 8192, &ta.rm.v, 64, nh, ntk, &ms.mld);
-      }
     }
-    if (has_next) ld_pending = 2;
     __syncthreads();
   }
   if (tid == 0) bulk_wait_all();  // every record tile written before the kernel ends
-  // wind down: make sure no MMA is still writing TMEM before freeing it, and
-  // that a pending set of row copies has landed (its missing copies issued first)
+  // wind down: make sure no MMA is still writing TMEM before freeing it
   if (abort && tid == 32) mma_commit(&ms.mfin);
   if (abort && tid == 0) {
     mma_commit(&ms.mfin);
     mbar_wait_ool(&ms.mfin, 0, a.status, 109);
-    if (ld_pending > 0) {
-      int sq_, ln_, jl_;
-      int64_t tk_;
-      a.map.info(pend_item / H, sq_, tk_, ln_, jl_);
-      const int ph_ = pend_item % H, pt_ = (int)tk_;
-      if (ld_pending == 1) {
-        tma_rows(sm + I_B1, &ta.rm.g, 0, ph_, pt_, &ms.mld);
-        tma_rows(sm + I_V, &ta.rm.v, 0, ph_, pt_, &ms.mld);
-        tma_rows(sm + I_V + 8192, &ta.rm.v, 64, ph_, pt_, &ms.mld);
-      }
-      mbar_wait_ool(&ms.mld, (it + 1) & 1, a.status, 110);
-    }
   }
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, 256);
