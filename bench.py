@@ -79,11 +79,9 @@ KERNEL_UNITS = {
 # DRAM traffic measured by ncu (dram__bytes_read.sum + dram__bytes_write.sum)
 # for the kernel as it stands, per chunk-head, keyed by kernel and workload:
 # captured on a B=2 launch (inputs still larger than L2), traffic being
-# proportional to the chunk-heads a launch processes (profiles/).  Since the
-# capture only the bounded wait's poll limit has changed (a branch that no
-# completed wait takes); no memory access has.
+# proportional to the chunk-heads a launch processes (profiles/).
 NCU_TRAFFIC = {
-    ("tc_grad", "layer_fwdbwd_bf16"): (454119168 + 152589312) / (2 * 64 * 16),
+    ("tc_grad", "layer_fwdbwd_bf16"): (454014464 + 135201536) / (2 * 64 * 16),
 }
 
 
