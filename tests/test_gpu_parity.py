@@ -146,6 +146,32 @@ def test_backward_with_saved_forward_results(with_cs, gscale):
         check(key, a[key], ref[key], io)
 
 
+def test_near_unit_gates_over_a_long_chunk_chain():
+    """g ~ -3e-4 per channel and token (decay ~0.9997) over 4096 tokens = 64
+    chunks: the state forgets almost nothing, so the bf16 operand roundings
+    of every chunk step add up the most here.  The forward (o, final state,
+    chunk states) and the backward through the saved buffer, as the training
+    step runs them, against the oracle."""
+    io = torch.bfloat16
+    B, T, H = 1, 4096, 2
+    inp = random_inputs(B, T, H, 128, 128, io, seed=77, gscale=4e-4)
+    d = to_dev(inp)
+    S0, dST = inp["S0"].cuda(), inp["dST"].cuda()
+    o, ST, cs, sv = api.chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["sign"], d["beta"], S0=S0,
+                                  save_chunk_states=True, save_for_backward=True)
+    got = api.chunk_bwd(d["q"], d["k"], d["v"], d["g"], d["sign"], d["beta"], d["dO"], S0=S0, dST=dST,
+                        saved=sv)
+    torch.cuda.synchronize()
+    o_ref, ST_ref, cs_ref = oracle_fwd_batched(inp, S0=inp["S0"], chunk=64)
+    errs = {"o": check("o", o, o_ref, io), "ST": check("ST", ST, ST_ref, io),
+            "chunk_states": check("chunk_states", cs, cs_ref.reshape(B, T // 64, H, 128, 128).transpose(0, 2, 1, 3, 4),
+                                  io)}
+    ref = oracle_bwd_batched(inp, inp["dO"], S0=inp["S0"], dST=inp["dST"])
+    for key in ("dq", "dk", "dv", "dg", "dbeta", "dS0"):
+        errs[key] = check(key, got[key], ref[key], io)
+    print("relative L2:", {k: "%.2e" % v for k, v in errs.items()})
+
+
 def test_saved_is_ignored_without_a_saved_form():
     io = torch.float32
     inp = random_inputs(1, 100, 2, 64, 64, io, seed=14)
