@@ -430,11 +430,13 @@ __global__ void __launch_bounds__(kIntraThreads, 2) tc_intra_kernel(const __grid
 // ===========================================================================
 constexpr int kStateThreads = 512;   // two warp groups of 256 (two warps per TMEM lane quadrant each)
 constexpr int kGroup = 256;
+constexpr int kTileStorer = 64;      // group A thread that issues the state tiles' bulk stores
 constexpr uint32_t S_REC0 = 0;
 constexpr uint32_t S_REC1 = REC_PAD;
 constexpr uint32_t S_TS = 2 * REC_PAD;          // S^T bf16, K-major [v][c] 128 x 128
 constexpr uint32_t S_TU = S_TS + 32768;         // U^T bf16, K-major [v][s] 128 x 64
-constexpr uint32_t S_MISC = S_TU + 16384;
+constexpr uint32_t S_OST = S_TU + 16384;        // output rows of a chunk, bf16 [64][128] (group B's staging)
+constexpr uint32_t S_MISC = S_OST + 16384;
 
 struct StateMisc {
   uint64_t mrec[2], m3, m4, mfin, sready, sdone;
@@ -563,12 +565,10 @@ __global__ void __launch_bounds__(kStateThreads, 1) tc_state_kernel(TcArgs ta) {
   fence_async_smem();
   tc_fence_before();
   __syncthreads();
-  if (!abort && tid == 0 && nc > 0) {
-    issue_mma3(0);
-    if (ta.state_tiles) {  // S_0 for the backward
-      bulk_s2g(const_cast<unsigned char *>(record(0)) + R7, sm + S_TS, 32768);
-      bulk_commit();
-    }
+  if (!abort && tid == 0 && nc > 0) issue_mma3(0);
+  if (!abort && tid == kTileStorer && nc > 0 && ta.state_tiles) {  // S_0 for the backward
+    bulk_s2g(const_cast<unsigned char *>(record(0)) + R7, sm + S_TS, 32768);
+    bulk_commit();
   }
 
   if (grpA) {
@@ -631,7 +631,7 @@ __global__ void __launch_bounds__(kStateThreads, 1) tc_state_kernel(TcArgs ta) {
         }
         mma_commit(&ms.m4);  // also on failure: the other arrival must not wait on a missing one
       }
-      if (gt == 0) bulk_wait_read_all();  // the last state tile has left S_TS
+      if (tid == kTileStorer) bulk_wait_read_all();  // the last state tile has left S_TS
       if (!wait_a(&ms.m4, j & 1, 204, ok)) { abort = true; break; }
       tc_fence_after();
       // the record buffer is free again: fetch chunk j + 2 into it
@@ -652,20 +652,20 @@ __global__ void __launch_bounds__(kStateThreads, 1) tc_state_kernel(TcArgs ta) {
           *reinterpret_cast<uint4 *>(sm + S_TS + kmaj_off(v, c0 + 8, 128)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
         }
         fence_async_smem();
-        tc_fence_before();
-        if (!wait_a(&ms.mrec[buf ^ 1], ((j + 1) >> 1) & 1, 205, true)) { abort = true; break; }
-        if (gt == 0) {
-          issue_mma3(j + 1);
-          if (ta.state_tiles) {  // S_{j+1} for the backward
-            bulk_s2g(const_cast<unsigned char *>(record(j + 1)) + R7, sm + S_TS, 32768);
-            bulk_commit();
-          }
-        }
       }
-      // S_{j+1} and O_j are in TMEM: hand them to group B
+      // S_{j+1} and O_j are in TMEM, and this warp has read S_{j+1}: hand them
+      // to group B (which scales S^T in place) before the next MMA3 is issued
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&ms.sready);
+      if (j + 1 < nc) {
+        if (!wait_a(&ms.mrec[buf ^ 1], ((j + 1) >> 1) & 1, 205, true)) { abort = true; break; }
+        if (gt == 0) issue_mma3(j + 1);
+        if (tid == kTileStorer && ta.state_tiles) {  // S_{j+1} for the backward (off the MMA issuer)
+          bulk_s2g(const_cast<unsigned char *>(record(j + 1)) + R7, sm + S_TS, 32768);
+          bulk_commit();
+        }
+      }
     }
   } else {
     for (int j = 0; j < nc && !abort; ++j) {
@@ -709,14 +709,26 @@ __global__ void __launch_bounds__(kStateThreads, 1) tc_state_kernel(TcArgs ta) {
       __syncwarp();
       if (lane == 0) mbar_arrive(&ms.sdone);
       if (ta.write_o) {
+        // rows through shared memory ([row][channel], this thread's column v),
+        // then out in 16-byte pieces: a warp writes two whole 256-byte rows per
+        // store instead of 64 bytes of one
+        unsigned char *ost = sm + S_OST;
 #pragma unroll
         for (int i = 0; i < 32; ++i)
-          if (32 * ch + i < len)
-            o[((size_t)(tok0 + 32 * ch + i) * H + h) * D + v] = __float2bfloat16_rn(i < 16 ? ov[i] : ow[i - 16]);
+          *reinterpret_cast<__nv_bfloat16 *>(ost + (uint32_t)((32 * ch + i) * D + v) * 2) =
+              __float2bfloat16_rn(i < 16 ? ov[i] : ow[i - 16]);
+        group_sync(2, kGroup);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int idx = gt + kGroup * k, row = idx >> 4, piece = idx & 15;
+          if (row < len)
+            *reinterpret_cast<uint4 *>(o + ((size_t)(tok0 + row) * H + h) * D + 8 * piece) =
+                *reinterpret_cast<const uint4 *>(ost + row * 256 + 16 * piece);
+        }
       }
     }
   }
-  if (tid == 0) bulk_wait_all();  // every state tile written before the kernel ends
+  if (tid == kTileStorer) bulk_wait_all();  // every state tile written before the kernel ends
   __syncthreads();
   if (abort && tid == 32) mma_commit(&ms.mfin);
   if (abort && tid == 0) {
