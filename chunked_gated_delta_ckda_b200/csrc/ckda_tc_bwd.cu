@@ -78,6 +78,7 @@ __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wai
 // ===========================================================================
 constexpr int kSbThreads = 512;  // two warp groups of 256 (two warps per TMEM lane quadrant each)
 constexpr int kSbGroup = 256;
+constexpr int kSbCopier = 64;  // group A thread that issues the record loads and the dS snapshots
 constexpr uint32_t RB_SIZE = 58368;            // compact record: R1 | R3 | R4 | R5
 constexpr uint32_t RB_R1 = 0, RB_R3 = 32768, RB_R4 = 40960, RB_R5 = 57344;
 constexpr uint32_t SB_RB0 = 0, SB_RB1 = RB_SIZE;
@@ -89,7 +90,7 @@ constexpr uint32_t SB_DUG = SB_DU + 16384;     // dU bf16 K-major [s][v] 64 rows
 constexpr uint32_t SB_MISC = SB_DUG + 16384;
 
 struct SbMisc {
-  uint64_t mrec[2], mu, ms, mfin, dsready, scaled, dudone;
+  uint64_t mrec[2], mdo[2], mu, ms, mfin, dsready, scaled, dudone;
   uint32_t tmem;
 };
 
@@ -103,7 +104,7 @@ struct SbMisc {
 // MMA of step s, and the dU tile out (staged transposed, bulk stored).
 // Hand-offs (one arrive per warp): dsready (A: dS^T has been read), scaled
 // (B: dS^T is scaled), dudone (B: the dU^T buffer has been read).
-__global__ void __launch_bounds__(kSbThreads, 1) tc_state_bwd_kernel(BwdTcArgs ta) {
+__global__ void __launch_bounds__(kSbThreads, 1) tc_state_bwd_kernel(const __grid_constant__ BwdTcArgs ta) {
   extern __shared__ unsigned char smem_raw[];
   unsigned char *sm = reinterpret_cast<unsigned char *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -140,6 +141,8 @@ __global__ void __launch_bounds__(kSbThreads, 1) tc_state_bwd_kernel(BwdTcArgs t
   if (tid == 0) {
     mbar_init(&ms.mrec[0], 1);
     mbar_init(&ms.mrec[1], 1);
+    mbar_init(&ms.mdo[0], 1);
+    mbar_init(&ms.mdo[1], 1);
     mbar_init(&ms.mu, 1);
     mbar_init(&ms.ms, 1);
     mbar_init(&ms.mfin, 1);
@@ -169,18 +172,24 @@ __global__ void __launch_bounds__(kSbThreads, 1) tc_state_bwd_kernel(BwdTcArgs t
     bulk_g2s(dst + RB_R1, src + R1, 32768, &ms.mrec[s & 1]);
     bulk_g2s(dst + RB_R3, src + R3, 25088, &ms.mrec[s & 1]);
   };
-  auto issue_dO = [&](int s) {  // group A
-    const int j = nc - 1 - s;
+  // dO rows of step s (two TMA boxes, K-major SW128 64 x 128) into buffer s & 1,
+  // issued by group B's first thread once that buffer's last readers (the
+  // MMAs of step s - 2) are done; a partial chunk's rows past its end are
+  // zeroed by group A before use
+  auto chunk_len = [&](int s) {
     int sq, len, jl;
     int64_t tok0;
-    a.map.info(first + j, sq, tok0, len, jl);
+    a.map.info(first + nc - 1 - s, sq, tok0, len, jl);
+    return len;
+  };
+  auto issue_dO = [&](int s) {
+    int sq, len, jl;
+    int64_t tok0;
+    a.map.info(first + nc - 1 - s, sq, tok0, len, jl);
     unsigned char *dst = ob[s & 1];
-    for (int e = gt; e < 64 * 16; e += kSbGroup) {
-      const int r = e >> 4, cc = e & 15;
-      const int rr = r < len ? r : 0;
-      cp_async16(dst + kmaj_off(r, cc * 8, 64), dO + ((size_t)(tok0 + rr) * H + h) * D + cc * 8, r < len);
-    }
-    cp_async_commit();
+    mbar_arrive_expect_tx(&ms.mdo[s & 1], 16384);
+    tma_rows(dst, &ta.rm.dO, 0, h, (int)tok0, &ms.mdo[s & 1]);
+    tma_rows(dst + 8192, &ta.rm.dO, 64, h, (int)tok0, &ms.mdo[s & 1]);
   };
   // dL/dS_{c+1} snapshot of chunk j: the bf16 dS^T operand tile as it stands
   // (one bulk store by group A's first thread, after the tile's writers have synchronised)
@@ -194,8 +203,8 @@ __global__ void __launch_bounds__(kSbThreads, 1) tc_state_bwd_kernel(BwdTcArgs t
     issue_record(0);
     if (nc > 1) issue_record(1);
   }
+  if (tid == kSbGroup && nc > 0) issue_dO(0);
   if (grpA) {
-    if (nc > 0) issue_dO(0);
     // dS_T (true frame) -> dS^T rows; bf16 copy for the MMA, fp32 in TMEM
     for (int c0 = 64 * ch; c0 < 64 * ch + 64; c0 += 16) {
       float sv[16];
@@ -218,13 +227,14 @@ __global__ void __launch_bounds__(kSbThreads, 1) tc_state_bwd_kernel(BwdTcArgs t
   fence_async_smem();
   tc_fence_before();
   __syncthreads();
-  if (tid == 0 && nc > 0) snapshot(nc - 1);
+  if (tid == kSbCopier && nc > 0) snapshot(nc - 1);
   if (grpA && nc > 0) {  // dS^T is in place: group B may scale it for step 0
     __syncwarp();
     if (lane == 0) mbar_arrive(&ms.dsready);
   }
 
   bool abort = false;
+  int n_do = (tid == kSbGroup && nc > 0) ? 1 : 0;  // dO loads issued (group B's first thread)
   if (grpA) {
     auto wait_a = [&](uint64_t *bar, uint32_t phase, uint32_t site, bool ok_in) -> bool {
       bool ok = ok_in;
@@ -237,11 +247,13 @@ __global__ void __launch_bounds__(kSbThreads, 1) tc_state_bwd_kernel(BwdTcArgs t
       unsigned char *rec = rb[b];
       unsigned char *ot = ob[b];
       const uint32_t du = 128 + 64 * b;  // dU^T buffer of this step
-      if (s + 1 < nc) issue_dO(s + 1);  // prefetch next dO into the other buffer
-      // dO of this step landed (all but the group just committed)
-      if (s + 1 < nc) asm volatile("cp.async.wait_group 1;" ::: "memory");
-      else cp_async_wait_all();
-      fence_async_smem();
+      const int len_s = chunk_len(s);
+      if (len_s < 64) {  // this step's dO: rows past the chunk are zeros, not the next tokens' rows
+        const bool okd = mbar_wait(&ms.mdo[b], (s >> 1) & 1, a.status, 310);
+        if (group_sync_or(1, kSbGroup, !okd)) { abort = true; break; }
+        zero_tail_rows(ot, 8192, len_s, gt, kSbGroup);
+        fence_async_smem();
+      }
       if (!wait_a(&ms.mrec[b], (s >> 1) & 1, 301, true)) { abort = true; break; }
       // dU^T = dO^T A_q + dS1^T Khat^T
       bool ok = true;
@@ -250,6 +262,7 @@ __global__ void __launch_bounds__(kSbThreads, 1) tc_state_bwd_kernel(BwdTcArgs t
         // rather than the one for step s - 2, whose buffer this step reuses,
         // keeps the parity wait unambiguous: B cannot run two steps ahead)
         if (s >= 1) ok = mbar_wait(&ms.dudone, (s - 1) & 1, a.status, 304);
+        if (ok && len_s == 64) ok = mbar_wait(&ms.mdo[b], (s >> 1) & 1, a.status, 310);  // this step's dO
         if (ok) {
           tc_fence_after();
           const uint32_t sO = smem_u32(ot), sRec = smem_u32(rec), sDS = smem_u32(sm + SB_DS);
@@ -300,11 +313,11 @@ __global__ void __launch_bounds__(kSbThreads, 1) tc_state_bwd_kernel(BwdTcArgs t
             mma_bf16(tmem, sdesc_off(sdesc(sDU, 16, 1024), kk * 32), sdesc_off(sdesc(sRec + RB_R1, 16, 1024), kk * 32), id2, true);
           mma_commit(&ms.ms);
         }
-        bulk_wait_read_all();  // the last snapshot has left the dS^T tile
       }
+      if (tid == kSbCopier) bulk_wait_read_all();  // the last snapshot has left the dS^T tile
       if (!wait_a(&ms.ms, s & 1, 303, ok)) { abort = true; break; }
       tc_fence_after();
-      if (gt == 0 && s + 2 < nc) issue_record(s + 2);
+      if (tid == kSbCopier && s + 2 < nc) issue_record(s + 2);
       // dS at the start of chunk j: next step's operand, snapshot of chunk j-1, or dS0
       for (int c0 = 64 * ch; c0 < 64 * ch + 64; c0 += 16) {
         float sv[16];
@@ -323,14 +336,13 @@ __global__ void __launch_bounds__(kSbThreads, 1) tc_state_bwd_kernel(BwdTcArgs t
       }
       fence_async_smem();
       tc_fence_before();
-      group_sync(1, kSbGroup);
-      if (gt == 0 && j > 0) snapshot(j - 1);
       if (j > 0) {  // dS^T has been read: group B may scale it for the next step
         __syncwarp();
         if (lane == 0) mbar_arrive(&ms.dsready);
       }
+      group_sync(1, kSbGroup);
+      if (tid == kSbCopier && j > 0) snapshot(j - 1);
     }
-    cp_async_wait_all();
   } else {
     for (int s = 0; s < nc && !abort; ++s) {
       const int b = s & 1;
@@ -339,6 +351,11 @@ __global__ void __launch_bounds__(kSbThreads, 1) tc_state_bwd_kernel(BwdTcArgs t
       bool ok = mbar_wait(&ms.dsready, s & 1, a.status, 306);
       if (ok) ok = mbar_wait(&ms.mrec[b], (s >> 1) & 1, a.status, 307);
       if (group_sync_or(2, kSbGroup, !ok)) { abort = true; break; }
+      // the MMAs of step s - 1 are done (dsready): the next step's dO into their buffer
+      if (gt == 0 && s + 1 < nc) {
+        issue_dO(s + 1);
+        ++n_do;
+      }
       tc_fence_after();
       {
         const float *dj = reinterpret_cast<const float *>(rb[b] + RB_R5);
@@ -379,7 +396,11 @@ __global__ void __launch_bounds__(kSbThreads, 1) tc_state_bwd_kernel(BwdTcArgs t
       }
     }
   }
-  if (gt == 0) bulk_wait_all();  // every tile written before the kernel ends
+  if (gt == 0 || tid == kSbCopier) bulk_wait_all();  // every tile written before the kernel ends
+  // dO rows still landing (after an abort) finish before the CTA leaves: the
+  // last load into each buffer (at most one per buffer is outstanding)
+  if (tid == kSbGroup)
+    for (int k = n_do > 2 ? n_do - 2 : 0; k < n_do; ++k) mbar_wait(&ms.mdo[k & 1], (k >> 1) & 1, a.status, 311);
   __syncthreads();
   if (abort && tid == 0) {
     mma_commit(&ms.mfin);
