@@ -78,7 +78,7 @@ __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wai
 // ===========================================================================
 constexpr int kSbThreads = 512;  // two warp groups of 256 (two warps per TMEM lane quadrant each)
 constexpr int kSbGroup = 256;
-constexpr int kSbCopier = 64;  // group A thread that issues the record loads and the dS snapshots
+constexpr int kSbCopier = 64;  // group A thread that issues the first dS snapshot (the others: group B)
 constexpr uint32_t RB_SIZE = 58368;            // compact record: R1 | R3 | R4 | R5
 constexpr uint32_t RB_R1 = 0, RB_R3 = 32768, RB_R4 = 40960, RB_R5 = 57344;
 constexpr uint32_t SB_RB0 = 0, SB_RB1 = RB_SIZE;
@@ -317,7 +317,6 @@ __global__ void __launch_bounds__(kSbThreads, 1) tc_state_bwd_kernel(const __gri
       if (tid == kSbCopier) bulk_wait_read_all();  // the last snapshot has left the dS^T tile
       if (!wait_a(&ms.ms, s & 1, 303, ok)) { abort = true; break; }
       tc_fence_after();
-      if (tid == kSbCopier && s + 2 < nc) issue_record(s + 2);
       // dS at the start of chunk j: next step's operand, snapshot of chunk j-1, or dS0
       for (int c0 = 64 * ch; c0 < 64 * ch + 64; c0 += 16) {
         float sv[16];
@@ -341,7 +340,6 @@ __global__ void __launch_bounds__(kSbThreads, 1) tc_state_bwd_kernel(const __gri
         if (lane == 0) mbar_arrive(&ms.dsready);
       }
       group_sync(1, kSbGroup);
-      if (tid == kSbCopier && j > 0) snapshot(j - 1);
     }
   } else {
     for (int s = 0; s < nc && !abort; ++s) {
@@ -351,10 +349,17 @@ __global__ void __launch_bounds__(kSbThreads, 1) tc_state_bwd_kernel(const __gri
       bool ok = mbar_wait(&ms.dsready, s & 1, a.status, 306);
       if (ok) ok = mbar_wait(&ms.mrec[b], (s >> 1) & 1, a.status, 307);
       if (group_sync_or(2, kSbGroup, !ok)) { abort = true; break; }
-      // the MMAs of step s - 1 are done (dsready): the next step's dO into their buffer
-      if (gt == 0 && s + 1 < nc) {
-        issue_dO(s + 1);
-        ++n_do;
+      // the MMAs of step s - 1 are done (dsready): the next step's dO into their
+      // buffer, the next record but one into the slot of step s - 1, and the
+      // dL/dS snapshot of the tile group A has just written (the chain's copies,
+      // issued off the chain)
+      if (gt == 0) {
+        if (s + 1 < nc) {
+          issue_dO(s + 1);
+          ++n_do;
+        }
+        if (s >= 1 && s + 1 < nc) issue_record(s + 1);
+        if (s >= 1) snapshot(nc - 1 - s);
       }
       tc_fence_after();
       {
@@ -369,6 +374,7 @@ __global__ void __launch_bounds__(kSbThreads, 1) tc_state_bwd_kernel(const __gri
         }
         tmem_wait_st();
       }
+      if (gt == 0) bulk_wait_read_all();  // the snapshot has left the dS^T tile (group A rewrites it after scaled)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&ms.scaled);
