@@ -257,26 +257,27 @@ __global__ void __launch_bounds__(kSbThreads, 1) tc_state_bwd_kernel(const __gri
       if (!wait_a(&ms.mrec[b], (s >> 1) & 1, 301, true)) { abort = true; break; }
       // dU^T = dO^T A_q + dS1^T Khat^T
       bool ok = true;
-      if (gt == 0) {
+      if (warp == 0) {  // the whole warp; one elected lane issues
         // group B has read the dU^T of step s - 1 (waiting for that completion
         // rather than the one for step s - 2, whose buffer this step reuses,
         // keeps the parity wait unambiguous: B cannot run two steps ahead)
         if (s >= 1) ok = mbar_wait(&ms.dudone, (s - 1) & 1, a.status, 304);
         if (ok && len_s == 64) ok = mbar_wait(&ms.mdo[b], (s >> 1) & 1, a.status, 310);  // this step's dO
+        ok = __all_sync(0xffffffffu, ok);
         if (ok) {
           tc_fence_after();
           const uint32_t sO = smem_u32(ot), sRec = smem_u32(rec), sDS = smem_u32(sm + SB_DS);
           const uint32_t id1 = idesc_bf16(128, 64, true, true);
           const uint32_t id2 = idesc_bf16(128, 64, false, true);
+          const uint64_t dO_ = sdesc(sO, 8192, 1024), dAq = sdesc(sRec + RB_R3, 8192, 1024);
+          const uint64_t dDS = sdesc(sDS, 16, 1024), dKh = sdesc(sRec + RB_R4, 8192, 1024);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            mma_bf16(tmem + du, sdesc_off(sdesc(sO, 8192, 1024), kk * 2048), sdesc_off(sdesc(sRec + RB_R3, 8192, 1024), kk * 2048),
-                     id1, kk > 0);
+            mma_bf16_warp(tmem + du, sdesc_off(dO_, kk * 2048), sdesc_off(dAq, kk * 2048), id1, kk > 0);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            mma_bf16(tmem + du, sdesc_off(sdesc(sDS, 16, 1024), (kk >> 2) * 16384 + (kk & 3) * 32),
-                     sdesc_off(sdesc(sRec + RB_R4, 8192, 1024), kk * 2048), id2, true);
-          mma_commit(&ms.mu);
+            mma_bf16_warp(tmem + du, sdesc_off(dDS, (kk >> 2) * 16384 + (kk & 3) * 32), sdesc_off(dKh, kk * 2048), id2, true);
+          mma_commit_warp(&ms.mu);
         }
       }
       if (!wait_a(&ms.mu, s & 1, 302, ok)) { abort = true; break; }
@@ -297,21 +298,21 @@ __global__ void __launch_bounds__(kSbThreads, 1) tc_state_bwd_kernel(const __gri
       group_sync(1, kSbGroup);
       // dS^T += dO^T QG - dU^T W  (dS^T scaled by group B first)
       ok = true;
-      if (gt == 0) {
+      if (warp == 0) {
         ok = mbar_wait(&ms.scaled, s & 1, a.status, 305);
+        ok = __all_sync(0xffffffffu, ok);
         if (ok) {
           tc_fence_after();
           const uint32_t sO = smem_u32(ot), sRec = smem_u32(rec), sDU = smem_u32(sm + SB_DU);
           const uint32_t id1 = idesc_bf16(128, 128, true, false);
           const uint32_t id2 = idesc_bf16(128, 128, false, false) | (1u << 13);  // negate A
+          const uint64_t dO_ = sdesc(sO, 8192, 1024), dQG = sdesc(sRec + RB_R1 + 16384, 16, 1024);
+          const uint64_t dDU = sdesc(sDU, 16, 1024), dW = sdesc(sRec + RB_R1, 16, 1024);
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_bf16(tmem, sdesc_off(sdesc(sO, 8192, 1024), kk * 2048), sdesc_off(sdesc(sRec + RB_R1 + 16384, 16, 1024), kk * 32),
-                     id1, true);
+          for (int kk = 0; kk < 4; ++kk) mma_bf16_warp(tmem, sdesc_off(dO_, kk * 2048), sdesc_off(dQG, kk * 32), id1, true);
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_bf16(tmem, sdesc_off(sdesc(sDU, 16, 1024), kk * 32), sdesc_off(sdesc(sRec + RB_R1, 16, 1024), kk * 32), id2, true);
-          mma_commit(&ms.ms);
+          for (int kk = 0; kk < 4; ++kk) mma_bf16_warp(tmem, sdesc_off(dDU, kk * 32), sdesc_off(dW, kk * 32), id2, true);
+          mma_commit_warp(&ms.ms);
         }
       }
       if (tid == kSbCopier) bulk_wait_read_all();  // the last snapshot has left the dS^T tile
@@ -408,8 +409,8 @@ __global__ void __launch_bounds__(kSbThreads, 1) tc_state_bwd_kernel(const __gri
   if (tid == kSbGroup)
     for (int k = n_do > 2 ? n_do - 2 : 0; k < n_do; ++k) mbar_wait(&ms.mdo[k & 1], (k >> 1) & 1, a.status, 311);
   __syncthreads();
-  if (abort && tid == 0) {
-    mma_commit(&ms.mfin);
+  if (abort && warp == 0) {  // the MMAs of warp 0 (issued by its elected lane) done
+    mma_commit_warp(&ms.mfin);
     mbar_wait(&ms.mfin, 0, a.status, 309);
   }
   __syncthreads();

@@ -514,15 +514,16 @@ __global__ void __launch_bounds__(kStateThreads, 1) tc_state_kernel(TcArgs ta) {
   auto record = [&](int j) -> const unsigned char * {
     return ta.recs + ((size_t)(first + j) * H + h) * REC;
   };
-  auto issue_mma3 = [&](int j) {
+  auto issue_mma3 = [&](int j) {  // by a whole warp
     tc_fence_after();
     const uint32_t id = idesc_bf16(128, 128, false, true);
-    const uint32_t sS = smem_u32(sm + S_TS), sR = smem_u32(recbuf[j & 1] + R1);
+    const uint32_t sS = smem_u32(sm + S_TS), sR = smem_u32(sm + (j & 1) * S_REC1 + R1);
+    const uint64_t dA = sdesc(sS, 16, 1024), dB = sdesc(sR, 16384, 1024);
 #pragma unroll
     for (int kk = 0; kk < 8; ++kk)
-      mma_bf16(tmem + 128 + 128 * (j & 1), sdesc_off(sdesc(sS, 16, 1024), (kk >> 2) * 16384 + (kk & 3) * 32),
-               sdesc_off(sdesc(sR, 16384, 1024), kk * 2048), id, kk > 0);
-    mma_commit(&ms.m3);
+      mma_bf16_warp(tmem + 128 + 128 * (j & 1), sdesc_off(dA, (kk >> 2) * 16384 + (kk & 3) * 32),
+                    sdesc_off(dB, kk * 2048), id, kk > 0);
+    mma_commit_warp(&ms.m3);
   };
   if (tid == 0) {
     for (int j = 0; j < 2 && j < nc; ++j) {
@@ -565,7 +566,7 @@ __global__ void __launch_bounds__(kStateThreads, 1) tc_state_kernel(TcArgs ta) {
   fence_async_smem();
   tc_fence_before();
   __syncthreads();
-  if (!abort && tid == 0 && nc > 0) issue_mma3(0);
+  if (!abort && warp == 0 && nc > 0) issue_mma3(0);
   if (!abort && tid == kTileStorer && nc > 0 && ta.state_tiles) {  // S_0 for the backward
     bulk_s2g(const_cast<unsigned char *>(record(0)) + R7, sm + S_TS, 32768);
     bulk_commit();
@@ -607,29 +608,28 @@ __global__ void __launch_bounds__(kStateThreads, 1) tc_state_kernel(TcArgs ta) {
       fence_async_smem();
       tc_fence_before();
       group_sync(1, kGroup);
-      // MMA4: O^T += U^T A_q^T (second thread, at once); MMA5: S^T += U^T Khat
-      // (this group's first thread, once group B has scaled S^T)
+      // MMA4: O^T += U^T A_q^T (warp 1, at once); MMA5: S^T += U^T Khat (warp 0,
+      // once group B has scaled S^T); each issued by one elected lane of its warp
       bool ok = true;
-      if (gt == 32) {
+      if (warp == 1) {
         tc_fence_after();
         const uint32_t id4 = idesc_bf16(128, 64, false, false);
+        const uint64_t dA = sdesc(smem_u32(sm + S_TU), 16, 1024), dB = sdesc(smem_u32(rec + R3), 16, 1024);
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_bf16(tmem + acc + 64, sdesc_off(sdesc(smem_u32(sm + S_TU), 16, 1024), kk * 32),
-                   sdesc_off(sdesc(smem_u32(rec + R3), 16, 1024), kk * 32), id4, true);
-        mma_commit(&ms.m4);
+        for (int kk = 0; kk < 4; ++kk) mma_bf16_warp(tmem + acc + 64, sdesc_off(dA, kk * 32), sdesc_off(dB, kk * 32), id4, true);
+        mma_commit_warp(&ms.m4);
       }
-      if (gt == 0) {
+      if (warp == 0) {
         if (j > 0) ok = mbar_wait(&ms.sdone, (j - 1) & 1, a.status, 206);
+        ok = __all_sync(0xffffffffu, ok);  // (the same lane issues and commits)
         if (ok) {
           tc_fence_after();
           const uint32_t id5 = idesc_bf16(128, 128, false, false);
+          const uint64_t dA = sdesc(smem_u32(sm + S_TU), 16, 1024), dB = sdesc(smem_u32(rec + R4), 16, 1024);
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_bf16(tmem + 0, sdesc_off(sdesc(smem_u32(sm + S_TU), 16, 1024), kk * 32),
-                     sdesc_off(sdesc(smem_u32(rec + R4), 16, 1024), kk * 32), id5, true);
+          for (int kk = 0; kk < 4; ++kk) mma_bf16_warp(tmem + 0, sdesc_off(dA, kk * 32), sdesc_off(dB, kk * 32), id5, true);
         }
-        mma_commit(&ms.m4);  // also on failure: the other arrival must not wait on a missing one
+        mma_commit_warp(&ms.m4);  // also on failure: the other arrival must not wait on a missing one
       }
       if (tid == kTileStorer) bulk_wait_read_all();  // the last state tile has left S_TS
       if (!wait_a(&ms.m4, j & 1, 204, ok)) { abort = true; break; }
@@ -660,7 +660,7 @@ __global__ void __launch_bounds__(kStateThreads, 1) tc_state_kernel(TcArgs ta) {
       if (lane == 0) mbar_arrive(&ms.sready);
       if (j + 1 < nc) {
         if (!wait_a(&ms.mrec[buf ^ 1], ((j + 1) >> 1) & 1, 205, true)) { abort = true; break; }
-        if (gt == 0) issue_mma3(j + 1);
+        if (warp == 0) issue_mma3(j + 1);
         if (tid == kTileStorer && ta.state_tiles) {  // S_{j+1} for the backward (off the MMA issuer)
           bulk_s2g(const_cast<unsigned char *>(record(j + 1)) + R7, sm + S_TS, 32768);
           bulk_commit();
@@ -730,9 +730,10 @@ __global__ void __launch_bounds__(kStateThreads, 1) tc_state_kernel(TcArgs ta) {
   }
   if (tid == kTileStorer) bulk_wait_all();  // every state tile written before the kernel ends
   __syncthreads();
-  if (abort && tid == 32) mma_commit(&ms.mfin);
-  if (abort && tid == 0) {
-    mma_commit(&ms.mfin);
+  // wind down: the MMAs of warps 0 and 1 (issued by their elected lanes) done
+  if (abort && warp == 1) mma_commit_warp(&ms.mfin);
+  if (abort && warp == 0) {
+    mma_commit_warp(&ms.mfin);
     mbar_wait(&ms.mfin, 0, a.status, 209);
   }
   __syncthreads();
