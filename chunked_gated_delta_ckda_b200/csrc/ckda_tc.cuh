@@ -302,6 +302,8 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t *>(&v);
 }
+// the 32 bits of a bf16 pair
+__device__ __forceinline__ uint32_t bf162_bits(__nv_bfloat162 v) { return *reinterpret_cast<uint32_t *>(&v); }
 // x = hi + lo with hi = bf16(x) and lo = bf16(x - hi): a pair of bf16 values
 // that carries ~16 significant bits into a tensor-core product
 __device__ __forceinline__ void split_bf16x2(float a, float b, uint32_t &hi, uint32_t &lo) {

@@ -1187,16 +1187,18 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
           const float2 oq = __fmul2_rn(p2, dqp), ok = __fmul2_rn(p2, dkp);
           const __nv_bfloat162 bq = __floats2bfloat162_rn(oq.x, oq.y), bk = __floats2bfloat162_rn(ok.x, ok.y);
           const __nv_bfloat162 bv = __floats2bfloat162_rn(dVv[i], dVv[i + 1]);  // lane c is value channel c here
-          const size_t off = off0 + i * rstride;
-          if (r < len) {
-            dq[off] = __low2bfloat16(bq);
-            dk[off] = __low2bfloat16(bk);
-            dv[off] = __low2bfloat16(bv);
-          }
-          if (r + 1 < len) {
-            dq[off + rstride] = __high2bfloat16(bq);
-            dk[off + rstride] = __high2bfloat16(bk);
-            dv[off + rstride] = __high2bfloat16(bv);
+          // lanes 2k, 2k + 1 (channels c, c ^ 1) swap halves: the even lane
+          // then holds row r of both channels, the odd one row r + 1, and one
+          // 4-byte store per lane writes two rows per warp instruction
+          const uint32_t pq = bf162_bits(bq), pk = bf162_bits(bk), pv = bf162_bits(bv);
+          const uint32_t xq = __shfl_xor_sync(0xffffffffu, pq, 1), xk = __shfl_xor_sync(0xffffffffu, pk, 1);
+          const uint32_t xv = __shfl_xor_sync(0xffffffffu, pv, 1);
+          const bool odd = lane & 1;
+          const size_t off = off0 + i * rstride + (odd ? rstride - 1 : 0);  // (row r + 1, channel c - 1) on odd lanes
+          if ((odd ? r + 1 : r) < len) {
+            *reinterpret_cast<uint32_t *>(dq + off) = odd ? __byte_perm(xq, pq, 0x7632) : __byte_perm(pq, xq, 0x5410);
+            *reinterpret_cast<uint32_t *>(dk + off) = odd ? __byte_perm(xk, pk, 0x7632) : __byte_perm(pk, xk, 0x5410);
+            *reinterpret_cast<uint32_t *>(dv + off) = odd ? __byte_perm(xv, pv, 0x7632) : __byte_perm(pv, xv, 0x5410);
           }
         }
         tmem_st4(lanebase + 16 * cq + 4 * b4, dg4);
@@ -1226,9 +1228,22 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
       tmem_wait_ld();
 #pragma unroll
       for (int ii = 15; ii >= 0; --ii) {
-        const int r = 16 * cq + ii;
         acc += dgs[ii];
-        if (r < len) a.dg[((size_t)(tok0 + r) * H + h) * D + c] = acc;
+        dgs[ii] = acc;
+      }
+      // the same pairing as above, 8 bytes per lane: rows 2m (even lanes) and
+      // 2m + 1 (odd lanes) of channels c & ~1, c | 1
+      {
+        const bool odd = lane & 1;
+        const size_t base = ((size_t)(tok0 + 16 * cq) * H + h) * D + (c & ~1);
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+          const float x = __shfl_xor_sync(0xffffffffu, odd ? dgs[2 * m] : dgs[2 * m + 1], 1);
+          const int r = 16 * cq + 2 * m + (odd ? 1 : 0);
+          if (r < len)
+            *reinterpret_cast<float2 *>(a.dg + base + (size_t)(2 * m + (odd ? 1 : 0)) * H * D) =
+                odd ? make_float2(x, dgs[2 * m + 1]) : make_float2(dgs[2 * m], x);
+        }
       }
       if (tid < 64 && tid < len)
         dbeta[(size_t)(tok0 + tid) * H + h] = __float2bfloat16_rn(
