@@ -11,9 +11,10 @@ only compiles it with gcc and marshals numpy arrays.
 Every function is pinned by ``tests/test_oracle_pins.py`` to facts the pages
 and the mathematics fix (orthogonality at |alpha| = 1, beta = 2; the 2-D
 rotation; non-expansiveness; closed forms; dense brute force; finite
-differences).  Parity of the gradient with the authors' own "backward
-convention" is unpinned: that appendix is not in the pages; the oracle returns
-the exact gradient of the recurrence.
+differences).  The backward is the exact gradient of the recurrence, pinned by
+finite differences; the pages refer to an appendix with a "backward
+convention" for the gate's magnitude floor that they do not contain, so no
+other convention is implemented or compared.
 """
 from __future__ import annotations
 
