@@ -423,7 +423,7 @@ __global__ void __launch_bounds__(kSbThreads, 1) tc_state_bwd_kernel(const __gri
 constexpr int kGThreads = 512;  // 16 warps: four per TMEM lane quadrant
 constexpr uint32_t G_A1 = 0;          // [Q~; K~l] K-major 128 x 128
 constexpr uint32_t G_B1 = 32768;      // K~r K-major 64 x 128
-constexpr uint32_t G_KG = 49152;      // KG (== K-major [j][c] 64 rows); later dM M^T parts
+constexpr uint32_t G_KG = 49152;      // g staging (with B1); later dM M^T parts
 constexpr uint32_t G_UV = 65536;      // [U; V] K-major 128 x 128
 constexpr uint32_t G_TT = 98304;      // T K-major [r][j] 64 x 64
 constexpr uint32_t G_OU = 106496;     // [dO; dU] K-major 128 x 128
@@ -557,7 +557,7 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = ms.tmem;
-  const uint32_t sA1 = smem_u32(sm + G_A1), sB1 = smem_u32(sm + G_B1), sKG = smem_u32(sm + G_KG);
+  const uint32_t sA1 = smem_u32(sm + G_A1), sB1 = smem_u32(sm + G_B1);
   const uint32_t sUV = smem_u32(sm + G_UV), sTT = smem_u32(sm + G_TT), sOU = smem_u32(sm + G_OU);
   const uint32_t sSC = smem_u32(sm + G_SC), sWN = smem_u32(sm + G_WN);
   float *dTf = reinterpret_cast<float *>(sm + G_DT);
@@ -698,7 +698,6 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
         st_bf16(sm + G_A1, kmaj_off(r, c, 128), qp * el);
         st_bf16(sm + G_A1, kmaj_off(64 + r, c, 128), kp * el);
         st_bf16(sm + G_B1, kmaj_off(r, c, 64), kp * er);
-        st_bf16(sm + G_KG, mnmaj_off(r, c, 64), kp * el * eGm);
       }
     } else {
       // (unrolled: the prep arrays must stay in registers, which a runtime
@@ -711,7 +710,7 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
         fb[r * D + c] = P.G[i];
         fb[64 * D + r * D + c] = kp;
         fb[128 * D + r * D + c] = qp;
-        st_bf16(sm + G_KG, mnmaj_off(r, c, 64), kp * fast_exp(P.G[i]));
+        st_bf16(sm + G_A1, kmaj_off(64 + r, c, 128), kp * fast_exp(P.G[i]));  // KG itself (A1 is idle here)
       }
     }
     fence_async_smem();
@@ -844,25 +843,31 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
     if (!wait_one(&ms.bar[3], ph, a.status, 406)) { abort = true; break; }
     tc_fence_after();
     if (has_next) issue_stage(0, next_item);
-    {  // dW = -dU S_c^T -> rows 64..127 of the S_c tile (K-major [i][c]); S_c is dead
+    {  // dW = -dU S_c^T -> rows 64..127 of the S_c tile (K-major [i][c]); S_c is dead.
+      // Fast path: stored as dW Diag(e^{Gam_m}) (channel c scaled by e^{Gam_m,c}),
+      // so that KG = K~l Diag(e^{Gam_m}) is never formed: dW KG^T = (dW Diag(e^{Gam_m})) K~l^T,
+      // and dKG comes out scaled by e^{Gam_m} too (the epilogue uses el for E there)
+      const float sc = fast ? -fast_exp(P.Gm) : -1.f;
       float w[16];
       tmem_ld16(lanebase + 320 + 16 * cq, w);
       tmem_wait_ld();
 #pragma unroll
-      for (int i = 0; i < 16; ++i) st_bf16(sm + G_SC, kmaj_off(64 + 16 * cq + i, c, 128), -w[i]);
+      for (int i = 0; i < 16; ++i) st_bf16(sm + G_SC, kmaj_off(64 + 16 * cq + i, c, 128), sc * w[i]);
     }
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
 
     // ---------------- D7 = [dO; dU][U; V]^T + [.; dW] KG^T (second part), dKG^T ----------------
+    // (KG^T read as the K~l rows 64..127 of A1 -- KG itself on the exact path --
+    // against the scaled dW)
     if (tid == 0) {
       tc_fence_after();
       const uint32_t id2 = idesc_bf16(128, 64, false, false);
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk)
         mma_bf16(tmem + 192, sdesc_off(sdesc(sSC, 16, 1024), (kk >> 2) * 16384 + (kk & 3) * 32),
-                 sdesc_off(sdesc(sKG, 16, 1024), (kk >> 2) * 8192 + (kk & 3) * 32), id2, true);
+                 sdesc_off(sdesc(sA1 + 8192, 16, 1024), (kk >> 2) * 16384 + (kk & 3) * 32), id2, true);
       mma_commit(&ms.bar[4]);
     } else if (tid == 32) {
       tc_fence_after();
@@ -1171,13 +1176,15 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
           const float2 dKh2 = make_float2(dKh[i], dKh[i + 1]);
           const float2 Kh = __fmul2_rn(__fmul2_rn(make_float2(pCs, pCs), kp), eC);   // Khat
           const float2 khd = __fmul2_rn(dKh2, Kh);                                     // dKhat . Khat
-          // dk' = x1 + y1 + dKG E + pC dKhat eC;  dq' = x2 + dQG E
-          const float2 dkp = __ffma2_rn(make_float2(pCs, pCs), __fmul2_rn(dKh2, eC), __ffma2_rn(dKG2, E, __fadd2_rn(x1, y1)));
+          // dk' = x1 + y1 + dKG E + pC dKhat eC;  dq' = x2 + dQG E (on the fast
+          // path the dKG accumulator already carries e^{Gam_m}: its factor is el)
+          const float2 EK = kFast ? el : E;
+          const float2 dkp = __ffma2_rn(make_float2(pCs, pCs), __fmul2_rn(dKh2, eC), __ffma2_rn(dKG2, EK, __fadd2_rn(x1, y1)));
           const float2 dqp = __ffma2_rn(dQG2, E, x2);
           // dL/dGam: k' x1 + q' x2 - k' y1 + dKG KG + dQG QG - dKhat Khat
           float2 dgv = __fmul2_rn(kp, __fadd2_rn(x1, make_float2(-y1.x, -y1.y)));
           dgv = __ffma2_rn(qp, x2, dgv);
-          dgv = __ffma2_rn(__fmul2_rn(dKG2, kp), E, dgv);
+          dgv = __ffma2_rn(__fmul2_rn(dKG2, kp), EK, dgv);
           dgv = __ffma2_rn(__fmul2_rn(dQG2, qp), E, dgv);
           dgv = __fadd2_rn(dgv, make_float2(-khd.x, -khd.y));
           dg4[i] = dgv.x;
