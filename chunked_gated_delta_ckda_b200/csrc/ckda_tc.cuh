@@ -328,8 +328,9 @@ constexpr uint32_t R5 = 73728;   // d[128] fp32
 constexpr uint32_t R6 = 74240;   // M = (I + Diag(beta) A)^{-1}: fp32 [64][65] (row stride 65)
 constexpr uint32_t R7 = 90880;   // S_c^T bf16, K-major [v][c] 128 x 128: the chunk-start state
                                  // (written by the state pass, read by the backward)
+constexpr uint32_t R8 = 123648;  // T = M Diag(beta) bf16, K-major [r][j] 64 x 64 (read by the backward)
 constexpr uint32_t REC_STATE = R6;  // R1 .. R5: the part the sequential state passes read
-constexpr uint32_t REC = 123648;    // bytes per (chunk, head) record
+constexpr uint32_t REC = 131840;    // bytes per (chunk, head) record
 
 // 2^x and 1/x with one MUFU instruction each (PTX ex2.approx / rcp.approx);
 // their relative error (~2^-22) is far below the bf16 operand rounding.

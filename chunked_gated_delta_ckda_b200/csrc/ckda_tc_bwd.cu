@@ -443,7 +443,9 @@ constexpr uint32_t G_FSUM = G_UV;               // float [2][4][128]
 constexpr uint32_t W_TILE = 16384;              // W^T half of the record's R1 tile
 constexpr uint32_t S_TILE = 32768;              // the record's S_c^T (bf16 K-major [v][c])
 constexpr uint32_t M_BYTES = 64 * LDF * 4;      // the record's M
-static_assert(M_BYTES == R7 - R6 && S_TILE == REC - R7, "record layout");
+constexpr uint32_t T_TILE = 8192;               // the record's T
+constexpr uint32_t G_SGN = G_DT;                // sign rows of the next item (dT is dead by then)
+static_assert(M_BYTES == R7 - R6 && S_TILE == R8 - R7 && T_TILE == REC - R8, "record layout");
 
 struct GMisc {
   uint64_t bar[7], mdu, mds, mfin, mrec, mld;
@@ -573,11 +575,11 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
   const int nitems = a.map.n_chunks() * H;
 
   // Every load of one item: the reverse pass's dU tile, the forward's W tile,
-  // M and S_c^T, and the row tensors (q, k staged in A1, g in B1 + KG, sign in
-  // TT -- the prep consumes them before those tiles are written -- V into
-  // rows 64.. of [U; V] and dO into rows 0..63 of [dO; dU], K-major SW128
-  // boxes).  Issued once the previous item's last readers of these regions
-  // are done (its phase E), so they overlap its final epilogue.
+  // M, S_c^T and T, and the row tensors (q, k staged in A1, g in B1 + KG, sign
+  // in the dT scratch -- the prep consumes them before those regions are
+  // written -- V into rows 64.. of [U; V] and dO into rows 0..63 of [dO; dU],
+  // K-major SW128 boxes).  Issued in stages as the previous item's last
+  // readers of these regions finish.
   // thread 0's count of issued load sets (each completes mld, mrec and mdu
   // once) and of the completions it has seen: an abort drains the rest
   uint32_t n_issued = 0, n_mld = 0, n_mrec = 0, n_mdu = 0;
@@ -585,10 +587,11 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
   // it fills are no longer read by the current item, so that the loads spread
   // over the item instead of piling up at its end:
   //   0 (after the third MMA group): dU and dO into [dO; dU]; the dS tile into L2
-  //   1 (after the fourth):          S_c^T into the S tile, sign into T
+  //   1 (after the fourth):          S_c^T into the S tile, the record's T into T
   //   2 (after the dM M^T products): M
   //   3 (after dL):                  V into rows 64.. of [U; V]
-  //   4 (after X, Y):                q, k into A1, g into B1 + KG, the W tile
+  //   4 (after X, Y):                q, k into A1, g into B1 + KG, the W tile, sign
+  //                                  into the dT scratch (dead by then)
   // One copy per warp (lane 0) within a stage.  The three byte counts of the
   // set are posted by thread 0 once the current item's phases of mld, mrec and
   // mdu have completed; a transiently negative transaction count is allowed
@@ -599,7 +602,7 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
   int staged = 0, pending_item = -1;
   auto post_bytes = [&]() {
     mbar_arrive_expect_tx(&ms.mdu, DU_TILE);
-    mbar_arrive_expect_tx(&ms.mrec, W_TILE + M_BYTES + S_TILE);
+    mbar_arrive_expect_tx(&ms.mrec, W_TILE + M_BYTES + S_TILE + T_TILE);
     mbar_arrive_expect_tx(&ms.mld, kRowBytesQK + kRowBytesG + (a.sign ? kRowBytesSign : 0) + 2 * 16384);
   };
   // copy `w` of stage `st` for item itm (w < number of copies of the stage)
@@ -619,7 +622,7 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
       else prefetch_l2(ta.dS_tiles + (size_t)itm * DS_TILE, DS_TILE);  // copied in mid-item
     } else if (st == 1) {
       if (w == 0) bulk_g2s(sm + G_SC, rec + R7, S_TILE, &ms.mrec);
-      else if (a.sign) tma_rows(sm + G_TT, &ta.rm.sign, 0, hh, t, &ms.mld);
+      else bulk_g2s(sm + G_TT, rec + R8, T_TILE, &ms.mrec);
     } else if (st == 2) {
       bulk_g2s(sm + G_MF, rec + R6, M_BYTES, &ms.mrec);
     } else if (st == 3) {
@@ -628,10 +631,11 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
       if (w == 0) bulk_g2s(sm + G_WN, rec + R1, W_TILE, &ms.mrec);
       else if (w <= 2) tma_rows(sm + G_A1 + kStageQ + 8192 * (w - 1), &ta.rm.q, 64 * (w - 1), hh, t, &ms.mld);
       else if (w <= 4) tma_rows(sm + G_A1 + kStageK + 8192 * (w - 3), &ta.rm.k, 64 * (w - 3), hh, t, &ms.mld);
-      else tma_rows(sm + G_B1, &ta.rm.g, 0, hh, t, &ms.mld);
+      else if (w == 5) tma_rows(sm + G_B1, &ta.rm.g, 0, hh, t, &ms.mld);
+      else if (a.sign) tma_rows(sm + G_SGN, &ta.rm.sign, 0, hh, t, &ms.mld);
     }
   };
-  constexpr int kStageCopies[5] = {5, 2, 1, 2, 6};
+  constexpr int kStageCopies[5] = {5, 2, 1, 2, 7};
   // stage st of the next item's set, issued by lane 0 of the first warps
   auto issue_stage = [&](int st, int itm) {
     if (tid == 0 && st == 0 && !posted) {  // (the first item: counts not posted yet)
@@ -671,7 +675,7 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
     if (!wait_all(&ms.mld, ph, a.status, 400)) { abort = true; break; }
     ++n_mld;
     PrepC P;
-    prepc_load(sm + G_A1, reinterpret_cast<const float *>(sm + G_B1), a.sign ? sm + G_TT : nullptr, len, c, cq,
+    prepc_load(sm + G_A1, reinterpret_cast<const float *>(sm + G_B1), a.sign ? sm + G_SGN : nullptr, len, c, cq,
                P, &ms.qt[0][0], &ms.qp[0][0]);
     if (len < 64) {  // V and dO rows past the chunk
       zero_tail_rows(sm + G_UV + 8192, 16384, len, tid, kGThreads);
@@ -713,23 +717,11 @@ __global__ void __launch_bounds__(kGThreads, 1) tc_grad_kernel(const __grid_cons
         st_bf16(sm + G_A1, kmaj_off(64 + r, c, 128), kp * fast_exp(P.G[i]));  // KG itself (A1 is idle here)
       }
     }
-    fence_async_smem();
-    __syncthreads();
+    fence_async_smem();  // (the wait below is the barrier before the MMAs read the tiles)
 
-    // ---------------- T = M Diag(beta) (M from the forward's record) ----------------
+    // ---------------- the record's tiles (W, M, S_c^T, T = M Diag(beta)) ----------------
     if (!wait_all(&ms.mrec, ph, a.status, 401)) { abort = true; break; }
     ++n_mrec;
-    {
-      const int r = tid >> 3, j0 = (tid & 7) * 8;
-      uint32_t pk[4];
-#pragma unroll
-      for (int m = 0; m < 4; ++m)
-        pk[m] = pack_bf16(Mf[r * LDF + j0 + 2 * m] * ms.beta[j0 + 2 * m],
-                          Mf[r * LDF + j0 + 2 * m + 1] * ms.beta[j0 + 2 * m + 1]);
-      *reinterpret_cast<uint4 *>(sm + G_TT + kmaj_off(r, j0, 64)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-    }
-    fence_async_smem();
-    __syncthreads();
 
     // ---------------- A (kept in TMEM for dbeta), U^T = V^T T^T - (W S)^T ----------------
     if (tid == 32) {  // A, by a second thread (its commit is part of this phase)

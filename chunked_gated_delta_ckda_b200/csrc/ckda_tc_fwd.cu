@@ -350,8 +350,9 @@ __global__ void __launch_bounds__(kIntraThreads, 2) tc_intra_kernel(const __grid
     }
     fence_async_smem();
     __syncthreads();
-    if (tid == 0) {  // M itself goes to the record too: the backward starts from it
+    if (tid == 0) {  // M and T go to the record too: the backward starts from them
       bulk_s2g(rec + R6, Mf, 64 * LDF * 4);
+      bulk_s2g(rec + R8, sm + I_T, 8192);
       bulk_commit();
     }
 
