@@ -81,7 +81,7 @@ KERNEL_UNITS = {
 # captured on a B=2 launch (inputs still larger than L2), traffic being
 # proportional to the chunk-heads a launch processes (profiles/).
 NCU_TRAFFIC = {
-    ("tc_grad", "layer_fwdbwd_bf16"): (454157056 + 135293952) / (2 * 64 * 16),
+    ("tc_grad", "layer_fwdbwd_bf16"): (470960896 + 135686912) / (2 * 64 * 16),
 }
 
 
