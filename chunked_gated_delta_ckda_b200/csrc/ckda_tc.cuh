@@ -246,10 +246,6 @@ __host__ __device__ __forceinline__ uint32_t mnmaj_off(int k, int mn, int kdim) 
   const int blk = mn >> 6, c = mn & 63;
   return (uint32_t)(blk * kdim * 128 + k * 128 + ((((c >> 3) ^ (k & 7)) << 4) | ((c & 7) << 1)));
 }
-// 16-byte chunk j (0..7) of row `row` in a 128-byte-swizzled row
-__host__ __device__ __forceinline__ uint32_t swz_chunk(int row, int j) {
-  return (uint32_t)(((j ^ (row & 7)) << 4));
-}
 
 // Instruction descriptor, kind::f16, bf16 x bf16 -> fp32.
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn, bool b_mn) {
@@ -348,51 +344,6 @@ __device__ __forceinline__ float fast_exp(float x) { return ex2_approx(x * kLog2
 
 __device__ __forceinline__ void st_bf16(unsigned char *base, uint32_t off, float x) {
   *reinterpret_cast<__nv_bfloat16 *>(base + off) = __float2bfloat16_rn(x);
-}
-
-// Chunk rows 32*hf .. 32*hf+31 of key channel c: local inclusive cumsum of g,
-// raw bf16 k | q << 16, sign bits.  Rows >= len are padding (g = 0, k = q = 0,
-// sign +1).  All loads are issued before any use (clamped row index).
-__device__ __forceinline__ void load_rows(const float *g, const int8_t *sign,
-                                          const __nv_bfloat16 *k, const __nv_bfloat16 *q,
-                                          int64_t tok0, int len, int h, int H, int c, int hf,
-                                          float (&G)[32], uint32_t (&kq)[32], uint32_t &neg) {
-  float acc = 0.f;
-  neg = 0;
-#pragma unroll
-  for (int b = 0; b < 2; ++b) {  // two batches of 16 rows: all loads of a batch in flight
-    float gg[16];
-    int sg[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const int r = 32 * hf + 16 * b + i;
-      const int rr = r < len ? r : len - 1;
-      const size_t off = ((size_t)(tok0 + rr) * H + h) * D + c;
-      gg[i] = g[off];
-      sg[i] = sign[off];
-      kq[16 * b + i] = (uint32_t)__bfloat16_as_ushort(k[off]) |
-                       ((uint32_t)__bfloat16_as_ushort(q[off]) << 16);
-    }
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const int ii = 16 * b + i;
-      const bool valid = 32 * hf + ii < len;
-      acc += valid ? gg[i] : 0.f;
-      G[ii] = acc;
-      if (!valid) kq[ii] = 0;
-      if (valid && sg[i] < 0) neg |= 1u << ii;
-    }
-  }
-}
-
-__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8]) {
-  uint32_t r[8];
-  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-                 "=r"(r[7])
-               : "r"(taddr));
-#pragma unroll
-  for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
 }
 
 // ---------------------------------------------------------------------------

@@ -65,13 +65,6 @@ __device__ __forceinline__ void tmem_st4(uint32_t taddr, const float (&v)[4]) {
 __device__ __forceinline__ void tmem_st1(uint32_t taddr, float v) {
   asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(__float_as_uint(v)) : "memory");
 }
-__device__ __forceinline__ void cp_async16(void *smem_dst, const void *gsrc, bool valid) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(smem_dst)), "l"(gsrc),
-               "r"(valid ? 16 : 0)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
 // ===========================================================================
 // reverse state pass
